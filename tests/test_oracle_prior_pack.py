@@ -1,0 +1,185 @@
+"""Pins of the oracle's mask-prior initialisation (Eq.9, Eq.10) and hard-mask packing.
+
+Checked against: the page's similarity values and mean inner product, combinatorial overlap
+counts, a brute force over candidates for the magnitude prior, the moments of N(0, 0.01),
+an independent unpacker of the packed format, and the page's 0.65 bits/param figure.
+"""
+import math
+from itertools import combinations
+
+import numpy as np
+import pytest
+
+from _golden import keyed, rows
+
+NM = [(2, 4), (4, 8)]
+
+
+def _energy_best(S, W):
+    """Brute force: candidate that keeps the largest sum of squared weights."""
+    energy = (W[:, None, :] ** 2 * S[None].astype(np.float64)).sum(-1)
+    return np.argmax(energy, 1)
+
+
+# ---------------------------------------------------------------- Eq.9 similarity
+
+def test_similarity_values_2of4_match_page(orc):
+    table = {int(r[0]): int(r[1]) for r in rows("prior_similarity_2of4.txt") if r[0] != "mean_inner_product"}
+    mean_ip = float(keyed("prior_similarity_2of4.txt")["mean_inner_product"][0])
+    rng = np.random.default_rng(0)
+    W = rng.normal(0, 0.02, size=(500, 4))
+    S = orc.candidates(2, 4)
+    pi, pidx, sim = orc.prior_init(2, 4, W, np.arange(500), alpha=3.0, init_std=0.0, seed=0)
+    for b in range(500):
+        m0 = S[pidx[b]]
+        ip = (S * m0).sum(1)
+        assert ip.mean() == mean_ip            # mean inner product over the candidates
+        for i in range(6):
+            assert sim[b, i] == table[int(ip[i])]
+        # counts of +1 / 0 / -1 are 1 / 4 / 1
+        assert sorted(sim[b]) == [-1, 0, 0, 0, 0, 1]
+
+
+def test_similarity_4of8_overlap_counts(orc):
+    """For 4:8 the overlap of a candidate with the prior is 4,3,2,1,0 for 1,16,36,16,1
+    candidates; the mean inner product is N^2/M = 2, so sim runs +2..-2 with mean 0."""
+    rng = np.random.default_rng(1)
+    W = rng.normal(0, 0.02, size=(50, 8))
+    _, pidx, sim = orc.prior_init(4, 8, W, np.arange(50), 3.0, 0.0, 0)
+    for b in range(50):
+        vals, counts = np.unique(sim[b], return_counts=True)
+        assert list(vals) == [-2, -1, 0, 1, 2]
+        assert list(counts) == [1, 16, 36, 16, 1]
+        assert sim[b].mean() == 0.0
+        # the closed form of the mean: each kept position lies in C(M-1, N-1) candidates
+        assert math.comb(7, 3) * 4 / math.comb(8, 4) == 2.0
+
+
+# ---------------------------------------------------------------- magnitude prior
+
+@pytest.mark.parametrize("n,m", NM)
+def test_magnitude_prior_is_energy_maximiser(orc, n, m):
+    rng = np.random.default_rng(2)
+    S = orc.candidates(n, m)
+    W = rng.normal(0, 0.02, size=(400, m))
+    _, pidx, _ = orc.prior_init(n, m, W, np.arange(400), 3.0, 0.0, 0)
+    np.testing.assert_array_equal(pidx, _energy_best(S, W))
+
+
+def test_magnitude_prior_ties_and_nan(orc):
+    S = orc.candidates(2, 4)
+    W = np.array([[0.5, -0.5, 0.5, 0.1],       # tie among 0,1,2 -> keep 0,1
+                  [np.nan, 0.1, 0.2, 0.3],     # NaN ranks last -> keep 2,3
+                  [0.0, 0.0, 0.0, 0.0],        # all equal -> keep 0,1
+                  [0.1, -0.3, 0.3, 0.05]])     # |.| tie between 1 and 2 -> keep 1,2
+    _, pidx, _ = orc.prior_init(2, 4, W, np.arange(4), 3.0, 0.0, 0)
+    kept = [tuple(np.flatnonzero(S[k])) for k in pidx]
+    assert kept == [(0, 1), (2, 3), (0, 1), (1, 2)]
+
+
+# ---------------------------------------------------------------- Eq.10 initialisation
+
+@pytest.mark.parametrize("n,m", NM)
+def test_deterministic_prior_argmax_reproduces_prior(orc, n, m):
+    """init_std = 0: pi = alpha * sim, so argmax(kappa * pi) is the prior candidate in every
+    block (and it is the unique maximum)."""
+    rng = np.random.default_rng(3)
+    W = rng.normal(0, 0.02, size=(1000, m))
+    pi, pidx, sim = orc.prior_init(n, m, W, np.arange(1000), alpha=3.0, init_std=0.0, seed=0)
+    np.testing.assert_array_equal(pi, 3.0 * sim)
+    k = orc.argmax(np.float32(3.0) * pi.astype(np.float32), orc.num_candidates(n, m))
+    np.testing.assert_array_equal(k, pidx)
+    assert np.all((pi == pi.max(1, keepdims=True)).sum(1) == 1)
+
+
+@pytest.mark.parametrize("n,m", NM)
+def test_random_init_is_normal_with_std_001(orc, n, m):
+    """alpha = 0 leaves the N(0, 0.01) draws (Table 7): zero mean, std 0.01, Box-Muller
+    pairs with E[r^2] = 2, and independent of the weights."""
+    C = orc.num_candidates(n, m)
+    nb = 40_000 if m == 4 else 4000
+    rng = np.random.default_rng(4)
+    W = rng.normal(0, 0.02, size=(nb, m))
+    pi, _, _ = orc.prior_init(n, m, W, np.arange(nb), alpha=0.0, init_std=0.01, seed=7)
+    z = pi.ravel() / 0.01
+    N = z.size
+    assert abs(z.mean()) < 5 / math.sqrt(N)
+    assert abs(z.var() - 1.0) < 5 * math.sqrt(2.0 / N)
+    assert abs(((z - z.mean()) ** 4).mean() / z.var() ** 2 - 3.0) < 5 * math.sqrt(24.0 / N)
+    pairs = pi[:, : (C // 2) * 2].reshape(nb, -1, 2) / 0.01
+    r2 = (pairs ** 2).sum(-1).ravel()
+    assert abs(r2.mean() - 2.0) < 5 * 2.0 / math.sqrt(r2.size)
+    pi2, _, _ = orc.prior_init(n, m, W * 3.0, np.arange(nb), alpha=0.0, init_std=0.01, seed=7)
+    np.testing.assert_array_equal(pi, pi2)
+
+
+@pytest.mark.parametrize("n,m", NM)
+def test_prior_bias_scales_with_block_std(orc, n, m):
+    """Eq.10: pi(alpha) - pi(0) = alpha * sigma(pi(0)) * sim, sigma the spread of the block's
+    random logits."""
+    rng = np.random.default_rng(5)
+    W = rng.normal(0, 0.02, size=(300, m))
+    p0, pidx, sim = orc.prior_init(n, m, W, np.arange(300), 0.0, 0.01, seed=9)
+    p3, pidx3, _ = orc.prior_init(n, m, W, np.arange(300), 3.0, 0.01, seed=9)
+    np.testing.assert_array_equal(pidx, pidx3)
+    sigma = p0.std(1, keepdims=True)
+    np.testing.assert_allclose(p3 - p0, 3.0 * sigma * sim, rtol=0, atol=1e-15)
+    # with the bias the prior candidate's logit rises by alpha*sigma*max(sim) over its draw
+    assert np.all(p3[np.arange(300), pidx] > p0[np.arange(300), pidx])
+
+
+# ---------------------------------------------------------------- hard mask and packing
+
+def _unpack(n, m, values, meta, rows_, cols, dtype):
+    """Independent reading of the packed format back into a dense matrix."""
+    dense = np.zeros((rows_, cols), dtype)
+    bpr = cols // m
+    for r in range(rows_):
+        for q in range(bpr):
+            if m == 4:
+                nib = (int(meta[r, q // 8]) >> (4 * (q % 8))) & 0xF
+                pos = [nib & 3, nib >> 2]
+            else:
+                code = int(meta[r, q])
+                pos = [(code >> (3 * t)) & 7 for t in range(4)]
+            assert pos == sorted(pos) and len(set(pos)) == n and max(pos) < m
+            for t in range(n):
+                dense[r, q * m + pos[t]] = values[r, q * n + t]
+    return dense
+
+
+@pytest.mark.parametrize("n,m", NM)
+@pytest.mark.parametrize("wbits", [np.uint16, np.uint32])
+def test_pack_roundtrip_is_masked_weight(orc, n, m, wbits):
+    rng = np.random.default_rng(6)
+    C = orc.num_candidates(n, m)
+    S = orc.candidates(n, m)
+    rows_, cols = 7, m * 21           # 21 blocks per row: a ragged last metadata word for 2:4
+    Wraw = rng.integers(1, np.iinfo(wbits).max, size=(rows_, cols), dtype=wbits)
+    pi = rng.normal(0, 1, size=(rows_ * cols // m, C)).astype(np.float32)
+    values, meta, cand = orc.hard_pack(n, m, Wraw, pi)
+    k = np.argmax(pi, 1)
+    np.testing.assert_array_equal(cand, k)
+    dense = _unpack(n, m, values, meta, rows_, cols, wbits)
+    mask = S[k].reshape(rows_, cols)
+    np.testing.assert_array_equal(dense, np.where(mask == 1, Wraw, 0))
+    if m == 4:
+        # unused nibbles of the last word are zero
+        assert np.all((meta[:, -1] >> (4 * (21 % 8))) == 0)
+
+
+def test_argmax_ties_and_nan(orc):
+    pi = np.array([[1.0, 3.0, 3.0, 0.0, 3.0, 2.0],
+                   [np.nan, 1.0, 2.0, np.nan, 2.0, 0.0],
+                   [np.nan] * 6,
+                   [-np.inf, -1.0, -np.inf, -1.0, -2.0, -3.0]], np.float32)
+    np.testing.assert_array_equal(orc.argmax(pi, 6), [1, 2, 0, 1])
+
+
+def test_mask_storage_bits_per_param(orc):
+    """A 2:4 mask is one of C(4,2) = 6 candidates per 4 weights: log2(6)/4 = 0.646 bits per
+    parameter, the page's 0.65 bits/param."""
+    page = float(keyed("paper_figures.txt")["mask_bits_per_param_2of4"][0])
+    C = orc.num_candidates(2, 4)
+    assert C == int(keyed("paper_figures.txt")["logits_per_block_2of4"][0])
+    assert round(math.log2(C) / 4, 2) == page
