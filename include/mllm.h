@@ -1,0 +1,190 @@
+/*
+ * mllm.h -- C ABI of libmllm, the B200 (sm_100a) implementation of MaskLLM's per-block
+ * differentiable N:M mask sampler.
+ *
+ * Source of the method: "MaskLLM: Learnable Semi-Structured Sparsity for Large Language
+ * Models" (arXiv 2409.17481), as summarised on the paper-graph-ui page; sections below are
+ * that page's. Every weight matrix is frozen; each block of M consecutive weights along a
+ * row carries C = C(M,N) learnable logits, one per candidate N:M mask (s.3.2). One
+ * training step calls mllm_sample_fwd for every matrix, the caller's network consumes the
+ * soft-masked weights and returns their gradient, then mllm_sample_bwd_adam updates the
+ * logits in place (s.3.4, Algorithm 1 step 2). mllm_prior_init runs once before training
+ * (Algorithm 1 step 1) and mllm_hard_pack once after it (Algorithm 1 step 3).
+ *
+ * Conventions shared by every call
+ *   Layout. A matrix is row-major [rows, cols] with cols % M == 0. Block b (0-based, in
+ *     row-major order) covers elements [b*M, b*M + M) of the flattened matrix, i.e. M
+ *     consecutive weights of one row. B = rows*cols/M blocks. Per-block arrays (logits and
+ *     the AdamW moments) are row-major [B, C] fp32. The candidate order is fixed:
+ *       2:4 (C = 6): [1,1,0,0] [1,0,1,0] [1,0,0,1] [0,1,0,1] [0,1,1,0] [0,0,1,1]
+ *                    (the page's listing, s.3.2 Eq.2; 1 = keep);
+ *       4:8 (C = 70): the 4-subsets of positions 0..7 in lexicographic order of their
+ *                    ascending index tuples, (0,1,2,3), (0,1,2,4), ..., (4,5,6,7).
+ *   Ownership. Every pointer inside mllm_matrix, and reg_sum_out / workspace, is device
+ *     memory owned by the caller and borrowed for the duration of the enqueued work. The
+ *     `mats` and `hp` arrays themselves are host memory, read during the call only. The
+ *     library allocates nothing and keeps no state between calls.
+ *   Streams. `stream` is a cudaStream_t (NULL = the legacy default stream). All work is
+ *     enqueued asynchronously on it; the call returns once enqueued.
+ *   Alignment. Every device pointer must be 16-byte aligned (MLLM_ERR_MISALIGNED).
+ *   Errors. Arguments are validated on the host before anything is enqueued; on any error
+ *     nothing is launched and no output is touched. A failed launch returns MLLM_ERR_CUDA
+ *     (mllm_last_cuda_error() gives the cudaError_t). No call waits on the device, so no
+ *     call can hang; device-side faults surface at the caller's next synchronisation.
+ *   Grouping. `n_mats > 1` processes all matrices of one layer in a single launch; each
+ *     matrix keeps its own buffers. Matrices with rows == 0 or cols == 0 are allowed and
+ *     contribute nothing.
+ *   Random numbers. Noise for candidate c of block b of a matrix at sampling step s comes
+ *     from Philox4x32-10 (Salmon et al., SC'11) with key (seed lo32, seed hi32) and counter
+ *     (gid lo32, gid hi32, s, c/6), gid = block_offset + b; field c%6 = bits [21(c%6),
+ *     21(c%6)+21) of the 128-bit output (word 0 least significant) is k, eps =
+ *     (2k+1)*2^-22, and g = -nlog(-nlog(eps)) with nlog the fp32 table-driven logarithm
+ *     fixed by the specification (Tang's method, a 128-entry table, a cubic remainder).
+ *     Step 0xFFFFFFFF is reserved for mllm_prior_init. The same (seed, step) gives
+ *     bit-identical noise in forward and backward; noise is recomputed, never stored.
+ */
+#ifndef MLLM_H
+#define MLLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLLM_ABI_VERSION 1
+
+typedef enum {
+    MLLM_OK = 0,
+    MLLM_ERR_INVALID_ARG = 1, /* null pointer, bad size, non-finite or out-of-range scalar */
+    MLLM_ERR_MISALIGNED = 2,  /* a device pointer is not 16-byte aligned */
+    MLLM_ERR_UNSUPPORTED = 3, /* N:M other than 2:4 or 4:8, or an unsupported dtype */
+    MLLM_ERR_WORKSPACE = 4,   /* workspace missing or smaller than mllm_workspace_bytes() */
+    MLLM_ERR_CUDA = 5         /* a CUDA launch or runtime call failed */
+} mllm_status;
+
+typedef enum {
+    MLLM_BF16 = 0, /* bfloat16 */
+    MLLM_F32 = 1   /* IEEE binary32 */
+} mllm_dtype;
+
+typedef struct {
+    int32_t n; /* weights kept per block: 2 or 4 */
+    int32_t m; /* block length: 4 or 8 */
+} mllm_nm;
+
+/* One frozen weight matrix and its buffers. Fields a call does not use may be NULL. */
+typedef struct {
+    const void *W;          /* [rows, cols] w_dtype, frozen weights (all calls) */
+    void *X_out;            /* [rows, cols] w_dtype, soft-masked weights W . M (fwd) */
+    const void *G;          /* [rows, cols] g_dtype, dL/dX from the network (bwd) */
+    int32_t w_dtype;        /* mllm_dtype of W and X_out */
+    int32_t g_dtype;        /* mllm_dtype of G */
+    int64_t rows, cols;     /* cols % M == 0 */
+    float *logits;          /* [B, C] fp32 logits pi (init writes; fwd reads; bwd updates) */
+    float *adam_m;          /* [B, C] fp32 AdamW first moment (init zeroes; bwd updates) */
+    float *adam_v;          /* [B, C] fp32 AdamW second moment (init zeroes; bwd updates) */
+    uint64_t block_offset;  /* global id of block 0, the Philox counter base */
+    float *soft_mask_out;   /* [rows, cols] fp32 soft mask M (fwd, optional, for inspection) */
+    float *grad_logits_out; /* [B, C] fp32 dL/dpi before AdamW (bwd, optional) */
+    void *pack_values;      /* [rows, cols*N/M] w_dtype kept weights (pack) */
+    void *pack_meta;        /* pack: 2:4 uint32 [rows, ceil(cols/32)]; 4:8 uint16 [rows, cols/8] */
+    uint8_t *cand_idx_out;  /* [B] uint8 argmax candidate index (pack, optional) */
+} mllm_matrix;
+
+/* Per-step scalars (s.3.4 Table 7 values in brackets; the schedules are the caller's). */
+typedef struct {
+    float kappa;        /* logit scale, > 0 (100 -> 500 linearly) */
+    float tau;          /* Gumbel-softmax temperature, > 0 (4 -> 0.05 linearly) */
+    float lambda;       /* sparse-weight regulariser strength, >= 0 (1e-5), Eq.8 */
+    float lr;           /* AdamW learning rate, >= 0 (5e-4 LLaMA-2, 1e-3 GPT-3) */
+    float beta1, beta2; /* AdamW betas in [0, 1) (0.9, 0.999) */
+    float eps;          /* AdamW epsilon, > 0 (1e-8) */
+    float weight_decay; /* decoupled weight decay, >= 0 (0.1) */
+    uint32_t adam_step; /* 1-based AdamW step t for the bias corrections 1 - beta^t */
+    uint32_t step;      /* sampling step s, the Philox counter word 2; != 0xFFFFFFFF */
+    uint64_t seed;      /* Philox key */
+    int32_t noise_on;   /* 0 replaces the Gumbel noise by zero */
+    int32_t reserved;   /* must be 0 */
+} mllm_hparams;
+
+/* Number of candidate masks C(M, N) (6 or 70), or 0 if unsupported. */
+int32_t mllm_num_candidates(mllm_nm nm);
+
+/* Mask-prior initialisation (s.3.4 "Mask Prior", Eq.9 and Eq.10; Algorithm 1 step 1).
+ * Per block: M0 = the N positions of largest |W| (equal magnitudes: lower position first;
+ * NaN ranks last); sim_i = M0.S_i - (mean over k of M0.S_k) = M0.S_i - N*N/M;
+ * pi0_i = init_std * n_i with n_i standard normal (Box-Muller: candidates 2p and 2p+1 take
+ * radius sqrt(-2 ln u_2p) and angle 2*pi*u_(2p+1), u_c the reserved-step uniform of
+ * candidate c); pi_i = pi0_i + alpha * sigma * sim_i with sigma the population standard
+ * deviation of pi0 over the block's C logits. init_std == 0 selects a deterministic mode
+ * (an addition, not on the pages): pi_i = alpha * sim_i, so argmax pi is the prior mask.
+ * Writes logits, and zeroes adam_m and adam_v when they are non-NULL.
+ * Reads W; needs logits. alpha >= 0 and init_std >= 0, both finite. */
+mllm_status mllm_prior_init(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, float alpha,
+                            float init_std, uint64_t seed, void *stream);
+
+/* Forward of the sampler (s.3.4 Eq.5-Eq.8, Algorithm 1 lines 1-5). Per block:
+ *   w_i = fma(kappa, pi_i, g_i) in fp32 (one rounding); y = softmax(w / tau) (Eq.6);
+ *   M_j = sum_i y_i S_ij (Eq.7); X_j = W_j * M_j rounded to nearest-even in w_dtype;
+ *   reg += sum_j (W_j M_j)^2 (Eq.8 without lambda, before rounding X).
+ * Writes X_out (and soft_mask_out when non-NULL). When reg_sum_out is non-NULL it receives
+ * the sum over all blocks of all matrices as one double; this needs a workspace of
+ * mllm_workspace_bytes() bytes, zero-filled before its first use (each call leaves it
+ * zero-filled when its work completes; calls sharing a workspace must be stream-ordered).
+ * The sum is deterministic for a given device. reg_sum_out == NULL skips the reduction and
+ * the workspace may be NULL. Reads W, logits. */
+mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                            const mllm_hparams *hp, double *reg_sum_out, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Backward to the logits fused with AdamW (s.3.2 "Frozen LLM Backbone"; s.3.4 Eq.8 and
+ * Algorithm 1 step 2; AdamW as in PyTorch, Loshchilov & Hutter decoupled decay).
+ * Recomputes the forward's noise, y and M for the same (seed, step), then per block:
+ *   u_j = G_j W_j - 2 lambda W_j^2 M_j                 (dL/dM for L = L_LM - lambda R)
+ *   dpi_i = (kappa/tau) y_i sum_j (S_ij - M_j) u_j     (1 - M_j formed as a sum of y)
+ *   pi <- pi (1 - lr wd); m <- b1 m + (1-b1) dpi; v <- b2 v + (1-b2) dpi^2;
+ *   pi <- pi - lr/(1-b1^t) * m / (sqrt(v)/sqrt(1-b2^t) + eps),  t = adam_step.
+ * Updates logits, adam_m, adam_v in place; writes grad_logits_out when non-NULL.
+ * Reads W, G. */
+mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                 const mllm_hparams *hp, void *stream);
+
+/* Hard-mask extraction and compressed export (s.3.2 "Information flow at inference";
+ * Algorithm 1 step 3). Per block: k = first index of the largest logit (NaN never wins;
+ * all-NaN gives 0), kept positions p_0 < ... < p_{N-1} of S_k;
+ *   pack_values[r, q*N + t] = W[r, q*M + p_t] (bit copy), for block q of row r;
+ *   2:4 pack_meta: nibble p_0 | p_1 << 2 in bits [4(q%8), 4(q%8)+4) of uint32 word q/8 of
+ *     row r; a row has ceil((cols/4)/8) words; unused high nibbles are written as zero;
+ *   4:8 pack_meta: uint16 per block, p_0 | p_1 << 3 | p_2 << 6 | p_3 << 9;
+ *   cand_idx_out[b] = k when non-NULL.
+ * Reads W, logits. */
+mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, void *stream);
+
+/* The Gumbel noise itself, for inspection and statistical tests: g_out[i*C + c] = noise
+ * of candidate c of the block with global id gids[i] at (seed, step). gids and g_out are
+ * device arrays of n_blocks and n_blocks*C entries; step may be any value, including the
+ * reserved one. */
+mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t *gids,
+                       int64_t n_blocks, float *g_out, void *stream);
+
+/* Workspace bytes mllm_sample_fwd needs for its regulariser sum (independent of sizes). */
+size_t mllm_workspace_bytes(void);
+
+/* Static description of a status code. */
+const char *mllm_status_string(mllm_status s);
+
+/* cudaError_t of the most recent MLLM_ERR_CUDA on the calling thread (0 if none). */
+int32_t mllm_last_cuda_error(void);
+
+/* ABI guards for bindings: MLLM_ABI_VERSION, sizeof(mllm_matrix), sizeof(mllm_hparams). */
+int32_t mllm_abi_version(void);
+size_t mllm_sizeof_matrix(void);
+size_t mllm_sizeof_hparams(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLLM_H */

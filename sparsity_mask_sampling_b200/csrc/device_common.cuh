@@ -1,0 +1,183 @@
+// device_common.cuh -- launch descriptors and the random-number path shared by the kernels.
+//
+// The noise is part of the specification (bit for bit): Philox4x32-10 (Salmon, Moraes, Dror,
+// Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) gives 128 bits per (seed,
+// block, step, group); six 21-bit fields k give uniforms eps = (2k+1) 2^-22 and the Gumbel
+// noise g = -nlog(-nlog(eps)) of MaskLLM's Eq.5 (paper-graph-ui summary, s.3.4 "Step 1").
+// nlog is the fp32 table-driven logarithm of P.T.P. Tang (ACM TOMS 16(4), 1990): a 7-bit
+// mantissa prefix selects a breakpoint F in [0.75, 1.5), r = x 2^-e / F - 1 with |r| < 2^-8,
+// ln(1+r) ~ r - r^2/2 + r^3/3. Only correctly rounded fp32 operations (fma, mul, add,
+// int->float) are used, so the bits are fixed by the definition on any IEEE machine.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace mllm {
+
+constexpr int kMaxMats = 16;             // matrices per launch; larger groups are chunked
+constexpr uint32_t kInitStep = 0xFFFFFFFFu;
+constexpr int kThreads = 256;            // threads per CTA for every sampler kernel
+
+// Logarithm table and constants, built once on the host from their definitions:
+// F_j = 1 + j/128 (j < 64) or (1 + j/128)/2 (j >= 64); c_j = fl32(1/F_j);
+// L_j = fl32(-ln c_j); ln2_hi = fl32(ln 2) with the low 8 mantissa bits cleared;
+// ln2_lo = fl32(ln 2 - ln2_hi); one_third = fl32(1/3).
+struct NoiseTab {
+    float2 cl[128];  // (c_j, L_j)
+    float ln2_hi, ln2_lo, one_third, pad;
+};
+
+// One matrix of a grouped launch. work_begin/work_count are in the kernel's work units
+// (tiles of kThreads pairs of blocks, or of packed words).
+struct MatDesc {
+    const void *W;
+    void *X;
+    const void *G;
+    float *pi, *m, *v;
+    float *soft, *grad;
+    void *pvals, *pmeta;
+    uint8_t *cidx;
+    int64_t rows, cols, nblocks;
+    uint64_t gid0;
+    int64_t work_begin, work_count;
+    int32_t w_f32, g_f32;
+};
+
+struct Group {
+    int32_t n;
+    int32_t pad;
+    int64_t total_work;
+    MatDesc d[kMaxMats];
+};
+
+// Scalars of one forward / backward launch, derived on the host from mllm_hparams.
+struct StepScalars {
+    float kappa;         // logit scale
+    float c2;            // fl32(log2(e) / tau): exp((w - max)/tau) = 2^((w - max) * c2)
+    float kappa_over_tau;// fl32(kappa / tau), the z -> pi chain factor
+    float two_lambda;    // 2 lambda
+    float decay;         // fl32(1 - lr * wd)
+    float beta1, one_minus_beta1, beta2, one_minus_beta2;
+    float step_size;     // fl32(lr / (1 - beta1^t))
+    float inv_sqrt_bc2;  // fl32(1 / sqrt(1 - beta2^t))
+    float eps;
+    uint32_t step;
+    uint32_t noise_on;
+    uint64_t seed;
+};
+
+__device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Index of the matrix that owns work unit t (uniform across the CTA).
+__device__ __forceinline__ int find_mat(const Group &g, int64_t t) {
+    int i = 0;
+    while (i + 1 < g.n && t >= g.d[i + 1].work_begin) ++i;
+    return i;
+}
+
+// ---------------------------------------------------------------------------- Philox
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t rk0 = k0 + (uint32_t)r * 0x9E3779B9u;  // Weyl key schedule
+        const uint32_t rk1 = k1 + (uint32_t)r * 0xBB67AE85u;
+        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ rk0, lo1, hi0 ^ c.w ^ rk1, lo0);
+    }
+    return c;
+}
+
+// The six 21-bit fields of the 128-bit output (x as a little-endian integer).
+__device__ __forceinline__ void fields21(uint4 x, uint32_t f[6]) {
+    constexpr uint32_t M21 = 0x1FFFFFu;
+    f[0] = x.x & M21;
+    f[1] = __funnelshift_r(x.x, x.y, 21) & M21;
+    f[2] = (x.y >> 10) & M21;
+    f[3] = __funnelshift_r(x.y, x.z, 31) & M21;
+    f[4] = __funnelshift_r(x.z, x.w, 20) & M21;
+    f[5] = (x.w >> 9) & M21;
+}
+
+__device__ __forceinline__ uint4 block_words(uint64_t seed, uint64_t gid, uint32_t step, uint32_t group) {
+    return philox4x32_10(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), step, group),
+                         (uint32_t)seed, (uint32_t)(seed >> 32));
+}
+
+// eps = (2k+1) 2^-22: the bit pattern of 1 + (2k+1) 2^-22 minus 1 (both exact).
+__device__ __forceinline__ float uniform_from_field(uint32_t k) {
+    return __fadd_rn(__uint_as_float(0x3F800002u | (k << 2)), -1.0f);
+}
+
+// ---------------------------------------------------------------------------- nlog
+
+__device__ __forceinline__ float nlog(float x, const float2 *__restrict__ tab, float ln2_hi,
+                                      float ln2_lo, float one_third) {
+    const uint32_t b = __float_as_uint(x);
+    const uint32_t ib = b + 0x8000u;               // nearest 7-bit mantissa prefix
+    const uint32_t j = (ib >> 16) & 0x7Fu;
+    const int32_t e = (int32_t)(ib >> 23) - 127 + (int32_t)(j >> 6);
+    const float mm = __uint_as_float(b - ((uint32_t)e << 23));  // x 2^-e, exact
+    const float2 cl = tab[j];
+    const float r = __fmaf_rn(mm, cl.x, -1.0f);
+    const float q = __fmaf_rn(r, one_third, -0.5f);
+    const float rq = __fmul_rn(r, q);
+    const float p = __fmaf_rn(rq, r, r);
+    const float ef = __int2float_rn(e);
+    const float hi = __fmaf_rn(ef, ln2_hi, cl.y);
+    const float lo = __fmaf_rn(ef, ln2_lo, p);
+    return __fadd_rn(hi, lo);
+}
+
+struct NlogCtx {
+    const float2 *tab;
+    float ln2_hi, ln2_lo, one_third;
+    __device__ __forceinline__ float operator()(float x) const {
+        return nlog(x, tab, ln2_hi, ln2_lo, one_third);
+    }
+};
+
+// g = -log(-log eps) for field k (the negations are exact).
+__device__ __forceinline__ float gumbel(uint32_t k, const NlogCtx &L) {
+    const float eps = uniform_from_field(k);
+    const float t = -L(eps);
+    return -L(t);
+}
+
+// Copy the table into shared memory (call with all threads, then __syncthreads()).
+__device__ __forceinline__ void load_tab(float2 *s_tab, const NoiseTab &tab) {
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) s_tab[i] = tab.cl[i];
+}
+
+// ---------------------------------------------------------------------------- misc
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Streaming (evict-first) global accesses for data touched once per call.
+__device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(uint4 *p, uint4 v) { __stcs(p, v); }
+
+}  // namespace mllm

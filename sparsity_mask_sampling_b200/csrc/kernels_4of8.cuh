@@ -1,0 +1,426 @@
+// kernels_4of8.cuh -- the 4:8 sampler kernels (C = 70 candidates per block of 8 weights).
+//
+// MaskLLM (paper-graph-ui summary of arXiv 2409.17481) s.3.2 / s.3.4, generalised from 2:4
+// to 4:8 as the method states (N:M with C(M,N) candidates); the candidate order is the
+// lexicographic order of the ascending position 4-tuples.
+//
+// Work mapping: one thread owns one block and walks all 70 candidates fully unrolled, so
+// every candidate's keep mask is a compile-time constant (no divergence, no table lookups).
+// A block's logits are 280 B, so a thread reading its own row would make each warp access
+// stride 280 B; instead a CTA stages its tile of kBlocksPerCta logit rows through shared
+// memory with coalesced copies, and AdamW runs as a flat, coalesced pass over the tile.
+#pragma once
+
+#include <type_traits>
+
+#include "device_common.cuh"
+
+namespace mllm {
+namespace k48 {
+
+constexpr int C = 70;
+constexpr int kCtaThreads = 128;
+constexpr int kBlocksPerCta = kCtaThreads;  // one block per thread
+constexpr int kTileFloats = kBlocksPerCta * C;
+constexpr int kBwdDynSmem = 2 * kTileFloats * (int)sizeof(float);
+
+// Keep mask (bit j = position j) of candidate i: the i-th 4-subset of {0..7} in
+// lexicographic order of ascending index tuples. Only ever evaluated at compile time.
+__host__ __device__ constexpr uint32_t cand_mask(int i) {
+    int r = 0;
+    for (int a = 0; a < 8; ++a)
+        for (int b = a + 1; b < 8; ++b)
+            for (int c = b + 1; c < 8; ++c)
+                for (int d = c + 1; d < 8; ++d)
+                    if (r++ == i) return (1u << a) | (1u << b) | (1u << c) | (1u << d);
+    return 0u;
+}
+
+// Compile-time loop: f(std::integral_constant<int, I>) for I in [B, E).
+template <int B, int E, class F>
+__device__ __forceinline__ void static_for(F &&f) {
+    if constexpr (B < E) {
+        f(std::integral_constant<int, B>{});
+        static_for<B + 1, E>(f);
+    }
+}
+
+// --------------------------------------------------------------------------- tile staging
+
+// Copy n floats global -> shared (n may be any count; src/dst 8-byte aligned).
+__device__ __forceinline__ void stage_in(float *dst, const float *src, int n) {
+    const int n2 = n >> 1;
+    const float2 *s2 = reinterpret_cast<const float2 *>(src);
+    float2 *d2 = reinterpret_cast<float2 *>(dst);
+    for (int i = threadIdx.x; i < n2; i += kCtaThreads) d2[i] = __ldcs(s2 + i);
+    if ((n & 1) && threadIdx.x == 0) dst[n - 1] = __ldcs(src + n - 1);
+}
+
+__device__ __forceinline__ void stage_out(float *dst, const float *src, int n) {
+    const int n2 = n >> 1;
+    const float2 *s2 = reinterpret_cast<const float2 *>(src);
+    float2 *d2 = reinterpret_cast<float2 *>(dst);
+    for (int i = threadIdx.x; i < n2; i += kCtaThreads) __stcs(d2 + i, s2[i]);
+    if ((n & 1) && threadIdx.x == 0) __stcs(dst + n - 1, src[n - 1]);
+}
+
+template <bool kF32>
+__device__ __forceinline__ void load8(const void *base, int64_t b, float w[8]) {
+    if (kF32) {
+        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + b * 8);
+        const float4 a = ld_stream(p), c = ld_stream(p + 1);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = c.x; w[5] = c.y; w[6] = c.z; w[7] = c.w;
+    } else {
+        const uint4 a = ld_stream(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(base) + b * 8));
+        w[0] = bf16lo(a.x); w[1] = bf16hi(a.x); w[2] = bf16lo(a.y); w[3] = bf16hi(a.y);
+        w[4] = bf16lo(a.z); w[5] = bf16hi(a.z); w[6] = bf16lo(a.w); w[7] = bf16hi(a.w);
+    }
+}
+
+template <bool kF32>
+__device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) {
+    if (kF32) {
+        float4 *p = reinterpret_cast<float4 *>(static_cast<float *>(base) + b * 8);
+        st_stream(p, make_float4(x[0], x[1], x[2], x[3]));
+        st_stream(p + 1, make_float4(x[4], x[5], x[6], x[7]));
+    } else {
+        st_stream(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(base) + b * 8),
+                  make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7])));
+    }
+}
+
+// --------------------------------------------------------------------------- per-block math
+
+// Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates, and their maximum.
+__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t seed, uint64_t gid,
+                                           const StepScalars &sc, const NlogCtx &L, float w[C]) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int gr = 0; gr < 12; ++gr) {
+        uint32_t f[6];
+        if (sc.noise_on) fields21(block_words(seed, gid, sc.step, (uint32_t)gr), f);
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int c = 6 * gr + k;
+            if (c < C) {
+                const float g = sc.noise_on ? gumbel(f[k], L) : 0.f;
+                w[c] = __fmaf_rn(sc.kappa, pi_row[c], g);
+                mx = fmaxf(mx, w[c]);
+            }
+        }
+    }
+    return mx;
+}
+
+// e_c = 2^((w_c - max) c2) in place; returns sum e; ms[j] = sum_{c: j in S_c} e_c and, when
+// kComp, mc[j] = sum_{c: j not in S_c} e_c.
+template <bool kComp>
+__device__ __forceinline__ float soft_sums(float w[C], float mx, float c2, float ms[8], float mc[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { ms[j] = 0.f; mc[j] = 0.f; }
+    float s = 0.f;
+    static_for<0, C>([&](auto I) {
+        constexpr int c = decltype(I)::value;
+        constexpr uint32_t mk = cand_mask(c);
+        const float e = ex2_approx(__fmul_rn(__fsub_rn(w[c], mx), c2));
+        w[c] = e;
+        s += e;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (mk & (1u << j)) ms[j] += e;
+            else if (kComp) mc[j] += e;
+        }
+    });
+    return s;
+}
+
+// --------------------------------------------------------------------------- kernels
+
+template <bool kW32>
+__global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant__ Group grp,
+                                                          const __grid_constant__ NoiseTab tab,
+                                                          const StepScalars sc, double *partials,
+                                                          unsigned int *ticket, double *reg_out,
+                                                          int accumulate) {
+    __shared__ float2 s_tab[128];
+    __shared__ __align__(16) float s_pi[kTileFloats];
+    load_tab(s_tab, tab);
+    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    float acc = 0.f;
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
+        const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
+        __syncthreads();  // previous tile's readers are done (and the table is loaded)
+        stage_in(s_pi, d.pi + tb0 * C, nb * C);
+        __syncthreads();
+        if ((int)threadIdx.x < nb) {
+            const int64_t b = tb0 + threadIdx.x;
+            float w[C], ms[8], mc[8], wt[8];
+            const float mx = perturbed(s_pi + threadIdx.x * C, sc.seed, d.gid0 + b, sc, L, w);
+            load8<kW32>(d.W, b, wt);
+            const float r = rcp_approx(soft_sums<false>(w, mx, sc.c2, ms, mc));
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                ms[j] = __fmul_rn(ms[j], r);
+                x[j] = __fmul_rn(wt[j], ms[j]);
+                acc = __fmaf_rn(x[j], x[j], acc);
+            }
+            store8<kW32>(d.X, b, x);
+            if (d.soft) {
+                float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
+                sp[0] = make_float4(ms[0], ms[1], ms[2], ms[3]);
+                sp[1] = make_float4(ms[4], ms[5], ms[6], ms[7]);
+            }
+        }
+    }
+    if (reg_out) {
+        // CTA-level deterministic reduction, then the last CTA combines all partials.
+        __shared__ double s_w[kCtaThreads / 32];
+        __shared__ bool s_last;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        __syncthreads();
+        if (lane == 0) s_w[warp] = (double)acc;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double tt = 0.0;
+            for (int i = 0; i < kCtaThreads / 32; ++i) tt += s_w[i];
+            partials[blockIdx.x] = tt;
+            __threadfence();
+            s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1);
+        }
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        double tt = 0.0;
+        for (unsigned int i = threadIdx.x; i < gridDim.x; i += kCtaThreads) tt += __ldcg(partials + i);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tt += __shfl_xor_sync(0xFFFFFFFFu, tt, o);
+        __syncthreads();
+        if (lane == 0) s_w[warp] = tt;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double tot = 0.0;
+            for (int i = 0; i < kCtaThreads / 32; ++i) tot += s_w[i];
+            *reg_out = accumulate ? (*reg_out + tot) : tot;
+            *ticket = 0u;
+        }
+    }
+}
+
+template <bool kW32, bool kG32>
+__global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_constant__ Group grp,
+                                                               const __grid_constant__ NoiseTab tab,
+                                                               const StepScalars sc) {
+    __shared__ float2 s_tab[128];
+    extern __shared__ __align__(16) float s_dyn[];  // [2 * kTileFloats]: logits, gradients
+    float *s_pi = s_dyn, *s_gr = s_dyn + kTileFloats;
+    load_tab(s_tab, tab);
+    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
+        const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
+        __syncthreads();
+        stage_in(s_pi, d.pi + tb0 * C, nb * C);
+        __syncthreads();
+        if ((int)threadIdx.x < nb) {
+            const int64_t b = tb0 + threadIdx.x;
+            float w[C], ms[8], mc[8], wt[8], gw[8];
+            const float mx = perturbed(s_pi + threadIdx.x * C, sc.seed, d.gid0 + b, sc, L, w);
+            load8<kW32>(d.W, b, wt);
+            load8<kG32>(d.G, b, gw);
+            const float r = rcp_approx(soft_sums<true>(w, mx, sc.c2, ms, mc));
+            float P[8], Q[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                ms[j] = __fmul_rn(ms[j], r);
+                mc[j] = __fmul_rn(mc[j], r);
+                const float wj = wt[j];
+                const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j],
+                                          __fmul_rn(gw[j], wj));
+                P[j] = __fmul_rn(mc[j], u);
+                Q[j] = __fmul_rn(ms[j], u);
+            }
+            const float cr = __fmul_rn(sc.kappa_over_tau, r);
+            float *grow = s_gr + threadIdx.x * C;
+            static_for<0, C>([&](auto I) {
+                constexpr int c = decltype(I)::value;
+                constexpr uint32_t mk = cand_mask(c);
+                float kept = 0.f, pruned = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (mk & (1u << j)) kept += P[j];
+                    else pruned += Q[j];
+                }
+                grow[c] = __fmul_rn(__fmul_rn(cr, w[c]), kept - pruned);
+            });
+        }
+        __syncthreads();
+        // AdamW over the tile as one flat, coalesced array.
+        const int n = nb * C;
+        float *pi = d.pi + tb0 * C, *mm = d.m + tb0 * C, *vv = d.v + tb0 * C;
+        float *gout = d.grad ? d.grad + tb0 * C : nullptr;
+        for (int i = threadIdx.x; i < n; i += kCtaThreads) {
+            float p = s_pi[i], m = __ldcs(mm + i), v = __ldcs(vv + i);
+            const float g = s_gr[i];
+            const float pd = __fmul_rn(p, sc.decay);
+            m = __fmaf_rn(sc.beta1, m, __fmul_rn(sc.one_minus_beta1, g));
+            v = __fmaf_rn(sc.beta2, v, __fmul_rn(sc.one_minus_beta2, __fmul_rn(g, g)));
+            const float denom = __fmaf_rn(__fsqrt_rn(v), sc.inv_sqrt_bc2, sc.eps);
+            p = __fmaf_rn(-sc.step_size, __fdividef(m, denom), pd);
+            __stcs(pi + i, p);
+            __stcs(mm + i, m);
+            __stcs(vv + i, v);
+            if (gout) __stcs(gout + i, g);
+        }
+    }
+}
+
+template <bool kW32>
+__global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constant__ Group grp,
+                                                            float alpha, float init_std, uint64_t seed) {
+    __shared__ __align__(16) float s_pi[kTileFloats];
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
+        const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
+        __syncthreads();
+        if ((int)threadIdx.x < nb) {
+            const int64_t b = tb0 + threadIdx.x;
+            float wt[8], key[8];
+            load8<kW32>(d.W, b, wt);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) key[j] = (wt[j] != wt[j]) ? -1.0f : fabsf(wt[j]);
+            uint32_t m0 = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                int rank = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k != j && (key[k] > key[j] || (key[k] == key[j] && k < j))) ++rank;
+                if (rank < 4) m0 |= 1u << j;
+            }
+            float *row = s_pi + threadIdx.x * C;
+            if (init_std == 0.f) {
+                static_for<0, C>([&](auto I) {
+                    constexpr int c = decltype(I)::value;
+                    row[c] = alpha * ((float)__popc(m0 & cand_mask(c)) - 2.0f);
+                });
+            } else {
+                float mu = 0.f;
+#pragma unroll
+                for (int gr = 0; gr < 12; ++gr) {
+                    uint32_t f[6];
+                    fields21(block_words(seed, d.gid0 + b, kInitStep, (uint32_t)gr), f);
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        const int c = 6 * gr + 2 * q;
+                        if (c < C) {
+                            const float u1 = uniform_from_field(f[2 * q]);
+                            const float u2 = uniform_from_field(f[2 * q + 1]);
+                            const float rad = sqrtf(-2.0f * logf(u1));
+                            float sn, cs;
+                            sincospif(2.0f * u2, &sn, &cs);
+                            row[c] = init_std * (rad * cs);
+                            row[c + 1] = init_std * (rad * sn);
+                            mu += row[c] + row[c + 1];
+                        }
+                    }
+                }
+                mu *= (1.0f / C);
+                float var = 0.f;
+                for (int c = 0; c < C; ++c) var = fmaf(row[c] - mu, row[c] - mu, var);
+                const float as = alpha * sqrtf(var * (1.0f / C));
+                static_for<0, C>([&](auto I) {
+                    constexpr int c = decltype(I)::value;
+                    row[c] = fmaf(as, (float)__popc(m0 & cand_mask(c)) - 2.0f, row[c]);
+                });
+            }
+        }
+        __syncthreads();
+        const int n = nb * C;
+        stage_out(d.pi + tb0 * C, s_pi, n);
+        for (int i = threadIdx.x; i < n; i += kCtaThreads) {
+            if (d.m) __stcs(d.m + tb0 * C + i, 0.f);
+            if (d.v) __stcs(d.v + tb0 * C + i, 0.f);
+        }
+    }
+}
+
+// Hard pack: one thread per block (tile staged through shared memory).
+template <bool kW32>
+__global__ void __launch_bounds__(kCtaThreads) pack_kernel(const __grid_constant__ Group grp) {
+    __shared__ __align__(16) float s_pi[kTileFloats];
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
+        const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
+        __syncthreads();
+        stage_in(s_pi, d.pi + tb0 * C, nb * C);
+        __syncthreads();
+        if ((int)threadIdx.x >= nb) continue;
+        const int64_t b = tb0 + threadIdx.x;
+        const float *row = s_pi + threadIdx.x * C;
+        int k = -1;
+        float best = 0.f;
+        for (int c = 0; c < C; ++c) {
+            const float p = row[c];
+            if (p == p && (k < 0 || p > best)) { k = c; best = p; }
+        }
+        if (k < 0) k = 0;
+        uint32_t mask = 0;
+        static_for<0, C>([&](auto I) {
+            constexpr int c = decltype(I)::value;
+            if (c == k) mask = cand_mask(c);
+        });
+        int pos[4], n = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) if (mask & (1u << j)) pos[n++ & 3] = j;
+        static_cast<uint16_t *>(d.pmeta)[b] = (uint16_t)(pos[0] | (pos[1] << 3) | (pos[2] << 6) | (pos[3] << 9));
+        if (d.cidx) d.cidx[b] = (uint8_t)k;
+        if (kW32) {
+            const float *W = static_cast<const float *>(d.W) + b * 8;
+            float4 o = make_float4(__ldcs(W + pos[0]), __ldcs(W + pos[1]), __ldcs(W + pos[2]), __ldcs(W + pos[3]));
+            __stcs(reinterpret_cast<float4 *>(static_cast<float *>(d.pvals) + b * 4), o);
+        } else {
+            const uint4 a = ld_stream(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(d.W) + b * 8));
+            const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+            uint32_t h[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) h[q] = (wv[pos[q] >> 1] >> (16 * (pos[q] & 1))) & 0xFFFFu;
+            __stcs(reinterpret_cast<uint2 *>(static_cast<uint16_t *>(d.pvals) + b * 4),
+                   make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16)));
+        }
+    }
+}
+
+}  // namespace k48
+
+// Gumbel noise of arbitrary blocks for inspection: one thread per block, C values each.
+__global__ void __launch_bounds__(kThreads) noise_kernel(const __grid_constant__ NoiseTab tab, int C,
+                                                         uint64_t seed, uint32_t step,
+                                                         const uint64_t *__restrict__ gids,
+                                                         int64_t n, float *__restrict__ out) {
+    __shared__ float2 s_tab[128];
+    load_tab(s_tab, tab);
+    __syncthreads();
+    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint64_t gid = gids[i];
+        for (int gr = 0; gr * 6 < C; ++gr) {
+            uint32_t f[6];
+            fields21(block_words(seed, gid, step, (uint32_t)gr), f);
+            for (int k = 0; k < 6; ++k) {
+                const int c = 6 * gr + k;
+                if (c < C) out[i * C + c] = gumbel(f[k], L);
+            }
+        }
+    }
+}
+
+}  // namespace mllm

@@ -1,0 +1,426 @@
+// mllm.cu -- host side of libmllm: argument validation, grouping, launch configuration and
+// the extern "C" entry points declared in include/mllm.h.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "mllm.h"
+#include "device_common.cuh"
+#include "kernels_2of4.cuh"
+#include "kernels_4of8.cuh"
+
+namespace mllm {
+namespace {
+
+thread_local int32_t g_last_cuda = 0;
+
+// Workspace layout of the forward's regulariser reduction: a ticket word, then one double
+// per CTA of the launch (the forward grid is capped at kMaxReduceCtas).
+constexpr int kMaxReduceCtas = 4096;
+constexpr size_t kWsPartialsOffset = 16;
+constexpr size_t kWorkspaceBytes = kWsPartialsOffset + sizeof(double) * kMaxReduceCtas;
+
+// ------------------------------------------------------------------------ noise table
+
+NoiseTab build_noise_tab() {
+    NoiseTab t{};
+    for (int j = 0; j < 128; ++j) {
+        const double F = (j < 64) ? (1.0 + j / 128.0) : (1.0 + j / 128.0) * 0.5;
+        const float c = (float)(1.0 / F);
+        t.cl[j] = make_float2(c, (float)(-std::log((double)c)));
+    }
+    const double ln2 = std::log(2.0);
+    float hi = (float)ln2;
+    uint32_t bits;
+    std::memcpy(&bits, &hi, 4);
+    bits &= 0xFFFFFF00u;  // clear 8 low mantissa bits: e * ln2_hi exact for |e| < 256
+    std::memcpy(&hi, &bits, 4);
+    t.ln2_hi = hi;
+    t.ln2_lo = (float)(ln2 - (double)hi);
+    t.one_third = (float)(1.0 / 3.0);
+    return t;
+}
+
+const NoiseTab &noise_tab() {
+    static const NoiseTab tab = build_noise_tab();
+    return tab;
+}
+
+// ------------------------------------------------------------------------ device info
+
+struct OccKey {
+    int dev;
+    const void *fn;
+};
+std::mutex g_occ_mu;
+std::vector<std::pair<OccKey, int>> g_occ;  // (device, kernel) -> resident CTAs per SM
+std::vector<int> g_sms;
+
+int sm_count(int dev) {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    if ((int)g_sms.size() <= dev) g_sms.resize(dev + 1, 0);
+    if (!g_sms[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 1;
+        g_sms[dev] = n;
+    }
+    return g_sms[dev];
+}
+
+// Resident CTAs per SM of a kernel on a device (first use also raises the kernel's dynamic
+// shared-memory limit when it needs more than the 48 KB default).
+int resident_ctas(int dev, const void *fn, int threads, int dyn_smem) {
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        for (auto &e : g_occ)
+            if (e.first.dev == dev && e.first.fn == fn) return e.second;
+    }
+    if (dyn_smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, dyn_smem) != cudaSuccess || n <= 0) n = 1;
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    g_occ.push_back({OccKey{dev, fn}, n});
+    return n;
+}
+
+int64_t grid_for(const void *fn, int threads, int dyn_smem, int64_t work, int64_t cap) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int64_t g = (int64_t)sm_count(dev) * resident_ctas(dev, fn, threads, dyn_smem);
+    return std::max<int64_t>(1, std::min<int64_t>({work, g, cap}));
+}
+
+mllm_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MLLM_OK;
+    g_last_cuda = (int32_t)e;
+    return MLLM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------ validation
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+enum Need : unsigned {
+    kNeedW = 1, kNeedX = 2, kNeedG = 4, kNeedPi = 8, kNeedMV = 16, kNeedPack = 32,
+};
+
+int num_cand(mllm_nm nm) {
+    if (nm.n == 2 && nm.m == 4) return 6;
+    if (nm.n == 4 && nm.m == 8) return 70;
+    return 0;
+}
+
+mllm_status check_ptr(const void *p, bool required) {
+    if (!p) return required ? MLLM_ERR_INVALID_ARG : MLLM_OK;
+    return aligned16(p) ? MLLM_OK : MLLM_ERR_MISALIGNED;
+}
+
+mllm_status validate_mats(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, unsigned need) {
+    if (!num_cand(nm)) return MLLM_ERR_UNSUPPORTED;
+    if (!mats || n_mats <= 0) return MLLM_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_mats; ++i) {
+        const mllm_matrix &a = mats[i];
+        if (a.rows < 0 || a.cols < 0 || a.cols % nm.m) return MLLM_ERR_INVALID_ARG;
+        if (a.rows > 0 && a.cols > ((int64_t)1 << 62) / a.rows) return MLLM_ERR_INVALID_ARG;
+        if (a.w_dtype != MLLM_BF16 && a.w_dtype != MLLM_F32) return MLLM_ERR_UNSUPPORTED;
+        if (a.w_dtype != mats[0].w_dtype) return MLLM_ERR_UNSUPPORTED;
+        if (need & kNeedG) {
+            if (a.g_dtype != MLLM_BF16 && a.g_dtype != MLLM_F32) return MLLM_ERR_UNSUPPORTED;
+            if (a.g_dtype != mats[0].g_dtype) return MLLM_ERR_UNSUPPORTED;
+        }
+        const bool any = a.rows > 0 && a.cols > 0;
+        mllm_status s;
+        if ((s = check_ptr(a.W, any && (need & kNeedW))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.X_out, any && (need & kNeedX))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.G, any && (need & kNeedG))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.logits, any && (need & kNeedPi))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.adam_m, any && (need & kNeedMV))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.adam_v, any && (need & kNeedMV))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.soft_mask_out, false)) != MLLM_OK) return s;
+        if ((s = check_ptr(a.grad_logits_out, false)) != MLLM_OK) return s;
+        if ((s = check_ptr(a.pack_values, any && (need & kNeedPack))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.pack_meta, any && (need & kNeedPack))) != MLLM_OK) return s;
+        if ((s = check_ptr(a.cand_idx_out, false)) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+bool finite(float x) { return std::isfinite(x); }
+
+mllm_status validate_fwd_hp(const mllm_hparams *hp) {
+    if (!hp) return MLLM_ERR_INVALID_ARG;
+    if (!finite(hp->kappa) || !(hp->kappa > 0.f)) return MLLM_ERR_INVALID_ARG;
+    if (!finite(hp->tau) || !(hp->tau > 0.f)) return MLLM_ERR_INVALID_ARG;
+    if (hp->step == kInitStep || hp->reserved != 0) return MLLM_ERR_INVALID_ARG;
+    const double c2 = 1.4426950408889634 / (double)hp->tau;
+    const double kt = (double)hp->kappa / (double)hp->tau;
+    if (!std::isfinite((float)c2) || !std::isfinite((float)kt)) return MLLM_ERR_INVALID_ARG;
+    return MLLM_OK;
+}
+
+mllm_status validate_bwd_hp(const mllm_hparams *hp) {
+    mllm_status s = validate_fwd_hp(hp);
+    if (s != MLLM_OK) return s;
+    if (!finite(hp->lambda) || hp->lambda < 0.f) return MLLM_ERR_INVALID_ARG;
+    if (!finite(hp->lr) || hp->lr < 0.f) return MLLM_ERR_INVALID_ARG;
+    if (!(hp->beta1 >= 0.f && hp->beta1 < 1.f)) return MLLM_ERR_INVALID_ARG;
+    if (!(hp->beta2 >= 0.f && hp->beta2 < 1.f)) return MLLM_ERR_INVALID_ARG;
+    if (!finite(hp->eps) || !(hp->eps > 0.f)) return MLLM_ERR_INVALID_ARG;
+    if (!finite(hp->weight_decay) || hp->weight_decay < 0.f) return MLLM_ERR_INVALID_ARG;
+    if (hp->adam_step < 1) return MLLM_ERR_INVALID_ARG;
+    return MLLM_OK;
+}
+
+StepScalars make_scalars(const mllm_hparams &hp) {
+    StepScalars s{};
+    const double t = (double)hp.adam_step;
+    s.kappa = hp.kappa;
+    s.c2 = (float)(1.4426950408889634 / (double)hp.tau);
+    s.kappa_over_tau = (float)((double)hp.kappa / (double)hp.tau);
+    s.two_lambda = 2.0f * hp.lambda;
+    s.decay = (float)(1.0 - (double)hp.lr * (double)hp.weight_decay);
+    s.beta1 = hp.beta1;
+    s.one_minus_beta1 = (float)(1.0 - (double)hp.beta1);
+    s.beta2 = hp.beta2;
+    s.one_minus_beta2 = (float)(1.0 - (double)hp.beta2);
+    const double bc1 = 1.0 - std::pow((double)hp.beta1, t);
+    const double bc2 = 1.0 - std::pow((double)hp.beta2, t);
+    s.step_size = (bc1 > 0.0) ? (float)((double)hp.lr / bc1) : 0.f;
+    s.inv_sqrt_bc2 = (bc2 > 0.0) ? (float)(1.0 / std::sqrt(bc2)) : 0.f;
+    s.eps = hp.eps;
+    s.step = hp.step;
+    s.noise_on = hp.noise_on ? 1u : 0u;
+    s.seed = hp.seed;
+    return s;
+}
+
+// ------------------------------------------------------------------------ grouping
+
+MatDesc make_desc(const mllm_matrix &a, int M) {
+    MatDesc d{};
+    d.W = a.W; d.X = a.X_out; d.G = a.G;
+    d.pi = a.logits; d.m = a.adam_m; d.v = a.adam_v;
+    d.soft = a.soft_mask_out; d.grad = a.grad_logits_out;
+    d.pvals = a.pack_values; d.pmeta = a.pack_meta; d.cidx = a.cand_idx_out;
+    d.rows = a.rows; d.cols = a.cols;
+    d.nblocks = (a.rows > 0 && a.cols > 0) ? a.rows * (a.cols / M) : 0;
+    d.gid0 = a.block_offset;
+    d.w_f32 = a.w_dtype == MLLM_F32;
+    d.g_f32 = a.g_dtype == MLLM_F32;
+    return d;
+}
+
+// Work units of one matrix for a kernel kind.
+enum class Kind { Sample24, Pack24, Sample48, Pack48 };
+
+int64_t work_units(const MatDesc &d, Kind k) {
+    if (d.nblocks == 0) return 0;
+    switch (k) {
+        case Kind::Sample24: {
+            const int64_t pairs = (d.nblocks + 1) / 2;
+            return (pairs + kThreads - 1) / kThreads;
+        }
+        case Kind::Pack24: {
+            const int64_t bpr = d.cols / 4, words = d.rows * ((bpr + 7) / 8);
+            return (words + kThreads - 1) / kThreads;
+        }
+        case Kind::Sample48:
+            return (d.nblocks + k48::kBlocksPerCta - 1) / k48::kBlocksPerCta;
+        case Kind::Pack48:
+            return (d.nblocks + k48::kBlocksPerCta - 1) / k48::kBlocksPerCta;
+    }
+    return 0;
+}
+
+// Split the call into groups of at most kMaxMats matrices with their work prefix sums.
+std::vector<Group> make_groups(const mllm_matrix *mats, int32_t n_mats, int M, Kind k) {
+    std::vector<Group> out;
+    for (int32_t i0 = 0; i0 < n_mats; i0 += kMaxMats) {
+        Group g{};
+        const int32_t n = std::min<int32_t>(kMaxMats, n_mats - i0);
+        int64_t acc = 0;
+        for (int32_t i = 0; i < n; ++i) {
+            MatDesc d = make_desc(mats[i0 + i], M);
+            d.work_begin = acc;
+            d.work_count = work_units(d, k);
+            acc += d.work_count;
+            g.d[i] = d;
+        }
+        g.n = n;
+        g.total_work = acc;
+        out.push_back(g);
+    }
+    return out;
+}
+
+}  // namespace
+}  // namespace mllm
+
+using namespace mllm;
+
+extern "C" {
+
+int32_t mllm_num_candidates(mllm_nm nm) { return num_cand(nm); }
+
+size_t mllm_workspace_bytes(void) { return kWorkspaceBytes; }
+
+int32_t mllm_abi_version(void) { return MLLM_ABI_VERSION; }
+size_t mllm_sizeof_matrix(void) { return sizeof(mllm_matrix); }
+size_t mllm_sizeof_hparams(void) { return sizeof(mllm_hparams); }
+int32_t mllm_last_cuda_error(void) { return g_last_cuda; }
+
+const char *mllm_status_string(mllm_status s) {
+    switch (s) {
+        case MLLM_OK: return "ok";
+        case MLLM_ERR_INVALID_ARG: return "invalid argument";
+        case MLLM_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+        case MLLM_ERR_UNSUPPORTED: return "unsupported N:M pattern or dtype";
+        case MLLM_ERR_WORKSPACE: return "workspace missing or too small";
+        case MLLM_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+mllm_status mllm_prior_init(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, float alpha,
+                            float init_std, uint64_t seed, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedPi);
+    if (s != MLLM_OK) return s;
+    if (!finite(alpha) || alpha < 0.f || !finite(init_std) || init_std < 0.f) return MLLM_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool w32 = mats[0].w_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
+    for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48)) {
+        if (g.total_work == 0) continue;
+        if (is24) {
+            const void *fn = w32 ? (const void *)k24::prior_kernel<true> : (const void *)k24::prior_kernel<false>;
+            const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k24::prior_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, alpha, init_std, seed);
+            else k24::prior_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, alpha, init_std, seed);
+        } else {
+            const void *fn = w32 ? (const void *)k48::prior_kernel<true> : (const void *)k48::prior_kernel<false>;
+            const int64_t grid = grid_for(fn, k48::kCtaThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k48::prior_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, alpha, init_std, seed);
+            else k48::prior_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, alpha, init_std, seed);
+        }
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                            const mllm_hparams *hp, double *reg_sum_out, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedX | kNeedPi);
+    if (s != MLLM_OK) return s;
+    if ((s = validate_fwd_hp(hp)) != MLLM_OK) return s;
+    if (reg_sum_out) {
+        if ((reinterpret_cast<uintptr_t>(reg_sum_out) & 7u) != 0) return MLLM_ERR_MISALIGNED;
+        if (!workspace || workspace_bytes < kWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StepScalars sc = make_scalars(*hp);
+    const bool w32 = mats[0].w_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
+    unsigned int *ticket = reg_sum_out ? static_cast<unsigned int *>(workspace) : nullptr;
+    double *partials = reg_sum_out ? reinterpret_cast<double *>(static_cast<char *>(workspace) + kWsPartialsOffset) : nullptr;
+    bool wrote_reg = false;
+    for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48)) {
+        if (g.total_work == 0) continue;
+        const int accumulate = wrote_reg ? 1 : 0;
+        if (is24) {
+            const void *fn = w32 ? (const void *)k24::fwd_kernel<true> : (const void *)k24::fwd_kernel<false>;
+            const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, kMaxReduceCtas);
+            if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+        } else {
+            const void *fn = w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>;
+            const int64_t grid = grid_for(fn, k48::kCtaThreads, 0, g.total_work, kMaxReduceCtas);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+        }
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+        wrote_reg = true;
+    }
+    if (reg_sum_out && !wrote_reg) {
+        if ((s = cuda_status(cudaMemsetAsync(reg_sum_out, 0, sizeof(double), st))) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                 const mllm_hparams *hp, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedG | kNeedPi | kNeedMV);
+    if (s != MLLM_OK) return s;
+    if ((s = validate_bwd_hp(hp)) != MLLM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StepScalars sc = make_scalars(*hp);
+    const bool w32 = mats[0].w_dtype == MLLM_F32, g32 = mats[0].g_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
+    for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48)) {
+        if (g.total_work == 0) continue;
+#define MLLM_LAUNCH_BWD(NS, THREADS, SMEM, W32, G32)                                              \
+    do {                                                                                         \
+        const void *fn = (const void *)NS::bwd_adam_kernel<W32, G32>;                            \
+        const int64_t grid = grid_for(fn, THREADS, SMEM, g.total_work, INT32_MAX);                 \
+        NS::bwd_adam_kernel<W32, G32><<<(unsigned)grid, THREADS, SMEM, st>>>(g, noise_tab(), sc); \
+    } while (0)
+        if (is24) {
+            if (w32 && g32) MLLM_LAUNCH_BWD(k24, kThreads, 0, true, true);
+            else if (w32) MLLM_LAUNCH_BWD(k24, kThreads, 0, true, false);
+            else if (g32) MLLM_LAUNCH_BWD(k24, kThreads, 0, false, true);
+            else MLLM_LAUNCH_BWD(k24, kThreads, 0, false, false);
+        } else {
+            if (w32 && g32) MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, true);
+            else if (w32) MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, false);
+            else if (g32) MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, true);
+            else MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, false);
+        }
+#undef MLLM_LAUNCH_BWD
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedPi | kNeedPack);
+    if (s != MLLM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool w32 = mats[0].w_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
+    for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Pack24 : Kind::Pack48)) {
+        if (g.total_work == 0) continue;
+        if (is24) {
+            const void *fn = w32 ? (const void *)k24::pack_kernel<true> : (const void *)k24::pack_kernel<false>;
+            const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k24::pack_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g);
+            else k24::pack_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g);
+        } else {
+            const void *fn = w32 ? (const void *)k48::pack_kernel<true> : (const void *)k48::pack_kernel<false>;
+            const int64_t grid = grid_for(fn, k48::kCtaThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k48::pack_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g);
+            else k48::pack_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g);
+        }
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t *gids,
+                       int64_t n_blocks, float *g_out, void *stream) {
+    const int C = num_cand(nm);
+    if (!C) return MLLM_ERR_UNSUPPORTED;
+    if (n_blocks < 0) return MLLM_ERR_INVALID_ARG;
+    if (n_blocks == 0) return MLLM_OK;
+    mllm_status s;
+    if ((s = check_ptr(gids, true)) != MLLM_OK) return s;
+    if ((s = check_ptr(g_out, true)) != MLLM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t grid = std::min<int64_t>((n_blocks + kThreads - 1) / kThreads, INT32_MAX);
+    noise_kernel<<<(unsigned)grid, kThreads, 0, st>>>(noise_tab(), C, seed, step, gids, n_blocks, g_out);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

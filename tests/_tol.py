@@ -1,0 +1,85 @@
+"""Parity tolerances between the CUDA path and the oracle.
+
+The bars are the stated ones: bit-exact for integer/index work (noise bits, hard masks,
+packed values and metadata); soft masks 1e-5 relative; W.M within 1 bf16 ulp (1e-5 relative
+when W is fp32); logit gradients and AdamW-updated logits 1e-4 relative; the regulariser
+1e-3 relative. How "relative" is read:
+  * soft mask: element-wise, |dM_j| <= 1e-5 M_ref_j (a sum of positive weights);
+  * gradient: a signed sum of terms, so relative to the magnitude of its summands,
+    |dg_i| <= 1e-4 (kappa/tau) y_i sum_j |S_ij - M_j| |u_j| (the oracle's `scale`);
+  * updated logits: relative to the block, |dpi_i| <= 1e-4 max_k |pi_ref_k|.
+Every bound also admits an absolute floor 1e-30 times the block's natural scale: fp32 soft
+index weights below 2^-126 flush to zero on the GPU (exp2 approximation with ftz) where the
+fp64 oracle keeps them; such differences are representational, not arithmetic.
+"""
+import numpy as np
+
+FLOOR = 1e-30
+
+
+def bf16_ulp(x):
+    """Spacing of bfloat16 numbers at |x| (8 significant bits, fp32 exponent range)."""
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -126)
+    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def assert_x_close(x_gpu, x_ref, w_dtype, W):
+    """Soft-masked weights: 1 bf16 ulp (bf16) or 1e-5 relative (fp32), floor |W| 1e-30."""
+    x_gpu = np.asarray(x_gpu, np.float64)
+    x_ref = np.asarray(x_ref, np.float64)
+    err = np.abs(x_gpu - x_ref)
+    if w_dtype == "bf16":
+        tol = bf16_ulp(x_ref)
+    else:
+        tol = 1e-5 * np.abs(x_ref)
+    tol = tol + FLOOR * np.abs(W)
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} X mismatches, worst {np.max(err / np.maximum(tol, 1e-300)):.3g} x tol"
+
+
+def assert_soft_close(ms_gpu, ms_ref):
+    err = np.abs(np.asarray(ms_gpu, np.float64) - ms_ref)
+    tol = 1e-5 * ms_ref + FLOOR
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} soft-mask mismatches, worst {np.max(err / tol):.3g} x tol"
+    return float(np.max(err / np.maximum(ms_ref, 1e-300)))
+
+
+def grad_floor(W, G, kappa, tau, lam):
+    """Per-block floor: 1e-30 (kappa/tau) sum_j (|G_j W_j| + 2 lambda W_j^2)."""
+    W = np.asarray(W, np.float64)
+    G = np.asarray(G, np.float64)
+    return FLOOR * (kappa / tau) * (np.abs(G * W) + 2 * lam * W * W).sum(1, keepdims=True)
+
+
+def assert_grad_close(g_gpu, g_ref, scale, floor):
+    err = np.abs(np.asarray(g_gpu, np.float64) - g_ref)
+    tol = 1e-4 * scale + floor
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} gradient mismatches, worst {np.max(err / tol):.3g} x tol"
+    return float(np.max(err / np.maximum(scale, 1e-300)))
+
+
+def assert_logits_close(p_gpu, p_ref):
+    p_ref = np.asarray(p_ref, np.float64)
+    err = np.abs(np.asarray(p_gpu, np.float64) - p_ref)
+    tol = 1e-4 * np.abs(p_ref).max(1, keepdims=True) + FLOOR
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} updated-logit mismatches, worst {np.max(err / tol):.3g} x tol"
+
+
+def assert_moments_close(m_gpu, v_gpu, m_ref, v_ref, g_ref, g_tol, beta1, beta2):
+    """AdamW moments carry the gradient's tolerance: dm <= (1-b1) dg, dv <= (1-b2)(2|g| dg + dg^2),
+    plus fp32 rounding (2^-22 relative)."""
+    m_err = np.abs(np.asarray(m_gpu, np.float64) - m_ref)
+    v_err = np.abs(np.asarray(v_gpu, np.float64) - v_ref)
+    m_tol = (1 - beta1) * g_tol + 2.0**-22 * np.abs(m_ref) + FLOOR
+    v_tol = (1 - beta2) * (2 * np.abs(g_ref) * g_tol + g_tol**2) + 2.0**-22 * v_ref + 1e-45
+    assert not (m_err > m_tol).any(), f"{(m_err > m_tol).sum()} first-moment mismatches"
+    assert not (v_err > v_tol).any(), f"{(v_err > v_tol).sum()} second-moment mismatches"
+
+
+def assert_reg_close(r_gpu, r_ref):
+    assert abs(r_gpu - r_ref) <= 1e-3 * abs(r_ref), (r_gpu, r_ref)

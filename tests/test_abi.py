@@ -1,0 +1,155 @@
+"""The C ABI library loads, exports every declared symbol, and rejects bad arguments on the
+host before touching a device (these calls make no CUDA call and run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    from sparsity_mask_sampling_b200 import _mllm
+    from sparsity_mask_sampling_b200.build import build
+
+    build()
+    _mllm.lib()
+    return _mllm
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(mllm_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(M):
+    names = _declared_functions()
+    assert len(names) >= 12, names
+    h = ctypes.CDLL(M.LIB_PATH)
+    for n in names:
+        assert hasattr(h, n), n
+
+
+def test_abi_guards(M):
+    L = M.lib()
+    assert L.mllm_abi_version() == M.ABI_VERSION
+    assert L.mllm_sizeof_matrix() == ctypes.sizeof(M.Matrix)
+    assert L.mllm_sizeof_hparams() == ctypes.sizeof(M.HParams)
+    assert M.mllm_workspace_bytes() >= 16 + 8 * 148
+
+
+def test_num_candidates(M):
+    assert M.mllm_num_candidates((2, 4)) == 6
+    assert M.mllm_num_candidates((4, 8)) == 70
+    assert M.mllm_num_candidates((1, 4)) == 0
+    assert M.mllm_num_candidates((2, 8)) == 0
+
+
+def test_status_strings(M):
+    for s in range(6):
+        assert M.mllm_status_string(s)
+
+
+def _mat(M, **kw):
+    base = dict(W=0x1000, X_out=0x2000, G=0x3000, w_dtype=0, g_dtype=0, rows=4, cols=8,
+                logits=0x4000, adam_m=0x5000, adam_v=0x6000, block_offset=0,
+                soft_mask_out=0, grad_logits_out=0, pack_values=0x7000, pack_meta=0x8000,
+                cand_idx_out=0)
+    base.update(kw)
+    return M.Matrix(**base)
+
+
+def _hp(M, **kw):
+    base = dict(kappa=100.0, tau=4.0, lambda_=1e-5, lr=5e-4, beta1=0.9, beta2=0.999, eps=1e-8,
+                weight_decay=0.1, adam_step=1, step=0, seed=0, noise_on=1, reserved=0)
+    base.update(kw)
+    return M.HParams(**base)
+
+
+def _fwd(M, mats, hp, nm=(2, 4), reg=0, ws=0x9000, wsb=None):
+    L = M.lib()
+    arr = (M.Matrix * len(mats))(*mats)
+    wsb = M.mllm_workspace_bytes() if wsb is None else wsb
+    return L.mllm_sample_fwd(ctypes.cast(arr, ctypes.c_void_p), len(mats), M.NM(*nm),
+                             ctypes.byref(hp), reg, ws, wsb, 0)
+
+
+def _bwd(M, mats, hp, nm=(2, 4)):
+    arr = (M.Matrix * len(mats))(*mats)
+    return M.lib().mllm_sample_bwd_adam(ctypes.cast(arr, ctypes.c_void_p), len(mats), M.NM(*nm),
+                                        ctypes.byref(hp), 0)
+
+
+def test_invalid_arguments_rejected(M):
+    L = M.lib()
+    hp = _hp(M)
+    # null matrix array / zero count
+    assert L.mllm_sample_fwd(None, 1, M.NM(2, 4), ctypes.byref(hp), 0, 0, 0, 0) == M.MLLM_ERR_INVALID_ARG
+    assert _fwd(M, [], hp) == M.MLLM_ERR_INVALID_ARG
+    # unsupported pattern
+    assert _fwd(M, [_mat(M)], hp, nm=(3, 4)) == M.MLLM_ERR_UNSUPPORTED
+    # cols not a multiple of M
+    assert _fwd(M, [_mat(M, cols=6)], hp) == M.MLLM_ERR_INVALID_ARG
+    assert _fwd(M, [_mat(M, cols=12)], hp, nm=(4, 8)) == M.MLLM_ERR_INVALID_ARG
+    assert _fwd(M, [_mat(M, rows=-1)], hp) == M.MLLM_ERR_INVALID_ARG
+    # missing required buffers
+    assert _fwd(M, [_mat(M, W=0)], hp) == M.MLLM_ERR_INVALID_ARG
+    assert _fwd(M, [_mat(M, X_out=0)], hp) == M.MLLM_ERR_INVALID_ARG
+    assert _fwd(M, [_mat(M, logits=0)], hp) == M.MLLM_ERR_INVALID_ARG
+    assert _bwd(M, [_mat(M, G=0)], hp) == M.MLLM_ERR_INVALID_ARG
+    assert _bwd(M, [_mat(M, adam_v=0)], hp) == M.MLLM_ERR_INVALID_ARG
+    # unknown dtype, mixed dtypes in one call
+    assert _fwd(M, [_mat(M, w_dtype=7)], hp) == M.MLLM_ERR_UNSUPPORTED
+    assert _fwd(M, [_mat(M), _mat(M, w_dtype=1)], hp) == M.MLLM_ERR_UNSUPPORTED
+
+
+def test_misaligned_pointers_rejected(M):
+    hp = _hp(M)
+    for field in ("W", "X_out", "logits", "soft_mask_out"):
+        assert _fwd(M, [_mat(M, **{field: 0x1008})], hp) == M.MLLM_ERR_MISALIGNED, field
+    for field in ("G", "adam_m", "adam_v", "grad_logits_out"):
+        assert _bwd(M, [_mat(M, **{field: 0x1004})], hp) == M.MLLM_ERR_MISALIGNED, field
+    assert _fwd(M, [_mat(M)], hp, reg=0x10004) == M.MLLM_ERR_MISALIGNED
+    assert _fwd(M, [_mat(M)], hp, reg=0x10000, ws=0x9008) == M.MLLM_ERR_MISALIGNED
+
+
+def test_workspace_checked(M):
+    hp = _hp(M)
+    assert _fwd(M, [_mat(M)], hp, reg=0x10000, ws=0) == M.MLLM_ERR_WORKSPACE
+    assert _fwd(M, [_mat(M)], hp, reg=0x10000, wsb=M.mllm_workspace_bytes() - 8) == M.MLLM_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("field,value", [
+    ("tau", 0.0), ("tau", -1.0), ("tau", float("inf")), ("tau", float("nan")), ("tau", 1e-39),
+    ("kappa", 0.0), ("kappa", float("nan")), ("step", 0xFFFFFFFF), ("reserved", 1)])
+def test_bad_forward_scalars(M, field, value):
+    assert _fwd(M, [_mat(M)], _hp(M, **{field: value})) == M.MLLM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field,value", [
+    ("lambda_", -1e-5), ("lr", float("nan")), ("beta1", 1.0), ("beta2", -0.1), ("eps", 0.0),
+    ("weight_decay", -0.1), ("adam_step", 0)])
+def test_bad_backward_scalars(M, field, value):
+    assert _bwd(M, [_mat(M)], _hp(M, **{field: value})) == M.MLLM_ERR_INVALID_ARG
+
+
+def test_prior_and_pack_validation(M):
+    L = M.lib()
+    arr = (M.Matrix * 1)(_mat(M))
+    p = ctypes.cast(arr, ctypes.c_void_p)
+    assert L.mllm_prior_init(p, 1, M.NM(2, 4), -1.0, 0.01, 0, 0) == M.MLLM_ERR_INVALID_ARG
+    assert L.mllm_prior_init(p, 1, M.NM(2, 4), 3.0, float("nan"), 0, 0) == M.MLLM_ERR_INVALID_ARG
+    bad = (M.Matrix * 1)(_mat(M, pack_meta=0))
+    assert L.mllm_hard_pack(ctypes.cast(bad, ctypes.c_void_p), 1, M.NM(2, 4), 0) == M.MLLM_ERR_INVALID_ARG
+    bad = (M.Matrix * 1)(_mat(M, pack_values=0x7004))
+    assert L.mllm_hard_pack(ctypes.cast(bad, ctypes.c_void_p), 1, M.NM(2, 4), 0) == M.MLLM_ERR_MISALIGNED
+    assert L.mllm_noise(M.NM(2, 4), 0, 0, 0x1000, -1, 0x2000, 0) == M.MLLM_ERR_INVALID_ARG
+    assert L.mllm_noise(M.NM(2, 5), 0, 0, 0x1000, 1, 0x2000, 0) == M.MLLM_ERR_UNSUPPORTED
+    assert L.mllm_noise(M.NM(2, 4), 0, 0, 0x1000, 0, 0x2000, 0) == M.MLLM_OK  # nothing to do

@@ -1,0 +1,339 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle, element by element.
+
+Inputs come from sparsity_mask_sampling_b200.inputs (seeded, on the CPU), are copied to the
+device for the kernels and handed to the oracle as the same bytes. Sizes span several CTA
+tiles and end in ragged tails (odd block counts, partial tiles, partial metadata words).
+"""
+import numpy as np
+import pytest
+import torch
+
+import _tol
+from sparsity_mask_sampling_b200 import (Hparams, MatrixBuffers, alloc_matrix, inputs, mllm_hard_pack,
+                                         mllm_noise, mllm_prior_init, mllm_sample_bwd_adam,
+                                         mllm_sample_fwd, mllm_workspace_bytes)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+C_OF = {(2, 4): 6, (4, 8): 70}
+
+
+@pytest.fixture(scope="module")
+def orc():
+    import oracle
+
+    oracle.build()
+    return oracle
+
+
+@pytest.fixture(scope="module")
+def ws():
+    return torch.zeros(mllm_workspace_bytes(), dtype=torch.uint8, device=DEV)
+
+
+def _wvals(W):
+    """Exact weight values as float64 [B, M] for the oracle."""
+    return W.float().double().numpy()
+
+
+class Case:
+    """One matrix: CPU inputs, device buffers, oracle views."""
+
+    def __init__(self, nm, rows, cols, w_dtype="bf16", seed=0, offset=0, pi_std=0.02, outliers=0.0):
+        n, m = nm
+        self.nm, self.rows, self.cols, self.C = nm, rows, cols, C_OF[nm]
+        self.B = rows * cols // m
+        self.w_dtype = w_dtype
+        self.W = inputs.weights(rows, cols, w_dtype, 0.02, seed, outlier_frac=outliers)
+        self.G = inputs.upstream_grad(rows, cols, w_dtype, 1e-3 if w_dtype == "bf16" else 1.0, seed + 1)
+        self.pi = inputs.logits(self.B, self.C, pi_std, seed + 2)
+        self.m0, self.v0 = inputs.moments(self.B, self.C, seed + 3)
+        self.offset = offset
+        self.gids = (np.arange(self.B, dtype=np.uint64) + np.uint64(offset))
+        self.mb = alloc_matrix(self.W.to(DEV), nm, offset, fwd=True, bwd=True, pack=True,
+                               soft_mask=True, grad_logits=True)
+        self.mb.G.copy_(self.G.to(DEV))
+        self.reset()
+
+    def reset(self):
+        self.mb.logits.copy_(self.pi.to(DEV))
+        self.mb.adam_m.copy_(self.m0.to(DEV))
+        self.mb.adam_v.copy_(self.v0.to(DEV))
+
+    @property
+    def Wv(self):
+        return _wvals(self.W).reshape(self.B, self.nm[1])
+
+    @property
+    def Gv(self):
+        return _wvals(self.G).reshape(self.B, self.nm[1])
+
+    def x_gpu(self):
+        return self.mb.X.float().double().cpu().numpy().reshape(self.B, self.nm[1])
+
+
+def _run_fwd(cases, nm, hp, ws):
+    reg = torch.zeros(1, dtype=torch.float64, device=DEV)
+    mllm_sample_fwd([c.mb for c in cases], nm, hp, reg, ws)
+    torch.cuda.synchronize()
+    return float(reg.item())
+
+
+def _check_fwd(orc, cases, hp, reg_gpu):
+    reg_ref = 0.0
+    for c in cases:
+        r = orc.sample_fwd(*c.nm, c.Wv, c.pi.numpy(), c.gids, hp.kappa, hp.tau, hp.seed, hp.step,
+                           noise_on=hp.noise_on)
+        reg_ref += r["reg"]
+        _tol.assert_soft_close(c.mb.soft_mask.cpu().numpy().reshape(c.B, c.nm[1]), r["msoft"])
+        _tol.assert_x_close(c.x_gpu(), r["x"], c.w_dtype, c.Wv)
+    _tol.assert_reg_close(reg_gpu, reg_ref)
+
+
+def _check_bwd(orc, cases, hp):
+    for c in cases:
+        g_ref, scale = orc.sample_bwd(*c.nm, c.Wv, c.Gv, c.pi.numpy(), c.gids, hp.kappa, hp.tau,
+                                      hp.lambda_, hp.seed, hp.step, noise_on=hp.noise_on)
+        floor = _tol.grad_floor(c.Wv, c.Gv, hp.kappa, hp.tau, hp.lambda_)
+        g_gpu = c.mb.grad_logits.cpu().numpy()
+        _tol.assert_grad_close(g_gpu, g_ref, scale, floor)
+        p_ref, m_ref, v_ref = orc.adamw(c.pi.numpy(), c.m0.numpy(), c.v0.numpy(), g_ref, np.float32(hp.lr),
+                                        np.float32(hp.beta1), np.float32(hp.beta2), np.float32(hp.eps),
+                                        np.float32(hp.weight_decay), hp.adam_step)
+        _tol.assert_logits_close(c.mb.logits.cpu().numpy(), p_ref)
+        _tol.assert_moments_close(c.mb.adam_m.cpu().numpy(), c.mb.adam_v.cpu().numpy(), m_ref, v_ref,
+                                  g_ref, 1e-4 * scale + floor, np.float32(hp.beta1), np.float32(hp.beta2))
+
+
+SHAPES_24 = [(64, 128), (3, 12), (1, 4), (300, 64), (77, 36), (256, 1024)]
+SHAPES_48 = [(64, 128), (3, 16), (1, 8), (130, 72), (40, 1024)]
+SCHED = [(4.0, 100.0), (1.0, 300.0), (0.05, 500.0)]
+
+
+# ------------------------------------------------------------------------------ noise
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_noise_bit_exact(orc, nm):
+    rng = np.random.default_rng(0)
+    n = 1 << 18 if nm == (2, 4) else 1 << 14
+    gids = rng.integers(0, 2**63, size=n, dtype=np.uint64)
+    gids[:1000] = np.arange(1000, dtype=np.uint64)
+    for seed, step in [(0, 0), (0x1234_5678_9ABC_DEF0, 77), (5, 0xFFFFFFFF)]:
+        out = torch.empty(n, C_OF[nm], dtype=torch.float32, device=DEV)
+        mllm_noise(nm, seed, step, torch.from_numpy(gids.view(np.int64)).to(DEV), out)
+        _, g_ref = orc.noise(*nm, seed, step, gids)
+        got = out.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), g_ref.view(np.uint32)), \
+            f"{np.sum(got != g_ref)} noise values differ"
+
+
+def test_noise_every_uniform_value(orc):
+    """Every 21-bit field value maps to the same g on both sides: the GPU noise of many
+    blocks covers all 2^21 uniforms (checked through the oracle's eps of the same blocks)."""
+    gids = np.arange(1 << 20, dtype=np.uint64)
+    out = torch.empty(len(gids), 6, dtype=torch.float32, device=DEV)
+    mllm_noise((2, 4), 9, 3, torch.from_numpy(gids.view(np.int64)).to(DEV), out)
+    eps, g_ref = orc.noise(2, 4, 9, 3, gids)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), g_ref.view(np.uint32))
+    assert len(np.unique(eps)) > 0.9 * (1 << 21)
+
+
+# ------------------------------------------------------------------------------ forward
+
+@pytest.mark.parametrize("nm,shapes", [((2, 4), SHAPES_24), ((4, 8), SHAPES_48)])
+@pytest.mark.parametrize("tau,kappa", SCHED)
+def test_forward_parity(orc, ws, nm, shapes, tau, kappa):
+    cases = []
+    off = 0
+    for i, (r, c) in enumerate(shapes):
+        cases.append(Case(nm, r, c, seed=10 * i, offset=off, outliers=0.01 if i == 0 else 0.0))
+        off += cases[-1].B + 12345
+    hp = Hparams(kappa=kappa, tau=tau, step=3, seed=0xC0FFEE)
+    reg = _run_fwd(cases, nm, hp, ws)
+    _check_fwd(orc, cases, hp, reg)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_forward_fp32_weights(orc, ws, nm):
+    """The tiny workload's fp32 weights: X within 1e-5 relative."""
+    cases = [Case(nm, 64, 128, w_dtype="f32", seed=0)]
+    hp = Hparams(kappa=100.0, tau=4.0, step=0, seed=0)
+    _check_fwd(orc, cases, hp, _run_fwd(cases, nm, hp, ws))
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_forward_noise_off_and_one_hot(orc, ws, nm):
+    cases = [Case(nm, 33, 64, seed=4)]
+    hp = Hparams(kappa=1.0, tau=1e-3, step=0, seed=1, noise_on=False)
+    _check_fwd(orc, cases, hp, _run_fwd(cases, nm, hp, ws))
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_forward_large_block_offsets(orc, ws, nm):
+    """Global block ids beyond 2^32 (the high counter word) and a 2^63 neighbourhood."""
+    cases = [Case(nm, 16, 64, seed=5, offset=2**32 - 7), Case(nm, 8, 64, seed=6, offset=2**63 + 11)]
+    hp = Hparams(kappa=200.0, tau=0.5, step=12, seed=2**40 + 3)
+    _check_fwd(orc, cases, hp, _run_fwd(cases, nm, hp, ws))
+
+
+def test_forward_empty_matrices(orc, ws):
+    """Empty matrices contribute nothing; a call with only empty matrices writes reg = 0."""
+    e = MatrixBuffers(W=torch.empty(0, 8, dtype=torch.bfloat16, device=DEV))
+    reg = torch.full((1,), 7.0, dtype=torch.float64, device=DEV)
+    mllm_sample_fwd([e], (2, 4), Hparams(), reg, ws)
+    torch.cuda.synchronize()
+    assert reg.item() == 0.0
+    cases = [Case((2, 4), 5, 8, seed=7)]
+    hp = Hparams(kappa=100.0, tau=1.0)
+    reg = torch.zeros(1, dtype=torch.float64, device=DEV)
+    mllm_sample_fwd([e, cases[0].mb, e], (2, 4), hp, reg, ws)
+    torch.cuda.synchronize()
+    _check_fwd(orc, cases, hp, reg.item())
+
+
+def test_forward_many_matrices_chunked(orc, ws):
+    """More matrices than one launch takes (16): the regulariser accumulates across chunks."""
+    cases, off = [], 0
+    for i in range(19):
+        cases.append(Case((2, 4), 3 + i, 16, seed=100 + i, offset=off))
+        off += cases[-1].B
+    hp = Hparams(kappa=150.0, tau=2.0, step=1, seed=3)
+    _check_fwd(orc, cases, hp, _run_fwd(cases, (2, 4), hp, ws))
+
+
+def test_forward_deterministic(ws):
+    cases = [Case((2, 4), 256, 1024, seed=8)]
+    hp = Hparams(kappa=100.0, tau=1.0, step=5, seed=9)
+    r1 = _run_fwd(cases, (2, 4), hp, ws)
+    x1 = cases[0].mb.X.clone()
+    r2 = _run_fwd(cases, (2, 4), hp, ws)
+    assert r1 == r2 and torch.equal(x1, cases[0].mb.X)
+
+
+def test_forward_without_regulariser(orc, ws):
+    cases = [Case((2, 4), 64, 64, seed=9)]
+    hp = Hparams(kappa=100.0, tau=1.0)
+    mllm_sample_fwd([cases[0].mb], (2, 4), hp, None, None)
+    torch.cuda.synchronize()
+    r = orc.sample_fwd(2, 4, cases[0].Wv, cases[0].pi.numpy(), cases[0].gids, 100.0, 1.0, 0, 0)
+    _tol.assert_x_close(cases[0].x_gpu(), r["x"], "bf16", cases[0].Wv)
+
+
+# ------------------------------------------------------------------------------ backward
+
+@pytest.mark.parametrize("nm,shapes", [((2, 4), SHAPES_24), ((4, 8), SHAPES_48)])
+@pytest.mark.parametrize("tau,kappa", SCHED)
+def test_backward_adam_parity(orc, nm, shapes, tau, kappa):
+    cases, off = [], 0
+    for i, (r, c) in enumerate(shapes):
+        cases.append(Case(nm, r, c, seed=20 * i + 1, offset=off, outliers=0.01 if i == 0 else 0.0))
+        off += cases[-1].B
+    hp = Hparams(kappa=kappa, tau=tau, lambda_=1e-5, lr=5e-4, adam_step=7, step=6, seed=0xBEEF)
+    mllm_sample_bwd_adam([c.mb for c in cases], nm, hp)
+    torch.cuda.synchronize()
+    _check_bwd(orc, cases, hp)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_backward_first_step_and_fp32(orc, nm):
+    """Adam step 1 from zero moments (sign-like update) with fp32 weights and gradients."""
+    c = Case(nm, 64, 128, w_dtype="f32", seed=30)
+    c.m0.zero_()
+    c.v0.zero_()
+    c.reset()
+    hp = Hparams(kappa=100.0, tau=4.0, lambda_=1e-5, lr=1e-3, adam_step=1, step=0, seed=0)
+    mllm_sample_bwd_adam([c.mb], nm, hp)
+    torch.cuda.synchronize()
+    _check_bwd(orc, [c], hp)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_backward_large_lambda_noise_off(orc, nm):
+    c = Case(nm, 40, 64, seed=31)
+    hp = Hparams(kappa=50.0, tau=0.7, lambda_=5.0, lr=1e-3, adam_step=3, step=2, seed=4, noise_on=False)
+    mllm_sample_bwd_adam([c.mb], nm, hp)
+    torch.cuda.synchronize()
+    _check_bwd(orc, [c], hp)
+
+
+def test_forward_backward_share_noise(orc, ws):
+    """Same (seed, step): the backward's recomputed soft mask is the forward's. Checked by
+    the gradient of a loss whose G equals the forward output: both match the oracle."""
+    c = Case((2, 4), 128, 256, seed=32)
+    hp = Hparams(kappa=300.0, tau=0.3, step=41, seed=77, adam_step=2)
+    _check_fwd(orc, [c], hp, _run_fwd([c], (2, 4), hp, ws))
+    mllm_sample_bwd_adam([c.mb], (2, 4), hp)
+    torch.cuda.synchronize()
+    _check_bwd(orc, [c], hp)
+
+
+# ------------------------------------------------------------------------------ prior init
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_prior_deterministic_bit_exact(orc, nm):
+    c = Case(nm, 96, 64, seed=40, outliers=0.05)
+    W = c.W.clone()
+    W[0, :4] = torch.tensor([0.5, -0.5, 0.5, 0.1])       # ties resolve to the lower position
+    c.mb.W.copy_(W.to(DEV))
+    mllm_prior_init([c.mb], nm, 3.0, 0.0, 0)
+    torch.cuda.synchronize()
+    pi_ref, pidx, _ = orc.prior_init(*nm, _wvals(W).reshape(c.B, nm[1]), c.gids, 3.0, 0.0, 0)
+    got = c.mb.logits.cpu().numpy()
+    assert np.array_equal(got, pi_ref.astype(np.float32))
+    assert np.array_equal(np.argmax(got, 1), pidx)
+    assert not c.mb.adam_m.any() and not c.mb.adam_v.any()
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_prior_random_parity(orc, nm):
+    c = Case(nm, 200, 128, seed=41, offset=2**33)
+    mllm_prior_init([c.mb], nm, 3.0, 0.01, 1234)
+    torch.cuda.synchronize()
+    pi_ref, _, _ = orc.prior_init(*nm, c.Wv, c.gids, 3.0, 0.01, 1234)
+    got = c.mb.logits.cpu().numpy().astype(np.float64)
+    err = np.abs(got - pi_ref)
+    tol = 1e-6 * np.abs(pi_ref).max(1, keepdims=True) + 1e-12
+    assert not (err > tol).any(), f"{(err > tol).sum()} prior logits differ, worst {np.max(err / tol):.3g}"
+    assert not c.mb.adam_m.any() and not c.mb.adam_v.any()
+
+
+# ------------------------------------------------------------------------------ hard pack
+
+@pytest.mark.parametrize("nm,shapes", [((2, 4), [(64, 128), (3, 12), (5, 36), (7, 4)]),
+                                       ((4, 8), [(64, 128), (3, 16), (5, 24)])])
+@pytest.mark.parametrize("w_dtype", ["bf16", "f32"])
+def test_pack_bit_exact(orc, nm, shapes, w_dtype):
+    cases = [Case(nm, r, c, w_dtype=w_dtype, seed=50 + i) for i, (r, c) in enumerate(shapes)]
+    for i, c in enumerate(cases):
+        # quantised logits produce ties (lowest index wins); a few NaNs never win
+        q = torch.round(c.pi * 200) / 200
+        if i == 0:
+            q[::7, 1] = float("nan")
+            q[::11] = float("nan")
+        c.pi = q
+        c.reset()
+        c.mb.cand_idx.fill_(255)
+    mllm_hard_pack([c.mb for c in cases], nm)
+    torch.cuda.synchronize()
+    view = np.uint16 if w_dtype == "bf16" else np.uint32
+    for c in cases:
+        raw = c.W.view(torch.int16 if w_dtype == "bf16" else torch.int32).numpy().view(view)
+        vals, meta, cand = orc.hard_pack(*nm, raw, c.pi.numpy())
+        assert np.array_equal(c.mb.cand_idx.cpu().numpy(), cand)
+        got_vals = c.mb.pack_values.view(torch.int16 if w_dtype == "bf16" else torch.int32).cpu().numpy().view(view)
+        assert np.array_equal(got_vals, vals)
+        got_meta = c.mb.pack_meta.cpu().numpy().view(meta.dtype)
+        assert np.array_equal(got_meta, meta)
+
+
+def test_pack_of_deterministic_prior_is_magnitude_mask(orc):
+    """init_std = 0 then pack: the packed values are the 2 largest-|w| of every block."""
+    c = Case((2, 4), 128, 256, seed=60)
+    mllm_prior_init([c.mb], (2, 4), 3.0, 0.0, 0)
+    mllm_hard_pack([c.mb], (2, 4))
+    torch.cuda.synchronize()
+    Wf = c.W.float().numpy().reshape(c.B, 4)
+    top2 = np.sort(np.argsort(-np.abs(Wf), 1, kind="stable")[:, :2], 1)
+    expect = np.take_along_axis(Wf, top2, 1).reshape(c.rows, -1)
+    assert np.array_equal(c.mb.pack_values.float().cpu().numpy(), expect)
