@@ -1,0 +1,562 @@
+"""Benchmark of the MaskLLM mask sampler's hot path on B200.
+
+One step = the forward of every weight matrix of the workload (one grouped launch per
+layer, layers 0 -> L-1) followed by the fused backward + AdamW of every matrix (layers
+L-1 -> 0), as in one training step of the method. Metric: blocks/s over the step
+(blocks = groups of M weights, each with its C logits), whole job; plus each kernel's
+achieved HBM bandwidth against the measured copy bandwidth.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Default workload: the full LLaMA-2-7B-shaped stack at 2:4 (32 layers x 7 matrices,
+1,619,001,344 blocks; logits and AdamW moments resident in HBM, ~130 GB). Under torchrun
+each rank runs its own stack (weak scaling, disjoint global block ids); the only exchange
+is an all-reduce of the step's regulariser sum.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mask-sampling blocks/sec (fwd, fused bwd+Adam) and % of B200 HBM roofline"
+UNIT = "blocks/s"
+# algorithmic HBM bytes per block: fwd reads W + logits, writes X; bwd+Adam reads W, G,
+# logits, m, v and writes logits, m, v; pack reads W + logits, writes values + metadata
+BYTES = {6: {"fwd": 40, "bwd": 160, "pack": 36.5, "init": 80},
+         70: {"fwd": 312, "bwd": 1712, "pack": 306, "init": 856}}
+FALLBACK_HBM_GBS = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        # samples under load: power above the midpoint of the observed range
+        if power and max(power) > min(power) + 50:
+            thr = (max(power) + min(power)) / 2
+            loaded = [s for s, p in zip(sm, power) if p >= thr]
+        else:
+            loaded = sm
+        return {"sm_mhz": float(np.median(loaded or sm)), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(sm), "samples_under_load": len(loaded), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+class Stack:
+    """Device state of the workload: resident W, logits, moments; pooled X and G."""
+
+    def __init__(self, w, dev, rank, seed_base=0):
+        import torch
+        import sparsity_mask_sampling_b200 as pkg
+        from sparsity_mask_sampling_b200 import configs, inputs
+
+        self.w = w
+        self.dev = dev
+        self.nm = w.nm
+        self.C = w.C
+        rank_offset = rank * w.total_blocks()
+        offs = configs.layer_block_offsets(w)
+        # X and G pools: two layers' worth, alternating (values do not change the cost)
+        self.pool = []
+        for p in range(2):
+            self.pool.append([(torch.empty(m.rows, m.cols, dtype=torch.bfloat16 if w.w_dtype == "bf16" else torch.float32, device=dev),
+                               inputs.upstream_grad(m.rows, m.cols, w.g_dtype, w.g_std, seed=seed_base + 1000 + 10 * p + i, device=dev))
+                              for i, m in enumerate(w.matrices)])
+        self.layers = []
+        self.bufs = []
+        for l in range(w.layers):
+            mats = []
+            for i, m in enumerate(w.matrices):
+                W = inputs.weights(m.rows, m.cols, w.w_dtype, w.w_std, seed=seed_base + 100 * l + i,
+                                   outlier_frac=w.outlier_frac, outlier_scale=w.outlier_scale, device=dev)
+                B = m.rows * m.cols // w.nm[1]
+                mb = pkg.MatrixBuffers(
+                    W=W, block_offset=rank_offset + offs[l][i],
+                    logits=torch.empty(B, w.C, dtype=torch.float32, device=dev),
+                    adam_m=torch.zeros(B, w.C, dtype=torch.float32, device=dev),
+                    adam_v=torch.zeros(B, w.C, dtype=torch.float32, device=dev))
+                mats.append(mb)
+            self.bufs.append(mats)
+            arr_views = []
+            for p in range(2):
+                for mb, (X, G) in zip(mats, self.pool[p]):
+                    mb.X, mb.G = X, G
+                arr_views.append(pkg.MatrixArray(mats))
+            self.layers.append(arr_views)  # [pool 0 view, pool 1 view]
+        self.ws = torch.zeros(pkg.mllm_workspace_bytes(), dtype=torch.uint8, device=dev)
+        self.reg = torch.zeros(w.layers, dtype=torch.float64, device=dev)
+        self.blocks = w.total_blocks()
+
+    def view(self, l):
+        return self.layers[l][l % 2]
+
+    def prior_init(self, seed=0):
+        import sparsity_mask_sampling_b200 as pkg
+
+        for l in range(self.w.layers):
+            pkg.mllm_prior_init(self.view(l), self.nm, self.w.alpha, self.w.init_std, seed)
+
+    def hparams(self, t, seed=0):
+        import sparsity_mask_sampling_b200 as pkg
+
+        T = max(self.w.steps, 1)
+        return pkg.Hparams(kappa=self.w.kappa_at(t % T), tau=self.w.tau_at(t % T), lambda_=self.w.lam,
+                           lr=self.w.lr, weight_decay=self.w.weight_decay, adam_step=t + 1, step=t,
+                           seed=seed).to_c()
+
+
+def run_step(stack, t, ev=None, g_ready=None, g_free=None, copy_fn=None):
+    """Enqueue one step. ev: optional dict of per-launch (start, end) event lists.
+    copy_fn(l, pool) enqueues the H2D copy of layer l's G (e2e leg)."""
+    import torch
+    import sparsity_mask_sampling_b200 as pkg
+
+    hp = stack.hparams(t)
+    nm = stack.nm
+    L = stack.w.layers
+    for l in range(L):
+        if ev is not None:
+            ev["fwd"][l][0].record()
+        pkg.mllm_sample_fwd(stack.view(l), nm, hp, stack.reg[l:l + 1], stack.ws)
+        if ev is not None:
+            ev["fwd"][l][1].record()
+    for l in reversed(range(L)):
+        if copy_fn is not None:
+            copy_fn(l)
+        if ev is not None:
+            ev["bwd"][l][0].record()
+        pkg.mllm_sample_bwd_adam(stack.view(l), nm, hp)
+        if ev is not None:
+            ev["bwd"][l][1].record()
+        if g_free is not None:
+            g_free[l % 2].record()
+
+
+def gpu_arm(args, w):
+    import torch
+    import torch.distributed as dist
+    import sparsity_mask_sampling_b200 as pkg
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pkg.lib()
+    hbm_peak, peak_kind = peaks()
+
+    t0 = time.time()
+    stack = Stack(w, dev, rank)
+    stack.prior_init(seed=0)
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] stack ready: {stack.blocks:,} blocks, {torch.cuda.memory_allocated(dev)/1e9:.1f} GB, {time.time()-t0:.1f}s")
+
+    # once-per-run rows: prior init and pack, timed on the device
+    init_ms = time_once(lambda: stack.prior_init(seed=0))
+    def reduce_all():
+        if world > 1:
+            dist.all_reduce(stack.reg, op=dist.ReduceOp.SUM)
+
+    # warm-up
+    for t in range(args.warmup):
+        run_step(stack, t)
+        reduce_all()
+    torch.cuda.synchronize()
+
+    # device-timed steps
+    L = w.layers
+    evs = [{k: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+            for k in ("fwd", "bwd")} for _ in range(args.steps)]
+    durs = {"fwd": [], "bwd": []}
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for k in range(args.steps):
+        run_step(stack, args.warmup + k, ev=evs[k])
+        reduce_all()
+    end.record()
+    torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    for ev in evs:
+        for name in ("fwd", "bwd"):
+            durs[name].extend(ev[name][l][0].elapsed_time(ev[name][l][1]) for l in range(L))
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    t_max = elapsed_ms
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    ms_per_step = t_max / args.steps
+    value = stack.blocks * world * args.steps / (t_max / 1e3)
+
+    # pack (once, after training)
+    pack_ms = time_pack(stack)
+
+    # end-to-end: upstream gradients from pinned host memory, regulariser read back
+    e2e = e2e_leg(args, stack, w, world, dist if world > 1 else None, dev)
+
+    blocks_per_layer = w.blocks_per_layer()
+    fb = BYTES[w.C]
+    kern = {}
+    for name in ("fwd", "bwd"):
+        d = np.array(durs[name])
+        avg_ms = float(d.mean())
+        achieved = blocks_per_layer * fb[name] / (avg_ms / 1e3) / 1e9
+        kern[name] = {"avg_launch_ms": avg_ms, "blocks_per_launch": blocks_per_layer,
+                      "bytes_per_block": fb[name], "achieved_gbs": achieved, "frac": achieved / hbm_peak}
+    traffic = traffic_from_profile("bwd", w)
+    roofline = {"bound": "hbm", "kernel": "bwd_adam (fused backward + AdamW)",
+                "achieved": round(kern["bwd"]["achieved_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(kern["bwd"]["achieved_gbs"] / hbm_peak, 4), "peak_kind": peak_kind,
+                "traffic": traffic}
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_of(w, world),
+            "roofline": roofline,
+            "kernels": {
+                "fwd": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in kern["fwd"].items()},
+                "bwd_adam": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in kern["bwd"].items()},
+                "pack_once": once_stats(pack_ms, stack.blocks, fb["pack"], hbm_peak),
+                "prior_init_once": once_stats(init_ms, stack.blocks, fb["init"], hbm_peak),
+            },
+            "e2e": e2e,
+            "gpu_launches": 2 * L * args.steps * n_groups(w),
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+def n_groups(w):
+    return math.ceil(len(w.matrices) / 16)
+
+
+def time_once(fn):
+    import torch
+
+    fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+def time_pack(stack):
+    import torch
+    import sparsity_mask_sampling_b200 as pkg
+    from sparsity_mask_sampling_b200 import buffers
+
+    # packed outputs of one layer are reused across layers (the pack runs once; only its cost matters)
+    w = stack.w
+    outs = []
+    for m in w.matrices:
+        (vs, (ms, mdt)) = buffers.pack_shapes(m.rows, m.cols, w.nm)
+        outs.append((torch.empty(vs, dtype=torch.bfloat16, device=stack.dev), torch.empty(ms, dtype=mdt, device=stack.dev),
+                     torch.empty(m.rows * m.cols // w.nm[1], dtype=torch.uint8, device=stack.dev)))
+    arrs = []
+    for l in range(w.layers):
+        for mb, (v, mt, ci) in zip(stack.bufs[l], outs):
+            mb.pack_values, mb.pack_meta, mb.cand_idx = v, mt, ci
+        arrs.append(pkg.MatrixArray(stack.bufs[l]))
+
+    def go():
+        for a in arrs:
+            pkg.mllm_hard_pack(a, w.nm)
+    return time_once(go)
+
+
+def once_stats(ms, blocks, bpb, peak):
+    gbs = blocks * bpb / (ms / 1e3) / 1e9
+    return {"ms": round(ms, 3), "blocks_per_s": blocks / (ms / 1e3), "achieved_gbs": round(gbs, 1),
+            "frac": round(gbs / peak, 4)}
+
+
+def e2e_leg(args, stack, w, world, dist, dev):
+    """Same steps through the public API with the step inputs on the host: each layer's
+    upstream gradients are copied from pinned host memory (a copy stream, overlapped with
+    the kernels), and the regulariser sums are read back to the host every step."""
+    import torch
+
+    L = w.layers
+    host_g = []
+    for p in range(2):
+        host_g.append([g.cpu().pin_memory() for (_, g) in stack.pool[p]])
+    h2d = sum(g.numel() * g.element_size() for (_, g) in stack.pool[0]) * L
+    reg_host = torch.empty(L, dtype=torch.float64, pin_memory=True)
+    d2h = reg_host.numel() * reg_host.element_size()
+    main = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    g_free = [torch.cuda.Event(), torch.cuda.Event()]
+    for e in g_free:
+        e.record(main)
+
+    def copy_fn(l):
+        p = l % 2
+        with torch.cuda.stream(copy):
+            copy.wait_event(g_free[p])
+            for (_, g), hg in zip(stack.pool[p], host_g[p]):
+                g.copy_(hg, non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(copy)
+        main.wait_event(ready)
+
+    steps = max(2, min(args.steps, 5))
+    for t in range(1):
+        run_step(stack, 1000 + t, g_free=g_free, copy_fn=copy_fn)
+        reg_host.copy_(stack.reg, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for t in range(steps):
+        run_step(stack, 2000 + t, g_free=g_free, copy_fn=copy_fn)
+        if dist is not None:
+            dist.all_reduce(stack.reg, op=dist.ReduceOp.SUM)
+        reg_host.copy_(stack.reg, non_blocking=True)
+        main.synchronize()
+        _ = float(reg_host.sum())
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if dist is not None:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    return {"value": stack.blocks * world * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def config_of(w, world):
+    return {"workload": w.name, "nm": f"{w.nm[0]}:{w.nm[1]}", "layers": w.layers,
+            "matrices_per_layer": len(w.matrices),
+            "shapes_out_in": [[m.rows, m.cols] for m in w.matrices],
+            "blocks_per_step_per_gpu": w.total_blocks(), "candidates": w.C,
+            "weights": f"{w.w_dtype} ~N(0,{w.w_std}^2), {w.outlier_frac:.0%} outlier input channels x{w.outlier_scale:g}",
+            "upstream_grad": f"{w.g_dtype} ~N(0,{w.g_std}^2)",
+            "tau": list(w.tau), "kappa": list(w.kappa), "lr": w.lr, "lambda": w.lam,
+            "launches": "one grouped launch per layer per kernel",
+            "l2": "inputs larger than L2 (each launch streams >= 280 MB); no flush",
+            "parallelism": f"dp{world} (independent shards)"}
+
+
+def traffic_from_profile(kernel, w):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (its sha256 is recorded there); otherwise None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(f"{kernel}_{w.nm[0]}of{w.nm[1]}")
+    if not ent or ent.get("source_sha256") != kernel_source_sha():
+        return None
+    return ent["dram_bytes_per_block"] * w.blocks_per_layer()
+
+
+def kernel_source_sha():
+    csrc = os.path.join(ROOT, "sparsity_mask_sampling_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+# ------------------------------------------------------------------------------ CPU (oracle)
+
+def make_sample(w, n_blocks, seed=0):
+    """A bounded sample of the workload's blocks: their global ids, weights, logits and
+    upstream gradients (seeded, same distributions as the GPU workload)."""
+    import torch
+    from sparsity_mask_sampling_b200 import inputs
+
+    rng = np.random.default_rng(seed)
+    gids = rng.integers(0, w.total_blocks(), size=n_blocks, dtype=np.uint64)
+    M = w.nm[1]
+    W = inputs.weights(n_blocks, M, w.w_dtype, w.w_std, seed=seed).float().double().numpy()
+    G = inputs.upstream_grad(n_blocks, M, w.g_dtype, w.g_std, seed=seed + 1).float().double().numpy()
+    pi = inputs.logits(n_blocks, w.C, 0.02, seed=seed + 2).numpy()
+    return gids, W, G, pi
+
+
+def oracle_step(orc, w, sample, t):
+    """The oracle on one sample for one step: forward, backward, AdamW."""
+    gids, W, G, pi = sample
+    kappa, tau = w.kappa_at(t % w.steps), w.tau_at(t % w.steps)
+    n, m = w.nm
+    orc.sample_fwd(n, m, W, pi, gids, kappa, tau, 0, t)
+    g, _ = orc.sample_bwd(n, m, W, G, pi, gids, kappa, tau, w.lam, 0, t)
+    z = np.zeros_like(g)
+    orc.adamw(pi, z, z, g, w.lr, 0.9, 0.999, 1e-8, w.weight_decay, t + 1)
+
+
+def cpu_run(w, n_blocks, threads, steps, t0=0):
+    import oracle as orc
+
+    orc.build()
+    per = max(1, n_blocks // threads)
+    samples = [make_sample(w, per, seed=17 + i) for i in range(threads)]
+    start = time.perf_counter()
+    with cf.ThreadPoolExecutor(threads) as ex:
+        for t in range(steps):
+            list(ex.map(lambda s: oracle_step(orc, w, s, t0 + t), samples))
+    return time.perf_counter() - start, per * threads
+
+
+def cpu_baseline(w, target_s=15.0):
+    threads = os.cpu_count() or 1
+    dt, n = cpu_run(w, 2000 * threads, threads, 1)
+    rate = n / dt
+    n_blocks = int(min(max(rate * target_s, 1000 * threads), 5e7))
+    dt, n = cpu_run(w, n_blocks, threads, 1)
+    return {"value": n / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n:,} blocks drawn from {w.name} (random global ids; weights, logits and "
+                      f"gradients from the same seeded distributions), one forward + backward + "
+                      f"AdamW step, {dt:.1f} s on {threads} threads"}
+
+
+def reference_arm(args, w):
+    """The oracle as it stands on the host cores: each step runs the oracle's forward,
+    backward and AdamW on a bounded sample of the workload's blocks."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    threads = os.cpu_count() or 1
+    dt, n = cpu_run(w, 2000 * threads, threads, 1)
+    per_step = int(min(max(n / dt * args.ref_step_seconds, 1000 * threads), 5e7))
+    cpu_run(w, per_step, threads, args.warmup)
+    dt, n = cpu_run(w, per_step, threads, args.steps, t0=args.warmup)
+    value = n * args.steps / dt
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, 1), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n:,} blocks per step drawn from {w.name}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama2_7b_stack_2of4")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warm-up raised to 3 steps")
+        args.warmup = 3
+    from sparsity_mask_sampling_b200 import configs
+
+    w = configs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        out = reference_arm(args, w)
+    else:
+        out = gpu_arm(args, w)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()
