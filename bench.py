@@ -123,8 +123,9 @@ class Stack:
         self.dev = dev
         self.nm = w.nm
         self.C = w.C
-        rank_offset = rank * w.total_blocks()
-        offs = configs.layer_block_offsets(w)
+        from sparsity_mask_sampling_b200 import sharding
+
+        offs = sharding.weak_block_offsets(w, rank)
         # X and G pools: two layers' worth, alternating (values do not change the cost)
         self.pool = []
         for p in range(2):
@@ -140,7 +141,7 @@ class Stack:
                                    outlier_frac=w.outlier_frac, outlier_scale=w.outlier_scale, device=dev)
                 B = m.rows * m.cols // w.nm[1]
                 mb = pkg.MatrixBuffers(
-                    W=W, block_offset=rank_offset + offs[l][i],
+                    W=W, block_offset=offs[l][i],
                     logits=torch.empty(B, w.C, dtype=torch.float32, device=dev),
                     adam_m=torch.zeros(B, w.C, dtype=torch.float32, device=dev),
                     adam_v=torch.zeros(B, w.C, dtype=torch.float32, device=dev))
