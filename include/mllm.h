@@ -23,7 +23,8 @@
  *   Ownership. Every pointer inside mllm_matrix, and reg_sum_out / workspace, is device
  *     memory owned by the caller and borrowed for the duration of the enqueued work. The
  *     `mats` and `hp` arrays themselves are host memory, read during the call only. The
- *     library allocates nothing and keeps no state between calls.
+ *     library allocates nothing and keeps no state between calls, except the fixed scratch
+ *     array of mllm_sample_fwd_noalloc (described there).
  *   Streams. `stream` is a cudaStream_t (NULL = the legacy default stream). All work is
  *     enqueued asynchronously on it; the call returns once enqueued.
  *   Alignment. Every device pointer must be 16-byte aligned (MLLM_ERR_MISALIGNED).
@@ -138,6 +139,27 @@ mllm_status mllm_prior_init(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
 mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
                             const mllm_hparams *hp, double *reg_sum_out, void *workspace,
                             size_t workspace_bytes, void *stream);
+
+/* Forward for callers that cannot allocate device memory (no counterpart in the paper;
+ * an addition of this library). Some callers own no allocator: a plugin whose host
+ * framework hands it only the tensors of the step and forbids cudaMalloc/cudaFree after
+ * start-up (they synchronise the device and fragment a fixed memory budget), or a runtime
+ * that exposes device memory to it only as the call's inputs and outputs. For them the
+ * scratch of the regulariser reduction (a ticket word and one double per CTA) lives in a
+ * fixed array inside this library instead of the `workspace` argument of mllm_sample_fwd.
+ * Semantics, outputs and arguments are otherwise those of mllm_sample_fwd.
+ *   Limit: the array holds 2048 per-CTA partial sums (16,400 bytes, 256-byte aligned); a
+ *     launch that would need more (a device with more than 2048 resident CTAs of the
+ *     kernel) is rejected with MLLM_ERR_WORKSPACE before anything is enqueued.
+ *   Set-up: the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture. Every GPU that loads the library holds the array until exit.
+ *   Sharing: all calls on a device share the one array and each call clears its ticket
+ *     word before launching; calls whose work overlaps on the GPU (different streams
+ *     without ordering between them) race on the array and must not be issued.
+ *   reg_sum_out must be non-NULL. Nothing is allocated: no cudaMalloc, no cudaFree. */
+mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                    const mllm_hparams *hp, double *reg_sum_out, void *stream);
 
 /* Backward to the logits fused with AdamW (s.3.2 "Frozen LLM Backbone"; s.3.4 Eq.8 and
  * Algorithm 1 step 2; AdamW as in PyTorch, Loshchilov & Hutter decoupled decay).

@@ -86,6 +86,7 @@ _SIGS = {
     "mllm_prior_init": (ctypes.c_int, [_P, ctypes.c_int32, NM, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, _P]),
     "mllm_sample_fwd": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P, ctypes.c_size_t, _P]),
     "mllm_sample_bwd_adam": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P]),
+    "mllm_sample_fwd_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P]),
     "mllm_hard_pack": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P]),
     "mllm_noise": (ctypes.c_int, [NM, ctypes.c_uint64, ctypes.c_uint32, _P, ctypes.c_int64, _P, _P]),
     "mllm_workspace_bytes": (ctypes.c_size_t, []),
@@ -245,6 +246,15 @@ def mllm_sample_fwd(mats, nm, hp: Hparams, reg_sum_out: Optional[torch.Tensor] =
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mllm_sample_fwd(a.ptr, a.n, _nm(nm), ctypes.byref(h), _ptr(reg_sum_out),
                                  _ptr(workspace), ws_bytes, _stream(stream)), "mllm_sample_fwd")
+
+
+def mllm_sample_fwd_noalloc(mats, nm, hp: Hparams, reg_sum_out: torch.Tensor, stream=None):
+    """mllm_sample_fwd for callers that cannot allocate: the reduction scratch is a fixed
+    array inside libmllm (no workspace argument). Calls on one device must not overlap."""
+    a = _mats(mats)
+    h = hp.to_c() if isinstance(hp, Hparams) else hp
+    _check(lib().mllm_sample_fwd_noalloc(a.ptr, a.n, _nm(nm), ctypes.byref(h), _ptr(reg_sum_out),
+                                         _stream(stream)), "mllm_sample_fwd_noalloc")
 
 
 def mllm_sample_bwd_adam(mats, nm, hp: Hparams, stream=None):

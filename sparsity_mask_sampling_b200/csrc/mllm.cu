@@ -255,6 +255,36 @@ std::vector<Group> make_groups(const mllm_matrix *mats, int32_t n_mats, int M, K
     return out;
 }
 
+// ------------------------------------------------------------------------ no-alloc scratch
+
+// Scratch of mllm_sample_fwd_noalloc: the ticket word at offset 0, per-CTA partial sums from
+// offset kWsPartialsOffset. A file-scope device array, so no allocation is ever made; its
+// device address is looked up once per device (host code cannot use the symbol itself).
+constexpr int kNoallocMaxCtas = 2048;
+constexpr size_t kNoallocBytes = kWsPartialsOffset + sizeof(double) * kNoallocMaxCtas;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+mllm_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (dev < 0 || dev >= kMaxDevices) return MLLM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_status(e);
+        if (!p) return MLLM_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MLLM_OK;
+}
+
 }  // namespace
 }  // namespace mllm
 
@@ -345,6 +375,52 @@ mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
         wrote_reg = true;
     }
     if (reg_sum_out && !wrote_reg) {
+        if ((s = cuda_status(cudaMemsetAsync(reg_sum_out, 0, sizeof(double), st))) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                    const mllm_hparams *hp, double *reg_sum_out, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedX | kNeedPi);
+    if (s != MLLM_OK) return s;
+    if ((s = validate_fwd_hp(hp)) != MLLM_OK) return s;
+    if (!reg_sum_out) return MLLM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(reg_sum_out) & 7u) != 0) return MLLM_ERR_MISALIGNED;
+    const bool w32 = mats[0].w_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
+    const void *fn = is24 ? (w32 ? (const void *)k24::fwd_kernel<true> : (const void *)k24::fwd_kernel<false>)
+                          : (w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>);
+    const int threads = is24 ? kThreads : k48::kCtaThreads;
+    const std::vector<Group> groups = make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48);
+    // every launch's scratch need (one partial per CTA) is checked before anything runs
+    for (const Group &g : groups) {
+        if (g.total_work == 0) continue;
+        if (grid_for(fn, threads, 0, g.total_work, kMaxReduceCtas) > kNoallocMaxCtas) return MLLM_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != MLLM_OK) return s;
+    unsigned int *ticket = static_cast<unsigned int *>(scratch);
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(scratch) + kWsPartialsOffset);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StepScalars sc = make_scalars(*hp);
+    bool wrote_reg = false;
+    for (const Group &g : groups) {
+        if (g.total_work == 0) continue;
+        if ((s = cuda_status(cudaMemsetAsync(ticket, 0, sizeof(unsigned int), st))) != MLLM_OK) return s;
+        const int accumulate = wrote_reg ? 1 : 0;
+        const int64_t grid = grid_for(fn, threads, 0, g.total_work, kMaxReduceCtas);
+        if (is24) {
+            if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+        } else {
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+        }
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+        wrote_reg = true;
+    }
+    if (!wrote_reg) {
         if ((s = cuda_status(cudaMemsetAsync(reg_sum_out, 0, sizeof(double), st))) != MLLM_OK) return s;
     }
     return MLLM_OK;
