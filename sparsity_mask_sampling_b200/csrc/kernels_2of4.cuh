@@ -409,5 +409,49 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const __grid_constant__ 
     }
 }
 
+// Hard pack when every row's block count is a multiple of 8, so each metadata word covers
+// 8 consecutive blocks of one row and its index is (global block)/8: one thread per pair of
+// blocks with whole-vector loads; four consecutive threads (lanes 4i..4i+3) assemble a word
+// with two shuffles and the first of them stores it.
+__device__ __forceinline__ uint32_t half_of(const uint4 &a, int idx) {  // bf16 idx of 8
+    const uint32_t w = (idx & 4) ? ((idx & 2) ? a.w : a.z) : ((idx & 2) ? a.y : a.x);
+    return (idx & 1) ? (w >> 16) : (w & 0xFFFFu);
+}
+
+template <bool kW32>
+__global__ void __launch_bounds__(kThreads) pack_pairs_kernel(const __grid_constant__ Group grp) {
+    const int lane = threadIdx.x & 31;
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
+        const bool valid = b0 < d.nblocks;  // nblocks is a multiple of 8 on this path
+        uint32_t byte = 0;
+        if (valid) {
+            float pi[12];
+            load12(d.pi, b0, true, pi);
+            const int k0 = argmax6(pi), k1 = argmax6(pi + 6);
+            const uint32_t m0 = cand_mask(k0), m1 = cand_mask(k1);
+            const int a0 = __ffs(m0) - 1, c0 = 31 - __clz(m0);
+            const int a1 = __ffs(m1) - 1, c1 = 31 - __clz(m1);
+            byte = (uint32_t)(a0 | (c0 << 2)) | ((uint32_t)(a1 | (c1 << 2)) << 4);
+            if (kW32) {
+                const float *W = static_cast<const float *>(d.W) + b0 * 4;
+                st_stream(reinterpret_cast<float4 *>(static_cast<float *>(d.pvals) + b0 * 2),
+                          make_float4(__ldcs(W + a0), __ldcs(W + c0), __ldcs(W + 4 + a1), __ldcs(W + 4 + c1)));
+            } else {
+                const uint4 a = ld_stream(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(d.W) + b0 * 4));
+                __stcs(reinterpret_cast<uint2 *>(static_cast<uint16_t *>(d.pvals) + b0 * 2),
+                       make_uint2(half_of(a, a0) | (half_of(a, c0) << 16),
+                                  half_of(a, 4 + a1) | (half_of(a, 4 + c1) << 16)));
+            }
+            if (d.cidx) *reinterpret_cast<uint16_t *>(d.cidx + b0) = (uint16_t)(k0 | (k1 << 8));
+        }
+        uint32_t word = byte << (8 * (lane & 3));
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+        word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+        if (valid && (lane & 3) == 0) static_cast<uint32_t *>(d.pmeta)[b0 / 8] = word;
+    }
+}
+
 }  // namespace k24
 }  // namespace mllm

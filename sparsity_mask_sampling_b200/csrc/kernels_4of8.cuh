@@ -47,21 +47,39 @@ __device__ __forceinline__ void static_for(F &&f) {
 
 // --------------------------------------------------------------------------- tile staging
 
-// Copy n floats global -> shared (n may be any count; src/dst 8-byte aligned).
+// Tile staging. A tile of nb blocks is nb*280 bytes, 16-byte aligned at its start (tiles
+// begin at multiples of kBlocksPerCta blocks). stage_in issues asynchronous 16-byte copies
+// (cp.async, no registers involved) for every whole 16-byte chunk, plus one 8-byte tail when
+// nb is odd, then waits for them; the caller synchronises the CTA afterwards.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void stage_in(float *dst, const float *src, int n) {
-    const int n2 = n >> 1;
-    const float2 *s2 = reinterpret_cast<const float2 *>(src);
-    float2 *d2 = reinterpret_cast<float2 *>(dst);
-    for (int i = threadIdx.x; i < n2; i += kCtaThreads) d2[i] = __ldcs(s2 + i);
-    if ((n & 1) && threadIdx.x == 0) dst[n - 1] = __ldcs(src + n - 1);
+    const int n4 = n >> 2;  // whole 16-byte chunks
+    for (int i = threadIdx.x; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
+    if ((n & 3) && threadIdx.x == 0) {  // n = nb*70 is even: at most one 8-byte tail
+        *reinterpret_cast<float2 *>(dst + 4 * n4) = __ldcs(reinterpret_cast<const float2 *>(src + 4 * n4));
+    }
+    cp_async_wait_all();
 }
 
 __device__ __forceinline__ void stage_out(float *dst, const float *src, int n) {
-    const int n2 = n >> 1;
-    const float2 *s2 = reinterpret_cast<const float2 *>(src);
-    float2 *d2 = reinterpret_cast<float2 *>(dst);
-    for (int i = threadIdx.x; i < n2; i += kCtaThreads) __stcs(d2 + i, s2[i]);
-    if ((n & 1) && threadIdx.x == 0) __stcs(dst + n - 1, src[n - 1]);
+    const int n4 = n >> 2;
+    for (int i = threadIdx.x; i < n4; i += kCtaThreads)
+        __stcs(reinterpret_cast<float4 *>(dst) + i, reinterpret_cast<const float4 *>(src)[i]);
+    if ((n & 3) && threadIdx.x == 0)
+        __stcs(reinterpret_cast<float2 *>(dst + 4 * n4), *reinterpret_cast<const float2 *>(src + 4 * n4));
+}
+
+// Ask L2 to fetch [p, p + bytes) now (a bulk prefetch; no data returns to the SM).
+__device__ __forceinline__ void prefetch_l2(const void *p, int bytes) {
+    bytes &= ~15;
+    if (bytes > 0) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 template <bool kF32>
@@ -133,6 +151,15 @@ __device__ __forceinline__ float soft_sums(float w[C], float mx, float c2, float
         }
     });
     return s;
+}
+
+// AdamW, PyTorch step order, one element.
+__device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, const StepScalars &s) {
+    const float pd = __fmul_rn(p, s.decay);
+    m = __fmaf_rn(s.beta1, m, __fmul_rn(s.one_minus_beta1, g));
+    v = __fmaf_rn(s.beta2, v, __fmul_rn(s.one_minus_beta2, __fmul_rn(g, g)));
+    const float denom = __fmaf_rn(__fsqrt_rn(v), s.inv_sqrt_bc2, s.eps);
+    p = __fmaf_rn(-s.step_size, __fdividef(m, denom), pd);
 }
 
 // --------------------------------------------------------------------------- kernels
@@ -226,6 +253,10 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
         __syncthreads();
+        if (threadIdx.x == 0) {
+            prefetch_l2(d.m + tb0 * C, nb * C * 4);
+            prefetch_l2(d.v + tb0 * C, nb * C * 4);
+        }
         stage_in(s_pi, d.pi + tb0 * C, nb * C);
         __syncthreads();
         if ((int)threadIdx.x < nb) {
@@ -261,22 +292,49 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
             });
         }
         __syncthreads();
-        // AdamW over the tile as one flat, coalesced array.
-        const int n = nb * C;
-        float *pi = d.pi + tb0 * C, *mm = d.m + tb0 * C, *vv = d.v + tb0 * C;
-        float *gout = d.grad ? d.grad + tb0 * C : nullptr;
-        for (int i = threadIdx.x; i < n; i += kCtaThreads) {
-            float p = s_pi[i], m = __ldcs(mm + i), v = __ldcs(vv + i);
-            const float g = s_gr[i];
-            const float pd = __fmul_rn(p, sc.decay);
-            m = __fmaf_rn(sc.beta1, m, __fmul_rn(sc.one_minus_beta1, g));
-            v = __fmaf_rn(sc.beta2, v, __fmul_rn(sc.one_minus_beta2, __fmul_rn(g, g)));
-            const float denom = __fmaf_rn(__fsqrt_rn(v), sc.inv_sqrt_bc2, sc.eps);
-            p = __fmaf_rn(-sc.step_size, __fdividef(m, denom), pd);
-            __stcs(pi + i, p);
-            __stcs(mm + i, m);
-            __stcs(vv + i, v);
-            if (gout) __stcs(gout + i, g);
+        // AdamW over the tile as one flat, coalesced array of float4: each thread first loads
+        // kUnroll vectors of m and v (prefetched into L2 at the start of the tile), then
+        // updates them, so every thread keeps 2*kUnroll loads in flight.
+        const int n = nb * C, n4 = n >> 2;
+        float *__restrict__ pi = d.pi + tb0 * C;
+        float *__restrict__ mm = d.m + tb0 * C;
+        float *__restrict__ vv = d.v + tb0 * C;
+        float *__restrict__ gout = d.grad ? d.grad + tb0 * C : nullptr;
+        constexpr int kUnroll = 6;
+        for (int i0 = threadIdx.x; i0 < n4; i0 += kCtaThreads * kUnroll) {
+            float4 m4[kUnroll], v4[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = i0 + u * kCtaThreads;
+                if (i < n4) {
+                    m4[u] = __ldcs(reinterpret_cast<const float4 *>(mm) + i);
+                    v4[u] = __ldcs(reinterpret_cast<const float4 *>(vv) + i);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int i = i0 + u * kCtaThreads;
+                if (i < n4) {
+                    float4 p4 = reinterpret_cast<const float4 *>(s_pi)[i];
+                    const float4 g4 = reinterpret_cast<const float4 *>(s_gr)[i];
+                    adamw(p4.x, m4[u].x, v4[u].x, g4.x, sc);
+                    adamw(p4.y, m4[u].y, v4[u].y, g4.y, sc);
+                    adamw(p4.z, m4[u].z, v4[u].z, g4.z, sc);
+                    adamw(p4.w, m4[u].w, v4[u].w, g4.w, sc);
+                    __stcs(reinterpret_cast<float4 *>(pi) + i, p4);
+                    __stcs(reinterpret_cast<float4 *>(mm) + i, m4[u]);
+                    __stcs(reinterpret_cast<float4 *>(vv) + i, v4[u]);
+                    if (gout) __stcs(reinterpret_cast<float4 *>(gout) + i, g4);
+                }
+            }
+        }
+        if ((n & 3) && threadIdx.x == 0) {  // 2-float tail of a tile with an odd block count
+            for (int i = 4 * n4; i < n; ++i) {
+                float p = s_pi[i], m = mm[i], v = vv[i];
+                adamw(p, m, v, s_gr[i], sc);
+                pi[i] = p; mm[i] = m; vv[i] = v;
+                if (gout) gout[i] = s_gr[i];
+            }
         }
     }
 }
@@ -343,11 +401,18 @@ __global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constan
             }
         }
         __syncthreads();
-        const int n = nb * C;
+        const int n = nb * C, n4 = n >> 2;
         stage_out(d.pi + tb0 * C, s_pi, n);
-        for (int i = threadIdx.x; i < n; i += kCtaThreads) {
-            if (d.m) __stcs(d.m + tb0 * C + i, 0.f);
-            if (d.v) __stcs(d.v + tb0 * C + i, 0.f);
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = threadIdx.x; i < n4; i += kCtaThreads) {
+            if (d.m) __stcs(reinterpret_cast<float4 *>(d.m + tb0 * C) + i, z4);
+            if (d.v) __stcs(reinterpret_cast<float4 *>(d.v + tb0 * C) + i, z4);
+        }
+        if ((n & 3) && threadIdx.x == 0) {
+            for (int i = 4 * n4; i < n; ++i) {
+                if (d.m) d.m[tb0 * C + i] = 0.f;
+                if (d.v) d.v[tb0 * C + i] = 0.f;
+            }
         }
     }
 }

@@ -466,6 +466,20 @@ mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool w32 = mats[0].w_dtype == MLLM_F32;
     const bool is24 = nm.m == 4;
+    // 2:4 rows of whole metadata words (cols % 32 == 0, every LLM shape) take the pair kernel
+    bool words_aligned = true;
+    for (int32_t i = 0; i < n_mats; ++i) words_aligned = words_aligned && ((mats[i].cols / 4) % 8 == 0);
+    if (is24 && words_aligned) {
+        for (const Group &g : make_groups(mats, n_mats, nm.m, Kind::Sample24)) {
+            if (g.total_work == 0) continue;
+            const void *fn = w32 ? (const void *)k24::pack_pairs_kernel<true> : (const void *)k24::pack_pairs_kernel<false>;
+            const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k24::pack_pairs_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g);
+            else k24::pack_pairs_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g);
+            if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+        }
+        return MLLM_OK;
+    }
     for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Pack24 : Kind::Pack48)) {
         if (g.total_work == 0) continue;
         if (is24) {

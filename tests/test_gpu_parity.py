@@ -301,6 +301,7 @@ def test_prior_random_parity(orc, nm):
 # ------------------------------------------------------------------------------ hard pack
 
 @pytest.mark.parametrize("nm,shapes", [((2, 4), [(64, 128), (3, 12), (5, 36), (7, 4)]),
+                                       ((2, 4), [(64, 128), (33, 256), (5, 32), (1, 96)]),
                                        ((4, 8), [(64, 128), (3, 16), (5, 24)])])
 @pytest.mark.parametrize("w_dtype", ["bf16", "f32"])
 def test_pack_bit_exact(orc, nm, shapes, w_dtype):
