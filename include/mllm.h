@@ -40,7 +40,8 @@
  *     (gid lo32, gid hi32, s, c/6), gid = block_offset + b; field c%6 = bits [21(c%6),
  *     21(c%6)+21) of the 128-bit output (word 0 least significant) is k, eps =
  *     (2k+1)*2^-22, and g = -nlog(-nlog(eps)) with nlog the fp32 table-driven logarithm
- *     fixed by the specification (Tang's method, a 128-entry table, a cubic remainder).
+ *     fixed by the specification (Tang's method: x = 2^e mm, a 7-bit mantissa prefix j,
+ *     r = fma(mm, c_j, -1), ln x = T[e][j] + (r - r^2/2 + r^3/3); see mllm_noise_table).
  *     Step 0xFFFFFFFF is reserved for mllm_prior_init. The same (seed, step) gives
  *     bit-identical noise in forward and backward; noise is recomputed, never stored.
  */
@@ -190,6 +191,11 @@ mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, 
  * reserved one. */
 mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t *gids,
                        int64_t n_blocks, float *g_out, void *stream);
+
+/* The logarithm table the noise uses, as compiled into the kernels (host memory, for
+ * inspection and tests): c_out[j] = fl32(1/F_j), j = 0..127, and t_out[(e + 22)*128 + j] =
+ * fl32(e ln2 - ln c_j) for e = -22..4 (27*128 entries). No device work. */
+mllm_status mllm_noise_table(float *c_out, float *t_out);
 
 /* Workspace bytes mllm_sample_fwd needs for its regulariser sum (independent of sizes). */
 size_t mllm_workspace_bytes(void);

@@ -142,11 +142,12 @@ def nlog_array(x) -> np.ndarray:
 
 
 def nlog_table():
+    """(c [128], T [27, 128] for exponents -22..4, (1/3, emin, emax)) of nlog."""
     c = np.zeros(128, np.float32)
-    L = np.zeros(128, np.float32)
+    T = np.zeros((27, 128), np.float32)
     k = np.zeros(3, np.float32)
-    lib().orc_nlog_table(_ptr(c), _ptr(L), _ptr(k))
-    return c, L, k
+    lib().orc_nlog_table(_ptr(c), _ptr(T), _ptr(k))
+    return c, T, k
 
 
 def noise(n, m, seed, step, gids):

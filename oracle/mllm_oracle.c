@@ -24,8 +24,8 @@
  *       random numbers: as easy as 1, 2, 3") -> 21-bit field k -> eps = (2k+1) 2^-22 ->
  *       t = -nlog(eps) -> g = -nlog(t), with nlog the fp32 table-driven logarithm below
  *       (the method of P.T.P. Tang, "Table-driven implementation of the logarithm function
- *       in IEEE floating-point arithmetic", ACM TOMS 16(4), 1990, with a 128-entry table
- *       and a degree-3 Taylor remainder);
+ *       in IEEE floating-point arithmetic", ACM TOMS 16(4), 1990: a table indexed by the
+ *       binary exponent and a 7-bit mantissa prefix, and a degree-3 Taylor remainder);
  *   (2) the perturbed logit w = fma(kappa, pi, g), one fp32 rounding.
  * The flag `round_w = 0` evaluates w = kappa*pi + g in double instead (used only by the
  * finite-difference and autograd pins, where a rounding step would be a staircase).
@@ -143,26 +143,26 @@ static uint32_t candidate_field(uint64_t seed, uint64_t gid, uint32_t step, int 
 /* x = 2^e * mm with mm within 2^-8 of a breakpoint F_j. j is the 7-bit mantissa prefix of
  * x rounded to nearest; prefixes j >= 64 (mantissa >= 1.5) move to the next binade, so
  * F_j = 1 + j/128 for j < 64 and (1 + j/128)/2 for j >= 64, both in [0.75, 1.5).
- * c_j = fl32(1/F_j), L_j = fl32(-ln c_j) (ln evaluated in double). With r = fma(mm, c_j, -1),
- * |r| < 2^-8, ln x = e ln2 + L_j + ln(1 + r), and ln(1 + r) = r - r^2/2 + r^3/3 + O(r^4).
- * ln2 is split (Cody & Waite) into LN2_HI, fp32(ln 2) with its low 8 mantissa bits
- * cleared so that e*LN2_HI is exact, and LN2_LO = fl32(ln 2 - LN2_HI). */
-static float NLOG_C[128], NLOG_L[128];
-static float LN2_HI, LN2_LO, ONE_THIRD;
+ * c_j = fl32(1/F_j). With r = fma(mm, c_j, -1), |r| < 2^-8,
+ *   ln x = e ln2 - ln c_j + ln(1 + r),  ln(1 + r) = r - r^2/2 + r^3/3 + O(r^4),
+ * and T[e][j] = fl32(e ln2 - ln c_j) (evaluated in double, rounded once) carries the first
+ * two terms. The noise only ever takes logarithms of x in [2^-22, 16) (eps >= 2^-22 and
+ * t = -ln eps <= 15.25), so e runs over [-22, 4]: 27 rows of 128 entries. Outside that
+ * domain nlog is not defined (this implementation returns NaN). */
+#define NLOG_EMIN (-22)
+#define NLOG_EMAX 4
+#define NLOG_ROWS (NLOG_EMAX - NLOG_EMIN + 1)
+static float NLOG_C[128], NLOG_T[NLOG_ROWS][128];
+static float ONE_THIRD;
 
 static void build_nlog(void) {
     for (int j = 0; j < 128; j++) {
         double F = (j < 64) ? (1.0 + j / 128.0) : (1.0 + j / 128.0) / 2.0;
-        float c = (float)(1.0 / F);
-        NLOG_C[j] = c;
-        NLOG_L[j] = (float)(-log((double)c));
+        NLOG_C[j] = (float)(1.0 / F);
     }
-    float ln2f = (float)M_LN2;
-    uint32_t b;
-    memcpy(&b, &ln2f, 4);
-    b &= 0xFFFFFF00u;
-    memcpy(&LN2_HI, &b, 4);
-    LN2_LO = (float)(M_LN2 - (double)LN2_HI);
+    for (int e = NLOG_EMIN; e <= NLOG_EMAX; e++)
+        for (int j = 0; j < 128; j++)
+            NLOG_T[e - NLOG_EMIN][j] = (float)((double)e * M_LN2 - log((double)NLOG_C[j]));
     ONE_THIRD = (float)(1.0 / 3.0);
 }
 
@@ -172,6 +172,7 @@ static float nlog(float x) {
     uint32_t ib = b + 0x8000u;                 /* round the mantissa at its 7-bit prefix */
     uint32_t j = (ib >> 16) & 0x7Fu;
     int32_t e = (int32_t)(ib >> 23) - 127 + (int32_t)(j >> 6);
+    if (!(x > 0.0f) || e < NLOG_EMIN || e > NLOG_EMAX) return NAN;
     uint32_t mb = b - ((uint32_t)e << 23);     /* mm = x * 2^-e, exact */
     float mm;
     memcpy(&mm, &mb, 4);
@@ -179,10 +180,7 @@ static float nlog(float x) {
     float q = fmaf(r, ONE_THIRD, -0.5f);
     float rq = r * q;
     float p = fmaf(rq, r, r);                  /* r - r^2/2 + r^3/3 */
-    float ef = (float)e;
-    float hi = fmaf(ef, LN2_HI, NLOG_L[j]);
-    float lo = fmaf(ef, LN2_LO, p);
-    return hi + lo;
+    return NLOG_T[e - NLOG_EMIN][j] + p;
 }
 
 float orc_nlog(float x) { return nlog(x); }
@@ -191,9 +189,14 @@ void orc_nlog_array(int64_t n, const float *x, float *out) {
     for (int64_t i = 0; i < n; i++) out[i] = nlog(x[i]);
 }
 
-void orc_nlog_table(float *c, float *L, float *consts) {
-    for (int j = 0; j < 128; j++) { c[j] = NLOG_C[j]; L[j] = NLOG_L[j]; }
-    consts[0] = LN2_HI; consts[1] = LN2_LO; consts[2] = ONE_THIRD;
+/* c [128], T [27 * 128] (row e - NLOG_EMIN), consts[0] = fl32(1/3), consts[1..2] = e range. */
+void orc_nlog_table(float *c, float *T, float *consts) {
+    for (int j = 0; j < 128; j++) c[j] = NLOG_C[j];
+    for (int r = 0; r < NLOG_ROWS; r++)
+        for (int j = 0; j < 128; j++) T[r * 128 + j] = NLOG_T[r][j];
+    consts[0] = ONE_THIRD;
+    consts[1] = (float)NLOG_EMIN;
+    consts[2] = (float)NLOG_EMAX;
 }
 
 /* eps = (2k+1) 2^-22, exact in fp32, strictly inside (0, 1). */

@@ -90,6 +90,7 @@ _SIGS = {
     "mllm_hard_pack": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P]),
     "mllm_noise": (ctypes.c_int, [NM, ctypes.c_uint64, ctypes.c_uint32, _P, ctypes.c_int64, _P, _P]),
     "mllm_workspace_bytes": (ctypes.c_size_t, []),
+    "mllm_noise_table": (ctypes.c_int, [_P, _P]),
     "mllm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mllm_last_cuda_error": (ctypes.c_int32, []),
     "mllm_abi_version": (ctypes.c_int32, []),
@@ -272,6 +273,16 @@ def mllm_hard_pack(mats, nm, stream=None):
 def mllm_noise(nm, seed: int, step: int, gids: torch.Tensor, g_out: torch.Tensor, stream=None):
     _check(lib().mllm_noise(_nm(nm), int(seed), int(step), _ptr(gids), int(gids.numel()),
                             _ptr(g_out), _stream(stream)), "mllm_noise")
+
+
+def mllm_noise_table():
+    """(c [128], T [27, 128]) of the noise logarithm as compiled into the kernels."""
+    import numpy as np
+
+    c = np.zeros(128, np.float32)
+    T = np.zeros((27, 128), np.float32)
+    _check(lib().mllm_noise_table(c.ctypes.data, T.ctypes.data), "mllm_noise_table")
+    return c, T
 
 
 def mllm_last_cuda_error() -> int:

@@ -5,9 +5,11 @@
 // block, step, group); six 21-bit fields k give uniforms eps = (2k+1) 2^-22 and the Gumbel
 // noise g = -nlog(-nlog(eps)) of MaskLLM's Eq.5 (paper-graph-ui summary, s.3.4 "Step 1").
 // nlog is the fp32 table-driven logarithm of P.T.P. Tang (ACM TOMS 16(4), 1990): a 7-bit
-// mantissa prefix selects a breakpoint F in [0.75, 1.5), r = x 2^-e / F - 1 with |r| < 2^-8,
-// ln(1+r) ~ r - r^2/2 + r^3/3. Only correctly rounded fp32 operations (fma, mul, add,
-// int->float) are used, so the bits are fixed by the definition on any IEEE machine.
+// mantissa prefix j selects a breakpoint F_j in [0.75, 1.5) and x = 2^e mm, r = mm c_j - 1
+// with c_j = fl32(1/F_j) and |r| < 2^-8; ln x = T[e][j] + (r - r^2/2 + r^3/3) with
+// T[e][j] = fl32(e ln2 - ln c_j). Only correctly rounded fp32 operations (fma, mul, add) act
+// on the data, so the bits are fixed by the definition on any IEEE machine. The noise takes
+// logarithms of x in [2^-22, 16) only, so e runs over [-22, 4].
 #pragma once
 
 #include <cstdint>
@@ -20,14 +22,48 @@ constexpr int kMaxMats = 16;             // matrices per launch; larger groups a
 constexpr uint32_t kInitStep = 0xFFFFFFFFu;
 constexpr int kThreads = 256;            // threads per CTA for every sampler kernel
 
-// Logarithm table and constants, built once on the host from their definitions:
-// F_j = 1 + j/128 (j < 64) or (1 + j/128)/2 (j >= 64); c_j = fl32(1/F_j);
-// L_j = fl32(-ln c_j); ln2_hi = fl32(ln 2) with the low 8 mantissa bits cleared;
-// ln2_lo = fl32(ln 2 - ln2_hi); one_third = fl32(1/3).
-struct NoiseTab {
-    float2 cl[128];  // (c_j, L_j)
-    float ln2_hi, ln2_lo, one_third, pad;
+// ---------------------------------------------------------------------------- nlog table
+
+constexpr int kNlogEmin = -22, kNlogEmax = 4;
+constexpr int kNlogRows = kNlogEmax - kNlogEmin + 1;  // 27
+constexpr int kNlogEntries = kNlogRows * 128;        // 3456 (c_j, T[e][j]) pairs, 27 KB
+
+// Natural logarithm in double, for building the table at compile time: x = m 2^k with m in
+// [0.75, 1.5), ln m = 2 atanh((m-1)/(m+1)) by its series (|s| <= 0.2, 40 terms). Accurate to a
+// few double ulps; every table entry lies more than 2^-20 fp32 ulp from a rounding boundary,
+// so rounding this to fp32 gives the correctly rounded entry.
+constexpr double kLn2 = 0.693147180559945309417232121458176568;
+constexpr double cx_ln(double x) {
+    int k = 0;
+    while (x >= 1.5) { x *= 0.5; ++k; }
+    while (x < 0.75) { x *= 2.0; --k; }
+    const double s = (x - 1.0) / (x + 1.0), s2 = s * s;
+    double term = s, sum = 0.0;
+    for (int i = 1; i < 80; i += 2) { sum += term / i; term *= s2; }
+    return 2.0 * sum + k * kLn2;
+}
+
+// The table in the order the kernels index it. With ib2 = bits(x) + 0x408000 (rounding the
+// mantissa at its 7-bit prefix, plus half a binade), ib2 >> 23 = e + 127 and bits 16..22 of
+// ib2 are j ^ 64 (prefixes j >= 64 carry into the exponent), so entry (ib2 >> 16) - 105*128
+// = (e + 22)*128 + (j ^ 64) holds (c_j, T[e][j]).
+struct NoiseTable {
+    float2 cT[kNlogEntries];
+    constexpr NoiseTable() : cT{} {
+        for (int row = 0; row < kNlogRows; ++row) {
+            const int e = row + kNlogEmin;
+            for (int jr = 0; jr < 128; ++jr) {
+                const int j = jr ^ 64;
+                const double F = (j < 64) ? (1.0 + j / 128.0) : (1.0 + j / 128.0) * 0.5;
+                const float c = (float)(1.0 / F);
+                cT[row * 128 + jr] = float2{c, (float)((double)e * kLn2 - cx_ln((double)c))};
+            }
+        }
+    }
 };
+__device__ const NoiseTable g_noise_table{};
+constexpr uint32_t kNlogIndexBias = (127u + kNlogEmin) * 128u;  // 13440
+constexpr float kOneThird = (float)(1.0 / 3.0);
 
 // One matrix of a grouped launch. work_begin/work_count are in the kernel's work units
 // (tiles of kThreads pairs of blocks, or of packed words).
@@ -114,42 +150,39 @@ __device__ __forceinline__ float uniform_from_field(uint32_t k) {
 
 // ---------------------------------------------------------------------------- nlog
 
-__device__ __forceinline__ float nlog(float x, const float2 *__restrict__ tab, float ln2_hi,
-                                      float ln2_lo, float one_third) {
+// nlog(x) for x in [2^-22, 16). kClamp bounds the table index (one instruction); it is
+// applied to the second logarithm, whose argument comes from arithmetic, not from bits.
+template <bool kClamp>
+__device__ __forceinline__ float nlog(float x, const float2 *__restrict__ tab) {
     const uint32_t b = __float_as_uint(x);
-    const uint32_t ib = b + 0x8000u;               // nearest 7-bit mantissa prefix
-    const uint32_t j = (ib >> 16) & 0x7Fu;
-    const int32_t e = (int32_t)(ib >> 23) - 127 + (int32_t)(j >> 6);
-    const float mm = __uint_as_float(b - ((uint32_t)e << 23));  // x 2^-e, exact
-    const float2 cl = tab[j];
-    const float r = __fmaf_rn(mm, cl.x, -1.0f);
-    const float q = __fmaf_rn(r, one_third, -0.5f);
+    const uint32_t ib2 = b + 0x408000u;
+    uint32_t idx = (ib2 >> 16) - kNlogIndexBias;
+    if (kClamp) idx = min(idx, (uint32_t)(kNlogEntries - 1));
+    const float2 cT = tab[idx];
+    const float mm = __uint_as_float(b - (ib2 & 0x7F800000u) + 0x3F800000u);  // x 2^-e, exact
+    const float r = __fmaf_rn(mm, cT.x, -1.0f);
+    const float q = __fmaf_rn(r, kOneThird, -0.5f);
     const float rq = __fmul_rn(r, q);
     const float p = __fmaf_rn(rq, r, r);
-    const float ef = __int2float_rn(e);
-    const float hi = __fmaf_rn(ef, ln2_hi, cl.y);
-    const float lo = __fmaf_rn(ef, ln2_lo, p);
-    return __fadd_rn(hi, lo);
+    return __fadd_rn(cT.y, p);
 }
 
 struct NlogCtx {
     const float2 *tab;
-    float ln2_hi, ln2_lo, one_third;
-    __device__ __forceinline__ float operator()(float x) const {
-        return nlog(x, tab, ln2_hi, ln2_lo, one_third);
-    }
 };
 
 // g = -log(-log eps) for field k (the negations are exact).
 __device__ __forceinline__ float gumbel(uint32_t k, const NlogCtx &L) {
     const float eps = uniform_from_field(k);
-    const float t = -L(eps);
-    return -L(t);
+    const float t = -nlog<false>(eps, L.tab);
+    return -nlog<true>(t, L.tab);
 }
 
-// Copy the table into shared memory (call with all threads, then __syncthreads()).
-__device__ __forceinline__ void load_tab(float2 *s_tab, const NoiseTab &tab) {
-    for (int i = threadIdx.x; i < 128; i += blockDim.x) s_tab[i] = tab.cl[i];
+// Copy the table into shared memory (all threads; __syncthreads() before use).
+__device__ __forceinline__ void load_tab(float2 *s_tab) {
+    const float4 *src = reinterpret_cast<const float4 *>(g_noise_table.cT);
+    float4 *dst = reinterpret_cast<float4 *>(s_tab);
+    for (int i = threadIdx.x; i < kNlogEntries / 2; i += blockDim.x) dst[i] = src[i];
 }
 
 // ---------------------------------------------------------------------------- misc

@@ -183,14 +183,13 @@ __device__ __forceinline__ void reduce_to_global(float acc, double *partials, un
 
 template <bool kW32>
 __global__ void __launch_bounds__(kThreads) fwd_kernel(const __grid_constant__ Group grp,
-                                                       const __grid_constant__ NoiseTab tab,
                                                        const StepScalars sc, double *partials,
                                                        unsigned int *ticket, double *reg_out,
                                                        int accumulate) {
-    __shared__ float2 s_tab[128];
-    load_tab(s_tab, tab);
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
+    load_tab(s_tab);
     __syncthreads();
-    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    const NlogCtx L{s_tab};
     float acc = 0.f;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
         const MatDesc &d = grp.d[find_mat(grp, t)];
@@ -227,12 +226,11 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const __grid_constant__ G
 
 template <bool kW32, bool kG32>
 __global__ void __launch_bounds__(kThreads) bwd_adam_kernel(const __grid_constant__ Group grp,
-                                                            const __grid_constant__ NoiseTab tab,
                                                             const StepScalars sc) {
-    __shared__ float2 s_tab[128];
-    load_tab(s_tab, tab);
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
+    load_tab(s_tab);
     __syncthreads();
-    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    const NlogCtx L{s_tab};
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
         const MatDesc &d = grp.d[find_mat(grp, t)];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;

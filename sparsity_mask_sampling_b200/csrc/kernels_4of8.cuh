@@ -22,6 +22,7 @@ constexpr int C = 70;
 constexpr int kCtaThreads = 128;
 constexpr int kBlocksPerCta = kCtaThreads;  // one block per thread
 constexpr int kTileFloats = kBlocksPerCta * C;
+constexpr int kFwdDynSmem = kTileFloats * (int)sizeof(float);
 constexpr int kBwdDynSmem = 2 * kTileFloats * (int)sizeof(float);
 
 // Keep mask (bit j = position j) of candidate i: the i-th 4-subset of {0..7} in
@@ -166,14 +167,14 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
 
 template <bool kW32>
 __global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant__ Group grp,
-                                                          const __grid_constant__ NoiseTab tab,
                                                           const StepScalars sc, double *partials,
                                                           unsigned int *ticket, double *reg_out,
                                                           int accumulate) {
-    __shared__ float2 s_tab[128];
-    __shared__ __align__(16) float s_pi[kTileFloats];
-    load_tab(s_tab, tab);
-    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
+    extern __shared__ __align__(16) float s_dyn[];  // [kTileFloats] logits of the tile
+    float *s_pi = s_dyn;
+    load_tab(s_tab);
+    const NlogCtx L{s_tab};
     float acc = 0.f;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
         const MatDesc &d = grp.d[find_mat(grp, t)];
@@ -241,13 +242,12 @@ __global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant_
 
 template <bool kW32, bool kG32>
 __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_constant__ Group grp,
-                                                               const __grid_constant__ NoiseTab tab,
                                                                const StepScalars sc) {
-    __shared__ float2 s_tab[128];
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
     extern __shared__ __align__(16) float s_dyn[];  // [2 * kTileFloats]: logits, gradients
     float *s_pi = s_dyn, *s_gr = s_dyn + kTileFloats;
-    load_tab(s_tab, tab);
-    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    load_tab(s_tab);
+    const NlogCtx L{s_tab};
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
         const MatDesc &d = grp.d[find_mat(grp, t)];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
@@ -467,14 +467,14 @@ __global__ void __launch_bounds__(kCtaThreads) pack_kernel(const __grid_constant
 }  // namespace k48
 
 // Gumbel noise of arbitrary blocks for inspection: one thread per block, C values each.
-__global__ void __launch_bounds__(kThreads) noise_kernel(const __grid_constant__ NoiseTab tab, int C,
+__global__ void __launch_bounds__(kThreads) noise_kernel(int C,
                                                          uint64_t seed, uint32_t step,
                                                          const uint64_t *__restrict__ gids,
                                                          int64_t n, float *__restrict__ out) {
-    __shared__ float2 s_tab[128];
-    load_tab(s_tab, tab);
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
+    load_tab(s_tab);
     __syncthreads();
-    const NlogCtx L{s_tab, tab.ln2_hi, tab.ln2_lo, tab.one_third};
+    const NlogCtx L{s_tab};
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const uint64_t gid = gids[i];
         for (int gr = 0; gr * 6 < C; ++gr) {

@@ -22,32 +22,6 @@ constexpr int kMaxReduceCtas = 4096;
 constexpr size_t kWsPartialsOffset = 16;
 constexpr size_t kWorkspaceBytes = kWsPartialsOffset + sizeof(double) * kMaxReduceCtas;
 
-// ------------------------------------------------------------------------ noise table
-
-NoiseTab build_noise_tab() {
-    NoiseTab t{};
-    for (int j = 0; j < 128; ++j) {
-        const double F = (j < 64) ? (1.0 + j / 128.0) : (1.0 + j / 128.0) * 0.5;
-        const float c = (float)(1.0 / F);
-        t.cl[j] = make_float2(c, (float)(-std::log((double)c)));
-    }
-    const double ln2 = std::log(2.0);
-    float hi = (float)ln2;
-    uint32_t bits;
-    std::memcpy(&bits, &hi, 4);
-    bits &= 0xFFFFFF00u;  // clear 8 low mantissa bits: e * ln2_hi exact for |e| < 256
-    std::memcpy(&hi, &bits, 4);
-    t.ln2_hi = hi;
-    t.ln2_lo = (float)(ln2 - (double)hi);
-    t.one_third = (float)(1.0 / 3.0);
-    return t;
-}
-
-const NoiseTab &noise_tab() {
-    static const NoiseTab tab = build_noise_tab();
-    return tab;
-}
-
 // ------------------------------------------------------------------------ device info
 
 struct OccKey {
@@ -69,15 +43,15 @@ int sm_count(int dev) {
     return g_sms[dev];
 }
 
-// Resident CTAs per SM of a kernel on a device (first use also raises the kernel's dynamic
-// shared-memory limit when it needs more than the 48 KB default).
+// Resident CTAs per SM of a kernel on a device (first use also sets the kernel's dynamic
+// shared-memory limit to what its launches request).
 int resident_ctas(int dev, const void *fn, int threads, int dyn_smem) {
     {
         std::lock_guard<std::mutex> lk(g_occ_mu);
         for (auto &e : g_occ)
             if (e.first.dev == dev && e.first.fn == fn) return e.second;
     }
-    if (dyn_smem > 48 * 1024) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+    if (dyn_smem > 0) cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, dyn_smem) != cudaSuccess || n <= 0) n = 1;
     std::lock_guard<std::mutex> lk(g_occ_mu);
@@ -296,6 +270,18 @@ int32_t mllm_num_candidates(mllm_nm nm) { return num_cand(nm); }
 
 size_t mllm_workspace_bytes(void) { return kWorkspaceBytes; }
 
+mllm_status mllm_noise_table(float *c_out, float *t_out) {
+    if (!c_out || !t_out) return MLLM_ERR_INVALID_ARG;
+    static constexpr NoiseTable tab{};  // the same compile-time table as g_noise_table
+    for (int row = 0; row < kNlogRows; ++row)
+        for (int jr = 0; jr < 128; ++jr) {
+            const int j = jr ^ 64;
+            if (row == 0) c_out[j] = tab.cT[jr].x;
+            t_out[row * 128 + j] = tab.cT[row * 128 + jr].y;
+        }
+    return MLLM_OK;
+}
+
 int32_t mllm_abi_version(void) { return MLLM_ABI_VERSION; }
 size_t mllm_sizeof_matrix(void) { return sizeof(mllm_matrix); }
 size_t mllm_sizeof_hparams(void) { return sizeof(mllm_hparams); }
@@ -363,13 +349,13 @@ mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
         if (is24) {
             const void *fn = w32 ? (const void *)k24::fwd_kernel<true> : (const void *)k24::fwd_kernel<false>;
             const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, kMaxReduceCtas);
-            if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
-            else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         } else {
             const void *fn = w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>;
-            const int64_t grid = grid_for(fn, k48::kCtaThreads, 0, g.total_work, kMaxReduceCtas);
-            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
-            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            const int64_t grid = grid_for(fn, k48::kCtaThreads, k48::kFwdDynSmem, g.total_work, kMaxReduceCtas);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         }
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -392,11 +378,12 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
     const void *fn = is24 ? (w32 ? (const void *)k24::fwd_kernel<true> : (const void *)k24::fwd_kernel<false>)
                           : (w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>);
     const int threads = is24 ? kThreads : k48::kCtaThreads;
+    const int dyn_smem = is24 ? 0 : k48::kFwdDynSmem;
     const std::vector<Group> groups = make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48);
     // every launch's scratch need (one partial per CTA) is checked before anything runs
     for (const Group &g : groups) {
         if (g.total_work == 0) continue;
-        if (grid_for(fn, threads, 0, g.total_work, kMaxReduceCtas) > kNoallocMaxCtas) return MLLM_ERR_WORKSPACE;
+        if (grid_for(fn, threads, dyn_smem, g.total_work, kMaxReduceCtas) > kNoallocMaxCtas) return MLLM_ERR_WORKSPACE;
     }
     void *scratch = nullptr;
     if ((s = noalloc_scratch(&scratch)) != MLLM_OK) return s;
@@ -409,13 +396,13 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
         if (g.total_work == 0) continue;
         if ((s = cuda_status(cudaMemsetAsync(ticket, 0, sizeof(unsigned int), st))) != MLLM_OK) return s;
         const int accumulate = wrote_reg ? 1 : 0;
-        const int64_t grid = grid_for(fn, threads, 0, g.total_work, kMaxReduceCtas);
+        const int64_t grid = grid_for(fn, threads, dyn_smem, g.total_work, kMaxReduceCtas);
         if (is24) {
-            if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
-            else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         } else {
-            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
-            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, noise_tab(), sc, partials, ticket, reg_sum_out, accumulate);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         }
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -441,7 +428,7 @@ mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_n
     do {                                                                                         \
         const void *fn = (const void *)NS::bwd_adam_kernel<W32, G32>;                            \
         const int64_t grid = grid_for(fn, THREADS, SMEM, g.total_work, INT32_MAX);                 \
-        NS::bwd_adam_kernel<W32, G32><<<(unsigned)grid, THREADS, SMEM, st>>>(g, noise_tab(), sc); \
+        NS::bwd_adam_kernel<W32, G32><<<(unsigned)grid, THREADS, SMEM, st>>>(g, sc); \
     } while (0)
         if (is24) {
             if (w32 && g32) MLLM_LAUNCH_BWD(k24, kThreads, 0, true, true);
@@ -509,7 +496,7 @@ mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t 
     if ((s = check_ptr(g_out, true)) != MLLM_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t grid = std::min<int64_t>((n_blocks + kThreads - 1) / kThreads, INT32_MAX);
-    noise_kernel<<<(unsigned)grid, kThreads, 0, st>>>(noise_tab(), C, seed, step, gids, n_blocks, g_out);
+    noise_kernel<<<(unsigned)grid, kThreads, 0, st>>>(C, seed, step, gids, n_blocks, g_out);
     return cuda_status(cudaGetLastError());
 }
 

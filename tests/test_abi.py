@@ -153,3 +153,15 @@ def test_prior_and_pack_validation(M):
     assert L.mllm_noise(M.NM(2, 4), 0, 0, 0x1000, -1, 0x2000, 0) == M.MLLM_ERR_INVALID_ARG
     assert L.mllm_noise(M.NM(2, 5), 0, 0, 0x1000, 1, 0x2000, 0) == M.MLLM_ERR_UNSUPPORTED
     assert L.mllm_noise(M.NM(2, 4), 0, 0, 0x1000, 0, 0x2000, 0) == M.MLLM_OK  # nothing to do
+
+
+def test_compiled_noise_table_matches_oracle_table(M):
+    """The kernels' compile-time logarithm table equals the oracle's, bit for bit (the
+    oracle's is pinned to 50-digit logarithms)."""
+    import numpy as np
+    import oracle
+
+    c, T = M.mllm_noise_table()
+    oc, oT, _ = oracle.nlog_table()
+    assert np.array_equal(c.view(np.uint32), oc.view(np.uint32))
+    assert np.array_equal(T.view(np.uint32), oT.view(np.uint32))

@@ -129,14 +129,16 @@ def test_noise_bit_exact(orc, nm):
 
 
 def test_noise_every_uniform_value(orc):
-    """Every 21-bit field value maps to the same g on both sides: the GPU noise of many
-    blocks covers all 2^21 uniforms (checked through the oracle's eps of the same blocks)."""
-    gids = np.arange(1 << 20, dtype=np.uint64)
+    """The 25M draws of 2^22 blocks reach (all but a handful of) the 2^21 possible uniforms,
+    and with them every row of the logarithm table both logarithms use; every value is
+    bit-identical to the oracle's."""
+    gids = np.arange(1 << 22, dtype=np.uint64)
     out = torch.empty(len(gids), 6, dtype=torch.float32, device=DEV)
     mllm_noise((2, 4), 9, 3, torch.from_numpy(gids.view(np.int64)).to(DEV), out)
     eps, g_ref = orc.noise(2, 4, 9, 3, gids)
-    assert np.array_equal(out.cpu().numpy().view(np.uint32), g_ref.view(np.uint32))
-    assert len(np.unique(eps)) > 0.9 * (1 << 21)
+    got = out.cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), g_ref.view(np.uint32)), f"{np.sum(got != g_ref)} differ"
+    assert len(np.unique(eps)) > (1 << 21) - 64
 
 
 # ------------------------------------------------------------------------------ forward

@@ -2,7 +2,7 @@
 
 None of these compare the oracle with itself: the candidate set is checked against the page's
 listing and combinatorial counts, Philox against its published known answers, the bit
-slicing against big-integer arithmetic, nlog against 50-digit logarithms, and the noise
+slicing against big-integer arithmetic, nlog's table against 50-digit logarithms, and the noise
 against the Gumbel distribution's closed-form moments and the Gumbel-Max theorem.
 """
 import math
@@ -107,28 +107,28 @@ def _ulp32(x):
 
 
 def test_nlog_table_correctly_rounded(orc):
-    """c_j = fl32(1/F_j) and L_j = fl32(-ln c_j), checked with 50-digit logarithms; each L_j
-    also lies far from an fp32 rounding boundary, so any accurate double logarithm rounds to
-    the same fp32 value."""
+    """c_j = fl32(1/F_j) and T[e][j] = fl32(e ln2 - ln c_j), checked with 50-digit
+    logarithms; every T entry also lies far from an fp32 rounding boundary (more than 2^-20
+    of an ulp), so any logarithm accurate to ~1e-15 rounds to the same fp32 value."""
     getcontext().prec = 50
-    c, L, consts = orc.nlog_table()
+    c, T, consts = orc.nlog_table()
+    third, emin, emax = consts
+    assert third == np.float32(1 / 3) and (emin, emax) == (-22, 4) and T.shape == (27, 128)
+    ln2 = Decimal(2).ln()
     for j in range(128):
         F = (1 + j / 128) if j < 64 else (1 + j / 128) / 2
         assert c[j] == np.float32(1.0 / F)
-        exact = -Decimal(float(c[j])).ln()
-        f32 = np.float32(float(exact))
-        assert L[j] == f32
-        if exact != 0:
-            ulp = Decimal(_ulp32(f32))
-            dist = abs(exact - Decimal(float(f32)))
-            assert dist < ulp / 2 - ulp * Decimal(2) ** -20   # not near a midpoint
-    ln2_hi, ln2_lo, third = consts
-    assert third == np.float32(1 / 3)
-    # LN2_HI has its low 8 mantissa bits clear, so e * LN2_HI is exact for |e| < 256
-    assert np.array([ln2_hi], np.float32).view(np.uint32)[0] & 0xFF == 0
-    ln2 = Decimal(2).ln()
-    # LN2_LO is ln 2 - LN2_HI rounded once to fp32
-    assert abs(Decimal(float(ln2_hi)) + Decimal(float(ln2_lo)) - ln2) <= Decimal(_ulp32(ln2_lo)) / 2
+        lnc = Decimal(float(c[j])).ln()
+        for r, e in enumerate(range(-22, 5)):
+            exact = e * ln2 - lnc
+            f32 = np.float32(float(exact))
+            assert T[r, j] == f32, (e, j)
+            if exact != 0:
+                ulp = Decimal(_ulp32(f32))
+                dist = abs(exact - Decimal(float(f32)))
+                assert dist < ulp / 2 - ulp * Decimal(2) ** -20, (e, j)   # not near a midpoint
+            else:
+                assert T[r, j] == 0.0
 
 
 def test_nlog_accuracy_on_noise_domain(orc):
@@ -136,13 +136,25 @@ def test_nlog_accuracy_on_noise_domain(orc):
     uniform the generator can produce and a dense sweep of the second logarithm's inputs."""
     k = np.arange(2**21, dtype=np.float64)
     eps = ((2 * k + 1) / 2.0**22).astype(np.float32)
-    t = np.concatenate([eps, np.geomspace(2.0e-7, 16.0, 400_000).astype(np.float32),
+    t = np.concatenate([eps, np.geomspace(2.0**-22, 16.0, 400_000).astype(np.float32),
                         np.float32(1.0) + np.arange(-2000, 2000, dtype=np.float32) * np.float32(2**-23)])
     got = orc.nlog_array(t).astype(np.float64)
     ref = np.log(t.astype(np.float64))
     err = np.abs(got - ref)
     tol = np.maximum(2.0 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64), 2.0**-30)
     assert np.all(err <= tol), float(np.max(err / tol))
+
+
+def test_noise_stays_in_nlog_domain(orc):
+    """For every possible uniform, both logarithms of the noise transform take arguments in
+    [2^-22, 16): eps >= 2^-22 and t = -nlog(eps) in [2^-22, 15.25]."""
+    k = np.arange(2**21, dtype=np.float64)
+    eps = ((2 * k + 1) / 2.0**22).astype(np.float32)
+    t = -orc.nlog_array(eps)
+    assert np.all(np.isfinite(t)) and t.min() >= np.float32(2.0**-22) and t.max() < 16.0
+    g = -orc.nlog_array(t)
+    assert np.all(np.isfinite(g))
+    assert np.isnan(orc.nlog(2.0**-23)) and np.isnan(orc.nlog(32.0)) and np.isnan(orc.nlog(-1.0))
 
 
 # ---------------------------------------------------------------- Gumbel noise (Eq.5)
