@@ -100,6 +100,11 @@ WORKLOADS = {
         name="general_4of8", nm=(4, 8),
         matrices=(MatrixShape("up", 11008, 4096), MatrixShape("down", 4096, 11008)),
         steps=50, tau=(2.0, 2.0), kappa=(100.0, 100.0), lr=5e-4, seeds=(0,)),
+    # one 4096x4096 matrix at 4:8 (2.1M blocks, 0.6 GB of logits): a small case of the 4:8
+    # kernels for profiler captures (inputs still larger than L2)
+    "square_4096_4of8": Workload(
+        name="square_4096_4of8", nm=(4, 8), matrices=(MatrixShape("w", 4096, 4096),),
+        steps=50, tau=(2.0, 2.0), kappa=(100.0, 100.0), lr=5e-4, seeds=(0,)),
 }
 
 

@@ -46,7 +46,16 @@ constexpr double cx_ln(double x) {
 // The table in the order the kernels index it. With ib2 = bits(x) + 0x408000 (rounding the
 // mantissa at its 7-bit prefix, plus half a binade), ib2 >> 23 = e + 127 and bits 16..22 of
 // ib2 are j ^ 64 (prefixes j >= 64 carry into the exponent), so entry (ib2 >> 16) - 105*128
-// = (e + 22)*128 + (j ^ 64) holds (c_j, T[e][j]).
+// = (e + 22)*128 + (j ^ 64) holds (c_j 2^-e, T[e][j]). Storing c_j scaled by 2^-e (exact)
+// lets the kernel form r = fma(x, c_j 2^-e, -1), which equals fma(x 2^-e, c_j, -1) bit for
+// bit, without reconstructing the reduced argument x 2^-e.
+constexpr double cx_pow2(int e) {
+    double p = 1.0;
+    for (; e > 0; --e) p *= 2.0;
+    for (; e < 0; ++e) p *= 0.5;
+    return p;
+}
+
 struct NoiseTable {
     float2 cT[kNlogEntries];
     constexpr NoiseTable() : cT{} {
@@ -56,13 +65,14 @@ struct NoiseTable {
                 const int j = jr ^ 64;
                 const double F = (j < 64) ? (1.0 + j / 128.0) : (1.0 + j / 128.0) * 0.5;
                 const float c = (float)(1.0 / F);
-                cT[row * 128 + jr] = float2{c, (float)((double)e * kLn2 - cx_ln((double)c))};
+                cT[row * 128 + jr] = float2{(float)((double)c * cx_pow2(-e)),
+                                            (float)((double)e * kLn2 - cx_ln((double)c))};
             }
         }
     }
 };
 __device__ const NoiseTable g_noise_table{};
-constexpr uint32_t kNlogIndexBias = (127u + kNlogEmin) * 128u;  // 13440
+constexpr uint32_t kNlogIndexBias = (uint32_t)(127 + kNlogEmin) * 128u;  // 13440
 constexpr float kOneThird = (float)(1.0 / 3.0);
 
 // One matrix of a grouped launch. work_begin/work_count are in the kernel's work units
@@ -138,6 +148,19 @@ __device__ __forceinline__ void fields21(uint4 x, uint32_t f[6]) {
     f[5] = (x.w >> 9) & M21;
 }
 
+// The same six fields k, each already placed as the float bits of 1 + (2k+1) 2^-22: the
+// field shifted to bits 2..22 (one funnel shift two places short of the field's offset)
+// merged with the constant bits 0x3F800002 (one three-input logic op).
+__device__ __forceinline__ void fields21_unit(uint4 x, uint32_t u[6]) {
+    constexpr uint32_t MK = 0x7FFFFCu, ONE = 0x3F800002u;
+    u[0] = ((x.x << 2) & MK) | ONE;
+    u[1] = (__funnelshift_r(x.x, x.y, 19) & MK) | ONE;
+    u[2] = ((x.y >> 8) & MK) | ONE;
+    u[3] = (__funnelshift_r(x.y, x.z, 29) & MK) | ONE;
+    u[4] = (__funnelshift_r(x.z, x.w, 18) & MK) | ONE;
+    u[5] = ((x.w >> 7) & MK) | ONE;
+}
+
 __device__ __forceinline__ uint4 block_words(uint64_t seed, uint64_t gid, uint32_t step, uint32_t group) {
     return philox4x32_10(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), step, group),
                          (uint32_t)seed, (uint32_t)(seed >> 32));
@@ -154,13 +177,11 @@ __device__ __forceinline__ float uniform_from_field(uint32_t k) {
 // applied to the second logarithm, whose argument comes from arithmetic, not from bits.
 template <bool kClamp>
 __device__ __forceinline__ float nlog(float x, const float2 *__restrict__ tab) {
-    const uint32_t b = __float_as_uint(x);
-    const uint32_t ib2 = b + 0x408000u;
+    const uint32_t ib2 = __float_as_uint(x) + 0x408000u;
     uint32_t idx = (ib2 >> 16) - kNlogIndexBias;
     if (kClamp) idx = min(idx, (uint32_t)(kNlogEntries - 1));
     const float2 cT = tab[idx];
-    const float mm = __uint_as_float(b - (ib2 & 0x7F800000u) + 0x3F800000u);  // x 2^-e, exact
-    const float r = __fmaf_rn(mm, cT.x, -1.0f);
+    const float r = __fmaf_rn(x, cT.x, -1.0f);  // = fma(x 2^-e, c_j, -1)
     const float q = __fmaf_rn(r, kOneThird, -0.5f);
     const float rq = __fmul_rn(r, q);
     const float p = __fmaf_rn(rq, r, r);
@@ -174,6 +195,13 @@ struct NlogCtx {
 // g = -log(-log eps) for field k (the negations are exact).
 __device__ __forceinline__ float gumbel(uint32_t k, const NlogCtx &L) {
     const float eps = uniform_from_field(k);
+    const float t = -nlog<false>(eps, L.tab);
+    return -nlog<true>(t, L.tab);
+}
+
+// The same from the bits of 1 + eps (fields21_unit): eps = that - 1, exact.
+__device__ __forceinline__ float gumbel_unit(uint32_t unit_bits, const NlogCtx &L) {
+    const float eps = __fadd_rn(__uint_as_float(unit_bits), -1.0f);
     const float t = -nlog<false>(eps, L.tab);
     return -nlog<true>(t, L.tab);
 }

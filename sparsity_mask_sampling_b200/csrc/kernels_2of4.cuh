@@ -99,10 +99,10 @@ __device__ __forceinline__ void noise6(uint64_t seed, uint64_t gid, uint32_t ste
         for (int i = 0; i < C; ++i) g[i] = 0.f;
         return;
     }
-    uint32_t f[6];
-    fields21(block_words(seed, gid, step, 0u), f);
+    uint32_t u[6];
+    fields21_unit(block_words(seed, gid, step, 0u), u);
 #pragma unroll
-    for (int i = 0; i < C; ++i) g[i] = gumbel(f[i], L);
+    for (int i = 0; i < C; ++i) g[i] = gumbel_unit(u[i], L);
 }
 
 // Unnormalised soft index e_i = 2^((w_i - max w) c2) with w_i = fma(kappa, pi_i, g_i), and

@@ -273,10 +273,11 @@ size_t mllm_workspace_bytes(void) { return kWorkspaceBytes; }
 mllm_status mllm_noise_table(float *c_out, float *t_out) {
     if (!c_out || !t_out) return MLLM_ERR_INVALID_ARG;
     static constexpr NoiseTable tab{};  // the same compile-time table as g_noise_table
+    constexpr int row0 = -kNlogEmin;    // e = 0, where the stored c_j 2^-e is c_j itself
     for (int row = 0; row < kNlogRows; ++row)
         for (int jr = 0; jr < 128; ++jr) {
             const int j = jr ^ 64;
-            if (row == 0) c_out[j] = tab.cT[jr].x;
+            if (row == row0) c_out[j] = tab.cT[row * 128 + jr].x;
             t_out[row * 128 + j] = tab.cT[row * 128 + jr].y;
         }
     return MLLM_OK;
