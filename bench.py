@@ -111,97 +111,6 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ GPU arm
 
-class Stack:
-    """Device state of the workload: resident W, logits, moments; pooled X and G."""
-
-    def __init__(self, w, dev, rank, seed_base=0):
-        import torch
-        import sparsity_mask_sampling_b200 as pkg
-        from sparsity_mask_sampling_b200 import configs, inputs
-
-        self.w = w
-        self.dev = dev
-        self.nm = w.nm
-        self.C = w.C
-        from sparsity_mask_sampling_b200 import sharding
-
-        offs = sharding.weak_block_offsets(w, rank)
-        # X and G pools: two layers' worth, alternating (values do not change the cost)
-        self.pool = []
-        for p in range(2):
-            self.pool.append([(torch.empty(m.rows, m.cols, dtype=torch.bfloat16 if w.w_dtype == "bf16" else torch.float32, device=dev),
-                               inputs.upstream_grad(m.rows, m.cols, w.g_dtype, w.g_std, seed=seed_base + 1000 + 10 * p + i, device=dev))
-                              for i, m in enumerate(w.matrices)])
-        self.layers = []
-        self.bufs = []
-        for l in range(w.layers):
-            mats = []
-            for i, m in enumerate(w.matrices):
-                W = inputs.weights(m.rows, m.cols, w.w_dtype, w.w_std, seed=seed_base + 100 * l + i,
-                                   outlier_frac=w.outlier_frac, outlier_scale=w.outlier_scale, device=dev)
-                B = m.rows * m.cols // w.nm[1]
-                mb = pkg.MatrixBuffers(
-                    W=W, block_offset=offs[l][i],
-                    logits=torch.empty(B, w.C, dtype=torch.float32, device=dev),
-                    adam_m=torch.zeros(B, w.C, dtype=torch.float32, device=dev),
-                    adam_v=torch.zeros(B, w.C, dtype=torch.float32, device=dev))
-                mats.append(mb)
-            self.bufs.append(mats)
-            arr_views = []
-            for p in range(2):
-                for mb, (X, G) in zip(mats, self.pool[p]):
-                    mb.X, mb.G = X, G
-                arr_views.append(pkg.MatrixArray(mats))
-            self.layers.append(arr_views)  # [pool 0 view, pool 1 view]
-        self.ws = torch.zeros(pkg.mllm_workspace_bytes(), dtype=torch.uint8, device=dev)
-        self.reg = torch.zeros(w.layers, dtype=torch.float64, device=dev)
-        self.blocks = w.total_blocks()
-
-    def view(self, l):
-        return self.layers[l][l % 2]
-
-    def prior_init(self, seed=0):
-        import sparsity_mask_sampling_b200 as pkg
-
-        for l in range(self.w.layers):
-            pkg.mllm_prior_init(self.view(l), self.nm, self.w.alpha, self.w.init_std, seed)
-
-    def hparams(self, t, seed=0):
-        import sparsity_mask_sampling_b200 as pkg
-
-        T = max(self.w.steps, 1)
-        return pkg.Hparams(kappa=self.w.kappa_at(t % T), tau=self.w.tau_at(t % T), lambda_=self.w.lam,
-                           lr=self.w.lr, weight_decay=self.w.weight_decay, adam_step=t + 1, step=t,
-                           seed=seed).to_c()
-
-
-def run_step(stack, t, ev=None, g_ready=None, g_free=None, copy_fn=None):
-    """Enqueue one step. ev: optional dict of per-launch (start, end) event lists.
-    copy_fn(l, pool) enqueues the H2D copy of layer l's G (e2e leg)."""
-    import torch
-    import sparsity_mask_sampling_b200 as pkg
-
-    hp = stack.hparams(t)
-    nm = stack.nm
-    L = stack.w.layers
-    for l in range(L):
-        if ev is not None:
-            ev["fwd"][l][0].record()
-        pkg.mllm_sample_fwd(stack.view(l), nm, hp, stack.reg[l:l + 1], stack.ws)
-        if ev is not None:
-            ev["fwd"][l][1].record()
-    for l in reversed(range(L)):
-        if copy_fn is not None:
-            copy_fn(l)
-        if ev is not None:
-            ev["bwd"][l][0].record()
-        pkg.mllm_sample_bwd_adam(stack.view(l), nm, hp)
-        if ev is not None:
-            ev["bwd"][l][1].record()
-        if g_free is not None:
-            g_free[l % 2].record()
-
-
 def gpu_arm(args, w):
     import torch
     import torch.distributed as dist
@@ -219,8 +128,10 @@ def gpu_arm(args, w):
     pkg.lib()
     hbm_peak, peak_kind = peaks()
 
+    from sparsity_mask_sampling_b200.stack import SamplerStack
+
     t0 = time.time()
-    stack = Stack(w, dev, rank)
+    stack = SamplerStack(w, dev, rank)
     stack.prior_init(seed=0)
     torch.cuda.synchronize()
     log(f"[rank {rank}] stack ready: {stack.blocks:,} blocks, {torch.cuda.memory_allocated(dev)/1e9:.1f} GB, {time.time()-t0:.1f}s")
@@ -233,7 +144,7 @@ def gpu_arm(args, w):
 
     # warm-up
     for t in range(args.warmup):
-        run_step(stack, t)
+        stack.step(t)
         reduce_all()
     torch.cuda.synchronize()
 
@@ -252,7 +163,7 @@ def gpu_arm(args, w):
     end = torch.cuda.Event(enable_timing=True)
     start.record()
     for k in range(args.steps):
-        run_step(stack, args.warmup + k, ev=evs[k])
+        stack.step(args.warmup + k, ev=evs[k])
         reduce_all()
     end.record()
     torch.cuda.synchronize()
@@ -395,7 +306,7 @@ def e2e_leg(args, stack, w, world, dist, dev):
 
     steps = max(2, min(args.steps, 5))
     for t in range(1):
-        run_step(stack, 1000 + t, g_free=g_free, copy_fn=copy_fn)
+        stack.step(1000 + t, g_free=g_free, copy_fn=copy_fn)
         reg_host.copy_(stack.reg, non_blocking=True)
     torch.cuda.synchronize()
     if dist is not None:
@@ -403,7 +314,7 @@ def e2e_leg(args, stack, w, world, dist, dev):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for t in range(steps):
-        run_step(stack, 2000 + t, g_free=g_free, copy_fn=copy_fn)
+        stack.step(2000 + t, g_free=g_free, copy_fn=copy_fn)
         if dist is not None:
             dist.all_reduce(stack.reg, op=dist.ReduceOp.SUM)
         reg_host.copy_(stack.reg, non_blocking=True)
