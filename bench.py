@@ -1,17 +1,23 @@
 """Benchmark of the MaskLLM mask sampler's hot path on B200.
 
-One step = the forward of every weight matrix of the workload (one grouped launch per
-layer, layers 0 -> L-1) followed by the fused backward + AdamW of every matrix (layers
-L-1 -> 0), as in one training step of the method. Metric: blocks/s over the step
-(blocks = groups of M weights, each with its C logits), whole job; plus each kernel's
-achieved HBM bandwidth against the measured copy bandwidth.
+One step = every block of every weight matrix of the workload gets one forward (noise, soft
+index, soft mask, W.M, regulariser) and one backward + AdamW, as in one training step of
+the method. Default loop ("fused"): the forward of step 0 runs once before timing; then per
+step and per layer (in reverse order, as a backward pass visits them) one launch does step
+t's backward + AdamW and, from the updated logits, step t+1's forward. "--loop separate"
+times the unfused form: per step a forward launch per layer, then a backward + AdamW launch
+per layer in reverse. Metric: blocks/s over whole steps (blocks = groups of M weights, each
+with its C logits), whole job; plus each kernel's achieved HBM bandwidth against the
+measured copy bandwidth.
 
-  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--loop fused|separate]
+                  [--impl reference]
 
 Default workload: the full LLaMA-2-7B-shaped stack at 2:4 (32 layers x 7 matrices,
-1,619,001,344 blocks; logits and AdamW moments resident in HBM, ~130 GB). Under torchrun
-each rank runs its own stack (weak scaling, disjoint global block ids); the only exchange
-is an all-reduce of the step's regulariser sum.
+1,619,001,344 blocks; logits and AdamW moments resident in HBM, ~130 GB, plus the next
+step's soft-masked weights of every layer, 13 GB). Under torchrun each rank runs its own
+stack (weak scaling, disjoint global block ids); the only exchange is an all-reduce of the
+step's regulariser sums.
 """
 from __future__ import annotations
 
@@ -35,8 +41,9 @@ METRIC = "mask-sampling blocks/sec (fwd, fused bwd+Adam) and % of B200 HBM roofl
 UNIT = "blocks/s"
 # algorithmic HBM bytes per block: fwd reads W + logits, writes X; bwd+Adam reads W, G,
 # logits, m, v and writes logits, m, v; pack reads W + logits, writes values + metadata
-BYTES = {6: {"fwd": 40, "bwd": 160, "pack": 36.5, "init": 80},
-         70: {"fwd": 312, "bwd": 1712, "pack": 306, "init": 856}}
+# the fused kernel reads W, G, logits, m, v and writes logits, m, v and the next step's X
+BYTES = {6: {"fwd": 40, "bwd": 160, "fused": 168, "pack": 36.5, "init": 80},
+         70: {"fwd": 312, "bwd": 1712, "fused": 1728, "pack": 306, "init": 856}}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -127,32 +134,45 @@ def gpu_arm(args, w):
     dev = torch.device("cuda", local)
     pkg.lib()
     hbm_peak, peak_kind = peaks()
+    fused = args.loop == "fused"
 
     from sparsity_mask_sampling_b200.stack import SamplerStack
 
     t0 = time.time()
-    stack = SamplerStack(w, dev, rank)
+    stack = SamplerStack(w, dev, rank, x_per_layer=fused)
     stack.prior_init(seed=0)
     torch.cuda.synchronize()
     log(f"[rank {rank}] stack ready: {stack.blocks:,} blocks, {torch.cuda.memory_allocated(dev)/1e9:.1f} GB, {time.time()-t0:.1f}s")
 
-    # once-per-run rows: prior init and pack, timed on the device
+    # once-per-run rows: prior init (pack after the timed steps), timed on the device
     init_ms = time_once(lambda: stack.prior_init(seed=0))
+
     def reduce_all():
         if world > 1:
             dist.all_reduce(stack.reg, op=dist.ReduceOp.SUM)
 
-    # warm-up
+    L = w.layers
+
+    def step(t, ev=None, **kw):
+        if fused:
+            stack.step_fused(t, ev=ev, **kw)
+        else:
+            stack.step(t, ev=ev, **kw)
+
+    # prologue (the first forward of a fused loop) and warm-up steps
+    if fused:
+        stack.forward_all(0)
     for t in range(args.warmup):
-        stack.step(t)
+        step(t)
         reduce_all()
     torch.cuda.synchronize()
 
-    # device-timed steps
-    L = w.layers
-    evs = [{k: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
-            for k in ("fwd", "bwd")} for _ in range(args.steps)]
-    durs = {"fwd": [], "bwd": []}
+    # device-timed steps: every block gets one forward and one backward + AdamW per step
+    if fused:
+        evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)] for _ in range(args.steps)]
+    else:
+        evs = [{k: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
+                for k in ("fwd", "bwd")} for _ in range(args.steps)]
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
@@ -163,17 +183,20 @@ def gpu_arm(args, w):
     end = torch.cuda.Event(enable_timing=True)
     start.record()
     for k in range(args.steps):
-        stack.step(args.warmup + k, ev=evs[k])
+        step(args.warmup + k, ev=evs[k])
         reduce_all()
     end.record()
     torch.cuda.synchronize()
     elapsed_ms = start.elapsed_time(end)
-    for ev in evs:
-        for name in ("fwd", "bwd"):
-            durs[name].extend(ev[name][l][0].elapsed_time(ev[name][l][1]) for l in range(L))
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
+    durs = {}
+    if fused:
+        durs["fused"] = [ev[l][0].elapsed_time(ev[l][1]) for ev in evs for l in range(L)]
+    else:
+        for name in ("fwd", "bwd"):
+            durs[name] = [ev[name][l][0].elapsed_time(ev[name][l][1]) for ev in evs for l in range(L)]
     t_max = elapsed_ms
     if world > 1:
         tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
@@ -182,42 +205,54 @@ def gpu_arm(args, w):
     ms_per_step = t_max / args.steps
     value = stack.blocks * world * args.steps / (t_max / 1e3)
 
+    # the two unfused kernels, one pass over every layer each (reference timings)
+    ref = standalone_timings(stack, L, 5000)
+
     # pack (once, after training)
     pack_ms = time_pack(stack)
 
     # end-to-end: upstream gradients from pinned host memory, regulariser read back
-    e2e = e2e_leg(args, stack, w, world, dist if world > 1 else None, dev)
+    e2e = e2e_leg(args, stack, w, world, dist if world > 1 else None, dev, step, fused)
 
     blocks_per_layer = w.blocks_per_layer()
     fb = BYTES[w.C]
-    kern = {}
-    for name in ("fwd", "bwd"):
-        d = np.array(durs[name])
-        avg_ms = float(d.mean())
-        achieved = blocks_per_layer * fb[name] / (avg_ms / 1e3) / 1e9
-        kern[name] = {"avg_launch_ms": avg_ms, "blocks_per_launch": blocks_per_layer,
-                      "bytes_per_block": fb[name], "achieved_gbs": achieved, "frac": achieved / hbm_peak}
-    traffic = traffic_from_profile("bwd", w)
-    roofline = {"bound": "hbm", "kernel": "bwd_adam (fused backward + AdamW)",
-                "achieved": round(kern["bwd"]["achieved_gbs"], 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(kern["bwd"]["achieved_gbs"] / hbm_peak, 4), "peak_kind": peak_kind,
-                "traffic": traffic}
+
+    def kstats(ms_list, bpb, name):
+        avg = float(np.mean(ms_list))
+        gbs = blocks_per_layer * bpb / (avg / 1e3) / 1e9
+        return {"kernel": name, "avg_launch_ms": round(avg, 4), "launches": len(ms_list),
+                "blocks_per_launch": blocks_per_layer, "bytes_per_block": bpb,
+                "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)}
+
+    kernels = {}
+    if fused:
+        kernels["bwd_adam_fwd"] = kstats(durs["fused"], fb["fused"],
+                                         "bwd_adam_fwd_kernel: backward + AdamW of step t, forward of step t+1")
+        dom = kernels["bwd_adam_fwd"]
+        traffic = traffic_from_profile("bwd_adam_fwd", w)
+    else:
+        kernels["fwd"] = kstats(durs["fwd"], fb["fwd"], "fwd_kernel")
+        kernels["bwd_adam"] = kstats(durs["bwd"], fb["bwd"], "bwd_adam_kernel")
+        dom = kernels["bwd_adam"]
+        traffic = traffic_from_profile("bwd", w)
+    kernels["fwd_standalone"] = kstats(ref["fwd"], fb["fwd"], "fwd_kernel (first step of a loop)")
+    kernels["bwd_adam_standalone"] = kstats(ref["bwd"], fb["bwd"], "bwd_adam_kernel (unfused)")
+    kernels["pack_once"] = once_stats(pack_ms, stack.blocks, fb["pack"], hbm_peak)
+    kernels["prior_init_once"] = once_stats(init_ms, stack.blocks, fb["init"], hbm_peak)
+    roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved_gbs"], "peak": hbm_peak,
+                "unit": "GB/s", "frac": round(dom["achieved_gbs"] / hbm_peak, 4), "peak_kind": peak_kind,
+                "bytes_per_block": dom["bytes_per_block"], "traffic": traffic}
     out = None
     if rank == 0:
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": config_of(w, world),
+            "config": config_of(w, world, args.loop),
             "roofline": roofline,
-            "kernels": {
-                "fwd": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in kern["fwd"].items()},
-                "bwd_adam": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in kern["bwd"].items()},
-                "pack_once": once_stats(pack_ms, stack.blocks, fb["pack"], hbm_peak),
-                "prior_init_once": once_stats(init_ms, stack.blocks, fb["init"], hbm_peak),
-            },
+            "kernels": kernels,
             "e2e": e2e,
-            "gpu_launches": 2 * L * args.steps * n_groups(w),
+            "gpu_launches": (1 if fused else 2) * L * args.steps * n_groups(w),
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -225,6 +260,24 @@ def gpu_arm(args, w):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return out
+
+
+def standalone_timings(stack, L, t):
+    """Per-launch device time of the unfused forward and backward + AdamW, each run once
+    over every layer (outside the timed steps)."""
+    import torch
+
+    hp = stack.hparams(t).to_c()
+    out = {"fwd": [], "bwd": []}
+    for name, fn in (("fwd", stack.forward), ("bwd", stack.backward)):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+        for l in range(L):
+            evs[l][0].record()
+            fn(l, hp)
+            evs[l][1].record()
+        torch.cuda.synchronize()
+        out[name] = [a.elapsed_time(b) for a, b in evs]
     return out
 
 
@@ -275,7 +328,7 @@ def once_stats(ms, blocks, bpb, peak):
             "frac": round(gbs / peak, 4)}
 
 
-def e2e_leg(args, stack, w, world, dist, dev):
+def e2e_leg(args, stack, w, world, dist, dev, step, fused):
     """Same steps through the public API with the step inputs on the host: each layer's
     upstream gradients are copied from pinned host memory (a copy stream, overlapped with
     the kernels), and the regulariser sums are read back to the host every step."""
@@ -305,16 +358,18 @@ def e2e_leg(args, stack, w, world, dist, dev):
         main.wait_event(ready)
 
     steps = max(2, min(args.steps, 5))
-    for t in range(1):
-        stack.step(1000 + t, g_free=g_free, copy_fn=copy_fn)
-        reg_host.copy_(stack.reg, non_blocking=True)
+    t0 = 2000
+    if fused:
+        stack.forward_all(t0 - 1)
+    step(t0 - 1, g_free=g_free, copy_fn=copy_fn)
+    reg_host.copy_(stack.reg, non_blocking=True)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for t in range(steps):
-        stack.step(2000 + t, g_free=g_free, copy_fn=copy_fn)
+        step(t0 + t, g_free=g_free, copy_fn=copy_fn)
         if dist is not None:
             dist.all_reduce(stack.reg, op=dist.ReduceOp.SUM)
         reg_host.copy_(stack.reg, non_blocking=True)
@@ -332,8 +387,11 @@ def e2e_leg(args, stack, w, world, dist, dev):
             "ms_per_step": ms / steps}
 
 
-def config_of(w, world):
-    return {"workload": w.name, "nm": f"{w.nm[0]}:{w.nm[1]}", "layers": w.layers,
+def config_of(w, world, loop="fused"):
+    return {"workload": w.name, "loop": {"fused": "fused: per layer one launch of step t's backward + AdamW "
+                                                  "with step t+1's forward (the first forward in the prologue)",
+                                         "separate": "separate: per layer a forward launch, then a backward + "
+                                                     "AdamW launch"}[loop], "nm": f"{w.nm[0]}:{w.nm[1]}", "layers": w.layers,
             "matrices_per_layer": len(w.matrices),
             "shapes_out_in": [[m.rows, m.cols] for m in w.matrices],
             "blocks_per_step_per_gpu": w.total_blocks(), "candidates": w.C,
@@ -438,7 +496,7 @@ def reference_arm(args, w):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w, 1), "impl": "reference",
+        "data": "synthetic", "config": config_of(w, 1, args.loop), "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{n:,} blocks per step drawn from {w.name}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -452,6 +510,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama2_7b_stack_2of4")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--loop", default="fused", choices=["fused", "separate"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)

@@ -174,6 +174,23 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
 mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
                                  const mllm_hparams *hp, void *stream);
 
+/* Backward + AdamW of step t fused with the forward of step t+1 (an addition of this
+ * library, not on the pages). A training step runs the forward of every layer, then the
+ * backward in reverse; the next step's forward of a layer needs exactly the logits this
+ * step's backward just wrote. This call does, for every block, mllm_sample_bwd_adam with
+ * `hp` followed by mllm_sample_fwd with `hp_next` on the updated logits, reading W and the
+ * logits once: logits, adam_m, adam_v get step t's update, X_out receives step t+1's
+ * soft-masked weights, grad_logits_out (optional) step t's gradient, soft_mask_out
+ * (optional) step t+1's soft mask, and reg_sum_out (optional, with the workspace as in
+ * mllm_sample_fwd) step t+1's regulariser. A loop then calls mllm_sample_fwd once for the
+ * first step and this call for every step after it. Results are identical to the two calls
+ * in sequence. 4:8 runs them as two launches; 2:4 is one fused launch.
+ * Reads W, G. hp is validated as for mllm_sample_bwd_adam, hp_next as for mllm_sample_fwd. */
+mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                     const mllm_hparams *hp, const mllm_hparams *hp_next,
+                                     double *reg_sum_out, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
 /* Hard-mask extraction and compressed export (s.3.2 "Information flow at inference";
  * Algorithm 1 step 3). Per block: k = first index of the largest logit (NaN never wins;
  * all-NaN gives 0), kept positions p_0 < ... < p_{N-1} of S_k;

@@ -87,6 +87,7 @@ _SIGS = {
     "mllm_sample_fwd": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P, ctypes.c_size_t, _P]),
     "mllm_sample_bwd_adam": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P]),
     "mllm_sample_fwd_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P]),
+    "mllm_sample_bwd_adam_fwd": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "mllm_hard_pack": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P]),
     "mllm_noise": (ctypes.c_int, [NM, ctypes.c_uint64, ctypes.c_uint32, _P, ctypes.c_int64, _P, _P]),
     "mllm_workspace_bytes": (ctypes.c_size_t, []),
@@ -263,6 +264,19 @@ def mllm_sample_bwd_adam(mats, nm, hp: Hparams, stream=None):
     h = hp.to_c() if isinstance(hp, Hparams) else hp
     _check(lib().mllm_sample_bwd_adam(a.ptr, a.n, _nm(nm), ctypes.byref(h), _stream(stream)),
            "mllm_sample_bwd_adam")
+
+
+def mllm_sample_bwd_adam_fwd(mats, nm, hp: Hparams, hp_next: Hparams,
+                             reg_sum_out: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward + AdamW with hp, then the next step's forward with hp_next, in one pass."""
+    a = _mats(mats)
+    h = hp.to_c() if isinstance(hp, Hparams) else hp
+    hn = hp_next.to_c() if isinstance(hp_next, Hparams) else hp_next
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mllm_sample_bwd_adam_fwd(a.ptr, a.n, _nm(nm), ctypes.byref(h), ctypes.byref(hn),
+                                          _ptr(reg_sum_out), _ptr(workspace), ws_bytes,
+                                          _stream(stream)), "mllm_sample_bwd_adam_fwd")
 
 
 def mllm_hard_pack(mats, nm, stream=None):

@@ -281,6 +281,96 @@ __global__ void __launch_bounds__(kThreads) bwd_adam_kernel(const __grid_constan
     }
 }
 
+// Backward + AdamW of step t fused with the forward of step t+1 (mllm_sample_bwd_adam_fwd):
+// per pair of blocks, the backward math of bwd_adam_kernel with step t's scalars (sb), then,
+// from the updated logits still in registers, the forward math of fwd_kernel with step t+1's
+// scalars (sf). W and the logits are read once for both; X of step t+1 is written.
+template <bool kW32, bool kG32>
+__global__ void __launch_bounds__(kThreads, 3) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
+                                                                const StepScalars sb, const StepScalars sf,
+                                                                double *partials, unsigned int *ticket,
+                                                                double *reg_out, int accumulate) {
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
+    load_tab(s_tab);
+    __syncthreads();
+    const NlogCtx L{s_tab};
+    float acc = 0.f;
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
+        if (b0 >= d.nblocks) continue;
+        const bool two = b0 + 1 < d.nblocks;
+        float w[8], gw[8], pi[12], mo[12], vo[12], x[8], msv[8];
+        load_vals<kW32>(d.W, b0, two, w);
+        load_vals<kG32>(d.G, b0, two, gw);
+        load12(d.pi, b0, two, pi);
+        load12(d.m, b0, two, mo);
+        load12(d.v, b0, two, vo);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint64_t gid = d.gid0 + b0 + h;
+            {   // backward + AdamW, step t
+                float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
+                noise6(sb.seed, gid, sb.step, sb.noise_on, L, g);
+                soft_index(pi + 6 * h, g, sb.kappa, sb.c2, e, r);
+                soft_mask(e, r, ms);
+                soft_mask_comp(e, r, mc);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float wj = w[4 * h + j];
+                    const float u = __fmaf_rn(-__fmul_rn(sb.two_lambda, __fmul_rn(wj, wj)), ms[j],
+                                              __fmul_rn(gw[4 * h + j], wj));
+                    P[j] = __fmul_rn(mc[j], u);
+                    Q[j] = __fmul_rn(ms[j], u);
+                }
+                float D[6];
+                D[0] = (P[0] + P[1]) - (Q[2] + Q[3]);
+                D[1] = (P[0] + P[2]) - (Q[1] + Q[3]);
+                D[2] = (P[0] + P[3]) - (Q[1] + Q[2]);
+                D[3] = (P[1] + P[3]) - (Q[0] + Q[2]);
+                D[4] = (P[1] + P[2]) - (Q[0] + Q[3]);
+                D[5] = (P[2] + P[3]) - (Q[0] + Q[1]);
+                const float cr = __fmul_rn(sb.kappa_over_tau, r);
+                float grad[6];
+#pragma unroll
+                for (int i = 0; i < C; ++i) {
+                    grad[i] = __fmul_rn(__fmul_rn(cr, e[i]), D[i]);
+                    adamw(pi[6 * h + i], mo[6 * h + i], vo[6 * h + i], grad[i], sb);
+                }
+                if (d.grad && (h == 0 || two)) {
+                    float2 *gp = reinterpret_cast<float2 *>(d.grad + (b0 + h) * C);
+                    gp[0] = make_float2(grad[0], grad[1]);
+                    gp[1] = make_float2(grad[2], grad[3]);
+                    gp[2] = make_float2(grad[4], grad[5]);
+                }
+            }
+            {   // forward, step t+1, from the updated logits
+                float g[6], e[6], r, ms[4];
+                noise6(sf.seed, gid, sf.step, sf.noise_on, L, g);
+                soft_index(pi + 6 * h, g, sf.kappa, sf.c2, e, r);
+                soft_mask(e, r, ms);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float xj = __fmul_rn(w[4 * h + j], ms[j]);
+                    x[4 * h + j] = xj;
+                    msv[4 * h + j] = ms[j];
+                    if (h == 0 || two) acc = __fmaf_rn(xj, xj, acc);
+                }
+            }
+        }
+        store12(d.pi, b0, two, pi);
+        store12(d.m, b0, two, mo);
+        store12(d.v, b0, two, vo);
+        store_vals<kW32>(d.X, b0, two, x);
+        if (d.soft) {
+            float4 *sp = reinterpret_cast<float4 *>(d.soft + b0 * 4);
+            sp[0] = make_float4(msv[0], msv[1], msv[2], msv[3]);
+            if (two) sp[1] = make_float4(msv[4], msv[5], msv[6], msv[7]);
+        }
+    }
+    if (reg_out) reduce_to_global(acc, partials, ticket, reg_out, accumulate);
+}
+
 // Prior candidate of one block: the two positions of largest |w| (ties: lower position;
 // NaN ranks last) as a 4-bit keep mask.
 __device__ __forceinline__ uint32_t top2_mask(const float *w) {

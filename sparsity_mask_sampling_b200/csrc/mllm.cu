@@ -448,6 +448,53 @@ mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_n
     return MLLM_OK;
 }
 
+mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                     const mllm_hparams *hp, const mllm_hparams *hp_next,
+                                     double *reg_sum_out, void *workspace, size_t workspace_bytes,
+                                     void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedX | kNeedG | kNeedPi | kNeedMV);
+    if (s != MLLM_OK) return s;
+    if ((s = validate_bwd_hp(hp)) != MLLM_OK) return s;
+    if ((s = validate_fwd_hp(hp_next)) != MLLM_OK) return s;
+    if (reg_sum_out) {
+        if ((reinterpret_cast<uintptr_t>(reg_sum_out) & 7u) != 0) return MLLM_ERR_MISALIGNED;
+        if (!workspace || workspace_bytes < kWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    }
+    if (nm.m != 4) {  // 4:8: the two kernels in sequence
+        if ((s = mllm_sample_bwd_adam(mats, n_mats, nm, hp, stream)) != MLLM_OK) return s;
+        return mllm_sample_fwd(mats, n_mats, nm, hp_next, reg_sum_out, workspace, workspace_bytes, stream);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StepScalars sb = make_scalars(*hp), sf = make_scalars(*hp_next);
+    const bool w32 = mats[0].w_dtype == MLLM_F32, g32 = mats[0].g_dtype == MLLM_F32;
+    unsigned int *ticket = reg_sum_out ? static_cast<unsigned int *>(workspace) : nullptr;
+    double *partials = reg_sum_out ? reinterpret_cast<double *>(static_cast<char *>(workspace) + kWsPartialsOffset) : nullptr;
+    bool wrote_reg = false;
+    for (const Group &g : make_groups(mats, n_mats, nm.m, Kind::Sample24)) {
+        if (g.total_work == 0) continue;
+        const int accumulate = wrote_reg ? 1 : 0;
+#define MLLM_LAUNCH_FUSED(W32, G32)                                                                    \
+    do {                                                                                                 \
+        const void *fn = (const void *)k24::bwd_adam_fwd_kernel<W32, G32>;                               \
+        const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, kMaxReduceCtas);                     \
+        k24::bwd_adam_fwd_kernel<W32, G32><<<(unsigned)grid, kThreads, 0, st>>>(g, sb, sf, partials, ticket, \
+                                                                              reg_sum_out, accumulate);  \
+    } while (0)
+        if (w32 && g32) MLLM_LAUNCH_FUSED(true, true);
+        else if (w32) MLLM_LAUNCH_FUSED(true, false);
+        else if (g32) MLLM_LAUNCH_FUSED(false, true);
+        else MLLM_LAUNCH_FUSED(false, false);
+#undef MLLM_LAUNCH_FUSED
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+        wrote_reg = true;
+    }
+    if (reg_sum_out && !wrote_reg) {
+        if ((s = cuda_status(cudaMemsetAsync(reg_sum_out, 0, sizeof(double), st))) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
 mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, void *stream) {
     mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedPi | kNeedPack);
     if (s != MLLM_OK) return s;

@@ -5,6 +5,10 @@ AdamW moments) and streams the per-step tensors (soft-masked weights X out, upst
 gradients G in) through a pool of two layers' worth of buffers, as a training loop would
 hand them to and from the frozen network. One training step = the forward of every layer
 (one grouped launch each) then the fused backward + AdamW in reverse layer order.
+
+With x_per_layer=True every matrix keeps its own X, as a loop that runs the fused call
+(step t's backward + AdamW and step t+1's forward in one launch per layer) needs: layer l's
+next-step X is produced during this step's backward and read at the next step's forward.
 """
 from __future__ import annotations
 
@@ -20,8 +24,10 @@ _DT = {"bf16": torch.bfloat16, "f32": torch.float32}
 
 
 class SamplerStack:
-    def __init__(self, w: Workload, device, rank: int = 0, seed_base: int = 0, rng_seed: int = 0):
+    def __init__(self, w: Workload, device, rank: int = 0, seed_base: int = 0, rng_seed: int = 0,
+                 x_per_layer: bool = False):
         self.w = w
+        self.x_per_layer = x_per_layer
         self.dev = torch.device(device)
         self.nm = w.nm
         self.C = w.C
@@ -37,6 +43,7 @@ class SamplerStack:
                               for i, m in enumerate(w.matrices)])
         self.bufs: List[List[M.MatrixBuffers]] = []
         self._views = []
+        self.own_x = []
         for l in range(w.layers):
             mats = []
             for i, m in enumerate(w.matrices):
@@ -50,6 +57,8 @@ class SamplerStack:
                     adam_v=torch.zeros(B, w.C, dtype=torch.float32, device=self.dev)))
             self.bufs.append(mats)
             self._views.append(None)
+            if x_per_layer:
+                self.own_x.append([torch.empty(m.rows, m.cols, dtype=wdt, device=self.dev) for m in w.matrices])
         self.ws = torch.zeros(M.mllm_workspace_bytes(), dtype=torch.uint8, device=self.dev)
         self.reg = torch.zeros(w.layers, dtype=torch.float64, device=self.dev)
         self.blocks = w.total_blocks()
@@ -59,16 +68,18 @@ class SamplerStack:
         """(Re)build the C matrix arrays; call after replacing any buffer of self.bufs."""
         self._views = []
         for l, mats in enumerate(self.bufs):
-            for mb, (X, G) in zip(mats, self.pool[l % 2]):
-                mb.X, mb.G = X, G
+            for i, (mb, (X, G)) in enumerate(zip(mats, self.pool[l % 2])):
+                mb.X = self.own_x[l][i] if self.x_per_layer else X
+                mb.G = G
             self._views.append(M.MatrixArray(mats))
 
     def view(self, l: int) -> M.MatrixArray:
         return self._views[l]
 
     def XG(self, l: int, i: int):
-        """The pooled (X, G) buffers layer l's matrix i uses."""
-        return self.pool[l % 2][i]
+        """The (X, G) buffers layer l's matrix i uses."""
+        X, G = self.pool[l % 2][i]
+        return (self.own_x[l][i] if self.x_per_layer else X), G
 
     def prior_init(self, seed: int = 0, alpha: Optional[float] = None, init_std: Optional[float] = None):
         a = self.w.alpha if alpha is None else alpha
@@ -87,6 +98,30 @@ class SamplerStack:
 
     def backward(self, l: int, hp):
         M.mllm_sample_bwd_adam(self.view(l), self.nm, hp)
+
+    def backward_forward(self, l: int, hp, hp_next):
+        M.mllm_sample_bwd_adam_fwd(self.view(l), self.nm, hp, hp_next, self.reg[l:l + 1], self.ws)
+
+    def forward_all(self, t: int):
+        """The forward of every layer for step t (the first step of a fused loop)."""
+        hp = self.hparams(t).to_c()
+        for l in range(self.w.layers):
+            self.forward(l, hp)
+
+    def step_fused(self, t: int, ev=None, copy_fn=None, g_free=None):
+        """Enqueue step t of a fused loop: per layer in reverse order, step t's backward +
+        AdamW and step t+1's forward in one launch (step t's forward ran before)."""
+        hp, hpn = self.hparams(t).to_c(), self.hparams(t + 1).to_c()
+        for l in reversed(range(self.w.layers)):
+            if copy_fn is not None:
+                copy_fn(l)
+            if ev is not None:
+                ev[l][0].record()
+            self.backward_forward(l, hp, hpn)
+            if ev is not None:
+                ev[l][1].record()
+            if g_free is not None:
+                g_free[l % 2].record()
 
     def step(self, t: int, ev=None, copy_fn=None, g_free=None):
         """Enqueue one training step on the current stream. ev: optional {"fwd", "bwd"} lists of

@@ -11,7 +11,7 @@ import torch
 import _tol
 from sparsity_mask_sampling_b200 import (Hparams, MatrixBuffers, alloc_matrix, inputs, mllm_hard_pack,
                                          mllm_noise, mllm_prior_init, mllm_sample_bwd_adam,
-                                         mllm_sample_fwd, mllm_workspace_bytes)
+                                         mllm_sample_bwd_adam_fwd, mllm_sample_fwd, mllm_workspace_bytes)
 
 pytestmark = pytest.mark.gpu
 
@@ -340,3 +340,39 @@ def test_pack_of_deterministic_prior_is_magnitude_mask(orc):
     top2 = np.sort(np.argsort(-np.abs(Wf), 1, kind="stable")[:, :2], 1)
     expect = np.take_along_axis(Wf, top2, 1).reshape(c.rows, -1)
     assert np.array_equal(c.mb.pack_values.float().cpu().numpy(), expect)
+
+
+# ------------------------------------------------------------------------------ fused step
+
+@pytest.mark.parametrize("nm,shapes", [((2, 4), SHAPES_24), ((4, 8), SHAPES_48)])
+@pytest.mark.parametrize("tau,kappa", [(4.0, 100.0), (0.05, 500.0)])
+def test_fused_backward_forward_is_the_sequence(orc, ws, nm, shapes, tau, kappa):
+    """mllm_sample_bwd_adam_fwd = mllm_sample_bwd_adam (step t) then mllm_sample_fwd (step
+    t+1): logits, moments, gradient, X, soft mask bit for bit, regulariser to rounding of
+    its summation order; and its backward part matches the oracle on identical inputs."""
+    cases, off = [], 0
+    for i, (r, c) in enumerate(shapes):
+        cases.append(Case(nm, r, c, seed=70 + i, offset=off))
+        off += cases[-1].B
+    hp = Hparams(kappa=kappa, tau=tau, lambda_=1e-5, lr=5e-4, adam_step=4, step=3, seed=0xACE)
+    hp_next = Hparams(kappa=kappa * 1.01, tau=tau * 0.99, step=4, seed=0xACE)
+    mats = [c.mb for c in cases]
+    mllm_sample_bwd_adam(mats, nm, hp)
+    reg_a = torch.zeros(1, dtype=torch.float64, device=DEV)
+    mllm_sample_fwd(mats, nm, hp_next, reg_a, ws)
+    torch.cuda.synchronize()
+    seq = [[t.clone() for t in (c.mb.logits, c.mb.adam_m, c.mb.adam_v, c.mb.grad_logits, c.mb.X, c.mb.soft_mask)]
+           for c in cases]
+    for c in cases:
+        c.reset()
+        c.mb.X.zero_()
+        c.mb.soft_mask.zero_()
+    reg_b = torch.zeros(1, dtype=torch.float64, device=DEV)
+    mllm_sample_bwd_adam_fwd(mats, nm, hp, hp_next, reg_b, ws)
+    torch.cuda.synchronize()
+    for c, ref in zip(cases, seq):
+        got = (c.mb.logits, c.mb.adam_m, c.mb.adam_v, c.mb.grad_logits, c.mb.X, c.mb.soft_mask)
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
+    assert abs(reg_a.item() - reg_b.item()) <= 1e-12 * abs(reg_a.item())
+    _check_bwd(orc, cases, hp)
