@@ -221,6 +221,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Square root to about one ulp in one instruction (keeps denormals; sqrt(0) = 0). The
+// AdamW denominator needs no correctly rounded root: its result is compared at 1e-4.
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float y;
+    asm("sqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float rcp_approx(float x) {
     float y;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -138,7 +138,7 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
     const float pd = __fmul_rn(p, s.decay);
     m = __fmaf_rn(s.beta1, m, __fmul_rn(s.one_minus_beta1, g));
     v = __fmaf_rn(s.beta2, v, __fmul_rn(s.one_minus_beta2, __fmul_rn(g, g)));
-    const float denom = __fmaf_rn(__fsqrt_rn(v), s.inv_sqrt_bc2, s.eps);
+    const float denom = __fmaf_rn(sqrt_approx(v), s.inv_sqrt_bc2, s.eps);
     p = __fmaf_rn(-s.step_size, __fdividef(m, denom), pd);
 }
 
