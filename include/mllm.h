@@ -127,6 +127,17 @@ int32_t mllm_num_candidates(mllm_nm nm);
 mllm_status mllm_prior_init(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, float alpha,
                             float init_std, uint64_t seed, void *stream);
 
+/* Mask-prior initialisation from a given prior mask (the transfer prior: s.3.4 "Mask
+ * Prior" takes M0 from any one-shot method or from a previous MaskLLM run; Table 5's
+ * domain-transfer masks start from the general mask). Exactly mllm_prior_init with M0 of
+ * block b = candidate prior_idx[i][b] of matrix i instead of the magnitude prior, where
+ * prior_idx is a host array of n_mats device pointers to uint8 [B] (for instance the
+ * cand_idx_out of an earlier mllm_hard_pack). An index >= C gives that block no prior
+ * (sim = 0: pi = pi0, or 0 in the deterministic mode). W is not read. */
+mllm_status mllm_prior_init_from_mask(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                      const uint8_t *const *prior_idx, float alpha,
+                                      float init_std, uint64_t seed, void *stream);
+
 /* Forward of the sampler (s.3.4 Eq.5-Eq.8, Algorithm 1 lines 1-5). Per block:
  *   w_i = fma(kappa, pi_i, g_i) in fp32 (one rounding); y = softmax(w / tau) (Eq.6);
  *   M_j = sum_i y_i S_ij (Eq.7); X_j = W_j * M_j rounded to nearest-even in w_dtype;
@@ -201,6 +212,30 @@ mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, ml
  *   cand_idx_out[b] = k when non-NULL.
  * Reads W, logits. */
 mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, void *stream);
+
+/* Mask difference (s.3.4 Fig. 5a between adjacent steps, Fig. 8 between methods):
+ * *count_out (device, uint64) = number of i < n with a[i] != b[i], for two device arrays of
+ * candidate indices (e.g. cand_idx_out of two mllm_hard_pack calls). Exact. */
+mllm_status mllm_mask_diff(const uint8_t *a, const uint8_t *b, int64_t n,
+                           unsigned long long *count_out, void *stream);
+
+/* Mask statistics over all blocks of the matrices (at most 16 per call), into out[0..3]
+ * (device doubles): out[0] = sum over blocks of max_i softmax(kappa pi)_i (mean maximum
+ * probability, Fig. 5b, is out[0]/B); out[1] = sum of |W| kept by the hard mask argmax pi;
+ * out[2] = sum of |W| kept by the magnitude mask (out[1]/out[2]: relative L1 norm of the
+ * kept weights, Fig. 6); out[3] = number of blocks whose hard mask is the magnitude mask.
+ * Needs the mllm_sample_fwd workspace; deterministic for a given device. Reads W, logits. */
+mllm_status mllm_mask_stats(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, float kappa,
+                            double *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Compact code of hard masks (the page stores learned 2:4 masks at 0.65 bits/param, the
+ * entropy log2(6)/4 of a candidate index): D candidate indices per uint32 word, word w =
+ * sum_{t<D} idx[wD + t] C^t (missing tail digits 0); 2:4: D = 12 (0.667 bits per weight),
+ * 4:8: base 70, D = 5 (0.8 bits per weight). words has ceil(n/D) entries. */
+mllm_status mllm_encode_candidates(mllm_nm nm, const uint8_t *idx, int64_t n, uint32_t *words,
+                                   void *stream);
+mllm_status mllm_decode_candidates(mllm_nm nm, const uint32_t *words, int64_t n, uint8_t *idx,
+                                   void *stream);
 
 /* The Gumbel noise itself, for inspection and statistical tests: g_out[i*C + c] = noise
  * of candidate c of the block with global id gids[i] at (seed, step). gids and g_out are

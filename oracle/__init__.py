@@ -64,9 +64,14 @@ _SIGS = {
     "orc_sample_bwd": (_I, [_I, _I, _I64, _P, _P, _P, _P, _F, _F, _F, _U64, _U32, _I, _I, _P, _P]),
     "orc_adamw": (None, [_I64, _P, _P, _P, _P, _D, _D, _D, _D, _D, _I64, _P, _P, _P]),
     "orc_prior_init": (_I, [_I, _I, _I64, _P, _P, _D, _D, _U64, _P, _P, _P]),
+    "orc_prior_init_from_index": (_I, [_I, _I, _I64, _P, _P, _D, _D, _U64, _P, _P]),
     "orc_argmax": (_I, [_I64, _I, _P, _P]),
     "orc_hard_pack": (_I, [_I, _I, _I64, _I64, _I, _P, _P, _P, _P, _P]),
     "orc_round_bf16": (None, [_I64, _P, _P]),
+    "orc_mask_diff": (_I64, [_I64, _P, _P]),
+    "orc_mask_stats": (_I, [_I, _I, _I64, _P, _P, _D, _P]),
+    "orc_encode_candidates": (_I, [_I, _I, _I64, _P, _P]),
+    "orc_decode_candidates": (_I, [_I, _I, _I64, _P, _P]),
 }
 
 
@@ -244,6 +249,22 @@ def prior_init(n, m, W, gids, alpha, init_std, seed):
     return pi, pidx, sim
 
 
+def prior_init_from_index(n, m, gids, prior_idx, alpha, init_std, seed):
+    """Eq.9-Eq.10 from a given prior candidate per block (index >= C: no prior).
+
+    Returns (pi [nb, C] float64, sim [nb, C])."""
+    C = num_candidates(n, m)
+    g_ids = _c(gids, np.uint64).ravel()
+    k = _c(prior_idx, np.int32).ravel()
+    nb = g_ids.size
+    pi = np.zeros((nb, C))
+    sim = np.zeros((nb, C))
+    rc = lib().orc_prior_init_from_index(n, m, nb, _ptr(g_ids), _ptr(k), float(alpha), float(init_std),
+                                         int(seed), _ptr(pi), _ptr(sim))
+    _check(rc, "prior_init_from_index")
+    return pi, sim
+
+
 def argmax(pi, C) -> np.ndarray:
     p = _c(pi, np.float32).reshape(-1, C)
     out = np.zeros(p.shape[0], np.int32)
@@ -285,3 +306,40 @@ def round_bf16(x) -> np.ndarray:
 def bf16_bits_to_float(bits) -> np.ndarray:
     """Exact value of bf16 bit patterns (a bit shift; no arithmetic of the method)."""
     return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------------------
+# Diagnostics and codec
+# ---------------------------------------------------------------------------------------
+
+def mask_diff(a, b) -> int:
+    """Number of blocks whose candidate index differs (Fig. 5a / Fig. 8 mask difference)."""
+    a = _c(a, np.uint8).ravel()
+    b = _c(b, np.uint8).ravel()
+    return int(lib().orc_mask_diff(a.size, _ptr(a), _ptr(b)))
+
+
+def mask_stats(n, m, W, pi, kappa):
+    """(sum of max softmax(kappa pi), L1 kept by argmax, L1 kept by magnitude, blocks where
+    the two masks agree); see orc_mask_stats."""
+    C = num_candidates(n, m)
+    W = _c(W, np.float64).reshape(-1, m)
+    pi = _c(pi, np.float32).reshape(-1, C)
+    out = np.zeros(4)
+    _check(lib().orc_mask_stats(n, m, W.shape[0], _ptr(W), _ptr(pi), float(kappa), _ptr(out)), "mask_stats")
+    return out
+
+
+def encode_candidates(n, m, idx) -> np.ndarray:
+    idx = _c(idx, np.uint8).ravel()
+    D = 12 if m == 4 else 5
+    out = np.zeros((idx.size + D - 1) // D, np.uint32)
+    _check(lib().orc_encode_candidates(n, m, idx.size, _ptr(idx), _ptr(out)), "encode")
+    return out
+
+
+def decode_candidates(n, m, words, nb) -> np.ndarray:
+    words = _c(words, np.uint32).ravel()
+    out = np.zeros(nb, np.uint8)
+    _check(lib().orc_decode_candidates(n, m, nb, _ptr(words), _ptr(out)), "decode")
+    return out

@@ -462,6 +462,49 @@ int orc_prior_init(int n, int m, int64_t nb, const double *W, const uint64_t *gi
     return ORC_OK;
 }
 
+/* Prior initialisation from a given prior mask per block (the transfer prior: s.3.4 "Mask
+ * Prior" takes M0 from any one-shot method or from a previous MaskLLM run, Table 5).
+ * M0 of block b = S_{prior_idx[b]}; an index >= C means the block has no prior: sim = 0, so
+ * pi = pi0 (or 0 in the deterministic mode). Otherwise exactly orc_prior_init with that M0. */
+int orc_prior_init_from_index(int n, int m, int64_t nb, const uint64_t *gid, const int32_t *prior_idx,
+                              double alpha, double init_std, uint64_t seed, double *pi_out,
+                              double *sim_out) {
+    int C = num_candidates(n, m);
+    if (!C) return ORC_ERR;
+    for (int64_t b = 0; b < nb; b++) {
+        double sim[70];
+        int32_t k = prior_idx[b];
+        if (k < 0 || k >= C) {
+            for (int i = 0; i < C; i++) sim[i] = 0.0;
+        } else {
+            const uint8_t *m0 = cand_row(n, m, k);
+            double ip[70], mean_ip = 0.0;
+            for (int i = 0; i < C; i++) {
+                const uint8_t *row = cand_row(n, m, i);
+                int sacc = 0;
+                for (int j = 0; j < m; j++) sacc += row[j] * m0[j];
+                ip[i] = (double)sacc;
+                mean_ip += ip[i];
+            }
+            mean_ip /= (double)C;
+            for (int i = 0; i < C; i++) sim[i] = ip[i] - mean_ip;
+        }
+        if (init_std == 0.0) {
+            for (int i = 0; i < C; i++) pi_out[b * C + i] = alpha * sim[i];
+        } else {
+            double nrm[70], pi0[70], mu = 0.0, var = 0.0;
+            init_normals(C, seed, gid[b], nrm);
+            for (int i = 0; i < C; i++) { pi0[i] = init_std * nrm[i]; mu += pi0[i]; }
+            mu /= (double)C;
+            for (int i = 0; i < C; i++) var += (pi0[i] - mu) * (pi0[i] - mu);
+            double sigma = sqrt(var / (double)C);
+            for (int i = 0; i < C; i++) pi_out[b * C + i] = pi0[i] + alpha * sigma * sim[i];
+        }
+        if (sim_out) for (int i = 0; i < C; i++) sim_out[b * C + i] = sim[i];
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------------------ */
 /* Hard mask and compressed export                                                       */
 /* ------------------------------------------------------------------------------------ */
@@ -519,6 +562,85 @@ int orc_hard_pack(int n, int m, int64_t rows, int64_t cols, int elem_bytes, cons
             }
             if (cand_idx) cand_idx[blk] = (uint8_t)k;
         }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Diagnostics of the learned masks (s.3.4 Figs. 5, 6, 8) and a candidate-index codec     */
+/* ------------------------------------------------------------------------------------ */
+
+/* Number of blocks whose hard mask (candidate index) differs between a and b: the mask
+ * difference between two masks (Fig. 8) or between adjacent steps (Fig. 5a). */
+int64_t orc_mask_diff(int64_t n, const uint8_t *a, const uint8_t *b) {
+    int64_t d = 0;
+    for (int64_t i = 0; i < n; i++) d += (a[i] != b[i]);
+    return d;
+}
+
+/* Mask statistics over nb blocks (W [nb, M] values, pi [nb, C]):
+ *   out[0] = sum over blocks of max_i p_i with p = softmax(kappa pi) (mean max probability,
+ *            Fig. 5b, is out[0] / nb);
+ *   out[1] = sum of |W_j| over the positions the hard mask (argmax pi) keeps;
+ *   out[2] = sum of |W_j| over the positions the magnitude mask (top-N |W|) keeps
+ *            (out[1] / out[2] is the relative L1 norm of the kept weights, Fig. 6);
+ *   out[3] = number of blocks whose hard mask equals the magnitude mask. */
+int orc_mask_stats(int n, int m, int64_t nb, const double *W, const float *pi, double kappa, double *out) {
+    int C = num_candidates(n, m);
+    if (!C) return ORC_ERR;
+    double s_maxp = 0.0, s_l1 = 0.0, s_l1_mag = 0.0, same = 0.0;
+    for (int64_t b = 0; b < nb; b++) {
+        const float *p = pi + b * C;
+        const double *w = W + b * m;
+        int k = argmax_first(p, C);
+        double mx = -INFINITY, sum = 0.0;
+        for (int i = 0; i < C; i++) if ((double)kappa * p[i] > mx) mx = (double)kappa * p[i];
+        for (int i = 0; i < C; i++) sum += exp((double)kappa * p[i] - mx);
+        s_maxp += 1.0 / sum;
+        uint8_t m0[8];
+        magnitude_prior(n, m, w, m0);
+        const uint8_t *row = cand_row(n, m, k);
+        int eq = 1;
+        for (int j = 0; j < m; j++) {
+            if (row[j]) s_l1 += fabs(w[j]);
+            if (m0[j]) s_l1_mag += fabs(w[j]);
+            if (row[j] != m0[j]) eq = 0;
+        }
+        same += eq;
+    }
+    out[0] = s_maxp; out[1] = s_l1; out[2] = s_l1_mag; out[3] = same;
+    return ORC_OK;
+}
+
+/* Candidate-index codec: D = 12 indices per uint32 for 2:4 (6^12 < 2^32, 0.667 bits per
+ * weight against log2(6)/4 = 0.646, the page's 0.65 bits/param) and D = 5 per uint32 for 4:8
+ * (70^5 < 2^32, 0.8 bits per weight). Word w = sum_{t<D} idx[wD + t] C^t (missing tail
+ * indices count as 0). */
+int orc_encode_candidates(int n, int m, int64_t nb, const uint8_t *idx, uint32_t *out) {
+    int C = num_candidates(n, m);
+    if (!C) return ORC_ERR;
+    int D = (m == 4) ? 12 : 5;
+    int64_t words = (nb + D - 1) / D;
+    for (int64_t wi = 0; wi < words; wi++) {
+        uint64_t v = 0, p = 1;
+        for (int t = 0; t < D; t++) {
+            int64_t i = wi * D + t;
+            if (i < nb) v += (uint64_t)idx[i] * p;
+            p *= (uint64_t)C;
+        }
+        out[wi] = (uint32_t)v;
+    }
+    return ORC_OK;
+}
+
+int orc_decode_candidates(int n, int m, int64_t nb, const uint32_t *in, uint8_t *idx) {
+    int C = num_candidates(n, m);
+    if (!C) return ORC_ERR;
+    int D = (m == 4) ? 12 : 5;
+    for (int64_t i = 0; i < nb; i++) {
+        uint64_t v = in[i / D];
+        for (int t = 0; t < (int)(i % D); t++) v /= (uint64_t)C;
+        idx[i] = (uint8_t)(v % (uint64_t)C);
+    }
     return ORC_OK;
 }
 

@@ -84,6 +84,7 @@ _P = ctypes.c_void_p
 _SIGS = {
     "mllm_num_candidates": (ctypes.c_int32, [NM]),
     "mllm_prior_init": (ctypes.c_int, [_P, ctypes.c_int32, NM, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, _P]),
+    "mllm_prior_init_from_mask": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, ctypes.c_float, ctypes.c_float, ctypes.c_uint64, _P]),
     "mllm_sample_fwd": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P, ctypes.c_size_t, _P]),
     "mllm_sample_bwd_adam": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P]),
     "mllm_sample_fwd_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P, _P, _P]),
@@ -91,6 +92,10 @@ _SIGS = {
     "mllm_hard_pack": (ctypes.c_int, [_P, ctypes.c_int32, NM, _P]),
     "mllm_noise": (ctypes.c_int, [NM, ctypes.c_uint64, ctypes.c_uint32, _P, ctypes.c_int64, _P, _P]),
     "mllm_workspace_bytes": (ctypes.c_size_t, []),
+    "mllm_mask_diff": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P]),
+    "mllm_mask_stats": (ctypes.c_int, [_P, ctypes.c_int32, NM, ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+    "mllm_encode_candidates": (ctypes.c_int, [NM, _P, ctypes.c_int64, _P, _P]),
+    "mllm_decode_candidates": (ctypes.c_int, [NM, _P, ctypes.c_int64, _P, _P]),
     "mllm_noise_table": (ctypes.c_int, [_P, _P]),
     "mllm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mllm_last_cuda_error": (ctypes.c_int32, []),
@@ -241,6 +246,15 @@ def mllm_prior_init(mats, nm, alpha: float, init_std: float, seed: int, stream=N
                                  _stream(stream)), "mllm_prior_init")
 
 
+def mllm_prior_init_from_mask(mats, nm, prior_idx, alpha: float, init_std: float, seed: int, stream=None):
+    """Prior init with M0 = candidate prior_idx[i][b] (uint8 device tensors, one per matrix)."""
+    a = _mats(mats)
+    ptrs = (ctypes.c_void_p * max(1, a.n))(*[_ptr(t) for t in prior_idx])
+    _check(lib().mllm_prior_init_from_mask(a.ptr, a.n, _nm(nm), ctypes.cast(ptrs, ctypes.c_void_p),
+                                           float(alpha), float(init_std), int(seed), _stream(stream)),
+           "mllm_prior_init_from_mask")
+
+
 def mllm_sample_fwd(mats, nm, hp: Hparams, reg_sum_out: Optional[torch.Tensor] = None,
                     workspace: Optional[torch.Tensor] = None, stream=None):
     a = _mats(mats)
@@ -297,6 +311,28 @@ def mllm_noise_table():
     T = np.zeros((27, 128), np.float32)
     _check(lib().mllm_noise_table(c.ctypes.data, T.ctypes.data), "mllm_noise_table")
     return c, T
+
+
+def mllm_mask_diff(a: torch.Tensor, b: torch.Tensor, count_out: torch.Tensor, stream=None):
+    _check(lib().mllm_mask_diff(_ptr(a), _ptr(b), int(a.numel()), _ptr(count_out), _stream(stream)),
+           "mllm_mask_diff")
+
+
+def mllm_mask_stats(mats, nm, kappa: float, out: torch.Tensor, workspace: torch.Tensor, stream=None):
+    a = _mats(mats)
+    _check(lib().mllm_mask_stats(a.ptr, a.n, _nm(nm), float(kappa), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "mllm_mask_stats")
+
+
+def mllm_encode_candidates(nm, idx: torch.Tensor, words: torch.Tensor, stream=None):
+    _check(lib().mllm_encode_candidates(_nm(nm), _ptr(idx), int(idx.numel()), _ptr(words), _stream(stream)),
+           "mllm_encode_candidates")
+
+
+def mllm_decode_candidates(nm, words: torch.Tensor, n: int, idx: torch.Tensor, stream=None):
+    _check(lib().mllm_decode_candidates(_nm(nm), _ptr(words), int(n), _ptr(idx), _stream(stream)),
+           "mllm_decode_candidates")
 
 
 def mllm_last_cuda_error() -> int:

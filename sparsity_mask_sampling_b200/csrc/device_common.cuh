@@ -85,6 +85,7 @@ struct MatDesc {
     float *soft, *grad;
     void *pvals, *pmeta;
     uint8_t *cidx;
+    const uint8_t *prior;  // prior candidate index per block (prior init from a given mask)
     int64_t rows, cols, nblocks;
     uint64_t gid0;
     int64_t work_begin, work_count;

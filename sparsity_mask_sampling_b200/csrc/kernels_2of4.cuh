@@ -394,7 +394,9 @@ __device__ __forceinline__ uint32_t cand_mask(int i) {
     return (0xC6A953u >> (4 * i)) & 0xFu;  // 0x3, 0x5, 0x9, 0xA, 0x6, 0xC
 }
 
-template <bool kW32>
+// Prior initialisation. kFromIdx = false: M0 is the magnitude prior of the block's weights;
+// kFromIdx = true: M0 is candidate d.prior[b] (an index >= C: no prior, sim = 0).
+template <bool kW32, bool kFromIdx>
 __global__ void __launch_bounds__(kThreads) prior_kernel(const __grid_constant__ Group grp,
                                                          float alpha, float init_std, uint64_t seed) {
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
@@ -403,13 +405,20 @@ __global__ void __launch_bounds__(kThreads) prior_kernel(const __grid_constant__
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
         float w[8], pi[12], zero[12];
-        load_vals<kW32>(d.W, b0, two, w);
+        if (!kFromIdx) load_vals<kW32>(d.W, b0, two, w);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint32_t m0 = top2_mask(w + 4 * h);
             float sim[6];
+            if (kFromIdx) {
+                const uint32_t k = (h == 0 || two) ? d.prior[b0 + h] : 255u;
+                const uint32_t m0 = cand_mask(k < C ? (int)k : 0);
 #pragma unroll
-            for (int i = 0; i < C; ++i) sim[i] = (float)__popc(m0 & cand_mask(i)) - 1.0f;  // N*N/M = 1
+                for (int i = 0; i < C; ++i) sim[i] = (k < C) ? (float)__popc(m0 & cand_mask(i)) - 1.0f : 0.0f;
+            } else {
+                const uint32_t m0 = top2_mask(w + 4 * h);
+#pragma unroll
+                for (int i = 0; i < C; ++i) sim[i] = (float)__popc(m0 & cand_mask(i)) - 1.0f;  // N*N/M = 1
+            }
             if (init_std == 0.f) {
 #pragma unroll
                 for (int i = 0; i < C; ++i) pi[6 * h + i] = alpha * sim[i];

@@ -37,6 +37,16 @@ __host__ __device__ constexpr uint32_t cand_mask(int i) {
     return 0u;
 }
 
+// The 70 keep masks as a device table, for lookups by a runtime index (the prior given as a
+// candidate index); built at compile time from cand_mask.
+struct Cand48Table {
+    uint8_t m[C];
+    constexpr Cand48Table() : m{} {
+        for (int i = 0; i < C; ++i) m[i] = (uint8_t)cand_mask(i);
+    }
+};
+__device__ const Cand48Table g_cand48{};
+
 // Compile-time loop: f(std::integral_constant<int, I>) for I in [B, E).
 template <int B, int E, class F>
 __device__ __forceinline__ void static_for(F &&f) {
@@ -339,7 +349,8 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
     }
 }
 
-template <bool kW32>
+// Prior initialisation; kFromIdx as for the 2:4 kernel (M0 = candidate d.prior[b], >= C: none).
+template <bool kW32, bool kFromIdx>
 __global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constant__ Group grp,
                                                             float alpha, float init_std, uint64_t seed) {
     __shared__ __align__(16) float s_pi[kTileFloats];
@@ -350,24 +361,31 @@ __global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constan
         __syncthreads();
         if ((int)threadIdx.x < nb) {
             const int64_t b = tb0 + threadIdx.x;
-            float wt[8], key[8];
-            load8<kW32>(d.W, b, wt);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) key[j] = (wt[j] != wt[j]) ? -1.0f : fabsf(wt[j]);
             uint32_t m0 = 0;
+            float shift = 2.0f;  // sim = |M0 & S_c| - N*N/M; no prior: every sim is 0
+            if (kFromIdx) {
+                const uint32_t k = d.prior[b];
+                if (k < (uint32_t)C) m0 = g_cand48.m[k];
+                else shift = 0.0f;
+            } else {
+                float wt[8], key[8];
+                load8<kW32>(d.W, b, wt);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                int rank = 0;
+                for (int j = 0; j < 8; ++j) key[j] = (wt[j] != wt[j]) ? -1.0f : fabsf(wt[j]);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    if (k != j && (key[k] > key[j] || (key[k] == key[j] && k < j))) ++rank;
-                if (rank < 4) m0 |= 1u << j;
+                for (int j = 0; j < 8; ++j) {
+                    int rank = 0;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        if (k != j && (key[k] > key[j] || (key[k] == key[j] && k < j))) ++rank;
+                    if (rank < 4) m0 |= 1u << j;
+                }
             }
             float *row = s_pi + threadIdx.x * C;
             if (init_std == 0.f) {
                 static_for<0, C>([&](auto I) {
                     constexpr int c = decltype(I)::value;
-                    row[c] = alpha * ((float)__popc(m0 & cand_mask(c)) - 2.0f);
+                    row[c] = alpha * ((float)__popc(m0 & cand_mask(c)) - shift);
                 });
             } else {
                 float mu = 0.f;
@@ -396,7 +414,7 @@ __global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constan
                 const float as = alpha * sqrtf(var * (1.0f / C));
                 static_for<0, C>([&](auto I) {
                     constexpr int c = decltype(I)::value;
-                    row[c] = fmaf(as, (float)__popc(m0 & cand_mask(c)) - 2.0f, row[c]);
+                    row[c] = fmaf(as, (float)__popc(m0 & cand_mask(c)) - shift, row[c]);
                 });
             }
         }

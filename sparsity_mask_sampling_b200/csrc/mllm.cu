@@ -10,6 +10,7 @@
 #include "device_common.cuh"
 #include "kernels_2of4.cuh"
 #include "kernels_4of8.cuh"
+#include "kernels_diag.cuh"
 
 namespace mllm {
 namespace {
@@ -229,6 +230,37 @@ std::vector<Group> make_groups(const mllm_matrix *mats, int32_t n_mats, int M, K
     return out;
 }
 
+// ------------------------------------------------------------------------ prior launcher
+
+template <bool kFromIdx>
+mllm_status launch_prior(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, const uint8_t *const *prior_idx,
+                         float alpha, float init_std, uint64_t seed, void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool w32 = mats[0].w_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
+    int32_t i0 = 0;
+    for (Group g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48)) {
+        if (kFromIdx)
+            for (int32_t i = 0; i < g.n; ++i) g.d[i].prior = prior_idx[i0 + i];
+        i0 += g.n;
+        if (g.total_work == 0) continue;
+        if (is24) {
+            const void *fn = w32 ? (const void *)k24::prior_kernel<true, kFromIdx> : (const void *)k24::prior_kernel<false, kFromIdx>;
+            const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k24::prior_kernel<true, kFromIdx><<<(unsigned)grid, kThreads, 0, st>>>(g, alpha, init_std, seed);
+            else k24::prior_kernel<false, kFromIdx><<<(unsigned)grid, kThreads, 0, st>>>(g, alpha, init_std, seed);
+        } else {
+            const void *fn = w32 ? (const void *)k48::prior_kernel<true, kFromIdx> : (const void *)k48::prior_kernel<false, kFromIdx>;
+            const int64_t grid = grid_for(fn, k48::kCtaThreads, 0, g.total_work, INT32_MAX);
+            if (w32) k48::prior_kernel<true, kFromIdx><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, alpha, init_std, seed);
+            else k48::prior_kernel<false, kFromIdx><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, alpha, init_std, seed);
+        }
+        mllm_status s = cuda_status(cudaGetLastError());
+        if (s != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
 // ------------------------------------------------------------------------ no-alloc scratch
 
 // Scratch of mllm_sample_fwd_noalloc: the ticket word at offset 0, per-CTA partial sums from
@@ -305,25 +337,21 @@ mllm_status mllm_prior_init(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
     mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedPi);
     if (s != MLLM_OK) return s;
     if (!finite(alpha) || alpha < 0.f || !finite(init_std) || init_std < 0.f) return MLLM_ERR_INVALID_ARG;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool w32 = mats[0].w_dtype == MLLM_F32;
-    const bool is24 = nm.m == 4;
-    for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48)) {
-        if (g.total_work == 0) continue;
-        if (is24) {
-            const void *fn = w32 ? (const void *)k24::prior_kernel<true> : (const void *)k24::prior_kernel<false>;
-            const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, INT32_MAX);
-            if (w32) k24::prior_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, alpha, init_std, seed);
-            else k24::prior_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, alpha, init_std, seed);
-        } else {
-            const void *fn = w32 ? (const void *)k48::prior_kernel<true> : (const void *)k48::prior_kernel<false>;
-            const int64_t grid = grid_for(fn, k48::kCtaThreads, 0, g.total_work, INT32_MAX);
-            if (w32) k48::prior_kernel<true><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, alpha, init_std, seed);
-            else k48::prior_kernel<false><<<(unsigned)grid, k48::kCtaThreads, 0, st>>>(g, alpha, init_std, seed);
-        }
-        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    return launch_prior<false>(mats, n_mats, nm, nullptr, alpha, init_std, seed, stream);
+}
+
+mllm_status mllm_prior_init_from_mask(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
+                                      const uint8_t *const *prior_idx, float alpha, float init_std,
+                                      uint64_t seed, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedPi);
+    if (s != MLLM_OK) return s;
+    if (!finite(alpha) || alpha < 0.f || !finite(init_std) || init_std < 0.f) return MLLM_ERR_INVALID_ARG;
+    if (!prior_idx) return MLLM_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_mats; ++i) {
+        const bool any = mats[i].rows > 0 && mats[i].cols > 0;
+        if ((s = check_ptr(prior_idx[i], any)) != MLLM_OK) return s;
     }
-    return MLLM_OK;
+    return launch_prior<true>(mats, n_mats, nm, prior_idx, alpha, init_std, seed, stream);
 }
 
 mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
@@ -531,6 +559,89 @@ mllm_status mllm_hard_pack(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, 
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
     }
     return MLLM_OK;
+}
+
+mllm_status mllm_mask_diff(const uint8_t *a, const uint8_t *b, int64_t n, unsigned long long *count_out,
+                           void *stream) {
+    if (n < 0) return MLLM_ERR_INVALID_ARG;
+    mllm_status s;
+    if ((s = check_ptr(count_out, true)) != MLLM_OK) return s;
+    if ((s = check_ptr(a, n > 0)) != MLLM_OK) return s;
+    if ((s = check_ptr(b, n > 0)) != MLLM_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = cuda_status(cudaMemsetAsync(count_out, 0, sizeof(unsigned long long), st))) != MLLM_OK) return s;
+    if (n == 0) return MLLM_OK;
+    const int64_t grid = grid_for((const void *)diag::mask_diff_kernel, kThreads, 0,
+                                  (n / 16 + kThreads - 1) / kThreads + 1, INT32_MAX);
+    diag::mask_diff_kernel<<<(unsigned)grid, kThreads, 0, st>>>(a, b, n, count_out);
+    return cuda_status(cudaGetLastError());
+}
+
+mllm_status mllm_mask_stats(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, float kappa, double *out,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+    mllm_status s = validate_mats(mats, n_mats, nm, kNeedW | kNeedPi);
+    if (s != MLLM_OK) return s;
+    if (!finite(kappa) || !(kappa > 0.f)) return MLLM_ERR_INVALID_ARG;
+    if ((s = check_ptr(out, true)) != MLLM_OK) return s;
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    if (n_mats > kMaxMats) return MLLM_ERR_UNSUPPORTED;  // one launch: one deterministic sum
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool w32 = mats[0].w_dtype == MLLM_F32, is24 = nm.m == 4;
+    Group g = make_groups(mats, n_mats, nm.m, Kind::Sample24)[0];
+    if (!is24) {  // 4:8: one block per thread
+        int64_t acc = 0;
+        for (int32_t i = 0; i < g.n; ++i) {
+            g.d[i].work_begin = acc;
+            g.d[i].work_count = (g.d[i].nblocks + kThreads - 1) / kThreads;
+            acc += g.d[i].work_count;
+        }
+        g.total_work = acc;
+    }
+    if (g.total_work == 0) return cuda_status(cudaMemsetAsync(out, 0, 4 * sizeof(double), st));
+    unsigned int *ticket = static_cast<unsigned int *>(workspace);
+    double *partials = reinterpret_cast<double *>(static_cast<char *>(workspace) + kWsPartialsOffset);
+    const void *fn = is24 ? (w32 ? (const void *)diag::stats24_kernel<true> : (const void *)diag::stats24_kernel<false>)
+                          : (w32 ? (const void *)diag::stats48_kernel<true> : (const void *)diag::stats48_kernel<false>);
+    const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, diag::kMaxStatCtas);
+    if (is24) {
+        if (w32) diag::stats24_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, kappa, partials, ticket, out);
+        else diag::stats24_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, kappa, partials, ticket, out);
+    } else {
+        if (w32) diag::stats48_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, kappa, partials, ticket, out);
+        else diag::stats48_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, kappa, partials, ticket, out);
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+static mllm_status codec_args(mllm_nm nm, const void *src, const void *dst, int64_t n, int *C, int *D) {
+    *C = num_cand(nm);
+    if (!*C) return MLLM_ERR_UNSUPPORTED;
+    *D = (nm.m == 4) ? 12 : 5;
+    if (n < 0) return MLLM_ERR_INVALID_ARG;
+    mllm_status s;
+    if ((s = check_ptr(src, n > 0)) != MLLM_OK) return s;
+    return check_ptr(dst, n > 0);
+}
+
+mllm_status mllm_encode_candidates(mllm_nm nm, const uint8_t *idx, int64_t n, uint32_t *words, void *stream) {
+    int C, D;
+    mllm_status s = codec_args(nm, idx, words, n, &C, &D);
+    if (s != MLLM_OK || n == 0) return s;
+    const int64_t w = (n + D - 1) / D;
+    const int64_t grid = std::min<int64_t>((w + kThreads - 1) / kThreads, 65535 * 16);
+    diag::encode_kernel<<<(unsigned)grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(idx, n, C, D, words);
+    return cuda_status(cudaGetLastError());
+}
+
+mllm_status mllm_decode_candidates(mllm_nm nm, const uint32_t *words, int64_t n, uint8_t *idx, void *stream) {
+    int C, D;
+    mllm_status s = codec_args(nm, words, idx, n, &C, &D);
+    if (s != MLLM_OK || n == 0) return s;
+    const int64_t w = (n + D - 1) / D;
+    const int64_t grid = std::min<int64_t>((w + kThreads - 1) / kThreads, 65535 * 16);
+    diag::decode_kernel<<<(unsigned)grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(words, n, C, D, idx);
+    return cuda_status(cudaGetLastError());
 }
 
 mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t *gids,

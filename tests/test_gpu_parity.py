@@ -10,7 +10,8 @@ import torch
 
 import _tol
 from sparsity_mask_sampling_b200 import (Hparams, MatrixBuffers, alloc_matrix, inputs, mllm_hard_pack,
-                                         mllm_noise, mllm_prior_init, mllm_sample_bwd_adam,
+                                         mllm_noise, mllm_prior_init, mllm_prior_init_from_mask,
+                                         mllm_sample_bwd_adam,
                                          mllm_sample_bwd_adam_fwd, mllm_sample_fwd, mllm_workspace_bytes)
 
 pytestmark = pytest.mark.gpu
@@ -376,3 +377,42 @@ def test_fused_backward_forward_is_the_sequence(orc, ws, nm, shapes, tau, kappa)
             assert torch.equal(a, b)
     assert abs(reg_a.item() - reg_b.item()) <= 1e-12 * abs(reg_a.item())
     _check_bwd(orc, cases, hp)
+
+
+# ------------------------------------------------------------------------------ transfer prior
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+@pytest.mark.parametrize("init_std", [0.0, 0.01])
+def test_prior_from_mask_parity(orc, nm, init_std):
+    """Prior init from given candidate indices (some >= C: no prior) against the oracle:
+    bit-exact in the deterministic mode, 1e-6 of the block's scale with random logits."""
+    C = C_OF[nm]
+    cases = [Case(nm, 64, 128, seed=80, offset=5), Case(nm, 7, 40 if nm == (2, 4) else 48, seed=81, offset=10**6)]
+    rng = np.random.default_rng(3)
+    idx = []
+    for c in cases:
+        k = rng.integers(0, C + 3, size=c.B).astype(np.uint8)   # a few >= C
+        idx.append(torch.from_numpy(k).to(DEV))
+    mllm_prior_init_from_mask([c.mb for c in cases], nm, idx, 3.0, init_std, 99)
+    torch.cuda.synchronize()
+    for c, k in zip(cases, idx):
+        ref, _ = orc.prior_init_from_index(*nm, c.gids, k.cpu().numpy().astype(np.int32), 3.0, init_std, 99)
+        got = c.mb.logits.cpu().numpy().astype(np.float64)
+        if init_std == 0.0:
+            assert np.array_equal(got, ref.astype(np.float32).astype(np.float64))
+        else:
+            tol = 1e-6 * np.abs(ref).max(1, keepdims=True) + 1e-12
+            assert not (np.abs(got - ref) > tol).any()
+        assert not c.mb.adam_m.any() and not c.mb.adam_v.any()
+
+
+def test_transfer_prior_round_trip(orc):
+    """A general mask (hard-packed candidate indices of one run) seeds the prior of the next:
+    in the deterministic mode its argmax is the general mask in every block."""
+    c = Case((2, 4), 128, 256, seed=82)
+    mllm_hard_pack([c.mb], (2, 4))
+    general = c.mb.cand_idx.clone()
+    d = Case((2, 4), 128, 256, seed=83)
+    mllm_prior_init_from_mask([d.mb], (2, 4), [general], 3.0, 0.0, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.argmax(d.mb.logits, 1).to(torch.uint8), general)

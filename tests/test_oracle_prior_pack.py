@@ -183,3 +183,35 @@ def test_mask_storage_bits_per_param(orc):
     C = orc.num_candidates(2, 4)
     assert C == int(keyed("paper_figures.txt")["logits_per_block_2of4"][0])
     assert round(math.log2(C) / 4, 2) == page
+
+
+# ---------------------------------------------------------------- transfer prior (given M0)
+
+@pytest.mark.parametrize("n,m", NM)
+def test_prior_from_index_equals_magnitude_prior_when_given_it(orc, n, m):
+    """Giving the magnitude prior's own candidate index reproduces prior_init exactly, in both
+    the random and the deterministic mode."""
+    rng = np.random.default_rng(12)
+    W = rng.normal(0, 0.02, size=(300, m))
+    gids = np.arange(300, dtype=np.uint64) + np.uint64(7)
+    for init_std in (0.0, 0.01):
+        pi, pidx, sim = orc.prior_init(n, m, W, gids, 3.0, init_std, 5)
+        pi2, sim2 = orc.prior_init_from_index(n, m, gids, pidx, 3.0, init_std, 5)
+        np.testing.assert_array_equal(pi, pi2)
+        np.testing.assert_array_equal(sim, sim2)
+
+
+@pytest.mark.parametrize("n,m", NM)
+def test_prior_from_index_any_mask_and_no_prior(orc, n, m):
+    """Any candidate can be the prior (deterministic mode: argmax = that candidate, sim takes
+    the page's values); an index >= C leaves the random logits alone."""
+    C = orc.num_candidates(n, m)
+    rng = np.random.default_rng(13)
+    k = rng.integers(0, C, size=500)
+    pi, sim = orc.prior_init_from_index(n, m, np.arange(500), k, 3.0, 0.0, 0)
+    np.testing.assert_array_equal(np.argmax(pi, 1), k)
+    assert np.all(np.sort(np.unique(sim)) == (np.array([-1, 0, 1]) if m == 4 else np.array([-2, -1, 0, 1, 2])))
+    none = np.full(500, C, np.int32)
+    p0, _ = orc.prior_init_from_index(n, m, np.arange(500), none, 3.0, 0.01, 9)
+    r0, _, _ = orc.prior_init(n, m, np.zeros((500, m)), np.arange(500), 0.0, 0.01, 9)
+    np.testing.assert_array_equal(p0, r0)
