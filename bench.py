@@ -208,8 +208,9 @@ def gpu_arm(args, w):
     # the two unfused kernels, one pass over every layer each (reference timings)
     ref = standalone_timings(stack, L, 5000)
 
-    # pack (once, after training)
+    # pack (once, after training), then the mask diagnostics, codec and transfer prior
     pack_ms = time_pack(stack)
+    extras = time_extras(stack, hbm_peak)
 
     # end-to-end: upstream gradients from pinned host memory, regulariser read back
     e2e = e2e_leg(args, stack, w, world, dist if world > 1 else None, dev, step, fused)
@@ -251,6 +252,7 @@ def gpu_arm(args, w):
             "config": config_of(w, world, args.loop),
             "roofline": roofline,
             "kernels": kernels,
+            "extras": extras,
             "e2e": e2e,
             "gpu_launches": (1 if fused else 2) * L * args.steps * n_groups(w),
             "clocks": clocks,
@@ -320,6 +322,40 @@ def time_pack(stack):
         for a in arrs:
             pkg.mllm_hard_pack(a, w.nm)
     return time_once(go)
+
+
+def time_extras(stack, peak):
+    """Once-per-run calls around training, timed over the whole stack on the device: mask
+    statistics (Fig. 5b/6), mask difference between two hard masks (Fig. 5a/8), the
+    candidate-index code, and a prior initialisation from a given mask (transfer)."""
+    import torch
+    import sparsity_mask_sampling_b200 as pkg
+
+    w = stack.w
+    L = w.layers
+    dev = stack.dev
+    B = stack.blocks
+    out = {}
+    stats = torch.zeros(4, dtype=torch.float64, device=dev)
+    out["mask_stats_once"] = once_stats(
+        time_once(lambda: [pkg.mllm_mask_stats(stack.view(l), w.nm, w.kappa[1], stats, stack.ws) for l in range(L)]),
+        B, (16 if w.w_dtype == "f32" else 8) + 4 * w.C, peak)
+    idx = [mb.cand_idx for mb in stack.bufs[0]]   # hard masks of one layer, reused per layer
+    other = [torch.roll(t, 1) for t in idx]
+    cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+    out["mask_diff_once"] = once_stats(
+        time_once(lambda: [pkg.mllm_mask_diff(a, b, cnt) for _ in range(L) for a, b in zip(idx, other)]), B, 2, peak)
+    D = 12 if w.nm == (2, 4) else 5
+    words = [torch.empty((t.numel() + D - 1) // D, dtype=torch.int32, device=dev) for t in idx]
+    out["encode_once"] = once_stats(
+        time_once(lambda: [pkg.mllm_encode_candidates(w.nm, t, wd) for _ in range(L) for t, wd in zip(idx, words)]),
+        B, 1 + 4.0 / D, peak)
+    pri = [idx] * L
+    arrs = [stack.view(l) for l in range(L)]
+    out["prior_from_mask_once"] = once_stats(
+        time_once(lambda: [pkg.mllm_prior_init_from_mask(arrs[l], w.nm, pri[l], w.alpha, w.init_std, 0) for l in range(L)]),
+        B, 1 + 12 * w.C, peak)
+    return out
 
 
 def once_stats(ms, blocks, bpb, peak):

@@ -16,10 +16,12 @@ from typing import List, Tuple
 
 
 def linear_schedule(x0: float, x1: float, t: int, T: int) -> float:
-    """x_t = x0 + (x1 - x0) t / (T - 1), endpoints included (t = 0 .. T-1)."""
+    """x_t = x0 + (x1 - x0) t / (T - 1), endpoints included (t = 0 .. T-1); evaluated as
+    x0 (1 - f) + x1 f, f = t / (T - 1), so that both endpoints are exact."""
     if T <= 1:
         return x0
-    return x0 + (x1 - x0) * t / (T - 1)
+    f = t / (T - 1)
+    return x0 * (1.0 - f) + x1 * f
 
 
 @dataclass(frozen=True)
