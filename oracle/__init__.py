@@ -11,7 +11,9 @@ Large Language Models"), cited by section and equation.
 
 Parity status per function (see the pins in tests/test_oracle_*.py):
   candidates, philox4x32_10, nlog, noise, soft_mask, sample_fwd, sample_bwd, adamw,
-  prior_init (deterministic mode, similarity, magnitude prior), hard_pack, round_bf16: pinned.
+  prior_init (deterministic mode, similarity, magnitude prior), prior_init_from_index,
+  hard_pack, round_bf16, mask_diff, mask_stats, encode/decode_candidates, sparse_linear:
+  pinned.
   prior_init random mode: the N(0, 0.01) draws are pinned statistically (moments) and the
   Eq.10 structure exactly; the individual Box-Muller bits are parity-by-tolerance only.
 """
@@ -72,6 +74,7 @@ _SIGS = {
     "orc_mask_stats": (_I, [_I, _I, _I64, _P, _P, _D, _P]),
     "orc_encode_candidates": (_I, [_I, _I, _I64, _P, _P]),
     "orc_decode_candidates": (_I, [_I, _I, _I64, _P, _P]),
+    "orc_sparse_linear": (_I, [_I, _I, _I64, _I64, _P, _P, _I64, _P, _P]),
 }
 
 
@@ -343,3 +346,18 @@ def decode_candidates(n, m, words, nb) -> np.ndarray:
     out = np.zeros(nb, np.uint8)
     _check(lib().orc_decode_candidates(n, m, nb, _ptr(words), _ptr(out)), "decode")
     return out
+
+
+def sparse_linear(n, m, values, meta, x) -> np.ndarray:
+    """Product with a hard-masked weight in hard_pack's compressed form (s.3.2, inference):
+    values [rows, cols*N/M] uint16 (bf16 bits), meta as hard_pack returns it, x [tokens, cols]
+    uint16 (bf16 bits). Returns y [tokens, rows] float64, y = x W*^T."""
+    values = _c(values, np.uint16)
+    rows = values.shape[0]
+    x = _c(x, np.uint16)
+    tokens, cols = x.shape
+    meta = _c(meta, np.uint32 if m == 4 else np.uint16)
+    y = np.zeros((tokens, rows))
+    _check(lib().orc_sparse_linear(n, m, rows, cols, _ptr(values), _ptr(meta), tokens, _ptr(x), _ptr(y)),
+           "sparse_linear")
+    return y

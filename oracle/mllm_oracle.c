@@ -645,6 +645,51 @@ int orc_decode_candidates(int n, int m, int64_t nb, const uint32_t *in, uint8_t 
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Deployment: the product with the hard-masked weight (s.3.2 "Information flow at       */
+/* inference": the learned mask is applied once and the sparse network is served)        */
+/* ------------------------------------------------------------------------------------ */
+
+static double bf16_to_double(uint16_t h) {
+    uint32_t bits = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &bits, 4);
+    return (double)f;
+}
+
+/* y = x W*^T for a matrix W* = W (.) M* given in orc_hard_pack's compressed form (bf16
+ * values, 2:4 nibble or 4:8 uint16 metadata), and activations x [tokens, cols] in bf16:
+ *   y[t*rows + r] = sum over blocks q of row r, over kept slots i < N,
+ *                   values[r, qN + i] * x[t, qM + p_i],
+ * p_i the i-th kept position decoded from the metadata. Every term is an exact product of
+ * two bf16 numbers; the sum runs in double in the order written. */
+int orc_sparse_linear(int n, int m, int64_t rows, int64_t cols, const uint16_t *values, const void *meta,
+                      int64_t tokens, const uint16_t *x, double *y) {
+    if (!num_candidates(n, m) || cols % m || rows < 0 || tokens < 0) return ORC_ERR;
+    int64_t bpr = cols / m, words = (bpr + 7) / 8;
+    for (int64_t t = 0; t < tokens; t++)
+        for (int64_t r = 0; r < rows; r++) {
+            double acc = 0.0;
+            for (int64_t q = 0; q < bpr; q++) {
+                int pos[4];
+                if (m == 4) {
+                    uint32_t w = ((const uint32_t *)meta)[r * words + q / 8];
+                    uint32_t nib = (w >> (4 * (q % 8))) & 0xFu;
+                    pos[0] = (int)(nib & 3u);
+                    pos[1] = (int)(nib >> 2);
+                } else {
+                    uint32_t code = ((const uint16_t *)meta)[r * bpr + q];
+                    for (int i = 0; i < 4; i++) pos[i] = (int)((code >> (3 * i)) & 7u);
+                }
+                for (int i = 0; i < n; i++)
+                    acc += bf16_to_double(values[r * bpr * n + q * n + i]) *
+                           bf16_to_double(x[t * cols + q * m + pos[i]]);
+            }
+            y[t * rows + r] = acc;
+        }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Rounding of the soft-masked weights to their storage type                             */
 /* ------------------------------------------------------------------------------------ */
 
