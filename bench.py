@@ -12,6 +12,9 @@ measured copy bandwidth.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--loop fused|separate]
                   [--impl reference]
+  python bench.py --mode sparse_linear [--workload NAME] [--steps K --warmup W]
+      (serving leg: the workload's matrices as packed hard masks, y = x W*^T per call for
+       1, 8 and 16 tokens, against dense cuBLAS; one JSON line)
 
 Default workload: the full LLaMA-2-7B-shaped stack at 2:4 (32 layers x 7 matrices,
 1,619,001,344 blocks; logits and AdamW moments resident in HBM, ~130 GB, plus the next
@@ -211,6 +214,7 @@ def gpu_arm(args, w):
     # pack (once, after training), then the mask diagnostics, codec and transfer prior
     pack_ms = time_pack(stack)
     extras = time_extras(stack, hbm_peak)
+    extras["sparse_linear"] = time_sparse_linear(stack, hbm_peak)
 
     # end-to-end: upstream gradients from pinned host memory, regulariser read back
     e2e = e2e_leg(args, stack, w, world, dist if world > 1 else None, dev, step, fused)
@@ -358,6 +362,79 @@ def time_extras(stack, peak):
     return out
 
 
+def time_median(fn, reps=5):
+    import torch
+
+    fn()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        out.append(s.elapsed_time(e))
+    return float(np.median(out))
+
+
+def time_sparse_linear(stack, peak, token_counts=(1, 8, 16)):
+    """Serving the learned sparse network (s.3.2, inference): y = x W*^T for every matrix of
+    the stack from its own packed hard mask (one mllm_sparse_linear call for all of them: a
+    launch per 16 matrices), as
+    one decode step of T tokens through all linear layers, beside the same products with the
+    dense bf16 weights through cuBLAS (torch.nn.functional.linear). Bytes are those of the
+    compressed weights, metadata, activations and outputs; the packed stack (7.3 GB for
+    LLaMA-2-7B at 2:4) is larger than L2, so every pass streams it from HBM."""
+    import torch
+    import torch.nn.functional as F
+    import sparsity_mask_sampling_b200 as pkg
+    from sparsity_mask_sampling_b200 import buffers
+
+    w = stack.w
+    if w.w_dtype != "bf16":
+        return None
+    dev = stack.dev
+    L = w.layers
+    packed = []
+    for l in range(L):
+        outs = []
+        for mb, m in zip(stack.bufs[l], w.matrices):
+            (vs, (ms, mdt)) = buffers.pack_shapes(m.rows, m.cols, w.nm)
+            mb.pack_values = torch.empty(vs, dtype=torch.bfloat16, device=dev)
+            mb.pack_meta = torch.empty(ms, dtype=mdt, device=dev)
+            mb.cand_idx = None
+            outs.append((mb.pack_values, mb.pack_meta))
+        pkg.mllm_hard_pack(pkg.MatrixArray(stack.bufs[l]), w.nm)
+        packed.append(outs)
+    wbytes = sum(v.numel() * 2 + mt.numel() * mt.element_size() for outs in packed for v, mt in outs)
+    dense_bytes = sum(mb.W.numel() * 2 for mats in stack.bufs for mb in mats)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    spl_ws = pkg.sparse_linear_workspace(dev)
+    res = {"launches_per_pass": math.ceil(L * len(w.matrices) / 16), "compressed_weight_gb": round(wbytes / 1e9, 3)}
+    for T in token_counts:
+        xs = {c: torch.randn(T, c, device=dev, generator=gen).to(torch.bfloat16) for c in {m.cols for m in w.matrices}}
+        ys = [torch.empty(T, m.rows, dtype=torch.float32, device=dev) for m in w.matrices]
+        arr = pkg.SparseOperandArray([(v, mt, xs[m.cols], y) for l in range(L)
+                                      for (v, mt), m, y in zip(packed[l], w.matrices, ys)])
+        io = L * sum(T * m.cols * 2 + T * m.rows * 4 for m in w.matrices)
+        ms = time_median(lambda: pkg.mllm_sparse_linear(arr, w.nm, T, spl_ws))
+        ms_dense = time_median(lambda: [F.linear(xs[mb.W.shape[1]], mb.W) for mats in stack.bufs for mb in mats])
+        gbs = (wbytes + io) / (ms / 1e3) / 1e9
+        res[f"tokens_{T}"] = {
+            "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "dense_cublas_ms": round(ms_dense, 4),
+            "dense_cublas_gbs": round((dense_bytes + io) / (ms_dense / 1e3) / 1e9, 1),
+            "speedup_vs_dense": round(ms_dense / ms, 3)}
+    for mats in stack.bufs:
+        for mb in mats:
+            mb.pack_values = mb.pack_meta = None
+    del packed
+    torch.cuda.empty_cache()
+    return res
+
+
 def once_stats(ms, blocks, bpb, peak):
     gbs = blocks * bpb / (ms / 1e3) / 1e9
     return {"ms": round(ms, 3), "blocks_per_s": blocks / (ms / 1e3), "achieved_gbs": round(gbs, 1),
@@ -441,25 +518,26 @@ def config_of(w, world, loop="fused"):
 
 def traffic_from_profile(kernel, w):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
-    kernel source (its sha256 is recorded there); otherwise None."""
+    source of the kernel (its sha256 is recorded there); otherwise None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     ent = d.get(f"{kernel}_{w.nm[0]}of{w.nm[1]}")
-    if not ent or ent.get("source_sha256") != kernel_source_sha():
+    if not ent or ent.get("source_sha256") != kernel_source_sha(w.nm):
         return None
     return ent["dram_bytes_per_block"] * w.blocks_per_layer()
 
 
-def kernel_source_sha():
+def kernel_source_sha(nm=(2, 4)):
+    """sha256 of the files that hold the sampler kernels' device code for a pattern (the
+    shared device helpers and the pattern's kernel file)."""
     csrc = os.path.join(ROOT, "sparsity_mask_sampling_b200", "csrc")
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(f.read())
+    for fn in ("device_common.cuh", "kernels_2of4.cuh" if nm == (2, 4) else "kernels_4of8.cuh"):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 
@@ -539,8 +617,96 @@ def reference_arm(args, w):
     }
 
 
+def random_packed(rows, cols, nm, dev, gen):
+    """A packed hard-masked bf16 matrix with random values and a random valid candidate per
+    block, in mllm_hard_pack's format (for timing; the content does not change the cost)."""
+    import torch
+    from itertools import combinations
+
+    n, m = nm
+    bpr = cols // m
+    vals = torch.randn(rows, bpr * n, device=dev, generator=gen).to(torch.bfloat16)
+    combos = list(combinations(range(m), n))
+    k = torch.randint(0, len(combos), (rows, bpr), device=dev, generator=gen)
+    if m == 4:
+        nib = torch.tensor([p[0] | p[1] << 2 for p in combos], device=dev, dtype=torch.int64)[k]
+        words = (bpr + 7) // 8
+        pad = torch.zeros(rows, words * 8, device=dev, dtype=torch.int64)
+        pad[:, :bpr] = nib
+        shifts = 4 * torch.arange(8, device=dev, dtype=torch.int64)
+        w = (pad.view(rows, words, 8) << shifts).sum(-1)
+        meta = torch.where(w >= 2 ** 31, w - 2 ** 32, w).to(torch.int32)
+    else:
+        meta = torch.tensor([p[0] | p[1] << 3 | p[2] << 6 | p[3] << 9 for p in combos], device=dev,
+                            dtype=torch.int16)[k]
+    return vals, meta
+
+
+def sparse_linear_arm(args, w):
+    """--mode sparse_linear: serving the learned sparse network (s.3.2, inference). Every
+    matrix of the workload as a packed hard-masked bf16 weight; one pass = y = x W*^T for all
+    of them (one mllm_sparse_linear call, a launch per 16 matrices) for T tokens, timed per
+    call with CUDA events (median of --steps calls after --warmup), beside the same products
+    with dense bf16 weights through cuBLAS (torch.nn.functional.linear)."""
+    import torch
+    import torch.nn.functional as F
+    import sparsity_mask_sampling_b200 as pkg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    pkg.lib()
+    hbm_peak, peak_kind = peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    shapes = [(m.rows, m.cols) for _ in range(w.layers) for m in w.matrices]
+    packed = [random_packed(r, c, w.nm, dev, gen) for r, c in shapes]
+    dense = [torch.randn(r, c, device=dev, generator=gen).to(torch.bfloat16) for r, c in shapes]
+    wbytes = sum(v.numel() * 2 + mt.numel() * mt.element_size() for v, mt in packed)
+    dbytes = sum(d.numel() * 2 for d in dense)
+    ws = pkg.sparse_linear_workspace(dev)
+
+    def med(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(args.steps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            out.append(s.elapsed_time(e))
+        return float(np.median(out))
+
+    res = {}
+    for T in (1, 8, 16):
+        xs = {c: torch.randn(T, c, device=dev, generator=gen).to(torch.bfloat16) for c in {c for _, c in shapes}}
+        ys = [torch.empty(T, r, dtype=torch.float32, device=dev) for r, _ in shapes]
+        arr = pkg.SparseOperandArray([(v, mt, xs[c], y) for (v, mt), (r, c), y in zip(packed, shapes, ys)])
+        io = sum(T * c * 2 + T * r * 4 for r, c in shapes)
+        ms = med(lambda: pkg.mllm_sparse_linear(arr, w.nm, T, ws))
+        ms_d = med(lambda: [F.linear(xs[d.shape[1]], d) for d in dense])
+        gbs = (wbytes + io) / (ms / 1e3) / 1e9
+        res[f"tokens_{T}"] = {"ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
+                              "dense_cublas_ms": round(ms_d, 4),
+                              "dense_cublas_gbs": round((dbytes + io) / (ms_d / 1e3) / 1e9, 1),
+                              "speedup_vs_dense": round(ms_d / ms, 3)}
+    t8 = res["tokens_8"]
+    return {"metric": "sparse_linear_bandwidth", "value": t8["achieved_gbs"], "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t8["ms"], "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic (random packed masks and values)",
+            "config": {"workload": w.name, "matrices": len(shapes), "nm": f"{w.nm[0]}:{w.nm[1]}",
+                       "compressed_weight_gb": round(wbytes / 1e9, 3), "launches_per_call": math.ceil(len(shapes) / 16),
+                       "tokens_timed": 8},
+            "roofline": {"bound": "hbm", "achieved": t8["achieved_gbs"], "peak": hbm_peak, "unit": "GB/s",
+                         "frac": t8["frac"], "peak_kind": peak_kind},
+            "tokens": res}
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--mode", default="train", choices=["train", "sparse_linear"])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -557,7 +723,9 @@ def main():
     from sparsity_mask_sampling_b200 import configs
 
     w = configs.WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.mode == "sparse_linear":
+        out = sparse_linear_arm(args, w)
+    elif args.impl == "reference":
         out = reference_arm(args, w)
     else:
         out = gpu_arm(args, w)

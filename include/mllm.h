@@ -237,6 +237,36 @@ mllm_status mllm_encode_candidates(mllm_nm nm, const uint8_t *idx, int64_t n, ui
 mllm_status mllm_decode_candidates(mllm_nm nm, const uint32_t *words, int64_t n, uint8_t *idx,
                                    void *stream);
 
+/* One operand of mllm_sparse_linear: a hard-masked weight W* = W (.) M* [rows, cols] in the
+ * compressed form mllm_hard_pack writes for a bf16 matrix, and the activations it multiplies.
+ * All four pointers are caller-owned device memory, 16-byte aligned. */
+typedef struct {
+    const void *pack_values;  /* [rows, cols*N/M] bf16: pack_values of mllm_hard_pack        */
+    const void *pack_meta;    /* pack_meta of mllm_hard_pack (2:4 uint32 words, 4:8 uint16)  */
+    const void *x;            /* [tokens, cols] bf16 activations, row-major                  */
+    float *y;                 /* [tokens, rows] fp32 output, row-major (overwritten)          */
+    int64_t rows, cols;       /* of the dense matrix; cols % M == 0                           */
+} mllm_sparse_operand;
+
+/* Serving the learned sparse network (s.3.2 "Information flow at inference": the mask is
+ * applied once and the N:M-sparse weights are used from then on): for every operand,
+ *   y[t, r] = sum over blocks q of row r and kept slots i < N of
+ *             pack_values[r, qN + i] * x[t, qM + p_i],
+ * i.e. y = x W*^T, with bf16 products accumulated in fp32 (tensor cores), for 1 <= tokens
+ * <= 16 (decode-sized batches; the kernel is bound by reading the compressed weight).
+ * Operands may differ in shape and are processed in one launch per 16 of them; rows == 0
+ * operands are skipped and cols == 0 gives y = 0 (pointers other than y may then be NULL).
+ * workspace: device memory of mllm_sparse_linear_workspace_bytes() bytes, zero-filled by the
+ * caller before its first use; every call leaves it zero-filled again (partial tiles of rows
+ * whose columns are split between warps, and one completion counter per warp). Calls that
+ * may run concurrently need separate workspaces. Deterministic on a given device: the
+ * summation order depends only on the shapes and the launch size. Works for 2:4 and 4:8. */
+mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, mllm_nm nm, int32_t tokens,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes mllm_sparse_linear needs (independent of sizes). */
+size_t mllm_sparse_linear_workspace_bytes(void);
+
 /* The Gumbel noise itself, for inspection and statistical tests: g_out[i*C + c] = noise
  * of candidate c of the block with global id gids[i] at (seed, step). gids and g_out are
  * device arrays of n_blocks and n_blocks*C entries; step may be any value, including the
@@ -258,10 +288,11 @@ const char *mllm_status_string(mllm_status s);
 /* cudaError_t of the most recent MLLM_ERR_CUDA on the calling thread (0 if none). */
 int32_t mllm_last_cuda_error(void);
 
-/* ABI guards for bindings: MLLM_ABI_VERSION, sizeof(mllm_matrix), sizeof(mllm_hparams). */
+/* ABI guards for bindings: MLLM_ABI_VERSION and the sizes of the structs. */
 int32_t mllm_abi_version(void);
 size_t mllm_sizeof_matrix(void);
 size_t mllm_sizeof_hparams(void);
+size_t mllm_sizeof_sparse_operand(void);
 
 #ifdef __cplusplus
 }

@@ -80,6 +80,17 @@ class HParams(ctypes.Structure):
     ]
 
 
+class SparseOperand(ctypes.Structure):
+    _fields_ = [
+        ("pack_values", ctypes.c_void_p),
+        ("pack_meta", ctypes.c_void_p),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("rows", ctypes.c_int64),
+        ("cols", ctypes.c_int64),
+    ]
+
+
 _P = ctypes.c_void_p
 _SIGS = {
     "mllm_num_candidates": (ctypes.c_int32, [NM]),
@@ -97,6 +108,9 @@ _SIGS = {
     "mllm_encode_candidates": (ctypes.c_int, [NM, _P, ctypes.c_int64, _P, _P]),
     "mllm_decode_candidates": (ctypes.c_int, [NM, _P, ctypes.c_int64, _P, _P]),
     "mllm_noise_table": (ctypes.c_int, [_P, _P]),
+    "mllm_sparse_linear": (ctypes.c_int, [_P, ctypes.c_int32, NM, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "mllm_sparse_linear_workspace_bytes": (ctypes.c_size_t, []),
+    "mllm_sizeof_sparse_operand": (ctypes.c_size_t, []),
     "mllm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mllm_last_cuda_error": (ctypes.c_int32, []),
     "mllm_abi_version": (ctypes.c_int32, []),
@@ -121,7 +135,8 @@ def lib() -> ctypes.CDLL:
             fn.argtypes = args
         if h.mllm_abi_version() != ABI_VERSION:
             raise ImportError("libmllm.so ABI version mismatch")
-        if h.mllm_sizeof_matrix() != ctypes.sizeof(Matrix) or h.mllm_sizeof_hparams() != ctypes.sizeof(HParams):
+        if (h.mllm_sizeof_matrix() != ctypes.sizeof(Matrix) or h.mllm_sizeof_hparams() != ctypes.sizeof(HParams)
+                or h.mllm_sizeof_sparse_operand() != ctypes.sizeof(SparseOperand)):
             raise ImportError("libmllm.so struct layout mismatch")
         _lib = h
     return _lib
@@ -333,6 +348,37 @@ def mllm_encode_candidates(nm, idx: torch.Tensor, words: torch.Tensor, stream=No
 def mllm_decode_candidates(nm, words: torch.Tensor, n: int, idx: torch.Tensor, stream=None):
     _check(lib().mllm_decode_candidates(_nm(nm), _ptr(words), int(n), _ptr(idx), _stream(stream)),
            "mllm_decode_candidates")
+
+
+class SparseOperandArray:
+    """C array of mllm_sparse_operand built from (pack_values, pack_meta, x, y) tensors:
+    rows = y.shape[1], cols = x.shape[1]. Keeps the tensors alive with the array."""
+
+    def __init__(self, ops: Sequence):
+        self.ops = [tuple(o) for o in ops]
+        self.arr = (SparseOperand * max(len(self.ops), 1))()
+        for i, (vals, meta, x, y) in enumerate(self.ops):
+            self.arr[i] = SparseOperand(_ptr(vals), _ptr(meta), _ptr(x), _ptr(y), int(y.shape[1]), int(x.shape[1]))
+        self.n = len(self.ops)
+        self.ptr = ctypes.cast(self.arr, ctypes.c_void_p)
+
+
+def mllm_sparse_linear_workspace_bytes() -> int:
+    return lib().mllm_sparse_linear_workspace_bytes()
+
+
+def sparse_linear_workspace(device) -> torch.Tensor:
+    """A zero-filled workspace for mllm_sparse_linear on `device`."""
+    return torch.zeros(mllm_sparse_linear_workspace_bytes(), dtype=torch.uint8, device=device)
+
+
+def mllm_sparse_linear(ops, nm, tokens: int, workspace: torch.Tensor, stream=None):
+    """y = x W*^T for every (pack_values, pack_meta, x [tokens, cols], y [tokens, rows]) of ops
+    (or a prepared SparseOperandArray); workspace from sparse_linear_workspace()."""
+    a = ops if isinstance(ops, SparseOperandArray) else SparseOperandArray(ops)
+    _check(lib().mllm_sparse_linear(a.ptr, a.n, _nm(nm), int(tokens), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "mllm_sparse_linear")
 
 
 def mllm_last_cuda_error() -> int:

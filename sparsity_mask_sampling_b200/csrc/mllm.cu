@@ -11,6 +11,7 @@
 #include "kernels_2of4.cuh"
 #include "kernels_4of8.cuh"
 #include "kernels_diag.cuh"
+#include "kernels_spl.cuh"
 
 namespace mllm {
 namespace {
@@ -228,6 +229,56 @@ std::vector<Group> make_groups(const mllm_matrix *mats, int32_t n_mats, int M, K
         out.push_back(g);
     }
     return out;
+}
+
+// ------------------------------------------------------------------------ sparse linear
+
+constexpr int kSplRowTiles = 2;   // row tiles of 16 per CTA task (4 warps per tile split k)
+constexpr int kSplDepth = 2;      // slabs in flight per warp
+
+mllm_status validate_operands(const mllm_sparse_operand *ops, int32_t n_ops, mllm_nm nm, int32_t tokens) {
+    if (!num_cand(nm)) return MLLM_ERR_UNSUPPORTED;
+    if (!ops || n_ops <= 0 || tokens < 1 || tokens > spl::kMaxTokens) return MLLM_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_ops; ++i) {
+        const mllm_sparse_operand &o = ops[i];
+        if (o.rows < 0 || o.cols < 0 || o.cols % nm.m) return MLLM_ERR_INVALID_ARG;
+        if (o.rows == 0) continue;
+        mllm_status s;
+        if ((s = check_ptr(o.y, true)) != MLLM_OK) return s;
+        const bool any = o.cols > 0;
+        if ((s = check_ptr(o.pack_values, any)) != MLLM_OK) return s;
+        if ((s = check_ptr(o.pack_meta, any)) != MLLM_OK) return s;
+        if ((s = check_ptr(o.x, any)) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+template <int kN, int kNT>
+mllm_status launch_spl_sk(const spl::SkGroup &g, float *part, unsigned int *tickets, cudaStream_t st) {
+    auto fn = spl::sparse_linear_sk_kernel<kN, kNT>;
+    constexpr int smem = spl::sk_smem_bytes<kNT>();
+    const int64_t grid = grid_for((const void *)fn, spl::kSkThreads, smem, INT32_MAX,
+                                  spl::kMaxSkWarps / spl::kSkWarps);
+    fn<<<(unsigned)grid, spl::kSkThreads, smem, st>>>(g, part, tickets);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int kNT>
+mllm_status launch_spl_sp(const spl::SkGroup &g, float *part, unsigned int *tickets, cudaStream_t st) {
+    auto fn = spl::sparse_linear_sp_kernel<kNT>;
+    constexpr int smem = spl::sp_smem_bytes<kNT>();
+    const int64_t grid = grid_for((const void *)fn, spl::kSkThreads, smem, INT32_MAX,
+                                  spl::kMaxSkWarps / spl::kSkWarps);
+    fn<<<(unsigned)grid, spl::kSkThreads, smem, st>>>(g, part, tickets);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int kN, bool kVec, int kNT>
+mllm_status launch_spl(const spl::OpGroup &g, cudaStream_t st) {
+    auto fn = spl::sparse_linear_kernel<kN, kVec, kNT, kSplRowTiles, kSplDepth>;
+    const int64_t grid = grid_for((const void *)fn, spl::kCtaThreads, 0, g.total_tasks, INT32_MAX);
+    fn<<<(unsigned)grid, spl::kCtaThreads, 0, st>>>(g);
+    return cuda_status(cudaGetLastError());
 }
 
 // ------------------------------------------------------------------------ prior launcher
@@ -643,6 +694,93 @@ mllm_status mllm_decode_candidates(mllm_nm nm, const uint32_t *words, int64_t n,
     diag::decode_kernel<<<(unsigned)grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(words, n, C, D, idx);
     return cuda_status(cudaGetLastError());
 }
+
+mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, mllm_nm nm, int32_t tokens,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+    mllm_status s = validate_operands(ops, n_ops, nm, tokens);
+    if (s != MLLM_OK) return s;
+    if (!workspace || workspace_bytes < spl::kSkWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *part = static_cast<float *>(workspace);
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) +
+                                                             (size_t)spl::kMaxSkWarps * 2 * 32 * spl::kSkPartFloats * sizeof(float));
+    std::vector<int32_t> order;
+    for (int32_t i = 0; i < n_ops; ++i) {
+        if (ops[i].rows == 0) continue;
+        if (ops[i].cols == 0) {  // y = 0
+            s = cuda_status(cudaMemsetAsync(ops[i].y, 0, sizeof(float) * (size_t)tokens * (size_t)ops[i].rows, st));
+            if (s != MLLM_OK) return s;
+            continue;
+        }
+        order.push_back(i);
+    }
+    // operands with the longest rows first (the tiled kernel's first wave takes them)
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int32_t a, int32_t b) { return ops[a].cols > ops[b].cols; });
+    const bool is24 = nm.m == 4, two = tokens > 8;
+    for (size_t i0 = 0; i0 < order.size(); i0 += kMaxMats) {
+        const size_t n = std::min<size_t>(kMaxMats, order.size() - i0);
+        bool vec = true, words = true;
+        for (size_t k = 0; k < n; ++k) {
+            vec = vec && (ops[order[i0 + k]].cols % 16 == 0);
+            words = words && (ops[order[i0 + k]].cols % 32 == 0);
+        }
+        if (vec) {  // streamed kernels: the launch's chunks split evenly over all warps
+                    // (2:4 with whole metadata words: sparse tensor cores; else expansion)
+            spl::SkGroup g{};
+            g.tokens = tokens;
+            int64_t acc = 0;
+            for (size_t k = 0; k < n; ++k) {
+                const mllm_sparse_operand &o = ops[order[i0 + k]];
+                spl::SkOp &d = g.d[k];
+                d.vals = static_cast<const uint32_t *>(o.pack_values);
+                d.meta = o.pack_meta;
+                d.x = static_cast<const uint32_t *>(o.x);
+                d.y = o.y;
+                d.rows = o.rows;
+                d.cols = o.cols;
+                d.nch = (o.cols + spl::kChunk - 1) / spl::kChunk;
+                d.ntiles = (o.rows + spl::kSkRows - 1) / spl::kSkRows;
+                d.chunk_begin = acc;
+                acc += d.nch * d.ntiles;
+            }
+            g.n = (int32_t)n;
+            g.total_chunks = acc;
+            if (is24 && words) s = two ? launch_spl_sp<2>(g, part, tickets, st) : launch_spl_sp<1>(g, part, tickets, st);
+            else if (is24) s = two ? launch_spl_sk<2, 2>(g, part, tickets, st) : launch_spl_sk<2, 1>(g, part, tickets, st);
+            else s = two ? launch_spl_sk<4, 2>(g, part, tickets, st) : launch_spl_sk<4, 1>(g, part, tickets, st);
+            if (s != MLLM_OK) return s;
+            continue;
+        }
+        spl::OpGroup g{};
+        g.tokens = tokens;
+        int64_t acc = 0;
+        const int64_t rows_per_task = 16 * kSplRowTiles;
+        for (size_t k = 0; k < n; ++k) {
+            const mllm_sparse_operand &o = ops[order[i0 + k]];
+            spl::Op &d = g.d[k];
+            d.vals = static_cast<const uint32_t *>(o.pack_values);
+            d.meta = o.pack_meta;
+            d.x = static_cast<const uint32_t *>(o.x);
+            d.y = o.y;
+            d.rows = o.rows;
+            d.cols = o.cols;
+            d.task_begin = acc;
+            acc += (o.rows + rows_per_task - 1) / rows_per_task;
+        }
+        g.n = (int32_t)n;
+        g.total_tasks = acc;
+        if (is24) s = two ? launch_spl<2, false, 2>(g, st) : launch_spl<2, false, 1>(g, st);
+        else s = two ? launch_spl<4, false, 2>(g, st) : launch_spl<4, false, 1>(g, st);
+        if (s != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+size_t mllm_sparse_linear_workspace_bytes(void) { return spl::kSkWorkspaceBytes; }
+
+size_t mllm_sizeof_sparse_operand(void) { return sizeof(mllm_sparse_operand); }
 
 mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t *gids,
                        int64_t n_blocks, float *g_out, void *stream) {

@@ -42,6 +42,7 @@ def test_abi_guards(M):
     assert L.mllm_abi_version() == M.ABI_VERSION
     assert L.mllm_sizeof_matrix() == ctypes.sizeof(M.Matrix)
     assert L.mllm_sizeof_hparams() == ctypes.sizeof(M.HParams)
+    assert L.mllm_sizeof_sparse_operand() == ctypes.sizeof(M.SparseOperand)
     assert M.mllm_workspace_bytes() >= 16 + 8 * 148
 
 
@@ -165,3 +166,36 @@ def test_compiled_noise_table_matches_oracle_table(M):
     oc, oT, _ = oracle.nlog_table()
     assert np.array_equal(c.view(np.uint32), oc.view(np.uint32))
     assert np.array_equal(T.view(np.uint32), oT.view(np.uint32))
+
+
+def _spl(M, ops, nm=(2, 4), tokens=8, ws=0x100000, wsb=None):
+    arr = (M.SparseOperand * max(len(ops), 1))(*ops)
+    wsb = M.mllm_sparse_linear_workspace_bytes() if wsb is None else wsb
+    return M.lib().mllm_sparse_linear(ctypes.cast(arr, ctypes.c_void_p) if ops else None, len(ops),
+                                      M.NM(*nm), tokens, ws, wsb, 0)
+
+
+def _op(M, **kw):
+    base = dict(pack_values=0x1000, pack_meta=0x2000, x=0x3000, y=0x4000, rows=32, cols=64)
+    base.update(kw)
+    return M.SparseOperand(**base)
+
+
+def test_sparse_linear_validation(M):
+    assert _spl(M, []) == M.MLLM_ERR_INVALID_ARG
+    assert _spl(M, [_op(M)], nm=(1, 4)) == M.MLLM_ERR_UNSUPPORTED
+    for tokens in (0, -1, 17):
+        assert _spl(M, [_op(M)], tokens=tokens) == M.MLLM_ERR_INVALID_ARG, tokens
+    assert _spl(M, [_op(M, cols=6)]) == M.MLLM_ERR_INVALID_ARG
+    assert _spl(M, [_op(M, cols=12)], nm=(4, 8)) == M.MLLM_ERR_INVALID_ARG
+    assert _spl(M, [_op(M, rows=-1)]) == M.MLLM_ERR_INVALID_ARG
+    for field in ("pack_values", "pack_meta", "x", "y"):
+        assert _spl(M, [_op(M, **{field: 0})]) == M.MLLM_ERR_INVALID_ARG, field
+        assert _spl(M, [_op(M), _op(M, **{field: 0x5008})]) == M.MLLM_ERR_MISALIGNED, field
+    # cols == 0 needs only y; rows == 0 needs nothing (these would launch, so only the
+    # rejected variants are called here)
+    assert _spl(M, [_op(M, cols=0, y=0)]) == M.MLLM_ERR_INVALID_ARG
+    # workspace
+    assert _spl(M, [_op(M)], ws=0) == M.MLLM_ERR_WORKSPACE
+    assert _spl(M, [_op(M)], wsb=M.mllm_sparse_linear_workspace_bytes() - 4) == M.MLLM_ERR_WORKSPACE
+    assert _spl(M, [_op(M)], ws=0x100008) == M.MLLM_ERR_MISALIGNED

@@ -1,0 +1,202 @@
+"""Parity of mllm_sparse_linear (y = x W*^T on the packed hard mask) with the oracle.
+
+The packed operands come from the oracle's own hard_pack of seeded weights and logits (no
+oracle input comes from the GPU); a second set of cases runs the whole chain on the GPU
+(hard_pack then sparse_linear) from the same seeded inputs. Sizes cover several k-chunks and
+row tiles, ragged tails (rows not a multiple of the 32-row task, columns not a multiple of
+the 64-column chunk, columns not a multiple of 16: the element-wise loader), every token
+count class (1, 8, 9, 16), grouped calls with empty operands, and the LLaMA-2-7B shapes at
+full size on sampled rows.
+"""
+from itertools import combinations
+
+import numpy as np
+import pytest
+import torch
+
+import _tol
+from sparsity_mask_sampling_b200 import (MatrixArray, MatrixBuffers, mllm_hard_pack, mllm_sparse_linear,
+                                         mllm_sparse_linear_workspace_bytes, sparse_linear_workspace)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+C_OF = {(2, 4): 6, (4, 8): 70}
+
+
+@pytest.fixture(scope="module")
+def ws():
+    return sparse_linear_workspace(DEV)
+
+
+def _tickets_clear(ws):
+    """The call leaves its completion counters (the workspace's last 4096 words) at zero."""
+    return not ws[-4 * 4096:].any()
+
+
+def _bf16_bits(rng, shape, std):
+    f = rng.normal(0.0, std, size=shape).astype(np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _val(bits):
+    return (np.asarray(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _dev16(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+def _dev_meta(meta):
+    meta = np.ascontiguousarray(meta)
+    return torch.from_numpy(meta.view(np.int32 if meta.dtype == np.uint32 else np.int16)).to(DEV)
+
+
+def _random_packed(rng, nm, rows, cols):
+    """A packed operand drawn directly: random bf16 values and a random valid candidate per
+    block, encoded as hard_pack encodes it (for full-size shapes, where [B, C] logits for the
+    oracle's hard_pack would take gigabytes of host memory)."""
+    n, m = nm
+    bpr = cols // m
+    values = _bf16_bits(rng, (rows, bpr * n), 0.02)
+    combos = list(combinations(range(m), n))
+    k = rng.integers(0, len(combos), size=(rows, bpr))
+    if m == 4:
+        nib = np.array([p[0] | p[1] << 2 for p in combos], np.uint64)[k]
+        words = (bpr + 7) // 8
+        pad = np.zeros((rows, words * 8), np.uint64)
+        pad[:, :bpr] = nib
+        meta = (pad.reshape(rows, words, 8) << (4 * np.arange(8, dtype=np.uint64))).sum(-1).astype(np.uint32)
+    else:
+        meta = np.array([p[0] | p[1] << 3 | p[2] << 6 | p[3] << 9 for p in combos], np.uint16)[k]
+    return values, meta
+
+
+class Operand:
+    def __init__(self, orc, nm, rows, cols, tokens, seed, direct=False):
+        rng = np.random.default_rng(seed)
+        n, m = nm
+        self.nm, self.rows, self.cols = nm, rows, cols
+        if direct:
+            self.values, self.meta = _random_packed(rng, nm, rows, cols)
+        else:
+            self.W = _bf16_bits(rng, (rows, cols), 0.02)
+            self.pi = rng.normal(0, 1, size=(rows * cols // m, C_OF[nm])).astype(np.float32)
+            self.values, self.meta, _ = orc.hard_pack(n, m, self.W, self.pi)
+        self.x = _bf16_bits(rng, (tokens, cols), 1.0)
+        self.d_values, self.d_meta = _dev16(self.values), _dev_meta(self.meta)
+        self.d_x = _dev16(self.x)
+        self.y = torch.full((tokens, rows), float("nan"), dtype=torch.float32, device=DEV)
+
+    def op(self):
+        return (self.d_values, self.d_meta, self.d_x, self.y)
+
+    def check(self, orc, rows_sel=None):
+        n, m = self.nm
+        vals, meta = self.values, self.meta
+        if rows_sel is not None:
+            vals, meta = vals[rows_sel], meta[rows_sel]
+        y_ref = orc.sparse_linear(n, m, vals, meta, self.x)
+        # sum_k |x_k w_k| for the tolerance: the same product with the sign bits cleared
+        absxw = orc.sparse_linear(n, m, vals & 0x7FFF, meta, self.x & 0x7FFF)
+        got = self.y.cpu().numpy().astype(np.float64)
+        if rows_sel is not None:
+            got = got[:, rows_sel]
+        return _tol.assert_spl_close(got, y_ref, absxw, self.cols)
+
+
+SHAPES = [(48, 256), (37, 1040), (70, 1088), (33, 84), (16, 40), (5, 8)]
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+@pytest.mark.parametrize("tokens", [1, 8, 9, 16])
+def test_sparse_linear_matches_oracle(orc, ws, nm, tokens):
+    shapes = [(r, c) for r, c in SHAPES if c % nm[1] == 0]
+    ops = [Operand(orc, nm, r, c, tokens, seed=10 * i + tokens) for i, (r, c) in enumerate(shapes)]
+    mllm_sparse_linear([o.op() for o in ops[:3]], nm, tokens, ws)       # one grouped call (vector loads)
+    for o in ops[3:]:
+        mllm_sparse_linear([o.op()], nm, tokens, ws)                    # element-wise loads
+    torch.cuda.synchronize()
+    for o in ops:
+        o.check(orc)
+    assert _tickets_clear(ws)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_grouped_call_with_empty_operands_and_determinism(orc, ws, nm):
+    tokens = 5
+    a = Operand(orc, nm, 40, 512, tokens, seed=1)
+    b = Operand(orc, nm, 24, 128, tokens, seed=2)
+    empty_rows = (a.d_values, a.d_meta, torch.empty(tokens, 0, device=DEV, dtype=torch.bfloat16),
+                  torch.empty(tokens, 0, device=DEV))
+    y0 = torch.full((tokens, 12), float("nan"), device=DEV)
+    no_cols = (None, None, torch.empty(tokens, 0, device=DEV, dtype=torch.bfloat16), y0)
+    mllm_sparse_linear([a.op(), empty_rows, no_cols, b.op()], nm, tokens, ws)
+    torch.cuda.synchronize()
+    a.check(orc)
+    b.check(orc)
+    assert torch.equal(y0, torch.zeros_like(y0))
+    first = a.y.clone()
+    for _ in range(3):
+        mllm_sparse_linear([a.op()], nm, tokens, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(first, a.y)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_gpu_chain_pack_then_linear(orc, ws, nm):
+    """hard_pack on the GPU, then sparse_linear on its output, against the oracle chain."""
+    n, m = nm
+    rows, cols, tokens = 96, 768, 8
+    o = Operand(orc, nm, rows, cols, tokens, seed=5)
+    W = _dev16(o.W)
+    mb = MatrixBuffers(W=W, logits=torch.from_numpy(o.pi).to(DEV))
+    mb.pack_values = torch.empty(rows, cols // m * n, dtype=torch.bfloat16, device=DEV)
+    mb.pack_meta = torch.empty(o.d_meta.shape, dtype=o.d_meta.dtype, device=DEV)
+    mllm_hard_pack(MatrixArray([mb]), nm)
+    mllm_sparse_linear([(mb.pack_values, mb.pack_meta, o.d_x, o.y)], nm, tokens, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(mb.pack_meta, o.d_meta)
+    o.check(orc)
+
+
+@pytest.mark.parametrize("nm,tokens", [((2, 4), 8), ((2, 4), 16), ((4, 8), 8)])
+def test_llama_shapes_full_size_sampled_rows(orc, ws, nm, tokens):
+    """q/o [4096, 4096], gate [11008, 4096], down [4096, 11008] in one grouped call, the
+    launch the benchmark times; the oracle checks 24 rows of each (first, last, random)."""
+    shapes = [(4096, 4096), (11008, 4096), (4096, 11008)]
+    ops = [Operand(orc, nm, r, c, tokens, seed=50 + i, direct=True) for i, (r, c) in enumerate(shapes)]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    for o in ops:
+        sel = np.unique(np.concatenate([[0, o.rows - 1], rng.choice(o.rows, 22, replace=False)]))
+        o.check(orc, sel)
+        assert torch.isfinite(o.y).all()
+    assert _tickets_clear(ws)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+@pytest.mark.parametrize("tokens", [3, 16])
+def test_tiles_cut_into_many_pieces(orc, ws, nm, tokens):
+    """Few rows and long rows: each 32-row tile is cut between hundreds of warps, whose
+    partial tiles the last arriving warp adds; repeated calls reuse the workspace."""
+    o = Operand(orc, nm, 40, 16384, tokens, seed=77, direct=True)
+    for _ in range(2):
+        mllm_sparse_linear([o.op()], nm, tokens, ws)
+    torch.cuda.synchronize()
+    o.check(orc)
+    assert _tickets_clear(ws)
+
+
+@pytest.mark.parametrize("tokens", [2, 8, 13])
+def test_2of4_tensor_core_path_ragged(orc, ws, tokens):
+    """2:4 with whole metadata words (cols % 32 == 0) runs on the sparse tensor cores: rows
+    not a multiple of the 32-row tile and a last 64-column chunk with only one 32-column
+    window in the matrix."""
+    nm = (2, 4)
+    ops = [Operand(orc, nm, r, c, tokens, seed=90 + i) for i, (r, c) in enumerate([(45, 96), (33, 160), (7, 32)])]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
+    torch.cuda.synchronize()
+    for o in ops:
+        o.check(orc)
+    assert _tickets_clear(ws)

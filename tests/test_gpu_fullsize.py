@@ -71,7 +71,7 @@ def _check_prior(orc, stack, samples):
         pi_ref, _, _ = orc.prior_init(*w.nm, s.W, s.gids, w.alpha, w.init_std, 0)
         got = s.mb.logits[s.idx_t].cpu().numpy().astype(np.float64)
         err = np.abs(got - pi_ref)
-        assert not (err > 1e-6 * np.abs(pi_ref).max(1, keepdims=True) + 1e-12).any()
+        assert (err <= 1e-6 * np.abs(pi_ref).max(1, keepdims=True) + 1e-12).all()
         assert not s.mb.adam_m[s.idx_t].any() and not s.mb.adam_v[s.idx_t].any()
         s.pi, s.m, s.v = pi_ref.astype(np.float32), np.zeros_like(pi_ref, np.float32), np.zeros_like(pi_ref, np.float32)
 
