@@ -620,8 +620,12 @@ __global__ void __launch_bounds__(kSkThreads, 1) sparse_linear_sk_kernel(const _
 constexpr int kSpRowBytes = 80;   // 64 bytes of values + 2 metadata words, padded
 constexpr int kSpTokBytes = 144;  // 64 columns of x (128 bytes), padded
 template <int kNT> constexpr int sp_stage_bytes() { return kSkRows * kSpRowBytes + 8 * kNT * kSpTokBytes; }
-template <int kNT> constexpr int sp_stages() { return kNT == 1 ? 6 : 5; }
-template <int kNT> constexpr int sp_smem_bytes() { return kSkWarps * sp_stages<kNT>() * sp_stage_bytes<kNT>(); }
+// 16 warps x 3 stages (up to 8 tokens) and 12 x 3 (16 tokens, more registers) keep ~110 KB
+// per SM in flight; more warps with shallower rings measured faster than 8 x 6 (latency of
+// each warp's own instruction chains, not bytes in flight, limited the deeper rings)
+template <int kNT> constexpr int sp_warps() { return kNT == 1 ? 16 : 12; }
+template <int kNT> constexpr int sp_stages() { return kNT == 1 ? 3 : 3; }
+template <int kNT> constexpr int sp_smem_bytes() { return sp_warps<kNT>() * sp_stages<kNT>() * sp_stage_bytes<kNT>(); }
 
 __device__ __forceinline__ void mma_sp_bf16_16832(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                   const uint32_t (&b)[4], uint32_t e) {
@@ -642,66 +646,115 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const unsigned cha
                  : "r"(a));
 }
 
-// Source pointers of one lane's copies for the tile the load cursor is in.
+// Copy state of one lane for the chunk the load cursor points at: source byte pointers
+// (advanced by one chunk per issue) and copy sizes (0 = zero-fill) of its pieces -- values of
+// rows 32*tile + lane/4 + 8k (16-byte quarter lane%4), metadata of row 32*tile + lane (two
+// words), x of tokens lane/8 + 4k (16-byte part lane%8).
 template <int kNT>
-struct SpSrc {
-    const uint32_t *v[4];   // values of rows 32*tile + lane/4 + 8k, 16-byte quarter lane%4
-    const uint32_t *m;      // metadata of row 32*tile + lane
-    const uint32_t *x[2 * kNT];  // x of token lane/8 + 4k, 16-byte part lane%8
-    unsigned vin, min_, xin;  // in-range bits
+struct SpLoad {
+    int op, j, nch;
+    int64_t tile;
+    const char *v[4], *m, *x[2 * kNT];
+    unsigned vsz[4], msz, xsz[2 * kNT];
 };
 
+// Positions the copy state at chunk j of tile `tile` of operand `op`.
 template <int kNT>
-__device__ __forceinline__ void sp_tile_src(const SkGroup &grp, const Cursor &c, int lane, SpSrc<kNT> &src) {
-    const SkOp &d = grp.d[c.op];
-    const int64_t wpr = d.cols >> 2, mw = d.cols >> 5;
-    src.vin = 0u;
+__device__ __forceinline__ void sp_load_at(const SkGroup &grp, int op, int64_t tile, int j, int lane, SpLoad<kNT> &L) {
+    const SkOp &d = grp.d[op];
+    L.op = op;
+    L.tile = tile;
+    L.j = j;
+    L.nch = (int)d.nch;
+    const int64_t vrow = d.cols, mrow = d.cols >> 3, xrow = d.cols << 1;  // bytes per row (2:4)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const int64_t r = c.tile * kSkRows + (lane >> 2) + 8 * k;
+        const int64_t r = tile * kSkRows + (lane >> 2) + 8 * k;
         const bool in = r < d.rows;
-        src.v[k] = d.vals + (in ? r * wpr : 0) + 4 * (lane & 3);
-        src.vin |= (unsigned)in << k;
+        L.v[k] = reinterpret_cast<const char *>(d.vals) + (in ? r * vrow : 0) + 16 * (lane & 3) + 64 * j;
+        L.vsz[k] = in ? 16u : 0u;
     }
-    const int64_t rm = c.tile * kSkRows + lane;
-    src.min_ = rm < d.rows;
-    src.m = static_cast<const uint32_t *>(d.meta) + (src.min_ ? rm * mw : 0);
-    src.xin = 0u;
+    const int64_t rm = tile * kSkRows + lane;
+    const bool min = rm < d.rows;
+    L.m = static_cast<const char *>(d.meta) + (min ? rm * mrow : 0) + 8 * j;
+    L.msz = min ? 4u : 0u;
 #pragma unroll
     for (int k = 0; k < 2 * kNT; ++k) {
         const int tok = (lane >> 3) + 4 * k;
         const bool in = tok < grp.tokens;
-        src.x[k] = d.x + (in ? (int64_t)tok * (d.cols >> 1) : 0) + 4 * (lane & 7);
-        src.xin |= (unsigned)in << k;
+        L.x[k] = reinterpret_cast<const char *>(d.x) + (in ? (int64_t)tok * xrow : 0) + 16 * (lane & 7) + 128 * j;
+        L.xsz[k] = in ? 16u : 0u;
     }
 }
 
+// Issues the copies of the current chunk into `stage` (a shared-memory address) and moves
+// the state to the next chunk of the sequence.
 template <int kNT>
-__device__ __forceinline__ void sp_issue(const SkGroup &grp, const Cursor &c, const SpSrc<kNT> &src,
-                                         unsigned char *stage, int lane) {
-    const int64_t cols = grp.d[c.op].cols, col0 = c.j * kChunk;
-    const bool whole = col0 + kChunk <= cols;  // every piece of the chunk is inside the row
-    const unsigned jw = (unsigned)c.j;         // chunk index (chunks per row < 2^26)
+__device__ __forceinline__ void sp_issue(const SkGroup &grp, SpLoad<kNT> &L, unsigned stage, int lane) {
+    const int cols = (int)grp.d[L.op].cols, col0 = L.j * kChunk;
+    const bool whole = col0 + kChunk <= cols;  // only a row's last chunk can be partial
+    const unsigned vdst = stage + (lane >> 2) * kSpRowBytes + 16 * (lane & 3);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const bool in = ((src.vin >> k) & 1u) && (whole || col0 + 16 * (lane & 3) < cols);
-        cp_async16_zfill(stage + ((lane >> 2) + 8 * k) * kSpRowBytes + 16 * (lane & 3), src.v[k] + 16u * jw, in);
+        const unsigned sz = (whole || col0 + 16 * (lane & 3) < cols) ? L.vsz[k] : 0u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(vdst + 8 * k * kSpRowBytes), "l"(L.v[k]),
+                     "r"(sz) : "memory");
+        L.v[k] += 64;
     }
+    const unsigned mdst = stage + lane * kSpRowBytes + 64;
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
-        const bool in = src.min_ && (whole || col0 + 32 * w < cols);
-        cp_async4_zfill(stage + lane * kSpRowBytes + 64 + 4 * w, src.m + 2u * jw + w, in);
+        const unsigned sz = (whole || col0 + 32 * w < cols) ? L.msz : 0u;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(mdst + 4 * w), "l"(L.m + 4 * w), "r"(sz)
+                     : "memory");
     }
+    L.m += 8;
+    const unsigned xdst = stage + kSkRows * kSpRowBytes + (lane >> 3) * kSpTokBytes + 16 * (lane & 7);
 #pragma unroll
     for (int k = 0; k < 2 * kNT; ++k) {
-        const bool in = ((src.xin >> k) & 1u) && (whole || col0 + 8 * (lane & 7) < cols);
-        cp_async16_zfill(stage + kSkRows * kSpRowBytes + ((lane >> 3) + 4 * k) * kSpTokBytes + 16 * (lane & 7),
-                         src.x[k] + 32u * jw, in);
+        const unsigned sz = (whole || col0 + 8 * (lane & 7) < cols) ? L.xsz[k] : 0u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(xdst + 4 * k * kSpTokBytes), "l"(L.x[k]),
+                     "r"(sz) : "memory");
+        L.x[k] += 128;
+    }
+    if (++L.j == L.nch) {  // next tile (or next operand)
+        const SkOp &d = grp.d[L.op];
+        if (L.tile + 1 < d.ntiles) sp_load_at<kNT>(grp, L.op, L.tile + 1, 0, lane, L);
+        else if (L.op + 1 < grp.n) sp_load_at<kNT>(grp, L.op + 1, 0, 0, lane, L);
+    }
+}
+
+// One stage: 2 windows x 2 row tiles x kNT mma.sp. kEdge: the stage may hold zero-filled
+// metadata words (rows past the matrix, or the window past its last column).
+template <int kNT, bool kEdge>
+__device__ __forceinline__ void sp_compute(const unsigned char *st, int lane, int g, int t, float (&acc)[2][kNT][4]) {
+    const unsigned char *pa = st + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kSpRowBytes + 16 * (lane >> 4);
+    const unsigned char *pb = st + kSkRows * kSpRowBytes + (lane & 7) * kSpTokBytes + 16 * (lane >> 3);
+    const uint32_t esel = (t & 1) ? 0x7632u : 0x5410u;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        uint32_t b[kNT][4];
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) ldmatrix_x4(b[nt], pb + 8 * nt * kSpTokBytes + 64 * w);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            uint32_t a[4];
+            ldmatrix_x4(a, pa + 16 * mt * kSpRowBytes + 32 * w);
+            const unsigned char *ra = st + (16 * mt + g) * kSpRowBytes;
+            uint32_t mg = lds32(ra + 64 + 4 * w), mg8 = lds32(ra + 8 * kSpRowBytes + 64 + 4 * w);
+            if constexpr (kEdge) {
+                mg = mg ? mg : 0x44444444u;
+                mg8 = mg8 ? mg8 : 0x44444444u;
+            }
+            const uint32_t e = __byte_perm(mg, mg8, esel);
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt) mma_sp_bf16_16832(acc[mt][nt], a[0], a[1], a[2], a[3], b[nt], e);
+        }
     }
 }
 
 template <int kNT>
-__global__ void __launch_bounds__(kSkThreads, 1) sparse_linear_sp_kernel(const __grid_constant__ SkGroup grp,
+__global__ void __launch_bounds__(32 * sp_warps<kNT>(), 1) sparse_linear_sp_kernel(const __grid_constant__ SkGroup grp,
                                                                          float *__restrict__ part,
                                                                          unsigned int *__restrict__ tickets) {
     constexpr int kD = sp_stages<kNT>();
@@ -709,71 +762,59 @@ __global__ void __launch_bounds__(kSkThreads, 1) sparse_linear_sp_kernel(const _
     extern __shared__ __align__(16) unsigned char s_ring[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t total = grp.total_chunks;
-    const int64_t GW = imin64((int64_t)gridDim.x * kSkWarps, total), gw = (int64_t)blockIdx.x * kSkWarps + warp;
+    constexpr int kW = sp_warps<kNT>();
+    const int64_t GW = imin64((int64_t)gridDim.x * kW, total), gw = (int64_t)blockIdx.x * kW + warp;
     if (gw >= GW) return;
-    const int64_t lo = gw * total / GW, hi = (gw + 1) * total / GW, n = hi - lo;
+    const int64_t lo = gw * total / GW, hi = (gw + 1) * total / GW;
+    const int n = (int)(hi - lo);  // chunks of this warp (< 2^31: a chunk holds > 2 KB of operands)
     unsigned char *ring = s_ring + (size_t)warp * kD * kStage;
-    Cursor ld = sk_decode(grp, lo), cc = ld;
-    SpSrc<kNT> src;
-    sp_tile_src<kNT>(grp, ld, lane, src);
+    const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+    const Cursor c0 = sk_decode(grp, lo);
+    SpLoad<kNT> L;
+    sp_load_at<kNT>(grp, c0.op, c0.tile, (int)c0.j, lane, L);
 #pragma unroll
     for (int s = 0; s < kD; ++s) {
-        if (s < n) {
-            sp_issue<kNT>(grp, ld, src, ring + s * kStage, lane);
-            sk_advance(grp, ld);
-            if (ld.j == 0 && s + 1 < n) sp_tile_src<kNT>(grp, ld, lane, src);
-        }
+        if (s < n) sp_issue<kNT>(grp, L, ring_s + s * kStage, lane);
         cp_async_commit();
     }
+    // compute cursor
+    int op = c0.op, j = (int)c0.j;
+    int64_t tile = c0.tile;
+    int nch = (int)grp.d[op].nch;
+    bool rows_edge = (tile + 1) * kSkRows > grp.d[op].rows, cols_edge = (grp.d[op].cols & (kChunk - 1)) != 0;
     float acc[2][kNT][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
     int s = 0;
-    for (int64_t f = 0; f < n; ++f) {
+    for (int f = 0; f < n; ++f) {
         cp_async_wait<kD - 1>();
         __syncwarp();  // every lane's copies of chunk f are visible to the warp
         const unsigned char *st = ring + s * kStage;
-        // ldmatrix row addresses of this lane: A (values) row 16mt + lane%8 + 8*(bit 3 of lane),
-        // 16-byte half lane/16 of the window; B (x) token 8nt + lane%8, 16-byte part lane/8
-        const unsigned char *pa = st + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kSpRowBytes + 16 * (lane >> 4);
-        const unsigned char *pb = st + kSkRows * kSpRowBytes + (lane & 7) * kSpTokBytes + 16 * (lane >> 3);
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            uint32_t b[kNT][4];
-#pragma unroll
-            for (int nt = 0; nt < kNT; ++nt) ldmatrix_x4(b[nt], pb + 8 * nt * kSpTokBytes + 64 * w);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                uint32_t a[4];
-                ldmatrix_x4(a, pa + 16 * mt * kSpRowBytes + 32 * w);
-                const unsigned char *ra = st + (16 * mt + g) * kSpRowBytes;
-                uint32_t mg = lds32(ra + 64 + 4 * w), mg8 = lds32(ra + 8 * kSpRowBytes + 64 + 4 * w);
-                mg = mg ? mg : 0x44444444u;
-                mg8 = mg8 ? mg8 : 0x44444444u;
-                const uint32_t e = __byte_perm(mg, mg8, (t & 1) ? 0x7632u : 0x5410u);
-#pragma unroll
-                for (int nt = 0; nt < kNT; ++nt) mma_sp_bf16_16832(acc[mt][nt], a[0], a[1], a[2], a[3], b[nt], e);
-            }
-        }
+        if (rows_edge || (cols_edge && j == nch - 1)) sp_compute<kNT, true>(st, lane, g, t, acc);
+        else sp_compute<kNT, false>(st, lane, g, t, acc);
         __syncwarp();  // the stage is read: it may be refilled
-        if (f + kD < n) {
-            sp_issue<kNT>(grp, ld, src, ring + s * kStage, lane);
-            sk_advance(grp, ld);
-            if (ld.j == 0 && f + kD + 1 < n) sp_tile_src<kNT>(grp, ld, lane, src);
-        }
+        if (f + kD < n) sp_issue<kNT>(grp, L, ring_s + s * kStage, lane);
         cp_async_commit();
         s = (s + 1 == kD) ? 0 : s + 1;
-        const SkOp &d = grp.d[cc.op];
-        if (cc.j == d.nch - 1 || f == n - 1) {
-            sk_finish<kNT>(grp, d, cc.tile, acc, part, tickets, gw, GW, total, lane, g, t);
+        if (j == nch - 1 || f == n - 1) {
+            sk_finish<kNT>(grp, grp.d[op], tile, acc, part, tickets, gw, GW, total, lane, g, t);
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                 for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
         }
-        if (f + 1 < n) sk_advance(grp, cc);
+        if (++j == nch && f + 1 < n) {
+            j = 0;
+            if (++tile == grp.d[op].ntiles) {
+                tile = 0;
+                ++op;
+                nch = (int)grp.d[op].nch;
+                cols_edge = (grp.d[op].cols & (kChunk - 1)) != 0;
+            }
+            rows_edge = (tile + 1) * kSkRows > grp.d[op].rows;
+        }
     }
     cp_async_wait<0>();
 }

@@ -241,7 +241,8 @@ mllm_status validate_operands(const mllm_sparse_operand *ops, int32_t n_ops, mll
     if (!ops || n_ops <= 0 || tokens < 1 || tokens > spl::kMaxTokens) return MLLM_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_ops; ++i) {
         const mllm_sparse_operand &o = ops[i];
-        if (o.rows < 0 || o.cols < 0 || o.cols % nm.m) return MLLM_ERR_INVALID_ARG;
+        if (o.rows < 0 || o.cols < 0 || o.cols % nm.m || o.rows > INT32_MAX || o.cols > INT32_MAX)
+            return MLLM_ERR_INVALID_ARG;
         if (o.rows == 0) continue;
         mllm_status s;
         if ((s = check_ptr(o.y, true)) != MLLM_OK) return s;
@@ -266,10 +267,9 @@ mllm_status launch_spl_sk(const spl::SkGroup &g, float *part, unsigned int *tick
 template <int kNT>
 mllm_status launch_spl_sp(const spl::SkGroup &g, float *part, unsigned int *tickets, cudaStream_t st) {
     auto fn = spl::sparse_linear_sp_kernel<kNT>;
-    constexpr int smem = spl::sp_smem_bytes<kNT>();
-    const int64_t grid = grid_for((const void *)fn, spl::kSkThreads, smem, INT32_MAX,
-                                  spl::kMaxSkWarps / spl::kSkWarps);
-    fn<<<(unsigned)grid, spl::kSkThreads, smem, st>>>(g, part, tickets);
+    constexpr int smem = spl::sp_smem_bytes<kNT>(), threads = 32 * spl::sp_warps<kNT>();
+    const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::sp_warps<kNT>());
+    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets);
     return cuda_status(cudaGetLastError());
 }
 
