@@ -617,31 +617,6 @@ def reference_arm(args, w):
     }
 
 
-def random_packed(rows, cols, nm, dev, gen):
-    """A packed hard-masked bf16 matrix with random values and a random valid candidate per
-    block, in mllm_hard_pack's format (for timing; the content does not change the cost)."""
-    import torch
-    from itertools import combinations
-
-    n, m = nm
-    bpr = cols // m
-    vals = torch.randn(rows, bpr * n, device=dev, generator=gen).to(torch.bfloat16)
-    combos = list(combinations(range(m), n))
-    k = torch.randint(0, len(combos), (rows, bpr), device=dev, generator=gen)
-    if m == 4:
-        nib = torch.tensor([p[0] | p[1] << 2 for p in combos], device=dev, dtype=torch.int64)[k]
-        words = (bpr + 7) // 8
-        pad = torch.zeros(rows, words * 8, device=dev, dtype=torch.int64)
-        pad[:, :bpr] = nib
-        shifts = 4 * torch.arange(8, device=dev, dtype=torch.int64)
-        w = (pad.view(rows, words, 8) << shifts).sum(-1)
-        meta = torch.where(w >= 2 ** 31, w - 2 ** 32, w).to(torch.int32)
-    else:
-        meta = torch.tensor([p[0] | p[1] << 3 | p[2] << 6 | p[3] << 9 for p in combos], device=dev,
-                            dtype=torch.int16)[k]
-    return vals, meta
-
-
 def sparse_linear_arm(args, w):
     """--mode sparse_linear: serving the learned sparse network (s.3.2, inference). Every
     matrix of the workload as a packed hard-masked bf16 weight; one pass = y = x W*^T for all
@@ -656,10 +631,12 @@ def sparse_linear_arm(args, w):
     torch.cuda.set_device(dev)
     pkg.lib()
     hbm_peak, peak_kind = peaks()
+    from sparsity_mask_sampling_b200 import inputs
+
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
     shapes = [(m.rows, m.cols) for _ in range(w.layers) for m in w.matrices]
-    packed = [random_packed(r, c, w.nm, dev, gen) for r, c in shapes]
+    packed = [inputs.packed_hard_mask(r, c, w.nm, seed=1000 + i, device=dev) for i, (r, c) in enumerate(shapes)]
     dense = [torch.randn(r, c, device=dev, generator=gen).to(torch.bfloat16) for r, c in shapes]
     wbytes = sum(v.numel() * 2 + mt.numel() * mt.element_size() for v, mt in packed)
     dbytes = sum(d.numel() * 2 for d in dense)

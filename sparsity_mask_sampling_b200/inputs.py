@@ -51,3 +51,31 @@ def moments(nblocks: int, C: int, seed=3, device="cpu"):
     m = torch.randn(nblocks, C, generator=g, device=device) * 1e-4
     v = torch.randn(nblocks, C, generator=g, device=device).abs() * 1e-8
     return m, v
+
+
+def packed_hard_mask(rows: int, cols: int, nm, seed=0, device="cpu", std=0.02):
+    """A hard-masked bf16 matrix already in mllm_hard_pack's compressed form: N(0, std^2)
+    values and a uniformly drawn candidate per block, encoded as the pack encodes kept
+    positions (2:4: nibble p0 | p1 << 2, 8 blocks per uint32 word of a row, unused nibbles
+    zero; 4:8: uint16 p0 | p1 << 3 | p2 << 6 | p3 << 9). Returns (values [rows, cols*N/M]
+    bf16, meta int32 [rows, ceil(cols/32)] or int16 [rows, cols/8]) -- a stand-in for a
+    trained model's packed weights, whose serving cost does not depend on the values."""
+    from itertools import combinations
+
+    n, m = nm
+    g = _gen(seed, device)
+    bpr = cols // m
+    vals = (torch.randn(rows, bpr * n, generator=g, device=device) * std).to(torch.bfloat16)
+    combos = list(combinations(range(m), n))
+    k = torch.randint(0, len(combos), (rows, bpr), generator=g, device=device)
+    if m == 4:
+        nib = torch.tensor([p[0] | p[1] << 2 for p in combos], device=device, dtype=torch.int64)[k]
+        words = (bpr + 7) // 8
+        pad = torch.zeros(rows, words * 8, device=device, dtype=torch.int64)
+        pad[:, :bpr] = nib
+        w = (pad.view(rows, words, 8) << (4 * torch.arange(8, device=device, dtype=torch.int64))).sum(-1)
+        meta = torch.where(w >= 2 ** 31, w - 2 ** 32, w).to(torch.int32)
+    else:
+        codes = [p[0] | p[1] << 3 | p[2] << 6 | p[3] << 9 for p in combos]
+        meta = torch.tensor(codes, device=device, dtype=torch.int16)[k]
+    return vals, meta

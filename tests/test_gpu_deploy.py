@@ -15,8 +15,9 @@ import pytest
 import torch
 
 import _tol
-from sparsity_mask_sampling_b200 import (MatrixArray, MatrixBuffers, mllm_hard_pack, mllm_sparse_linear,
-                                         mllm_sparse_linear_workspace_bytes, sparse_linear_workspace)
+from sparsity_mask_sampling_b200 import (MatrixArray, MatrixBuffers, configs, inputs, mllm_hard_pack,
+                                         mllm_sparse_linear, mllm_sparse_linear_workspace_bytes,
+                                         sparse_linear_workspace)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -199,4 +200,33 @@ def test_2of4_tensor_core_path_ragged(orc, ws, tokens):
     torch.cuda.synchronize()
     for o in ops:
         o.check(orc)
+    assert _tickets_clear(ws)
+
+
+def test_full_stack_call_as_benchmarked(orc, ws):
+    """The benchmark's serving call: the 224 matrices of the 32-layer LLaMA-2-7B stack as
+    packed 2:4 hard masks (7.3 GB; inputs.packed_hard_mask with the benchmark's seeds), one
+    call of 14 launches at 8 tokens; the oracle checks sampled rows of matrices in the first,
+    middle and last layers (every shape), and every output is written."""
+    w = configs.WORKLOADS["llama2_7b_stack_2of4"]
+    T = 8
+    shapes = [(m.rows, m.cols) for _ in range(w.layers) for m in w.matrices]
+    packed = [inputs.packed_hard_mask(r, c, w.nm, seed=1000 + i, device=DEV) for i, (r, c) in enumerate(shapes)]
+    xs = {c: inputs.weights(T, c, "bf16", 1.0, seed=c, device=DEV) for c in {c for _, c in shapes}}
+    ys = [torch.full((T, r), float("nan"), device=DEV) for r, _ in shapes]
+    mllm_sparse_linear([(v, mt, xs[c], y) for (v, mt), (r, c), y in zip(packed, shapes, ys)], w.nm, T, ws)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    for i in [0, 4, 6, 7 * 15 + 1, 7 * 15 + 5, 7 * 31 + 3, len(shapes) - 1]:
+        (v, mt), (r, c) = packed[i], shapes[i]
+        sel = np.unique(np.concatenate([[0, r - 1], rng.choice(r, 14, replace=False)]))
+        sel_t = torch.from_numpy(sel).to(DEV)
+        vals = v[sel_t].view(torch.int16).cpu().numpy().view(np.uint16)
+        meta = mt[sel_t].cpu().numpy().view(np.uint32)
+        x = xs[c].view(torch.int16).cpu().numpy().view(np.uint16)
+        y_ref = orc.sparse_linear(2, 4, vals, meta, x)
+        absxw = orc.sparse_linear(2, 4, vals & 0x7FFF, meta, x & 0x7FFF)
+        got = ys[i][:, sel_t].cpu().numpy().astype(np.float64)
+        _tol.assert_spl_close(got, y_ref, absxw, c)
+    assert all(bool(torch.isfinite(y).all()) for y in ys)
     assert _tickets_clear(ws)
