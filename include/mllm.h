@@ -258,8 +258,11 @@ typedef struct {
  * operands are skipped and cols == 0 gives y = 0 (pointers other than y may then be NULL).
  * workspace: device memory of mllm_sparse_linear_workspace_bytes() bytes, zero-filled by the
  * caller before its first use; every call leaves it zero-filled again (partial tiles of rows
- * whose columns are split between warps, and one completion counter per warp). Calls that
- * may run concurrently need separate workspaces. Deterministic on a given device: the
+ * whose columns are split between warps, one completion counter per warp, and an error word
+ * -- the uint32 at byte offset workspace_bytes - 16 -- that a call sets to nonzero if one of
+ * its asynchronous copies never completed within a bounded wait, in which case that call's
+ * y is invalid; it is never expected to be set). Calls that may run concurrently need
+ * separate workspaces. Deterministic on a given device: the
  * summation order depends only on the shapes and the launch size. Works for 2:4 and 4:8. */
 mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, mllm_nm nm, int32_t tokens,
                                void *workspace, size_t workspace_bytes, void *stream);

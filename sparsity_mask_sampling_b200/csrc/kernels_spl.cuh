@@ -21,6 +21,8 @@
 // chunk); hardware sparse tensor cores only take 2:4, so both patterns expand to dense tiles.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (type only; maps are encoded through the runtime's driver entry point)
+
 #include "device_common.cuh"
 
 namespace mllm {
@@ -353,10 +355,10 @@ template <int kNT> constexpr int sk_lane_bytes() { return 80 + 32 * kNT; }  // v
 template <int kNT> constexpr int sk_stages() { return kNT == 1 ? 6 : 5; }
 template <int kNT> constexpr int sk_smem_bytes() { return kSkWarps * sk_stages<kNT>() * 32 * sk_lane_bytes<kNT>(); }
 // workspace: two partial tiles per warp (2 m-tiles x kNT x 4 floats per lane, kNT <= 2),
-// then one ticket per warp
+// then one ticket per warp, then an error word (set when a bulk copy never completes)
 constexpr size_t kSkPartFloats = 2 * 2 * 4;
 constexpr size_t kSkWorkspaceBytes = (size_t)kMaxSkWarps * 2 * 32 * kSkPartFloats * sizeof(float) +
-                                     (size_t)kMaxSkWarps * sizeof(unsigned int);
+                                     (size_t)kMaxSkWarps * sizeof(unsigned int) + 16;  // + error word
 
 struct SkOp {
     const uint32_t *vals;
@@ -817,6 +819,188 @@ __global__ void __launch_bounds__(32 * sp_warps<kNT>(), 1) sparse_linear_sp_kern
         }
     }
     cp_async_wait<0>();
+}
+
+// ------------------------------------------------------------------ 2:4, tensor copies (TMA)
+
+// The same product for rows of whole 128-column stages (cols % 128 == 0, every LLM shape),
+// fed by the tensor memory accelerator: per 32-row x 128-column stage one lane issues four
+// tiled copies (cp.async.bulk.tensor.2d) -- the 32 x 64 box of compressed values, the 32 x 4
+// box of metadata words and two 8kNT x 64 boxes of x -- completing on the stage's mbarrier.
+// Boxes past the matrix (rows, tokens) are zero-filled by the copy engine. Values and x land
+// with the 128-byte swizzle (16-byte chunk c of box row r at chunk c ^ (r % 8)), so the
+// ldmatrix reads below are free of bank conflicts. Each tensor map describes one operand
+// (values, metadata, x) and is passed with the launch. Waits are bounded: a copy that never
+// lands sets the workspace's error word and the warp returns after a bounded wait for its
+// other stages. Work split and partial tiles as in the kernels above, 128-column chunks.
+
+constexpr int kTmChunk = 128;
+constexpr unsigned kTmSpinLimit = 1u << 24;
+template <int kNT> constexpr int tm_xbox_bytes() { return 8 * kNT * 128; }
+template <int kNT> constexpr int tm_stage_tx() { return 32 * 128 + 2 * tm_xbox_bytes<kNT>() + 32 * 16; }
+template <int kNT> constexpr int tm_stage_bytes() { return (tm_stage_tx<kNT>() + 1023) / 1024 * 1024; }
+template <int kNT> constexpr int tm_warps() { return 8; }
+template <int kNT> constexpr int tm_stages() { return 3; }
+template <int kNT> constexpr int tm_smem_bytes() { return tm_warps<kNT>() * tm_stages<kNT>() * tm_stage_bytes<kNT>() + 1024; }
+
+struct TmMaps {
+    CUtensorMap vals;  // bf16 [rows, cols/2], box 64 x 32, 128-byte swizzle
+    CUtensorMap meta;  // uint32 [rows, cols/32], box 4 x 32
+    CUtensorMap x;     // bf16 [tokens, cols], box 64 x 8kNT, 128-byte swizzle
+};
+
+struct TmGroup {
+    SkGroup g;
+    TmMaps maps[kMaxMats];
+};
+
+__device__ __forceinline__ void mbar_init(unsigned bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(unsigned bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0u;
+}
+__device__ __forceinline__ void tma_load_2d(unsigned dst, const CUtensorMap *map, int x, int y, unsigned bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+// Warp-uniform bounded wait for phase `parity` of a stage's barrier.
+__device__ __forceinline__ bool tm_wait(unsigned bar, unsigned parity) {
+    for (unsigned it = 0; it < kTmSpinLimit; ++it)
+        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+    return false;
+}
+
+template <int kNT>
+__device__ __forceinline__ void tm_issue(const TmGroup &tg, const Cursor &c, unsigned stage, unsigned bar) {
+    const TmMaps &mp = tg.maps[c.op];
+    const int j = (int)c.j, row0 = (int)(c.tile * kSkRows);
+    mbar_arrive_tx(bar, (unsigned)tm_stage_tx<kNT>());
+    tma_load_2d(stage, &mp.vals, 64 * j, row0, bar);
+    tma_load_2d(stage + 4096, &mp.x, 128 * j, 0, bar);
+    tma_load_2d(stage + 4096 + tm_xbox_bytes<kNT>(), &mp.x, 128 * j + 64, 0, bar);
+    tma_load_2d(stage + 4096 + 2 * tm_xbox_bytes<kNT>(), &mp.meta, 4 * j, row0, bar);
+}
+
+template <int kNT, bool kEdge>
+__device__ __forceinline__ void tm_compute(const unsigned char *st, int lane, int g, int t, float (&acc)[2][kNT][4]) {
+    const unsigned char *meta = st + 4096 + 2 * tm_xbox_bytes<kNT>();
+    const uint32_t esel = (t & 1) ? 0x7632u : 0x5410u;
+    const int ar = (lane & 7) + 8 * ((lane >> 3) & 1);  // A box row of this lane (+16 mt)
+    const int br = lane & 7;                             // x box row (token) of this lane (+8 nt)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const unsigned char *xb = st + 4096 + (w >> 1) * tm_xbox_bytes<kNT>();
+        uint32_t b[kNT][4];
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+            const int r = br + 8 * nt, c = 4 * (w & 1) + (lane >> 3);
+            ldmatrix_x4(b[nt], xb + r * 128 + ((c ^ (r & 7)) << 4));
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            const int r = ar + 16 * mt, c = 2 * w + (lane >> 4);
+            uint32_t a[4];
+            ldmatrix_x4(a, st + r * 128 + ((c ^ (r & 7)) << 4));
+            const unsigned char *ra = meta + (16 * mt + g) * 16 + 4 * w;
+            uint32_t mg = lds32(ra), mg8 = lds32(ra + 8 * 16);
+            if constexpr (kEdge) {
+                mg = mg ? mg : 0x44444444u;
+                mg8 = mg8 ? mg8 : 0x44444444u;
+            }
+            const uint32_t e = __byte_perm(mg, mg8, esel);
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt) mma_sp_bf16_16832(acc[mt][nt], a[0], a[1], a[2], a[3], b[nt], e);
+        }
+    }
+}
+
+template <int kNT>
+__global__ void __launch_bounds__(32 * tm_warps<kNT>(), 1) sparse_linear_tma_kernel(
+    const __grid_constant__ TmGroup tg, float *__restrict__ part, unsigned int *__restrict__ tickets,
+    unsigned int *__restrict__ err) {
+    constexpr int kW = tm_warps<kNT>(), kD = tm_stages<kNT>(), kStage = tm_stage_bytes<kNT>();
+    extern __shared__ unsigned char s_dyn_tm[];
+    __shared__ __align__(8) unsigned long long s_bar[kW][kD];
+    const SkGroup &grp = tg.g;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int64_t total = grp.total_chunks;
+    const int64_t GW = imin64((int64_t)gridDim.x * kW, total), gw = (int64_t)blockIdx.x * kW + warp;
+    if (gw >= GW) return;  // no block-wide barrier follows
+    const int64_t lo = gw * total / GW, hi = (gw + 1) * total / GW;
+    const int n = (int)(hi - lo);
+    // 1024-byte aligned ring (the swizzle pattern repeats every 1024 bytes)
+    const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_tm);
+    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
+    unsigned char *ring = s_dyn_tm + pad + (size_t)warp * kD * kStage;
+    const unsigned ring_s = dyn_s + pad + (unsigned)(warp * kD * kStage);
+    const unsigned bar0 = (unsigned)__cvta_generic_to_shared(&s_bar[warp][0]);
+    if (lane == 0) {
+        for (int s = 0; s < kD; ++s) mbar_init(bar0 + 8 * s, 1u);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    __syncwarp();
+    Cursor ld = sk_decode(grp, lo), cc = ld;
+#pragma unroll
+    for (int s = 0; s < kD; ++s)
+        if (s < n) {
+            if (lane == 0) tm_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+            sk_advance(grp, ld);
+        }
+    bool rows_edge = (cc.tile + 1) * kSkRows > grp.d[cc.op].rows;
+    float acc[2][kNT][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+    unsigned phase = 0u;  // bit s: parity of the next phase of stage s
+    int s = 0;
+    for (int f = 0; f < n; ++f) {
+        if (!tm_wait(bar0 + 8 * s, (phase >> s) & 1u)) {
+            if (lane == 0) atomicOr(err, 1u);
+            for (int q = 1; q < kD && f + q < n; ++q) {
+                const int sq = (s + q) % kD;
+                tm_wait(bar0 + 8 * sq, (phase >> sq) & 1u);
+            }
+            return;
+        }
+        phase ^= 1u << s;
+        const unsigned char *st = ring + s * kStage;
+        if (rows_edge) tm_compute<kNT, true>(st, lane, g, t, acc);
+        else tm_compute<kNT, false>(st, lane, g, t, acc);
+        __syncwarp();        // every lane has read the stage
+        fence_proxy_async();  // generic reads before the stage's next asynchronous writes
+        if (f + kD < n) {
+            if (lane == 0) tm_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+            sk_advance(grp, ld);
+        }
+        s = (s + 1 == kD) ? 0 : s + 1;
+        const SkOp &d = grp.d[cc.op];
+        if (cc.j == d.nch - 1 || f == n - 1) {
+            sk_finish<kNT>(grp, d, cc.tile, acc, part, tickets, gw, GW, total, lane, g, t);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+        }
+        if (f + 1 < n) {
+            sk_advance(grp, cc);
+            rows_edge = (cc.tile + 1) * kSkRows > grp.d[cc.op].rows;
+        }
+    }
 }
 
 }  // namespace spl

@@ -1,6 +1,7 @@
 // mllm.cu -- host side of libmllm: argument validation, grouping, launch configuration and
 // the extern "C" entry points declared in include/mllm.h.
 #include <algorithm>
+#include <cudaTypedefs.h>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -270,6 +271,56 @@ mllm_status launch_spl_sp(const spl::SkGroup &g, float *part, unsigned int *tick
     constexpr int smem = spl::sp_smem_bytes<kNT>(), threads = 32 * spl::sp_warps<kNT>();
     const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::sp_warps<kNT>());
     fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets);
+    return cuda_status(cudaGetLastError());
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A 2-D row-major tensor [outer, inner] with rows of row_bytes, copied in boxes of
+// box_outer x box_inner elements.
+bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    const auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The three maps of a 2:4 operand for the TMA kernel (cols % 128 == 0).
+bool encode_operand(spl::TmMaps *mp, const mllm_sparse_operand &o, int32_t tokens, int kNT) {
+    const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
+    return encode_2d(&mp->vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+           encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4, 32,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           encode_2d(&mp->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
+                     (uint32_t)(8 * kNT), CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int kNT>
+mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
+                           cudaStream_t st) {
+    auto fn = spl::sparse_linear_tma_kernel<kNT>;
+    constexpr int smem = spl::tm_smem_bytes<kNT>(), threads = 32 * spl::tm_warps<kNT>();
+    const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::tm_warps<kNT>());
+    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err);
     return cuda_status(cudaGetLastError());
 }
 
@@ -705,6 +756,7 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
     float *part = static_cast<float *>(workspace);
     unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) +
                                                              (size_t)spl::kMaxSkWarps * 2 * 32 * spl::kSkPartFloats * sizeof(float));
+    unsigned int *err = tickets + spl::kMaxSkWarps;
     std::vector<int32_t> order;
     for (int32_t i = 0; i < n_ops; ++i) {
         if (ops[i].rows == 0) continue;
@@ -721,32 +773,51 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
     const bool is24 = nm.m == 4, two = tokens > 8;
     for (size_t i0 = 0; i0 < order.size(); i0 += kMaxMats) {
         const size_t n = std::min<size_t>(kMaxMats, order.size() - i0);
-        bool vec = true, words = true;
+        bool vec = true, words = true, stages = true;
         for (size_t k = 0; k < n; ++k) {
             vec = vec && (ops[order[i0 + k]].cols % 16 == 0);
             words = words && (ops[order[i0 + k]].cols % 32 == 0);
+            stages = stages && (ops[order[i0 + k]].cols % spl::kTmChunk == 0);
         }
         if (vec) {  // streamed kernels: the launch's chunks split evenly over all warps
-                    // (2:4 with whole metadata words: sparse tensor cores; else expansion)
-            spl::SkGroup g{};
-            g.tokens = tokens;
-            int64_t acc = 0;
-            for (size_t k = 0; k < n; ++k) {
-                const mllm_sparse_operand &o = ops[order[i0 + k]];
-                spl::SkOp &d = g.d[k];
-                d.vals = static_cast<const uint32_t *>(o.pack_values);
-                d.meta = o.pack_meta;
-                d.x = static_cast<const uint32_t *>(o.x);
-                d.y = o.y;
-                d.rows = o.rows;
-                d.cols = o.cols;
-                d.nch = (o.cols + spl::kChunk - 1) / spl::kChunk;
-                d.ntiles = (o.rows + spl::kSkRows - 1) / spl::kSkRows;
-                d.chunk_begin = acc;
-                acc += d.nch * d.ntiles;
+            // 2:4 in whole 128-column stages: tensor copies (falls back if a map cannot be
+            // encoded); other 2:4 with whole metadata words: sparse tensor cores via cp.async;
+            // else block expansion
+            const bool tma = is24 && stages;
+            auto group_of = [&](int64_t chunk) {
+                spl::SkGroup g{};
+                g.tokens = tokens;
+                int64_t acc = 0;
+                for (size_t k = 0; k < n; ++k) {
+                    const mllm_sparse_operand &o = ops[order[i0 + k]];
+                    spl::SkOp &d = g.d[k];
+                    d.vals = static_cast<const uint32_t *>(o.pack_values);
+                    d.meta = o.pack_meta;
+                    d.x = static_cast<const uint32_t *>(o.x);
+                    d.y = o.y;
+                    d.rows = o.rows;
+                    d.cols = o.cols;
+                    d.nch = (o.cols + chunk - 1) / chunk;
+                    d.ntiles = (o.rows + spl::kSkRows - 1) / spl::kSkRows;
+                    d.chunk_begin = acc;
+                    acc += d.nch * d.ntiles;
+                }
+                g.n = (int32_t)n;
+                g.total_chunks = acc;
+                return g;
+            };
+            if (tma) {
+                static thread_local spl::TmGroup tg;
+                tg.g = group_of(spl::kTmChunk);
+                bool ok = true;
+                for (size_t k = 0; k < n && ok; ++k) ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1);
+                if (ok) {
+                    s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
+                    if (s != MLLM_OK) return s;
+                    continue;
+                }
             }
-            g.n = (int32_t)n;
-            g.total_chunks = acc;
+            const spl::SkGroup g = group_of(spl::kChunk);
             if (is24 && words) s = two ? launch_spl_sp<2>(g, part, tickets, st) : launch_spl_sp<1>(g, part, tickets, st);
             else if (is24) s = two ? launch_spl_sk<2, 2>(g, part, tickets, st) : launch_spl_sk<2, 1>(g, part, tickets, st);
             else s = two ? launch_spl_sk<4, 2>(g, part, tickets, st) : launch_spl_sk<4, 1>(g, part, tickets, st);

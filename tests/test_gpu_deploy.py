@@ -30,8 +30,9 @@ def ws():
 
 
 def _tickets_clear(ws):
-    """The call leaves its completion counters (the workspace's last 4096 words) at zero."""
-    return not ws[-4 * 4096:].any()
+    """The call leaves its completion counters and error word (the workspace's tail: 4096
+    tickets, then the error word and padding) at zero."""
+    return not ws[-(4 * 4096 + 16):].any()
 
 
 def _bf16_bits(rng, shape, std):
