@@ -16,6 +16,10 @@ measured copy bandwidth.
       (serving leg: the workload's matrices as packed hard masks, y = x W*^T per call for
        1, 8 and 16 tokens, against dense cuBLAS; one JSON line)
 
+The training line also carries "extras": once-per-run calls timed over the whole stack
+(mask statistics, mask difference, candidate code, prior from a given mask) and the
+serving product on the stack's own learned masks.
+
 Default workload: the full LLaMA-2-7B-shaped stack at 2:4 (32 layers x 7 matrices,
 1,619,001,344 blocks; logits and AdamW moments resident in HBM, ~130 GB, plus the next
 step's soft-masked weights of every layer, 13 GB). Under torchrun each rank runs its own
