@@ -592,10 +592,14 @@ def cpu_baseline(w, target_s=15.0):
     rate = n / dt
     n_blocks = int(min(max(rate * target_s, 1000 * threads), 5e7))
     dt, n = cpu_run(w, n_blocks, threads, 1)
+    # the same on one core, on a sample of ~2 s
+    dt1, n1 = cpu_run(w, max(1000, int(rate / threads * 2.0)), 1, 1)
     return {"value": n / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "value_1_core": n1 / dt1,
             "sample": f"{n:,} blocks drawn from {w.name} (random global ids; weights, logits and "
                       f"gradients from the same seeded distributions), one forward + backward + "
-                      f"AdamW step, {dt:.1f} s on {threads} threads"}
+                      f"AdamW step, {dt:.1f} s on {threads} threads; value_1_core: {n1:,} blocks, "
+                      f"{dt1:.1f} s on 1 thread"}
 
 
 def reference_arm(args, w):
