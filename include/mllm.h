@@ -270,6 +270,15 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
 /* Workspace bytes mllm_sparse_linear needs (independent of sizes). */
 size_t mllm_sparse_linear_workspace_bytes(void);
 
+/* Test of the bounded waits of mllm_sparse_linear's copy pipeline (no counterpart in the
+ * paper): one launch of the 2:4 kernel for one operand (cols % 128 == 0, tokens <= 8) in which
+ * the first pipeline stage of every warp is armed but never filled, so that every warp's wait
+ * runs out after its 1 s bound, sets the workspace's error word and returns. Takes about a
+ * second; y is left invalid and the workspace must be zero-filled again afterwards. Nothing
+ * faults and the context stays usable. MLLM_ERR_UNSUPPORTED for other shapes. */
+mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int32_t tokens, void *workspace,
+                                             size_t workspace_bytes, void *stream);
+
 /* The Gumbel noise itself, for inspection and statistical tests: g_out[i*C + c] = noise
  * of candidate c of the block with global id gids[i] at (seed, step). gids and g_out are
  * device arrays of n_blocks and n_blocks*C entries; step may be any value, including the

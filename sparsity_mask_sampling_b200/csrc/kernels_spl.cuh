@@ -830,12 +830,13 @@ __global__ void __launch_bounds__(32 * sp_warps<kNT>(), 1) sparse_linear_sp_kern
 // Boxes past the matrix (rows, tokens) are zero-filled by the copy engine. Values and x land
 // with the 128-byte swizzle (16-byte chunk c of box row r at chunk c ^ (r % 8)), so the
 // ldmatrix reads below are free of bank conflicts. Each tensor map describes one operand
-// (values, metadata, x) and is passed with the launch. Waits are bounded: a copy that never
-// lands sets the workspace's error word and the warp returns after a bounded wait for its
-// other stages. Work split and partial tiles as in the kernels above, 128-column chunks.
+// (values, metadata, x) and is passed with the launch. Waits are bounded (1 s): a copy that
+// never lands sets the workspace's error word and the warp returns after a bounded wait for
+// its other stages. arm_only_first (tests only) arms every warp's first stage without
+// filling it, so that this path runs. Work split and partial tiles as in the kernels above, 128-column chunks.
 
 constexpr int kTmChunk = 128;
-constexpr unsigned kTmSpinLimit = 1u << 24;
+constexpr unsigned long long kTmWaitNs = 1000000000ull;  // bound of one wait: 1 s (a stage lands in us)
 template <int kNT> constexpr int tm_xbox_bytes() { return 8 * kNT * 128; }
 template <int kNT> constexpr int tm_stage_tx() { return 32 * 128 + 2 * tm_xbox_bytes<kNT>() + 32 * 16; }
 template <int kNT> constexpr int tm_stage_bytes() { return (tm_stage_tx<kNT>() + 1023) / 1024 * 1024; }
@@ -877,11 +878,21 @@ __device__ __forceinline__ void tma_load_2d(unsigned dst, const CUtensorMap *map
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
-// Warp-uniform bounded wait for phase `parity` of a stage's barrier.
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
+    return t;
+}
+
+// Warp-uniform wait for phase `parity` of a stage's barrier, bounded by kTmWaitNs of lane
+// 0's clock; false if it ran out.
 __device__ __forceinline__ bool tm_wait(unsigned bar, unsigned parity) {
-    for (unsigned it = 0; it < kTmSpinLimit; ++it)
+    if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+    const unsigned long long t0 = __shfl_sync(0xFFFFFFFFu, globaltimer_ns(), 0);
+    while (true) {
         if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
-    return false;
+        if (__shfl_sync(0xFFFFFFFFu, globaltimer_ns(), 0) - t0 > kTmWaitNs) return false;
+    }
 }
 
 template <int kNT>
@@ -931,7 +942,7 @@ __device__ __forceinline__ void tm_compute(const unsigned char *st, int lane, in
 template <int kNT>
 __global__ void __launch_bounds__(32 * tm_warps<kNT>(), 1) sparse_linear_tma_kernel(
     const __grid_constant__ TmGroup tg, float *__restrict__ part, unsigned int *__restrict__ tickets,
-    unsigned int *__restrict__ err) {
+    unsigned int *__restrict__ err, int arm_only_first) {
     constexpr int kW = tm_warps<kNT>(), kD = tm_stages<kNT>(), kStage = tm_stage_bytes<kNT>();
     extern __shared__ unsigned char s_dyn_tm[];
     __shared__ __align__(8) unsigned long long s_bar[kW][kD];
@@ -957,7 +968,12 @@ __global__ void __launch_bounds__(32 * tm_warps<kNT>(), 1) sparse_linear_tma_ker
 #pragma unroll
     for (int s = 0; s < kD; ++s)
         if (s < n) {
-            if (lane == 0) tm_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+            if (lane == 0) {
+                if (s == 0 && arm_only_first)  // test of the bounded wait: a stage nothing fills
+                    mbar_arrive_tx(bar0, (unsigned)tm_stage_tx<kNT>());
+                else
+                    tm_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+            }
             sk_advance(grp, ld);
         }
     bool rows_edge = (cc.tile + 1) * kSkRows > grp.d[cc.op].rows;

@@ -316,11 +316,11 @@ bool encode_operand(spl::TmMaps *mp, const mllm_sparse_operand &o, int32_t token
 
 template <int kNT>
 mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
-                           cudaStream_t st) {
+                           cudaStream_t st, int arm_only_first = 0) {
     auto fn = spl::sparse_linear_tma_kernel<kNT>;
     constexpr int smem = spl::tm_smem_bytes<kNT>(), threads = 32 * spl::tm_warps<kNT>();
     const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::tm_warps<kNT>());
-    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err);
+    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err, arm_only_first);
     return cuda_status(cudaGetLastError());
 }
 
@@ -850,6 +850,36 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
 }
 
 size_t mllm_sparse_linear_workspace_bytes(void) { return spl::kSkWorkspaceBytes; }
+
+mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int32_t tokens, void *workspace,
+                                             size_t workspace_bytes, void *stream) {
+    const mllm_nm nm{2, 4};
+    mllm_status s = validate_operands(op, 1, nm, tokens);
+    if (s != MLLM_OK) return s;
+    if (!workspace || workspace_bytes < spl::kSkWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    if (op->rows == 0 || op->cols == 0 || op->cols % spl::kTmChunk || tokens > 8) return MLLM_ERR_UNSUPPORTED;
+    float *part = static_cast<float *>(workspace);
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) +
+                                                             (size_t)spl::kMaxSkWarps * 2 * 32 * spl::kSkPartFloats * sizeof(float));
+    static thread_local spl::TmGroup tg;
+    tg.g = spl::SkGroup{};
+    tg.g.tokens = tokens;
+    spl::SkOp &d = tg.g.d[0];
+    d.vals = static_cast<const uint32_t *>(op->pack_values);
+    d.meta = op->pack_meta;
+    d.x = static_cast<const uint32_t *>(op->x);
+    d.y = op->y;
+    d.rows = op->rows;
+    d.cols = op->cols;
+    d.nch = op->cols / spl::kTmChunk;
+    d.ntiles = (op->rows + spl::kSkRows - 1) / spl::kSkRows;
+    d.chunk_begin = 0;
+    tg.g.n = 1;
+    tg.g.total_chunks = d.nch * d.ntiles;
+    if (!encode_operand(&tg.maps[0], *op, tokens, 1)) return MLLM_ERR_UNSUPPORTED;
+    return launch_spl_tma<1>(tg, part, tickets, tickets + spl::kMaxSkWarps, static_cast<cudaStream_t>(stream), 1);
+}
 
 size_t mllm_sizeof_sparse_operand(void) { return sizeof(mllm_sparse_operand); }
 

@@ -199,3 +199,19 @@ def test_sparse_linear_validation(M):
     assert _spl(M, [_op(M)], ws=0) == M.MLLM_ERR_WORKSPACE
     assert _spl(M, [_op(M)], wsb=M.mllm_sparse_linear_workspace_bytes() - 4) == M.MLLM_ERR_WORKSPACE
     assert _spl(M, [_op(M)], ws=0x100008) == M.MLLM_ERR_MISALIGNED
+
+
+def test_timeout_check_validation(M):
+    L = M.lib()
+    wsb = M.mllm_sparse_linear_workspace_bytes()
+
+    def call(op, tokens=4, ws=0x100000):
+        arr = (M.SparseOperand * 1)(op)
+        return L.mllm_sparse_linear_check_timeout(ctypes.cast(arr, ctypes.c_void_p), tokens, ws, wsb, 0)
+
+    # shapes the 2:4 tensor-copy pipeline does not take, rejected before any launch
+    assert call(_op(M, cols=64)) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=128), tokens=9) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=128, rows=0)) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=128), ws=0) == M.MLLM_ERR_WORKSPACE
+    assert call(_op(M, cols=128, x=0)) == M.MLLM_ERR_INVALID_ARG

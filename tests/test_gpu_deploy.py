@@ -16,8 +16,8 @@ import torch
 
 import _tol
 from sparsity_mask_sampling_b200 import (MatrixArray, MatrixBuffers, configs, inputs, mllm_hard_pack,
-                                         mllm_sparse_linear, mllm_sparse_linear_workspace_bytes,
-                                         sparse_linear_workspace)
+                                         mllm_sparse_linear, mllm_sparse_linear_check_timeout,
+                                         mllm_sparse_linear_workspace_bytes, sparse_linear_workspace)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -230,4 +230,25 @@ def test_full_stack_call_as_benchmarked(orc, ws):
         got = ys[i][:, sel_t].cpu().numpy().astype(np.float64)
         _tol.assert_spl_close(got, y_ref, absxw, c)
     assert all(bool(torch.isfinite(y).all()) for y in ys)
+    assert _tickets_clear(ws)
+
+
+def test_bounded_wait_reports_error_and_context_survives(orc):
+    """Failure detection of the copy pipeline: a launch whose first stage per warp is armed
+    but never filled makes every warp's bounded wait (1 s) run out; the call sets the
+    workspace's error word, returns, and the next call on a re-zeroed workspace is exact."""
+    import time
+
+    nm, tokens = (2, 4), 4
+    ws = sparse_linear_workspace(DEV)
+    o = Operand(orc, nm, 64, 256, tokens, seed=31)
+    t0 = time.time()
+    mllm_sparse_linear_check_timeout(o.op(), tokens, ws)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 60
+    assert int(ws[-16:-12].view(torch.int32).item()) != 0
+    ws.zero_()
+    mllm_sparse_linear([o.op()], nm, tokens, ws)
+    torch.cuda.synchronize()
+    o.check(orc)
     assert _tickets_clear(ws)
