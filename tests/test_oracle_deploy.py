@@ -95,3 +95,38 @@ def test_sparse_linear_homogeneous_and_empty(orc, n, m):
     np.testing.assert_array_equal(orc.sparse_linear(n, m, values, meta, x2),
                                   2.0 * orc.sparse_linear(n, m, values, meta, x))
     assert orc.sparse_linear(n, m, values, meta, x[:0]).shape == (0, rows_)
+
+
+@pytest.mark.parametrize("n,m", NM)
+def test_packed_input_generator_is_valid_pack(orc, n, m):
+    """inputs.packed_hard_mask (the serving benchmark's operands) encodes a valid candidate
+    per block exactly as hard_pack does: decoding it through the oracle's product with
+    one-hot activations keeps N nonzero positions per block, ascending, and round-trips
+    through hard_pack of the decoded dense matrix with logits favouring those candidates."""
+    import torch
+
+    from sparsity_mask_sampling_b200 import inputs
+
+    rows_, bpr = 6, 21
+    cols = bpr * m
+    v, mt = inputs.packed_hard_mask(rows_, cols, (n, m), seed=5)
+    values = v.view(torch.int16).numpy().view(np.uint16)
+    meta = mt.numpy().view(np.uint32 if m == 4 else np.uint16)
+    eye = np.zeros((cols, cols), np.uint16)
+    np.fill_diagonal(eye, 0x3F80)
+    dense = orc.sparse_linear(n, m, values, meta, eye).T          # [rows, cols] = W*
+    kept = (dense != 0).reshape(rows_, bpr, m)
+    assert (kept.sum(-1) == n).all()
+    S = _cands(n, m)
+    k = np.array([np.flatnonzero((S == kb).all(1))[0] for kb in kept.reshape(-1, m).astype(np.float64)])
+    pi = np.full((rows_ * bpr, orc.num_candidates(n, m)), -1.0, np.float32)
+    pi[np.arange(rows_ * bpr), k] = 1.0
+    W = np.zeros((rows_, cols), np.uint16)
+    W[dense != 0] = _bits_of(dense[dense != 0])
+    v2, m2, _ = orc.hard_pack(n, m, W, pi)
+    np.testing.assert_array_equal(v2, values)
+    np.testing.assert_array_equal(m2, meta)
+
+
+def _bits_of(vals):
+    return (np.asarray(vals, np.float32).view(np.uint32) >> 16).astype(np.uint16)
