@@ -7,18 +7,28 @@
 // call (decode). At that size the product is bound by reading the compressed weight from
 // HBM: 2:4 moves 2.25 bytes per weight pair instead of 4 dense.
 //
-// Mapping. A warp owns a tile of 16 rows; per chunk of 64 columns each thread (g = lane/4,
-// t = lane%4) loads, for rows g and g+8 of the tile, the compressed values and metadata of
-// columns 16t..16t+15 (one 16-byte vector and one 32-bit metadata word per row) and the same
-// 16 columns of x for token g (and g+8). It expands its blocks to dense bf16 pairs in
-// registers -- byte permutes whose selectors come from a small shared-memory table indexed by
-// the metadata -- and issues four bf16 mma.sync m16n8k16 steps. The order of the k-sum is
-// free, so the k-slots {2t, 2t+1, 2t+8, 2t+9} of step s are mapped to columns 16t+4s..16t+4s+3
-// of the chunk, for A and B alike: every thread then reads whole vectors of its own columns.
-// The kWarps warps of a CTA work on kMT row tiles, kKS = kWarps/kMT warps per tile taking
-// every kKS-th chunk; the partial tiles are added in shared memory in warp order, so the
-// result is deterministic. 4:8 uses the same mapping (a thread owns two 4:8 blocks per
-// chunk); hardware sparse tensor cores only take 2:4, so both patterns expand to dense tiles.
+// Four kernels, chosen per launch by the operands' widths (host side, mllm.cu):
+//   sparse_linear_tma_kernel  2:4, cols % 128 == 0 (every LLM shape): sparse tensor cores
+//                             (mma.sp) fed by tiled tensor copies; the fast path;
+//   sparse_linear_sp_kernel   2:4, cols % 32 == 0: the same arithmetic fed by cp.async;
+//   sparse_linear_sk_kernel   4:8 (no hardware sparse path) and 2:4 with cols % 16 == 0:
+//                             blocks expanded to dense bf16 in registers, dense mma.sync;
+//   sparse_linear_kernel      any cols % M == 0: the expansion with element-wise loads.
+// The last three split the launch's chunks evenly over all warps (stream-K); the first
+// kernel below splits whole row tiles over CTAs and is kept for the element-wise case.
+//
+// Mapping of the expansion kernels. A warp owns a tile of 16 rows; per chunk of 64 columns
+// each thread (g = lane/4, t = lane%4) loads, for rows g and g+8 of the tile, the compressed
+// values and metadata of columns 16t..16t+15 (one 16-byte vector and one 32-bit metadata word
+// per row) and the same 16 columns of x for token g (and g+8). It expands its blocks to dense
+// bf16 pairs in registers -- byte permutes whose selectors come from a small shared-memory
+// table indexed by the metadata -- and issues four bf16 mma.sync m16n8k16 steps. The order of
+// the k-sum is free, so the k-slots {2t, 2t+1, 2t+8, 2t+9} of step s are mapped to columns
+// 16t+4s..16t+4s+3 of the chunk, for A and B alike: every thread then reads whole vectors of
+// its own columns. In the tiled kernel the kWarps warps of a CTA work on kMT row tiles, kKS =
+// kWarps/kMT warps per tile taking every kKS-th chunk; the partial tiles are added in shared
+// memory in warp order, so the result is deterministic. 4:8 uses the same mapping (a thread
+// owns two 4:8 blocks per chunk).
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (type only; maps are encoded through the runtime's driver entry point)
@@ -355,7 +365,7 @@ template <int kNT> constexpr int sk_lane_bytes() { return 80 + 32 * kNT; }  // v
 template <int kNT> constexpr int sk_stages() { return kNT == 1 ? 6 : 5; }
 template <int kNT> constexpr int sk_smem_bytes() { return kSkWarps * sk_stages<kNT>() * 32 * sk_lane_bytes<kNT>(); }
 // workspace: two partial tiles per warp (2 m-tiles x kNT x 4 floats per lane, kNT <= 2),
-// then one ticket per warp, then an error word (set when a bulk copy never completes)
+// then one ticket per warp, then an error word (set when a tensor copy never completes)
 constexpr size_t kSkPartFloats = 2 * 2 * 4;
 constexpr size_t kSkWorkspaceBytes = (size_t)kMaxSkWarps * 2 * 32 * kSkPartFloats * sizeof(float) +
                                      (size_t)kMaxSkWarps * sizeof(unsigned int) + 16;  // + error word
