@@ -215,3 +215,29 @@ def test_prior_from_index_any_mask_and_no_prior(orc, n, m):
     p0, _ = orc.prior_init_from_index(n, m, np.arange(500), none, 3.0, 0.01, 9)
     r0, _, _ = orc.prior_init(n, m, np.zeros((500, m)), np.arange(500), 0.0, 0.01, 9)
     np.testing.assert_array_equal(p0, r0)
+
+
+@pytest.mark.parametrize("n,m", NM)
+def test_eq10_argmax_is_prior_exactly_when_the_bias_covers_the_draws(orc, n, m):
+    """Eq.10 with random draws: the prior candidate p is the argmax of pi = pi0 + alpha sigma
+    sim exactly when, for every other candidate j, pi0_j - pi0_p < alpha sigma (sim_p - sim_j)
+    (sigma the spread of the block's draws). Checked block by block against the oracle's own
+    argmax; with alpha = 3 the prior wins in most blocks (~95 % at 2:4, ~85 % at 4:8, where 16
+    candidates sit one similarity step below it), with alpha = 0 in about 1/C."""
+    C = orc.num_candidates(n, m)
+    nb = 4000
+    rng = np.random.default_rng(21)
+    W = rng.normal(0, 0.02, size=(nb, m))
+    gids = np.arange(nb)
+    p0, pidx, sim = orc.prior_init(n, m, W, gids, 0.0, 0.01, seed=3)
+    for alpha, lo, hi in ((3.0, 0.75, 1.0), (0.0, 0.5 / C, 2.0 / C)):
+        p, _, _ = orc.prior_init(n, m, W, gids, alpha, 0.01, seed=3)
+        k = orc.argmax(p.astype(np.float32), C)
+        sigma = p0.std(1)
+        sp = sim[np.arange(nb), pidx]
+        lhs = p0 - p0[np.arange(nb), pidx][:, None]
+        rhs = alpha * sigma[:, None] * (sp[:, None] - sim)
+        others = np.arange(C)[None, :] != pidx[:, None]
+        predicate = np.all((lhs < rhs) | ~others, axis=1)
+        np.testing.assert_array_equal(k == pidx, predicate)
+        assert lo <= predicate.mean() <= hi, (alpha, predicate.mean())
