@@ -301,6 +301,35 @@ def test_prior_random_parity(orc, nm):
     assert not c.mb.adam_m.any() and not c.mb.adam_v.any()
 
 
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_prior_random_argmax_predicate_on_device(orc, nm):
+    """Eq.10 on the device's own outputs, a property at any size: the draws pi0 (alpha = 0)
+    and the biased logits (alpha = 3) of the same seed give argmax = magnitude prior exactly
+    in the blocks where alpha sigma (sim_p - sim_j) exceeds every draw gap pi0_j - pi0_p; the
+    prior index and sim come from the oracle (they are exact functions of W)."""
+    c = Case(nm, 512, 256, seed=43, offset=7)
+    C = C_OF[nm]
+    mllm_prior_init([c.mb], nm, 0.0, 0.01, 99)
+    torch.cuda.synchronize()
+    p0 = c.mb.logits.cpu().numpy().astype(np.float64)
+    mllm_prior_init([c.mb], nm, 3.0, 0.01, 99)
+    torch.cuda.synchronize()
+    p3 = c.mb.logits.cpu().numpy()
+    _, pidx, sim = orc.prior_init(*nm, c.Wv, c.gids, 3.0, 0.0, 0)
+    nb = p0.shape[0]
+    k = orc.argmax(p3, C)
+    sigma = p0.std(1)
+    sp = sim[np.arange(nb), pidx]
+    lhs = p0 - p0[np.arange(nb), pidx][:, None]
+    rhs = 3.0 * sigma[:, None] * (sp[:, None] - sim)
+    others = np.arange(C)[None, :] != pidx[:, None]
+    margin = np.where(others, rhs - lhs, np.inf).min(1)
+    decided = np.abs(margin) > 1e-6 * np.abs(p3).max(1)   # away from fp32 rounding of the test
+    predicate = margin > 0
+    assert decided.mean() > 0.99
+    np.testing.assert_array_equal((k == pidx)[decided], predicate[decided])
+
+
 # ------------------------------------------------------------------------------ hard pack
 
 @pytest.mark.parametrize("nm,shapes", [((2, 4), [(64, 128), (3, 12), (5, 36), (7, 4)]),
