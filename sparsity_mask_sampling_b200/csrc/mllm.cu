@@ -767,9 +767,18 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
         }
         order.push_back(i);
     }
-    // operands with the longest rows first (the tiled kernel's first wave takes them)
-    std::stable_sort(order.begin(), order.end(),
-                     [&](int32_t a, int32_t b) { return ops[a].cols > ops[b].cols; });
+    // operands grouped by the kernel their width allows (so that a launch of 16 does not fall
+    // back for one odd operand), then the longest rows first (the tiled kernel's first wave
+    // takes them)
+    auto width_class = [&](int64_t cols) {
+        if (nm.m == 4 && cols % spl::kTmChunk == 0) return 0;
+        if (cols % 32 == 0) return 1;
+        return cols % 16 == 0 ? 2 : 3;
+    };
+    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
+        const int ca = width_class(ops[a].cols), cb = width_class(ops[b].cols);
+        return ca != cb ? ca < cb : ops[a].cols > ops[b].cols;
+    });
     const bool is24 = nm.m == 4, two = tokens > 8;
     for (size_t i0 = 0; i0 < order.size(); i0 += kMaxMats) {
         const size_t n = std::min<size_t>(kMaxMats, order.size() - i0);

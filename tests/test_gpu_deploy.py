@@ -252,3 +252,18 @@ def test_bounded_wait_reports_error_and_context_survives(orc):
     torch.cuda.synchronize()
     o.check(orc)
     assert _tickets_clear(ws)
+
+
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_many_operands_of_mixed_widths_in_one_call(orc, ws, nm):
+    """More than 16 operands whose widths take different kernels (multiples of 128, of 32, of
+    16, and odd multiples of M) in one call: the call groups them per kernel and per 16."""
+    m = nm[1]
+    widths = [256, 384, 96, 160, 48, 80, 4 * m * 3, 128, 1024, 32 * m, 16 * 3, 8 * m + m]
+    widths = [c for c in widths if c % m == 0]
+    ops = [Operand(orc, nm, 17 + 5 * i, widths[i % len(widths)], 6, seed=200 + i) for i in range(22)]
+    mllm_sparse_linear([o.op() for o in ops], nm, 6, ws)
+    torch.cuda.synchronize()
+    for o in ops:
+        o.check(orc)
+    assert _tickets_clear(ws)
