@@ -14,7 +14,7 @@ measured copy bandwidth.
                   [--impl reference]
   python bench.py --mode sparse_linear [--workload NAME] [--steps K --warmup W]
       (serving leg: the workload's matrices as packed hard masks, y = x W*^T per call for
-       1, 8 and 16 tokens, against dense cuBLAS; one JSON line)
+       1, 8, 16, 32 and 64 tokens, against dense cuBLAS; one JSON line)
 
 The training line also carries "extras": once-per-run calls timed over the whole stack
 (mask statistics, mask difference, candidate code, prior from a given mask) and the
@@ -382,7 +382,7 @@ def time_median(fn, reps=5):
     return float(np.median(out))
 
 
-def time_sparse_linear(stack, peak, token_counts=(1, 8, 16)):
+def time_sparse_linear(stack, peak, token_counts=(1, 8, 16, 32, 64)):
     """Serving the learned sparse network (s.3.2, inference): y = x W*^T for every matrix of
     the stack from its own packed hard mask (one mllm_sparse_linear call for all of them: a
     launch per 16 matrices), as
@@ -628,7 +628,7 @@ def reference_arm(args, w):
 def sparse_linear_arm(args, w):
     """--mode sparse_linear: serving the learned sparse network (s.3.2, inference). Every
     matrix of the workload as a packed hard-masked bf16 weight; one pass = y = x W*^T for all
-    of them (one mllm_sparse_linear call, a launch per 16 matrices) for T tokens, timed per
+    of them (one mllm_sparse_linear call, a launch per 16 matrices) for T = 1-64 tokens, timed per
     call with CUDA events (median of --steps calls after --warmup), beside the same products
     with dense bf16 weights through cuBLAS (torch.nn.functional.linear)."""
     import torch
@@ -665,7 +665,7 @@ def sparse_linear_arm(args, w):
         return float(np.median(out))
 
     res = {}
-    for T in (1, 8, 16):
+    for T in (1, 8, 16, 32, 64):
         xs = {c: torch.randn(T, c, device=dev, generator=gen).to(torch.bfloat16) for c in {c for _, c in shapes}}
         ys = [torch.empty(T, r, dtype=torch.float32, device=dev) for r, _ in shapes]
         arr = pkg.SparseOperandArray([(v, mt, xs[c], y) for (v, mt), (r, c), y in zip(packed, shapes, ys)])

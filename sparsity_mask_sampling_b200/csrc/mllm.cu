@@ -324,6 +324,16 @@ mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tic
     return cuda_status(cudaGetLastError());
 }
 
+template <int kNT>
+mllm_status launch_spl_tmab(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
+                            cudaStream_t st) {
+    auto fn = spl::sparse_linear_tmab_kernel<kNT>;
+    constexpr int smem = spl::tb_smem_bytes<kNT>(), threads = 32 * spl::kTbWarps;
+    const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kTbMaxCtas);
+    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err);
+    return cuda_status(cudaGetLastError());
+}
+
 template <int kN, bool kVec, int kNT>
 mllm_status launch_spl(const spl::OpGroup &g, cudaStream_t st) {
     auto fn = spl::sparse_linear_kernel<kN, kVec, kNT, kSplRowTiles, kSplDepth>;
@@ -391,6 +401,146 @@ mllm_status noalloc_scratch(void **out) {
     }
     *out = g_noalloc_ptr[dev];
     return MLLM_OK;
+}
+
+// The per-warp kernels for up to 16 tokens; every operand has rows > 0 and cols > 0.
+mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mllm_nm nm, int32_t tokens, float *part,
+                                unsigned int *tickets, unsigned int *err, cudaStream_t st) {
+    mllm_status s = MLLM_OK;
+    std::vector<int32_t> order(ops.size());
+    for (size_t i = 0; i < ops.size(); ++i) order[i] = (int32_t)i;
+    // operands grouped by the kernel their width allows (so that a launch of 16 does not fall
+    // back for one odd operand), then the longest rows first (the tiled kernel's first wave
+    // takes them)
+    auto width_class = [&](int64_t cols) {
+        if (nm.m == 4 && cols % spl::kTmChunk == 0) return 0;
+        if (cols % 32 == 0) return 1;
+        return cols % 16 == 0 ? 2 : 3;
+    };
+    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
+        const int ca = width_class(ops[a].cols), cb = width_class(ops[b].cols);
+        return ca != cb ? ca < cb : ops[a].cols > ops[b].cols;
+    });
+    const bool is24 = nm.m == 4, two = tokens > 8;
+    for (size_t i0 = 0; i0 < order.size(); i0 += kMaxMats) {
+        const size_t n = std::min<size_t>(kMaxMats, order.size() - i0);
+        bool vec = true, words = true, stages = true;
+        for (size_t k = 0; k < n; ++k) {
+            vec = vec && (ops[order[i0 + k]].cols % 16 == 0);
+            words = words && (ops[order[i0 + k]].cols % 32 == 0);
+            stages = stages && (ops[order[i0 + k]].cols % spl::kTmChunk == 0);
+        }
+        if (vec) {  // streamed kernels: the launch's chunks split evenly over all warps
+            // 2:4 in whole 128-column stages: tensor copies (falls back if a map cannot be
+            // encoded); other 2:4 with whole metadata words: sparse tensor cores via cp.async;
+            // else block expansion
+            const bool tma = is24 && stages;
+            auto group_of = [&](int64_t chunk) {
+                spl::SkGroup g{};
+                g.tokens = tokens;
+                int64_t acc = 0;
+                for (size_t k = 0; k < n; ++k) {
+                    const mllm_sparse_operand &o = ops[order[i0 + k]];
+                    spl::SkOp &d = g.d[k];
+                    d.vals = static_cast<const uint32_t *>(o.pack_values);
+                    d.meta = o.pack_meta;
+                    d.x = static_cast<const uint32_t *>(o.x);
+                    d.y = o.y;
+                    d.rows = o.rows;
+                    d.cols = o.cols;
+                    d.nch = (o.cols + chunk - 1) / chunk;
+                    d.ntiles = (o.rows + spl::kSkRows - 1) / spl::kSkRows;
+                    d.chunk_begin = acc;
+                    acc += d.nch * d.ntiles;
+                }
+                g.n = (int32_t)n;
+                g.total_chunks = acc;
+                return g;
+            };
+            if (tma) {
+                static thread_local spl::TmGroup tg;
+                tg.g = group_of(spl::kTmChunk);
+                bool ok = true;
+                for (size_t k = 0; k < n && ok; ++k) ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1);
+                if (ok) {
+                    s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
+                    if (s != MLLM_OK) return s;
+                    continue;
+                }
+            }
+            const spl::SkGroup g = group_of(spl::kChunk);
+            if (is24 && words) s = two ? launch_spl_sp<2>(g, part, tickets, st) : launch_spl_sp<1>(g, part, tickets, st);
+            else if (is24) s = two ? launch_spl_sk<2, 2>(g, part, tickets, st) : launch_spl_sk<2, 1>(g, part, tickets, st);
+            else s = two ? launch_spl_sk<4, 2>(g, part, tickets, st) : launch_spl_sk<4, 1>(g, part, tickets, st);
+            if (s != MLLM_OK) return s;
+            continue;
+        }
+        spl::OpGroup g{};
+        g.tokens = tokens;
+        int64_t acc = 0;
+        const int64_t rows_per_task = 16 * kSplRowTiles;
+        for (size_t k = 0; k < n; ++k) {
+            const mllm_sparse_operand &o = ops[order[i0 + k]];
+            spl::Op &d = g.d[k];
+            d.vals = static_cast<const uint32_t *>(o.pack_values);
+            d.meta = o.pack_meta;
+            d.x = static_cast<const uint32_t *>(o.x);
+            d.y = o.y;
+            d.rows = o.rows;
+            d.cols = o.cols;
+            d.task_begin = acc;
+            acc += (o.rows + rows_per_task - 1) / rows_per_task;
+        }
+        g.n = (int32_t)n;
+        g.total_tasks = acc;
+        if (is24) s = two ? launch_spl<2, false, 2>(g, st) : launch_spl<2, false, 1>(g, st);
+        else s = two ? launch_spl<4, false, 2>(g, st) : launch_spl<4, false, 1>(g, st);
+        if (s != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+
+// 17-64 tokens for 2:4 operands with cols % 128 == 0: the batched kernel, 16 operands per
+// launch (false if a tensor map cannot be encoded; nothing is launched then).
+bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, float *part,
+                           unsigned int *tickets, unsigned int *err, cudaStream_t st, mllm_status *status) {
+    const int nt = tokens > 32 ? 8 : 4;
+    for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
+        const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
+        static thread_local spl::TmGroup tg;
+        tg.g = spl::SkGroup{};
+        tg.g.tokens = tokens;
+        int64_t acc = 0;
+        for (size_t k = 0; k < n; ++k) {
+            const mllm_sparse_operand &o = ops[i0 + k];
+            spl::SkOp &d = tg.g.d[k];
+            d.vals = static_cast<const uint32_t *>(o.pack_values);
+            d.meta = o.pack_meta;
+            d.x = static_cast<const uint32_t *>(o.x);
+            d.y = o.y;
+            d.rows = o.rows;
+            d.cols = o.cols;
+            d.nch = o.cols / spl::kTmChunk;
+            d.ntiles = (o.rows + spl::kTbRows - 1) / spl::kTbRows;
+            d.chunk_begin = acc;
+            acc += d.nch * d.ntiles;
+            const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
+            if (!(encode_2d(&tg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
+                            spl::kTbRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  encode_2d(&tg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4,
+                            spl::kTbRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  encode_2d(&tg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
+                            (uint32_t)(8 * nt), CU_TENSOR_MAP_SWIZZLE_128B)))
+                return false;
+        }
+        tg.g.n = (int32_t)n;
+        tg.g.total_chunks = acc;
+        *status = nt == 8 ? launch_spl_tmab<8>(tg, part, tickets, err, st) : launch_spl_tmab<4>(tg, part, tickets, err, st);
+        if (*status != MLLM_OK) return true;
+    }
+    *status = MLLM_OK;
+    return true;
 }
 
 }  // namespace
@@ -754,10 +904,9 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
     if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *part = static_cast<float *>(workspace);
-    unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) +
-                                                             (size_t)spl::kMaxSkWarps * 2 * 32 * spl::kSkPartFloats * sizeof(float));
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + spl::kPartBytes);
     unsigned int *err = tickets + spl::kMaxSkWarps;
-    std::vector<int32_t> order;
+    std::vector<mllm_sparse_operand> act, batched;
     for (int32_t i = 0; i < n_ops; ++i) {
         if (ops[i].rows == 0) continue;
         if (ops[i].cols == 0) {  // y = 0
@@ -765,94 +914,22 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
             if (s != MLLM_OK) return s;
             continue;
         }
-        order.push_back(i);
+        if (tokens > spl::kMaxTileTokens && nm.m == 4 && ops[i].cols % spl::kTmChunk == 0) batched.push_back(ops[i]);
+        else act.push_back(ops[i]);
     }
-    // operands grouped by the kernel their width allows (so that a launch of 16 does not fall
-    // back for one odd operand), then the longest rows first (the tiled kernel's first wave
-    // takes them)
-    auto width_class = [&](int64_t cols) {
-        if (nm.m == 4 && cols % spl::kTmChunk == 0) return 0;
-        if (cols % 32 == 0) return 1;
-        return cols % 16 == 0 ? 2 : 3;
-    };
-    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
-        const int ca = width_class(ops[a].cols), cb = width_class(ops[b].cols);
-        return ca != cb ? ca < cb : ops[a].cols > ops[b].cols;
-    });
-    const bool is24 = nm.m == 4, two = tokens > 8;
-    for (size_t i0 = 0; i0 < order.size(); i0 += kMaxMats) {
-        const size_t n = std::min<size_t>(kMaxMats, order.size() - i0);
-        bool vec = true, words = true, stages = true;
-        for (size_t k = 0; k < n; ++k) {
-            vec = vec && (ops[order[i0 + k]].cols % 16 == 0);
-            words = words && (ops[order[i0 + k]].cols % 32 == 0);
-            stages = stages && (ops[order[i0 + k]].cols % spl::kTmChunk == 0);
+    if (!batched.empty() && !sparse_linear_batched(batched, tokens, part, tickets, err, st, &s))
+        act.insert(act.end(), batched.begin(), batched.end());  // maps not encodable: token groups
+    if (s != MLLM_OK) return s;
+    if (act.empty()) return MLLM_OK;
+    if (tokens <= spl::kMaxTileTokens) return sparse_linear_small(act, nm, tokens, part, tickets, err, st);
+    // more tokens than the per-warp kernels take: groups of 16 tokens (x and y rows offset)
+    for (int32_t t0 = 0; t0 < tokens; t0 += spl::kMaxTileTokens) {
+        std::vector<mllm_sparse_operand> grp = act;
+        for (mllm_sparse_operand &o : grp) {
+            o.x = static_cast<const char *>(o.x) + (size_t)t0 * (size_t)o.cols * 2;
+            o.y = o.y + (size_t)t0 * (size_t)o.rows;
         }
-        if (vec) {  // streamed kernels: the launch's chunks split evenly over all warps
-            // 2:4 in whole 128-column stages: tensor copies (falls back if a map cannot be
-            // encoded); other 2:4 with whole metadata words: sparse tensor cores via cp.async;
-            // else block expansion
-            const bool tma = is24 && stages;
-            auto group_of = [&](int64_t chunk) {
-                spl::SkGroup g{};
-                g.tokens = tokens;
-                int64_t acc = 0;
-                for (size_t k = 0; k < n; ++k) {
-                    const mllm_sparse_operand &o = ops[order[i0 + k]];
-                    spl::SkOp &d = g.d[k];
-                    d.vals = static_cast<const uint32_t *>(o.pack_values);
-                    d.meta = o.pack_meta;
-                    d.x = static_cast<const uint32_t *>(o.x);
-                    d.y = o.y;
-                    d.rows = o.rows;
-                    d.cols = o.cols;
-                    d.nch = (o.cols + chunk - 1) / chunk;
-                    d.ntiles = (o.rows + spl::kSkRows - 1) / spl::kSkRows;
-                    d.chunk_begin = acc;
-                    acc += d.nch * d.ntiles;
-                }
-                g.n = (int32_t)n;
-                g.total_chunks = acc;
-                return g;
-            };
-            if (tma) {
-                static thread_local spl::TmGroup tg;
-                tg.g = group_of(spl::kTmChunk);
-                bool ok = true;
-                for (size_t k = 0; k < n && ok; ++k) ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1);
-                if (ok) {
-                    s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
-                    if (s != MLLM_OK) return s;
-                    continue;
-                }
-            }
-            const spl::SkGroup g = group_of(spl::kChunk);
-            if (is24 && words) s = two ? launch_spl_sp<2>(g, part, tickets, st) : launch_spl_sp<1>(g, part, tickets, st);
-            else if (is24) s = two ? launch_spl_sk<2, 2>(g, part, tickets, st) : launch_spl_sk<2, 1>(g, part, tickets, st);
-            else s = two ? launch_spl_sk<4, 2>(g, part, tickets, st) : launch_spl_sk<4, 1>(g, part, tickets, st);
-            if (s != MLLM_OK) return s;
-            continue;
-        }
-        spl::OpGroup g{};
-        g.tokens = tokens;
-        int64_t acc = 0;
-        const int64_t rows_per_task = 16 * kSplRowTiles;
-        for (size_t k = 0; k < n; ++k) {
-            const mllm_sparse_operand &o = ops[order[i0 + k]];
-            spl::Op &d = g.d[k];
-            d.vals = static_cast<const uint32_t *>(o.pack_values);
-            d.meta = o.pack_meta;
-            d.x = static_cast<const uint32_t *>(o.x);
-            d.y = o.y;
-            d.rows = o.rows;
-            d.cols = o.cols;
-            d.task_begin = acc;
-            acc += (o.rows + rows_per_task - 1) / rows_per_task;
-        }
-        g.n = (int32_t)n;
-        g.total_tasks = acc;
-        if (is24) s = two ? launch_spl<2, false, 2>(g, st) : launch_spl<2, false, 1>(g, st);
-        else s = two ? launch_spl<4, false, 2>(g, st) : launch_spl<4, false, 1>(g, st);
+        s = sparse_linear_small(grp, nm, std::min<int32_t>(spl::kMaxTileTokens, tokens - t0), part, tickets, err, st);
         if (s != MLLM_OK) return s;
     }
     return MLLM_OK;
@@ -869,8 +946,7 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int3
     if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
     if (op->rows == 0 || op->cols == 0 || op->cols % spl::kTmChunk || tokens > 8) return MLLM_ERR_UNSUPPORTED;
     float *part = static_cast<float *>(workspace);
-    unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) +
-                                                             (size_t)spl::kMaxSkWarps * 2 * 32 * spl::kSkPartFloats * sizeof(float));
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + spl::kPartBytes);
     static thread_local spl::TmGroup tg;
     tg.g = spl::SkGroup{};
     tg.g.tokens = tokens;

@@ -184,7 +184,7 @@ def _op(M, **kw):
 def test_sparse_linear_validation(M):
     assert _spl(M, []) == M.MLLM_ERR_INVALID_ARG
     assert _spl(M, [_op(M)], nm=(1, 4)) == M.MLLM_ERR_UNSUPPORTED
-    for tokens in (0, -1, 17):
+    for tokens in (0, -1, 65):
         assert _spl(M, [_op(M)], tokens=tokens) == M.MLLM_ERR_INVALID_ARG, tokens
     assert _spl(M, [_op(M, cols=6)]) == M.MLLM_ERR_INVALID_ARG
     assert _spl(M, [_op(M, cols=12)], nm=(4, 8)) == M.MLLM_ERR_INVALID_ARG

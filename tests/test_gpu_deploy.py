@@ -267,3 +267,44 @@ def test_many_operands_of_mixed_widths_in_one_call(orc, ws, nm):
     for o in ops:
         o.check(orc)
     assert _tickets_clear(ws)
+
+
+@pytest.mark.parametrize("tokens", [17, 32, 33, 64])
+def test_batched_decode_2of4(orc, ws, tokens):
+    """17-64 tokens at 2:4: the batched kernel (128-row tiles shared by four warps) for widths
+    that are multiples of 128 (ragged rows, tiles cut between CTAs), token groups of 16 for
+    the others, in one call."""
+    nm = (2, 4)
+    shapes = [(45, 256), (130, 1024), (7, 128), (64, 96), (33, 40)]
+    ops = [Operand(orc, nm, r, c, tokens, seed=300 + i) for i, (r, c) in enumerate(shapes)]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
+    torch.cuda.synchronize()
+    for o in ops:
+        o.check(orc)
+    assert _tickets_clear(ws)
+
+
+@pytest.mark.parametrize("tokens", [24, 64])
+def test_batched_decode_4of8_token_groups(orc, ws, tokens):
+    nm = (4, 8)
+    ops = [Operand(orc, nm, r, c, tokens, seed=320 + i) for i, (r, c) in enumerate([(40, 256), (19, 72)])]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
+    torch.cuda.synchronize()
+    for o in ops:
+        o.check(orc)
+    assert _tickets_clear(ws)
+
+
+def test_batched_decode_full_size_64_tokens(orc, ws):
+    """q [4096, 4096], gate [11008, 4096], down [4096, 11008] at 64 tokens in one call."""
+    nm, tokens = (2, 4), 64
+    ops = [Operand(orc, nm, r, c, tokens, seed=340 + i, direct=True)
+           for i, (r, c) in enumerate([(4096, 4096), (11008, 4096), (4096, 11008)])]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    for o in ops:
+        sel = np.unique(np.concatenate([[0, o.rows - 1], rng.choice(o.rows, 14, replace=False)]))
+        o.check(orc, sel)
+        assert torch.isfinite(o.y).all()
+    assert _tickets_clear(ws)
