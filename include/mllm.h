@@ -273,7 +273,8 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
 size_t mllm_sparse_linear_workspace_bytes(void);
 
 /* Test of the bounded waits of mllm_sparse_linear's copy pipeline (no counterpart in the
- * paper): one launch of the 2:4 kernel for one operand (cols % 128 == 0, tokens <= 8) in which
+ * paper): one launch of the 2:4 kernel for one operand (cols % 128 == 0, 1 <= tokens <= 64:
+ * the per-warp kernel up to 16 tokens, the batched kernel above) in which
  * the first pipeline stage of every warp is armed but never filled, so that every warp's wait
  * runs out after its 1 s bound, sets the workspace's error word and returns. Takes about a
  * second; y is left invalid and the workspace must be zero-filled again afterwards. Nothing

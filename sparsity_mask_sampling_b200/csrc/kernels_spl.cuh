@@ -1119,7 +1119,7 @@ __device__ __forceinline__ void tb_store(const SkOp &d, int64_t tile, int warp, 
 template <int kNT>
 __global__ void __launch_bounds__(32 * kTbWarps, 1) sparse_linear_tmab_kernel(
     const __grid_constant__ TmGroup tg, float *__restrict__ part, unsigned int *__restrict__ tickets,
-    unsigned int *__restrict__ err) {
+    unsigned int *__restrict__ err, int arm_only_first) {
     constexpr int kD = kTbStages, kStage = tb_stage_bytes<kNT>();
     constexpr int kSlot = 32 * 2 * kNT * 4;  // floats of one warp's partial tile
     extern __shared__ unsigned char s_dyn_tb[];
@@ -1144,7 +1144,12 @@ __global__ void __launch_bounds__(32 * kTbWarps, 1) sparse_linear_tmab_kernel(
     __syncthreads();
     Cursor ld = sk_decode(grp, lo), cc = ld;
     for (int s = 0; s < kD && s < n; ++s) {
-        if (threadIdx.x == 0) tb_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+        if (threadIdx.x == 0) {
+            if (s == 0 && arm_only_first)  // test of the bounded wait: a stage nothing fills
+                mbar_arrive_tx(bar0, (unsigned)tb_stage_tx<kNT>());
+            else
+                tb_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+        }
         sk_advance(grp, ld);
     }
     bool rows_edge = (cc.tile + 1) * kTbRows > grp.d[cc.op].rows;

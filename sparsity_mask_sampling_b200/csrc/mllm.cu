@@ -326,11 +326,11 @@ mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tic
 
 template <int kNT>
 mllm_status launch_spl_tmab(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
-                            cudaStream_t st) {
+                            cudaStream_t st, int arm_only_first = 0) {
     auto fn = spl::sparse_linear_tmab_kernel<kNT>;
     constexpr int smem = spl::tb_smem_bytes<kNT>(), threads = 32 * spl::kTbWarps;
     const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kTbMaxCtas);
-    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err);
+    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err, arm_only_first);
     return cuda_status(cudaGetLastError());
 }
 
@@ -504,7 +504,8 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
 // 17-64 tokens for 2:4 operands with cols % 128 == 0: the batched kernel, 16 operands per
 // launch (false if a tensor map cannot be encoded; nothing is launched then).
 bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, float *part,
-                           unsigned int *tickets, unsigned int *err, cudaStream_t st, mllm_status *status) {
+                           unsigned int *tickets, unsigned int *err, cudaStream_t st, mllm_status *status,
+                           int arm_only_first = 0) {
     const int nt = tokens > 32 ? 8 : 4;
     for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
         const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
@@ -536,7 +537,8 @@ bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t 
         }
         tg.g.n = (int32_t)n;
         tg.g.total_chunks = acc;
-        *status = nt == 8 ? launch_spl_tmab<8>(tg, part, tickets, err, st) : launch_spl_tmab<4>(tg, part, tickets, err, st);
+        *status = nt == 8 ? launch_spl_tmab<8>(tg, part, tickets, err, st, arm_only_first)
+                          : launch_spl_tmab<4>(tg, part, tickets, err, st, arm_only_first);
         if (*status != MLLM_OK) return true;
     }
     *status = MLLM_OK;
@@ -944,9 +946,16 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int3
     if (s != MLLM_OK) return s;
     if (!workspace || workspace_bytes < spl::kSkWorkspaceBytes) return MLLM_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
-    if (op->rows == 0 || op->cols == 0 || op->cols % spl::kTmChunk || tokens > 8) return MLLM_ERR_UNSUPPORTED;
+    if (op->rows == 0 || op->cols == 0 || op->cols % spl::kTmChunk) return MLLM_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *part = static_cast<float *>(workspace);
     unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + spl::kPartBytes);
+    unsigned int *err = tickets + spl::kMaxSkWarps;
+    if (tokens > spl::kMaxTileTokens) {  // the batched kernel
+        const std::vector<mllm_sparse_operand> ops(1, *op);
+        if (!sparse_linear_batched(ops, tokens, part, tickets, err, st, &s, 1)) return MLLM_ERR_UNSUPPORTED;
+        return s;
+    }
     static thread_local spl::TmGroup tg;
     tg.g = spl::SkGroup{};
     tg.g.tokens = tokens;
@@ -962,8 +971,9 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int3
     d.chunk_begin = 0;
     tg.g.n = 1;
     tg.g.total_chunks = d.nch * d.ntiles;
-    if (!encode_operand(&tg.maps[0], *op, tokens, 1)) return MLLM_ERR_UNSUPPORTED;
-    return launch_spl_tma<1>(tg, part, tickets, tickets + spl::kMaxSkWarps, static_cast<cudaStream_t>(stream), 1);
+    const int nt = tokens > 8 ? 2 : 1;
+    if (!encode_operand(&tg.maps[0], *op, tokens, nt)) return MLLM_ERR_UNSUPPORTED;
+    return nt == 2 ? launch_spl_tma<2>(tg, part, tickets, err, st, 1) : launch_spl_tma<1>(tg, part, tickets, err, st, 1);
 }
 
 size_t mllm_sizeof_sparse_operand(void) { return sizeof(mllm_sparse_operand); }

@@ -211,7 +211,7 @@ def test_timeout_check_validation(M):
 
     # shapes the 2:4 tensor-copy pipeline does not take, rejected before any launch
     assert call(_op(M, cols=64)) == M.MLLM_ERR_UNSUPPORTED
-    assert call(_op(M, cols=128), tokens=9) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=128), tokens=65) == M.MLLM_ERR_INVALID_ARG
     assert call(_op(M, cols=128, rows=0)) == M.MLLM_ERR_UNSUPPORTED
     assert call(_op(M, cols=128), ws=0) == M.MLLM_ERR_WORKSPACE
     assert call(_op(M, cols=128, x=0)) == M.MLLM_ERR_INVALID_ARG

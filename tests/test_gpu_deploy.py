@@ -233,13 +233,15 @@ def test_full_stack_call_as_benchmarked(orc, ws):
     assert _tickets_clear(ws)
 
 
-def test_bounded_wait_reports_error_and_context_survives(orc):
-    """Failure detection of the copy pipeline: a launch whose first stage per warp is armed
-    but never filled makes every warp's bounded wait (1 s) run out; the call sets the
-    workspace's error word, returns, and the next call on a re-zeroed workspace is exact."""
+@pytest.mark.parametrize("tokens", [4, 40])
+def test_bounded_wait_reports_error_and_context_survives(orc, tokens):
+    """Failure detection of the copy pipelines (per-warp kernel at 4 tokens, batched kernel at
+    40): a launch whose first stage is armed but never filled makes the bounded waits (1 s) run
+    out; the call sets the workspace's error word, returns, and the next call on a re-zeroed
+    workspace is exact."""
     import time
 
-    nm, tokens = (2, 4), 4
+    nm = (2, 4)
     ws = sparse_linear_workspace(DEV)
     o = Operand(orc, nm, 64, 256, tokens, seed=31)
     t0 = time.time()
