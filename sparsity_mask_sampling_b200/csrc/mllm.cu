@@ -303,23 +303,28 @@ bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The three maps of a 2:4 operand for the TMA kernel (cols % 128 == 0).
-bool encode_operand(spl::TmMaps *mp, const mllm_sparse_operand &o, int32_t tokens, int kNT) {
+// The three maps of an operand for the TMA kernel (cols % 128 == 0).
+bool encode_operand(spl::TmMaps *mp, const mllm_sparse_operand &o, int32_t tokens, int kNT, int kN = 2) {
     const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
-    return encode_2d(&mp->vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64, 32,
+    const bool meta_ok =
+        kN == 2 ? encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4, 32,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)
+                : encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT16, o.pack_meta, cols / 8, rows, cols / 4, 16, 32,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
+    return meta_ok &&
+           encode_2d(&mp->vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64, 32,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-           encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4, 32,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) &&
            encode_2d(&mp->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
                      (uint32_t)(8 * kNT), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int kNT>
+template <int kNT, int kN = 2>
 mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
                            cudaStream_t st, int arm_only_first = 0) {
-    auto fn = spl::sparse_linear_tma_kernel<kNT>;
-    constexpr int smem = spl::tm_smem_bytes<kNT>(), threads = 32 * spl::tm_warps<kNT>();
-    const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::tm_warps<kNT>());
+    auto fn = spl::sparse_linear_tma_kernel<kNT, kN>;
+    constexpr int smem = spl::tm_smem_bytes<kNT, kN>(), threads = 32 * spl::tm_warps<kNT, kN>();
+    const int64_t grid =
+        grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::tm_warps<kNT, kN>());
     fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err, arm_only_first);
     return cuda_status(cudaGetLastError());
 }
@@ -413,7 +418,7 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
     // back for one odd operand), then the longest rows first (the tiled kernel's first wave
     // takes them)
     auto width_class = [&](int64_t cols) {
-        if (nm.m == 4 && cols % spl::kTmChunk == 0) return 0;
+        if (cols % spl::kTmChunk == 0) return 0;
         if (cols % 32 == 0) return 1;
         return cols % 16 == 0 ? 2 : 3;
     };
@@ -434,7 +439,7 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
             // 2:4 in whole 128-column stages: tensor copies (falls back if a map cannot be
             // encoded); other 2:4 with whole metadata words: sparse tensor cores via cp.async;
             // else block expansion
-            const bool tma = is24 && stages;
+            const bool tma = stages;
             auto group_of = [&](int64_t chunk) {
                 spl::SkGroup g{};
                 g.tokens = tokens;
@@ -461,9 +466,11 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
                 static thread_local spl::TmGroup tg;
                 tg.g = group_of(spl::kTmChunk);
                 bool ok = true;
-                for (size_t k = 0; k < n && ok; ++k) ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1);
+                for (size_t k = 0; k < n && ok; ++k)
+                    ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1, is24 ? 2 : 4);
                 if (ok) {
-                    s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
+                    if (is24) s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
+                    else s = two ? launch_spl_tma<2, 4>(tg, part, tickets, err, st) : launch_spl_tma<1, 4>(tg, part, tickets, err, st);
                     if (s != MLLM_OK) return s;
                     continue;
                 }
