@@ -310,3 +310,37 @@ def test_batched_decode_full_size_64_tokens(orc, ws):
         o.check(orc, sel)
         assert torch.isfinite(o.y).all()
     assert _tickets_clear(ws)
+
+
+def test_side_streams_and_concurrent_host_threads(orc):
+    """The stream argument is honoured (work on a side stream, then that stream's sync) and
+    two host threads can drive the library at once with their own workspaces and streams
+    (the binding releases the GIL; the library keeps per-thread launch state)."""
+    import threading
+
+    nm, tokens = (2, 4), 8
+    sets = [[Operand(orc, nm, r, c, tokens, seed=400 + 10 * k + i) for i, (r, c) in enumerate([(96, 512), (33, 256)])]
+            for k in range(2)]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    wss = [sparse_linear_workspace(DEV) for _ in range(2)]
+    torch.cuda.synchronize()  # inputs were placed on the default stream
+    errors = []
+
+    def run(k):
+        try:
+            for _ in range(20):
+                mllm_sparse_linear([o.op() for o in sets[k]], nm, tokens, wss[k], stream=streams[k].cuda_stream)
+            streams[k].synchronize()
+        except Exception as e:  # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(k,)) for k in range(2)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors
+    for k in range(2):
+        for o in sets[k]:
+            o.check(orc)
+        assert _tickets_clear(wss[k])
