@@ -141,33 +141,18 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Loads the slab of columns col0..col0+15 (col0 = 64*chunk + 16t). kVec: cols % 16 == 0, so
-// the slab lies wholly inside or wholly outside the row and every piece is one aligned
-// vector; otherwise each block and each x element is loaded on its own with a bounds check.
-template <int kN, bool kVec, int kNT>
+// Loads the slab of columns col0..col0+15 (col0 = 64*chunk + 16t) of rows r0, r1, one block
+// and one x element at a time with bounds checks (any cols % M == 0; zeros past the matrix).
+template <int kN, int kNT>
 __device__ __forceinline__ void load_slab(Slab<kNT> &s, const Op &d, int64_t r0, int64_t r1, int64_t col0,
-                                          int g, int t, int tokens) {
+                                          int g, int tokens) {
     const int64_t cols = d.cols, bpr = cols / (2 * kN);
     const int64_t wpr = cols >> 2;  // value words per row
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int64_t r = h ? r1 : r0;
-        s.v[h] = z;
-        s.m[h] = 0u;
-        if (r >= d.rows) continue;
-        if constexpr (kVec) {
-            if (col0 >= cols) continue;
-            s.v[h] = __ldcs(reinterpret_cast<const uint4 *>(d.vals + r * wpr + (col0 >> 2)));
-            if constexpr (kN == 2) {
-                const int64_t mw = (bpr + 7) >> 3;
-                s.m[h] = __ldcs(static_cast<const uint32_t *>(d.meta) + r * mw + (col0 >> 5)) >> (16 * (t & 1));
-            } else {
-                s.m[h] = __ldcs(reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(d.meta) + r * bpr +
-                                                                   (col0 >> 3)));
-            }
-        } else {
-            uint32_t v[4] = {0u, 0u, 0u, 0u}, m = 0u;
+        uint32_t v[4] = {0u, 0u, 0u, 0u}, m = 0u;
+        if (r < d.rows) {
             if constexpr (kN == 2) {
                 const int64_t mw = (bpr + 7) >> 3;
 #pragma unroll
@@ -190,33 +175,25 @@ __device__ __forceinline__ void load_slab(Slab<kNT> &s, const Op &d, int64_t r0,
                     }
                 }
             }
-            s.v[h] = make_uint4(v[0], v[1], v[2], v[3]);
-            s.m[h] = m;
         }
+        s.v[h] = make_uint4(v[0], v[1], v[2], v[3]);
+        s.m[h] = m;
     }
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
         const int tok = g + 8 * nt;
-        s.x[nt][0] = z;
-        s.x[nt][1] = z;
-        if (tok >= tokens) continue;
-        if constexpr (kVec) {
-            if (col0 >= cols) continue;
-            const uint4 *p = reinterpret_cast<const uint4 *>(d.x + tok * (cols >> 1) + (col0 >> 1));
-            s.x[nt][0] = __ldg(p);
-            s.x[nt][1] = __ldg(p + 1);
-        } else {
+        uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (tok < tokens) {
             const uint16_t *xr = reinterpret_cast<const uint16_t *>(d.x) + tok * cols;
-            uint32_t w[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int64_t c = col0 + 2 * j;
                 const uint32_t lo = c < cols ? xr[c] : 0u, hi = c + 1 < cols ? xr[c + 1] : 0u;
                 w[j] = lo | hi << 16;
             }
-            s.x[nt][0] = make_uint4(w[0], w[1], w[2], w[3]);
-            s.x[nt][1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
+        s.x[nt][0] = make_uint4(w[0], w[1], w[2], w[3]);
+        s.x[nt][1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
 }
 
@@ -267,7 +244,7 @@ __device__ __forceinline__ void mma_slab(const Slab<kNT> &s, const uint2 *tab24,
 
 // kNT n8 tiles of tokens (1: up to 8, 2: up to 16); kMT row tiles per CTA task; kDepth
 // slabs in flight per warp.
-template <int kN, bool kVec, int kNT, int kMT, int kDepth>
+template <int kN, int kNT, int kMT, int kDepth>
 __global__ void __launch_bounds__(kCtaThreads) sparse_linear_kernel(const __grid_constant__ OpGroup grp) {
     constexpr int kKS = kWarps / kMT;
     static_assert(kWarps % kMT == 0, "row tiles must divide the warps");
@@ -296,7 +273,7 @@ __global__ void __launch_bounds__(kCtaThreads) sparse_linear_kernel(const __grid
 #pragma unroll
         for (int i = 0; i < kDepth; ++i) {
             const int64_t c = ks + (int64_t)i * kKS;
-            if (c < nch) load_slab<kN, kVec, kNT>(ring[i], d, r0, r1, c * kChunk + 16 * t, g, t, grp.tokens);
+            if (c < nch) load_slab<kN, kNT>(ring[i], d, r0, r1, c * kChunk + 16 * t, g, grp.tokens);
         }
         for (int64_t c0 = ks; c0 < nch; c0 += (int64_t)kDepth * kKS) {
 #pragma unroll
@@ -306,7 +283,7 @@ __global__ void __launch_bounds__(kCtaThreads) sparse_linear_kernel(const __grid
                     mma_slab<kN, kNT>(ring[i], s_tab24, s_sel48, s_msk48, acc);
                     const int64_t cn = c + (int64_t)kDepth * kKS;
                     if (cn < nch)
-                        load_slab<kN, kVec, kNT>(ring[i], d, r0, r1, cn * kChunk + 16 * t, g, t, grp.tokens);
+                        load_slab<kN, kNT>(ring[i], d, r0, r1, cn * kChunk + 16 * t, g, grp.tokens);
                 }
             }
         }

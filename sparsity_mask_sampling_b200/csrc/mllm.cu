@@ -339,9 +339,9 @@ mllm_status launch_spl_tmab(const spl::TmGroup &g, float *part, unsigned int *ti
     return cuda_status(cudaGetLastError());
 }
 
-template <int kN, bool kVec, int kNT>
+template <int kN, int kNT>
 mllm_status launch_spl(const spl::OpGroup &g, cudaStream_t st) {
-    auto fn = spl::sparse_linear_kernel<kN, kVec, kNT, kSplRowTiles, kSplDepth>;
+    auto fn = spl::sparse_linear_kernel<kN, kNT, kSplRowTiles, kSplDepth>;
     const int64_t grid = grid_for((const void *)fn, spl::kCtaThreads, 0, g.total_tasks, INT32_MAX);
     fn<<<(unsigned)grid, spl::kCtaThreads, 0, st>>>(g);
     return cuda_status(cudaGetLastError());
@@ -500,8 +500,8 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
         }
         g.n = (int32_t)n;
         g.total_tasks = acc;
-        if (is24) s = two ? launch_spl<2, false, 2>(g, st) : launch_spl<2, false, 1>(g, st);
-        else s = two ? launch_spl<4, false, 2>(g, st) : launch_spl<4, false, 1>(g, st);
+        if (is24) s = two ? launch_spl<2, 2>(g, st) : launch_spl<2, 1>(g, st);
+        else s = two ? launch_spl<4, 2>(g, st) : launch_spl<4, 1>(g, st);
         if (s != MLLM_OK) return s;
     }
     return MLLM_OK;
