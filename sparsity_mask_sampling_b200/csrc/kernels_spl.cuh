@@ -7,7 +7,9 @@
 // call (decode). At that size the product is bound by reading the compressed weight from
 // HBM: 2:4 moves 2.25 bytes per weight pair instead of 4 dense.
 //
-// Four kernels, chosen per launch by the operands' widths (host side, mllm.cu):
+// Up to 16 tokens, four kernels, chosen per launch by the operands' widths (host side, mllm.cu);
+// 17-64 tokens of 2:4 operands with cols % 128 == 0 run on the fifth-generation tensor cores
+// (kernels_umma.cuh), other operands as groups of 16 tokens:
 //   sparse_linear_tma_kernel  2:4, cols % 128 == 0 (every LLM shape): sparse tensor cores
 //                             (mma.sp) fed by tiled tensor copies; the fast path;
 //   sparse_linear_sp_kernel   2:4, cols % 32 == 0: the same arithmetic fed by cp.async;
@@ -345,12 +347,13 @@ template <int kNT> constexpr int sk_smem_bytes() { return kSkWarps * sk_stages<k
 // workspace: two partial tiles per warp (2 m-tiles x kNT x 4 floats per lane, kNT <= 2),
 // then one ticket per warp, then an error word (set when a tensor copy never completes)
 constexpr size_t kSkPartFloats = 2 * 2 * 4;
-// batched kernel (17-64 tokens, below): two partial tiles of 128 rows x 64 tokens per CTA
-constexpr int kTbWarps = 4, kTbRows = 32 * kTbWarps, kTbMaxCtas = 320;
-constexpr size_t kTbPartFloats = (size_t)kTbWarps * 32 * 2 * 8 * 4;  // per CTA and slot
+// batched kernel (17-64 tokens, kernels_umma.cuh): two partial tiles of 128 rows x 64 tokens
+// per CTA, at most kBatchMaxCtas CTAs
+constexpr int kBatchRows = 128, kBatchMaxCtas = 320;
+constexpr size_t kBatchPartFloats = (size_t)kBatchRows * kMaxTokens;  // per CTA and slot
 constexpr size_t kSpPartBytes = (size_t)kMaxSkWarps * 2 * 32 * kSkPartFloats * sizeof(float);
-constexpr size_t kTbPartBytes = (size_t)kTbMaxCtas * 2 * kTbPartFloats * sizeof(float);
-constexpr size_t kPartBytes = kSpPartBytes > kTbPartBytes ? kSpPartBytes : kTbPartBytes;
+constexpr size_t kBatchPartBytes = (size_t)kBatchMaxCtas * 2 * kBatchPartFloats * sizeof(float);
+constexpr size_t kPartBytes = kSpPartBytes > kBatchPartBytes ? kSpPartBytes : kBatchPartBytes;
 constexpr size_t kSkWorkspaceBytes = kPartBytes + (size_t)kMaxSkWarps * sizeof(unsigned int) + 16;  // + error word
 
 struct SkOp {
@@ -1055,212 +1058,6 @@ __global__ void __launch_bounds__(32 * tm_warps<kNT, kN>(), 1) sparse_linear_tma
         if (f + 1 < n) {
             sk_advance(grp, cc);
             rows_edge = (cc.tile + 1) * kSkRows > grp.d[cc.op].rows;
-        }
-    }
-}
-
-// ------------------------------------------------------------------ 2:4, batched decode
-
-// 17-64 tokens (2:4, cols % 128 == 0). A warp's private x stages would not fit, so the four
-// warps of a CTA share one pipeline over 128-row tiles: per 128-column stage one thread issues
-// the 128 x 64 box of values, the 128 x 4 box of metadata words and two 8kNT x 64 boxes of x;
-// each warp multiplies its 32 rows with all kNT token tiles. The chunk sequence is split
-// evenly over CTAs (stream-K at CTA granularity); a tile cut between CTAs leaves per-warp
-// partial tiles in the workspace, and the last CTA to arrive (a ticket per tile) adds them
-// in CTA order. Block barriers guard the refill of a stage; waits are bounded as above.
-
-template <int kNT> constexpr int tb_xbox_bytes() { return 8 * kNT * 128; }
-template <int kNT> constexpr int tb_stage_tx() { return kTbRows * 128 + 2 * tb_xbox_bytes<kNT>() + kTbRows * 16; }
-template <int kNT> constexpr int tb_stage_bytes() { return (tb_stage_tx<kNT>() + 1023) / 1024 * 1024; }
-constexpr int kTbStages = 3;
-template <int kNT> constexpr int tb_smem_bytes() { return kTbStages * tb_stage_bytes<kNT>() + 1024; }
-
-template <int kNT>
-__device__ __forceinline__ void tb_issue(const TmGroup &tg, const Cursor &c, unsigned stage, unsigned bar) {
-    const TmMaps &mp = tg.maps[c.op];
-    const int j = (int)c.j, row0 = (int)(c.tile * kTbRows);
-    mbar_arrive_tx(bar, (unsigned)tb_stage_tx<kNT>());
-    tma_load_2d(stage, &mp.vals, 64 * j, row0, bar);
-    tma_load_2d(stage + kTbRows * 128, &mp.x, 128 * j, 0, bar);
-    tma_load_2d(stage + kTbRows * 128 + tb_xbox_bytes<kNT>(), &mp.x, 128 * j + 64, 0, bar);
-    tma_load_2d(stage + kTbRows * 128 + 2 * tb_xbox_bytes<kNT>(), &mp.meta, 4 * j, row0, bar);
-}
-
-template <int kNT, bool kEdge>
-__device__ __forceinline__ void tb_compute(const unsigned char *st, int warp, int lane, int g, int t,
-                                           float (&acc)[2][kNT][4]) {
-    const unsigned char *xs = st + kTbRows * 128;
-    const unsigned char *meta = xs + 2 * tb_xbox_bytes<kNT>();
-    const uint32_t esel = (t & 1) ? 0x7632u : 0x5410u;
-    const int ar = 32 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
-    const int br = lane & 7;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const unsigned char *xb = xs + (w >> 1) * tb_xbox_bytes<kNT>();
-        uint32_t a[2][4], e[2];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            const int r = ar + 16 * mt, c = 2 * w + (lane >> 4);
-            ldmatrix_x4(a[mt], st + r * 128 + ((c ^ (r & 7)) << 4));
-            const unsigned char *ra = meta + (32 * warp + 16 * mt + g) * 16 + 4 * w;
-            uint32_t mg = lds32(ra), mg8 = lds32(ra + 8 * 16);
-            if constexpr (kEdge) {
-                mg = mg ? mg : 0x44444444u;
-                mg8 = mg8 ? mg8 : 0x44444444u;
-            }
-            e[mt] = __byte_perm(mg, mg8, esel);
-        }
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-            uint32_t b[4];
-            const int r = br + 8 * nt, c = 4 * (w & 1) + (lane >> 3);
-            ldmatrix_x4(b, xb + r * 128 + ((c ^ (r & 7)) << 4));
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) mma_sp_bf16_16832(acc[mt][nt], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b, e[mt]);
-        }
-    }
-}
-
-template <int kNT>
-__device__ __forceinline__ void tb_store(const SkOp &d, int64_t tile, int warp, const float (&acc)[2][kNT][4], int g,
-                                         int t, int tokens) {
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t r = tile * kTbRows + 32 * warp + 16 * mt + 8 * h + g;
-                if (r >= d.rows) continue;
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tok = 8 * nt + 2 * t + e;
-                    if (tok < tokens) d.y[tok * d.rows + r] = acc[mt][nt][2 * h + e];
-                }
-            }
-}
-
-template <int kNT>
-__global__ void __launch_bounds__(32 * kTbWarps, 1) sparse_linear_tmab_kernel(
-    const __grid_constant__ TmGroup tg, float *__restrict__ part, unsigned int *__restrict__ tickets,
-    unsigned int *__restrict__ err, int arm_only_first) {
-    constexpr int kD = kTbStages, kStage = tb_stage_bytes<kNT>();
-    constexpr int kSlot = 32 * 2 * kNT * 4;  // floats of one warp's partial tile
-    extern __shared__ unsigned char s_dyn_tb[];
-    __shared__ __align__(8) unsigned long long s_bar[kD];
-    __shared__ int s_last;
-    const SkGroup &grp = tg.g;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int64_t total = grp.total_chunks;
-    const int64_t G = imin64((int64_t)gridDim.x, total), cta = blockIdx.x;
-    if (cta >= G) return;  // the whole CTA: no barrier is left waiting
-    const int64_t lo = cta * total / G, hi = (cta + 1) * total / G;
-    const int n = (int)(hi - lo);
-    const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_tb);
-    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
-    unsigned char *ring = s_dyn_tb + pad;
-    const unsigned ring_s = dyn_s + pad;
-    const unsigned bar0 = (unsigned)__cvta_generic_to_shared(&s_bar[0]);
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kD; ++s) mbar_init(bar0 + 8 * s, 1u);
-        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    }
-    __syncthreads();
-    Cursor ld = sk_decode(grp, lo), cc = ld;
-    for (int s = 0; s < kD && s < n; ++s) {
-        if (threadIdx.x == 0) {
-            if (s == 0 && arm_only_first)  // test of the bounded wait: a stage nothing fills
-                mbar_arrive_tx(bar0, (unsigned)tb_stage_tx<kNT>());
-            else
-                tb_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
-        }
-        sk_advance(grp, ld);
-    }
-    bool rows_edge = (cc.tile + 1) * kTbRows > grp.d[cc.op].rows;
-    float acc[2][kNT][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
-    unsigned phase = 0u;
-    int s = 0;
-    for (int f = 0; f < n; ++f) {
-        const bool ok = tm_wait(bar0 + 8 * s, (phase >> s) & 1u);
-        if (__syncthreads_or(!ok)) {
-            // a copy never landed: flag it, give the other stages a bounded time, leave
-            if (threadIdx.x == 0) atomicOr(err, 1u);
-            for (int q = 1; q < kD && f + q < n; ++q) {
-                const int sq = (s + q) % kD;
-                tm_wait(bar0 + 8 * sq, (phase >> sq) & 1u);
-            }
-            return;
-        }
-        phase ^= 1u << s;
-        const unsigned char *st = ring + s * kStage;
-        if (rows_edge) tb_compute<kNT, true>(st, warp, lane, g, t, acc);
-        else tb_compute<kNT, false>(st, warp, lane, g, t, acc);
-        __syncthreads();  // every warp has read the stage
-        if (f + kD < n) {
-            if (threadIdx.x == 0) {
-                fence_proxy_async();
-                tb_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
-            }
-            sk_advance(grp, ld);
-        }
-        s = (s + 1 == kD) ? 0 : s + 1;
-        const SkOp &d = grp.d[cc.op];
-        if (cc.j == d.nch - 1 || f == n - 1) {  // end of this CTA's piece of the tile
-            const int64_t a = d.chunk_begin + cc.tile * d.nch, b = a + d.nch;
-            const int64_t c1 = ((a + 1) * G - 1) / total, c2 = (b * G - 1) / total;
-            if (c1 == c2) {
-                tb_store<kNT>(d, cc.tile, warp, acc, g, t, grp.tokens);
-            } else {
-                const int64_t lo1 = c1 * total / G;
-                const int slot = (cta == c1 && lo1 < a) ? 1 : 0;
-                float4 *mine = reinterpret_cast<float4 *>(part + ((cta * 2 + slot) * kTbWarps + warp) * kSlot) + lane * (2 * kNT);
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int nt = 0; nt < kNT; ++nt)
-                        __stcg(mine + mt * kNT + nt, make_float4(acc[mt][nt][0], acc[mt][nt][1], acc[mt][nt][2], acc[mt][nt][3]));
-                __threadfence();
-                __syncthreads();
-                if (threadIdx.x == 0) s_last = (atomicAdd(tickets + c1, 1u) == (unsigned int)(c2 - c1));
-                __syncthreads();
-                if (s_last) {
-                    __threadfence();
-                    float sum[2][kNT][4];
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                        for (int nt = 0; nt < kNT; ++nt) sum[mt][nt][0] = sum[mt][nt][1] = sum[mt][nt][2] = sum[mt][nt][3] = 0.f;
-                    for (int64_t q = c1; q <= c2; ++q) {
-                        const int sid = (q == c1 && lo1 < a) ? 1 : 0;
-                        const float4 *p = reinterpret_cast<const float4 *>(part + ((q * 2 + sid) * kTbWarps + warp) * kSlot) + lane * (2 * kNT);
-#pragma unroll
-                        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                            for (int nt = 0; nt < kNT; ++nt) {
-                                const float4 v = __ldcg(p + mt * kNT + nt);
-                                sum[mt][nt][0] += v.x;
-                                sum[mt][nt][1] += v.y;
-                                sum[mt][nt][2] += v.z;
-                                sum[mt][nt][3] += v.w;
-                            }
-                    }
-                    tb_store<kNT>(d, cc.tile, warp, sum, g, t, grp.tokens);
-                    __syncthreads();
-                    if (threadIdx.x == 0) tickets[c1] = 0u;
-                }
-            }
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < kNT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
-        }
-        if (f + 1 < n) {
-            sk_advance(grp, cc);
-            rows_edge = (cc.tile + 1) * kTbRows > grp.d[cc.op].rows;
         }
     }
 }

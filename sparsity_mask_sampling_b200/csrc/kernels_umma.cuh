@@ -1,0 +1,357 @@
+// kernels_umma.cuh -- batched decode (17-64 tokens) of the 2:4 serving product on the
+// fifth-generation tensor cores: tcgen05.mma.sp with operands in shared memory, sparsity
+// metadata and accumulators in tensor memory.
+//
+// The product is y = x W*^T with W* = W (.) M* in the form mllm_hard_pack writes (two kept
+// bf16 values and one 4-bit position code per block of four weights); MaskLLM serves the
+// masked network this way after training (paper-graph-ui summary of arXiv 2409.17481, s.3.2
+// "Information flow at inference"). It is an HBM stream: every compressed weight is read once.
+//
+// Tile: 128 rows of W* (the MMA's M) x all kNTok tokens (its N, tokens rounded up to 16) x
+// 128 columns per pipeline stage (four MMAs of K = 32). Per stage the tensor memory
+// accelerator lands, on one mbarrier, the 128 x 64 box of compressed values and two kNTok x 64
+// boxes of x (both with the 128-byte swizzle, the K-major layout the MMA's shared-memory
+// descriptors name) and the 128 x 4 box of metadata words. Roles in a CTA of five warps:
+//   warp 4       the copy warp: refills a stage when the MMAs that read it have completed
+//                (their tcgen05.commit arrives on the stage's "empty" barrier);
+//   warps 0-3    per stage, each thread builds the metadata word of its tensor-memory lane
+//                and stores it with tcgen05.st; after a barrier thread 0 issues the four
+//                MMAs and commits them; at the end of a tile each warp reads its 32 rows of
+//                the accumulator with tcgen05.ld and stores y (or a partial tile).
+// Metadata in tensor memory, M = 128, 16-bit types, one column per MMA (the address an MMA
+// names is even; the descriptor's selector bits stay 0): lane
+// L = (m % 8) + 8 h + 16 (m / 16) holds, for row m (m % 16 < 8) and K half h, the four
+// 4-bit codes of blocks 4h .. 4h+3 in its low 16 bits and those of row m + 8 in its high 16
+// bits -- the same per-quad distribution as the metadata of mma.sp m16n8k32, so a byte permute
+// of the packed words of rows m and m + 8 gives it. Rows past the matrix are zero-filled by
+// the copy engine; their zero words are replaced by a valid code (values there are zero).
+// Tensor memory per CTA: 128 columns (accumulator at 0 .. kNTok-1, the metadata of MMA j of
+// stage s at column 64 + 8s + 2j). A CTA takes more than a fifth of an SM's shared memory, so at most
+// four are resident and their 512 columns fit; the allocation never waits on another CTA.
+//
+// Work split: the 128-column chunks of all tiles of all operands of a launch form one sequence,
+// split into equal contiguous ranges over the CTAs (stream-K). A tile cut between CTAs leaves
+// one partial tile per piece in the workspace (slot 1 for a CTA's last piece when that CTA
+// also had earlier work, else slot 0); the last CTA to arrive (a ticket per tile, keyed by the
+// tile's first CTA) adds the pieces in CTA order and stores y, so results are deterministic. Every wait is
+// bounded (kTmWaitNs); a timeout sets the workspace's error word, the CTA stops issuing,
+// waits (bounded) for the copies and MMAs it has in flight, frees its tensor memory and exits.
+// arm_only_first (tests only) arms stage 0 without filling it, so that this path runs.
+#pragma once
+
+#include "kernels_spl.cuh"
+
+namespace mllm {
+namespace spl {
+
+constexpr int kUmRows = kBatchRows;          // MMA M: rows of a tile (128)
+constexpr int kUmStages = 3;
+constexpr int kUmThreads = 160;              // 4 MMA/epilogue warps + the copy warp
+constexpr int kUmCtasPerSm = 2;              // resident CTAs the grid is sized for
+constexpr unsigned kUmTmemCols = 128;
+constexpr unsigned kUmMetaCol = 64;
+constexpr size_t kUmPartFloats = kBatchPartFloats;  // one partial tile: 128 rows x 64 tokens
+
+template <int kNTok> constexpr int um_xbox_bytes() { return kNTok * 128; }
+template <int kNTok> constexpr int um_stage_tx() { return kUmRows * 128 + 2 * um_xbox_bytes<kNTok>() + kUmRows * 16; }
+template <int kNTok> constexpr int um_stage_bytes() { return (um_stage_tx<kNTok>() + 1023) / 1024 * 1024; }
+template <int kNTok> constexpr int um_smem_bytes() { return kUmStages * um_stage_bytes<kNTok>() + 1024; }
+
+// Instruction descriptor of kind::f16: sparse, f32 accumulator, bf16 A and B (both
+// K-major), N = kNTok, M = 128.
+template <int kNTok> constexpr uint32_t um_idesc() {
+    return (1u << 2) | (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNTok >> 3) << 17) |
+           ((uint32_t)(kUmRows >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t um_desc(unsigned saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void umma_sp(unsigned d_tmem, uint64_t adesc, uint64_t bdesc, unsigned e_tmem,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %5, 0;\n"
+        " tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(unsigned bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// The metadata of a stage's four MMAs, one per even column (taddr, +2, +4, +6).
+__device__ __forceinline__ void tmem_st_meta(unsigned taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %5, %2, %5, %3, %5, %4, %5};\n" ::"r"(taddr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(0u)
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// 16 consecutive accumulator columns of this thread's lane; the wait names the registers so
+// that no use is scheduled before the data is there.
+__device__ __forceinline__ void tmem_ld16(unsigned taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Barrier of the four MMA/epilogue warps (id 1), OR-reducing a predicate.
+__device__ __forceinline__ bool um_bar_or(bool p) {
+    unsigned r;
+    asm volatile(
+        "{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n barrier.cta.red.or.pred b, 1, 128, a;\n"
+        " selp.u32 %0, 1, 0, b;\n}\n"
+        : "=r"(r)
+        : "r"((unsigned)p)
+        : "memory");
+    return r != 0u;
+}
+__device__ __forceinline__ void um_bar() { asm volatile("barrier.cta.sync 1, 128;\n" ::: "memory"); }
+
+// Warp-uniform bounded wait that also gives up once *abort is set.
+__device__ __forceinline__ bool um_wait(unsigned bar, unsigned parity, const volatile int *abort) {
+    const unsigned long long t0 = __shfl_sync(0xFFFFFFFFu, globaltimer_ns(), 0);
+    while (true) {
+        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+        if (__any_sync(0xFFFFFFFFu, *abort != 0)) return false;
+        if (__shfl_sync(0xFFFFFFFFu, globaltimer_ns(), 0) - t0 > kTmWaitNs) return false;
+    }
+}
+
+template <int kNTok>
+__device__ __forceinline__ void um_issue(const TmGroup &tg, const Cursor &c, unsigned stage, unsigned bar) {
+    const TmMaps &mp = tg.maps[c.op];
+    const int j = (int)c.j, row0 = (int)(c.tile * kUmRows);
+    mbar_arrive_tx(bar, (unsigned)um_stage_tx<kNTok>());
+    tma_load_2d(stage, &mp.vals, 64 * j, row0, bar);
+    tma_load_2d(stage + kUmRows * 128, &mp.x, 128 * j, 0, bar);
+    tma_load_2d(stage + kUmRows * 128 + um_xbox_bytes<kNTok>(), &mp.x, 128 * j + 64, 0, bar);
+    tma_load_2d(stage + kUmRows * 128 + 2 * um_xbox_bytes<kNTok>(), &mp.meta, 4 * j, row0, bar);
+}
+
+template <int kNTok>
+__device__ __forceinline__ void um_store(const SkOp &d, int64_t tile, int warp, int lane, const float (&v)[kNTok],
+                                         int tokens) {
+    const int64_t r = tile * kUmRows + 32 * warp + lane;
+    if (r >= d.rows) return;
+#pragma unroll
+    for (int tok = 0; tok < kNTok; ++tok)
+        if (tok < tokens) d.y[tok * d.rows + r] = v[tok];
+}
+
+template <int kNTok>
+__global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_kernel(const __grid_constant__ TmGroup tg,
+                                                                          float *__restrict__ part,
+                                                                          unsigned int *__restrict__ tickets,
+                                                                          unsigned int *__restrict__ err,
+                                                                          int arm_only_first) {
+    static_assert(kNTok % 16 == 0 && kNTok >= 16 && kNTok <= kMaxTokens, "N of an M = 128 MMA");
+    static_assert(um_smem_bytes<kNTok>() * 5 > 233472, "at most four CTAs per SM: 4 x 128 TMEM columns");
+    static_assert(kUmCtasPerSm * (um_smem_bytes<kNTok>() + 2048) <= 233472, "kUmCtasPerSm CTAs fit an SM");
+    constexpr int kD = kUmStages, kStage = um_stage_bytes<kNTok>();
+    constexpr uint32_t kIdesc = um_idesc<kNTok>();
+    extern __shared__ unsigned char s_dyn_um[];
+    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_acc;
+    __shared__ unsigned s_tmem;
+    __shared__ volatile int s_abort;
+    __shared__ int s_last;
+    const SkGroup &grp = tg.g;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t total = grp.total_chunks;
+    const int64_t G = imin64((int64_t)gridDim.x, total), cta = blockIdx.x;
+    if (cta >= G) return;  // the whole CTA, before any barrier or allocation
+    const int64_t lo = cta * total / G, hi = (cta + 1) * total / G;
+    const int n = (int)(hi - lo);
+    const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_um);
+    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
+    const unsigned char *ring = s_dyn_um + pad;
+    const unsigned ring_s = dyn_s + pad;
+    const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
+    const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
+    const unsigned accb = (unsigned)__cvta_generic_to_shared(&s_acc);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kD; ++s) {
+            mbar_init(full0 + 8 * s, 1u);
+            mbar_init(empty0 + 8 * s, 1u);
+        }
+        mbar_init(accb, 1u);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 0) {
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(&s_tmem);
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst),
+                     "r"(kUmTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const unsigned tbase = s_tmem;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ copy warp
+        Cursor ld = sk_decode(grp, lo);
+        int issued = 0;
+        for (int f = 0; f < n; ++f) {
+            const int s = f % kD;
+            if (f >= kD && !um_wait(empty0 + 8 * s, ((f / kD) - 1) & 1, &s_abort)) {
+                if (lane == 0 && !s_abort) {
+                    atomicOr(err, 1u);
+                    s_abort = 1;
+                }
+                break;
+            }
+            if (lane == 0) {
+                if (f == 0 && arm_only_first)  // test of the bounded wait: a stage nothing fills
+                    mbar_arrive_tx(full0, (unsigned)um_stage_tx<kNTok>());
+                else {
+                    fence_proxy_async();
+                    um_issue<kNTok>(tg, ld, ring_s + s * kStage, full0 + 8 * s);
+                }
+            }
+            ++issued;
+            sk_advance(grp, ld);
+        }
+        // every copy this warp started has landed (bounded) before the CTA's memory is released
+        for (int s = 0; s < kD && s < issued; ++s) {
+            const int last = s + ((issued - 1 - s) / kD) * kD;  // the latest fill of stage s
+            tm_wait(full0 + 8 * s, (last / kD) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ MMA / epilogue warps
+        const unsigned tlane = tbase + ((unsigned)(32 * warp) << 16);
+        const int h = (lane >> 3) & 1;
+        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of the tile
+        const uint32_t esel = h ? 0x7632u : 0x5410u;
+        Cursor cc = sk_decode(grp, lo);
+        bool fresh = true;       // next MMA starts a tile piece (overwrites the accumulator)
+        unsigned acc_phase = 0u;
+        int mma_commits = 0;     // stages whose MMAs thread 0 has committed
+        bool failed = false;
+        for (int f = 0; f < n; ++f) {
+            const int s = f % kD;
+            const bool ok = um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort);
+            if (ok) {
+                tc_fence_after();
+                const unsigned char *meta = ring + s * kStage + kUmRows * 128 + 2 * um_xbox_bytes<kNTok>();
+                const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
+                const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
+                uint32_t e[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    e[j] = __byte_perm(a4[j] ? a4[j] : 0x44444444u, b4[j] ? b4[j] : 0x44444444u, esel);
+                tmem_st_meta(tlane + kUmMetaCol + 8 * s, e[0], e[1], e[2], e[3]);
+            }
+            tc_fence_before();
+            if (um_bar_or(!ok)) {
+                failed = true;
+                break;
+            }
+            const SkOp &d = grp.d[cc.op];
+            const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+                const unsigned st = ring_s + s * kStage;
+                const uint64_t a0 = um_desc(st), b0 = um_desc(st + kUmRows * 128),
+                               b1 = um_desc(st + kUmRows * 128 + um_xbox_bytes<kNTok>());
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    umma_sp(tbase, a0 + (uint64_t)(2 * j), ((j >> 1) ? b1 : b0) + (uint64_t)(4 * (j & 1)),
+                            tbase + kUmMetaCol + 8 * s + 2 * j, kIdesc, (fresh && j == 0) ? 0u : 1u);
+                umma_commit(empty0 + 8 * s);
+                if (piece_end) umma_commit(accb);
+            }
+            ++mma_commits;
+            fresh = false;
+            if (piece_end) {
+                // ---------------------------------------------------- epilogue of a tile piece
+                const bool acc_ok = um_wait(accb, acc_phase, &s_abort);
+                acc_phase ^= 1u;
+                if (um_bar_or(!acc_ok)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float v[kNTok];
+#pragma unroll
+                for (int q = 0; q < kNTok / 16; ++q) tmem_ld16(tlane + 16 * q, v + 16 * q);
+                tc_fence_before();
+                const int64_t a = d.chunk_begin + cc.tile * d.nch, b = a + d.nch;
+                const int64_t c1 = ((a + 1) * G - 1) / total, c2 = (b * G - 1) / total;
+                if (c1 == c2) {
+                    um_store<kNTok>(d, cc.tile, warp, lane, v, grp.tokens);
+                } else {
+                    const int64_t lo1 = c1 * total / G;
+                    const int slot = (cta == c1 && lo1 < a) ? 1 : 0;
+                    float *mine = part + (size_t)(cta * 2 + slot) * kUmPartFloats + 32 * warp + lane;
+#pragma unroll
+                    for (int tok = 0; tok < kNTok; ++tok) __stcg(mine + tok * kUmRows, v[tok]);
+                    __threadfence();
+                    um_bar();
+                    if (threadIdx.x == 0) s_last = (atomicAdd(tickets + c1, 1u) == (unsigned int)(c2 - c1));
+                    um_bar();
+                    if (s_last) {
+                        __threadfence();
+                        float sum[kNTok];
+#pragma unroll
+                        for (int tok = 0; tok < kNTok; ++tok) sum[tok] = 0.f;
+                        for (int64_t q = c1; q <= c2; ++q) {
+                            const int sid = (q == c1 && lo1 < a) ? 1 : 0;
+                            const float *p = part + (size_t)(q * 2 + sid) * kUmPartFloats + 32 * warp + lane;
+#pragma unroll
+                            for (int tok = 0; tok < kNTok; ++tok) sum[tok] += __ldcg(p + tok * kUmRows);
+                        }
+                        um_store<kNTok>(d, cc.tile, warp, lane, sum, grp.tokens);
+                        um_bar();
+                        if (threadIdx.x == 0) tickets[c1] = 0u;
+                    }
+                }
+                fresh = true;
+            }
+            sk_advance(grp, cc);
+        }
+        if (failed) {
+            if (threadIdx.x == 0 && !s_abort) {
+                atomicOr(err, 1u);
+                s_abort = 1;
+            }
+            // MMAs already issued complete before the tensor memory is released: wait (bounded)
+            // for the commit of the latest issued stage
+            if (mma_commits > 0) {
+                const int f = mma_commits - 1;
+                tm_wait(empty0 + 8 * (f % kD), (f / kD) & 1);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kUmTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace spl
+}  // namespace mllm

@@ -13,6 +13,7 @@
 #include "kernels_4of8.cuh"
 #include "kernels_diag.cuh"
 #include "kernels_spl.cuh"
+#include "kernels_umma.cuh"
 
 namespace mllm {
 namespace {
@@ -329,13 +330,19 @@ mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tic
     return cuda_status(cudaGetLastError());
 }
 
-template <int kNT>
-mllm_status launch_spl_tmab(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
+template <int kNTok>
+mllm_status launch_spl_umma(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
                             cudaStream_t st, int arm_only_first = 0) {
-    auto fn = spl::sparse_linear_tmab_kernel<kNT>;
-    constexpr int smem = spl::tb_smem_bytes<kNT>(), threads = 32 * spl::kTbWarps;
-    const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kTbMaxCtas);
-    fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err, arm_only_first);
+    auto fn = spl::sparse_linear_umma_kernel<kNTok>;
+    constexpr int smem = spl::um_smem_bytes<kNTok>();
+    // The occupancy query reports one resident CTA per SM for this kernel, although its launch
+    // bounds and shared memory admit kUmCtasPerSm (and a profile of a launch shows that
+    // limit); the grid is sized from those limits. No CTA waits on another, so any grid is correct.
+    int dev = 0;
+    cudaGetDevice(&dev);
+    resident_ctas(dev, (const void *)fn, spl::kUmThreads, smem);  // sets the dynamic shared-memory limit
+    const int64_t grid = std::min<int64_t>((int64_t)sm_count(dev) * spl::kUmCtasPerSm, spl::kBatchMaxCtas);
+    fn<<<(unsigned)grid, spl::kUmThreads, smem, st>>>(g, part, tickets, err, arm_only_first);
     return cuda_status(cudaGetLastError());
 }
 
@@ -508,12 +515,12 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
 }
 
 
-// 17-64 tokens for 2:4 operands with cols % 128 == 0: the batched kernel, 16 operands per
+// 17-64 tokens for 2:4 operands with cols % 128 == 0: the tensor-memory kernel, 16 operands per
 // launch (false if a tensor map cannot be encoded; nothing is launched then).
 bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, float *part,
                            unsigned int *tickets, unsigned int *err, cudaStream_t st, mllm_status *status,
                            int arm_only_first = 0) {
-    const int nt = tokens > 32 ? 8 : 4;
+    const int ntok = (tokens + 15) / 16 * 16 < 32 ? 32 : (tokens + 15) / 16 * 16;  // the MMA's N
     for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
         const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
         static thread_local spl::TmGroup tg;
@@ -530,22 +537,23 @@ bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t 
             d.rows = o.rows;
             d.cols = o.cols;
             d.nch = o.cols / spl::kTmChunk;
-            d.ntiles = (o.rows + spl::kTbRows - 1) / spl::kTbRows;
+            d.ntiles = (o.rows + spl::kUmRows - 1) / spl::kUmRows;
             d.chunk_begin = acc;
             acc += d.nch * d.ntiles;
             const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
             if (!(encode_2d(&tg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
-                            spl::kTbRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
                   encode_2d(&tg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4,
-                            spl::kTbRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   encode_2d(&tg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
-                            (uint32_t)(8 * nt), CU_TENSOR_MAP_SWIZZLE_128B)))
+                            (uint32_t)ntok, CU_TENSOR_MAP_SWIZZLE_128B)))
                 return false;
         }
         tg.g.n = (int32_t)n;
         tg.g.total_chunks = acc;
-        *status = nt == 8 ? launch_spl_tmab<8>(tg, part, tickets, err, st, arm_only_first)
-                          : launch_spl_tmab<4>(tg, part, tickets, err, st, arm_only_first);
+        *status = ntok == 64   ? launch_spl_umma<64>(tg, part, tickets, err, st, arm_only_first)
+                  : ntok == 48 ? launch_spl_umma<48>(tg, part, tickets, err, st, arm_only_first)
+                               : launch_spl_umma<32>(tg, part, tickets, err, st, arm_only_first);
         if (*status != MLLM_OK) return true;
     }
     *status = MLLM_OK;
@@ -958,7 +966,7 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int3
     float *part = static_cast<float *>(workspace);
     unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + spl::kPartBytes);
     unsigned int *err = tickets + spl::kMaxSkWarps;
-    if (tokens > spl::kMaxTileTokens) {  // the batched kernel
+    if (tokens > spl::kMaxTileTokens) {  // the tensor-memory kernel
         const std::vector<mllm_sparse_operand> ops(1, *op);
         if (!sparse_linear_batched(ops, tokens, part, tickets, err, st, &s, 1)) return MLLM_ERR_UNSUPPORTED;
         return s;

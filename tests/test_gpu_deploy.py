@@ -271,11 +271,11 @@ def test_many_operands_of_mixed_widths_in_one_call(orc, ws, nm):
     assert _tickets_clear(ws)
 
 
-@pytest.mark.parametrize("tokens", [17, 32, 33, 64])
+@pytest.mark.parametrize("tokens", [17, 32, 33, 48, 49, 64])
 def test_batched_decode_2of4(orc, ws, tokens):
-    """17-64 tokens at 2:4: the batched kernel (128-row tiles shared by four warps) for widths
-    that are multiples of 128 (ragged rows, tiles cut between CTAs), token groups of 16 for
-    the others, in one call."""
+    """17-64 tokens at 2:4: the tensor-memory kernel (128-row tiles, N = tokens rounded up to
+    16, at least 32) for widths that are multiples of 128 (ragged rows, tiles cut between
+    CTAs), token groups of 16 for the others, in one call."""
     nm = (2, 4)
     shapes = [(45, 256), (130, 1024), (7, 128), (64, 96), (33, 40)]
     ops = [Operand(orc, nm, r, c, tokens, seed=300 + i) for i, (r, c) in enumerate(shapes)]
@@ -312,13 +312,15 @@ def test_batched_decode_full_size_64_tokens(orc, ws):
     assert _tickets_clear(ws)
 
 
-def test_side_streams_and_concurrent_host_threads(orc):
+@pytest.mark.parametrize("tokens", [8, 40])
+def test_side_streams_and_concurrent_host_threads(orc, tokens):
     """The stream argument is honoured (work on a side stream, then that stream's sync) and
     two host threads can drive the library at once with their own workspaces and streams
-    (the binding releases the GIL; the library keeps per-thread launch state)."""
+    (the binding releases the GIL; the library keeps per-thread launch state). At 40 tokens
+    the two streams' tensor-memory kernels share SMs (each CTA holds 128 TMEM columns)."""
     import threading
 
-    nm, tokens = (2, 4), 8
+    nm = (2, 4)
     sets = [[Operand(orc, nm, r, c, tokens, seed=400 + 10 * k + i) for i, (r, c) in enumerate([(96, 512), (33, 256)])]
             for k in range(2)]
     streams = [torch.cuda.Stream() for _ in range(2)]
