@@ -274,11 +274,13 @@ size_t mllm_sparse_linear_workspace_bytes(void);
 
 /* Test of the bounded waits of mllm_sparse_linear's copy pipeline (no counterpart in the
  * paper): one launch of the 2:4 kernel for one operand (cols % 128 == 0, 1 <= tokens <= 64:
- * the per-warp kernel up to 16 tokens, the batched kernel above) in which
- * the first pipeline stage of every warp is armed but never filled, so that every warp's wait
- * runs out after its 1 s bound, sets the workspace's error word and returns. Takes about a
- * second; y is left invalid and the workspace must be zero-filled again afterwards. Nothing
- * faults and the context stays usable. MLLM_ERR_UNSUPPORTED for other shapes. */
+ * the per-warp kernel up to 16 tokens, the tensor-memory kernel above) in which
+ * the first pipeline stage of every warp (per-warp kernel) or CTA (tensor-memory kernel) is
+ * armed but never filled, so that its wait runs out after the 1 s bound, sets the workspace's
+ * error word and the kernel winds down (bounded waits for what it has in flight) and returns.
+ * Takes one to two seconds; y is left invalid and the workspace must be zero-filled again
+ * afterwards. Nothing faults and the context stays usable. MLLM_ERR_UNSUPPORTED for other
+ * shapes. */
 mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int32_t tokens, void *workspace,
                                              size_t workspace_bytes, void *stream);
 
