@@ -178,10 +178,11 @@ def test_llama_shapes_full_size_sampled_rows(orc, ws, nm, tokens):
 
 
 @pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
-@pytest.mark.parametrize("tokens", [3, 16])
+@pytest.mark.parametrize("tokens", [3, 16, 40])
 def test_tiles_cut_into_many_pieces(orc, ws, nm, tokens):
-    """Few rows and long rows: each 32-row tile is cut between hundreds of warps, whose
-    partial tiles the last arriving warp adds; repeated calls reuse the workspace."""
+    """Few rows and long rows: each tile is cut between hundreds of warps (32-row tiles) or,
+    at 40 tokens and 2:4, between 128 CTAs (one 128-row tile of 128 chunks), whose partial
+    tiles the last arriving warp or CTA adds; repeated calls reuse the workspace."""
     o = Operand(orc, nm, 40, 16384, tokens, seed=77, direct=True)
     for _ in range(2):
         mllm_sparse_linear([o.op()], nm, tokens, ws)
@@ -256,15 +257,18 @@ def test_bounded_wait_reports_error_and_context_survives(orc, tokens):
     assert _tickets_clear(ws)
 
 
-@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
-def test_many_operands_of_mixed_widths_in_one_call(orc, ws, nm):
+@pytest.mark.parametrize("nm,tokens", [((2, 4), 6), ((4, 8), 6), ((2, 4), 40)])
+def test_many_operands_of_mixed_widths_in_one_call(orc, ws, nm, tokens):
     """More than 16 operands whose widths take different kernels (multiples of 128, of 32, of
-    16, and odd multiples of M) in one call: the call groups them per kernel and per 16."""
+    16, and odd multiples of M) in one call: the call groups them per kernel and per 16 (at
+    40 tokens: 2:4 widths that are multiples of 128 in two tensor-memory launches, the
+    others in groups of 16 tokens)."""
     m = nm[1]
     widths = [256, 384, 96, 160, 48, 80, 4 * m * 3, 128, 1024, 32 * m, 16 * 3, 8 * m + m]
     widths = [c for c in widths if c % m == 0]
-    ops = [Operand(orc, nm, 17 + 5 * i, widths[i % len(widths)], 6, seed=200 + i) for i in range(22)]
-    mllm_sparse_linear([o.op() for o in ops], nm, 6, ws)
+    n_ops = 22 if tokens <= 16 else 40
+    ops = [Operand(orc, nm, 17 + 5 * i, widths[i % len(widths)], tokens, seed=200 + i) for i in range(n_ops)]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
     torch.cuda.synchronize()
     for o in ops:
         o.check(orc)
