@@ -273,16 +273,16 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
 size_t mllm_sparse_linear_workspace_bytes(void);
 
 /* Test of the bounded waits of mllm_sparse_linear's copy pipeline (no counterpart in the
- * paper): one launch of the 2:4 kernel for one operand (cols % 128 == 0, 1 <= tokens <= 64:
- * the per-warp kernel up to 16 tokens, the tensor-memory kernel above) in which
+ * paper): one launch of the 2:4 or 4:8 kernel for one operand (cols % 128 == 0,
+ * 1 <= tokens <= 64: the per-warp kernel up to 16 tokens, the tensor-memory kernel above) in which
  * the first pipeline stage of every warp (per-warp kernel) or CTA (tensor-memory kernel) is
  * armed but never filled, so that its wait runs out after the 1 s bound, sets the workspace's
  * error word and the kernel winds down (bounded waits for what it has in flight) and returns.
  * Takes one to two seconds; y is left invalid and the workspace must be zero-filled again
  * afterwards. Nothing faults and the context stays usable. MLLM_ERR_UNSUPPORTED for other
  * shapes. */
-mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int32_t tokens, void *workspace,
-                                             size_t workspace_bytes, void *stream);
+mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, mllm_nm nm, int32_t tokens,
+                                             void *workspace, size_t workspace_bytes, void *stream);
 
 /* The Gumbel noise itself, for inspection and statistical tests: g_out[i*C + c] = noise
  * of candidate c of the block with global id gids[i] at (seed, step). gids and g_out are

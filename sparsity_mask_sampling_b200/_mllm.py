@@ -110,7 +110,7 @@ _SIGS = {
     "mllm_noise_table": (ctypes.c_int, [_P, _P]),
     "mllm_sparse_linear": (ctypes.c_int, [_P, ctypes.c_int32, NM, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "mllm_sparse_linear_workspace_bytes": (ctypes.c_size_t, []),
-    "mllm_sparse_linear_check_timeout": (ctypes.c_int, [_P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "mllm_sparse_linear_check_timeout": (ctypes.c_int, [_P, NM, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "mllm_sizeof_sparse_operand": (ctypes.c_size_t, []),
     "mllm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mllm_last_cuda_error": (ctypes.c_int32, []),
@@ -382,11 +382,11 @@ def mllm_sparse_linear(ops, nm, tokens: int, workspace: torch.Tensor, stream=Non
            "mllm_sparse_linear")
 
 
-def mllm_sparse_linear_check_timeout(op, tokens: int, workspace: torch.Tensor, stream=None):
+def mllm_sparse_linear_check_timeout(op, nm, tokens: int, workspace: torch.Tensor, stream=None):
     """One (pack_values, pack_meta, x, y) operand through the timeout test of the copy
     pipeline (see include/mllm.h): the call's error word ends nonzero."""
     a = SparseOperandArray([op])
-    _check(lib().mllm_sparse_linear_check_timeout(a.ptr, int(tokens), _ptr(workspace),
+    _check(lib().mllm_sparse_linear_check_timeout(a.ptr, _nm(nm), int(tokens), _ptr(workspace),
                                                   workspace.numel() * workspace.element_size(), _stream(stream)),
            "mllm_sparse_linear_check_timeout")
 

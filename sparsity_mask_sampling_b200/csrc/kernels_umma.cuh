@@ -114,18 +114,20 @@ __device__ __forceinline__ void tmem_ld16(unsigned taddr, float *v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Barrier of the four MMA/epilogue warps (id 1), OR-reducing a predicate.
+// Barrier (id 1) of the kCount threads that are not the copy warp, OR-reducing a predicate.
+template <int kCount>
 __device__ __forceinline__ bool um_bar_or(bool p) {
     unsigned r;
     asm volatile(
-        "{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n barrier.cta.red.or.pred b, 1, 128, a;\n"
+        "{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n barrier.cta.red.or.pred b, 1, %2, a;\n"
         " selp.u32 %0, 1, 0, b;\n}\n"
         : "=r"(r)
-        : "r"((unsigned)p)
+        : "r"((unsigned)p), "n"(kCount)
         : "memory");
     return r != 0u;
 }
-__device__ __forceinline__ void um_bar() { asm volatile("barrier.cta.sync 1, 128;\n" ::: "memory"); }
+template <int kCount>
+__device__ __forceinline__ void um_bar() { asm volatile("barrier.cta.sync 1, %0;\n" ::"n"(kCount) : "memory"); }
 
 // Warp-uniform bounded wait that also gives up once *abort is set.
 __device__ __forceinline__ bool um_wait(unsigned bar, unsigned parity, const volatile int *abort) {
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                 tmem_st_meta(tlane + kUmMetaCol + 8 * s, e[0], e[1], e[2], e[3]);
             }
             tc_fence_before();
-            if (um_bar_or(!ok)) {
+            if (um_bar_or<128>(!ok)) {
                 failed = true;
                 break;
             }
@@ -288,7 +290,7 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                 // ---------------------------------------------------- epilogue of a tile piece
                 const bool acc_ok = um_wait(accb, acc_phase, &s_abort);
                 acc_phase ^= 1u;
-                if (um_bar_or(!acc_ok)) {
+                if (um_bar_or<128>(!acc_ok)) {
                     failed = true;
                     break;
                 }
@@ -308,9 +310,9 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
 #pragma unroll
                     for (int tok = 0; tok < kNTok; ++tok) __stcg(mine + tok * kUmRows, v[tok]);
                     __threadfence();
-                    um_bar();
+                    um_bar<128>();
                     if (threadIdx.x == 0) s_last = (atomicAdd(tickets + c1, 1u) == (unsigned int)(c2 - c1));
-                    um_bar();
+                    um_bar<128>();
                     if (s_last) {
                         __threadfence();
                         float sum[kNTok];
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                             for (int tok = 0; tok < kNTok; ++tok) sum[tok] += __ldcg(p + tok * kUmRows);
                         }
                         um_store<kNTok>(d, cc.tile, warp, lane, sum, grp.tokens);
-                        um_bar();
+                        um_bar<128>();
                         if (threadIdx.x == 0) tickets[c1] = 0u;
                     }
                 }
@@ -352,6 +354,339 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                      : "memory");
     }
 }
+
+// ------------------------------------------------------------------ 4:8 on the dense tensor cores
+//
+// 4:8 has no hardware sparse mode. Per 128-column stage, kU8Warps warps expand the compressed
+// tile into a dense 128 x 128 bf16 tile in shared memory (two 128 x 64 atoms in the K-major,
+// 128-byte swizzled layout of the MMA's descriptors), and one thread issues eight dense
+// tcgen05.mma (kind::f16, K = 16) on it. A 4:8 block (four kept values in position order and
+// the code p0 | p1 << 3 | p2 << 6 | p3 << 9) expands into exactly one 16-byte chunk of eight
+// bf16. Word i of the chunk (positions 2i, 2i+1) is prmt(prmt(v0v1, 0, A[p0p1].i), v2v3,
+// B[p2p3].i): table A places the first pair and zero-fills, table B places the second pair
+// and keeps the rest (u8_table_entry). Each CTA builds both 64-entry tables in shared memory,
+// 16 interleaved copies each, so that the lookups of a half-warp never share a bank. Thread t
+// expands row t % 128, part t / 128 of the stage (64 / kU8Warps blocks, within one atom).
+// A stage: values 16 KB | x, two kNTok x 64 boxes | metadata, 128 rows x 16 codes (4 KB) |
+// the dense tile (32 KB). One CTA per SM with three stages; tensor memory holds only the
+// accumulator (64 columns). Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 and the
+// token slice w / 4. Copy warp, bounded waits, work split and partial tiles as above.
+
+constexpr int kU8Warps = 16;         // expansion / epilogue warps (a multiple of 4, at most 16)
+constexpr int kU8Threads = 32 * kU8Warps + 32;  // + the copy warp
+constexpr int kU8NStep = 8 * (kU8Warps / 4) > 16 ? 8 * (kU8Warps / 4) : 16;  // N is a multiple of this
+constexpr int kU8Stages = 3;
+constexpr unsigned kU8TmemCols = 64;
+
+template <int kNTok> constexpr int u8_tx() { return kUmRows * 128 + 2 * um_xbox_bytes<kNTok>() + kUmRows * 32; }
+template <int kNTok> constexpr int u8_a_off() { return (u8_tx<kNTok>() + 1023) / 1024 * 1024; }
+template <int kNTok> constexpr int u8_stage_bytes() { return u8_a_off<kNTok>() + 2 * kUmRows * 128; }
+constexpr int kU8TabCopies = 16;     // one copy per lane of a half-warp: conflict-free 8-byte lookups
+constexpr int kU8TabBytes = 2 * 64 * kU8TabCopies * 8;  // tables A and B
+template <int kNTok> constexpr int u8_smem_bytes() { return kU8Stages * u8_stage_bytes<kNTok>() + 1024 + kU8TabBytes; }
+
+// Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
+// N = kNTok, M = 128.
+template <int kNTok> constexpr uint32_t u8_idesc() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNTok >> 3) << 17) | ((uint32_t)(kUmRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_dense(unsigned d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 8 consecutive accumulator columns of this thread's lane (see tmem_ld16).
+__device__ __forceinline__ void tmem_ld8(unsigned taddr, float *v) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Entry q = pa | pb << 3 of expansion table A (second = false) or B (second = true): the
+// byte-permute selectors of the four words of a dense chunk (x: words 0, 1; y: words 2, 3)
+// for a value pair at positions pa < pb. Table A places the first pair (v0 v1, bytes 0-3 of
+// the permute's sources) and takes zero bytes (4-7, a zero operand) elsewhere; table B places
+// the second pair (v2 v3, bytes 4-7) over that result and keeps its bytes (0-3) elsewhere.
+__device__ __forceinline__ uint2 u8_table_entry(int q, bool second) {
+    const int pa = q & 7, pb = q >> 3;
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t sel = 0u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int pos = 2 * i + h;
+            const uint32_t base = second ? 4u : 0u, other = second ? 2u * h : 4u;
+            const uint32_t b0 = pos == pa ? base : (pos == pb ? base + 2u : other);  // first source byte
+            sel |= (b0 | (b0 + 1u) << 4) << (8 * h);
+        }
+        w[i] = sel;
+    }
+    return make_uint2(w[0] | w[1] << 16, w[2] | w[3] << 16);
+}
+
+template <int kNTok>
+__device__ __forceinline__ void u8_issue(const TmGroup &tg, const Cursor &c, unsigned stage, unsigned bar) {
+    const TmMaps &mp = tg.maps[c.op];
+    const int j = (int)c.j, row0 = (int)(c.tile * kUmRows);
+    mbar_arrive_tx(bar, (unsigned)u8_tx<kNTok>());
+    tma_load_2d(stage, &mp.vals, 64 * j, row0, bar);
+    tma_load_2d(stage + kUmRows * 128, &mp.x, 128 * j, 0, bar);
+    tma_load_2d(stage + kUmRows * 128 + um_xbox_bytes<kNTok>(), &mp.x, 128 * j + 64, 0, bar);
+    tma_load_2d(stage + kUmRows * 128 + 2 * um_xbox_bytes<kNTok>(), &mp.meta, 16 * j, row0, bar);
+}
+
+// Row r, part pt of a stage (kBlk = 64 / kU8Warps blocks from block kBlk pt; a part lies in
+// one atom) into the dense tile.
+__device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char *dense, const uint2 *tab_a,
+                                          const uint2 *tab_b, int meta_off, int r, int pt) {
+    constexpr int kBlk = 64 / kU8Warps;  // 8 or 4 blocks, 2 per 16-byte value chunk
+    const int b0 = kBlk * pt, atom = b0 >> 3;
+    uint32_t codes[kBlk / 2];
+    if constexpr (kBlk == 8) {
+        const uint4 cw = lds128(st + meta_off + r * 32 + b0 * 2);
+        codes[0] = cw.x; codes[1] = cw.y; codes[2] = cw.z; codes[3] = cw.w;
+    } else {
+        const uint2 cw = *reinterpret_cast<const uint2 *>(st + meta_off + r * 32 + b0 * 2);
+        codes[0] = cw.x; codes[1] = cw.y;
+    }
+    unsigned char *row = dense + atom * (kUmRows * 128) + r * 128;
+#pragma unroll
+    for (int c = 0; c < kBlk / 2; ++c) {
+        const int cl = (b0 >> 1) + c;  // value chunk within the row
+        const uint4 v = lds128(st + r * 128 + ((cl ^ (r & 7)) << 4));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
+            const uint32_t code = (codes[c] >> (16 * h)) & 0xFFFu;
+            const uint2 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
+            uint4 o;
+            o.x = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
+            o.y = __byte_perm(__byte_perm(lo, 0u, sa.x >> 16), hi, sb.x >> 16);
+            o.z = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
+            o.w = __byte_perm(__byte_perm(lo, 0u, sa.y >> 16), hi, sb.y >> 16);
+            const int b = (2 * cl + h) & 7;  // dense chunk within the atom
+            *reinterpret_cast<uint4 *>(row + ((b ^ (r & 7)) << 4)) = o;
+        }
+    }
+}
+
+template <int kHalf>
+__device__ __forceinline__ void u8_store(const SkOp &d, int64_t tile, int q, int lane, int tok0,
+                                         const float (&v)[kHalf], int tokens) {
+    const int64_t r = tile * kUmRows + 32 * q + lane;
+    if (r >= d.rows) return;
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i)
+        if (tok0 + i < tokens) d.y[(tok0 + i) * d.rows + r] = v[i];
+}
+
+template <int kNTok>
+__global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(const __grid_constant__ TmGroup tg,
+                                                                            float *__restrict__ part,
+                                                                            unsigned int *__restrict__ tickets,
+                                                                            unsigned int *__restrict__ err,
+                                                                            int arm_only_first) {
+    static_assert(kNTok % 16 == 0 && kNTok >= 16 && kNTok <= kMaxTokens, "N of an M = 128 MMA");
+    static_assert(2 * (u8_smem_bytes<kNTok>() + 1024) > 233472, "one CTA per SM");
+    static_assert(kU8Warps % 4 == 0 && kU8Warps <= 16 && kNTok % (8 * (kU8Warps / 4)) == 0,
+                  "each epilogue warp takes a multiple of 8 token columns");
+    constexpr int kD = kU8Stages, kStage = u8_stage_bytes<kNTok>(), kAOff = u8_a_off<kNTok>();
+    constexpr int kMetaOff = kUmRows * 128 + 2 * um_xbox_bytes<kNTok>();
+    constexpr int kHalf = kNTok / (kU8Warps / 4);  // token columns per epilogue warp
+    constexpr int kBar = 32 * kU8Warps;
+    constexpr uint32_t kIdesc = u8_idesc<kNTok>();
+    extern __shared__ unsigned char s_dyn_u8[];
+    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_acc;
+    __shared__ unsigned s_tmem;
+    __shared__ volatile int s_abort;
+    __shared__ int s_last;
+    const SkGroup &grp = tg.g;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t total = grp.total_chunks;
+    const int64_t G = imin64((int64_t)gridDim.x, total), cta = blockIdx.x;
+    if (cta >= G) return;  // the whole CTA, before any barrier or allocation
+    const int64_t lo = cta * total / G, hi = (cta + 1) * total / G;
+    const int n = (int)(hi - lo);
+    const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_u8);
+    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
+    unsigned char *ring = s_dyn_u8 + pad;
+    const unsigned ring_s = dyn_s + pad;
+    uint2 *tab = reinterpret_cast<uint2 *>(ring + kD * kStage);  // A: entries [0, 64), B: [64, 128), x copies
+    const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
+    const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
+    const unsigned accb = (unsigned)__cvta_generic_to_shared(&s_acc);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kD; ++s) {
+            mbar_init(full0 + 8 * s, 1u);
+            mbar_init(empty0 + 8 * s, 1u);
+        }
+        mbar_init(accb, 1u);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    for (int i = threadIdx.x; i < 2 * 64 * kU8TabCopies; i += blockDim.x)  // entry e, copy c at e * copies + c
+        tab[i] = u8_table_entry((i / kU8TabCopies) & 63, i >= 64 * kU8TabCopies);
+    if (warp == 0) {
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(&s_tmem);
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst),
+                     "r"(kU8TmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const unsigned tbase = s_tmem;
+
+    if (warp == kU8Warps) {
+        // ------------------------------------------------------------ copy warp
+        Cursor ld = sk_decode(grp, lo);
+        int issued = 0;
+        for (int f = 0; f < n; ++f) {
+            const int s = f % kD;
+            if (f >= kD && !um_wait(empty0 + 8 * s, ((f / kD) - 1) & 1, &s_abort)) {
+                if (lane == 0 && !s_abort) {
+                    atomicOr(err, 1u);
+                    s_abort = 1;
+                }
+                break;
+            }
+            if (lane == 0) {
+                if (f == 0 && arm_only_first)  // test of the bounded wait: a stage nothing fills
+                    mbar_arrive_tx(full0, (unsigned)u8_tx<kNTok>());
+                else {
+                    fence_proxy_async();
+                    u8_issue<kNTok>(tg, ld, ring_s + s * kStage, full0 + 8 * s);
+                }
+            }
+            ++issued;
+            sk_advance(grp, ld);
+        }
+        for (int s = 0; s < kD && s < issued; ++s) {
+            const int last = s + ((issued - 1 - s) / kD) * kD;
+            tm_wait(full0 + 8 * s, (last / kD) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ expansion / MMA / epilogue warps
+        const int r = threadIdx.x & (kUmRows - 1), pt = threadIdx.x >> 7;
+        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
+        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
+        Cursor cc = sk_decode(grp, lo);
+        bool fresh = true;
+        unsigned acc_phase = 0u;
+        int mma_commits = 0;
+        bool failed = false;
+        for (int f = 0; f < n; ++f) {
+            const int s = f % kD;
+            unsigned char *st = ring + s * kStage;
+            const bool ok = um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort);
+            if (ok) {
+                u8_expand(st, st + kAOff, tab + (lane & (kU8TabCopies - 1)),
+                          tab + 64 * kU8TabCopies + (lane & (kU8TabCopies - 1)), kMetaOff, r, pt);
+                fence_proxy_async();  // the dense tile, written here, is read by the tensor cores
+            }
+            if (um_bar_or<kBar>(!ok)) {
+                failed = true;
+                break;
+            }
+            const SkOp &d = grp.d[cc.op];
+            const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+                const unsigned sa = ring_s + s * kStage;
+                const uint64_t a0 = um_desc(sa + kAOff), a1 = um_desc(sa + kAOff + kUmRows * 128),
+                               b0 = um_desc(sa + kUmRows * 128),
+                               b1 = um_desc(sa + kUmRows * 128 + um_xbox_bytes<kNTok>());
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    umma_dense(tbase, ((j >> 2) ? a1 : a0) + (uint64_t)(2 * (j & 3)),
+                               ((j >> 2) ? b1 : b0) + (uint64_t)(2 * (j & 3)), kIdesc, (fresh && j == 0) ? 0u : 1u);
+                umma_commit(empty0 + 8 * s);
+                if (piece_end) umma_commit(accb);
+            }
+            ++mma_commits;
+            fresh = false;
+            if (piece_end) {
+                const bool acc_ok = um_wait(accb, acc_phase, &s_abort);
+                acc_phase ^= 1u;
+                if (um_bar_or<kBar>(!acc_ok)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float v[kHalf];
+#pragma unroll
+                for (int k = 0; k < kHalf / 8; ++k) tmem_ld8(tq + 8 * k, v + 8 * k);
+                tc_fence_before();
+                const int64_t a = d.chunk_begin + cc.tile * d.nch, b = a + d.nch;
+                const int64_t c1 = ((a + 1) * G - 1) / total, c2 = (b * G - 1) / total;
+                const int tok0 = ch * kHalf;
+                if (c1 == c2) {
+                    u8_store<kHalf>(d, cc.tile, q, lane, tok0, v, grp.tokens);
+                } else {
+                    const int64_t lo1 = c1 * total / G;
+                    const int slot = (cta == c1 && lo1 < a) ? 1 : 0;
+                    float *mine = part + (size_t)(cta * 2 + slot) * kUmPartFloats + (size_t)tok0 * kUmRows + 32 * q + lane;
+#pragma unroll
+                    for (int i = 0; i < kHalf; ++i) __stcg(mine + i * kUmRows, v[i]);
+                    __threadfence();
+                    um_bar<kBar>();
+                    if (threadIdx.x == 0) s_last = (atomicAdd(tickets + c1, 1u) == (unsigned int)(c2 - c1));
+                    um_bar<kBar>();
+                    if (s_last) {
+                        __threadfence();
+                        float sum[kHalf];
+#pragma unroll
+                        for (int i = 0; i < kHalf; ++i) sum[i] = 0.f;
+                        for (int64_t qq = c1; qq <= c2; ++qq) {
+                            const int sid = (qq == c1 && lo1 < a) ? 1 : 0;
+                            const float *p = part + (size_t)(qq * 2 + sid) * kUmPartFloats + (size_t)tok0 * kUmRows + 32 * q + lane;
+#pragma unroll
+                            for (int i = 0; i < kHalf; ++i) sum[i] += __ldcg(p + i * kUmRows);
+                        }
+                        u8_store<kHalf>(d, cc.tile, q, lane, tok0, sum, grp.tokens);
+                        um_bar<kBar>();
+                        if (threadIdx.x == 0) tickets[c1] = 0u;
+                    }
+                }
+                fresh = true;
+            }
+            sk_advance(grp, cc);
+        }
+        if (failed) {
+            if (threadIdx.x == 0 && !s_abort) {
+                atomicOr(err, 1u);
+                s_abort = 1;
+            }
+            if (mma_commits > 0) {
+                const int f = mma_commits - 1;
+                tm_wait(empty0 + 8 * (f % kD), (f / kD) & 1);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kU8TmemCols)
+                     : "memory");
+    }
+}
+
 
 }  // namespace spl
 }  // namespace mllm

@@ -346,6 +346,19 @@ mllm_status launch_spl_umma(const spl::TmGroup &g, float *part, unsigned int *ti
     return cuda_status(cudaGetLastError());
 }
 
+template <int kNTok>
+mllm_status launch_spl_umma48(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
+                              cudaStream_t st, int arm_only_first = 0) {
+    auto fn = spl::sparse_linear_umma48_kernel<kNTok>;
+    constexpr int smem = spl::u8_smem_bytes<kNTok>();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    resident_ctas(dev, (const void *)fn, spl::kU8Threads, smem);  // sets the dynamic shared-memory limit
+    const int64_t grid = std::min<int64_t>((int64_t)sm_count(dev), spl::kBatchMaxCtas);  // one CTA per SM
+    fn<<<(unsigned)grid, spl::kU8Threads, smem, st>>>(g, part, tickets, err, arm_only_first);
+    return cuda_status(cudaGetLastError());
+}
+
 template <int kN, int kNT>
 mllm_status launch_spl(const spl::OpGroup &g, cudaStream_t st) {
     auto fn = spl::sparse_linear_kernel<kN, kNT, kSplRowTiles, kSplDepth>;
@@ -515,12 +528,15 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
 }
 
 
-// 17-64 tokens for 2:4 operands with cols % 128 == 0: the tensor-memory kernel, 16 operands per
-// launch (false if a tensor map cannot be encoded; nothing is launched then).
-bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, float *part,
+// 17-64 tokens for operands with cols % 128 == 0: the tensor-memory kernels (2:4 sparse MMA,
+// 4:8 expanded to dense), 16 operands per launch (false if a tensor map cannot be encoded;
+// nothing is launched then).
+bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, mllm_nm nm, int32_t tokens, float *part,
                            unsigned int *tickets, unsigned int *err, cudaStream_t st, mllm_status *status,
                            int arm_only_first = 0) {
-    const int ntok = (tokens + 15) / 16 * 16 < 32 ? 32 : (tokens + 15) / 16 * 16;  // the MMA's N
+    const bool is24 = nm.m == 4;
+    const int step = is24 ? 16 : spl::kU8NStep;  // the MMA's N: tokens rounded up to a step, at least 32
+    const int ntok = (tokens + step - 1) / step * step < 32 ? 32 : (tokens + step - 1) / step * step;
     for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
         const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
         static thread_local spl::TmGroup tg;
@@ -543,17 +559,27 @@ bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, int32_t 
             const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
             if (!(encode_2d(&tg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
                             spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
-                  encode_2d(&tg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4,
-                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  (is24 ? encode_2d(&tg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows,
+                                    cols / 8, 4, spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE)
+                        : encode_2d(&tg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT16, o.pack_meta, cols / 8, rows,
+                                    cols / 4, 16, spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
                   encode_2d(&tg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
                             (uint32_t)ntok, CU_TENSOR_MAP_SWIZZLE_128B)))
                 return false;
         }
         tg.g.n = (int32_t)n;
         tg.g.total_chunks = acc;
-        *status = ntok == 64   ? launch_spl_umma<64>(tg, part, tickets, err, st, arm_only_first)
-                  : ntok == 48 ? launch_spl_umma<48>(tg, part, tickets, err, st, arm_only_first)
-                               : launch_spl_umma<32>(tg, part, tickets, err, st, arm_only_first);
+        if (is24)
+            *status = ntok == 64   ? launch_spl_umma<64>(tg, part, tickets, err, st, arm_only_first)
+                      : ntok == 48 ? launch_spl_umma<48>(tg, part, tickets, err, st, arm_only_first)
+                                   : launch_spl_umma<32>(tg, part, tickets, err, st, arm_only_first);
+        else if (ntok == 64)
+            *status = launch_spl_umma48<64>(tg, part, tickets, err, st, arm_only_first);
+        else if constexpr (48 % spl::kU8NStep == 0)
+            *status = ntok == 48 ? launch_spl_umma48<48>(tg, part, tickets, err, st, arm_only_first)
+                                 : launch_spl_umma48<32>(tg, part, tickets, err, st, arm_only_first);
+        else
+            *status = launch_spl_umma48<32>(tg, part, tickets, err, st, arm_only_first);
         if (*status != MLLM_OK) return true;
     }
     *status = MLLM_OK;
@@ -931,10 +957,10 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
             if (s != MLLM_OK) return s;
             continue;
         }
-        if (tokens > spl::kMaxTileTokens && nm.m == 4 && ops[i].cols % spl::kTmChunk == 0) batched.push_back(ops[i]);
+        if (tokens > spl::kMaxTileTokens && ops[i].cols % spl::kTmChunk == 0) batched.push_back(ops[i]);
         else act.push_back(ops[i]);
     }
-    if (!batched.empty() && !sparse_linear_batched(batched, tokens, part, tickets, err, st, &s))
+    if (!batched.empty() && !sparse_linear_batched(batched, nm, tokens, part, tickets, err, st, &s))
         act.insert(act.end(), batched.begin(), batched.end());  // maps not encodable: token groups
     if (s != MLLM_OK) return s;
     if (act.empty()) return MLLM_OK;
@@ -954,9 +980,8 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
 
 size_t mllm_sparse_linear_workspace_bytes(void) { return spl::kSkWorkspaceBytes; }
 
-mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int32_t tokens, void *workspace,
-                                             size_t workspace_bytes, void *stream) {
-    const mllm_nm nm{2, 4};
+mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, mllm_nm nm, int32_t tokens,
+                                             void *workspace, size_t workspace_bytes, void *stream) {
     mllm_status s = validate_operands(op, 1, nm, tokens);
     if (s != MLLM_OK) return s;
     if (!workspace || workspace_bytes < spl::kSkWorkspaceBytes) return MLLM_ERR_WORKSPACE;
@@ -968,7 +993,7 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int3
     unsigned int *err = tickets + spl::kMaxSkWarps;
     if (tokens > spl::kMaxTileTokens) {  // the tensor-memory kernel
         const std::vector<mllm_sparse_operand> ops(1, *op);
-        if (!sparse_linear_batched(ops, tokens, part, tickets, err, st, &s, 1)) return MLLM_ERR_UNSUPPORTED;
+        if (!sparse_linear_batched(ops, nm, tokens, part, tickets, err, st, &s, 1)) return MLLM_ERR_UNSUPPORTED;
         return s;
     }
     static thread_local spl::TmGroup tg;
@@ -987,8 +1012,11 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, int3
     tg.g.n = 1;
     tg.g.total_chunks = d.nch * d.ntiles;
     const int nt = tokens > 8 ? 2 : 1;
-    if (!encode_operand(&tg.maps[0], *op, tokens, nt)) return MLLM_ERR_UNSUPPORTED;
-    return nt == 2 ? launch_spl_tma<2>(tg, part, tickets, err, st, 1) : launch_spl_tma<1>(tg, part, tickets, err, st, 1);
+    const bool is24 = nm.m == 4;
+    if (!encode_operand(&tg.maps[0], *op, tokens, nt, is24 ? 2 : 4)) return MLLM_ERR_UNSUPPORTED;
+    if (is24)
+        return nt == 2 ? launch_spl_tma<2>(tg, part, tickets, err, st, 1) : launch_spl_tma<1>(tg, part, tickets, err, st, 1);
+    return nt == 2 ? launch_spl_tma<2, 4>(tg, part, tickets, err, st, 1) : launch_spl_tma<1, 4>(tg, part, tickets, err, st, 1);
 }
 
 size_t mllm_sizeof_sparse_operand(void) { return sizeof(mllm_sparse_operand); }

@@ -205,12 +205,15 @@ def test_timeout_check_validation(M):
     L = M.lib()
     wsb = M.mllm_sparse_linear_workspace_bytes()
 
-    def call(op, tokens=4, ws=0x100000):
+    def call(op, tokens=4, ws=0x100000, nm=(2, 4)):
         arr = (M.SparseOperand * 1)(op)
-        return L.mllm_sparse_linear_check_timeout(ctypes.cast(arr, ctypes.c_void_p), tokens, ws, wsb, 0)
+        return L.mllm_sparse_linear_check_timeout(ctypes.cast(arr, ctypes.c_void_p), M.NM(*nm), tokens, ws, wsb, 0)
 
-    # shapes the 2:4 tensor-copy pipeline does not take, rejected before any launch
+    # shapes the tensor-copy pipelines do not take, rejected before any launch
     assert call(_op(M, cols=64)) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=64), nm=(4, 8)) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=128), nm=(3, 8)) == M.MLLM_ERR_UNSUPPORTED
+    assert call(_op(M, cols=132), nm=(4, 8)) == M.MLLM_ERR_INVALID_ARG
     assert call(_op(M, cols=128), tokens=65) == M.MLLM_ERR_INVALID_ARG
     assert call(_op(M, cols=128, rows=0)) == M.MLLM_ERR_UNSUPPORTED
     assert call(_op(M, cols=128), ws=0) == M.MLLM_ERR_WORKSPACE

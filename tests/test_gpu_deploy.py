@@ -234,19 +234,18 @@ def test_full_stack_call_as_benchmarked(orc, ws):
     assert _tickets_clear(ws)
 
 
-@pytest.mark.parametrize("tokens", [4, 40])
-def test_bounded_wait_reports_error_and_context_survives(orc, tokens):
-    """Failure detection of the copy pipelines (per-warp kernel at 4 tokens, batched kernel at
-    40): a launch whose first stage is armed but never filled makes the bounded waits (1 s) run
-    out; the call sets the workspace's error word, returns, and the next call on a re-zeroed
-    workspace is exact."""
+@pytest.mark.parametrize("nm,tokens", [((2, 4), 4), ((2, 4), 40), ((4, 8), 4), ((4, 8), 40)])
+def test_bounded_wait_reports_error_and_context_survives(orc, nm, tokens):
+    """Failure detection of the copy pipelines (per-warp kernels at 4 tokens, tensor-memory
+    kernels at 40): a launch whose first stage is armed but never filled makes the bounded
+    waits (1 s) run out; the call sets the workspace's error word, returns, and the next call
+    on a re-zeroed workspace is exact."""
     import time
 
-    nm = (2, 4)
     ws = sparse_linear_workspace(DEV)
     o = Operand(orc, nm, 64, 256, tokens, seed=31)
     t0 = time.time()
-    mllm_sparse_linear_check_timeout(o.op(), tokens, ws)
+    mllm_sparse_linear_check_timeout(o.op(), nm, tokens, ws)
     torch.cuda.synchronize()
     assert time.time() - t0 < 60
     assert int(ws[-16:-12].view(torch.int32).item()) != 0
@@ -290,10 +289,14 @@ def test_batched_decode_2of4(orc, ws, tokens):
     assert _tickets_clear(ws)
 
 
-@pytest.mark.parametrize("tokens", [24, 64])
-def test_batched_decode_4of8_token_groups(orc, ws, tokens):
+@pytest.mark.parametrize("tokens", [17, 24, 33, 48, 64])
+def test_batched_decode_4of8(orc, ws, tokens):
+    """17-64 tokens at 4:8: the tensor-memory kernel (blocks expanded to a dense tile in shared
+    memory, dense tcgen05.mma) for widths that are multiples of 128 (ragged rows, tiles cut
+    between CTAs), token groups of 16 for the others, in one call."""
     nm = (4, 8)
-    ops = [Operand(orc, nm, r, c, tokens, seed=320 + i) for i, (r, c) in enumerate([(40, 256), (19, 72)])]
+    shapes = [(40, 256), (130, 1024), (7, 128), (19, 72), (33, 40)]
+    ops = [Operand(orc, nm, r, c, tokens, seed=320 + i) for i, (r, c) in enumerate(shapes)]
     mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
     torch.cuda.synchronize()
     for o in ops:
@@ -301,9 +304,10 @@ def test_batched_decode_4of8_token_groups(orc, ws, tokens):
     assert _tickets_clear(ws)
 
 
-def test_batched_decode_full_size_64_tokens(orc, ws):
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
+def test_batched_decode_full_size_64_tokens(orc, ws, nm):
     """q [4096, 4096], gate [11008, 4096], down [4096, 11008] at 64 tokens in one call."""
-    nm, tokens = (2, 4), 64
+    tokens = 64
     ops = [Operand(orc, nm, r, c, tokens, seed=340 + i, direct=True)
            for i, (r, c) in enumerate([(4096, 4096), (11008, 4096), (4096, 11008)])]
     mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
