@@ -7,11 +7,12 @@
 // call (decode). At that size the product is bound by reading the compressed weight from
 // HBM: 2:4 moves 2.25 bytes per weight pair instead of 4 dense.
 //
-// Up to 16 tokens, four kernels, chosen per launch by the operands' widths (host side, mllm.cu);
-// 17-64 tokens of 2:4 operands with cols % 128 == 0 run on the fifth-generation tensor cores
-// (kernels_umma.cuh), other operands as groups of 16 tokens:
-//   sparse_linear_tma_kernel  2:4, cols % 128 == 0 (every LLM shape): sparse tensor cores
-//                             (mma.sp) fed by tiled tensor copies; the fast path;
+// Operands with cols % 128 == 0 (every LLM shape) run on the fifth-generation tensor cores
+// (kernels_umma.cuh) -- 2:4 above 16 tokens, 4:8 at any token count. The rest run here, up to
+// 16 tokens per launch (more as groups of 16), on four kernels chosen per launch by the
+// operands' widths (host side, mllm.cu):
+//   sparse_linear_tma_kernel  2:4, cols % 128 == 0, 1-16 tokens: sparse tensor cores (mma.sp)
+//                             fed by tiled tensor copies;
 //   sparse_linear_sp_kernel   2:4, cols % 32 == 0: the same arithmetic fed by cp.async;
 //   sparse_linear_sk_kernel   4:8 (no hardware sparse path) and 2:4 with cols % 16 == 0:
 //                             blocks expanded to dense bf16 in registers, dense mma.sync;
@@ -833,22 +834,20 @@ __global__ void __launch_bounds__(32 * sp_warps<kNT>(), 1) sparse_linear_sp_kern
 
 constexpr int kTmChunk = 128;
 constexpr unsigned long long kTmWaitNs = 1000000000ull;  // bound of one wait: 1 s (a stage lands in us)
-// kN = 2 (2:4, mma.sp) or 4 (4:8, blocks expanded to dense bf16, mma.sync). A stage's metadata
-// box: 2:4 32 rows x 4 uint32 words, 4:8 32 rows x 16 uint16 codes.
+// A stage's metadata box: 32 rows x 4 uint32 words.
 template <int kNT> constexpr int tm_xbox_bytes() { return 8 * kNT * 128; }
-template <int kN> constexpr int tm_meta_bytes() { return kN == 2 ? 32 * 16 : 32 * 32; }
-template <int kNT, int kN = 2> constexpr int tm_stage_tx() { return 32 * 128 + 2 * tm_xbox_bytes<kNT>() + tm_meta_bytes<kN>(); }
-template <int kNT, int kN = 2> constexpr int tm_stage_bytes() { return (tm_stage_tx<kNT, kN>() + 1023) / 1024 * 1024; }
-template <int kNT, int kN = 2> constexpr int tm_warps() { return (kN == 4 && kNT == 2) ? 7 : 8; }
-template <int kNT, int kN = 2> constexpr int tm_stages() { return 3; }
-template <int kNT, int kN = 2> constexpr int tm_smem_bytes() {
-    return tm_warps<kNT, kN>() * tm_stages<kNT, kN>() * tm_stage_bytes<kNT, kN>() + 1024;
-}
+template <int kNT> constexpr int tm_stage_tx() { return 32 * 128 + 2 * tm_xbox_bytes<kNT>() + 32 * 16; }
+template <int kNT> constexpr int tm_stage_bytes() { return (tm_stage_tx<kNT>() + 1023) / 1024 * 1024; }
+constexpr int kTmWarps = 8, kTmStages = 3;
+template <int kNT> constexpr int tm_smem_bytes() { return kTmWarps * kTmStages * tm_stage_bytes<kNT>() + 1024; }
 
+// Tensor maps of one operand. The per-warp kernel (2:4) uses 32-row boxes and x boxes of 8kNT
+// tokens; the tensor-memory kernels (kernels_umma.cuh) 128-row boxes, x boxes of N tokens and,
+// for 4:8, uint16 metadata [rows, cols/8] in boxes of 16 x 128.
 struct TmMaps {
-    CUtensorMap vals;  // bf16 [rows, cols/2], box 64 x 32, 128-byte swizzle
-    CUtensorMap meta;  // 2:4: uint32 [rows, cols/32], box 4 x 32; 4:8: uint16 [rows, cols/8], box 16 x 32
-    CUtensorMap x;     // bf16 [tokens, cols], box 64 x 8kNT, 128-byte swizzle
+    CUtensorMap vals;  // bf16 [rows, cols/2], box 64 x rows, 128-byte swizzle
+    CUtensorMap meta;  // 2:4: uint32 [rows, cols/32], box 4 x rows
+    CUtensorMap x;     // bf16 [tokens, cols], box 64 x tokens, 128-byte swizzle
 };
 
 struct TmGroup {
@@ -896,49 +895,18 @@ __device__ __forceinline__ bool tm_wait(unsigned bar, unsigned parity) {
     }
 }
 
-template <int kNT, int kN = 2>
+template <int kNT>
 __device__ __forceinline__ void tm_issue(const TmGroup &tg, const Cursor &c, unsigned stage, unsigned bar) {
     const TmMaps &mp = tg.maps[c.op];
     const int j = (int)c.j, row0 = (int)(c.tile * kSkRows);
-    mbar_arrive_tx(bar, (unsigned)tm_stage_tx<kNT, kN>());
+    mbar_arrive_tx(bar, (unsigned)tm_stage_tx<kNT>());
     tma_load_2d(stage, &mp.vals, 64 * j, row0, bar);
     tma_load_2d(stage + 4096, &mp.x, 128 * j, 0, bar);
     tma_load_2d(stage + 4096 + tm_xbox_bytes<kNT>(), &mp.x, 128 * j + 64, 0, bar);
-    tma_load_2d(stage + 4096 + 2 * tm_xbox_bytes<kNT>(), &mp.meta, (kN == 2 ? 4 : 16) * j, row0, bar);
+    tma_load_2d(stage + 4096 + 2 * tm_xbox_bytes<kNT>(), &mp.meta, 4 * j, row0, bar);
 }
 
 __device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
-
-// 4:8 stage: two 64-column windows; in each, lane (g, t) takes blocks 2t, 2t+1 of rows
-// 16 mt + g and + 8 (16-byte chunk 4w + t of the swizzled values row, two uint16 codes) and
-// x columns 16t..16t+15 of tokens g + 8 nt, and runs the expansion kernels' four mma.sync
-// steps (same k-slot mapping).
-template <int kNT>
-__device__ __forceinline__ void tm_compute48(const unsigned char *st, int g, int t, const uint4 *sel48,
-                                             const uint4 *msk48, float (&acc)[2][kNT][4]) {
-    const unsigned char *meta = st + 4096 + 2 * tm_xbox_bytes<kNT>();
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-        const unsigned char *xb = st + 4096 + w * tm_xbox_bytes<kNT>();
-        Slab<kNT> sl;
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-            const int r = g + 8 * nt;
-            sl.x[nt][0] = lds128(xb + r * 128 + (((2 * t) ^ (r & 7)) << 4));
-            sl.x[nt][1] = lds128(xb + r * 128 + (((2 * t + 1) ^ (r & 7)) << 4));
-        }
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = 16 * mt + 8 * h + g;
-                sl.v[h] = lds128(st + r * 128 + (((4 * w + t) ^ (r & 7)) << 4));
-                sl.m[h] = lds32(meta + r * 32 + 16 * w + 4 * t);
-            }
-            mma_slab<4, kNT>(sl, nullptr, sel48, msk48, acc[mt]);
-        }
-    }
-}
 
 template <int kNT, bool kEdge>
 __device__ __forceinline__ void tm_compute(const unsigned char *st, int lane, int g, int t, float (&acc)[2][kNT][4]) {
@@ -973,21 +941,13 @@ __device__ __forceinline__ void tm_compute(const unsigned char *st, int lane, in
     }
 }
 
-template <int kNT, int kN = 2>
-__global__ void __launch_bounds__(32 * tm_warps<kNT, kN>(), 1) sparse_linear_tma_kernel(
+template <int kNT>
+__global__ void __launch_bounds__(32 * kTmWarps, 1) sparse_linear_tma_kernel(
     const __grid_constant__ TmGroup tg, float *__restrict__ part, unsigned int *__restrict__ tickets,
     unsigned int *__restrict__ err, int arm_only_first) {
-    constexpr int kW = tm_warps<kNT, kN>(), kD = tm_stages<kNT, kN>(), kStage = tm_stage_bytes<kNT, kN>();
+    constexpr int kW = kTmWarps, kD = kTmStages, kStage = tm_stage_bytes<kNT>();
     extern __shared__ unsigned char s_dyn_tm[];
     __shared__ __align__(8) unsigned long long s_bar[kW][kD];
-    __shared__ uint4 s_sel48[kN == 4 ? 256 : 1], s_msk48[kN == 4 ? 256 : 1];
-    if constexpr (kN == 4) {
-        for (int i = threadIdx.x; i < 256; i += 32 * kW) {
-            s_sel48[i] = make_uint4(g_sel48.sel[i][0], g_sel48.sel[i][1], g_sel48.sel[i][2], g_sel48.sel[i][3]);
-            s_msk48[i] = make_uint4(g_sel48.mask[i][0], g_sel48.mask[i][1], g_sel48.mask[i][2], g_sel48.mask[i][3]);
-        }
-        __syncthreads();
-    }
     const SkGroup &grp = tg.g;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int64_t total = grp.total_chunks;
@@ -1012,9 +972,9 @@ __global__ void __launch_bounds__(32 * tm_warps<kNT, kN>(), 1) sparse_linear_tma
         if (s < n) {
             if (lane == 0) {
                 if (s == 0 && arm_only_first)  // test of the bounded wait: a stage nothing fills
-                    mbar_arrive_tx(bar0, (unsigned)tm_stage_tx<kNT, kN>());
+                    mbar_arrive_tx(bar0, (unsigned)tm_stage_tx<kNT>());
                 else
-                    tm_issue<kNT, kN>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+                    tm_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
             }
             sk_advance(grp, ld);
         }
@@ -1037,13 +997,12 @@ __global__ void __launch_bounds__(32 * tm_warps<kNT, kN>(), 1) sparse_linear_tma
         }
         phase ^= 1u << s;
         const unsigned char *st = ring + s * kStage;
-        if constexpr (kN == 4) tm_compute48<kNT>(st, g, t, s_sel48, s_msk48, acc);
-        else if (rows_edge) tm_compute<kNT, true>(st, lane, g, t, acc);
+        if (rows_edge) tm_compute<kNT, true>(st, lane, g, t, acc);
         else tm_compute<kNT, false>(st, lane, g, t, acc);
         __syncwarp();        // every lane has read the stage
         fence_proxy_async();  // generic reads before the stage's next asynchronous writes
         if (f + kD < n) {
-            if (lane == 0) tm_issue<kNT, kN>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
+            if (lane == 0) tm_issue<kNT>(tg, ld, ring_s + s * kStage, bar0 + 8 * s);
             sk_advance(grp, ld);
         }
         s = (s + 1 == kD) ? 0 : s + 1;

@@ -1,6 +1,7 @@
-// kernels_umma.cuh -- batched decode (17-64 tokens) of the 2:4 serving product on the
-// fifth-generation tensor cores: tcgen05.mma.sp with operands in shared memory, sparsity
-// metadata and accumulators in tensor memory.
+// kernels_umma.cuh -- the serving product on the fifth-generation tensor cores: 2:4 at 17-64
+// tokens with tcgen05.mma.sp (operands in shared memory, sparsity metadata and accumulators in
+// tensor memory), and 4:8 at 1-64 tokens with blocks expanded to a dense tile in shared memory
+// and dense tcgen05.mma (below, "4:8 on the dense tensor cores").
 //
 // The product is y = x W*^T with W* = W (.) M* in the form mllm_hard_pack writes (two kept
 // bf16 values and one 4-bit position code per block of four weights); MaskLLM serves the
@@ -81,6 +82,9 @@ __device__ __forceinline__ void umma_sp(unsigned d_tmem, uint64_t adesc, uint64_
 __device__ __forceinline__ void umma_commit(unsigned bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
                  : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
@@ -366,14 +370,18 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
 // B[p2p3].i): table A places the first pair and zero-fills, table B places the second pair
 // and keeps the rest (u8_table_entry). Each CTA builds both 64-entry tables in shared memory,
 // 16 interleaved copies each, so that the lookups of a half-warp never share a bank. Thread t
-// expands row t % 128, part t / 128 of the stage (64 / kU8Warps blocks, within one atom).
+// expands row t % 128, part t / 128 of the stage (64 / kU8Warps blocks, within one atom), and
+// arrives on the stage's "expanded" barrier; a separate MMA warp waits for all arrivals and
+// issues the stage's MMAs, so the expanding warps never wait on one another within a tile
+// (they meet once per tile, for the epilogue).
 // A stage: values 16 KB | x, two kNTok x 64 boxes | metadata, 128 rows x 16 codes (4 KB) |
 // the dense tile (32 KB). One CTA per SM with three stages; tensor memory holds only the
 // accumulator (64 columns). Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 and the
-// token slice w / 4. Copy warp, bounded waits, work split and partial tiles as above.
+// token slice w / 4. Copy warp, bounded waits, work split and partial tiles as above; a warp
+// whose wait runs out stops working and leaves with the others at the end of the tile.
 
 constexpr int kU8Warps = 16;         // expansion / epilogue warps (a multiple of 4, at most 16)
-constexpr int kU8Threads = 32 * kU8Warps + 32;  // + the copy warp
+constexpr int kU8Threads = 32 * kU8Warps + 64;  // + the copy warp and the MMA warp
 constexpr int kU8NStep = 8 * (kU8Warps / 4) > 16 ? 8 * (kU8Warps / 4) : 16;  // N is a multiple of this
 constexpr int kU8Stages = 3;
 constexpr unsigned kU8TmemCols = 64;
@@ -510,7 +518,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
     constexpr int kBar = 32 * kU8Warps;
     constexpr uint32_t kIdesc = u8_idesc<kNTok>();
     extern __shared__ unsigned char s_dyn_u8[];
-    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_acc;
+    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_exp[kD], s_acc;
     __shared__ unsigned s_tmem;
     __shared__ volatile int s_abort;
     __shared__ int s_last;
@@ -528,11 +536,13 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
     uint2 *tab = reinterpret_cast<uint2 *>(ring + kD * kStage);  // A: entries [0, 64), B: [64, 128), x copies
     const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
     const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
+    const unsigned exp0 = (unsigned)__cvta_generic_to_shared(&s_exp[0]);
     const unsigned accb = (unsigned)__cvta_generic_to_shared(&s_acc);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kD; ++s) {
             mbar_init(full0 + 8 * s, 1u);
             mbar_init(empty0 + 8 * s, 1u);
+            mbar_init(exp0 + 8 * s, (unsigned)kBar);  // every expanding thread arrives once per stage
         }
         mbar_init(accb, 1u);
         s_abort = 0;
@@ -580,32 +590,23 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
             const int last = s + ((issued - 1 - s) / kD) * kD;
             tm_wait(full0 + 8 * s, (last / kD) & 1);
         }
-    } else {
-        // ------------------------------------------------------------ expansion / MMA / epilogue warps
-        const int r = threadIdx.x & (kUmRows - 1), pt = threadIdx.x >> 7;
-        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
-        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
+    } else if (warp == kU8Warps + 1) {
+        // ------------------------------------------------------------ MMA warp
         Cursor cc = sk_decode(grp, lo);
         bool fresh = true;
-        unsigned acc_phase = 0u;
-        int mma_commits = 0;
-        bool failed = false;
+        int commits = 0;
         for (int f = 0; f < n; ++f) {
             const int s = f % kD;
-            unsigned char *st = ring + s * kStage;
-            const bool ok = um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort);
-            if (ok) {
-                u8_expand(st, st + kAOff, tab + (lane & (kU8TabCopies - 1)),
-                          tab + 64 * kU8TabCopies + (lane & (kU8TabCopies - 1)), kMetaOff, r, pt);
-                fence_proxy_async();  // the dense tile, written here, is read by the tensor cores
-            }
-            if (um_bar_or<kBar>(!ok)) {
-                failed = true;
+            if (!um_wait(exp0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                if (lane == 0 && !s_abort) {
+                    atomicOr(err, 1u);
+                    s_abort = 1;
+                }
                 break;
             }
             const SkOp &d = grp.d[cc.op];
             const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
-            if (threadIdx.x == 0) {
+            if (lane == 0) {
                 tc_fence_after();
                 const unsigned sa = ring_s + s * kStage;
                 const uint64_t a0 = um_desc(sa + kAOff), a1 = um_desc(sa + kAOff + kUmRows * 128),
@@ -618,10 +619,46 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
                 umma_commit(empty0 + 8 * s);
                 if (piece_end) umma_commit(accb);
             }
-            ++mma_commits;
-            fresh = false;
+            __syncwarp();
+            ++commits;
+            fresh = piece_end;
+            sk_advance(grp, cc);
+        }
+        if (commits > 0) {  // every MMA has completed (bounded) before the tensor memory is released
+            const int f = commits - 1;
+            tm_wait(empty0 + 8 * (f % kD), (f / kD) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ expansion / epilogue warps
+        const int r = threadIdx.x & (kUmRows - 1), pt = threadIdx.x >> 7;
+        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
+        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
+        const uint2 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
+        Cursor cc = sk_decode(grp, lo);
+        unsigned acc_phase = 0u;
+        bool failed = false;
+        for (int f = 0; f < n; ++f) {
+            const int s = f % kD;
+            unsigned char *st = ring + s * kStage;
+            // A warp whose wait ran out stops working but keeps its place in the loop, so that
+            // it meets the others at the end of the tile, where all of them leave together.
+            if (!failed) {
+                if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                    u8_expand(st, st + kAOff, tab_a, tab_b, kMetaOff, r, pt);
+                    fence_proxy_async();  // the dense tile, written here, is read by the tensor cores
+                    mbar_arrive(exp0 + 8 * s);
+                } else {
+                    failed = true;
+                    if (lane == 0 && !s_abort) {
+                        atomicOr(err, 1u);
+                        s_abort = 1;
+                    }
+                }
+            }
+            const SkOp &d = grp.d[cc.op];
+            const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
             if (piece_end) {
-                const bool acc_ok = um_wait(accb, acc_phase, &s_abort);
+                const bool acc_ok = !failed && um_wait(accb, acc_phase, &s_abort);
                 acc_phase ^= 1u;
                 if (um_bar_or<kBar>(!acc_ok)) {
                     failed = true;
@@ -631,7 +668,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
                 float v[kHalf];
 #pragma unroll
                 for (int k = 0; k < kHalf / 8; ++k) tmem_ld8(tq + 8 * k, v + 8 * k);
-                tc_fence_before();
+                tc_fence_before();  // these reads precede the next piece's first MMA (after its arrivals)
                 const int64_t a = d.chunk_begin + cc.tile * d.nch, b = a + d.nch;
                 const int64_t c1 = ((a + 1) * G - 1) / total, c2 = (b * G - 1) / total;
                 const int tok0 = ch * kHalf;
@@ -663,19 +700,12 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
                         if (threadIdx.x == 0) tickets[c1] = 0u;
                     }
                 }
-                fresh = true;
             }
             sk_advance(grp, cc);
         }
-        if (failed) {
-            if (threadIdx.x == 0 && !s_abort) {
-                atomicOr(err, 1u);
-                s_abort = 1;
-            }
-            if (mma_commits > 0) {
-                const int f = mma_commits - 1;
-                tm_wait(empty0 + 8 * (f % kD), (f / kD) & 1);
-            }
+        if (failed && threadIdx.x == 0 && !s_abort) {
+            atomicOr(err, 1u);
+            s_abort = 1;
         }
     }
     tc_fence_before();
@@ -686,7 +716,6 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
                      : "memory");
     }
 }
-
 
 }  // namespace spl
 }  // namespace mllm

@@ -305,27 +305,22 @@ bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_
 }
 
 // The three maps of an operand for the TMA kernel (cols % 128 == 0).
-bool encode_operand(spl::TmMaps *mp, const mllm_sparse_operand &o, int32_t tokens, int kNT, int kN = 2) {
+bool encode_operand(spl::TmMaps *mp, const mllm_sparse_operand &o, int32_t tokens, int kNT) {
     const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
-    const bool meta_ok =
-        kN == 2 ? encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4, 32,
-                            CU_TENSOR_MAP_SWIZZLE_NONE)
-                : encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT16, o.pack_meta, cols / 8, rows, cols / 4, 16, 32,
-                            CU_TENSOR_MAP_SWIZZLE_NONE);
-    return meta_ok &&
+    return encode_2d(&mp->meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4, 32,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) &&
            encode_2d(&mp->vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64, 32,
                      CU_TENSOR_MAP_SWIZZLE_128B) &&
            encode_2d(&mp->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
                      (uint32_t)(8 * kNT), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int kNT, int kN = 2>
+template <int kNT>
 mllm_status launch_spl_tma(const spl::TmGroup &g, float *part, unsigned int *tickets, unsigned int *err,
                            cudaStream_t st, int arm_only_first = 0) {
-    auto fn = spl::sparse_linear_tma_kernel<kNT, kN>;
-    constexpr int smem = spl::tm_smem_bytes<kNT, kN>(), threads = 32 * spl::tm_warps<kNT, kN>();
-    const int64_t grid =
-        grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::tm_warps<kNT, kN>());
+    auto fn = spl::sparse_linear_tma_kernel<kNT>;
+    constexpr int smem = spl::tm_smem_bytes<kNT>(), threads = 32 * spl::kTmWarps;
+    const int64_t grid = grid_for((const void *)fn, threads, smem, INT32_MAX, spl::kMaxSkWarps / spl::kTmWarps);
     fn<<<(unsigned)grid, threads, smem, st>>>(g, part, tickets, err, arm_only_first);
     return cuda_status(cudaGetLastError());
 }
@@ -458,8 +453,9 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
         if (vec) {  // streamed kernels: the launch's chunks split evenly over all warps
             // 2:4 in whole 128-column stages: tensor copies (falls back if a map cannot be
             // encoded); other 2:4 with whole metadata words: sparse tensor cores via cp.async;
-            // else block expansion
-            const bool tma = stages;
+            // else (and 4:8 whose maps could not be encoded for the tensor-memory kernel)
+            // block expansion
+            const bool tma = stages && is24;
             auto group_of = [&](int64_t chunk) {
                 spl::SkGroup g{};
                 g.tokens = tokens;
@@ -487,10 +483,9 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
                 tg.g = group_of(spl::kTmChunk);
                 bool ok = true;
                 for (size_t k = 0; k < n && ok; ++k)
-                    ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1, is24 ? 2 : 4);
+                    ok = encode_operand(&tg.maps[k], ops[order[i0 + k]], tokens, two ? 2 : 1);
                 if (ok) {
-                    if (is24) s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
-                    else s = two ? launch_spl_tma<2, 4>(tg, part, tickets, err, st) : launch_spl_tma<1, 4>(tg, part, tickets, err, st);
+                    s = two ? launch_spl_tma<2>(tg, part, tickets, err, st) : launch_spl_tma<1>(tg, part, tickets, err, st);
                     if (s != MLLM_OK) return s;
                     continue;
                 }
@@ -528,9 +523,9 @@ mllm_status sparse_linear_small(const std::vector<mllm_sparse_operand> &ops, mll
 }
 
 
-// 17-64 tokens for operands with cols % 128 == 0: the tensor-memory kernels (2:4 sparse MMA,
-// 4:8 expanded to dense), 16 operands per launch (false if a tensor map cannot be encoded;
-// nothing is launched then).
+// Operands with cols % 128 == 0 on the tensor-memory kernels (2:4 sparse MMA above 16 tokens,
+// 4:8 expanded to dense at any token count), 16 operands per launch (false if a tensor map
+// cannot be encoded; nothing is launched then).
 bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, mllm_nm nm, int32_t tokens, float *part,
                            unsigned int *tickets, unsigned int *err, cudaStream_t st, mllm_status *status,
                            int arm_only_first = 0) {
@@ -957,7 +952,8 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
             if (s != MLLM_OK) return s;
             continue;
         }
-        if (tokens > spl::kMaxTileTokens && ops[i].cols % spl::kTmChunk == 0) batched.push_back(ops[i]);
+        // the tensor-memory kernels: 2:4 above 16 tokens, 4:8 (expanded to dense) at any count
+        if (ops[i].cols % spl::kTmChunk == 0 && (tokens > spl::kMaxTileTokens || nm.m == 8)) batched.push_back(ops[i]);
         else act.push_back(ops[i]);
     }
     if (!batched.empty() && !sparse_linear_batched(batched, nm, tokens, part, tickets, err, st, &s))
@@ -991,7 +987,7 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, mllm
     float *part = static_cast<float *>(workspace);
     unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + spl::kPartBytes);
     unsigned int *err = tickets + spl::kMaxSkWarps;
-    if (tokens > spl::kMaxTileTokens) {  // the tensor-memory kernel
+    if (tokens > spl::kMaxTileTokens || nm.m == 8) {  // the tensor-memory kernel
         const std::vector<mllm_sparse_operand> ops(1, *op);
         if (!sparse_linear_batched(ops, nm, tokens, part, tickets, err, st, &s, 1)) return MLLM_ERR_UNSUPPORTED;
         return s;
@@ -1011,12 +1007,9 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, mllm
     d.chunk_begin = 0;
     tg.g.n = 1;
     tg.g.total_chunks = d.nch * d.ntiles;
-    const int nt = tokens > 8 ? 2 : 1;
-    const bool is24 = nm.m == 4;
-    if (!encode_operand(&tg.maps[0], *op, tokens, nt, is24 ? 2 : 4)) return MLLM_ERR_UNSUPPORTED;
-    if (is24)
-        return nt == 2 ? launch_spl_tma<2>(tg, part, tickets, err, st, 1) : launch_spl_tma<1>(tg, part, tickets, err, st, 1);
-    return nt == 2 ? launch_spl_tma<2, 4>(tg, part, tickets, err, st, 1) : launch_spl_tma<1, 4>(tg, part, tickets, err, st, 1);
+    const int nt = tokens > 8 ? 2 : 1;  // 2:4 up to 16 tokens: the per-warp kernel
+    if (!encode_operand(&tg.maps[0], *op, tokens, nt)) return MLLM_ERR_UNSUPPORTED;
+    return nt == 2 ? launch_spl_tma<2>(tg, part, tickets, err, st, 1) : launch_spl_tma<1>(tg, part, tickets, err, st, 1);
 }
 
 size_t mllm_sizeof_sparse_operand(void) { return sizeof(mllm_sparse_operand); }
