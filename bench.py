@@ -12,7 +12,7 @@ measured copy bandwidth.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--loop fused|separate]
                   [--impl reference]
-  python bench.py --mode sparse_linear [--workload NAME] [--steps K --warmup W]
+  python bench.py --mode sparse_linear [--workload NAME] [--serve-nm 2:4|4:8] [--steps K --warmup W]
       (serving leg: the workload's matrices as packed hard masks, y = x W*^T per call for
        1, 8, 16, 32 and 64 tokens, against dense cuBLAS; one JSON line)
 
@@ -701,6 +701,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
+    ap.add_argument("--serve-nm", default=None, choices=["2:4", "4:8"],
+                    help="--mode sparse_linear: pack the workload's matrices with this pattern instead of its own")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warm-up raised to 3 steps")
@@ -708,6 +710,12 @@ def main():
     from sparsity_mask_sampling_b200 import configs
 
     w = configs.WORKLOADS[args.workload]
+    if args.serve_nm is not None:
+        if args.mode != "sparse_linear":
+            ap.error("--serve-nm applies to --mode sparse_linear")
+        import dataclasses
+        nm = tuple(int(v) for v in args.serve_nm.split(":"))
+        w = dataclasses.replace(w, nm=nm, name=f"{w.name} packed {args.serve_nm}")
     if args.mode == "sparse_linear":
         out = sparse_linear_arm(args, w)
     elif args.impl == "reference":
