@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
 // bf16. Word i of the chunk (positions 2i, 2i+1) is prmt(prmt(v0v1, 0, A[p0p1].i), v2v3,
 // B[p2p3].i): table A places the first pair and zero-fills, table B places the second pair
 // and keeps the rest (u8_table_entry). Each CTA builds both 64-entry tables in shared memory,
-// 16 interleaved copies each, so that the lookups of a half-warp never share a bank. Thread t
+// 8 interleaved copies each, so that the 16-byte lookups of a quarter-warp never share a bank. Thread t
 // expands row t % 128, part t / 128 of the stage (64 / kU8Warps blocks, within one atom), and
 // arrives on the stage's "expanded" barrier; a separate MMA warp waits for all arrivals and
 // issues the stage's MMAs, so the expanding warps never wait on one another within a tile
@@ -389,8 +389,8 @@ constexpr unsigned kU8TmemCols = 64;
 template <int kNTok> constexpr int u8_tx() { return kUmRows * 128 + 2 * um_xbox_bytes<kNTok>() + kUmRows * 32; }
 template <int kNTok> constexpr int u8_a_off() { return (u8_tx<kNTok>() + 1023) / 1024 * 1024; }
 template <int kNTok> constexpr int u8_stage_bytes() { return u8_a_off<kNTok>() + 2 * kUmRows * 128; }
-constexpr int kU8TabCopies = 16;     // one copy per lane of a half-warp: conflict-free 8-byte lookups
-constexpr int kU8TabBytes = 2 * 64 * kU8TabCopies * 8;  // tables A and B
+constexpr int kU8TabCopies = 8;      // one copy per lane of a quarter-warp: conflict-free 16-byte lookups
+constexpr int kU8TabBytes = 2 * 64 * kU8TabCopies * 16;  // tables A and B
 template <int kNTok> constexpr int u8_smem_bytes() { return kU8Stages * u8_stage_bytes<kNTok>() + 1024 + kU8TabBytes; }
 
 // Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
@@ -424,11 +424,11 @@ __device__ __forceinline__ void tmem_ld8(unsigned taddr, float *v) {
 }
 
 // Entry q = pa | pb << 3 of expansion table A (second = false) or B (second = true): the
-// byte-permute selectors of the four words of a dense chunk (x: words 0, 1; y: words 2, 3)
-// for a value pair at positions pa < pb. Table A places the first pair (v0 v1, bytes 0-3 of
+// byte-permute selectors of the four words of a dense chunk (one per component) for a value
+// pair at positions pa < pb. Table A places the first pair (v0 v1, bytes 0-3 of
 // the permute's sources) and takes zero bytes (4-7, a zero operand) elsewhere; table B places
 // the second pair (v2 v3, bytes 4-7) over that result and keeps its bytes (0-3) elsewhere.
-__device__ __forceinline__ uint2 u8_table_entry(int q, bool second) {
+__device__ __forceinline__ uint4 u8_table_entry(int q, bool second) {
     const int pa = q & 7, pb = q >> 3;
     uint32_t w[4];
 #pragma unroll
@@ -443,7 +443,7 @@ __device__ __forceinline__ uint2 u8_table_entry(int q, bool second) {
         }
         w[i] = sel;
     }
-    return make_uint2(w[0] | w[1] << 16, w[2] | w[3] << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 template <int kNTok>
@@ -459,8 +459,8 @@ __device__ __forceinline__ void u8_issue(const TmGroup &tg, const Cursor &c, uns
 
 // Row r, part pt of a stage (kBlk = 64 / kU8Warps blocks from block kBlk pt; a part lies in
 // one atom) into the dense tile.
-__device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char *dense, const uint2 *tab_a,
-                                          const uint2 *tab_b, int meta_off, int r, int pt) {
+__device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char *dense, const uint4 *tab_a,
+                                          const uint4 *tab_b, int meta_off, int r, int pt) {
     constexpr int kBlk = 64 / kU8Warps;  // 8 or 4 blocks, 2 per 16-byte value chunk
     const int b0 = kBlk * pt, atom = b0 >> 3;
     uint32_t codes[kBlk / 2];
@@ -480,12 +480,12 @@ __device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char
         for (int h = 0; h < 2; ++h) {
             const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
             const uint32_t code = (codes[c] >> (16 * h)) & 0xFFFu;
-            const uint2 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
+            const uint4 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
             uint4 o;
             o.x = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
-            o.y = __byte_perm(__byte_perm(lo, 0u, sa.x >> 16), hi, sb.x >> 16);
-            o.z = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
-            o.w = __byte_perm(__byte_perm(lo, 0u, sa.y >> 16), hi, sb.y >> 16);
+            o.y = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
+            o.z = __byte_perm(__byte_perm(lo, 0u, sa.z), hi, sb.z);
+            o.w = __byte_perm(__byte_perm(lo, 0u, sa.w), hi, sb.w);
             const int b = (2 * cl + h) & 7;  // dense chunk within the atom
             *reinterpret_cast<uint4 *>(row + ((b ^ (r & 7)) << 4)) = o;
         }
@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
     const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
     unsigned char *ring = s_dyn_u8 + pad;
     const unsigned ring_s = dyn_s + pad;
-    uint2 *tab = reinterpret_cast<uint2 *>(ring + kD * kStage);  // A: entries [0, 64), B: [64, 128), x copies
+    uint4 *tab = reinterpret_cast<uint4 *>(ring + kD * kStage);  // A: entries [0, 64), B: [64, 128), x copies
     const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
     const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
     const unsigned exp0 = (unsigned)__cvta_generic_to_shared(&s_exp[0]);
@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
         const int r = threadIdx.x & (kUmRows - 1), pt = threadIdx.x >> 7;
         const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
         const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
-        const uint2 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
+        const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
         Cursor cc = sk_decode(grp, lo);
         unsigned acc_phase = 0u;
         bool failed = false;

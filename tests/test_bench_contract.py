@@ -48,3 +48,11 @@ def test_warmup_is_raised_to_three():
               "--ref-step-seconds", "0.1"], timeout=120)
     assert r.returncode == 0, r.stderr[-2000:]
     assert json.loads(r.stdout.strip().splitlines()[-1])["warmup"] == 3
+
+
+def test_serve_nm_is_only_for_the_serving_mode():
+    """--serve-nm repacks a workload for the serving benchmark only; the training step keeps
+    the workload's own pattern (its 4:8 state would not fit for the full stack)."""
+    r = _run(["--serve-nm", "4:8", "--workload", "tiny_2of4", "--steps", "1"], timeout=120)
+    assert r.returncode != 0
+    assert "--serve-nm applies to --mode sparse_linear" in r.stderr
