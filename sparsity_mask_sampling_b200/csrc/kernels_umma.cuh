@@ -12,13 +12,15 @@
 // 128 columns per pipeline stage (four MMAs of K = 32). Per stage the tensor memory
 // accelerator lands, on one mbarrier, the 128 x 64 box of compressed values and two kNTok x 64
 // boxes of x (both with the 128-byte swizzle, the K-major layout the MMA's shared-memory
-// descriptors name) and the 128 x 4 box of metadata words. Roles in a CTA of five warps:
+// descriptors name) and the 128 x 4 box of metadata words. Roles in a CTA of six warps:
 //   warp 4       the copy warp: refills a stage when the MMAs that read it have completed
 //                (their tcgen05.commit arrives on the stage's "empty" barrier);
-//   warps 0-3    per stage, each thread builds the metadata word of its tensor-memory lane
-//                and stores it with tcgen05.st; after a barrier thread 0 issues the four
-//                MMAs and commits them; at the end of a tile each warp reads its 32 rows of
-//                the accumulator with tcgen05.ld and stores y (or a partial tile).
+//   warps 0-3    per stage, each thread builds the metadata word of its tensor-memory lane,
+//                stores it with tcgen05.st and arrives on the stage's "metadata" barrier; at
+//                the end of a tile each warp reads its 32 rows of the accumulator with
+//                tcgen05.ld and stores y (or a partial tile);
+//   warp 5       the MMA warp: once all 128 metadata threads have arrived, one lane issues
+//                the stage's four MMAs and commits them.
 // Metadata in tensor memory, M = 128, 16-bit types, one column per MMA (the address an MMA
 // names is even; the descriptor's selector bits stay 0): lane
 // L = (m % 8) + 8 h + 16 (m / 16) holds, for row m (m % 16 < 8) and K half h, the four
@@ -47,7 +49,7 @@ namespace spl {
 
 constexpr int kUmRows = kBatchRows;          // MMA M: rows of a tile (128)
 constexpr int kUmStages = 3;
-constexpr int kUmThreads = 160;              // 4 MMA/epilogue warps + the copy warp
+constexpr int kUmThreads = 192;              // 4 metadata/epilogue warps, the copy warp, the MMA warp
 constexpr int kUmCtasPerSm = 2;              // resident CTAs the grid is sized for
 constexpr unsigned kUmTmemCols = 128;
 constexpr unsigned kUmMetaCol = 64;
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
     constexpr int kD = kUmStages, kStage = um_stage_bytes<kNTok>();
     constexpr uint32_t kIdesc = um_idesc<kNTok>();
     extern __shared__ unsigned char s_dyn_um[];
-    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_acc;
+    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_meta[kD], s_acc;
     __shared__ unsigned s_tmem;
     __shared__ volatile int s_abort;
     __shared__ int s_last;
@@ -193,11 +195,13 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
     const unsigned ring_s = dyn_s + pad;
     const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
     const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
+    const unsigned meta0 = (unsigned)__cvta_generic_to_shared(&s_meta[0]);
     const unsigned accb = (unsigned)__cvta_generic_to_shared(&s_acc);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kD; ++s) {
             mbar_init(full0 + 8 * s, 1u);
             mbar_init(empty0 + 8 * s, 1u);
+            mbar_init(meta0 + 8 * s, 128u);  // every metadata thread arrives once per stage
         }
         mbar_init(accb, 1u);
         s_abort = 0;
@@ -244,39 +248,23 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
             const int last = s + ((issued - 1 - s) / kD) * kD;  // the latest fill of stage s
             tm_wait(full0 + 8 * s, (last / kD) & 1);
         }
-    } else {
-        // ------------------------------------------------------------ MMA / epilogue warps
-        const unsigned tlane = tbase + ((unsigned)(32 * warp) << 16);
-        const int h = (lane >> 3) & 1;
-        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of the tile
-        const uint32_t esel = h ? 0x7632u : 0x5410u;
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA warp
         Cursor cc = sk_decode(grp, lo);
-        bool fresh = true;       // next MMA starts a tile piece (overwrites the accumulator)
-        unsigned acc_phase = 0u;
-        int mma_commits = 0;     // stages whose MMAs thread 0 has committed
-        bool failed = false;
+        bool fresh = true;  // the next MMA starts a tile piece (overwrites the accumulator)
+        int commits = 0;
         for (int f = 0; f < n; ++f) {
             const int s = f % kD;
-            const bool ok = um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort);
-            if (ok) {
-                tc_fence_after();
-                const unsigned char *meta = ring + s * kStage + kUmRows * 128 + 2 * um_xbox_bytes<kNTok>();
-                const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
-                const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
-                uint32_t e[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    e[j] = __byte_perm(a4[j] ? a4[j] : 0x44444444u, b4[j] ? b4[j] : 0x44444444u, esel);
-                tmem_st_meta(tlane + kUmMetaCol + 8 * s, e[0], e[1], e[2], e[3]);
-            }
-            tc_fence_before();
-            if (um_bar_or<128>(!ok)) {
-                failed = true;
+            if (!um_wait(meta0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                if (lane == 0 && !s_abort) {
+                    atomicOr(err, 1u);
+                    s_abort = 1;
+                }
                 break;
             }
             const SkOp &d = grp.d[cc.op];
             const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
-            if (threadIdx.x == 0) {
+            if (lane == 0) {
                 tc_fence_after();
                 const unsigned st = ring_s + s * kStage;
                 const uint64_t a0 = um_desc(st), b0 = um_desc(st + kUmRows * 128),
@@ -288,11 +276,54 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                 umma_commit(empty0 + 8 * s);
                 if (piece_end) umma_commit(accb);
             }
-            ++mma_commits;
-            fresh = false;
+            __syncwarp();
+            ++commits;
+            fresh = piece_end;
+            sk_advance(grp, cc);
+        }
+        if (commits > 0) {  // every MMA has completed (bounded) before the tensor memory is released
+            const int f = commits - 1;
+            tm_wait(empty0 + 8 * (f % kD), (f / kD) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ metadata / epilogue warps
+        const unsigned tlane = tbase + ((unsigned)(32 * warp) << 16);
+        const int h = (lane >> 3) & 1;
+        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of the tile
+        const uint32_t esel = h ? 0x7632u : 0x5410u;
+        Cursor cc = sk_decode(grp, lo);
+        unsigned acc_phase = 0u;
+        bool failed = false;
+        for (int f = 0; f < n; ++f) {
+            const int s = f % kD;
+            // A warp whose wait ran out stops working but keeps its place in the loop, so that
+            // it meets the others at the end of the tile, where all of them leave together.
+            if (!failed) {
+                if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                    tc_fence_after();
+                    const unsigned char *meta = ring + s * kStage + kUmRows * 128 + 2 * um_xbox_bytes<kNTok>();
+                    const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
+                    const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
+                    uint32_t e[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        e[j] = __byte_perm(a4[j] ? a4[j] : 0x44444444u, b4[j] ? b4[j] : 0x44444444u, esel);
+                    tmem_st_meta(tlane + kUmMetaCol + 8 * s, e[0], e[1], e[2], e[3]);
+                    tc_fence_before();
+                    mbar_arrive(meta0 + 8 * s);
+                } else {
+                    failed = true;
+                    if (lane == 0 && !s_abort) {
+                        atomicOr(err, 1u);
+                        s_abort = 1;
+                    }
+                }
+            }
+            const SkOp &d = grp.d[cc.op];
+            const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
             if (piece_end) {
                 // ---------------------------------------------------- epilogue of a tile piece
-                const bool acc_ok = um_wait(accb, acc_phase, &s_abort);
+                const bool acc_ok = !failed && um_wait(accb, acc_phase, &s_abort);
                 acc_phase ^= 1u;
                 if (um_bar_or<128>(!acc_ok)) {
                     failed = true;
@@ -302,7 +333,7 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                 float v[kNTok];
 #pragma unroll
                 for (int q = 0; q < kNTok / 16; ++q) tmem_ld16(tlane + 16 * q, v + 16 * q);
-                tc_fence_before();
+                tc_fence_before();  // these reads precede the next piece's first MMA (after its arrivals)
                 const int64_t a = d.chunk_begin + cc.tile * d.nch, b = a + d.nch;
                 const int64_t c1 = ((a + 1) * G - 1) / total, c2 = (b * G - 1) / total;
                 if (c1 == c2) {
@@ -333,21 +364,12 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
                         if (threadIdx.x == 0) tickets[c1] = 0u;
                     }
                 }
-                fresh = true;
             }
             sk_advance(grp, cc);
         }
-        if (failed) {
-            if (threadIdx.x == 0 && !s_abort) {
-                atomicOr(err, 1u);
-                s_abort = 1;
-            }
-            // MMAs already issued complete before the tensor memory is released: wait (bounded)
-            // for the commit of the latest issued stage
-            if (mma_commits > 0) {
-                const int f = mma_commits - 1;
-                tm_wait(empty0 + 8 * (f % kD), (f / kD) & 1);
-            }
+        if (failed && threadIdx.x == 0 && !s_abort) {
+            atomicOr(err, 1u);
+            s_abort = 1;
         }
     }
     tc_fence_before();
