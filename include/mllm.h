@@ -163,9 +163,11 @@ mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
  *   Limit: the array holds 2048 per-CTA partial sums (16,400 bytes, 256-byte aligned); a
  *     launch that would need more (a device with more than 2048 resident CTAs of the
  *     kernel) is rejected with MLLM_ERR_WORKSPACE before anything is enqueued.
- *   Set-up: the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture. Every GPU that loads the library holds the array until exit.
+ *   Set-up: every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress), so an address never outlives a device reset or a context;
+ *     the first call on a device may load the library's device code there, so make that
+ *     first call before any stream capture. Every GPU that loads the library holds the
+ *     array until exit.
  *   Sharing: all calls on a device share the one array and each call clears its ticket
  *     word before launching; calls whose work overlaps on the GPU (different streams
  *     without ordering between them) race on the array and must not be issued.

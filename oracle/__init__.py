@@ -14,8 +14,10 @@ Parity status per function (see the pins in tests/test_oracle_*.py):
   prior_init (deterministic mode, similarity, magnitude prior), prior_init_from_index,
   hard_pack, round_bf16, mask_diff, mask_stats, encode/decode_candidates, sparse_linear:
   pinned.
-  prior_init random mode: the N(0, 0.01) draws are pinned statistically (moments) and the
-  Eq.10 structure exactly; the individual Box-Muller bits are parity-by-tolerance only.
+  prior_init random mode: the N(0, 0.01) draws are pinned by their moments, each
+  Box-Muller pair against its two uniforms (radius and angle identities at fp64 rounding,
+  uniforms from the known-answer Philox), and the Eq.10 structure exactly. The GPU takes the
+  logarithm, sine and cosine in fp32, so GPU parity there is by tolerance (1e-6).
 """
 from __future__ import annotations
 

@@ -396,30 +396,22 @@ mllm_status launch_prior(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm, co
 // ------------------------------------------------------------------------ no-alloc scratch
 
 // Scratch of mllm_sample_fwd_noalloc: the ticket word at offset 0, per-CTA partial sums from
-// offset kWsPartialsOffset. A file-scope device array, so no allocation is ever made; its
-// device address is looked up once per device (host code cannot use the symbol itself).
+// offset kWsPartialsOffset. A file-scope device array, so no allocation is ever made. Host
+// code cannot use the symbol itself (it names a host-side stand-in), so the array's device
+// address on the current device is looked up with cudaGetSymbolAddress. That is done on every
+// call rather than cached: a device reset or a new context may place the module, and with it
+// the array, elsewhere, and a stale address would make the launch touch memory it does not own.
+// Once the module is loaded on a device the lookup is a host-side table query.
 constexpr int kNoallocMaxCtas = 2048;
 constexpr size_t kNoallocBytes = kWsPartialsOffset + sizeof(double) * kNoallocMaxCtas;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[kMaxDevices] = {};
-
 mllm_status noalloc_scratch(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_status(e);
-    if (dev < 0 || dev >= kMaxDevices) return MLLM_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_status(e);
-        if (!p) return MLLM_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    if (!p) return MLLM_ERR_CUDA;
+    *out = p;
     return MLLM_OK;
 }
 

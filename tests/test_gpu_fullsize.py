@@ -1,4 +1,4 @@
-"""Parity at the workloads' full sizes, in the launch configuration the benchmark times.
+"""Parity at the workloads' full sizes, in the launch configurations the benchmark times.
 
 Each workload is built at its real shapes with SamplerStack (one grouped launch per layer,
 global block ids as in the benchmark, up to 1.6e9 for the 32-layer stack) and driven
@@ -13,6 +13,12 @@ step depend only on those inputs; every checked step is thus compared on identic
 inputs, however far into the schedule (no input of the oracle ever comes from the GPU).
 The regulariser of each checked layer is checked against a property that holds at any
 size: the sum of squares of the layer's soft-masked weights.
+
+The *_fused_loop tests drive the benchmark's timed loop itself (forward of step 0, then per
+step one launch per layer of step t's backward + AdamW with step t+1's forward), so the
+kernel the benchmark reports is checked at the benchmark's sizes and grid: its CTAs walk
+many tiles each. There step t+1's soft-masked weights are compared with the oracle's
+forward from the oracle's own updated logits.
 """
 import numpy as np
 import pytest
@@ -182,11 +188,103 @@ def _run(orc, name, check_steps, layers=None, seed=0, rng_seed=0):
     torch.cuda.empty_cache()
 
 
-def test_gpt3_843m_layer_every_step_three_seeds(orc):
+def _check_next_forward(orc, stack, samples, t_next):
+    """X of step t_next (written by the previous launch) in the sampled blocks against the
+    oracle's forward from the oracle's own state, and every checked layer's regulariser
+    against the sum of squares of its soft-masked weights."""
+    w = stack.w
+    n, M = w.nm
+    hp = stack.hparams(t_next)
+    for s in samples:
+        X, _ = stack.XG(s.l, s.i)
+        got = X.view(-1, M)[s.idx_t].float().double().cpu().numpy()
+        fwd = orc.sample_fwd(n, M, s.W, s.pi, s.gids, hp.kappa, hp.tau, hp.seed, hp.step)
+        _tol.assert_x_close(got, fwd["x"], w.w_dtype, s.W)
+    for l in sorted({s.l for s in samples}):
+        r_x = sum(float((stack.XG(l, i)[0].double() ** 2).sum()) for i in range(len(w.matrices)))
+        r = float(stack.reg[l].item())
+        assert abs(r - r_x) <= 1e-3 * r, (l, r, r_x)
+
+
+def _run_fused(orc, name, check_steps, layers=None, seed=0, rng_seed=0):
+    """The benchmark's own loop (SamplerStack.forward_all, then one step_fused per step: per
+    layer one launch of step t's backward + AdamW and step t+1's forward), at full size.
+    Before a checked step the oracle's state is written into the sampled blocks; after it
+    the sampled logits and moments are compared with the oracle's AdamW on the oracle's
+    gradient, and the next step's soft-masked weights with the oracle's forward from the
+    oracle's updated logits (no oracle input comes from the GPU)."""
+    w = configs.WORKLOADS[name]
+    n, M = w.nm
+    torch.cuda.empty_cache()
+    stack = SamplerStack(w, DEV, rng_seed=rng_seed, x_per_layer=True)
+    stack.prior_init(seed=0)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(seed)
+    layers = layers if layers is not None else sorted({0, w.layers // 2, w.layers - 1})
+    samples = [Sample(stack, l, i, rng) for l in layers for i in range(len(w.matrices))]
+    _check_prior(orc, stack, samples)
+    for s in samples:
+        s.put_state(s.pi, s.m, s.v)
+    stack.forward_all(0)
+    torch.cuda.synchronize()
+    _check_next_forward(orc, stack, samples, 0)
+    f32 = np.float32
+    for t in range(max(check_steps) + 1):
+        if t not in check_steps:
+            stack.step_fused(t)
+            _advance(orc, stack, samples, t)
+            continue
+        for s in samples:
+            s.put_state(s.pi, s.m, s.v)
+        stack.step_fused(t)
+        torch.cuda.synchronize()
+        hp = stack.hparams(t)
+        for s in samples:
+            g_ref, scale = orc.sample_bwd(n, M, s.W, s.G, s.pi, s.gids, hp.kappa, hp.tau, hp.lambda_, hp.seed,
+                                          hp.step)
+            p_ref, m_ref, v_ref = orc.adamw(s.pi, s.m, s.v, g_ref, f32(hp.lr), f32(hp.beta1), f32(hp.beta2),
+                                            f32(hp.eps), f32(hp.weight_decay), hp.adam_step)
+            floor = _tol.grad_floor(s.W, s.G, hp.kappa, hp.tau, hp.lambda_)
+            pe = _tol.assert_logits_close(s.mb.logits[s.idx_t].cpu().numpy(), p_ref)
+            print(f"{name} step {t} layer {s.l} matrix {s.i}: worst per-element relative error of the "
+                  f"updated logits {pe:.3g}")
+            _tol.assert_moments_close(s.mb.adam_m[s.idx_t].cpu().numpy(), s.mb.adam_v[s.idx_t].cpu().numpy(),
+                                      m_ref, v_ref, g_ref, 1e-4 * scale + floor, f32(hp.beta1), f32(hp.beta2))
+            s.pi, s.m, s.v = p_ref.astype(np.float32), m_ref.astype(np.float32), v_ref.astype(np.float32)
+        _check_next_forward(orc, stack, samples, t + 1)
+    _check_pack(orc, stack, samples)
+    del stack
+    torch.cuda.empty_cache()
+
+
+def test_gpt3_843m_layer_every_step_all_seeds(orc):
     """GPT-3-843M-shaped layer, tau 4 -> 0.05 and kappa 100 -> 500 over 10 steps, every step
-    checked; noise seeds 1, 5 and 10 of the workload's ten runs."""
-    for rs in (1, 5, 10):
+    checked, for each of the workload's ten runs (noise seeds 1..10)."""
+    for rs in configs.WORKLOADS["gpt3_843m_layer_2of4"].seeds:
         _run(orc, "gpt3_843m_layer_2of4", check_steps=set(range(10)), rng_seed=rs, seed=rs)
+
+
+def test_gpt3_843m_layer_fused_loop(orc):
+    """The GPT-3-843M-shaped layer through the benchmark's fused loop, every step checked."""
+    _run_fused(orc, "gpt3_843m_layer_2of4", check_steps=set(range(10)), rng_seed=3, seed=3)
+
+
+def test_llama2_7b_layer_fused_loop(orc):
+    """One LLaMA-2-7B layer (50.6 M blocks) through the benchmark's fused loop: steps 0, 50
+    and 99 of its 100-step schedule checked (logits, moments, next X, regulariser)."""
+    _run_fused(orc, "llama2_7b_layer_2of4", check_steps={0, 50, 99})
+
+
+def test_llama2_7b_full_stack_fused_loop(orc):
+    """All 32 layers in the benchmark's fused loop (its exact launches: 1,619,001,344 blocks,
+    logits, moments and every layer's next-step X resident): the first, a middle and the
+    last layer checked at steps 0 and 9."""
+    _run_fused(orc, "llama2_7b_stack_2of4", check_steps={0, 9})
+
+
+def test_general_4of8_fused_loop(orc):
+    """4:8 through the fused loop (the call runs its two kernels), steps 0 and 49 checked."""
+    _run_fused(orc, "general_4of8", check_steps={0, 49})
 
 
 def test_llama2_7b_layer(orc):

@@ -445,3 +445,53 @@ def test_transfer_prior_round_trip(orc):
     mllm_prior_init_from_mask([d.mb], (2, 4), [general], 3.0, 0.0, 0)
     torch.cuda.synchronize()
     assert torch.equal(torch.argmax(d.mb.logits, 1).to(torch.uint8), general)
+
+
+# ------------------------------------------------------------------------------ grid stride
+
+@pytest.mark.parametrize("nm,shape", [((2, 4), (4096, 4096)), ((4, 8), (1024, 4096))])
+def test_fused_step_walks_many_tiles_per_cta(orc, ws, nm, shape):
+    """One matrix with far more tiles than the persistent grid has CTAs (2:4: 4096 x 4096 =
+    2.1 M pairs = 8,192 tiles of 256 pairs against 148 SMs x 3 CTAs; 4:8: 524 K blocks =
+    4,096 tiles of 128), so every CTA walks many tiles and carries its regulariser partial
+    across them. The fused call equals the two calls in sequence bit for bit; on a strided
+    sample of blocks its backward matches the oracle on identical inputs and its next-step
+    soft-masked weights match the oracle's forward from the oracle's updated logits; the
+    regulariser equals the sum of squares of the soft-masked weights."""
+    n, m = nm
+    c = Case(nm, *shape, seed=90, offset=3 * 2**32 + 11)
+    hp = Hparams(kappa=300.0, tau=0.5, lambda_=1e-5, lr=5e-4, adam_step=7, step=6, seed=0xD15C)
+    hp_next = Hparams(kappa=310.0, tau=0.45, step=7, seed=0xD15C)
+    mllm_sample_bwd_adam([c.mb], nm, hp)
+    reg_a = torch.zeros(1, dtype=torch.float64, device=DEV)
+    mllm_sample_fwd([c.mb], nm, hp_next, reg_a, ws)
+    torch.cuda.synchronize()
+    seq = [t.clone() for t in (c.mb.logits, c.mb.adam_m, c.mb.adam_v, c.mb.grad_logits, c.mb.X, c.mb.soft_mask)]
+    c.reset()
+    c.mb.X.zero_()
+    c.mb.soft_mask.zero_()
+    reg_b = torch.zeros(1, dtype=torch.float64, device=DEV)
+    mllm_sample_bwd_adam_fwd([c.mb], nm, hp, hp_next, reg_b, ws)
+    torch.cuda.synchronize()
+    for a, b in zip((c.mb.logits, c.mb.adam_m, c.mb.adam_v, c.mb.grad_logits, c.mb.X, c.mb.soft_mask), seq):
+        assert torch.equal(a, b)
+    assert abs(reg_a.item() - reg_b.item()) <= 1e-12 * abs(reg_a.item())
+    r_x = float((c.mb.X.double() ** 2).sum())
+    assert abs(reg_b.item() - r_x) <= 1e-3 * r_x
+    idx = np.arange(0, c.B, 13 if m == 4 else 7)
+    it = torch.from_numpy(idx).to(DEV)
+    W, G = c.Wv[idx], c.Gv[idx]
+    pi, m0, v0 = c.pi.numpy()[idx], c.m0.numpy()[idx], c.v0.numpy()[idx]
+    gids = c.gids[idx]
+    g_ref, scale = orc.sample_bwd(n, m, W, G, pi, gids, hp.kappa, hp.tau, hp.lambda_, hp.seed, hp.step)
+    floor = _tol.grad_floor(W, G, hp.kappa, hp.tau, hp.lambda_)
+    _tol.assert_grad_close(c.mb.grad_logits[it].cpu().numpy(), g_ref, scale, floor)
+    f32 = np.float32
+    p_ref, m_ref, v_ref = orc.adamw(pi, m0, v0, g_ref, f32(hp.lr), f32(hp.beta1), f32(hp.beta2), f32(hp.eps),
+                                    f32(hp.weight_decay), hp.adam_step)
+    _tol.assert_logits_close(c.mb.logits[it].cpu().numpy(), p_ref)
+    _tol.assert_moments_close(c.mb.adam_m[it].cpu().numpy(), c.mb.adam_v[it].cpu().numpy(), m_ref, v_ref,
+                              g_ref, 1e-4 * scale + floor, f32(hp.beta1), f32(hp.beta2))
+    fwd = orc.sample_fwd(n, m, W, p_ref.astype(np.float32), gids, hp_next.kappa, hp_next.tau, hp_next.seed,
+                         hp_next.step)
+    _tol.assert_x_close(c.mb.X.view(-1, m)[it].float().double().cpu().numpy(), fwd["x"], "bf16", W)

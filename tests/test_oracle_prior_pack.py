@@ -113,6 +113,51 @@ def test_random_init_is_normal_with_std_001(orc, n, m):
     np.testing.assert_array_equal(pi, pi2)
 
 
+def _init_uniforms(orc, C, seed, gids):
+    """u_c = (2k+1) 2^-22 of the reserved init step (0xFFFFFFFF), k the 21-bit field c%6 of
+    Philox(counter (gid lo, gid hi, 0xFFFFFFFF, c//6), key (seed lo, seed hi)), computed
+    here from the known-answer-pinned Philox and big-integer slicing of its 128 bits."""
+    u = np.zeros((len(gids), C))
+    for b, gid in enumerate(int(g) for g in gids):
+        for grp in range((C + 5) // 6):
+            words = orc.philox4x32_10([gid & 0xFFFFFFFF, gid >> 32, 0xFFFFFFFF, grp],
+                                      [seed & 0xFFFFFFFF, seed >> 32])
+            big = sum(int(words[i]) << (32 * i) for i in range(4))
+            for f in range(6):
+                c = 6 * grp + f
+                if c < C:
+                    u[b, c] = (2 * ((big >> (21 * f)) & ((1 << 21) - 1)) + 1) / 2.0 ** 22
+    return u
+
+
+@pytest.mark.parametrize("n,m", NM)
+def test_box_muller_pairs_follow_their_uniforms(orc, n, m):
+    """Each pair (2p, 2p+1) of the initial N(0,1) draws is one Box-Muller transform of the
+    reserved-step uniforms: radius from u_2p, angle from u_2p+1, so
+    n_2p^2 + n_2p+1^2 = -2 ln u_2p and atan2(n_2p+1, n_2p) = 2 pi u_2p+1 (mod 2 pi), to fp64
+    rounding. A cosine taken for both members, a reused radius or angle, swapped roles of the
+    two uniforms or a pair drawn from the wrong candidates all fail here, although they keep
+    every one-dimensional moment; the two members of a pair are uncorrelated."""
+    C = orc.num_candidates(n, m)
+    nb = 1500 if m == 4 else 150
+    seed = 0x5EED_0000_0000_0007
+    gids = np.arange(nb, dtype=np.uint64) * np.uint64(7919) + np.uint64(2**33 + 12345)
+    # no prior (index >= C) and init_std 1: the logits are the draws themselves
+    z, _ = orc.prior_init_from_index(n, m, gids, np.full(nb, C, np.int32), 3.0, 1.0, seed)
+    u = _init_uniforms(orc, C, seed, gids)
+    P = C // 2
+    a, b = z[:, 0:2 * P:2], z[:, 1:2 * P:2]
+    u1, u2 = u[:, 0:2 * P:2], u[:, 1:2 * P:2]
+    np.testing.assert_allclose(a * a + b * b, -2.0 * np.log(u1), rtol=1e-13, atol=0)
+    ang = np.mod(np.arctan2(b, a), 2 * np.pi)
+    d = np.abs(ang - 2 * np.pi * u2)
+    d = np.minimum(d, 2 * np.pi - d)
+    assert d.max() < 1e-12, d.max()
+    # pair members uncorrelated (a mix-up like n_2p+1 = n_2p would give E = 1)
+    prod = (a * b).ravel()
+    assert abs(prod.mean()) < 5.0 / math.sqrt(prod.size)
+
+
 @pytest.mark.parametrize("n,m", NM)
 def test_prior_bias_scales_with_block_std(orc, n, m):
     """Eq.10: pi(alpha) - pi(0) = alpha * sigma(pi(0)) * sim, sigma the spread of the block's

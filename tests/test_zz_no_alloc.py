@@ -5,17 +5,20 @@ forbids cudaMalloc/cudaFree once running, or a runtime that only passes the step
 cannot provide the workspace that mllm_sample_fwd needs for its regulariser reduction. The
 no-alloc entry point keeps that scratch in a fixed array inside the library. Here it is
 called through the C ABI twice in a row, and each call's outputs are compared with the
-workspace-based entry point on the same inputs, within the parity tolerances of the tests
-(regulariser 1e-3 relative, soft-masked weights within 1 bf16 ulp).
+workspace-based entry point on the same inputs. Both entry points launch the same kernels
+with the same grids and reduce in the same order, so the soft-masked weights and the
+regulariser must be identical bit for bit (any wrong partial slot or stale ticket would
+show); this is stricter than the oracle parity tolerances (1e-3 relative, 1 bf16 ulp). A
+layer of more than 16 matrices is split into several launches, which exercises the paths
+only the no-alloc call has between launches: the ticket cleared before each launch and the
+later launches adding to the regulariser.
 
 This file is named to be collected last, so a run that stops at the first failure has run
 every other test before it. It needs nothing from the other test files and passes alone.
 """
-import numpy as np
 import pytest
 import torch
 
-import _tol
 from sparsity_mask_sampling_b200 import (Hparams, MllmError, alloc_matrix, inputs, mllm_sample_fwd,
                                          mllm_sample_fwd_noalloc, mllm_workspace_bytes)
 from sparsity_mask_sampling_b200.build import build
@@ -42,7 +45,9 @@ def _layer(nm, shapes, seed):
 
 
 @pytest.mark.parametrize("nm,shapes", [((2, 4), [(512, 1024), (77, 36), (1, 4)]),
-                                       ((4, 8), [(256, 512), (3, 16)])])
+                                       ((4, 8), [(256, 512), (3, 16)]),
+                                       ((2, 4), [(8, 16)] * 20),
+                                       ((4, 8), [(8, 16), (5, 24)] * 9)])
 def test_noalloc_forward_matches_workspace_forward_twice(nm, shapes):
     mats = _layer(nm, shapes, seed=7)
     ws = torch.zeros(mllm_workspace_bytes(), dtype=torch.uint8, device=DEV)
@@ -56,10 +61,9 @@ def test_noalloc_forward_matches_workspace_forward_twice(nm, shapes):
         reg = torch.full((1,), -1.0, dtype=torch.float64, device=DEV)
         mllm_sample_fwd_noalloc(mats, nm, hp, reg)
         torch.cuda.synchronize()
-        _tol.assert_reg_close(reg.item(), reg_ref.item())
+        assert reg.item() == reg_ref.item()
         for m, xr in zip(mats, x_ref):
-            W = m.W.float().double().cpu().numpy()
-            _tol.assert_x_close(m.X.float().double().cpu().numpy(), xr.float().double().cpu().numpy(), "bf16", W)
+            assert torch.equal(m.X, xr)
 
 
 def test_noalloc_requires_regulariser_output():
