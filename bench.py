@@ -12,6 +12,9 @@ measured copy bandwidth.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--loop fused|separate]
                   [--impl reference]
+  python bench.py --mode masked_linear [--tokens T] [--steps K]
+      (the sampler inside the frozen network's linear layers of a LLaMA-2-7B layer: fused
+       mllm_masked_linear_* calls against the sampler calls + cuBLAS GEMMs)
   python bench.py --mode sparse_linear [--workload NAME] [--serve-nm 2:4|4:8] [--steps K --warmup W]
       (serving leg: the workload's matrices as packed hard masks, y = x W*^T per call for
        1, 8, 16, 32 and 64 tokens, against dense cuBLAS; one JSON line)
@@ -225,6 +228,14 @@ def gpu_arm(args, w):
 
     blocks_per_layer = w.blocks_per_layer()
     fb = BYTES[w.C]
+    stack_blocks = stack.blocks
+
+    # the other workloads, each at its full shape: every call timed on its own
+    if not args.no_configs:
+        del stack
+        torch.cuda.empty_cache()
+        extras["configs"] = config_legs(args, dev, hbm_peak, cpu=(world == 1 and rank == 0 and not args.no_cpu_baseline))
+        extras["masked_linear"] = masked_linear_leg(dev, hbm_peak, reps=args.config_reps)
 
     def kstats(ms_list, bpb, name):
         avg = float(np.mean(ms_list))
@@ -246,8 +257,8 @@ def gpu_arm(args, w):
         traffic = traffic_from_profile("bwd", w)
     kernels["fwd_standalone"] = kstats(ref["fwd"], fb["fwd"], "fwd_kernel (first step of a loop)")
     kernels["bwd_adam_standalone"] = kstats(ref["bwd"], fb["bwd"], "bwd_adam_kernel (unfused)")
-    kernels["pack_once"] = once_stats(pack_ms, stack.blocks, fb["pack"], hbm_peak)
-    kernels["prior_init_once"] = once_stats(init_ms, stack.blocks, fb["init"], hbm_peak)
+    kernels["pack_once"] = once_stats(pack_ms, stack_blocks, fb["pack"], hbm_peak)
+    kernels["prior_init_once"] = once_stats(init_ms, stack_blocks, fb["init"], hbm_peak)
     roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved_gbs"], "peak": hbm_peak,
                 "unit": "GB/s", "frac": round(dom["achieved_gbs"] / hbm_peak, 4), "peak_kind": peak_kind,
                 "bytes_per_block": dom["bytes_per_block"], "traffic": traffic}
@@ -545,6 +556,228 @@ def kernel_source_sha(nm=(2, 4)):
     return h.hexdigest()
 
 
+# ------------------------------------------------------------------------------ other workloads
+
+CONFIG_LEGS = ("tiny_2of4", "gpt3_843m_layer_2of4", "llama2_7b_layer_2of4", "general_4of8")
+
+
+def config_legs(args, dev, peak, cpu=True):
+    """Every workload other than the headline stack, at its full shape: the forward, the
+    backward + AdamW, the fused step call (backward + AdamW of step t with the forward of
+    step t+1) and the hard pack, each timed alone as the median of `reps` calls with CUDA
+    events, L2 flushed (a 1 GB write) before every call. The tiny workload is reported as
+    latency (us per call; no roofline claim at 2,048 blocks). Each workload carries the
+    oracle's rates on the host cores for the same calls (all threads and 1 thread)."""
+    from sparsity_mask_sampling_b200 import configs
+
+    out = {}
+    for name in CONFIG_LEGS:
+        w = configs.WORKLOADS[name]
+        out[name] = config_leg(w, dev, peak, reps=args.config_reps)
+        if cpu:
+            out[name]["cpu_baseline"] = cpu_kernel_rates(w, seconds=args.config_cpu_seconds)
+    return out
+
+
+def config_leg(w, dev, peak, reps=10):
+    import torch
+    import sparsity_mask_sampling_b200 as pkg
+    from sparsity_mask_sampling_b200 import buffers
+    from sparsity_mask_sampling_b200.stack import SamplerStack
+
+    stack = SamplerStack(w, dev, x_per_layer=True)
+    stack.prior_init(seed=0)
+    for mats in stack.bufs:
+        for mb, m in zip(mats, w.matrices):
+            (vs, (ms, mdt)) = buffers.pack_shapes(m.rows, m.cols, w.nm)
+            mb.pack_values = torch.empty(vs, dtype=mb.W.dtype, device=dev)
+            mb.pack_meta = torch.empty(ms, dtype=mdt, device=dev)
+            mb.cand_idx = torch.empty(m.rows * m.cols // w.nm[1], dtype=torch.uint8, device=dev)
+    stack.rebuild_views()
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    L = w.layers
+    t = 5  # a step inside the schedule
+    hp, hpn = stack.hparams(t).to_c(), stack.hparams(t + 1).to_c()
+    calls = {
+        "fwd": lambda: [stack.forward(l, hp) for l in range(L)],
+        "bwd_adam": lambda: [stack.backward(l, hp) for l in range(L)],
+        "bwd_adam_fwd": lambda: [stack.backward_forward(l, hp, hpn) for l in range(L)],
+        "pack": lambda: [pkg.mllm_hard_pack(stack.view(l), w.nm) for l in range(L)],
+    }
+    fb = BYTES[w.C]
+    bpb = {"fwd": fb["fwd"], "bwd_adam": fb["bwd"], "bwd_adam_fwd": fb["fused"], "pack": fb["pack"]}
+    if w.w_dtype == "f32":  # fp32 W, X and G: 8 more bytes per block for each of them
+        bpb = {"fwd": 56, "bwd_adam": 176, "bwd_adam_fwd": 192, "pack": 50.5}
+    blocks = stack.blocks
+    res = {"blocks": blocks, "nm": f"{w.nm[0]}:{w.nm[1]}", "reps": reps,
+           "timing": "median of the reps, each call alone on the device after a 1 GB L2 flush"}
+    for k, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        ms_list = []
+        for _ in range(reps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            ms_list.append(s.elapsed_time(e))
+        ms = float(np.median(ms_list))
+        gbs = blocks * bpb[k] / (ms / 1e3) / 1e9
+        ent = {"ms": round(ms, 4), "blocks_per_s": blocks / (ms / 1e3), "bytes_per_block": bpb[k],
+               "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        if blocks < 1e5:
+            ent = {"us": round(ms * 1e3, 2), "blocks_per_s": blocks / (ms / 1e3), "bytes_per_block": bpb[k],
+                   "note": "latency: launch-bound at this size, no roofline claim"}
+        res[k] = ent
+    del stack, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def masked_linear_leg(dev, peak, tokens=256, reps=10):
+    """The sampler inside the frozen network's linear layers (s.3.2 "Frozen LLM Backbone"), on
+    the LLaMA-2-7B layer's seven matrices at `tokens` tokens (seeded synthetic activations A
+    and output gradients dY, bf16). Fused: mllm_masked_linear_fwd (Y = A X^T with X made in
+    shared memory) and mllm_masked_linear_bwd_adam (G = dY^T A in tensor memory, then the
+    logits' backward + AdamW from it). Unfused, on the same box: mllm_sample_fwd writes X, then
+    cuBLAS Y = A X^T (torch F.linear); cuBLAS G = dY^T A (bf16 out), then mllm_sample_bwd_adam
+    reads it. Each call timed alone (median of reps, CUDA events, L2 flushed before each)."""
+    import torch
+    import torch.nn.functional as F
+    import sparsity_mask_sampling_b200 as pkg
+    from sparsity_mask_sampling_b200 import configs, inputs
+
+    w = configs.WORKLOADS["llama2_7b_layer_2of4"]
+    mats, ios_f, ios_b, As, dYs = [], [], [], [], []
+    off = 0
+    for i, m in enumerate(w.matrices):
+        W = inputs.weights(m.rows, m.cols, "bf16", 0.02, seed=100 + i, outlier_frac=0.01, device=dev)
+        mb = pkg.alloc_matrix(W, (2, 4), off, fwd=True, bwd=True)
+        mb.logits.copy_(inputs.logits(m.rows * m.cols // 4, 6, 0.02, seed=200 + i, device=dev))
+        A = inputs.weights(tokens, m.cols, "bf16", 1.0, seed=300 + i, device=dev)
+        dY = inputs.upstream_grad(tokens, m.rows, "bf16", 1e-3, seed=400 + i, device=dev)
+        y = torch.empty(tokens, m.rows, dtype=torch.float32, device=dev)
+        mats.append(mb)
+        ios_f.append((A, y, None))
+        ios_b.append((A, None, dY))
+        As.append(A)
+        dYs.append(dY)
+        off += m.rows * m.cols // 4
+    arr = pkg.MatrixArray(mats)
+    fused_mats = [pkg.MatrixBuffers(W=mb.W, logits=mb.logits, adam_m=mb.adam_m, adam_v=mb.adam_v,
+                                    block_offset=mb.block_offset) for mb in mats]
+    farr = pkg.MatrixArray(fused_mats)
+    mlws = pkg.masked_linear_workspace(dev)
+    ws = torch.zeros(pkg.mllm_workspace_bytes(), dtype=torch.uint8, device=dev)
+    reg = torch.zeros(1, dtype=torch.float64, device=dev)
+    hp = pkg.Hparams(kappa=300.0, tau=1.0, lambda_=1e-5, lr=5e-4, adam_step=5, step=4, seed=0)
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(reps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            out.append(s.elapsed_time(e))
+        return float(np.median(out))
+
+    def unfused_fwd():
+        pkg.mllm_sample_fwd(arr, (2, 4), hp, reg, ws)
+        for mb, (A, y, _) in zip(mats, ios_f):
+            y.copy_(F.linear(A, mb.X))
+
+    def unfused_bwd():
+        for mb, A, dY in zip(mats, As, dYs):
+            torch.matmul(dY.t(), A, out=mb.G)
+        pkg.mllm_sample_bwd_adam(arr, (2, 4), hp)
+
+    t = {
+        "fused_fwd_ms": timed(lambda: pkg.mllm_masked_linear_fwd(farr, ios_f, (2, 4), tokens, hp, mlws, reg)),
+        "unfused_fwd_ms": timed(unfused_fwd),
+        "fused_bwd_adam_ms": timed(lambda: pkg.mllm_masked_linear_bwd_adam(farr, ios_b, (2, 4), tokens, hp, mlws)),
+        "unfused_bwd_adam_ms": timed(unfused_bwd),
+    }
+    blocks = w.blocks_per_layer()
+    flops = 2.0 * tokens * blocks * 4  # one product per weight per token
+    res = {"workload": w.name, "tokens": tokens, "blocks": blocks,
+           "timing": "median of the reps, each call alone after a 1 GB L2 flush"}
+    for k, v in t.items():
+        res[k] = round(v, 4)
+    res["fwd_speedup"] = round(t["unfused_fwd_ms"] / t["fused_fwd_ms"], 3)
+    res["bwd_adam_speedup"] = round(t["unfused_bwd_adam_ms"] / t["fused_bwd_adam_ms"], 3)
+    # HBM bytes per block and step. Fused: forward reads W + logits (32), backward reads W and
+    # logits/m/v and writes logits/m/v (152). Unfused as timed here: sampler forward 40 + the
+    # GEMM's read of X 8, the GEMM's write of G 8 + sampler backward 160. (A loop built on the
+    # sampler's own fused step, which reads W and the logits once per step, moves 168 + 16 =
+    # 184, as the fused layer does; what the fused layer saves there is the X and G buffers.)
+    res["hbm_bytes_per_block_per_step"] = {"fused": 32 + 152, "unfused_as_timed": 48 + 168,
+                                           "unfused_with_fused_sampler_step": 168 + 16}
+    res["bytes_saved_per_block_per_step"] = 48 + 168 - (32 + 152)
+    res["buffers_not_held_gb_per_layer"] = round(blocks * 16 / 1e9, 3)  # X and G, bf16
+    res["fused_fwd_tflops"] = round(flops / (t["fused_fwd_ms"] / 1e3) / 1e12, 1)
+    res["fused_fwd_gbs"] = round(blocks * 32 / (t["fused_fwd_ms"] / 1e3) / 1e9, 1)
+    res["fused_bwd_adam_gbs"] = round(blocks * 152 / (t["fused_bwd_adam_ms"] / 1e3) / 1e9, 1)
+    del mats, fused_mats, arr, farr, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def _rate(fn, samples, threads):
+    start = time.perf_counter()
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(fn, samples))
+    return time.perf_counter() - start
+
+
+def cpu_kernel_rates(w, seconds=1.0):
+    """The oracle's forward, backward + AdamW and hard pack on the host cores (all threads,
+    then 1 thread), each on a bounded random sample of the workload's blocks sized to take
+    about `seconds`; blocks/s per call."""
+    import oracle as orc
+
+    orc.build()
+    n, m = w.nm
+    t = 5
+    kappa, tau = w.kappa_at(t % w.steps), w.tau_at(t % w.steps)
+
+    def fwd(s):
+        gids, W, G, pi = s
+        orc.sample_fwd(n, m, W, pi, gids, kappa, tau, 0, t)
+
+    def bwd(s):
+        gids, W, G, pi = s
+        g, _ = orc.sample_bwd(n, m, W, G, pi, gids, kappa, tau, w.lam, 0, t)
+        z = np.zeros_like(g)
+        orc.adamw(pi, z, z, g, w.lr, 0.9, 0.999, 1e-8, w.weight_decay, t + 1)
+
+    def pack(s):
+        gids, W, G, pi = s
+        raw = np.ascontiguousarray(W.astype(np.float32)).view(np.uint32).reshape(-1, 8 * m)
+        orc.hard_pack(n, m, raw, pi)
+
+    threads = os.cpu_count() or 1
+    out = {"cores": threads, "kind": "oracle", "unit": "blocks/s"}
+    for name, fn in (("fwd", fwd), ("bwd_adam", bwd), ("pack", pack)):
+        probe = [make_sample(w, 2048, seed=31)]
+        dt = max(_rate(fn, probe, 1), 1e-6)
+        per_thread = int(min(max(2048 / dt * seconds, 2048), 4e6)) // 8 * 8
+        samples = [make_sample(w, per_thread, seed=41 + i) for i in range(threads)]
+        dt_n = _rate(fn, samples, threads)
+        dt_1 = _rate(fn, samples[:1], 1)
+        out[name] = {"value": per_thread * threads / dt_n, "value_1_core": per_thread / dt_1}
+    out["sample"] = (f"per call and thread count, random blocks of {w.name} (same seeded distributions), "
+                     f"sized for about {seconds:g} s per thread")
+    return out
+
+
 # ------------------------------------------------------------------------------ CPU (oracle)
 
 def make_sample(w, n_blocks, seed=0):
@@ -691,7 +924,7 @@ def sparse_linear_arm(args, w):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--mode", default="train", choices=["train", "sparse_linear"])
+    ap.add_argument("--mode", default="train", choices=["train", "sparse_linear", "masked_linear"])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -701,6 +934,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' per-call timings")
+    ap.add_argument("--tokens", type=int, default=256, help="--mode masked_linear: tokens per call (1-256)")
+    ap.add_argument("--config-reps", type=int, default=10)
+    ap.add_argument("--config-cpu-seconds", type=float, default=1.0)
     ap.add_argument("--serve-nm", default=None, choices=["2:4", "4:8"],
                     help="--mode sparse_linear: pack the workload's matrices with this pattern instead of its own")
     args = ap.parse_args()
@@ -718,6 +955,16 @@ def main():
         w = dataclasses.replace(w, nm=nm, name=f"{w.name} packed {args.serve_nm}")
     if args.mode == "sparse_linear":
         out = sparse_linear_arm(args, w)
+    elif args.mode == "masked_linear":
+        import torch
+
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(dev)
+        r = masked_linear_leg(dev, peaks()[0], tokens=args.tokens, reps=args.steps)
+        out = {"metric": "masked linear layer, fused vs sampler + cuBLAS (ms per call)", "mode": "masked_linear",
+               "value": r["fused_fwd_ms"] + r["fused_bwd_adam_ms"], "unit": "ms", "higher_is_better": False,
+               "n_gpus": 1, "steps": args.steps, "dtype": "bf16 operands, fp32 accumulation", "data": "synthetic",
+               "config": {"workload": r["workload"], "tokens": r["tokens"]}, "result": r}
     elif args.impl == "reference":
         out = reference_arm(args, w)
     else:

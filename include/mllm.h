@@ -197,12 +197,56 @@ mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_n
  * (optional) step t+1's soft mask, and reg_sum_out (optional, with the workspace as in
  * mllm_sample_fwd) step t+1's regulariser. A loop then calls mllm_sample_fwd once for the
  * first step and this call for every step after it. Results are identical to the two calls
- * in sequence. 4:8 runs them as two launches; 2:4 is one fused launch.
+ * in sequence. One launch per group of matrices for both patterns.
  * Reads W, G. hp is validated as for mllm_sample_bwd_adam, hp_next as for mllm_sample_fwd. */
 mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
                                      const mllm_hparams *hp, const mllm_hparams *hp_next,
                                      double *reg_sum_out, void *workspace, size_t workspace_bytes,
                                      void *stream);
+
+/* Activations of one matrix's linear layer for the mllm_masked_linear_* calls (device
+ * memory, caller-owned, 16-byte aligned). */
+typedef struct {
+    const void *x;  /* [tokens, cols] bf16: the layer's input A, row-major                  */
+    float *y;       /* [tokens, rows] fp32: the layer's output Y = A X^T (forward; overwritten) */
+    const void *dy; /* [tokens, rows] bf16: dL/dY, the gradient of the output (backward)     */
+} mllm_linear_io;
+
+/* The sampler's forward inside the frozen network's linear layer (s.3.2 "Frozen LLM
+ * Backbone": every linear layer multiplies by the soft-masked weight; s.3.4 Eq.5-Eq.8):
+ *   Y[t, r] = sum_k A[t, k] X[r, k],  X = W (.) M in bf16, exactly the X of mllm_sample_fwd
+ * (same noise, same arithmetic, bit for bit), for 1 <= tokens <= 256, with the products on the
+ * tensor cores (bf16 operands, fp32 accumulation). X is made tile by tile in shared memory
+ * and never written to global memory (unless X_out is non-NULL, for inspection; soft_mask_out
+ * likewise). reg_sum_out (optional) receives the regulariser sum of the call as in
+ * mllm_sample_fwd. Matrix i uses io[i]; its W is bf16, cols % 64 == 0; 2:4 only
+ * (MLLM_ERR_UNSUPPORTED otherwise). workspace: mllm_masked_linear_workspace_bytes() bytes,
+ * zero-filled before its first use; every call leaves it zero-filled (partial tiles of rows
+ * split between CTAs, completion tickets, the regulariser's partials and an error word -- the
+ * uint32 at byte offset mllm_masked_linear_workspace_bytes() - 16 -- that a call sets if one of
+ * its bounded waits ran out, in which case its outputs are invalid; never expected). Calls sharing a workspace must
+ * be stream-ordered. Deterministic for a given device. Reads W, logits, x. */
+mllm_status mllm_masked_linear_fwd(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats,
+                                   mllm_nm nm, int32_t tokens, const mllm_hparams *hp, double *reg_sum_out,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* The weight side of the same layer's backward fused with the logits' backward and AdamW
+ * (s.3.2 "Frozen LLM Backbone": the frozen weights take no update, the gradient reaching the
+ * soft-masked weight goes to the logits; s.3.4 Eq.8, Algorithm 1 step 2): per matrix
+ *   G[r, k] = sum_t dY[t, r] A[t, k]     (dL/dX of Y = A X^T; tensor cores, fp32 accumulation)
+ * and then, per block, exactly mllm_sample_bwd_adam with G in fp32 in place of the upstream
+ * gradient: the noise of hp's step recomputed, dpi through Eq.7 and Eq.6 with the
+ * regulariser's term, AdamW on logits, adam_m, adam_v in place (grad_logits_out receives dpi
+ * when non-NULL). G is formed tile by tile in tensor and shared memory and never written to
+ * global memory. io[i].x and io[i].dy are the forward's activations and dL/dY; 1 <= tokens
+ * <= 256; W bf16, cols % 64 == 0, rows % 8 == 0, 2:4 only (MLLM_ERR_UNSUPPORTED otherwise).
+ * workspace as for mllm_masked_linear_fwd (only its error word is used here). Reads W, x, dy. */
+mllm_status mllm_masked_linear_bwd_adam(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats,
+                                        mllm_nm nm, int32_t tokens, const mllm_hparams *hp, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of the mllm_masked_linear_* calls (independent of sizes). */
+size_t mllm_masked_linear_workspace_bytes(void);
 
 /* Hard-mask extraction and compressed export (s.3.2 "Information flow at inference";
  * Algorithm 1 step 3). Per block: k = first index of the largest logit (NaN never wins;
@@ -312,6 +356,7 @@ int32_t mllm_abi_version(void);
 size_t mllm_sizeof_matrix(void);
 size_t mllm_sizeof_hparams(void);
 size_t mllm_sizeof_sparse_operand(void);
+size_t mllm_sizeof_linear_io(void);
 
 #ifdef __cplusplus
 }

@@ -12,8 +12,8 @@ Large Language Models"), cited by section and equation.
 Parity status per function (see the pins in tests/test_oracle_*.py):
   candidates, philox4x32_10, nlog, noise, soft_mask, sample_fwd, sample_bwd, adamw,
   prior_init (deterministic mode, similarity, magnitude prior), prior_init_from_index,
-  hard_pack, round_bf16, mask_diff, mask_stats, encode/decode_candidates, sparse_linear:
-  pinned.
+  hard_pack, round_bf16, mask_diff, mask_stats, encode/decode_candidates, sparse_linear,
+  masked_linear_fwd, masked_linear_bwd: pinned.
   prior_init random mode: the N(0, 0.01) draws are pinned by their moments, each
   Box-Muller pair against its two uniforms (radius and angle identities at fp64 rounding,
   uniforms from the known-answer Philox), and the Eq.10 structure exactly. The GPU takes the
@@ -311,6 +311,44 @@ def round_bf16(x) -> np.ndarray:
 def bf16_bits_to_float(bits) -> np.ndarray:
     """Exact value of bf16 bit patterns (a bit shift; no arithmetic of the method)."""
     return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------------------
+# The sampler inside the frozen network's linear layer
+# ---------------------------------------------------------------------------------------
+
+def masked_linear_fwd(n, m, W, pi, gids, A, kappa, tau, seed, step, noise_on=True, round_w=True):
+    """Forward of one frozen linear layer whose weight is the soft-masked W (s.3.2 "Frozen
+    LLM Backbone": every linear layer of the network multiplies by W . M on its forward
+    pass): X = W . M from the sampler's forward (Eq.5-Eq.7), stored in bf16 (nearest, ties
+    to even), then Y = A X^T for activations A [T, cols], as a plain fp64 matrix product.
+
+    W [rows, cols] and A [T, cols] are float64 values; pi [rows*cols/M, C] fp32; gids the
+    blocks' global ids. Returns a dict: y [T, rows]; x [rows, cols] (W . M unrounded);
+    x_bits [rows, cols] uint16 (its bf16 storage); reg (sum of unrounded x^2, Eq.8)."""
+    W = np.asarray(W, np.float64)
+    rows, cols = W.shape
+    f = sample_fwd(n, m, W.reshape(-1, m), pi, gids, kappa, tau, seed, step, noise_on=noise_on,
+                   round_w=round_w)
+    x = f["x"].reshape(rows, cols)
+    bits = round_bf16(x)
+    xr = bf16_bits_to_float(bits).astype(np.float64)
+    y = np.asarray(A, np.float64) @ xr.T
+    return {"y": y, "x": x, "x_bits": bits, "reg": f["reg"]}
+
+
+def masked_linear_bwd(n, m, W, pi, gids, A, dY, kappa, tau, lam, seed, step, noise_on=True, round_w=True):
+    """Weight side of the same layer's backward: the layer's weight X = W . M receives
+    dL/dX = dY^T A (the gradient of Y = A X^T with respect to X), and the logits receive
+    that gradient through Eq.7 and Eq.6 together with the regulariser's (sample_bwd); W
+    stays frozen (s.3.2). dY [T, rows] and A [T, cols] float64 values.
+    Returns (grad [B, C], scale [B, C] as sample_bwd gives it, G = dY^T A [rows, cols])."""
+    W = np.asarray(W, np.float64)
+    rows, cols = W.shape
+    G = np.asarray(dY, np.float64).T @ np.asarray(A, np.float64)
+    g, scale = sample_bwd(n, m, W.reshape(-1, m), G.reshape(-1, m), pi, gids, kappa, tau, lam, seed, step,
+                          noise_on=noise_on, round_w=round_w)
+    return g, scale, G
 
 
 # ---------------------------------------------------------------------------------------

@@ -9,7 +9,8 @@ from ._mllm import (  # noqa: F401
     mllm_decode_candidates, mllm_encode_candidates, mllm_hard_pack, mllm_last_cuda_error,
     mllm_mask_diff, mllm_mask_stats, mllm_noise, mllm_num_candidates, mllm_prior_init, mllm_prior_init_from_mask,
     mllm_sample_bwd_adam, mllm_sample_bwd_adam_fwd, mllm_sample_fwd, mllm_sample_fwd_noalloc, mllm_sparse_linear, mllm_sparse_linear_check_timeout, mllm_sparse_linear_workspace_bytes,
-    sparse_linear_workspace,
+    sparse_linear_workspace, mllm_masked_linear_fwd, mllm_masked_linear_workspace_bytes,
+    masked_linear_workspace, mllm_masked_linear_bwd_adam,
     mllm_status_string, mllm_workspace_bytes, lib, SparseOperandArray,
 )
 from .buffers import alloc_matrix, pack_shapes  # noqa: F401

@@ -91,6 +91,14 @@ class SparseOperand(ctypes.Structure):
     ]
 
 
+class LinearIO(ctypes.Structure):
+    _fields_ = [
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("dy", ctypes.c_void_p),
+    ]
+
+
 _P = ctypes.c_void_p
 _SIGS = {
     "mllm_num_candidates": (ctypes.c_int32, [NM]),
@@ -112,6 +120,10 @@ _SIGS = {
     "mllm_sparse_linear_workspace_bytes": (ctypes.c_size_t, []),
     "mllm_sparse_linear_check_timeout": (ctypes.c_int, [_P, NM, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "mllm_sizeof_sparse_operand": (ctypes.c_size_t, []),
+    "mllm_sizeof_linear_io": (ctypes.c_size_t, []),
+    "mllm_masked_linear_fwd": (ctypes.c_int, [_P, _P, ctypes.c_int32, NM, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]),
+    "mllm_masked_linear_workspace_bytes": (ctypes.c_size_t, []),
+    "mllm_masked_linear_bwd_adam": (ctypes.c_int, [_P, _P, ctypes.c_int32, NM, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
     "mllm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mllm_last_cuda_error": (ctypes.c_int32, []),
     "mllm_abi_version": (ctypes.c_int32, []),
@@ -137,7 +149,8 @@ def lib() -> ctypes.CDLL:
         if h.mllm_abi_version() != ABI_VERSION:
             raise ImportError("libmllm.so ABI version mismatch")
         if (h.mllm_sizeof_matrix() != ctypes.sizeof(Matrix) or h.mllm_sizeof_hparams() != ctypes.sizeof(HParams)
-                or h.mllm_sizeof_sparse_operand() != ctypes.sizeof(SparseOperand)):
+                or h.mllm_sizeof_sparse_operand() != ctypes.sizeof(SparseOperand)
+                or h.mllm_sizeof_linear_io() != ctypes.sizeof(LinearIO)):
             raise ImportError("libmllm.so struct layout mismatch")
         _lib = h
     return _lib
@@ -393,3 +406,45 @@ def mllm_sparse_linear_check_timeout(op, nm, tokens: int, workspace: torch.Tenso
 
 def mllm_last_cuda_error() -> int:
     return lib().mllm_last_cuda_error()
+
+
+def mllm_masked_linear_workspace_bytes() -> int:
+    return lib().mllm_masked_linear_workspace_bytes()
+
+
+def masked_linear_workspace(device) -> torch.Tensor:
+    """A zero-filled workspace for the mllm_masked_linear_* calls on `device`."""
+    return torch.zeros(mllm_masked_linear_workspace_bytes(), dtype=torch.uint8, device=device)
+
+
+def _linear_io(ios):
+    """C array of mllm_linear_io from (x, y, dy) tuples (entries may be None)."""
+    arr = (LinearIO * max(1, len(ios)))()
+    for i, (x, y, dy) in enumerate(ios):
+        arr[i] = LinearIO(_ptr(x), _ptr(y), _ptr(dy))
+    return arr
+
+
+def mllm_masked_linear_fwd(mats, ios, nm, tokens: int, hp: Hparams, workspace: torch.Tensor,
+                           reg_sum_out: Optional[torch.Tensor] = None, stream=None):
+    """Y = A (W . M)^T for every matrix, the soft-masked weight made on the fly: ios[i] =
+    (x [tokens, cols] bf16, y [tokens, rows] fp32, None)."""
+    a = _mats(mats)
+    io = _linear_io(ios)
+    h = hp.to_c() if isinstance(hp, Hparams) else hp
+    _check(lib().mllm_masked_linear_fwd(a.ptr, ctypes.cast(io, ctypes.c_void_p), a.n, _nm(nm), int(tokens),
+                                        ctypes.byref(h), _ptr(reg_sum_out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "mllm_masked_linear_fwd")
+
+
+def mllm_masked_linear_bwd_adam(mats, ios, nm, tokens: int, hp: Hparams, workspace: torch.Tensor, stream=None):
+    """G = dY^T A per matrix, then the logits' backward + AdamW from G (never stored):
+    ios[i] = (x [tokens, cols] bf16, None, dy [tokens, rows] bf16)."""
+    a = _mats(mats)
+    io = _linear_io(ios)
+    h = hp.to_c() if isinstance(hp, Hparams) else hp
+    _check(lib().mllm_masked_linear_bwd_adam(a.ptr, ctypes.cast(io, ctypes.c_void_p), a.n, _nm(nm), int(tokens),
+                                             ctypes.byref(h), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "mllm_masked_linear_bwd_adam")

@@ -79,6 +79,23 @@ __device__ __forceinline__ void stage_in(float *dst, const float *src, int n) {
     cp_async_wait_all();
 }
 
+// The same copies without the wait: the tile lands while the CTA works on something else;
+// the caller waits (cp_async_wait_pending) and synchronises the CTA before reading it. The 8-byte
+// tail of an odd block count goes through an 8-byte cp.async.
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void stage_in_async(float *dst, const float *src, int n) {
+    const int n4 = n >> 2;
+    for (int i = threadIdx.x; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
+    if ((n & 3) && threadIdx.x == 0) cp_async8(dst + 4 * n4, src + 4 * n4);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_pending() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void stage_out(float *dst, const float *src, int n) {
     const int n4 = n >> 2;
     for (int i = threadIdx.x; i < n4; i += kCtaThreads)
@@ -173,6 +190,139 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
     p = __fmaf_rn(-s.step_size, __fdividef(m, denom), pd);
 }
 
+// Gradient of one block's logits (Eq.6-Eq.8 backward, noise of step sc.step) into grow[C]:
+// dpi_c = (kappa/tau) y_c (sum_{j in S_c} P_j - sum_{j not in S_c} Q_j), P_j = (1 - M_j) u_j,
+// Q_j = M_j u_j, u_j = G_j W_j - 2 lambda W_j^2 M_j.
+__device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8], const float gw[8], uint64_t gid,
+                                         const StepScalars &sc, const NlogCtx &L, float *grow) {
+    float w[C], ms[8], mc[8];
+    const float mx = perturbed(pi_row, sc.seed, gid, sc, L, w);
+    const float r = rcp_approx(soft_sums<true>(w, mx, sc.c2, ms, mc));
+    float P[8], Q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        ms[j] = __fmul_rn(ms[j], r);
+        mc[j] = __fmul_rn(mc[j], r);
+        const float wj = wt[j];
+        const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j], __fmul_rn(gw[j], wj));
+        P[j] = __fmul_rn(mc[j], u);
+        Q[j] = __fmul_rn(ms[j], u);
+    }
+    const float cr = __fmul_rn(sc.kappa_over_tau, r);
+    static_for<0, C>([&](auto I) {
+        constexpr int c = decltype(I)::value;
+        constexpr uint32_t mk = cand_mask(c);
+        float kept = 0.f, pruned = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (mk & (1u << j)) kept += P[j];
+            else pruned += Q[j];
+        }
+        grow[c] = __fmul_rn(__fmul_rn(cr, w[c]), kept - pruned);
+    });
+}
+
+// Forward of one block (Eq.5-Eq.8): soft mask ms[8] and soft-masked weights x[8] (fp32),
+// regulariser partial added to acc.
+__device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], uint64_t gid, const StepScalars &sc,
+                                        const NlogCtx &L, float ms[8], float x[8], float &acc) {
+    float w[C], mc[8];
+    const float mx = perturbed(pi_row, sc.seed, gid, sc, L, w);
+    const float r = rcp_approx(soft_sums<false>(w, mx, sc.c2, ms, mc));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        ms[j] = __fmul_rn(ms[j], r);
+        x[j] = __fmul_rn(wt[j], ms[j]);
+        acc = __fmaf_rn(x[j], x[j], acc);
+    }
+}
+
+// AdamW over a tile as one flat, coalesced array of float4: logits and gradients from shared
+// memory, m and v from global memory (each thread first loads kUnroll vectors of each, so it
+// keeps 2*kUnroll loads in flight). Updated logits, m, v (and the gradient when gout) are
+// stored; with kKeep the updated logits are also written back to s_pi.
+template <bool kKeep>
+__device__ __forceinline__ void adam_tile(float *s_pi, const float *s_gr, int n, float *__restrict__ pi,
+                                          float *__restrict__ mm, float *__restrict__ vv,
+                                          float *__restrict__ gout, const StepScalars &sc) {
+    const int n4 = n >> 2;
+    constexpr int kUnroll = 6;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += kCtaThreads * kUnroll) {
+        float4 m4[kUnroll], v4[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kCtaThreads;
+            if (i < n4) {
+                m4[u] = __ldcs(reinterpret_cast<const float4 *>(mm) + i);
+                v4[u] = __ldcs(reinterpret_cast<const float4 *>(vv) + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kCtaThreads;
+            if (i < n4) {
+                float4 p4 = reinterpret_cast<const float4 *>(s_pi)[i];
+                const float4 g4 = reinterpret_cast<const float4 *>(s_gr)[i];
+                adamw(p4.x, m4[u].x, v4[u].x, g4.x, sc);
+                adamw(p4.y, m4[u].y, v4[u].y, g4.y, sc);
+                adamw(p4.z, m4[u].z, v4[u].z, g4.z, sc);
+                adamw(p4.w, m4[u].w, v4[u].w, g4.w, sc);
+                if (kKeep) reinterpret_cast<float4 *>(s_pi)[i] = p4;
+                __stcs(reinterpret_cast<float4 *>(pi) + i, p4);
+                __stcs(reinterpret_cast<float4 *>(mm) + i, m4[u]);
+                __stcs(reinterpret_cast<float4 *>(vv) + i, v4[u]);
+                if (gout) __stcs(reinterpret_cast<float4 *>(gout) + i, g4);
+            }
+        }
+    }
+    if ((n & 3) && threadIdx.x == 0) {  // 2-float tail of a tile with an odd block count
+        for (int i = 4 * n4; i < n; ++i) {
+            float p = s_pi[i], m = mm[i], v = vv[i];
+            adamw(p, m, v, s_gr[i], sc);
+            if (kKeep) s_pi[i] = p;
+            pi[i] = p; mm[i] = m; vv[i] = v;
+            if (gout) gout[i] = s_gr[i];
+        }
+    }
+}
+
+// CTA-level deterministic reduction of the regulariser partials, then the last CTA (ticket)
+// combines all per-CTA partials in index order and resets the ticket.
+__device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned int *ticket, double *reg_out,
+                                           int accumulate) {
+    __shared__ double s_w[kCtaThreads / 32];
+    __shared__ bool s_last;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) s_w[warp] = (double)acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double tt = 0.0;
+        for (int i = 0; i < kCtaThreads / 32; ++i) tt += s_w[i];
+        partials[blockIdx.x] = tt;
+        __threadfence();
+        s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    double tt = 0.0;
+    for (unsigned int i = threadIdx.x; i < gridDim.x; i += kCtaThreads) tt += __ldcg(partials + i);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tt += __shfl_xor_sync(0xFFFFFFFFu, tt, o);
+    __syncthreads();
+    if (lane == 0) s_w[warp] = tt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double tot = 0.0;
+        for (int i = 0; i < kCtaThreads / 32; ++i) tot += s_w[i];
+        *reg_out = accumulate ? (*reg_out + tot) : tot;
+        *ticket = 0u;
+    }
+}
+
 // --------------------------------------------------------------------------- kernels
 
 template <bool kW32>
@@ -195,17 +345,9 @@ __global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant_
         __syncthreads();
         if ((int)threadIdx.x < nb) {
             const int64_t b = tb0 + threadIdx.x;
-            float w[C], ms[8], mc[8], wt[8];
-            const float mx = perturbed(s_pi + threadIdx.x * C, sc.seed, d.gid0 + b, sc, L, w);
+            float wt[8], ms[8], x[8];
             load8<kW32>(d.W, b, wt);
-            const float r = rcp_approx(soft_sums<false>(w, mx, sc.c2, ms, mc));
-            float x[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                ms[j] = __fmul_rn(ms[j], r);
-                x[j] = __fmul_rn(wt[j], ms[j]);
-                acc = __fmaf_rn(x[j], x[j], acc);
-            }
+            fwd_row(s_pi + threadIdx.x * C, wt, d.gid0 + b, sc, L, ms, x, acc);
             store8<kW32>(d.X, b, x);
             if (d.soft) {
                 float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
@@ -214,40 +356,7 @@ __global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant_
             }
         }
     }
-    if (reg_out) {
-        // CTA-level deterministic reduction, then the last CTA combines all partials.
-        __shared__ double s_w[kCtaThreads / 32];
-        __shared__ bool s_last;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        __syncthreads();
-        if (lane == 0) s_w[warp] = (double)acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double tt = 0.0;
-            for (int i = 0; i < kCtaThreads / 32; ++i) tt += s_w[i];
-            partials[blockIdx.x] = tt;
-            __threadfence();
-            s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1);
-        }
-        __syncthreads();
-        if (!s_last) return;
-        __threadfence();
-        double tt = 0.0;
-        for (unsigned int i = threadIdx.x; i < gridDim.x; i += kCtaThreads) tt += __ldcg(partials + i);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tt += __shfl_xor_sync(0xFFFFFFFFu, tt, o);
-        __syncthreads();
-        if (lane == 0) s_w[warp] = tt;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double tot = 0.0;
-            for (int i = 0; i < kCtaThreads / 32; ++i) tot += s_w[i];
-            *reg_out = accumulate ? (*reg_out + tot) : tot;
-            *ticket = 0u;
-        }
-    }
+    if (reg_out) reduce_reg(acc, partials, ticket, reg_out, accumulate);
 }
 
 template <bool kW32, bool kG32>
@@ -271,82 +380,78 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
         __syncthreads();
         if ((int)threadIdx.x < nb) {
             const int64_t b = tb0 + threadIdx.x;
-            float w[C], ms[8], mc[8], wt[8], gw[8];
-            const float mx = perturbed(s_pi + threadIdx.x * C, sc.seed, d.gid0 + b, sc, L, w);
+            float wt[8], gw[8];
             load8<kW32>(d.W, b, wt);
             load8<kG32>(d.G, b, gw);
-            const float r = rcp_approx(soft_sums<true>(w, mx, sc.c2, ms, mc));
-            float P[8], Q[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                ms[j] = __fmul_rn(ms[j], r);
-                mc[j] = __fmul_rn(mc[j], r);
-                const float wj = wt[j];
-                const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j],
-                                          __fmul_rn(gw[j], wj));
-                P[j] = __fmul_rn(mc[j], u);
-                Q[j] = __fmul_rn(ms[j], u);
-            }
-            const float cr = __fmul_rn(sc.kappa_over_tau, r);
-            float *grow = s_gr + threadIdx.x * C;
-            static_for<0, C>([&](auto I) {
-                constexpr int c = decltype(I)::value;
-                constexpr uint32_t mk = cand_mask(c);
-                float kept = 0.f, pruned = 0.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (mk & (1u << j)) kept += P[j];
-                    else pruned += Q[j];
-                }
-                grow[c] = __fmul_rn(__fmul_rn(cr, w[c]), kept - pruned);
-            });
+            grad_row(s_pi + threadIdx.x * C, wt, gw, d.gid0 + b, sc, L, s_gr + threadIdx.x * C);
         }
         __syncthreads();
-        // AdamW over the tile as one flat, coalesced array of float4: each thread first loads
-        // kUnroll vectors of m and v (prefetched into L2 at the start of the tile), then
-        // updates them, so every thread keeps 2*kUnroll loads in flight.
-        const int n = nb * C, n4 = n >> 2;
-        float *__restrict__ pi = d.pi + tb0 * C;
-        float *__restrict__ mm = d.m + tb0 * C;
-        float *__restrict__ vv = d.v + tb0 * C;
-        float *__restrict__ gout = d.grad ? d.grad + tb0 * C : nullptr;
-        constexpr int kUnroll = 6;
-        for (int i0 = threadIdx.x; i0 < n4; i0 += kCtaThreads * kUnroll) {
-            float4 m4[kUnroll], v4[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int i = i0 + u * kCtaThreads;
-                if (i < n4) {
-                    m4[u] = __ldcs(reinterpret_cast<const float4 *>(mm) + i);
-                    v4[u] = __ldcs(reinterpret_cast<const float4 *>(vv) + i);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int i = i0 + u * kCtaThreads;
-                if (i < n4) {
-                    float4 p4 = reinterpret_cast<const float4 *>(s_pi)[i];
-                    const float4 g4 = reinterpret_cast<const float4 *>(s_gr)[i];
-                    adamw(p4.x, m4[u].x, v4[u].x, g4.x, sc);
-                    adamw(p4.y, m4[u].y, v4[u].y, g4.y, sc);
-                    adamw(p4.z, m4[u].z, v4[u].z, g4.z, sc);
-                    adamw(p4.w, m4[u].w, v4[u].w, g4.w, sc);
-                    __stcs(reinterpret_cast<float4 *>(pi) + i, p4);
-                    __stcs(reinterpret_cast<float4 *>(mm) + i, m4[u]);
-                    __stcs(reinterpret_cast<float4 *>(vv) + i, v4[u]);
-                    if (gout) __stcs(reinterpret_cast<float4 *>(gout) + i, g4);
-                }
-            }
-        }
-        if ((n & 3) && threadIdx.x == 0) {  // 2-float tail of a tile with an odd block count
-            for (int i = 4 * n4; i < n; ++i) {
-                float p = s_pi[i], m = mm[i], v = vv[i];
-                adamw(p, m, v, s_gr[i], sc);
-                pi[i] = p; mm[i] = m; vv[i] = v;
-                if (gout) gout[i] = s_gr[i];
-            }
-        }
+        adam_tile<false>(s_pi, s_gr, nb * C, d.pi + tb0 * C, d.m + tb0 * C, d.v + tb0 * C,
+                         d.grad ? d.grad + tb0 * C : nullptr, sc);
     }
+}
+
+// Backward + AdamW of step t fused with the forward of step t+1 (mllm_sample_bwd_adam_fwd):
+// per tile, the gradient of every block (noise of step t) into one buffer, the flat AdamW
+// pass (updated logits kept in shared memory), then the forward of step t+1 from the updated
+// logits. The tile's logits are read from HBM once. Two tile buffers alternate: while a tile's
+// forward runs, the next tile's logits land in the buffer its gradients used, and its m, v
+// are fetched into L2 at the start of the tile, ahead of the AdamW pass.
+template <bool kW32, bool kG32>
+__global__ void __launch_bounds__(kCtaThreads) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
+                                                                   const StepScalars sb, const StepScalars sf,
+                                                                   double *partials, unsigned int *ticket,
+                                                                   double *reg_out, int accumulate) {
+    __shared__ __align__(16) float2 s_tab[kNlogEntries];
+    extern __shared__ __align__(16) float s_dyn[];  // [2 * kTileFloats]: two tile buffers
+    load_tab(s_tab);
+    const NlogCtx L{s_tab};
+    float acc = 0.f;
+    int cur = 0;
+    auto stage = [&](float *dst, int64_t t) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
+        stage_in_async(dst, d.pi + tb0 * C, (int)imin64(kBlocksPerCta, d.nblocks - tb0) * C);
+    };
+    if ((int64_t)blockIdx.x < grp.total_work) stage(s_dyn, blockIdx.x);
+    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+        const MatDesc &d = grp.d[find_mat(grp, t)];
+        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
+        const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
+        float *s_pi = s_dyn + cur * kTileFloats, *s_gr = s_dyn + (cur ^ 1) * kTileFloats;
+        cp_async_wait_pending();
+        __syncthreads();  // the tile's logits (and the table) are in; the other buffer is free
+        if (threadIdx.x == 0) {
+            prefetch_l2(d.m + tb0 * C, nb * C * 4);
+            prefetch_l2(d.v + tb0 * C, nb * C * 4);
+        }
+        const bool mine = (int)threadIdx.x < nb;
+        const int64_t b = tb0 + threadIdx.x;
+        float wt[8];
+        if (mine) {
+            float gw[8];
+            load8<kW32>(d.W, b, wt);
+            load8<kG32>(d.G, b, gw);
+            grad_row(s_pi + threadIdx.x * C, wt, gw, d.gid0 + b, sb, L, s_gr + threadIdx.x * C);
+        }
+        __syncthreads();
+        adam_tile<true>(s_pi, s_gr, nb * C, d.pi + tb0 * C, d.m + tb0 * C, d.v + tb0 * C,
+                        d.grad ? d.grad + tb0 * C : nullptr, sb);
+        __syncthreads();  // updated logits in s_pi; the gradient buffer is free
+        if (t + gridDim.x < grp.total_work) stage(s_gr, t + gridDim.x);
+        if (mine) {
+            float ms[8], x[8];
+            fwd_row(s_pi + threadIdx.x * C, wt, d.gid0 + b, sf, L, ms, x, acc);
+            store8<kW32>(d.X, b, x);
+            if (d.soft) {
+                float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
+                sp[0] = make_float4(ms[0], ms[1], ms[2], ms[3]);
+                sp[1] = make_float4(ms[4], ms[5], ms[6], ms[7]);
+            }
+        }
+        cur ^= 1;
+    }
+    if (reg_out) reduce_reg(acc, partials, ticket, reg_out, accumulate);
 }
 
 // Prior initialisation; kFromIdx as for the 2:4 kernel (M0 = candidate d.prior[b], >= C: none).

@@ -14,6 +14,7 @@
 #include "kernels_diag.cuh"
 #include "kernels_spl.cuh"
 #include "kernels_umma.cuh"
+#include "kernels_mlin.cuh"
 
 namespace mllm {
 namespace {
@@ -573,6 +574,107 @@ bool sparse_linear_batched(const std::vector<mllm_sparse_operand> &ops, mllm_nm 
     return true;
 }
 
+// ------------------------------------------------------------------------ masked linear layer
+
+// Tokens rounded up to the MMA's N (32, 64, 128 or 256).
+int mlin_n(int32_t tokens) { return tokens <= 32 ? 32 : tokens <= 64 ? 64 : tokens <= 128 ? 128 : 256; }
+
+mllm_status validate_mlin(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats, mllm_nm nm,
+                          int32_t tokens, unsigned need, bool fwd) {
+    mllm_status s = validate_mats(mats, n_mats, nm, need);
+    if (s != MLLM_OK) return s;
+    if (nm.m != 4) return MLLM_ERR_UNSUPPORTED;
+    if (!io || tokens < 1 || tokens > mlin::kMaxTokens) return MLLM_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_mats; ++i) {
+        const mllm_matrix &a = mats[i];
+        if (a.w_dtype != MLLM_BF16) return MLLM_ERR_UNSUPPORTED;
+        if (a.cols % mlin::kChunk) return MLLM_ERR_UNSUPPORTED;
+        if (a.rows > INT32_MAX || a.cols > INT32_MAX) return MLLM_ERR_INVALID_ARG;
+        const bool any = a.rows > 0 && a.cols > 0;
+        if ((s = check_ptr(io[i].x, any)) != MLLM_OK) return s;
+        if ((s = check_ptr(fwd ? (const void *)io[i].y : io[i].dy, any)) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+// The call's matrices in groups of at most kMaxMats, each with its chunk sequence and the
+// activations' tensor maps (box 64 columns x N tokens, 128-byte swizzle). False if a map
+// cannot be encoded.
+bool mlin_groups(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats, int32_t tokens, int N,
+                 std::vector<mlin::Group> *out) {
+    for (int32_t i0 = 0; i0 < n_mats; i0 += kMaxMats) {
+        mlin::Group g{};
+        g.tokens = tokens;
+        int64_t acc = 0;
+        int32_t k = 0;
+        for (int32_t i = i0; i < std::min<int32_t>(n_mats, i0 + kMaxMats); ++i) {
+            const mllm_matrix &a = mats[i];
+            if (a.rows == 0 || a.cols == 0) continue;
+            mlin::Op &d = g.d[k];
+            d.W = a.W; d.pi = a.logits; d.m = a.adam_m; d.v = a.adam_v;
+            d.y = io[i].y; d.X = a.X_out; d.soft = a.soft_mask_out; d.grad = a.grad_logits_out;
+            d.gid0 = a.block_offset;
+            d.rows = a.rows; d.cols = a.cols;
+            d.nch = a.cols / mlin::kChunk;
+            d.ntiles = (a.rows + mlin::kRows - 1) / mlin::kRows;
+            d.chunk_begin = acc;
+            acc += d.nch * d.ntiles;
+            if (!encode_2d(&g.x[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, io[i].x, (uint64_t)a.cols, (uint64_t)tokens,
+                           2 * (uint64_t)a.cols, 64, (uint32_t)N, CU_TENSOR_MAP_SWIZZLE_128B))
+                return false;
+            ++k;
+        }
+        g.n = k;
+        g.total_chunks = acc;
+        if (k > 0) out->push_back(g);
+    }
+    return true;
+}
+
+template <int kN>
+mllm_status launch_mlin_fwd(const mlin::Group &g, const StepScalars &sc, unsigned char *ws, double *reg,
+                            int accumulate, cudaStream_t st) {
+    auto fn = mlin::masked_linear_fwd_kernel<kN>;
+    constexpr int smem = mlin::smem_bytes<kN>();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    resident_ctas(dev, (const void *)fn, mlin::kThreads, smem);  // sets the dynamic shared-memory limit
+    const int64_t grid = std::min<int64_t>({(int64_t)sm_count(dev), g.total_chunks, (int64_t)mlin::kMaxCtas});
+    fn<<<(unsigned)grid, mlin::kThreads, smem, st>>>(g, sc, ws, reg, accumulate);
+    return cuda_status(cudaGetLastError());
+}
+
+bool mlin_bwd_groups(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats, int32_t tokens,
+                     std::vector<mlin::BwdGroup> *out) {
+    for (int32_t i0 = 0; i0 < n_mats; i0 += kMaxMats) {
+        mlin::BwdGroup g{};
+        g.tokens = tokens;
+        int64_t acc = 0;
+        int32_t k = 0;
+        for (int32_t i = i0; i < std::min<int32_t>(n_mats, i0 + kMaxMats); ++i) {
+            const mllm_matrix &a = mats[i];
+            if (a.rows == 0 || a.cols == 0) continue;
+            mlin::Op &d = g.d[k];
+            d.W = a.W; d.pi = a.logits; d.m = a.adam_m; d.v = a.adam_v; d.grad = a.grad_logits_out;
+            d.gid0 = a.block_offset;
+            d.rows = a.rows; d.cols = a.cols;
+            g.ctiles[k] = (a.cols + mlin::kBwdCols - 1) / mlin::kBwdCols;
+            g.tile_begin[k] = acc;
+            acc += g.ctiles[k] * ((a.rows + mlin::kRows - 1) / mlin::kRows);
+            if (!encode_2d(&g.dy[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, io[i].dy, (uint64_t)a.rows, (uint64_t)tokens,
+                           2 * (uint64_t)a.rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                !encode_2d(&g.x[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, io[i].x, (uint64_t)a.cols, (uint64_t)tokens,
+                           2 * (uint64_t)a.cols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+                return false;
+            ++k;
+        }
+        g.n = k;
+        g.total_tiles = acc;
+        if (k > 0) out->push_back(g);
+    }
+    return true;
+}
+
 }  // namespace
 }  // namespace mllm
 
@@ -771,30 +873,34 @@ mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, ml
         if (!workspace || workspace_bytes < kWorkspaceBytes) return MLLM_ERR_WORKSPACE;
         if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
     }
-    if (nm.m != 4) {  // 4:8: the two kernels in sequence
-        if ((s = mllm_sample_bwd_adam(mats, n_mats, nm, hp, stream)) != MLLM_OK) return s;
-        return mllm_sample_fwd(mats, n_mats, nm, hp_next, reg_sum_out, workspace, workspace_bytes, stream);
-    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const StepScalars sb = make_scalars(*hp), sf = make_scalars(*hp_next);
     const bool w32 = mats[0].w_dtype == MLLM_F32, g32 = mats[0].g_dtype == MLLM_F32;
+    const bool is24 = nm.m == 4;
     unsigned int *ticket = reg_sum_out ? static_cast<unsigned int *>(workspace) : nullptr;
     double *partials = reg_sum_out ? reinterpret_cast<double *>(static_cast<char *>(workspace) + kWsPartialsOffset) : nullptr;
     bool wrote_reg = false;
-    for (const Group &g : make_groups(mats, n_mats, nm.m, Kind::Sample24)) {
+    for (const Group &g : make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48)) {
         if (g.total_work == 0) continue;
         const int accumulate = wrote_reg ? 1 : 0;
-#define MLLM_LAUNCH_FUSED(W32, G32)                                                                    \
+#define MLLM_LAUNCH_FUSED(NS, THREADS, SMEM, W32, G32)                                                 \
     do {                                                                                                 \
-        const void *fn = (const void *)k24::bwd_adam_fwd_kernel<W32, G32>;                               \
-        const int64_t grid = grid_for(fn, kThreads, 0, g.total_work, kMaxReduceCtas);                     \
-        k24::bwd_adam_fwd_kernel<W32, G32><<<(unsigned)grid, kThreads, 0, st>>>(g, sb, sf, partials, ticket, \
-                                                                              reg_sum_out, accumulate);  \
+        const void *fn = (const void *)NS::bwd_adam_fwd_kernel<W32, G32>;                                \
+        const int64_t grid = grid_for(fn, THREADS, SMEM, g.total_work, kMaxReduceCtas);                   \
+        NS::bwd_adam_fwd_kernel<W32, G32><<<(unsigned)grid, THREADS, SMEM, st>>>(g, sb, sf, partials, ticket, \
+                                                                               reg_sum_out, accumulate); \
     } while (0)
-        if (w32 && g32) MLLM_LAUNCH_FUSED(true, true);
-        else if (w32) MLLM_LAUNCH_FUSED(true, false);
-        else if (g32) MLLM_LAUNCH_FUSED(false, true);
-        else MLLM_LAUNCH_FUSED(false, false);
+        if (is24) {
+            if (w32 && g32) MLLM_LAUNCH_FUSED(k24, kThreads, 0, true, true);
+            else if (w32) MLLM_LAUNCH_FUSED(k24, kThreads, 0, true, false);
+            else if (g32) MLLM_LAUNCH_FUSED(k24, kThreads, 0, false, true);
+            else MLLM_LAUNCH_FUSED(k24, kThreads, 0, false, false);
+        } else {
+            if (w32 && g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, true);
+            else if (w32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, false);
+            else if (g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, true);
+            else MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, false);
+        }
 #undef MLLM_LAUNCH_FUSED
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -1005,6 +1111,66 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, mllm
 }
 
 size_t mllm_sizeof_sparse_operand(void) { return sizeof(mllm_sparse_operand); }
+size_t mllm_sizeof_linear_io(void) { return sizeof(mllm_linear_io); }
+
+size_t mllm_masked_linear_workspace_bytes(void) { return mlin::kWorkspaceBytes; }
+
+mllm_status mllm_masked_linear_bwd_adam(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats,
+                                        mllm_nm nm, int32_t tokens, const mllm_hparams *hp, void *workspace,
+                                        size_t workspace_bytes, void *stream) {
+    mllm_status s = validate_mlin(mats, io, n_mats, nm, tokens, kNeedW | kNeedPi | kNeedMV, false);
+    if (s != MLLM_OK) return s;
+    if ((s = validate_bwd_hp(hp)) != MLLM_OK) return s;
+    for (int32_t i = 0; i < n_mats; ++i)
+        if (mats[i].rows % 8) return MLLM_ERR_UNSUPPORTED;  // dY rows are whole 16-byte units
+    if (!workspace || workspace_bytes < mlin::kWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    std::vector<mlin::BwdGroup> groups;
+    if (!mlin_bwd_groups(mats, io, n_mats, tokens, &groups)) return MLLM_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StepScalars sc = make_scalars(*hp);
+    auto fn = mlin::masked_linear_bwd_adam_kernel;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    resident_ctas(dev, (const void *)fn, mlin::kThreads, mlin::kBwdSmem);  // sets the dynamic shared-memory limit
+    for (const mlin::BwdGroup &g : groups) {
+        const int64_t grid = std::min<int64_t>({(int64_t)sm_count(dev), g.total_tiles, (int64_t)mlin::kMaxCtas});
+        fn<<<(unsigned)grid, mlin::kThreads, mlin::kBwdSmem, st>>>(g, sc, static_cast<unsigned char *>(workspace));
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
+
+mllm_status mllm_masked_linear_fwd(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats, mllm_nm nm,
+                                   int32_t tokens, const mllm_hparams *hp, double *reg_sum_out, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    mllm_status s = validate_mlin(mats, io, n_mats, nm, tokens, kNeedW | kNeedPi, true);
+    if (s != MLLM_OK) return s;
+    if ((s = validate_fwd_hp(hp)) != MLLM_OK) return s;
+    if (reg_sum_out && (reinterpret_cast<uintptr_t>(reg_sum_out) & 7u) != 0) return MLLM_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < mlin::kWorkspaceBytes) return MLLM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
+    const int N = mlin_n(tokens);
+    std::vector<mlin::Group> groups;
+    if (!mlin_groups(mats, io, n_mats, tokens, N, &groups)) return MLLM_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StepScalars sc = make_scalars(*hp);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    bool wrote_reg = false;
+    for (const mlin::Group &g : groups) {
+        const int accumulate = wrote_reg ? 1 : 0;
+        s = N == 32    ? launch_mlin_fwd<32>(g, sc, ws, reg_sum_out, accumulate, st)
+            : N == 64  ? launch_mlin_fwd<64>(g, sc, ws, reg_sum_out, accumulate, st)
+            : N == 128 ? launch_mlin_fwd<128>(g, sc, ws, reg_sum_out, accumulate, st)
+                       : launch_mlin_fwd<256>(g, sc, ws, reg_sum_out, accumulate, st);
+        if (s != MLLM_OK) return s;
+        wrote_reg = true;
+    }
+    if (reg_sum_out && !wrote_reg) {
+        if ((s = cuda_status(cudaMemsetAsync(reg_sum_out, 0, sizeof(double), st))) != MLLM_OK) return s;
+    }
+    return MLLM_OK;
+}
 
 mllm_status mllm_noise(mllm_nm nm, uint64_t seed, uint32_t step, const uint64_t *gids,
                        int64_t n_blocks, float *g_out, void *stream) {

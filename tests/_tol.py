@@ -101,3 +101,32 @@ def assert_spl_close(y_gpu, y_ref, absxw, cols):
     bad = ~(err <= tol)  # NaN fails
     assert not bad.any(), f"{bad.sum()} y mismatches, worst {np.max(err / np.maximum(tol, 1e-300)):.3g} x tol"
     return float(np.max(err / np.maximum(absxw, 1e-300)))
+
+
+def assert_masked_linear_close(y_gpu, y_ref, A, x_ref, round_bf16):
+    """Y = A X^T with X = bf16(W * M) made inside the GEMM, against the oracle's fp64 product
+    with its own bf16 X. Two sources of difference, each bounded:
+      * an element of X may round to the neighbouring bf16 value when its unrounded value
+        lies within the soft-mask tolerance (1e-5 relative) plus the fp32 product's rounding
+        (2^-23) of a rounding midpoint; such elements are found by rounding both ends of that
+        interval (round_bf16 of the oracle), and each may move Y by |A| times the gap;
+      * the tensor cores add the exact bf16 x bf16 products into fp32, one k16 step after
+        another (ceil(cols/16) steps) plus the partial tiles of rows split between CTAs (at
+        most 8 more additions), each off by at most 2 ulp (2^-22) of a running sum bounded
+        by sum_k |A_k X_k|.
+    A [T, cols], x_ref [rows, cols] unrounded float64; y [T, rows]."""
+    A = np.asarray(A, np.float64)
+    x_ref = np.asarray(x_ref, np.float64)
+    delta = 1e-5 + 2.0 ** -23
+    lo = round_bf16(x_ref * (1 - delta)).astype(np.uint32) << 16
+    hi = round_bf16(x_ref * (1 + delta)).astype(np.uint32) << 16
+    lo_v = lo.view(np.float32).astype(np.float64)
+    hi_v = hi.view(np.float32).astype(np.float64)
+    gap = np.abs(hi_v - lo_v)  # 0 where the whole interval rounds to one value
+    xb = (round_bf16(x_ref).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    cols = A.shape[1]
+    bound = np.abs(A) @ gap.T + ((cols + 15) // 16 + 8) * 2.0 ** -22 * (np.abs(A) @ np.abs(xb).T)
+    err = np.abs(np.asarray(y_gpu, np.float64) - y_ref)
+    bad = ~(err <= bound + 1e-30)  # NaN fails
+    assert not bad.any(), f"{bad.sum()} Y mismatches, worst {np.max(err / np.maximum(bound, 1e-300)):.3g} x tol"
+    return float(np.max(err / np.maximum(np.abs(A) @ np.abs(xb).T, 1e-300)))

@@ -475,7 +475,9 @@ def test_fused_step_walks_many_tiles_per_cta(orc, ws, nm, shape):
     torch.cuda.synchronize()
     for a, b in zip((c.mb.logits, c.mb.adam_m, c.mb.adam_v, c.mb.grad_logits, c.mb.X, c.mb.soft_mask), seq):
         assert torch.equal(a, b)
-    assert abs(reg_a.item() - reg_b.item()) <= 1e-12 * abs(reg_a.item())
+    # the two kernels run different grids, so each CTA's fp32 partial covers other tiles: the
+    # sums agree to the rounding of that order (a few fp32 ulps per tile a CTA adds)
+    assert abs(reg_a.item() - reg_b.item()) <= 1e-6 * abs(reg_a.item())
     r_x = float((c.mb.X.double() ** 2).sum())
     assert abs(reg_b.item() - r_x) <= 1e-3 * r_x
     idx = np.arange(0, c.B, 13 if m == 4 else 7)
