@@ -70,6 +70,31 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def bf16_peak():
+    """Dense bf16 tensor-core TFLOP/s (burst) and its kind."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def tensor_stats(T, shapes_rows_cols, ms):
+    """Prefill-sized products are bound by the tensor cores: the dense-equivalent rate
+    2 T rows cols / time, against the 2:4 sparse peak, twice the dense bf16 peak (the
+    nominal ratio of the sparse mode)."""
+    flops = 2.0 * T * sum(r * c for r, c in shapes_rows_cols)
+    peak, kind = bf16_peak()
+    tf = flops / (ms / 1e3) / 1e12
+    return {"tflops_dense_equiv": round(tf, 1), "tensor_peak_tflops": 2 * peak, "tensor_peak_kind": kind,
+            "tensor_frac": round(tf / (2 * peak), 4)}
+
+
 # ------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -359,16 +384,24 @@ def time_extras(stack, peak):
     out["mask_stats_once"] = once_stats(
         time_once(lambda: [pkg.mllm_mask_stats(stack.view(l), w.nm, w.kappa[1], stats, stack.ws) for l in range(L)]),
         B, (16 if w.w_dtype == "f32" else 8) + 4 * w.C, peak)
-    idx = [mb.cand_idx for mb in stack.bufs[0]]   # hard masks of one layer, reused per layer
-    other = [torch.roll(t, 1) for t in idx]
+    # the whole stack's hard masks as one array (each matrix's candidate indices a view at its
+    # global block offset), so that the mask difference and the candidate code take one launch
+    flat = torch.empty(B, dtype=torch.uint8, device=dev)
+    base = stack.bufs[0][0].block_offset
+    for mats in stack.bufs:
+        for mb in mats:
+            nb = mb.W.numel() // w.nm[1]
+            mb.cand_idx = flat[mb.block_offset - base: mb.block_offset - base + nb]
+        pkg.mllm_hard_pack(pkg.MatrixArray(mats), w.nm)
+    idx = [mb.cand_idx for mb in stack.bufs[0]]
+    other = torch.roll(flat, 1)
     cnt = torch.zeros(1, dtype=torch.int64, device=dev)
-    out["mask_diff_once"] = once_stats(
-        time_once(lambda: [pkg.mllm_mask_diff(a, b, cnt) for _ in range(L) for a, b in zip(idx, other)]), B, 2, peak)
+    out["mask_diff_once"] = once_stats(time_once(lambda: pkg.mllm_mask_diff(flat, other, cnt)), B, 2, peak)
     D = 12 if w.nm == (2, 4) else 5
-    words = [torch.empty((t.numel() + D - 1) // D, dtype=torch.int32, device=dev) for t in idx]
-    out["encode_once"] = once_stats(
-        time_once(lambda: [pkg.mllm_encode_candidates(w.nm, t, wd) for _ in range(L) for t, wd in zip(idx, words)]),
-        B, 1 + 4.0 / D, peak)
+    words = torch.empty((B + D - 1) // D, dtype=torch.int32, device=dev)
+    out["encode_once"] = once_stats(time_once(lambda: pkg.mllm_encode_candidates(w.nm, flat, words)),
+                                    B, 1 + 4.0 / D, peak)
+    del other, words
     pri = [idx] * L
     arrs = [stack.view(l) for l in range(L)]
     out["prior_from_mask_once"] = once_stats(
@@ -393,7 +426,7 @@ def time_median(fn, reps=5):
     return float(np.median(out))
 
 
-def time_sparse_linear(stack, peak, token_counts=(1, 8, 16, 32, 64)):
+def time_sparse_linear(stack, peak, token_counts=(1, 8, 16, 32, 64, 128, 512, 2048)):
     """Serving the learned sparse network (s.3.2, inference): y = x W*^T for every matrix of
     the stack from its own packed hard mask (one mllm_sparse_linear call for all of them: a
     launch per 16 matrices), as
@@ -442,6 +475,8 @@ def time_sparse_linear(stack, peak, token_counts=(1, 8, 16, 32, 64)):
             "dense_cublas_ms": round(ms_dense, 4),
             "dense_cublas_gbs": round((dense_bytes + io) / (ms_dense / 1e3) / 1e9, 1),
             "speedup_vs_dense": round(ms_dense / ms, 3)}
+        if T > 64:
+            res[f"tokens_{T}"].update(tensor_stats(T, [(m.rows, m.cols) for _ in range(L) for m in w.matrices], ms))
     for mats in stack.bufs:
         for mb in mats:
             mb.pack_values = mb.pack_meta = None
@@ -898,7 +933,7 @@ def sparse_linear_arm(args, w):
         return float(np.median(out))
 
     res = {}
-    for T in (1, 8, 16, 32, 64):
+    for T in (1, 8, 16, 32, 64, 128, 512, 2048):
         xs = {c: torch.randn(T, c, device=dev, generator=gen).to(torch.bfloat16) for c in {c for _, c in shapes}}
         ys = [torch.empty(T, r, dtype=torch.float32, device=dev) for r, _ in shapes]
         arr = pkg.SparseOperandArray([(v, mt, xs[c], y) for (v, mt), (r, c), y in zip(packed, shapes, ys)])
@@ -910,6 +945,8 @@ def sparse_linear_arm(args, w):
                               "dense_cublas_ms": round(ms_d, 4),
                               "dense_cublas_gbs": round((dbytes + io) / (ms_d / 1e3) / 1e9, 1),
                               "speedup_vs_dense": round(ms_d / ms, 3)}
+        if T > 64:
+            res[f"tokens_{T}"].update(tensor_stats(T, shapes, ms))
     t8 = res["tokens_8"]
     return {"metric": "sparse_linear_bandwidth", "value": t8["achieved_gbs"], "unit": "GB/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t8["ms"], "higher_is_better": True,

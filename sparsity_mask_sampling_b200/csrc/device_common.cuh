@@ -113,6 +113,7 @@ struct StepScalars {
     uint32_t step;
     uint32_t noise_on;
     uint64_t seed;
+    uint32_t rk[20];     // Philox round keys of the seed: rk[2r], rk[2r+1] = k0 + r W0, k1 + r W1
 };
 
 __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -126,15 +127,25 @@ __device__ __forceinline__ int find_mat(const Group &g, int64_t t) {
 
 // ---------------------------------------------------------------------------- Philox
 
+// One Philox round: the two 32 x 32 -> 64-bit products (one wide multiply each), then the
+// S-box and the round key.
+__device__ __forceinline__ uint4 philox_round(uint4 c, uint32_t rk0, uint32_t rk1) {
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c.x, p1 = (uint64_t)0xCD9E8D57u * c.z;
+    return make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ rk0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ rk1, (uint32_t)p0);
+}
+
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
-    for (int r = 0; r < 10; ++r) {
-        const uint32_t rk0 = k0 + (uint32_t)r * 0x9E3779B9u;  // Weyl key schedule
-        const uint32_t rk1 = k1 + (uint32_t)r * 0xBB67AE85u;
-        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-        c = make_uint4(hi1 ^ c.y ^ rk0, lo1, hi0 ^ c.w ^ rk1, lo0);
-    }
+    for (int r = 0; r < 10; ++r)  // Weyl key schedule
+        c = philox_round(c, k0 + (uint32_t)r * 0x9E3779B9u, k1 + (uint32_t)r * 0xBB67AE85u);
+    return c;
+}
+
+// The same with the round keys of the launch's seed precomputed on the host (StepScalars::rk):
+// in an unrolled loop they are read straight from the kernel's parameters.
+__device__ __forceinline__ uint4 philox4x32_10_rk(uint4 c, const uint32_t (&rk)[20]) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) c = philox_round(c, rk[2 * r], rk[2 * r + 1]);
     return c;
 }
 
@@ -165,6 +176,11 @@ __device__ __forceinline__ void fields21_unit(uint4 x, uint32_t u[6]) {
 __device__ __forceinline__ uint4 block_words(uint64_t seed, uint64_t gid, uint32_t step, uint32_t group) {
     return philox4x32_10(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), step, group),
                          (uint32_t)seed, (uint32_t)(seed >> 32));
+}
+
+// block_words for a launch's step (seed and step from the step's scalars).
+__device__ __forceinline__ uint4 block_words(const StepScalars &sc, uint64_t gid, uint32_t group) {
+    return philox4x32_10_rk(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), sc.step, group), sc.rk);
 }
 
 // eps = (2k+1) 2^-22: the bit pattern of 1 + (2k+1) 2^-22 minus 1 (both exact).

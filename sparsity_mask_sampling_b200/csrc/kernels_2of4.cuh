@@ -91,16 +91,15 @@ __device__ __forceinline__ void store12(float *base, int64_t b0, bool two, const
 
 // --------------------------------------------------------------------------- per-block math
 
-// Gumbel noise of the block's six candidates: one Philox call, six fields.
-__device__ __forceinline__ void noise6(uint64_t seed, uint64_t gid, uint32_t step, bool on,
-                                       const NlogCtx &L, float g[6]) {
-    if (!on) {
+// Gumbel noise of the block's six candidates at the step of sc: one Philox call, six fields.
+__device__ __forceinline__ void noise6(const StepScalars &sc, uint64_t gid, const NlogCtx &L, float g[6]) {
+    if (!sc.noise_on) {
 #pragma unroll
         for (int i = 0; i < C; ++i) g[i] = 0.f;
         return;
     }
     uint32_t u[6];
-    fields21_unit(block_words(seed, gid, step, 0u), u);
+    fields21_unit(block_words(sc, gid, 0u), u);
 #pragma unroll
     for (int i = 0; i < C; ++i) g[i] = gumbel_unit(u[i], L);
 }
@@ -113,8 +112,11 @@ __device__ __forceinline__ void soft_index(const float *pi, const float g[6], fl
 #pragma unroll
     for (int i = 0; i < C; ++i) w[i] = __fmaf_rn(kappa, pi[i], g[i]);
     const float mx = fmaxf(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])), fmaxf(w[4], w[5]));
+    // (w_i - max) c2 as one fused step, w_i c2 - fl(max c2): the rounding of fl(max c2) is the
+    // same for all six and cancels in the normalisation
+    const float mc = __fmul_rn(mx, c2);
 #pragma unroll
-    for (int i = 0; i < C; ++i) e[i] = ex2_approx(__fmul_rn(__fsub_rn(w[i], mx), c2));
+    for (int i = 0; i < C; ++i) e[i] = ex2_approx(__fmaf_rn(w[i], c2, -mc));
     const float s = __fadd_rn(__fadd_rn(__fadd_rn(e[0], e[1]), __fadd_rn(e[2], e[3])), __fadd_rn(e[4], e[5]));
     r = rcp_approx(s);
 }
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const __grid_constant__ G
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             float g[6], e[6], r, ms[4];
-            noise6(sc.seed, d.gid0 + b0 + h, sc.step, sc.noise_on, L, g);
+            noise6(sc, d.gid0 + b0 + h, L, g);
             soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, r);
             soft_mask(e, r, ms);
 #pragma unroll
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) bwd_adam_kernel(const __grid_constan
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
-            noise6(sc.seed, d.gid0 + b0 + h, sc.step, sc.noise_on, L, g);
+            noise6(sc, d.gid0 + b0 + h, L, g);
             soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, r);
             soft_mask(e, r, ms);
             soft_mask_comp(e, r, mc);
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_adam_fwd_kernel(const __grid_
             const uint64_t gid = d.gid0 + b0 + h;
             {   // backward + AdamW, step t
                 float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
-                noise6(sb.seed, gid, sb.step, sb.noise_on, L, g);
+                noise6(sb, gid, L, g);
                 soft_index(pi + 6 * h, g, sb.kappa, sb.c2, e, r);
                 soft_mask(e, r, ms);
                 soft_mask_comp(e, r, mc);
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_adam_fwd_kernel(const __grid_
             }
             {   // forward, step t+1, from the updated logits
                 float g[6], e[6], r, ms[4];
-                noise6(sf.seed, gid, sf.step, sf.noise_on, L, g);
+                noise6(sf, gid, L, g);
                 soft_index(pi + 6 * h, g, sf.kappa, sf.c2, e, r);
                 soft_mask(e, r, ms);
 #pragma unroll

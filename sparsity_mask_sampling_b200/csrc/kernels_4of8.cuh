@@ -139,13 +139,13 @@ __device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) 
 // --------------------------------------------------------------------------- per-block math
 
 // Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates, and their maximum.
-__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t seed, uint64_t gid,
-                                           const StepScalars &sc, const NlogCtx &L, float w[C]) {
+__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
+                                           const NlogCtx &L, float w[C]) {
     float mx = -INFINITY;
 #pragma unroll
     for (int gr = 0; gr < 12; ++gr) {
         uint32_t f[6];
-        if (sc.noise_on) fields21(block_words(seed, gid, sc.step, (uint32_t)gr), f);
+        if (sc.noise_on) fields21(block_words(sc, gid, (uint32_t)gr), f);
 #pragma unroll
         for (int k = 0; k < 6; ++k) {
             const int c = 6 * gr + k;
@@ -166,10 +166,11 @@ __device__ __forceinline__ float soft_sums(float w[C], float mx, float c2, float
 #pragma unroll
     for (int j = 0; j < 8; ++j) { ms[j] = 0.f; mc[j] = 0.f; }
     float s = 0.f;
+    const float mc2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
     static_for<0, C>([&](auto I) {
         constexpr int c = decltype(I)::value;
         constexpr uint32_t mk = cand_mask(c);
-        const float e = ex2_approx(__fmul_rn(__fsub_rn(w[c], mx), c2));
+        const float e = ex2_approx(__fmaf_rn(w[c], c2, -mc2));
         w[c] = e;
         s += e;
 #pragma unroll
@@ -196,7 +197,7 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
 __device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8], const float gw[8], uint64_t gid,
                                          const StepScalars &sc, const NlogCtx &L, float *grow) {
     float w[C], ms[8], mc[8];
-    const float mx = perturbed(pi_row, sc.seed, gid, sc, L, w);
+    const float mx = perturbed(pi_row, gid, sc, L, w);
     const float r = rcp_approx(soft_sums<true>(w, mx, sc.c2, ms, mc));
     float P[8], Q[8];
 #pragma unroll
@@ -227,7 +228,7 @@ __device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8],
 __device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], uint64_t gid, const StepScalars &sc,
                                         const NlogCtx &L, float ms[8], float x[8], float &acc) {
     float w[C], mc[8];
-    const float mx = perturbed(pi_row, sc.seed, gid, sc, L, w);
+    const float mx = perturbed(pi_row, gid, sc, L, w);
     const float r = rcp_approx(soft_sums<false>(w, mx, sc.c2, ms, mc));
 #pragma unroll
     for (int j = 0; j < 8; ++j) {

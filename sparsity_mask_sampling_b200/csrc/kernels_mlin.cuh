@@ -143,7 +143,7 @@ __device__ __forceinline__ void gen_stage(unsigned char *tile, const Op &d, int6
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float g[6], e[6], rr, ms[4];
-                k24::noise6(sc.seed, d.gid0 + b0 + h, sc.step, sc.noise_on, L, g);
+                k24::noise6(sc, d.gid0 + b0 + h, L, g);
                 k24::soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, rr);
                 k24::soft_mask(e, rr, ms);
 #pragma unroll
@@ -478,7 +478,7 @@ __device__ __forceinline__ void pair_bwd_adam(const Op &d, int64_t b0, const flo
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
-        k24::noise6(sc.seed, d.gid0 + b0 + h, sc.step, sc.noise_on, L, g);
+        k24::noise6(sc, d.gid0 + b0 + h, L, g);
         k24::soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, r);
         k24::soft_mask(e, r, ms);
         k24::soft_mask_comp(e, r, mc);

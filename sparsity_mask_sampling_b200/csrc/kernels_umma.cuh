@@ -381,6 +381,242 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
     }
 }
 
+// ------------------------------------------------------------------ 2:4 prefill (more than 64 tokens)
+//
+// The same sparse MMA (M = 128 rows, K = 32 per instruction, metadata in tensor memory) with
+// N = 128 tokens. A unit of work is (operand, tile of 128 rows, chunk of 128 tokens) over all
+// the operand's columns; the units of a launch are ordered operand, row tile, token chunk, so a
+// CTA's consecutive units share one strip of compressed weights (read from HBM once, then from
+// L2). The host hands each CTA a contiguous range of whole units, balanced by their columns;
+// no unit is split between CTAs, so nothing is reduced across CTAs. The copy warp addresses
+// the token chunk through the activations' tensor map (rows past the call's tokens are
+// zero-filled) and the epilogue stores only rows of y inside it. Roles, stages, barriers,
+// bounded waits and wind-down as in sparse_linear_umma_kernel.
+
+constexpr int kPfTok = 128;                   // MMA N: tokens per unit
+constexpr int kPfMaxCtas = 160;
+constexpr unsigned kPfTmemCols = 256;         // accumulator 0..127, metadata from column 128
+constexpr unsigned kPfMetaCol = 128;
+
+struct PfOp {
+    const void *meta;
+    float *y;
+    int64_t rows, cols;
+    int64_t nch;         // 128-column chunks
+    int64_t ntiles;      // row tiles
+    int64_t nt;          // token chunks
+    int64_t unit_begin;  // first unit of this operand in the launch
+};
+
+struct PfGroup {
+    int32_t n;
+    int32_t tokens;
+    int32_t ubeg[kPfMaxCtas + 1];  // units [ubeg[c], ubeg[c+1]) belong to CTA c
+    PfOp d[kMaxMats];
+    TmMaps maps[kMaxMats];          // vals and meta as for the batched kernel; x boxes 64 x 128 tokens
+};
+
+struct PfCur {
+    int op;
+    int64_t tile, tc;
+};
+
+__device__ __forceinline__ PfCur pf_decode(const PfGroup &g, int64_t u) {
+    int i = 0;
+    while (i + 1 < g.n && u >= g.d[i + 1].unit_begin) ++i;
+    const int64_t r = u - g.d[i].unit_begin;
+    return PfCur{i, r / g.d[i].nt, r % g.d[i].nt};
+}
+
+__device__ __forceinline__ void pf_issue(const PfGroup &g, const PfCur &c, int64_t j, unsigned stage, unsigned bar) {
+    const TmMaps &mp = g.maps[c.op];
+    const int row0 = (int)(c.tile * kUmRows), tok0 = (int)(c.tc * kPfTok);
+    mbar_arrive_tx(bar, (unsigned)um_stage_tx<kPfTok>());
+    tma_load_2d(stage, &mp.vals, (int)(64 * j), row0, bar);
+    tma_load_2d(stage + kUmRows * 128, &mp.x, (int)(128 * j), tok0, bar);
+    tma_load_2d(stage + kUmRows * 128 + um_xbox_bytes<kPfTok>(), &mp.x, (int)(128 * j + 64), tok0, bar);
+    tma_load_2d(stage + kUmRows * 128 + 2 * um_xbox_bytes<kPfTok>(), &mp.meta, (int)(4 * j), row0, bar);
+}
+
+__global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(const __grid_constant__ PfGroup pg,
+                                                                            unsigned int *__restrict__ err) {
+    static_assert(um_smem_bytes<kPfTok>() + 1024 <= 232448, "fits one SM");
+    constexpr int kD = kUmStages, kStage = um_stage_bytes<kPfTok>();
+    constexpr uint32_t kIdesc = um_idesc<kPfTok>();
+    extern __shared__ unsigned char s_dyn_pf[];
+    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_meta[kD], s_acc;
+    __shared__ unsigned s_tmem;
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const int64_t u0 = pg.ubeg[cta], u1 = pg.ubeg[cta + 1];
+    const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_pf);
+    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
+    const unsigned char *ring = s_dyn_pf + pad;
+    const unsigned ring_s = dyn_s + pad;
+    const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
+    const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
+    const unsigned meta0 = (unsigned)__cvta_generic_to_shared(&s_meta[0]);
+    const unsigned accb = (unsigned)__cvta_generic_to_shared(&s_acc);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kD; ++s) {
+            mbar_init(full0 + 8 * s, 1u);
+            mbar_init(empty0 + 8 * s, 1u);
+            mbar_init(meta0 + 8 * s, 128u);
+        }
+        mbar_init(accb, 1u);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 0) {
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(&s_tmem);
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst),
+                     "r"(kPfTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const unsigned tbase = s_tmem;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ copy warp
+        int f = 0, issued = 0;
+        bool stop = false;
+        for (int64_t u = u0; u < u1 && !stop; ++u) {
+            const PfCur c = pf_decode(pg, u);
+            const int64_t nch = pg.d[c.op].nch;
+            for (int64_t j = 0; j < nch; ++j, ++f) {
+                const int s = f % kD;
+                if (f >= kD && !um_wait(empty0 + 8 * s, ((f / kD) - 1) & 1, &s_abort)) {
+                    if (lane == 0 && !s_abort) {
+                        atomicOr(err, 1u);
+                        s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    fence_proxy_async();
+                    pf_issue(pg, c, j, ring_s + s * kStage, full0 + 8 * s);
+                }
+                ++issued;
+            }
+        }
+        for (int s = 0; s < kD && s < issued; ++s) {
+            const int last = s + ((issued - 1 - s) / kD) * kD;
+            tm_wait(full0 + 8 * s, (last / kD) & 1);
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA warp
+        int f = 0, commits = 0;
+        bool stop = false;
+        for (int64_t u = u0; u < u1 && !stop; ++u) {
+            const PfCur c = pf_decode(pg, u);
+            const int64_t nch = pg.d[c.op].nch;
+            for (int64_t j = 0; j < nch; ++j, ++f) {
+                const int s = f % kD;
+                if (!um_wait(meta0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                    if (lane == 0 && !s_abort) {
+                        atomicOr(err, 1u);
+                        s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const unsigned st = ring_s + s * kStage;
+                    const uint64_t a0 = um_desc(st), b0 = um_desc(st + kUmRows * 128),
+                                   b1 = um_desc(st + kUmRows * 128 + um_xbox_bytes<kPfTok>());
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        umma_sp(tbase, a0 + (uint64_t)(2 * q), ((q >> 1) ? b1 : b0) + (uint64_t)(4 * (q & 1)),
+                                tbase + kPfMetaCol + 8 * s + 2 * q, kIdesc, (j == 0 && q == 0) ? 0u : 1u);
+                    umma_commit(empty0 + 8 * s);
+                    if (j == nch - 1) umma_commit(accb);
+                }
+                __syncwarp();
+                ++commits;
+            }
+        }
+        if (commits > 0) {
+            const int ff = commits - 1;
+            tm_wait(empty0 + 8 * (ff % kD), (ff / kD) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ metadata / epilogue warps
+        const unsigned tlane = tbase + ((unsigned)(32 * warp) << 16);
+        const int h = (lane >> 3) & 1;
+        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of the tile
+        const uint32_t esel = h ? 0x7632u : 0x5410u;
+        unsigned acc_phase = 0u;
+        bool failed = false;
+        int f = 0;
+        for (int64_t u = u0; u < u1; ++u) {
+            const PfCur c = pf_decode(pg, u);
+            const PfOp &d = pg.d[c.op];
+            for (int64_t j = 0; j < d.nch; ++j, ++f) {
+                const int s = f % kD;
+                if (!failed) {
+                    if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                        tc_fence_after();
+                        const unsigned char *meta = ring + s * kStage + kUmRows * 128 + 2 * um_xbox_bytes<kPfTok>();
+                        const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
+                        const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
+                        uint32_t e[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            e[q] = __byte_perm(a4[q] ? a4[q] : 0x44444444u, b4[q] ? b4[q] : 0x44444444u, esel);
+                        tmem_st_meta(tlane + kPfMetaCol + 8 * s, e[0], e[1], e[2], e[3]);
+                        tc_fence_before();
+                        mbar_arrive(meta0 + 8 * s);
+                    } else {
+                        failed = true;
+                        if (lane == 0 && !s_abort) {
+                            atomicOr(err, 1u);
+                            s_abort = 1;
+                        }
+                    }
+                }
+            }
+            // ---------------------------------------------------- epilogue of the unit
+            const bool acc_ok = !failed && um_wait(accb, acc_phase, &s_abort);
+            acc_phase ^= 1u;
+            if (um_bar_or<128>(!acc_ok)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            const int64_t r = c.tile * kUmRows + 32 * warp + lane;
+            const int tok0 = (int)(c.tc * kPfTok);
+#pragma unroll 1
+            for (int k = 0; k < kPfTok; k += 16) {
+                float v[16];
+                tmem_ld16(tlane + k, v);
+                if (r < d.rows) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (tok0 + k + i < pg.tokens) d.y[(int64_t)(tok0 + k + i) * d.rows + r] = v[i];
+                }
+            }
+            tc_fence_before();  // these reads precede the next unit's first MMA (after its arrivals)
+        }
+        if (failed && threadIdx.x == 0 && !s_abort) {
+            atomicOr(err, 1u);
+            s_abort = 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kPfTmemCols)
+                     : "memory");
+    }
+}
+
 // ------------------------------------------------------------------ 4:8 on the dense tensor cores
 //
 // 4:8 has no hardware sparse mode. Per 128-column stage, kU8Warps warps expand the compressed

@@ -172,6 +172,10 @@ StepScalars make_scalars(const mllm_hparams &hp) {
     s.step = hp.step;
     s.noise_on = hp.noise_on ? 1u : 0u;
     s.seed = hp.seed;
+    for (int r = 0; r < 10; ++r) {  // Philox4x32-10 key schedule (Weyl sequence), mod 2^32
+        s.rk[2 * r] = (uint32_t)hp.seed + (uint32_t)r * 0x9E3779B9u;
+        s.rk[2 * r + 1] = (uint32_t)(hp.seed >> 32) + (uint32_t)r * 0xBB67AE85u;
+    }
     return s;
 }
 
@@ -236,12 +240,13 @@ std::vector<Group> make_groups(const mllm_matrix *mats, int32_t n_mats, int M, K
 
 // ------------------------------------------------------------------------ sparse linear
 
+constexpr int kMaxCallTokens = 16384;  // tokens per mllm_sparse_linear call
 constexpr int kSplRowTiles = 2;   // row tiles of 16 per CTA task (4 warps per tile split k)
 constexpr int kSplDepth = 2;      // slabs in flight per warp
 
 mllm_status validate_operands(const mllm_sparse_operand *ops, int32_t n_ops, mllm_nm nm, int32_t tokens) {
     if (!num_cand(nm)) return MLLM_ERR_UNSUPPORTED;
-    if (!ops || n_ops <= 0 || tokens < 1 || tokens > spl::kMaxTokens) return MLLM_ERR_INVALID_ARG;
+    if (!ops || n_ops <= 0 || tokens < 1 || tokens > kMaxCallTokens) return MLLM_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_ops; ++i) {
         const mllm_sparse_operand &o = ops[i];
         if (o.rows < 0 || o.cols < 0 || o.cols % nm.m || o.rows > INT32_MAX || o.cols > INT32_MAX)
@@ -414,6 +419,67 @@ mllm_status noalloc_scratch(void **out) {
     if (!p) return MLLM_ERR_CUDA;
     *out = p;
     return MLLM_OK;
+}
+
+// 2:4 operands with cols % 128 == 0 above 64 tokens on the prefill kernel, 16 operands per
+// launch: units (operand, 128-row tile, 128-token chunk) split into contiguous whole-unit
+// ranges over the CTAs, balanced by columns. False if a tensor map cannot be encoded (nothing
+// is launched then).
+bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, unsigned int *err,
+                           cudaStream_t st, mllm_status *status) {
+    auto fn = spl::sparse_linear_prefill_kernel;
+    constexpr int smem = spl::um_smem_bytes<spl::kPfTok>();
+    int dev = 0;
+    cudaGetDevice(&dev);
+    resident_ctas(dev, (const void *)fn, spl::kUmThreads, smem);  // sets the dynamic shared-memory limit
+    for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
+        const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
+        static thread_local spl::PfGroup pg;
+        pg = spl::PfGroup{};
+        pg.tokens = tokens;
+        const int64_t nt = (tokens + spl::kPfTok - 1) / spl::kPfTok;
+        int64_t units = 0, chunks = 0;
+        for (size_t k = 0; k < n; ++k) {
+            const mllm_sparse_operand &o = ops[i0 + k];
+            spl::PfOp &d = pg.d[k];
+            d.meta = o.pack_meta;
+            d.y = o.y;
+            d.rows = o.rows;
+            d.cols = o.cols;
+            d.nch = o.cols / spl::kTmChunk;
+            d.ntiles = (o.rows + spl::kUmRows - 1) / spl::kUmRows;
+            d.nt = nt;
+            d.unit_begin = units;
+            units += d.ntiles * nt;
+            chunks += d.ntiles * nt * d.nch;
+            const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
+            if (!(encode_2d(&pg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  encode_2d(&pg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4,
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  encode_2d(&pg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
+                            (uint32_t)spl::kPfTok, CU_TENSOR_MAP_SWIZZLE_128B)))
+                return false;
+        }
+        pg.n = (int32_t)n;
+        const int64_t G = std::min<int64_t>({(int64_t)sm_count(dev), units, (int64_t)spl::kPfMaxCtas});
+        // unit u (first chunk at position p) goes to CTA floor(p G / chunks): contiguous ranges
+        int64_t u = 0, pos = 0;
+        for (int64_t c = 0; c <= G; ++c) {
+            while (u < units) {
+                int i = 0;
+                while (i + 1 < (int)n && u >= pg.d[i + 1].unit_begin) ++i;
+                if ((pos * G) / chunks >= c) break;
+                pos += pg.d[i].nch;
+                ++u;
+            }
+            pg.ubeg[c] = (int32_t)(c == G ? units : u);
+        }
+        fn<<<(unsigned)G, spl::kUmThreads, smem, st>>>(pg, err);
+        if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
+    }
+    *status = MLLM_OK;
+    return true;
 }
 
 // The per-warp kernels for up to 16 tokens; every operand has rows > 0 and cols > 0.
@@ -1054,8 +1120,30 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
         if (ops[i].cols % spl::kTmChunk == 0 && (tokens > spl::kMaxTileTokens || nm.m == 8)) batched.push_back(ops[i]);
         else act.push_back(ops[i]);
     }
-    if (!batched.empty() && !sparse_linear_batched(batched, nm, tokens, part, tickets, err, st, &s))
+    if (tokens > spl::kMaxTokens) {
+        // prefill-sized calls: 2:4 on the prefill kernel; 4:8 through the batched kernel in
+        // groups of 64 tokens (x and y rows offset)
+        if (!batched.empty() && nm.m == 4) {
+            if (!sparse_linear_prefill(batched, tokens, err, st, &s)) act.insert(act.end(), batched.begin(), batched.end());
+            if (s != MLLM_OK) return s;
+        } else if (!batched.empty()) {
+            for (int32_t t0 = 0; t0 < tokens; t0 += spl::kMaxTokens) {
+                std::vector<mllm_sparse_operand> grp = batched;
+                for (mllm_sparse_operand &o : grp) {
+                    o.x = static_cast<const char *>(o.x) + (size_t)t0 * (size_t)o.cols * 2;
+                    o.y = o.y + (size_t)t0 * (size_t)o.rows;
+                }
+                if (!sparse_linear_batched(grp, nm, std::min<int32_t>(spl::kMaxTokens, tokens - t0), part, tickets, err,
+                                           st, &s)) {
+                    act.insert(act.end(), batched.begin(), batched.end());
+                    break;
+                }
+                if (s != MLLM_OK) return s;
+            }
+        }
+    } else if (!batched.empty() && !sparse_linear_batched(batched, nm, tokens, part, tickets, err, st, &s)) {
         act.insert(act.end(), batched.begin(), batched.end());  // maps not encodable: token groups
+    }
     if (s != MLLM_OK) return s;
     if (act.empty()) return MLLM_OK;
     if (tokens <= spl::kMaxTileTokens) return sparse_linear_small(act, nm, tokens, part, tickets, err, st);
@@ -1080,7 +1168,8 @@ mllm_status mllm_sparse_linear_check_timeout(const mllm_sparse_operand *op, mllm
     if (s != MLLM_OK) return s;
     if (!workspace || workspace_bytes < spl::kSkWorkspaceBytes) return MLLM_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MLLM_ERR_MISALIGNED;
-    if (op->rows == 0 || op->cols == 0 || op->cols % spl::kTmChunk) return MLLM_ERR_UNSUPPORTED;
+    if (op->rows == 0 || op->cols == 0 || op->cols % spl::kTmChunk || tokens > spl::kMaxTokens)
+        return MLLM_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float *part = static_cast<float *>(workspace);
     unsigned int *tickets = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + spl::kPartBytes);

@@ -184,7 +184,7 @@ def _op(M, **kw):
 def test_sparse_linear_validation(M):
     assert _spl(M, []) == M.MLLM_ERR_INVALID_ARG
     assert _spl(M, [_op(M)], nm=(1, 4)) == M.MLLM_ERR_UNSUPPORTED
-    for tokens in (0, -1, 65):
+    for tokens in (0, -1, 16385):
         assert _spl(M, [_op(M)], tokens=tokens) == M.MLLM_ERR_INVALID_ARG, tokens
     assert _spl(M, [_op(M, cols=6)]) == M.MLLM_ERR_INVALID_ARG
     assert _spl(M, [_op(M, cols=12)], nm=(4, 8)) == M.MLLM_ERR_INVALID_ARG
@@ -214,7 +214,45 @@ def test_timeout_check_validation(M):
     assert call(_op(M, cols=64), nm=(4, 8)) == M.MLLM_ERR_UNSUPPORTED
     assert call(_op(M, cols=128), nm=(3, 8)) == M.MLLM_ERR_UNSUPPORTED
     assert call(_op(M, cols=132), nm=(4, 8)) == M.MLLM_ERR_INVALID_ARG
-    assert call(_op(M, cols=128), tokens=65) == M.MLLM_ERR_INVALID_ARG
+    assert call(_op(M, cols=128), tokens=65) == M.MLLM_ERR_UNSUPPORTED  # prefill sizes: not this test
+    assert call(_op(M, cols=128), tokens=16385) == M.MLLM_ERR_INVALID_ARG
     assert call(_op(M, cols=128, rows=0)) == M.MLLM_ERR_UNSUPPORTED
     assert call(_op(M, cols=128), ws=0) == M.MLLM_ERR_WORKSPACE
     assert call(_op(M, cols=128, x=0)) == M.MLLM_ERR_INVALID_ARG
+
+
+def _mlin(M, mats, ios, tokens=32, nm=(2, 4), bwd=False, ws=0x9000, wsb=None, hp=None):
+    L = M.lib()
+    arr = (M.Matrix * max(1, len(mats)))(*mats)
+    io = (M.LinearIO * max(1, len(ios)))(*ios)
+    wsb = M.mllm_masked_linear_workspace_bytes() if wsb is None else wsb
+    hp = _hp(M) if hp is None else hp
+    if bwd:
+        return L.mllm_masked_linear_bwd_adam(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(io, ctypes.c_void_p),
+                                             len(mats), M.NM(*nm), tokens, ctypes.byref(hp), ws, wsb, 0)
+    return L.mllm_masked_linear_fwd(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(io, ctypes.c_void_p), len(mats),
+                                    M.NM(*nm), tokens, ctypes.byref(hp), 0, ws, wsb, 0)
+
+
+def test_masked_linear_validation(M):
+    """The masked linear layer's calls reject what they do not support before any launch."""
+    assert ctypes.sizeof(M.LinearIO) == M.lib().mllm_sizeof_linear_io()
+    mat = _mat(M, rows=128, cols=128)
+    io = M.LinearIO(x=0xA000, y=0xB000, dy=0xC000)
+    for bwd in (False, True):
+        assert _mlin(M, [mat], [io], nm=(4, 8), bwd=bwd) == M.MLLM_ERR_UNSUPPORTED
+        assert _mlin(M, [_mat(M, rows=128, cols=128, w_dtype=1)], [io], bwd=bwd) == M.MLLM_ERR_UNSUPPORTED
+        assert _mlin(M, [_mat(M, rows=128, cols=96)], [io], bwd=bwd) == M.MLLM_ERR_UNSUPPORTED
+        for tokens in (0, -1, 257):
+            assert _mlin(M, [mat], [io], tokens=tokens, bwd=bwd) == M.MLLM_ERR_INVALID_ARG, tokens
+        assert _mlin(M, [mat], [M.LinearIO(x=0, y=0xB000, dy=0xC000)], bwd=bwd) == M.MLLM_ERR_INVALID_ARG
+        assert _mlin(M, [mat], [M.LinearIO(x=0xA008, y=0xB000, dy=0xC000)], bwd=bwd) == M.MLLM_ERR_MISALIGNED
+        assert _mlin(M, [mat], [io], bwd=bwd, ws=0) == M.MLLM_ERR_WORKSPACE
+        assert _mlin(M, [mat], [io], bwd=bwd, wsb=M.mllm_masked_linear_workspace_bytes() - 16) == M.MLLM_ERR_WORKSPACE
+        assert _mlin(M, [mat], [io], bwd=bwd, ws=0x9008) == M.MLLM_ERR_MISALIGNED
+    assert _mlin(M, [mat], [M.LinearIO(x=0xA000, y=0, dy=0xC000)]) == M.MLLM_ERR_INVALID_ARG
+    assert _mlin(M, [mat], [M.LinearIO(x=0xA000, y=0xB000, dy=0)], bwd=True) == M.MLLM_ERR_INVALID_ARG
+    assert _mlin(M, [_mat(M, rows=100, cols=128)], [io], bwd=True) == M.MLLM_ERR_UNSUPPORTED  # rows % 8
+    assert _mlin(M, [_mat(M, rows=128, cols=128, adam_m=0)], [io], bwd=True) == M.MLLM_ERR_INVALID_ARG
+    assert _mlin(M, [mat], [io], bwd=True, hp=_hp(M, adam_step=0)) == M.MLLM_ERR_INVALID_ARG
+    assert _mlin(M, [mat], [io], hp=_hp(M, tau=0.0)) == M.MLLM_ERR_INVALID_ARG
