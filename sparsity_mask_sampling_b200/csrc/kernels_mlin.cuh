@@ -48,6 +48,7 @@ using spl::tc_fence_before;
 using spl::tm_wait;
 using spl::tma_load_2d;
 using spl::tmem_ld16;
+using spl::tmem_ld8;
 using spl::um_bar;
 using spl::um_bar_or;
 using spl::um_desc;
@@ -57,7 +58,7 @@ using spl::umma_dense;
 
 constexpr int kRows = 128;          // MMA M: rows of W per tile
 constexpr int kChunk = 64;          // columns of W per stage (one 128-byte atom of bf16)
-constexpr int kProdWarps = 8;       // producer / epilogue warps
+constexpr int kProdWarps = 16;      // producer / epilogue warps
 constexpr int kProd = 32 * kProdWarps;
 constexpr int kThreads = kProd + 64;  // + the copy warp and the MMA warp
 constexpr int kStages = 3;
@@ -124,15 +125,17 @@ __device__ __forceinline__ void advance(const Group &g, Cur &c) {
     }
 }
 
-// The producers' part of a stage: rows r0 + 32 i (i < 4) and pair slot c (columns 8c .. 8c+7
+// The producers' part of a stage: rows r0 + 64 i (i < 2) and pair slot c (columns 8c .. 8c+7
 // of the chunk) of the 128 x 64 tile of X, computed by the 2:4 forward's arithmetic (k24) and
 // written as one 16-byte chunk at its 128-byte-swizzled place. Rows past the matrix are zero.
+constexpr int kRowStep = kProd / 8;            // rows a producer steps by (8 pair slots per row)
+constexpr int kPairsPerThread = kRows / kRowStep;
 __device__ __forceinline__ void gen_stage(unsigned char *tile, const Op &d, int64_t row_tile, int64_t j, int c,
                                           int r0, const StepScalars &sc, const NlogCtx &L, float &acc) {
     const int64_t bpr = d.cols >> 2;
-#pragma unroll 1
-    for (int i = 0; i < 4; ++i) {
-        const int r = r0 + 32 * i;
+#pragma unroll
+    for (int i = 0; i < kPairsPerThread; ++i) {
+        const int r = r0 + kRowStep * i;
         const int64_t row = row_tile * kRows + r;
         uint4 packed = make_uint4(0u, 0u, 0u, 0u);
         if (row < d.rows) {
@@ -209,11 +212,13 @@ template <int kN>
 __global__ void __launch_bounds__(kThreads, 1) masked_linear_fwd_kernel(const __grid_constant__ Group grp,
                                                                         const StepScalars sc, unsigned char *ws,
                                                                         double *reg_out, int accumulate) {
-    static_assert(kN % 32 == 0 && kN >= 32 && kN <= kMaxTokens, "N of an M = 128 MMA, two halves of 16k");
+    static_assert(kN % 32 == 0 && kN >= 32 && kN <= kMaxTokens, "N of an M = 128 MMA");
+    static_assert(kN % (8 * (kProdWarps / 4)) == 0, "each epilogue warp takes a multiple of 8 token columns");
     static_assert(smem_bytes<kN>() + 2 * kNlogEntries * 4 + 1024 <= 232448, "fits one SM");
     constexpr int kD = kStages, kStage = stage_bytes<kN>();
     constexpr uint32_t kIdesc = spl::u8_idesc<kN>();  // dense, f32 accumulator, bf16 K-major, M = 128
-    constexpr int kHalf = kN / 2;                       // token columns per epilogue warp
+    constexpr int kSlices = kProdWarps / 4;              // epilogue warps per TMEM lane quarter
+    constexpr int kHalf = kN / kSlices;                  // token columns per epilogue warp (a multiple of 8)
     extern __shared__ unsigned char s_dyn_ml[];
     __shared__ __align__(16) float2 s_tab[kNlogEntries];
     __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_gen[kD], s_acc;
@@ -325,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) masked_linear_fwd_kernel(const __
         // ------------------------------------------------------------ producer / epilogue warps
         const NlogCtx L{s_tab};
         const int pc = threadIdx.x & 7, r0 = threadIdx.x >> 3;
-        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token half of the epilogue
+        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
         const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
         Cur cc = decode(grp, lo);
         unsigned acc_phase = 0u;
@@ -361,10 +366,10 @@ __global__ void __launch_bounds__(kThreads, 1) masked_linear_fwd_kernel(const __
                 const int tok0 = ch * kHalf;
                 if (c1 == c2) {
 #pragma unroll 1
-                    for (int k = 0; k < kHalf; k += 16) {
-                        float v[16];
-                        tmem_ld16(tq + k, v);
-                        store_cols<kN>(d, cc.tile, q, lane, tok0 + k, v, 16, grp.tokens);
+                    for (int k = 0; k < kHalf; k += 8) {
+                        float v[8];
+                        tmem_ld8(tq + k, v);
+                        store_cols<kN>(d, cc.tile, q, lane, tok0 + k, v, 8, grp.tokens);
                     }
                     tc_fence_before();  // these reads precede the next piece's first MMA
                 } else {
@@ -372,11 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1) masked_linear_fwd_kernel(const __
                     const int slot = (cta == c1 && lo1 < a) ? 1 : 0;
                     float *mine = part + (size_t)(cta * 2 + slot) * kPartFloats + (size_t)tok0 * kRows + 32 * q + lane;
 #pragma unroll 1
-                    for (int k = 0; k < kHalf; k += 16) {
-                        float v[16];
-                        tmem_ld16(tq + k, v);
+                    for (int k = 0; k < kHalf; k += 8) {
+                        float v[8];
+                        tmem_ld8(tq + k, v);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) __stcg(mine + (size_t)(k + i) * kRows, v[i]);
+                        for (int i = 0; i < 8; ++i) __stcg(mine + (size_t)(k + i) * kRows, v[i]);
                     }
                     tc_fence_before();
                     __threadfence();
@@ -386,18 +391,18 @@ __global__ void __launch_bounds__(kThreads, 1) masked_linear_fwd_kernel(const __
                     if (s_last) {
                         __threadfence();
 #pragma unroll 1
-                        for (int k = 0; k < kHalf; k += 16) {
-                            float sum[16];
+                        for (int k = 0; k < kHalf; k += 8) {
+                            float sum[8];
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) sum[i] = 0.f;
+                            for (int i = 0; i < 8; ++i) sum[i] = 0.f;
                             for (int64_t qq = c1; qq <= c2; ++qq) {
                                 const int sid = (qq == c1 && lo1 < a) ? 1 : 0;
                                 const float *p = part + (size_t)(qq * 2 + sid) * kPartFloats +
                                                  (size_t)(tok0 + k) * kRows + 32 * q + lane;
 #pragma unroll
-                                for (int i = 0; i < 16; ++i) sum[i] += __ldcg(p + (size_t)i * kRows);
+                                for (int i = 0; i < 8; ++i) sum[i] += __ldcg(p + (size_t)i * kRows);
                             }
-                            store_cols<kN>(d, cc.tile, q, lane, tok0 + k, sum, 16, grp.tokens);
+                            store_cols<kN>(d, cc.tile, q, lane, tok0 + k, sum, 8, grp.tokens);
                         }
                         um_bar<kProd>();
                         if (threadIdx.x == 0) tickets[c1] = 0u;
@@ -636,8 +641,9 @@ __global__ void __launch_bounds__(kThreads, 1) masked_linear_bwd_adam_kernel(con
     } else {
         // ------------------------------------------------------------ epilogue warps
         const NlogCtx L{s_tab};
-        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, column half
-        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * 64);
+        constexpr int kCw = kBwdCols / (kProdWarps / 4);  // accumulator columns per epilogue warp
+        const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, column slice
+        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kCw);
         const int tid = threadIdx.x;
         bool failed = false;
         for (int it = 0; it < ntile; ++it) {
@@ -651,9 +657,9 @@ __global__ void __launch_bounds__(kThreads, 1) masked_linear_bwd_adam_kernel(con
             bwd_decode(grp, cta + (int64_t)it * G, op, rt, ct);
             const Op &d = grp.d[op];
             tc_fence_after();
-            float *grow = s_g + (32 * q + lane) * kGPitch + ch * 64;
+            float *grow = s_g + (32 * q + lane) * kGPitch + ch * kCw;
 #pragma unroll 1
-            for (int k = 0; k < 64; k += 16) {
+            for (int k = 0; k < kCw; k += 16) {
                 float v[16];
                 tmem_ld16(tq + k, v);
 #pragma unroll

@@ -385,12 +385,15 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
 //
 // The same sparse MMA (M = 128 rows, K = 32 per instruction, metadata in tensor memory) with
 // N = 128 tokens. A unit of work is (operand, tile of 128 rows, chunk of 128 tokens) over all
-// the operand's columns; the units of a launch are ordered operand, row tile, token chunk, so a
-// CTA's consecutive units share one strip of compressed weights (read from HBM once, then from
-// L2). The host hands each CTA a contiguous range of whole units, balanced by their columns;
-// no unit is split between CTAs, so nothing is reduced across CTAs. The copy warp addresses
-// the token chunk through the activations' tensor map (rows past the call's tokens are
-// zero-filled) and the epilogue stores only rows of y inside it. Roles, stages, barriers,
+// the operand's columns; no unit is split between CTAs, so nothing is reduced across CTAs.
+// CTA c takes units c, c + G, c + 2G, ... of a sequence ordered so that the G units in flight
+// at any time share few weight strips and all token chunks: per operand, groups of R row tiles
+// (R = ceil(G / token chunks)), within a group token chunk by token chunk, within a chunk the
+// group's row tiles. The strips and chunks of the activations in flight then fit in L2, so a
+// strip is read from HBM about once per group instead of once per token chunk. The host
+// orders the operands by decreasing columns (the longest units first). The copy warp
+// addresses the token chunk through the activations' tensor map (rows past the call's tokens
+// are zero-filled) and the epilogue stores only rows of y inside it. Roles, stages, barriers,
 // bounded waits and wind-down as in sparse_linear_umma_kernel.
 
 constexpr int kPfTok = 128;                   // MMA N: tokens per unit
@@ -405,15 +408,16 @@ struct PfOp {
     int64_t nch;         // 128-column chunks
     int64_t ntiles;      // row tiles
     int64_t nt;          // token chunks
+    int64_t rgroup;      // row tiles per group of the unit order
     int64_t unit_begin;  // first unit of this operand in the launch
 };
 
 struct PfGroup {
     int32_t n;
     int32_t tokens;
-    int32_t ubeg[kPfMaxCtas + 1];  // units [ubeg[c], ubeg[c+1]) belong to CTA c
+    int64_t total_units;
     PfOp d[kMaxMats];
-    TmMaps maps[kMaxMats];          // vals and meta as for the batched kernel; x boxes 64 x 128 tokens
+    TmMaps maps[kMaxMats];  // vals and meta as for the batched kernel; x boxes 64 x 128 tokens
 };
 
 struct PfCur {
@@ -424,8 +428,11 @@ struct PfCur {
 __device__ __forceinline__ PfCur pf_decode(const PfGroup &g, int64_t u) {
     int i = 0;
     while (i + 1 < g.n && u >= g.d[i + 1].unit_begin) ++i;
-    const int64_t r = u - g.d[i].unit_begin;
-    return PfCur{i, r / g.d[i].nt, r % g.d[i].nt};
+    const PfOp &d = g.d[i];
+    const int64_t idx = u - d.unit_begin, per = d.rgroup * d.nt;
+    const int64_t grp = idx / per, rem = idx % per;
+    const int64_t rg = d.ntiles - grp * d.rgroup < d.rgroup ? d.ntiles - grp * d.rgroup : d.rgroup;
+    return PfCur{i, grp * d.rgroup + rem % rg, rem / rg};
 }
 
 __device__ __forceinline__ void pf_issue(const PfGroup &g, const PfCur &c, int64_t j, unsigned stage, unsigned bar) {
@@ -448,8 +455,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
     __shared__ unsigned s_tmem;
     __shared__ volatile int s_abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cta = blockIdx.x;
-    const int64_t u0 = pg.ubeg[cta], u1 = pg.ubeg[cta + 1];
+    const int64_t G = gridDim.x, u0 = blockIdx.x, u1 = pg.total_units;
     const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_pf);
     const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
     const unsigned char *ring = s_dyn_pf + pad;
@@ -484,7 +490,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         // ------------------------------------------------------------ copy warp
         int f = 0, issued = 0;
         bool stop = false;
-        for (int64_t u = u0; u < u1 && !stop; ++u) {
+        for (int64_t u = u0; u < u1 && !stop; u += G) {
             const PfCur c = pf_decode(pg, u);
             const int64_t nch = pg.d[c.op].nch;
             for (int64_t j = 0; j < nch; ++j, ++f) {
@@ -512,7 +518,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         // ------------------------------------------------------------ MMA warp
         int f = 0, commits = 0;
         bool stop = false;
-        for (int64_t u = u0; u < u1 && !stop; ++u) {
+        for (int64_t u = u0; u < u1 && !stop; u += G) {
             const PfCur c = pf_decode(pg, u);
             const int64_t nch = pg.d[c.op].nch;
             for (int64_t j = 0; j < nch; ++j, ++f) {
@@ -554,7 +560,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         unsigned acc_phase = 0u;
         bool failed = false;
         int f = 0;
-        for (int64_t u = u0; u < u1; ++u) {
+        for (int64_t u = u0; u < u1; u += G) {
             const PfCur c = pf_decode(pg, u);
             const PfOp &d = pg.d[c.op];
             for (int64_t j = 0; j < d.nch; ++j, ++f) {

@@ -422,11 +422,14 @@ mllm_status noalloc_scratch(void **out) {
 }
 
 // 2:4 operands with cols % 128 == 0 above 64 tokens on the prefill kernel, 16 operands per
-// launch: units (operand, 128-row tile, 128-token chunk) split into contiguous whole-unit
-// ranges over the CTAs, balanced by columns. False if a tensor map cannot be encoded (nothing
+// launch (longest rows first): units (operand, 128-row tile, 128-token chunk) dealt round-robin
+// over the CTAs in the kernel's group order. False if a tensor map cannot be encoded (nothing
 // is launched then).
-bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, unsigned int *err,
+bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32_t tokens, unsigned int *err,
                            cudaStream_t st, mllm_status *status) {
+    std::vector<mllm_sparse_operand> ops = ops_in;
+    std::stable_sort(ops.begin(), ops.end(),
+                     [](const mllm_sparse_operand &a, const mllm_sparse_operand &b) { return a.cols > b.cols; });
     auto fn = spl::sparse_linear_prefill_kernel;
     constexpr int smem = spl::um_smem_bytes<spl::kPfTok>();
     int dev = 0;
@@ -438,7 +441,8 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops, int32_t 
         pg = spl::PfGroup{};
         pg.tokens = tokens;
         const int64_t nt = (tokens + spl::kPfTok - 1) / spl::kPfTok;
-        int64_t units = 0, chunks = 0;
+        const int64_t G0 = std::min<int64_t>((int64_t)sm_count(dev), (int64_t)spl::kPfMaxCtas);
+        int64_t units = 0;
         for (size_t k = 0; k < n; ++k) {
             const mllm_sparse_operand &o = ops[i0 + k];
             spl::PfOp &d = pg.d[k];
@@ -449,9 +453,9 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops, int32_t 
             d.nch = o.cols / spl::kTmChunk;
             d.ntiles = (o.rows + spl::kUmRows - 1) / spl::kUmRows;
             d.nt = nt;
+            d.rgroup = std::max<int64_t>(1, (G0 + nt - 1) / nt);
             d.unit_begin = units;
             units += d.ntiles * nt;
-            chunks += d.ntiles * nt * d.nch;
             const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
             if (!(encode_2d(&pg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
                             spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -462,19 +466,8 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops, int32_t 
                 return false;
         }
         pg.n = (int32_t)n;
-        const int64_t G = std::min<int64_t>({(int64_t)sm_count(dev), units, (int64_t)spl::kPfMaxCtas});
-        // unit u (first chunk at position p) goes to CTA floor(p G / chunks): contiguous ranges
-        int64_t u = 0, pos = 0;
-        for (int64_t c = 0; c <= G; ++c) {
-            while (u < units) {
-                int i = 0;
-                while (i + 1 < (int)n && u >= pg.d[i + 1].unit_begin) ++i;
-                if ((pos * G) / chunks >= c) break;
-                pos += pg.d[i].nch;
-                ++u;
-            }
-            pg.ubeg[c] = (int32_t)(c == G ? units : u);
-        }
+        pg.total_units = units;
+        const int64_t G = std::min<int64_t>(G0, units);
         fn<<<(unsigned)G, spl::kUmThreads, smem, st>>>(pg, err);
         if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
     }
