@@ -4,18 +4,11 @@
 // to 4:8 as the method states (N:M with C(M,N) candidates); the candidate order is the
 // lexicographic order of the ascending position 4-tuples.
 //
-// Work mapping of the sampler kernels (forward, backward + AdamW, fused step): a CTA of
-// kSampThreads = 256 threads takes a tile of kBlocksPerCta = 128 blocks; thread t works on
-// block t % 128, and its warp group h = t / 128 takes half of the block's candidates (h = 0:
-// candidates 0..35, Philox groups 0..5; h = 1: 36..69, groups 6..11), fully unrolled, so that
+// Work mapping: one thread owns one block and walks all 70 candidates fully unrolled, so
 // every candidate's keep mask is a compile-time constant (no divergence, no table lookups).
-// The two halves meet twice per soft mask through shared memory: their maxima, then their
-// partial sums (sum e, and per position the kept and pruned sums), which every thread adds in
-// the fixed order half 0 + half 1, so that the forward and the backward form identical soft
-// masks. A block's logits are 280 B, so a thread reading its own row from global memory would
-// make each warp access stride 280 B; instead a CTA stages its tile's logit rows through
-// shared memory with coalesced copies, and AdamW runs as a flat, coalesced pass over the tile.
-// The prior initialisation and the hard pack keep one thread per block (kCtaThreads).
+// A block's logits are 280 B, so a thread reading its own row would make each warp access
+// stride 280 B; instead a CTA stages its tile of kBlocksPerCta logit rows through shared
+// memory with coalesced copies, and AdamW runs as a flat, coalesced pass over the tile.
 #pragma once
 
 #include <type_traits>
@@ -26,19 +19,11 @@ namespace mllm {
 namespace k48 {
 
 constexpr int C = 70;
-constexpr int kCtaThreads = 128;            // prior init and hard pack: one thread per block
-constexpr int kBlocksPerCta = kCtaThreads;  // blocks per tile (every kernel)
-constexpr int kSampThreads = 2 * kBlocksPerCta;  // sampler kernels: two threads per block
+constexpr int kCtaThreads = 128;
+constexpr int kBlocksPerCta = kCtaThreads;  // one block per thread
 constexpr int kTileFloats = kBlocksPerCta * C;
-constexpr int kParts = 17;                  // partial sums a half hands over: sum e, 8 kept, 8 pruned
-constexpr int kFwdParts = 9;                // the forward's: sum e, 8 kept
-constexpr int kXchgFloats = 2 * kFwdParts * kBlocksPerCta + 2 * kBlocksPerCta;  // forward partials + maxima
-// forward: tile + exchange; backward: tile + gradients (the exchange's partials overlay the
-// gradient buffer) + maxima; fused: two tile buffers + the forward's exchange (with the
-// 27 KB table: three, two and two CTAs per SM)
-constexpr int kFwdDynSmem = (kTileFloats + kXchgFloats) * (int)sizeof(float);
-constexpr int kBwdDynSmem = (2 * kTileFloats + 2 * kBlocksPerCta) * (int)sizeof(float);
-constexpr int kFusedDynSmem = (2 * kTileFloats + kXchgFloats) * (int)sizeof(float);
+constexpr int kFwdDynSmem = kTileFloats * (int)sizeof(float);
+constexpr int kBwdDynSmem = 2 * kTileFloats * (int)sizeof(float);
 
 // Keep mask (bit j = position j) of candidate i: the i-th 4-subset of {0..7} in
 // lexicographic order of ascending index tuples. Only ever evaluated at compile time.
@@ -87,7 +72,7 @@ __device__ __forceinline__ void cp_async_wait_all() {
 
 __device__ __forceinline__ void stage_in(float *dst, const float *src, int n) {
     const int n4 = n >> 2;  // whole 16-byte chunks
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
+    for (int i = threadIdx.x; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
     if ((n & 3) && threadIdx.x == 0) {  // n = nb*70 is even: at most one 8-byte tail
         *reinterpret_cast<float2 *>(dst + 4 * n4) = __ldcs(reinterpret_cast<const float2 *>(src + 4 * n4));
     }
@@ -103,7 +88,7 @@ __device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
 }
 __device__ __forceinline__ void stage_in_async(float *dst, const float *src, int n) {
     const int n4 = n >> 2;
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
+    for (int i = threadIdx.x; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
     if ((n & 3) && threadIdx.x == 0) cp_async8(dst + 4 * n4, src + 4 * n4);
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -113,7 +98,7 @@ __device__ __forceinline__ void cp_async_wait_pending() {
 
 __device__ __forceinline__ void stage_out(float *dst, const float *src, int n) {
     const int n4 = n >> 2;
-    for (int i = threadIdx.x; i < n4; i += blockDim.x)
+    for (int i = threadIdx.x; i < n4; i += kCtaThreads)
         __stcs(reinterpret_cast<float4 *>(dst) + i, reinterpret_cast<const float4 *>(src)[i]);
     if ((n & 3) && threadIdx.x == 0)
         __stcs(reinterpret_cast<float2 *>(dst + 4 * n4), *reinterpret_cast<const float2 *>(src + 4 * n4));
@@ -153,18 +138,12 @@ __device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) 
 
 // --------------------------------------------------------------------------- per-block math
 
-// Candidates of half H: [kC0<H>, kC0<H> + kCn<H>), Philox groups [6H, 6H + 6).
-template <int H> constexpr int kC0 = 36 * H;
-template <int H> constexpr int kCn = H ? C - 36 : 36;
-
-// Perturbed logits w_c = fma(kappa, pi_c, g_c) of the half's candidates (w[c - kC0]), and
-// their maximum.
-template <int H>
-__device__ __forceinline__ float perturbed_half(const float *pi_row, uint64_t gid, const StepScalars &sc,
-                                                const NlogCtx &L, float w[36]) {
+// Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates, and their maximum.
+__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
+                                           const NlogCtx &L, float w[C]) {
     float mx = -INFINITY;
 #pragma unroll
-    for (int gr = 6 * H; gr < 6 * H + 6; ++gr) {
+    for (int gr = 0; gr < 12; ++gr) {
         uint32_t f[6];
         if (sc.noise_on) fields21(block_words(sc, gid, (uint32_t)gr), f);
 #pragma unroll
@@ -172,95 +151,35 @@ __device__ __forceinline__ float perturbed_half(const float *pi_row, uint64_t gi
             const int c = 6 * gr + k;
             if (c < C) {
                 const float g = sc.noise_on ? gumbel(f[k], L) : 0.f;
-                w[c - kC0<H>] = __fmaf_rn(sc.kappa, pi_row[c], g);
-                mx = fmaxf(mx, w[c - kC0<H>]);
+                w[c] = __fmaf_rn(sc.kappa, pi_row[c], g);
+                mx = fmaxf(mx, w[c]);
             }
         }
     }
     return mx;
 }
 
-// Over the half's candidates: e_c = 2^((w_c - max) c2) in place (w c2 - fl(max c2): a
-// common rounding that cancels in the normalisation); part[0] = sum e, part[1 + j] = sum of e
-// over candidates keeping position j, and with kComp part[9 + j] = sum over those pruning it.
-template <int H, bool kComp>
-__device__ __forceinline__ void soft_half(float w[36], float mx, float c2, float part[kParts]) {
+// e_c = 2^((w_c - max) c2) in place; returns sum e; ms[j] = sum_{c: j in S_c} e_c and, when
+// kComp, mc[j] = sum_{c: j not in S_c} e_c.
+template <bool kComp>
+__device__ __forceinline__ float soft_sums(float w[C], float mx, float c2, float ms[8], float mc[8]) {
 #pragma unroll
-    for (int k = 0; k < kParts; ++k) part[k] = 0.f;
-    const float mc2 = __fmul_rn(mx, c2);
-    static_for<kC0<H>, kC0<H> + kCn<H>>([&](auto I) {
+    for (int j = 0; j < 8; ++j) { ms[j] = 0.f; mc[j] = 0.f; }
+    float s = 0.f;
+    const float mc2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
+    static_for<0, C>([&](auto I) {
         constexpr int c = decltype(I)::value;
         constexpr uint32_t mk = cand_mask(c);
-        const float e = ex2_approx(__fmaf_rn(w[c - kC0<H>], c2, -mc2));
-        w[c - kC0<H>] = e;
-        part[0] += e;
+        const float e = ex2_approx(__fmaf_rn(w[c], c2, -mc2));
+        w[c] = e;
+        s += e;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            if (mk & (1u << j)) part[1 + j] += e;
-            else if (kComp) part[9 + j] += e;
+            if (mk & (1u << j)) ms[j] += e;
+            else if (kComp) mc[j] += e;
         }
     });
-}
-
-// Gradients of the half's candidates from the combined sums tot (sum e, kept and pruned sums
-// per position) and the half's e values: dpi_c = (kappa/tau) y_c (sum_{j in S_c} P_j -
-// sum_{j not in S_c} Q_j), P_j = (1 - M_j) u_j, Q_j = M_j u_j, u_j = G_j W_j - 2 lambda W_j^2 M_j.
-template <int H>
-__device__ __forceinline__ void grads_half(const float e[36], const float tot[kParts], const float wt[8],
-                                           const float gw[8], const StepScalars &sc, float *grow) {
-    const float r = rcp_approx(tot[0]);
-    float P[8], Q[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float ms = __fmul_rn(tot[1 + j], r), mc = __fmul_rn(tot[9 + j], r);
-        const float wj = wt[j];
-        const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms, __fmul_rn(gw[j], wj));
-        P[j] = __fmul_rn(mc, u);
-        Q[j] = __fmul_rn(ms, u);
-    }
-    const float cr = __fmul_rn(sc.kappa_over_tau, r);
-    static_for<kC0<H>, kC0<H> + kCn<H>>([&](auto I) {
-        constexpr int c = decltype(I)::value;
-        constexpr uint32_t mk = cand_mask(c);
-        float kept = 0.f, pruned = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (mk & (1u << j)) kept += P[j];
-            else pruned += Q[j];
-        }
-        grow[c] = __fmul_rn(__fmul_rn(cr, e[c - kC0<H>]), kept - pruned);
-    });
-}
-
-// The soft index of a tile's blocks, split between the two halves (h = thread / 128), in two
-// phases that every thread of the CTA calls (one CTA barrier each, outside any branch; active
-// = the thread's block exists). Phase 1: the half's perturbed logits w (into e[]) and the
-// exchange of maxima; returns the block's maximum. Phase 2: e = 2^((w - max) c2) in place and
-// the half's partial sums, the exchange of partial sums; tot[0 .. kN) receives the combined
-// sums (half 0 + half 1, the same order in every kernel).
-__device__ __forceinline__ float soft_phase1(bool active, int h, int blk, const float *pi_row, uint64_t gid,
-                                             const StepScalars &sc, const NlogCtx &L, float *xm, float e[36]) {
-    float mx = -INFINITY;
-    if (active) mx = h ? perturbed_half<1>(pi_row, gid, sc, L, e) : perturbed_half<0>(pi_row, gid, sc, L, e);
-    xm[h * kBlocksPerCta + blk] = mx;
-    __syncthreads();
-    return fmaxf(xm[blk], xm[kBlocksPerCta + blk]);
-}
-template <int kN>
-__device__ __forceinline__ void soft_phase2(bool active, int h, int blk, float mx, float c2, float *xp, float e[36],
-                                            float tot[kN]) {
-    constexpr bool kComp = kN > kFwdParts;
-    if (active) {
-        float part[kParts];
-        if (h) soft_half<1, kComp>(e, mx, c2, part);
-        else soft_half<0, kComp>(e, mx, c2, part);
-#pragma unroll
-        for (int k = 0; k < kN; ++k) xp[(h * kN + k) * kBlocksPerCta + blk] = part[k];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kN; ++k)
-        tot[k] = __fadd_rn(xp[k * kBlocksPerCta + blk], xp[(kN + k) * kBlocksPerCta + blk]);
+    return s;
 }
 
 // AdamW, PyTorch step order, one element.
@@ -272,6 +191,53 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
     p = __fmaf_rn(-s.step_size, __fdividef(m, denom), pd);
 }
 
+// Gradient of one block's logits (Eq.6-Eq.8 backward, noise of step sc.step) into grow[C]:
+// dpi_c = (kappa/tau) y_c (sum_{j in S_c} P_j - sum_{j not in S_c} Q_j), P_j = (1 - M_j) u_j,
+// Q_j = M_j u_j, u_j = G_j W_j - 2 lambda W_j^2 M_j.
+__device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8], const float gw[8], uint64_t gid,
+                                         const StepScalars &sc, const NlogCtx &L, float *grow) {
+    float w[C], ms[8], mc[8];
+    const float mx = perturbed(pi_row, gid, sc, L, w);
+    const float r = rcp_approx(soft_sums<true>(w, mx, sc.c2, ms, mc));
+    float P[8], Q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        ms[j] = __fmul_rn(ms[j], r);
+        mc[j] = __fmul_rn(mc[j], r);
+        const float wj = wt[j];
+        const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j], __fmul_rn(gw[j], wj));
+        P[j] = __fmul_rn(mc[j], u);
+        Q[j] = __fmul_rn(ms[j], u);
+    }
+    const float cr = __fmul_rn(sc.kappa_over_tau, r);
+    static_for<0, C>([&](auto I) {
+        constexpr int c = decltype(I)::value;
+        constexpr uint32_t mk = cand_mask(c);
+        float kept = 0.f, pruned = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (mk & (1u << j)) kept += P[j];
+            else pruned += Q[j];
+        }
+        grow[c] = __fmul_rn(__fmul_rn(cr, w[c]), kept - pruned);
+    });
+}
+
+// Forward of one block (Eq.5-Eq.8): soft mask ms[8] and soft-masked weights x[8] (fp32),
+// regulariser partial added to acc.
+__device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], uint64_t gid, const StepScalars &sc,
+                                        const NlogCtx &L, float ms[8], float x[8], float &acc) {
+    float w[C], mc[8];
+    const float mx = perturbed(pi_row, gid, sc, L, w);
+    const float r = rcp_approx(soft_sums<false>(w, mx, sc.c2, ms, mc));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        ms[j] = __fmul_rn(ms[j], r);
+        x[j] = __fmul_rn(wt[j], ms[j]);
+        acc = __fmaf_rn(x[j], x[j], acc);
+    }
+}
+
 // AdamW over a tile as one flat, coalesced array of float4: logits and gradients from shared
 // memory, m and v from global memory (each thread first loads kUnroll vectors of each, so it
 // keeps 2*kUnroll loads in flight). Updated logits, m, v (and the gradient when gout) are
@@ -281,12 +247,12 @@ __device__ __forceinline__ void adam_tile(float *s_pi, const float *s_gr, int n,
                                           float *__restrict__ mm, float *__restrict__ vv,
                                           float *__restrict__ gout, const StepScalars &sc) {
     const int n4 = n >> 2;
-    constexpr int kUnroll = 3;
-    for (int i0 = threadIdx.x; i0 < n4; i0 += kSampThreads * kUnroll) {
+    constexpr int kUnroll = 6;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += kCtaThreads * kUnroll) {
         float4 m4[kUnroll], v4[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int i = i0 + u * kSampThreads;
+            const int i = i0 + u * kCtaThreads;
             if (i < n4) {
                 m4[u] = __ldcs(reinterpret_cast<const float4 *>(mm) + i);
                 v4[u] = __ldcs(reinterpret_cast<const float4 *>(vv) + i);
@@ -294,7 +260,7 @@ __device__ __forceinline__ void adam_tile(float *s_pi, const float *s_gr, int n,
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int i = i0 + u * kSampThreads;
+            const int i = i0 + u * kCtaThreads;
             if (i < n4) {
                 float4 p4 = reinterpret_cast<const float4 *>(s_pi)[i];
                 const float4 g4 = reinterpret_cast<const float4 *>(s_gr)[i];
@@ -325,7 +291,7 @@ __device__ __forceinline__ void adam_tile(float *s_pi, const float *s_gr, int n,
 // combines all per-CTA partials in index order and resets the ticket.
 __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned int *ticket, double *reg_out,
                                            int accumulate) {
-    __shared__ double s_w[kSampThreads / 32];
+    __shared__ double s_w[kCtaThreads / 32];
     __shared__ bool s_last;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
@@ -335,7 +301,7 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
     __syncthreads();
     if (threadIdx.x == 0) {
         double tt = 0.0;
-        for (int i = 0; i < kSampThreads / 32; ++i) tt += s_w[i];
+        for (int i = 0; i < kCtaThreads / 32; ++i) tt += s_w[i];
         partials[blockIdx.x] = tt;
         __threadfence();
         s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1);
@@ -344,7 +310,7 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
     if (!s_last) return;
     __threadfence();
     double tt = 0.0;
-    for (unsigned int i = threadIdx.x; i < gridDim.x; i += kSampThreads) tt += __ldcg(partials + i);
+    for (unsigned int i = threadIdx.x; i < gridDim.x; i += kCtaThreads) tt += __ldcg(partials + i);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tt += __shfl_xor_sync(0xFFFFFFFFu, tt, o);
     __syncthreads();
@@ -352,7 +318,7 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
     __syncthreads();
     if (threadIdx.x == 0) {
         double tot = 0.0;
-        for (int i = 0; i < kSampThreads / 32; ++i) tot += s_w[i];
+        for (int i = 0; i < kCtaThreads / 32; ++i) tot += s_w[i];
         *reg_out = accumulate ? (*reg_out + tot) : tot;
         *ticket = 0u;
     }
@@ -360,81 +326,14 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
 
 // --------------------------------------------------------------------------- kernels
 
-// W of one block: positions 4h .. 4h+3 (the forward's half) or all eight.
-template <bool kF32>
-__device__ __forceinline__ void load4(const void *base, int64_t b, int h, float w[4]) {
-    if (kF32) {
-        const float4 a = __ldcs(reinterpret_cast<const float4 *>(static_cast<const float *>(base) + b * 8 + 4 * h));
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    } else {
-        const uint2 a = __ldcs(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(base) + b * 8 + 4 * h));
-        w[0] = bf16lo(a.x); w[1] = bf16hi(a.x); w[2] = bf16lo(a.y); w[3] = bf16hi(a.y);
-    }
-}
-template <bool kF32>
-__device__ __forceinline__ void store4(void *base, int64_t b, int h, const float x[4]) {
-    if (kF32) {
-        __stcs(reinterpret_cast<float4 *>(static_cast<float *>(base) + b * 8 + 4 * h), make_float4(x[0], x[1], x[2], x[3]));
-    } else {
-        __stcs(reinterpret_cast<uint2 *>(static_cast<uint16_t *>(base) + b * 8 + 4 * h),
-               make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3])));
-    }
-}
-
-// The forward of a tile whose logits are in s_pi (both halves; two CTA barriers): X of step
-// sc (positions 4h .. 4h+3 from each half), the soft mask when requested, squares added to acc.
 template <bool kW32>
-__device__ __forceinline__ void fwd_tile(const MatDesc &d, int64_t tb0, int nb, const float *s_pi, float *xm,
-                                         float *xp, const StepScalars &sc, const NlogCtx &L, float &acc) {
-    const int h = threadIdx.x / kBlocksPerCta, blk = threadIdx.x % kBlocksPerCta;
-    const bool active = blk < nb;
-    const int64_t b = tb0 + blk;
-    float e[36], tot[kFwdParts], wt[4] = {0.f, 0.f, 0.f, 0.f};
-    const float mx = soft_phase1(active, h, blk, s_pi + blk * C, d.gid0 + b, sc, L, xm, e);
-    if (active) load4<kW32>(d.W, b, h, wt);
-    soft_phase2<kFwdParts>(active, h, blk, mx, sc.c2, xp, e, tot);
-    if (!active) return;
-    const float r = rcp_approx(tot[0]);
-    float ms[4], x[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        ms[j] = __fmul_rn(h ? tot[5 + j] : tot[1 + j], r);
-        x[j] = __fmul_rn(wt[j], ms[j]);
-        acc = __fmaf_rn(x[j], x[j], acc);
-    }
-    store4<kW32>(d.X, b, h, x);
-    if (d.soft) __stcs(reinterpret_cast<float4 *>(d.soft + b * 8 + 4 * h), make_float4(ms[0], ms[1], ms[2], ms[3]));
-}
-
-// The gradients of a tile whose logits are in s_pi into s_gr (both halves; three CTA
-// barriers: the exchange's partials overlay s_gr until both halves have read them).
-template <bool kW32, bool kG32>
-__device__ __forceinline__ void grad_tile(const MatDesc &d, int64_t tb0, int nb, const float *s_pi, float *s_gr,
-                                          float *xm, const StepScalars &sc, const NlogCtx &L) {
-    const int h = threadIdx.x / kBlocksPerCta, blk = threadIdx.x % kBlocksPerCta;
-    const bool active = blk < nb;
-    const int64_t b = tb0 + blk;
-    float e[36], tot[kParts], wt[8], gw[8];
-    const float mx = soft_phase1(active, h, blk, s_pi + blk * C, d.gid0 + b, sc, L, xm, e);
-    if (active) {  // issued here, used after the next exchange
-        load8<kW32>(d.W, b, wt);
-        load8<kG32>(d.G, b, gw);
-    }
-    soft_phase2<kParts>(active, h, blk, mx, sc.c2, s_gr, e, tot);
-    __syncthreads();  // both halves have read the partials before the gradients overwrite them
-    if (!active) return;
-    if (h) grads_half<1>(e, tot, wt, gw, sc, s_gr + blk * C);
-    else grads_half<0>(e, tot, wt, gw, sc, s_gr + blk * C);
-}
-
-template <bool kW32>
-__global__ void __launch_bounds__(kSampThreads, 3) fwd_kernel(const __grid_constant__ Group grp,
-                                                           const StepScalars sc, double *partials,
-                                                           unsigned int *ticket, double *reg_out,
-                                                           int accumulate) {
+__global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant__ Group grp,
+                                                          const StepScalars sc, double *partials,
+                                                          unsigned int *ticket, double *reg_out,
+                                                          int accumulate) {
     __shared__ __align__(16) float2 s_tab[kNlogEntries];
-    extern __shared__ __align__(16) float s_dyn[];  // logits of the tile | partials | maxima
-    float *s_pi = s_dyn, *xp = s_dyn + kTileFloats, *xm = xp + 2 * kFwdParts * kBlocksPerCta;
+    extern __shared__ __align__(16) float s_dyn[];  // [kTileFloats] logits of the tile
+    float *s_pi = s_dyn;
     load_tab(s_tab);
     const NlogCtx L{s_tab};
     float acc = 0.f;
@@ -445,17 +344,28 @@ __global__ void __launch_bounds__(kSampThreads, 3) fwd_kernel(const __grid_const
         __syncthreads();  // previous tile's readers are done (and the table is loaded)
         stage_in(s_pi, d.pi + tb0 * C, nb * C);
         __syncthreads();
-        fwd_tile<kW32>(d, tb0, nb, s_pi, xm, xp, sc, L, acc);
+        if ((int)threadIdx.x < nb) {
+            const int64_t b = tb0 + threadIdx.x;
+            float wt[8], ms[8], x[8];
+            load8<kW32>(d.W, b, wt);
+            fwd_row(s_pi + threadIdx.x * C, wt, d.gid0 + b, sc, L, ms, x, acc);
+            store8<kW32>(d.X, b, x);
+            if (d.soft) {
+                float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
+                sp[0] = make_float4(ms[0], ms[1], ms[2], ms[3]);
+                sp[1] = make_float4(ms[4], ms[5], ms[6], ms[7]);
+            }
+        }
     }
     if (reg_out) reduce_reg(acc, partials, ticket, reg_out, accumulate);
 }
 
 template <bool kW32, bool kG32>
-__global__ void __launch_bounds__(kSampThreads, 2) bwd_adam_kernel(const __grid_constant__ Group grp,
-                                                                const StepScalars sc) {
+__global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_constant__ Group grp,
+                                                               const StepScalars sc) {
     __shared__ __align__(16) float2 s_tab[kNlogEntries];
-    extern __shared__ __align__(16) float s_dyn[];  // logits | gradients (partials first) | maxima
-    float *s_pi = s_dyn, *s_gr = s_dyn + kTileFloats, *xm = s_dyn + 2 * kTileFloats;
+    extern __shared__ __align__(16) float s_dyn[];  // [2 * kTileFloats]: logits, gradients
+    float *s_pi = s_dyn, *s_gr = s_dyn + kTileFloats;
     load_tab(s_tab);
     const NlogCtx L{s_tab};
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
@@ -469,7 +379,13 @@ __global__ void __launch_bounds__(kSampThreads, 2) bwd_adam_kernel(const __grid_
         }
         stage_in(s_pi, d.pi + tb0 * C, nb * C);
         __syncthreads();
-        grad_tile<kW32, kG32>(d, tb0, nb, s_pi, s_gr, xm, sc, L);
+        if ((int)threadIdx.x < nb) {
+            const int64_t b = tb0 + threadIdx.x;
+            float wt[8], gw[8];
+            load8<kW32>(d.W, b, wt);
+            load8<kG32>(d.G, b, gw);
+            grad_row(s_pi + threadIdx.x * C, wt, gw, d.gid0 + b, sc, L, s_gr + threadIdx.x * C);
+        }
         __syncthreads();
         adam_tile<false>(s_pi, s_gr, nb * C, d.pi + tb0 * C, d.m + tb0 * C, d.v + tb0 * C,
                          d.grad ? d.grad + tb0 * C : nullptr, sc);
@@ -477,19 +393,18 @@ __global__ void __launch_bounds__(kSampThreads, 2) bwd_adam_kernel(const __grid_
 }
 
 // Backward + AdamW of step t fused with the forward of step t+1 (mllm_sample_bwd_adam_fwd):
-// per tile, the gradients of every block (noise of step t) into one buffer, the flat AdamW
+// per tile, the gradient of every block (noise of step t) into one buffer, the flat AdamW
 // pass (updated logits kept in shared memory), then the forward of step t+1 from the updated
 // logits. The tile's logits are read from HBM once. Two tile buffers alternate: while a tile's
 // forward runs, the next tile's logits land in the buffer its gradients used, and its m, v
 // are fetched into L2 at the start of the tile, ahead of the AdamW pass.
 template <bool kW32, bool kG32>
-__global__ void __launch_bounds__(kSampThreads, 2) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
-                                                                    const StepScalars sb, const StepScalars sf,
-                                                                    double *partials, unsigned int *ticket,
-                                                                    double *reg_out, int accumulate) {
+__global__ void __launch_bounds__(kCtaThreads) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
+                                                                   const StepScalars sb, const StepScalars sf,
+                                                                   double *partials, unsigned int *ticket,
+                                                                   double *reg_out, int accumulate) {
     __shared__ __align__(16) float2 s_tab[kNlogEntries];
-    extern __shared__ __align__(16) float s_dyn[];  // two tile buffers | forward partials | maxima
-    float *xp = s_dyn + 2 * kTileFloats, *xm = xp + 2 * kFwdParts * kBlocksPerCta;
+    extern __shared__ __align__(16) float s_dyn[];  // [2 * kTileFloats]: two tile buffers
     load_tab(s_tab);
     const NlogCtx L{s_tab};
     float acc = 0.f;
@@ -511,13 +426,30 @@ __global__ void __launch_bounds__(kSampThreads, 2) bwd_adam_fwd_kernel(const __g
             prefetch_l2(d.m + tb0 * C, nb * C * 4);
             prefetch_l2(d.v + tb0 * C, nb * C * 4);
         }
-        grad_tile<kW32, kG32>(d, tb0, nb, s_pi, s_gr, xm, sb, L);
+        const bool mine = (int)threadIdx.x < nb;
+        const int64_t b = tb0 + threadIdx.x;
+        float wt[8];
+        if (mine) {
+            float gw[8];
+            load8<kW32>(d.W, b, wt);
+            load8<kG32>(d.G, b, gw);
+            grad_row(s_pi + threadIdx.x * C, wt, gw, d.gid0 + b, sb, L, s_gr + threadIdx.x * C);
+        }
         __syncthreads();
         adam_tile<true>(s_pi, s_gr, nb * C, d.pi + tb0 * C, d.m + tb0 * C, d.v + tb0 * C,
                         d.grad ? d.grad + tb0 * C : nullptr, sb);
         __syncthreads();  // updated logits in s_pi; the gradient buffer is free
         if (t + gridDim.x < grp.total_work) stage(s_gr, t + gridDim.x);
-        fwd_tile<kW32>(d, tb0, nb, s_pi, xm, xp, sf, L, acc);
+        if (mine) {
+            float ms[8], x[8];
+            fwd_row(s_pi + threadIdx.x * C, wt, d.gid0 + b, sf, L, ms, x, acc);
+            store8<kW32>(d.X, b, x);
+            if (d.soft) {
+                float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
+                sp[0] = make_float4(ms[0], ms[1], ms[2], ms[3]);
+                sp[1] = make_float4(ms[4], ms[5], ms[6], ms[7]);
+            }
+        }
         cur ^= 1;
     }
     if (reg_out) reduce_reg(acc, partials, ticket, reg_out, accumulate);

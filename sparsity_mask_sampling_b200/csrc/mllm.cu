@@ -825,9 +825,9 @@ mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
             else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         } else {
             const void *fn = w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>;
-            const int64_t grid = grid_for(fn, k48::kSampThreads, k48::kFwdDynSmem, g.total_work, kMaxReduceCtas);
-            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kSampThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
-            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kSampThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            const int64_t grid = grid_for(fn, k48::kCtaThreads, k48::kFwdDynSmem, g.total_work, kMaxReduceCtas);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         }
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -849,7 +849,7 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
     const bool is24 = nm.m == 4;
     const void *fn = is24 ? (w32 ? (const void *)k24::fwd_kernel<true> : (const void *)k24::fwd_kernel<false>)
                           : (w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>);
-    const int threads = is24 ? kThreads : k48::kSampThreads;
+    const int threads = is24 ? kThreads : k48::kCtaThreads;
     const int dyn_smem = is24 ? 0 : k48::kFwdDynSmem;
     const std::vector<Group> groups = make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48);
     // every launch's scratch need (one partial per CTA) is checked before anything runs
@@ -873,8 +873,8 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
             if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
             else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         } else {
-            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kSampThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
-            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kSampThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         }
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -908,10 +908,10 @@ mllm_status mllm_sample_bwd_adam(const mllm_matrix *mats, int32_t n_mats, mllm_n
             else if (g32) MLLM_LAUNCH_BWD(k24, kThreads, 0, false, true);
             else MLLM_LAUNCH_BWD(k24, kThreads, 0, false, false);
         } else {
-            if (w32 && g32) MLLM_LAUNCH_BWD(k48, k48::kSampThreads, k48::kBwdDynSmem, true, true);
-            else if (w32) MLLM_LAUNCH_BWD(k48, k48::kSampThreads, k48::kBwdDynSmem, true, false);
-            else if (g32) MLLM_LAUNCH_BWD(k48, k48::kSampThreads, k48::kBwdDynSmem, false, true);
-            else MLLM_LAUNCH_BWD(k48, k48::kSampThreads, k48::kBwdDynSmem, false, false);
+            if (w32 && g32) MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, true);
+            else if (w32) MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, false);
+            else if (g32) MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, true);
+            else MLLM_LAUNCH_BWD(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, false);
         }
 #undef MLLM_LAUNCH_BWD
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
@@ -955,10 +955,10 @@ mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, ml
             else if (g32) MLLM_LAUNCH_FUSED(k24, kThreads, 0, false, true);
             else MLLM_LAUNCH_FUSED(k24, kThreads, 0, false, false);
         } else {
-            if (w32 && g32) MLLM_LAUNCH_FUSED(k48, k48::kSampThreads, k48::kFusedDynSmem, true, true);
-            else if (w32) MLLM_LAUNCH_FUSED(k48, k48::kSampThreads, k48::kFusedDynSmem, true, false);
-            else if (g32) MLLM_LAUNCH_FUSED(k48, k48::kSampThreads, k48::kFusedDynSmem, false, true);
-            else MLLM_LAUNCH_FUSED(k48, k48::kSampThreads, k48::kFusedDynSmem, false, false);
+            if (w32 && g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, true);
+            else if (w32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, false);
+            else if (g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, true);
+            else MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, false);
         }
 #undef MLLM_LAUNCH_FUSED
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
