@@ -384,31 +384,41 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
 // ------------------------------------------------------------------ 2:4 prefill (more than 64 tokens)
 //
 // The same sparse MMA (M = 128 rows, K = 32 per instruction, metadata in tensor memory) with
-// N = 128 tokens. A unit of work is (operand, tile of 128 rows, chunk of 128 tokens) over all
-// the operand's columns; no unit is split between CTAs, so nothing is reduced across CTAs.
-// CTA c takes units c, c + G, c + 2G, ... of a sequence ordered so that the G units in flight
-// at any time share few weight strips and all token chunks: per operand, groups of R row tiles
-// (R = ceil(G / token chunks)), within a group token chunk by token chunk, within a chunk the
-// group's row tiles. The strips and chunks of the activations in flight then fit in L2, so a
-// strip is read from HBM about once per group instead of once per token chunk. The host
-// orders the operands by decreasing columns (the longest units first). The copy warp
-// addresses the token chunk through the activations' tensor map (rows past the call's tokens
-// are zero-filled) and the epilogue stores only rows of y inside it. Roles, stages, barriers,
-// bounded waits and wind-down as in sparse_linear_umma_kernel.
+// N = 128 tokens. A unit of work is (operand, pair of 128-row tiles, chunk of 128 tokens) over
+// all the operand's columns: per 128-column stage the copy warp lands both tiles' compressed
+// values and metadata and one 128-token box of the activations, and the MMA warp issues four
+// MMAs per tile into two accumulators (TMEM columns 0-127 and 128-255) with the same
+// activation operand, so every staged activation byte feeds two tiles. No unit is split
+// between CTAs, so nothing is reduced across CTAs. CTA c takes units c, c + G, c + 2G, ... of a
+// sequence ordered so that the G units in flight at any time share few weight strips and all
+// token chunks: per operand, groups of R row-tile pairs (R = ceil(G / token chunks)), within
+// a group token chunk by token chunk, within a chunk the group's pairs. The strips and chunks
+// in flight then fit in L2, so a strip is read from HBM about once per group instead of once
+// per token chunk. The host orders the operands by decreasing columns (the longest units
+// first). Tokens past the call are zero-filled by the activations' tensor map, rows past the
+// matrix by the weights' (their metadata words read zero and are replaced by a valid code),
+// and the epilogue stores only rows and tokens inside the call. Roles, barriers, bounded
+// waits and wind-down as in sparse_linear_umma_kernel.
 
 constexpr int kPfTok = 128;                   // MMA N: tokens per unit
 constexpr int kPfMaxCtas = 160;
-constexpr unsigned kPfTmemCols = 256;         // accumulator 0..127, metadata from column 128
-constexpr unsigned kPfMetaCol = 128;
+constexpr unsigned kPfTmemCols = 512;         // accumulators 0..255, metadata from column 256
+constexpr unsigned kPfMetaCol = 256;
+constexpr int kPfTileBytes = kUmRows * 128;   // one tile's compressed values in a stage (16 KB)
+constexpr int kPfXOff = 2 * kPfTileBytes;     // the activations' two 128 x 64 boxes
+constexpr int kPfMetaOff = kPfXOff + 2 * kPfTok * 128;  // both tiles' metadata (2 x 2 KB)
+constexpr int kPfStageTx = kPfMetaOff + 2 * kUmRows * 16;
+constexpr int kPfStage = (kPfStageTx + 1023) / 1024 * 1024;
+constexpr int kPfSmem = kUmStages * kPfStage + 1024;
 
 struct PfOp {
     const void *meta;
     float *y;
     int64_t rows, cols;
     int64_t nch;         // 128-column chunks
-    int64_t ntiles;      // row tiles
+    int64_t npairs;      // pairs of row tiles
     int64_t nt;          // token chunks
-    int64_t rgroup;      // row tiles per group of the unit order
+    int64_t rgroup;      // row-tile pairs per group of the unit order
     int64_t unit_begin;  // first unit of this operand in the launch
 };
 
@@ -422,7 +432,7 @@ struct PfGroup {
 
 struct PfCur {
     int op;
-    int64_t tile, tc;
+    int64_t pair, tc;
 };
 
 __device__ __forceinline__ PfCur pf_decode(const PfGroup &g, int64_t u) {
@@ -431,24 +441,27 @@ __device__ __forceinline__ PfCur pf_decode(const PfGroup &g, int64_t u) {
     const PfOp &d = g.d[i];
     const int64_t idx = u - d.unit_begin, per = d.rgroup * d.nt;
     const int64_t grp = idx / per, rem = idx % per;
-    const int64_t rg = d.ntiles - grp * d.rgroup < d.rgroup ? d.ntiles - grp * d.rgroup : d.rgroup;
+    const int64_t rg = d.npairs - grp * d.rgroup < d.rgroup ? d.npairs - grp * d.rgroup : d.rgroup;
     return PfCur{i, grp * d.rgroup + rem % rg, rem / rg};
 }
 
 __device__ __forceinline__ void pf_issue(const PfGroup &g, const PfCur &c, int64_t j, unsigned stage, unsigned bar) {
     const TmMaps &mp = g.maps[c.op];
-    const int row0 = (int)(c.tile * kUmRows), tok0 = (int)(c.tc * kPfTok);
-    mbar_arrive_tx(bar, (unsigned)um_stage_tx<kPfTok>());
+    const int row0 = (int)(c.pair * 2 * kUmRows), tok0 = (int)(c.tc * kPfTok);
+    mbar_arrive_tx(bar, (unsigned)kPfStageTx);
     tma_load_2d(stage, &mp.vals, (int)(64 * j), row0, bar);
-    tma_load_2d(stage + kUmRows * 128, &mp.x, (int)(128 * j), tok0, bar);
-    tma_load_2d(stage + kUmRows * 128 + um_xbox_bytes<kPfTok>(), &mp.x, (int)(128 * j + 64), tok0, bar);
-    tma_load_2d(stage + kUmRows * 128 + 2 * um_xbox_bytes<kPfTok>(), &mp.meta, (int)(4 * j), row0, bar);
+    tma_load_2d(stage + kPfTileBytes, &mp.vals, (int)(64 * j), row0 + kUmRows, bar);
+    tma_load_2d(stage + kPfXOff, &mp.x, (int)(128 * j), tok0, bar);
+    tma_load_2d(stage + kPfXOff + kPfTok * 128, &mp.x, (int)(128 * j + 64), tok0, bar);
+    tma_load_2d(stage + kPfMetaOff, &mp.meta, (int)(4 * j), row0, bar);
+    tma_load_2d(stage + kPfMetaOff + kUmRows * 16, &mp.meta, (int)(4 * j), row0 + kUmRows, bar);
 }
 
 __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(const __grid_constant__ PfGroup pg,
                                                                             unsigned int *__restrict__ err) {
-    static_assert(um_smem_bytes<kPfTok>() + 1024 <= 232448, "fits one SM");
-    constexpr int kD = kUmStages, kStage = um_stage_bytes<kPfTok>();
+    static_assert(kPfSmem + 1024 <= 232448, "fits one SM");
+    static_assert(kPfMetaCol + 2 * 8 * kUmStages <= kPfTmemCols, "metadata columns fit");
+    constexpr int kD = kUmStages;
     constexpr uint32_t kIdesc = um_idesc<kPfTok>();
     extern __shared__ unsigned char s_dyn_pf[];
     __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_meta[kD], s_acc;
@@ -505,7 +518,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
                 }
                 if (lane == 0) {
                     fence_proxy_async();
-                    pf_issue(pg, c, j, ring_s + s * kStage, full0 + 8 * s);
+                    pf_issue(pg, c, j, ring_s + s * kPfStage, full0 + 8 * s);
                 }
                 ++issued;
             }
@@ -533,13 +546,17 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
                 }
                 if (lane == 0) {
                     tc_fence_after();
-                    const unsigned st = ring_s + s * kStage;
-                    const uint64_t a0 = um_desc(st), b0 = um_desc(st + kUmRows * 128),
-                                   b1 = um_desc(st + kUmRows * 128 + um_xbox_bytes<kPfTok>());
+                    const unsigned st = ring_s + s * kPfStage;
+                    const uint64_t b0 = um_desc(st + kPfXOff), b1 = um_desc(st + kPfXOff + kPfTok * 128);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        umma_sp(tbase, a0 + (uint64_t)(2 * q), ((q >> 1) ? b1 : b0) + (uint64_t)(4 * (q & 1)),
-                                tbase + kPfMetaCol + 8 * s + 2 * q, kIdesc, (j == 0 && q == 0) ? 0u : 1u);
+                    for (int t = 0; t < 2; ++t) {
+                        const uint64_t a0 = um_desc(st + t * kPfTileBytes);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            umma_sp(tbase + t * kPfTok, a0 + (uint64_t)(2 * q),
+                                    ((q >> 1) ? b1 : b0) + (uint64_t)(4 * (q & 1)),
+                                    tbase + kPfMetaCol + 8 * (kD * t + s) + 2 * q, kIdesc, (j == 0 && q == 0) ? 0u : 1u);
+                    }
                     umma_commit(empty0 + 8 * s);
                     if (j == nch - 1) umma_commit(accb);
                 }
@@ -555,7 +572,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         // ------------------------------------------------------------ metadata / epilogue warps
         const unsigned tlane = tbase + ((unsigned)(32 * warp) << 16);
         const int h = (lane >> 3) & 1;
-        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of the tile
+        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of a tile
         const uint32_t esel = h ? 0x7632u : 0x5410u;
         unsigned acc_phase = 0u;
         bool failed = false;
@@ -568,14 +585,17 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
                 if (!failed) {
                     if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
                         tc_fence_after();
-                        const unsigned char *meta = ring + s * kStage + kUmRows * 128 + 2 * um_xbox_bytes<kPfTok>();
-                        const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
-                        const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
-                        uint32_t e[4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            e[q] = __byte_perm(a4[q] ? a4[q] : 0x44444444u, b4[q] ? b4[q] : 0x44444444u, esel);
-                        tmem_st_meta(tlane + kPfMetaCol + 8 * s, e[0], e[1], e[2], e[3]);
+                        for (int t = 0; t < 2; ++t) {
+                            const unsigned char *meta = ring + s * kPfStage + kPfMetaOff + t * kUmRows * 16;
+                            const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
+                            const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
+                            uint32_t e[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                e[q] = __byte_perm(a4[q] ? a4[q] : 0x44444444u, b4[q] ? b4[q] : 0x44444444u, esel);
+                            tmem_st_meta(tlane + kPfMetaCol + 8 * (kD * t + s), e[0], e[1], e[2], e[3]);
+                        }
                         tc_fence_before();
                         mbar_arrive(meta0 + 8 * s);
                     } else {
@@ -595,16 +615,19 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
                 break;
             }
             tc_fence_after();
-            const int64_t r = c.tile * kUmRows + 32 * warp + lane;
             const int tok0 = (int)(c.tc * kPfTok);
 #pragma unroll 1
-            for (int k = 0; k < kPfTok; k += 16) {
-                float v[16];
-                tmem_ld16(tlane + k, v);
-                if (r < d.rows) {
+            for (int t = 0; t < 2; ++t) {
+                const int64_t r = (c.pair * 2 + t) * kUmRows + 32 * warp + lane;
+#pragma unroll 1
+                for (int k = 0; k < kPfTok; k += 16) {
+                    float v[16];
+                    tmem_ld16(tlane + t * kPfTok + k, v);
+                    if (r < d.rows) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (tok0 + k + i < pg.tokens) d.y[(int64_t)(tok0 + k + i) * d.rows + r] = v[i];
+                        for (int i = 0; i < 16; ++i)
+                            if (tok0 + k + i < pg.tokens) d.y[(int64_t)(tok0 + k + i) * d.rows + r] = v[i];
+                    }
                 }
             }
             tc_fence_before();  // these reads precede the next unit's first MMA (after its arrivals)

@@ -422,8 +422,8 @@ mllm_status noalloc_scratch(void **out) {
 }
 
 // 2:4 operands with cols % 128 == 0 above 64 tokens on the prefill kernel, 16 operands per
-// launch (longest rows first): units (operand, 128-row tile, 128-token chunk) dealt round-robin
-// over the CTAs in the kernel's group order. False if a tensor map cannot be encoded (nothing
+// launch (longest rows first): units (operand, pair of 128-row tiles, 128-token chunk) dealt
+// round-robin over the CTAs in the kernel's group order. False if a tensor map cannot be encoded (nothing
 // is launched then).
 bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32_t tokens, unsigned int *err,
                            cudaStream_t st, mllm_status *status) {
@@ -431,7 +431,7 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
     std::stable_sort(ops.begin(), ops.end(),
                      [](const mllm_sparse_operand &a, const mllm_sparse_operand &b) { return a.cols > b.cols; });
     auto fn = spl::sparse_linear_prefill_kernel;
-    constexpr int smem = spl::um_smem_bytes<spl::kPfTok>();
+    constexpr int smem = spl::kPfSmem;
     int dev = 0;
     cudaGetDevice(&dev);
     resident_ctas(dev, (const void *)fn, spl::kUmThreads, smem);  // sets the dynamic shared-memory limit
@@ -451,11 +451,11 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
             d.rows = o.rows;
             d.cols = o.cols;
             d.nch = o.cols / spl::kTmChunk;
-            d.ntiles = (o.rows + spl::kUmRows - 1) / spl::kUmRows;
+            d.npairs = (o.rows + 2 * spl::kUmRows - 1) / (2 * spl::kUmRows);
             d.nt = nt;
             d.rgroup = std::max<int64_t>(1, (G0 + nt - 1) / nt);
             d.unit_begin = units;
-            units += d.ntiles * nt;
+            units += d.npairs * nt;
             const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
             if (!(encode_2d(&pg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
                             spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
