@@ -397,10 +397,14 @@ __global__ void __launch_bounds__(kUmThreads, kUmCtasPerSm) sparse_linear_umma_k
 // per token chunk. The host orders the operands by decreasing columns (the longest units
 // first). Tokens past the call are zero-filled by the activations' tensor map, rows past the
 // matrix by the weights' (their metadata words read zero and are replaced by a valid code),
-// and the epilogue stores only rows and tokens inside the call. Roles, barriers, bounded
-// waits and wind-down as in sparse_linear_umma_kernel.
+// and the epilogue stores only rows and tokens inside the call. Warps 0-3 turn the first
+// tile's metadata into TMEM, warps 4-7 the second tile's; warps 0-15 store the accumulators
+// (4 per tile and half of the tokens; the MMA pipe idles while they drain, so more warps
+// shorten the gap); warp 16 copies, warp 17 issues the MMAs. Barriers, bounded waits and
+// wind-down as in sparse_linear_umma_kernel.
 
 constexpr int kPfTok = 128;                   // MMA N: tokens per unit
+constexpr int kPfThreads = 576;               // 16 metadata/epilogue warps (8 per tile), the copy warp, the MMA warp
 constexpr int kPfMaxCtas = 160;
 constexpr unsigned kPfTmemCols = 512;         // accumulators 0..255, metadata from column 256
 constexpr unsigned kPfMetaCol = 256;
@@ -457,7 +461,7 @@ __device__ __forceinline__ void pf_issue(const PfGroup &g, const PfCur &c, int64
     tma_load_2d(stage + kPfMetaOff + kUmRows * 16, &mp.meta, (int)(4 * j), row0 + kUmRows, bar);
 }
 
-__global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(const __grid_constant__ PfGroup pg,
+__global__ void __launch_bounds__(kPfThreads, 1) sparse_linear_prefill_kernel(const __grid_constant__ PfGroup pg,
                                                                             unsigned int *__restrict__ err) {
     static_assert(kPfSmem + 1024 <= 232448, "fits one SM");
     static_assert(kPfMetaCol + 2 * 8 * kUmStages <= kPfTmemCols, "metadata columns fit");
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         for (int s = 0; s < kD; ++s) {
             mbar_init(full0 + 8 * s, 1u);
             mbar_init(empty0 + 8 * s, 1u);
-            mbar_init(meta0 + 8 * s, 128u);
+            mbar_init(meta0 + 8 * s, 256u);  // every metadata thread of both tiles arrives once per stage
         }
         mbar_init(accb, 1u);
         s_abort = 0;
@@ -499,7 +503,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
     tc_fence_after();
     const unsigned tbase = s_tmem;
 
-    if (warp == 4) {
+    if (warp == 16) {
         // ------------------------------------------------------------ copy warp
         int f = 0, issued = 0;
         bool stop = false;
@@ -527,7 +531,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
             const int last = s + ((issued - 1 - s) / kD) * kD;
             tm_wait(full0 + 8 * s, (last / kD) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == 17) {
         // ------------------------------------------------------------ MMA warp
         int f = 0, commits = 0;
         bool stop = false;
@@ -570,9 +574,13 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         }
     } else {
         // ------------------------------------------------------------ metadata / epilogue warps
-        const unsigned tlane = tbase + ((unsigned)(32 * warp) << 16);
+        // warps 0-3 and 8-11 take row tile 0 of the pair, warps 4-7 and 12-15 row tile 1 (TMEM
+        // lane quarter warp % 4); warps 0-7 also turn the metadata into TMEM. Each warp stores
+        // half of its lanes' 128 accumulator columns (warps 0-7 the first half).
+        const int t = (warp >> 2) & 1, wq = warp & 3, half = warp >> 3;
+        const unsigned tlane = tbase + ((unsigned)(32 * wq) << 16);
         const int h = (lane >> 3) & 1;
-        const int ra = 32 * warp + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of a tile
+        const int ra = 32 * wq + 16 * (lane >> 4) + (lane & 7);  // rows ra and ra + 8 of the tile
         const uint32_t esel = h ? 0x7632u : 0x5410u;
         unsigned acc_phase = 0u;
         bool failed = false;
@@ -580,22 +588,19 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
         for (int64_t u = u0; u < u1; u += G) {
             const PfCur c = pf_decode(pg, u);
             const PfOp &d = pg.d[c.op];
-            for (int64_t j = 0; j < d.nch; ++j, ++f) {
+            for (int64_t j = 0; j < d.nch && half == 0; ++j, ++f) {
                 const int s = f % kD;
                 if (!failed) {
                     if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
                         tc_fence_after();
+                        const unsigned char *meta = ring + s * kPfStage + kPfMetaOff + t * kUmRows * 16;
+                        const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
+                        const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
+                        uint32_t e[4];
 #pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            const unsigned char *meta = ring + s * kPfStage + kPfMetaOff + t * kUmRows * 16;
-                            const uint4 wa = lds128(meta + ra * 16), wb = lds128(meta + (ra + 8) * 16);
-                            const uint32_t a4[4] = {wa.x, wa.y, wa.z, wa.w}, b4[4] = {wb.x, wb.y, wb.z, wb.w};
-                            uint32_t e[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                e[q] = __byte_perm(a4[q] ? a4[q] : 0x44444444u, b4[q] ? b4[q] : 0x44444444u, esel);
-                            tmem_st_meta(tlane + kPfMetaCol + 8 * (kD * t + s), e[0], e[1], e[2], e[3]);
-                        }
+                        for (int q = 0; q < 4; ++q)
+                            e[q] = __byte_perm(a4[q] ? a4[q] : 0x44444444u, b4[q] ? b4[q] : 0x44444444u, esel);
+                        tmem_st_meta(tlane + kPfMetaCol + 8 * (kD * t + s), e[0], e[1], e[2], e[3]);
                         tc_fence_before();
                         mbar_arrive(meta0 + 8 * s);
                     } else {
@@ -610,27 +615,25 @@ __global__ void __launch_bounds__(kUmThreads, 1) sparse_linear_prefill_kernel(co
             // ---------------------------------------------------- epilogue of the unit
             const bool acc_ok = !failed && um_wait(accb, acc_phase, &s_abort);
             acc_phase ^= 1u;
-            if (um_bar_or<128>(!acc_ok)) {
+            if (um_bar_or<512>(!acc_ok)) {
                 failed = true;
                 break;
             }
             tc_fence_after();
             const int tok0 = (int)(c.tc * kPfTok);
+            const int64_t r = (c.pair * 2 + t) * kUmRows + 32 * wq + lane;
 #pragma unroll 1
-            for (int t = 0; t < 2; ++t) {
-                const int64_t r = (c.pair * 2 + t) * kUmRows + 32 * warp + lane;
-#pragma unroll 1
-                for (int k = 0; k < kPfTok; k += 16) {
-                    float v[16];
-                    tmem_ld16(tlane + t * kPfTok + k, v);
-                    if (r < d.rows) {
+            for (int k = half * (kPfTok / 2); k < (half + 1) * (kPfTok / 2); k += 16) {
+                float v[16];
+                tmem_ld16(tlane + t * kPfTok + k, v);
+                if (r < d.rows) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (tok0 + k + i < pg.tokens) d.y[(int64_t)(tok0 + k + i) * d.rows + r] = v[i];
-                    }
+                    for (int i = 0; i < 16; ++i)
+                        if (tok0 + k + i < pg.tokens) d.y[(int64_t)(tok0 + k + i) * d.rows + r] = v[i];
                 }
             }
-            tc_fence_before();  // these reads precede the next unit's first MMA (after its arrivals)
+            tc_fence_before();
+            um_bar<512>();  // every read of the accumulators precedes the next unit's first arrival
         }
         if (failed && threadIdx.x == 0 && !s_abort) {
             atomicOr(err, 1u);

@@ -434,7 +434,7 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
     constexpr int smem = spl::kPfSmem;
     int dev = 0;
     cudaGetDevice(&dev);
-    resident_ctas(dev, (const void *)fn, spl::kUmThreads, smem);  // sets the dynamic shared-memory limit
+    resident_ctas(dev, (const void *)fn, spl::kPfThreads, smem);  // sets the dynamic shared-memory limit
     for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
         const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
         static thread_local spl::PfGroup pg;
@@ -468,7 +468,7 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
         pg.n = (int32_t)n;
         pg.total_units = units;
         const int64_t G = std::min<int64_t>(G0, units);
-        fn<<<(unsigned)G, spl::kUmThreads, smem, st>>>(pg, err);
+        fn<<<(unsigned)G, spl::kPfThreads, smem, st>>>(pg, err);
         if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
     }
     *status = MLLM_OK;
