@@ -125,6 +125,13 @@ __device__ __forceinline__ int find_mat(const Group &g, int64_t t) {
     return i;
 }
 
+// The same searching forward from matrix i, the owner of a smaller unit: a CTA's grid-stride
+// walk visits its units in increasing order, so the search resumes where the last one ended.
+__device__ __forceinline__ int next_mat(const Group &g, int i, int64_t t) {
+    while (i + 1 < g.n && t >= g.d[i + 1].work_begin) ++i;
+    return i;
+}
+
 // ---------------------------------------------------------------------------- Philox
 
 // One Philox round: the two 32 x 32 -> 64-bit products (one wide multiply each), then the
@@ -190,13 +197,13 @@ __device__ __forceinline__ float uniform_from_field(uint32_t k) {
 
 // ---------------------------------------------------------------------------- nlog
 
-// nlog(x) for x in [2^-22, 16). kClamp bounds the table index (one instruction); it is
-// applied to the second logarithm, whose argument comes from arithmetic, not from bits.
-template <bool kClamp>
+// nlog(x) for x in [2^-22, 16). Both logarithms of the noise stay in that domain: the first
+// takes eps in [2^-22, 1), and its result t = -nlog(eps), the second's argument, lies in
+// [2^-22 + 2^-45, 15.25] for every one of the 2^21 fields (an exhaustive property of the
+// definition), so the table index needs no clamp.
 __device__ __forceinline__ float nlog(float x, const float2 *__restrict__ tab) {
     const uint32_t ib2 = __float_as_uint(x) + 0x408000u;
-    uint32_t idx = (ib2 >> 16) - kNlogIndexBias;
-    if (kClamp) idx = min(idx, (uint32_t)(kNlogEntries - 1));
+    const uint32_t idx = (ib2 >> 16) - kNlogIndexBias;
     const float2 cT = tab[idx];
     const float r = __fmaf_rn(x, cT.x, -1.0f);  // = fma(x 2^-e, c_j, -1)
     const float q = __fmaf_rn(r, kOneThird, -0.5f);
@@ -212,15 +219,15 @@ struct NlogCtx {
 // g = -log(-log eps) for field k (the negations are exact).
 __device__ __forceinline__ float gumbel(uint32_t k, const NlogCtx &L) {
     const float eps = uniform_from_field(k);
-    const float t = -nlog<false>(eps, L.tab);
-    return -nlog<true>(t, L.tab);
+    const float t = -nlog(eps, L.tab);
+    return -nlog(t, L.tab);
 }
 
 // The same from the bits of 1 + eps (fields21_unit): eps = that - 1, exact.
 __device__ __forceinline__ float gumbel_unit(uint32_t unit_bits, const NlogCtx &L) {
     const float eps = __fadd_rn(__uint_as_float(unit_bits), -1.0f);
-    const float t = -nlog<false>(eps, L.tab);
-    return -nlog<true>(t, L.tab);
+    const float t = -nlog(eps, L.tab);
+    return -nlog(t, L.tab);
 }
 
 // Copy the table into shared memory (all threads; __syncthreads() before use).

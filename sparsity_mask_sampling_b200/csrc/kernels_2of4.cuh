@@ -193,8 +193,10 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const __grid_constant__ G
     __syncthreads();
     const NlogCtx L{s_tab};
     float acc = 0.f;
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
@@ -233,8 +235,10 @@ __global__ void __launch_bounds__(kThreads) bwd_adam_kernel(const __grid_constan
     load_tab(s_tab);
     __syncthreads();
     const NlogCtx L{s_tab};
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
@@ -297,8 +301,10 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_adam_fwd_kernel(const __grid_
     __syncthreads();
     const NlogCtx L{s_tab};
     float acc = 0.f;
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
@@ -401,8 +407,10 @@ __device__ __forceinline__ uint32_t cand_mask(int i) {
 template <bool kW32, bool kFromIdx>
 __global__ void __launch_bounds__(kThreads) prior_kernel(const __grid_constant__ Group grp,
                                                          float alpha, float init_std, uint64_t seed) {
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
@@ -473,8 +481,10 @@ __device__ __forceinline__ int argmax6(const float *p) {
 // Hard pack: one thread per metadata word (8 blocks of one row).
 template <bool kW32>
 __global__ void __launch_bounds__(kThreads) pack_kernel(const __grid_constant__ Group grp) {
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t bpr = d.cols / 4, words = (bpr + 7) / 8;
         const int64_t widx = (t - d.work_begin) * kThreads + threadIdx.x;
         if (widx >= d.rows * words) continue;
@@ -520,8 +530,10 @@ __device__ __forceinline__ uint32_t half_of(const uint4 &a, int idx) {  // bf16 
 template <bool kW32>
 __global__ void __launch_bounds__(kThreads) pack_pairs_kernel(const __grid_constant__ Group grp) {
     const int lane = threadIdx.x & 31;
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         const bool valid = b0 < d.nblocks;  // nblocks is a multiple of 8 on this path
         uint32_t byte = 0;

@@ -337,8 +337,10 @@ __global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant_
     load_tab(s_tab);
     const NlogCtx L{s_tab};
     float acc = 0.f;
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
         __syncthreads();  // previous tile's readers are done (and the table is loaded)
@@ -368,8 +370,10 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
     float *s_pi = s_dyn, *s_gr = s_dyn + kTileFloats;
     load_tab(s_tab);
     const NlogCtx L{s_tab};
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
         __syncthreads();
@@ -415,8 +419,10 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_fwd_kernel(const __grid_
         stage_in_async(dst, d.pi + tb0 * C, (int)imin64(kBlocksPerCta, d.nblocks - tb0) * C);
     };
     if ((int64_t)blockIdx.x < grp.total_work) stage(s_dyn, blockIdx.x);
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
         float *s_pi = s_dyn + cur * kTileFloats, *s_gr = s_dyn + (cur ^ 1) * kTileFloats;
@@ -460,8 +466,10 @@ template <bool kW32, bool kFromIdx>
 __global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constant__ Group grp,
                                                             float alpha, float init_std, uint64_t seed) {
     __shared__ __align__(16) float s_pi[kTileFloats];
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
         __syncthreads();
@@ -545,8 +553,10 @@ __global__ void __launch_bounds__(kCtaThreads) prior_kernel(const __grid_constan
 template <bool kW32>
 __global__ void __launch_bounds__(kCtaThreads) pack_kernel(const __grid_constant__ Group grp) {
     __shared__ __align__(16) float s_pi[kTileFloats];
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
         __syncthreads();

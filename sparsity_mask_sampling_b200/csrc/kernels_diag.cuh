@@ -81,8 +81,10 @@ template <bool kW32>
 __global__ void __launch_bounds__(kThreads) stats24_kernel(const __grid_constant__ Group grp, float kappa,
                                                            double *partials, unsigned int *ticket, double *out) {
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
@@ -117,8 +119,10 @@ template <bool kW32>
 __global__ void __launch_bounds__(kThreads) stats48_kernel(const __grid_constant__ Group grp, float kappa,
                                                            double *partials, unsigned int *ticket, double *out) {
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
+        mi = next_mat(grp, mi, t);
+        const MatDesc &d = grp.d[mi];
         const int64_t b = (t - d.work_begin) * kThreads + threadIdx.x;
         if (b >= d.nblocks) continue;
         float w[8];
