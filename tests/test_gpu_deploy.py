@@ -362,8 +362,9 @@ def test_side_streams_and_concurrent_host_threads(orc, tokens):
 @pytest.mark.parametrize("tokens", [65, 128, 200, 512])
 def test_prefill_sized_calls(orc, ws, nm, tokens):
     """More than 64 tokens: 2:4 operands whose columns are whole 128-column stages run on the
-    prefill kernel (units of 128 rows x 128 tokens), the others in groups of 16 tokens; 4:8 in
-    groups of 64 tokens. Ragged rows and token chunks, several operands in one call."""
+    prefill kernel (units of two 128-row tiles x 128 tokens), the others in groups of 16
+    tokens; 4:8 in groups of 64 tokens. Ragged rows and token chunks, several operands in one
+    call."""
     shapes = [(300, 512), (128, 1024), (37, 1040), (200, 128)]
     ops = [Operand(orc, nm, r, c, tokens, seed=900 + 10 * i + tokens) for i, (r, c) in enumerate(shapes)]
     mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
@@ -383,6 +384,8 @@ def test_prefill_llama_layer_sampled_rows(orc, ws, tokens):
     mllm_sparse_linear([o.op() for o in ops], (2, 4), tokens, ws)
     torch.cuda.synchronize()
     for o in ops:
-        rows = np.unique(np.concatenate([[0, 127, 128, o.rows - 1], rng.choice(o.rows, 5, replace=False)]))
+        # both tiles of the first units and the edges of every 128-row tile among them
+        quarters = [0, 127, 128, 255, 256, 383, 384, 511, 512, 1023]
+        rows = np.unique(np.concatenate([quarters, [o.rows - 1], rng.choice(o.rows, 5, replace=False)]))
         o.check(orc, rows_sel=rows)
     assert _tickets_clear(ws)
