@@ -14,7 +14,6 @@
 #include "kernels_diag.cuh"
 #include "kernels_spl.cuh"
 #include "kernels_umma.cuh"
-#include "kernels_pf_pair.cuh"
 #include "kernels_mlin.cuh"
 
 namespace mllm {
@@ -470,79 +469,6 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
         pg.total_units = units;
         const int64_t G = std::min<int64_t>(G0, units);
         fn<<<(unsigned)G, spl::kPfThreads, smem, st>>>(pg, err);
-        if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
-    }
-    *status = MLLM_OK;
-    return true;
-}
-
-// Clusters of sparse_linear_prefill_pair_kernel that can be resident at once (each takes two
-// SMs of one GPC); the persistent grid is sized to it so that no cluster waits for a wave.
-int64_t pair_clusters(int dev) {
-    static std::mutex mu;
-    static int cached[64] = {0};
-    std::lock_guard<std::mutex> lk(mu);
-    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
-    const void *fn = (const void *)spl::sparse_linear_prefill_pair_kernel;
-    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, spl::kP2Smem);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * spl::kP2MaxPairs, 1, 1);
-    cfg.blockDim = dim3(spl::kPfThreads, 1, 1);
-    cfg.dynamicSmemBytes = spl::kP2Smem;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        n = sm_count(dev) / 2;
-    }
-    n = std::min(n, spl::kP2MaxPairs);
-    if (dev >= 0 && dev < 64) cached[dev] = n;
-    return n;
-}
-
-// 2:4 at prefill sizes on SM pairs: units of (operand, 512 rows, 128 tokens); operand order
-// and unit order as for the single-SM kernel. Returns false when a tensor map cannot be
-// encoded (the caller then runs 64-token groups).
-bool sparse_linear_prefill_pair(const std::vector<mllm_sparse_operand> &ops_in, int32_t tokens, unsigned int *err,
-                                cudaStream_t st, mllm_status *status) {
-    std::vector<mllm_sparse_operand> ops = ops_in;
-    std::stable_sort(ops.begin(), ops.end(),
-                     [](const mllm_sparse_operand &a, const mllm_sparse_operand &b) { return a.cols > b.cols; });
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const int64_t P0 = pair_clusters(dev);
-    for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
-        const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
-        static thread_local spl::PfGroup pg;
-        pg = spl::PfGroup{};
-        pg.tokens = tokens;
-        const int64_t nt = (tokens + spl::kPfTok - 1) / spl::kPfTok;
-        int64_t units = 0;
-        for (size_t k = 0; k < n; ++k) {
-            const mllm_sparse_operand &o = ops[i0 + k];
-            spl::PfOp &d = pg.d[k];
-            d.meta = o.pack_meta;
-            d.y = o.y;
-            d.rows = o.rows;
-            d.cols = o.cols;
-            d.nch = o.cols / spl::kTmChunk;
-            d.npairs = (o.rows + spl::kP2RowUnit - 1) / spl::kP2RowUnit;  // row units of 512
-            d.nt = nt;
-            d.rgroup = std::max<int64_t>(1, (P0 + nt - 1) / nt);
-            d.unit_begin = units;
-            units += d.npairs * nt;
-            const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
-            if (!(encode_2d(&pg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 64,
-                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
-                  encode_2d(&pg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT32, o.pack_meta, cols / 32, rows, cols / 8, 4,
-                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                  encode_2d(&pg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
-                            (uint32_t)spl::kP2Half, CU_TENSOR_MAP_SWIZZLE_128B)))
-                return false;
-        }
-        pg.n = (int32_t)n;
-        pg.total_units = units;
-        const int64_t P = std::min<int64_t>(P0, units);
-        spl::sparse_linear_prefill_pair_kernel<<<(unsigned)(2 * P), spl::kPfThreads, spl::kP2Smem, st>>>(pg, err);
         if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
     }
     *status = MLLM_OK;
