@@ -1,0 +1,256 @@
+// kernels_pf48.cuh -- the 4:8 serving product at prefill sizes (more than 64 tokens).
+//
+// y = x W*^T from the packed 4:8 hard mask (MaskLLM serves the masked network from its hard
+// mask after training: paper-graph-ui summary of arXiv 2409.17481, s.3.2 "Information flow at
+// inference"; s.5 Table 16 times 128- and 2048-token prompts). 4:8 has no hardware sparse
+// mode, so each stage of compressed blocks is expanded to a dense bf16 tile in shared memory
+// (the byte-permute expansion of sparse_linear_umma48_kernel, same selector tables) and fed to
+// dense tcgen05.mma (kind::f16). Unlike the decode kernel, which expands every weight once per
+// group of at most 64 tokens, a stage here is expanded once for 256 tokens: the MMA's N is 256
+// and the accumulator (128 rows x 256 tokens of fp32) fills 256 tensor-memory columns.
+//
+// A unit is (operand, 128-row tile, 256-token chunk) over all columns, in stages of 64 columns
+// (eight 4:8 blocks per row). Per stage the copy warp lands, on one mbarrier, the 256 x 64 box
+// of x (128-byte swizzle, the MMA's K-major layout), the 128 x 32 box of compressed values and
+// the 128 x 8 box of codes; the 16 expansion warps write the 128 x 64 dense atom (128-byte
+// swizzle) and arrive on the stage's "expanded" barrier; the MMA warp issues four MMAs
+// (K = 16) and commits them to the stage's "empty" barrier, and at a unit's last stage to the
+// accumulator barrier; then the same 16 warps store the unit's y (warp w: TMEM lane quarter
+// w % 4, tokens 64 (w / 4) ... + 63). Units are dealt round-robin to one CTA per SM in the
+// order of the 2:4 prefill kernel (row-tile groups, token chunk by token chunk), so a weight
+// strip is read from HBM about once per launch. Rows and tokens past the call are zero-filled
+// by the tensor maps and not stored. Every wait is bounded; a timeout sets the error word and
+// the CTA winds down as the other tensor-memory kernels do.
+#pragma once
+
+#include "kernels_umma.cuh"
+
+namespace mllm {
+namespace spl {
+
+constexpr int kP8Tok = 256;                              // MMA N: tokens per unit
+constexpr int kP8Stages = 3;
+constexpr int kP8XOff = 0;                               // x: 256 tokens x 64 columns (32 KB)
+constexpr int kP8DenseOff = kP8Tok * 128;                // the dense atom: 128 rows x 64 columns (16 KB)
+constexpr int kP8ValOff = kP8DenseOff + kUmRows * 128;   // values: 128 rows x 32 bf16 (8 KB, unswizzled)
+constexpr int kP8MetaOff = kP8ValOff + kUmRows * 64;     // codes: 128 rows x 8 uint16 (2 KB)
+constexpr int kP8StageTx = kP8Tok * 128 + kUmRows * 64 + kUmRows * 16;  // bytes the copy engine lands
+constexpr int kP8Stage = (kP8MetaOff + kUmRows * 16 + 1023) / 1024 * 1024;
+constexpr int kP8Smem = kP8Stages * kP8Stage + 1024 + kU8TabBytes;
+constexpr unsigned kP8TmemCols = 256;
+constexpr int kP8Threads = 32 * kU8Warps + 64;           // 16 expansion/epilogue warps, copy, MMA
+
+// Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
+// N = 256, M = 128.
+constexpr uint32_t p8_idesc() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kP8Tok >> 3) << 17) | ((uint32_t)(kUmRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void p8_issue(const PfGroup &g, const PfCur &c, int64_t j, unsigned stage, unsigned bar) {
+    const TmMaps &mp = g.maps[c.op];
+    const int row0 = (int)(c.pair * kUmRows), tok0 = (int)(c.tc * kP8Tok);
+    mbar_arrive_tx(bar, (unsigned)kP8StageTx);
+    tma_load_2d(stage + kP8XOff, &mp.x, (int)(64 * j), tok0, bar);
+    tma_load_2d(stage + kP8ValOff, &mp.vals, (int)(32 * j), row0, bar);
+    tma_load_2d(stage + kP8MetaOff, &mp.meta, (int)(8 * j), row0, bar);
+}
+
+// Thread (r, pt) of the stage: row r, blocks 2 pt and 2 pt + 1 (one 16-byte value chunk, one
+// word of two codes) into dense chunks 2 pt + h of row r. Four consecutive threads share a
+// row, so a quarter-warp reads 128 contiguous bytes of values.
+__device__ __forceinline__ void p8_expand(unsigned char *st, const uint4 *tab_a, const uint4 *tab_b, int r, int pt) {
+    const uint4 v = lds128(st + kP8ValOff + r * 64 + pt * 16);
+    const uint32_t cw = lds32(st + kP8MetaOff + r * 16 + pt * 4);
+    unsigned char *row = st + kP8DenseOff + r * 128;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
+        const uint32_t code = (cw >> (16 * h)) & 0xFFFu;
+        const uint4 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
+        uint4 o;
+        o.x = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
+        o.y = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
+        o.z = __byte_perm(__byte_perm(lo, 0u, sa.z), hi, sb.z);
+        o.w = __byte_perm(__byte_perm(lo, 0u, sa.w), hi, sb.w);
+        const int b = 2 * pt + h;
+        *reinterpret_cast<uint4 *>(row + ((b ^ (r & 7)) << 4)) = o;
+    }
+}
+
+__global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(const __grid_constant__ PfGroup pg,
+                                                                              unsigned int *__restrict__ err) {
+    static_assert(kP8Smem + 1024 <= 232448, "fits one SM");
+    static_assert(kU8Warps == 16, "four threads per row, 128 rows");
+    constexpr int kD = kP8Stages;
+    constexpr int kBar = 32 * kU8Warps;
+    constexpr uint32_t kIdesc = p8_idesc();
+    extern __shared__ unsigned char s_dyn_p8[];
+    __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_exp[kD], s_acc;
+    __shared__ unsigned s_tmem;
+    __shared__ volatile int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t G = gridDim.x, u0 = blockIdx.x, u1 = pg.total_units;
+    const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_p8);
+    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
+    unsigned char *ring = s_dyn_p8 + pad;
+    const unsigned ring_s = dyn_s + pad;
+    uint4 *tab = reinterpret_cast<uint4 *>(ring + kD * kP8Stage);  // A: entries [0, 64), B: [64, 128), x copies
+    const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
+    const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
+    const unsigned exp0 = (unsigned)__cvta_generic_to_shared(&s_exp[0]);
+    const unsigned accb = (unsigned)__cvta_generic_to_shared(&s_acc);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kD; ++s) {
+            mbar_init(full0 + 8 * s, 1u);
+            mbar_init(empty0 + 8 * s, 1u);
+            mbar_init(exp0 + 8 * s, (unsigned)kBar);  // every expanding thread arrives once per stage
+        }
+        mbar_init(accb, 1u);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    for (int i = threadIdx.x; i < 2 * 64 * kU8TabCopies; i += blockDim.x)  // entry e, copy c at e * copies + c
+        tab[i] = u8_table_entry((i / kU8TabCopies) & 63, i >= 64 * kU8TabCopies);
+    if (warp == 0) {
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(&s_tmem);
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst),
+                     "r"(kP8TmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const unsigned tbase = s_tmem;
+
+    if (warp == kU8Warps) {
+        // ------------------------------------------------------------ copy warp
+        int f = 0, issued = 0;
+        bool stop = false;
+        for (int64_t u = u0; u < u1 && !stop; u += G) {
+            const PfCur c = pf_decode(pg, u);
+            const int64_t nch = pg.d[c.op].nch;
+            for (int64_t j = 0; j < nch; ++j, ++f) {
+                const int s = f % kD;
+                if (f >= kD && !um_wait(empty0 + 8 * s, ((f / kD) - 1) & 1, &s_abort)) {
+                    if (lane == 0 && !s_abort) {
+                        atomicOr(err, 1u);
+                        s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    fence_proxy_async();
+                    p8_issue(pg, c, j, ring_s + s * kP8Stage, full0 + 8 * s);
+                }
+                ++issued;
+            }
+        }
+        for (int s = 0; s < kD && s < issued; ++s) {
+            const int last = s + ((issued - 1 - s) / kD) * kD;
+            tm_wait(full0 + 8 * s, (last / kD) & 1);
+        }
+    } else if (warp == kU8Warps + 1) {
+        // ------------------------------------------------------------ MMA warp
+        int f = 0, commits = 0;
+        bool stop = false;
+        for (int64_t u = u0; u < u1 && !stop; u += G) {
+            const PfCur c = pf_decode(pg, u);
+            const int64_t nch = pg.d[c.op].nch;
+            for (int64_t j = 0; j < nch; ++j, ++f) {
+                const int s = f % kD;
+                if (!um_wait(exp0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                    if (lane == 0 && !s_abort) {
+                        atomicOr(err, 1u);
+                        s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const unsigned st = ring_s + s * kP8Stage;
+                    const uint64_t a0 = um_desc(st + kP8DenseOff), b0 = um_desc(st + kP8XOff);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_dense(tbase, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), kIdesc,
+                                   (j == 0 && k == 0) ? 0u : 1u);
+                    umma_commit(empty0 + 8 * s);
+                    if (j == nch - 1) umma_commit(accb);
+                }
+                __syncwarp();
+                ++commits;
+            }
+        }
+        if (commits > 0) {
+            const int ff = commits - 1;
+            tm_wait(empty0 + 8 * (ff % kD), (ff / kD) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ expansion / epilogue warps
+        const int r = threadIdx.x >> 2, pt = threadIdx.x & 3;  // expansion: row, part
+        const int q = warp & 3, sl = warp >> 2;                // epilogue: TMEM lane quarter, token slice
+        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(64 * sl);
+        const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
+        unsigned acc_phase = 0u;
+        bool failed = false;
+        int f = 0;
+        for (int64_t u = u0; u < u1; u += G) {
+            const PfCur c = pf_decode(pg, u);
+            const PfOp &d = pg.d[c.op];
+            for (int64_t j = 0; j < d.nch; ++j, ++f) {
+                const int s = f % kD;
+                if (!failed) {
+                    if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
+                        p8_expand(ring + s * kP8Stage, tab_a, tab_b, r, pt);
+                        fence_proxy_async();  // the dense atom, written here, is read by the tensor cores
+                        mbar_arrive(exp0 + 8 * s);
+                    } else {
+                        failed = true;
+                        if (lane == 0 && !s_abort) {
+                            atomicOr(err, 1u);
+                            s_abort = 1;
+                        }
+                    }
+                }
+            }
+            // ---------------------------------------------------- epilogue of the unit
+            const bool acc_ok = !failed && um_wait(accb, acc_phase, &s_abort);
+            acc_phase ^= 1u;
+            if (um_bar_or<kBar>(!acc_ok)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            const int tok0 = (int)(c.tc * kP8Tok) + 64 * sl;
+            const int64_t row = c.pair * kUmRows + 32 * q + lane;
+#pragma unroll 1
+            for (int k = 0; k < 64; k += 16) {
+                float v[16];
+                tmem_ld16(tq + k, v);
+                if (row < d.rows) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (tok0 + k + i < pg.tokens) d.y[(int64_t)(tok0 + k + i) * d.rows + row] = v[i];
+                }
+            }
+            tc_fence_before();
+            um_bar<kBar>();  // every read of the accumulator precedes the next unit's first arrival
+        }
+        if (failed && threadIdx.x == 0 && !s_abort) {
+            atomicOr(err, 1u);
+            s_abort = 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kP8TmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace spl
+}  // namespace mllm

@@ -14,6 +14,7 @@
 #include "kernels_diag.cuh"
 #include "kernels_spl.cuh"
 #include "kernels_umma.cuh"
+#include "kernels_pf48.cuh"
 #include "kernels_mlin.cuh"
 
 namespace mllm {
@@ -469,6 +470,59 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
         pg.total_units = units;
         const int64_t G = std::min<int64_t>(G0, units);
         fn<<<(unsigned)G, spl::kPfThreads, smem, st>>>(pg, err);
+        if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
+    }
+    *status = MLLM_OK;
+    return true;
+}
+
+// 4:8 at prefill sizes: units of (operand, 128 rows, 256 tokens) over 64-column stages, each
+// stage expanded to dense once; operand and unit order as for the 2:4 prefill kernel. Returns
+// false when a tensor map cannot be encoded (the caller then runs 64-token groups).
+bool sparse_linear_prefill48(const std::vector<mllm_sparse_operand> &ops_in, int32_t tokens, unsigned int *err,
+                             cudaStream_t st, mllm_status *status) {
+    std::vector<mllm_sparse_operand> ops = ops_in;
+    std::stable_sort(ops.begin(), ops.end(),
+                     [](const mllm_sparse_operand &a, const mllm_sparse_operand &b) { return a.cols > b.cols; });
+    auto fn = spl::sparse_linear_prefill48_kernel;
+    constexpr int smem = spl::kP8Smem;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    resident_ctas(dev, (const void *)fn, spl::kP8Threads, smem);  // sets the dynamic shared-memory limit
+    for (size_t i0 = 0; i0 < ops.size(); i0 += kMaxMats) {
+        const size_t n = std::min<size_t>(kMaxMats, ops.size() - i0);
+        static thread_local spl::PfGroup pg;
+        pg = spl::PfGroup{};
+        pg.tokens = tokens;
+        const int64_t nt = (tokens + spl::kP8Tok - 1) / spl::kP8Tok;
+        const int64_t G0 = std::min<int64_t>((int64_t)sm_count(dev), (int64_t)spl::kPfMaxCtas);
+        int64_t units = 0;
+        for (size_t k = 0; k < n; ++k) {
+            const mllm_sparse_operand &o = ops[i0 + k];
+            spl::PfOp &d = pg.d[k];
+            d.meta = o.pack_meta;
+            d.y = o.y;
+            d.rows = o.rows;
+            d.cols = o.cols;
+            d.nch = o.cols / 64;                                   // 64-column stages
+            d.npairs = (o.rows + spl::kUmRows - 1) / spl::kUmRows;  // 128-row tiles
+            d.nt = nt;
+            d.rgroup = std::max<int64_t>(1, (G0 + nt - 1) / nt);
+            d.unit_begin = units;
+            units += d.npairs * nt;
+            const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
+            if (!(encode_2d(&pg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 32,
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  encode_2d(&pg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT16, o.pack_meta, cols / 8, rows, cols / 4, 8,
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  encode_2d(&pg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
+                            (uint32_t)spl::kP8Tok, CU_TENSOR_MAP_SWIZZLE_128B)))
+                return false;
+        }
+        pg.n = (int32_t)n;
+        pg.total_units = units;
+        const int64_t G = std::min<int64_t>(G0, units);
+        fn<<<(unsigned)G, spl::kP8Threads, smem, st>>>(pg, err);
         if ((*status = cuda_status(cudaGetLastError())) != MLLM_OK) return true;
     }
     *status = MLLM_OK;
@@ -1114,12 +1168,18 @@ mllm_status mllm_sparse_linear(const mllm_sparse_operand *ops, int32_t n_ops, ml
         else act.push_back(ops[i]);
     }
     if (tokens > spl::kMaxTokens) {
-        // prefill-sized calls: 2:4 on the prefill kernel; 4:8 through the batched kernel in
-        // groups of 64 tokens (x and y rows offset)
+        // prefill-sized calls: on the prefill kernels (2:4 sparse MMA, 4:8 expanded once per
+        // stage for 256 tokens); if a tensor map cannot be encoded, 4:8 through the batched
+        // kernel in groups of 64 tokens (x and y rows offset)
+        bool grouped = false;
         if (!batched.empty() && nm.m == 4) {
             if (!sparse_linear_prefill(batched, tokens, err, st, &s)) act.insert(act.end(), batched.begin(), batched.end());
             if (s != MLLM_OK) return s;
         } else if (!batched.empty()) {
+            grouped = !sparse_linear_prefill48(batched, tokens, err, st, &s);
+            if (s != MLLM_OK) return s;
+        }
+        if (grouped) {
             for (int32_t t0 = 0; t0 < tokens; t0 += spl::kMaxTokens) {
                 std::vector<mllm_sparse_operand> grp = batched;
                 for (mllm_sparse_operand &o : grp) {

@@ -361,10 +361,10 @@ def test_side_streams_and_concurrent_host_threads(orc, tokens):
 @pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
 @pytest.mark.parametrize("tokens", [65, 128, 200, 512])
 def test_prefill_sized_calls(orc, ws, nm, tokens):
-    """More than 64 tokens: 2:4 operands whose columns are whole 128-column stages run on the
-    prefill kernel (units of two 128-row tiles x 128 tokens), the others in groups of 16
-    tokens; 4:8 in groups of 64 tokens. Ragged rows and token chunks, several operands in one
-    call."""
+    """More than 64 tokens: operands whose columns are whole 128-column stages run on the
+    prefill kernels (2:4: units of two 128-row tiles x 128 tokens; 4:8: 128 rows x 256
+    tokens, each stage expanded once), the others in groups of 16 tokens. Ragged rows and
+    token chunks, several operands in one call."""
     shapes = [(300, 512), (128, 1024), (37, 1040), (200, 128)]
     ops = [Operand(orc, nm, r, c, tokens, seed=900 + 10 * i + tokens) for i, (r, c) in enumerate(shapes)]
     mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
@@ -374,14 +374,16 @@ def test_prefill_sized_calls(orc, ws, nm, tokens):
     assert _tickets_clear(ws)
 
 
+@pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
 @pytest.mark.parametrize("tokens", [128, 512, 2048])
-def test_prefill_llama_layer_sampled_rows(orc, ws, tokens):
-    """The LLaMA-2-7B layer's seven 2:4 matrices at prefill sizes (the page's 128- and
-    2048-token prompts), in one call; y checked on sampled rows, all tokens."""
+def test_prefill_llama_layer_sampled_rows(orc, ws, nm, tokens):
+    """The LLaMA-2-7B layer's seven matrices at prefill sizes (the page's 128- and
+    2048-token prompts), packed 2:4 (sparse MMA) or 4:8 (expanded once per stage for 256
+    tokens), in one call; y checked on sampled rows, all tokens."""
     w = configs.WORKLOADS["llama2_7b_layer_2of4"]
     rng = np.random.default_rng(tokens)
-    ops = [Operand(orc, (2, 4), m.rows, m.cols, tokens, seed=950 + i, direct=True) for i, m in enumerate(w.matrices)]
-    mllm_sparse_linear([o.op() for o in ops], (2, 4), tokens, ws)
+    ops = [Operand(orc, nm, m.rows, m.cols, tokens, seed=950 + i, direct=True) for i, m in enumerate(w.matrices)]
+    mllm_sparse_linear([o.op() for o in ops], nm, tokens, ws)
     torch.cuda.synchronize()
     for o in ops:
         # both tiles of the first units and the edges of every 128-row tile among them
