@@ -7,16 +7,17 @@
 // (the byte-permute expansion of sparse_linear_umma48_kernel, same selector tables) and fed to
 // dense tcgen05.mma (kind::f16). Unlike the decode kernel, which expands every weight once per
 // group of at most 64 tokens, a stage here is expanded once for 256 tokens: the MMA's N is 256
-// and the accumulator (128 rows x 256 tokens of fp32) fills 256 tensor-memory columns.
+// and the accumulator (128 rows x 256 tokens of fp32) fills 256 tensor-memory columns (calls
+// of at most 128 tokens use N = 128 and 128 columns, with four stages instead of three).
 //
-// A unit is (operand, 128-row tile, 256-token chunk) over all columns, in stages of 64 columns
-// (eight 4:8 blocks per row). Per stage the copy warp lands, on one mbarrier, the 256 x 64 box
+// A unit is (operand, 128-row tile, N-token chunk) over all columns, in stages of 64 columns
+// (eight 4:8 blocks per row). Per stage the copy warp lands, on one mbarrier, the N x 64 box
 // of x (128-byte swizzle, the MMA's K-major layout), the 128 x 32 box of compressed values and
 // the 128 x 8 box of codes; the 16 expansion warps write the 128 x 64 dense atom (128-byte
 // swizzle) and arrive on the stage's "expanded" barrier; the MMA warp issues four MMAs
 // (K = 16) and commits them to the stage's "empty" barrier, and at a unit's last stage to the
 // accumulator barrier; then the same 16 warps store the unit's y (warp w: TMEM lane quarter
-// w % 4, tokens 64 (w / 4) ... + 63). Units are dealt round-robin to one CTA per SM in the
+// w % 4, a quarter of the unit's tokens). Units are dealt round-robin to one CTA per SM in the
 // order of the 2:4 prefill kernel (row-tile groups, token chunk by token chunk), so a weight
 // strip is read from HBM about once per launch. Rows and tokens past the call are zero-filled
 // by the tensor maps and not stored. Every wait is bounded; a timeout sets the error word and
@@ -28,40 +29,45 @@
 namespace mllm {
 namespace spl {
 
-constexpr int kP8Tok = 256;                              // MMA N: tokens per unit
-constexpr int kP8Stages = 3;
-constexpr int kP8XOff = 0;                               // x: 256 tokens x 64 columns (32 KB)
-constexpr int kP8DenseOff = kP8Tok * 128;                // the dense atom: 128 rows x 64 columns (16 KB)
-constexpr int kP8ValOff = kP8DenseOff + kUmRows * 128;   // values: 128 rows x 32 bf16 (8 KB, unswizzled)
-constexpr int kP8MetaOff = kP8ValOff + kUmRows * 64;     // codes: 128 rows x 8 uint16 (2 KB)
-constexpr int kP8StageTx = kP8Tok * 128 + kUmRows * 64 + kUmRows * 16;  // bytes the copy engine lands
-constexpr int kP8Stage = (kP8MetaOff + kUmRows * 16 + 1023) / 1024 * 1024;
-constexpr int kP8Smem = kP8Stages * kP8Stage + 1024 + kU8TabBytes;
-constexpr unsigned kP8TmemCols = 256;
+// Tokens per unit (the MMA's N): 256, or 128 for calls of at most 128 tokens (a 256-token
+// unit would compute half of its columns on zero-filled tokens).
+template <int kTok> struct P8 {
+    static constexpr int kXOff = 0;                              // x: kTok tokens x 64 columns
+    static constexpr int kDenseOff = kTok * 128;                 // the dense atom: 128 rows x 64 columns (16 KB)
+    static constexpr int kValOff = kDenseOff + kUmRows * 128;    // values: 128 rows x 32 bf16 (8 KB, unswizzled)
+    static constexpr int kMetaOff = kValOff + kUmRows * 64;      // codes: 128 rows x 8 uint16 (2 KB)
+    static constexpr int kStageTx = kTok * 128 + kUmRows * 64 + kUmRows * 16;  // bytes the copy engine lands
+    static constexpr int kStage = (kMetaOff + kUmRows * 16 + 1023) / 1024 * 1024;
+    static constexpr int kStages = kTok == 256 ? 3 : 4;
+    static constexpr int kSmem = kStages * kStage + 1024 + kU8TabBytes;
+    static constexpr unsigned kTmemCols = kTok;
+    // Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
+    // N = kTok, M = 128.
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTok >> 3) << 17) | ((uint32_t)(kUmRows >> 4) << 24);
+};
 constexpr int kP8Threads = 32 * kU8Warps + 64;           // 16 expansion/epilogue warps, copy, MMA
 
-// Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
-// N = 256, M = 128.
-constexpr uint32_t p8_idesc() {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kP8Tok >> 3) << 17) | ((uint32_t)(kUmRows >> 4) << 24);
-}
-
+template <int kTok>
 __device__ __forceinline__ void p8_issue(const PfGroup &g, const PfCur &c, int64_t j, unsigned stage, unsigned bar) {
+    using K = P8<kTok>;
     const TmMaps &mp = g.maps[c.op];
-    const int row0 = (int)(c.pair * kUmRows), tok0 = (int)(c.tc * kP8Tok);
-    mbar_arrive_tx(bar, (unsigned)kP8StageTx);
-    tma_load_2d(stage + kP8XOff, &mp.x, (int)(64 * j), tok0, bar);
-    tma_load_2d(stage + kP8ValOff, &mp.vals, (int)(32 * j), row0, bar);
-    tma_load_2d(stage + kP8MetaOff, &mp.meta, (int)(8 * j), row0, bar);
+    const int row0 = (int)(c.pair * kUmRows), tok0 = (int)(c.tc * kTok);
+    mbar_arrive_tx(bar, (unsigned)K::kStageTx);
+    tma_load_2d(stage + K::kXOff, &mp.x, (int)(64 * j), tok0, bar);
+    tma_load_2d(stage + K::kValOff, &mp.vals, (int)(32 * j), row0, bar);
+    tma_load_2d(stage + K::kMetaOff, &mp.meta, (int)(8 * j), row0, bar);
 }
 
 // Thread (r, pt) of the stage: row r, blocks 2 pt and 2 pt + 1 (one 16-byte value chunk, one
 // word of two codes) into dense chunks 2 pt + h of row r. Four consecutive threads share a
 // row, so a quarter-warp reads 128 contiguous bytes of values.
+template <int kTok>
 __device__ __forceinline__ void p8_expand(unsigned char *st, const uint4 *tab_a, const uint4 *tab_b, int r, int pt) {
-    const uint4 v = lds128(st + kP8ValOff + r * 64 + pt * 16);
-    const uint32_t cw = lds32(st + kP8MetaOff + r * 16 + pt * 4);
-    unsigned char *row = st + kP8DenseOff + r * 128;
+    using K = P8<kTok>;
+    const uint4 v = lds128(st + K::kValOff + r * 64 + pt * 16);
+    const uint32_t cw = lds32(st + K::kMetaOff + r * 16 + pt * 4);
+    unsigned char *row = st + K::kDenseOff + r * 128;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
@@ -77,13 +83,15 @@ __device__ __forceinline__ void p8_expand(unsigned char *st, const uint4 *tab_a,
     }
 }
 
+template <int kTok>
 __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(const __grid_constant__ PfGroup pg,
                                                                               unsigned int *__restrict__ err) {
-    static_assert(kP8Smem + 1024 <= 232448, "fits one SM");
+    using K = P8<kTok>;
+    static_assert(K::kSmem + 1024 <= 232448, "fits one SM");
     static_assert(kU8Warps == 16, "four threads per row, 128 rows");
-    constexpr int kD = kP8Stages;
+    constexpr int kD = K::kStages, kP8Stage = K::kStage, kQTok = kTok / 4;  // epilogue: tokens per warp
     constexpr int kBar = 32 * kU8Warps;
-    constexpr uint32_t kIdesc = p8_idesc();
+    constexpr uint32_t kIdesc = K::kIdesc;
     extern __shared__ unsigned char s_dyn_p8[];
     __shared__ __align__(8) unsigned long long s_full[kD], s_empty[kD], s_exp[kD], s_acc;
     __shared__ unsigned s_tmem;
@@ -114,7 +122,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
     if (warp == 0) {
         const unsigned dst = (unsigned)__cvta_generic_to_shared(&s_tmem);
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst),
-                     "r"(kP8TmemCols)
+                     "r"(K::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
@@ -142,7 +150,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
                 }
                 if (lane == 0) {
                     fence_proxy_async();
-                    p8_issue(pg, c, j, ring_s + s * kP8Stage, full0 + 8 * s);
+                    p8_issue<kTok>(pg, c, j, ring_s + s * kP8Stage, full0 + 8 * s);
                 }
                 ++issued;
             }
@@ -171,7 +179,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
                 if (lane == 0) {
                     tc_fence_after();
                     const unsigned st = ring_s + s * kP8Stage;
-                    const uint64_t a0 = um_desc(st + kP8DenseOff), b0 = um_desc(st + kP8XOff);
+                    const uint64_t a0 = um_desc(st + K::kDenseOff), b0 = um_desc(st + K::kXOff);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         umma_dense(tbase, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), kIdesc,
@@ -191,7 +199,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
         // ------------------------------------------------------------ expansion / epilogue warps
         const int r = threadIdx.x >> 2, pt = threadIdx.x & 3;  // expansion: row, part
         const int q = warp & 3, sl = warp >> 2;                // epilogue: TMEM lane quarter, token slice
-        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(64 * sl);
+        const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(kQTok * sl);
         const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
         unsigned acc_phase = 0u;
         bool failed = false;
@@ -203,7 +211,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
                 const int s = f % kD;
                 if (!failed) {
                     if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
-                        p8_expand(ring + s * kP8Stage, tab_a, tab_b, r, pt);
+                        p8_expand<kTok>(ring + s * kP8Stage, tab_a, tab_b, r, pt);
                         fence_proxy_async();  // the dense atom, written here, is read by the tensor cores
                         mbar_arrive(exp0 + 8 * s);
                     } else {
@@ -223,10 +231,10 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
                 break;
             }
             tc_fence_after();
-            const int tok0 = (int)(c.tc * kP8Tok) + 64 * sl;
+            const int tok0 = (int)(c.tc * kTok) + kQTok * sl;
             const int64_t row = c.pair * kUmRows + 32 * q + lane;
 #pragma unroll 1
-            for (int k = 0; k < 64; k += 16) {
+            for (int k = 0; k < kQTok; k += 16) {
                 float v[16];
                 tmem_ld16(tq + k, v);
                 if (row < d.rows) {
@@ -247,7 +255,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kP8TmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(K::kTmemCols)
                      : "memory");
     }
 }

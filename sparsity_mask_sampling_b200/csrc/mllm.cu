@@ -476,16 +476,17 @@ bool sparse_linear_prefill(const std::vector<mllm_sparse_operand> &ops_in, int32
     return true;
 }
 
-// 4:8 at prefill sizes: units of (operand, 128 rows, 256 tokens) over 64-column stages, each
+// 4:8 at prefill sizes: units of (operand, 128 rows, kTok tokens) over 64-column stages, each
 // stage expanded to dense once; operand and unit order as for the 2:4 prefill kernel. Returns
 // false when a tensor map cannot be encoded (the caller then runs 64-token groups).
-bool sparse_linear_prefill48(const std::vector<mllm_sparse_operand> &ops_in, int32_t tokens, unsigned int *err,
-                             cudaStream_t st, mllm_status *status) {
+template <int kTok>
+bool sparse_linear_prefill48_n(const std::vector<mllm_sparse_operand> &ops_in, int32_t tokens, unsigned int *err,
+                               cudaStream_t st, mllm_status *status) {
     std::vector<mllm_sparse_operand> ops = ops_in;
     std::stable_sort(ops.begin(), ops.end(),
                      [](const mllm_sparse_operand &a, const mllm_sparse_operand &b) { return a.cols > b.cols; });
-    auto fn = spl::sparse_linear_prefill48_kernel;
-    constexpr int smem = spl::kP8Smem;
+    auto fn = spl::sparse_linear_prefill48_kernel<kTok>;
+    constexpr int smem = spl::P8<kTok>::kSmem;
     int dev = 0;
     cudaGetDevice(&dev);
     resident_ctas(dev, (const void *)fn, spl::kP8Threads, smem);  // sets the dynamic shared-memory limit
@@ -494,7 +495,7 @@ bool sparse_linear_prefill48(const std::vector<mllm_sparse_operand> &ops_in, int
         static thread_local spl::PfGroup pg;
         pg = spl::PfGroup{};
         pg.tokens = tokens;
-        const int64_t nt = (tokens + spl::kP8Tok - 1) / spl::kP8Tok;
+        const int64_t nt = (tokens + kTok - 1) / kTok;
         const int64_t G0 = std::min<int64_t>((int64_t)sm_count(dev), (int64_t)spl::kPfMaxCtas);
         int64_t units = 0;
         for (size_t k = 0; k < n; ++k) {
@@ -516,7 +517,7 @@ bool sparse_linear_prefill48(const std::vector<mllm_sparse_operand> &ops_in, int
                   encode_2d(&pg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT16, o.pack_meta, cols / 8, rows, cols / 4, 8,
                             spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   encode_2d(&pg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
-                            (uint32_t)spl::kP8Tok, CU_TENSOR_MAP_SWIZZLE_128B)))
+                            (uint32_t)kTok, CU_TENSOR_MAP_SWIZZLE_128B)))
                 return false;
         }
         pg.n = (int32_t)n;
@@ -527,6 +528,12 @@ bool sparse_linear_prefill48(const std::vector<mllm_sparse_operand> &ops_in, int
     }
     *status = MLLM_OK;
     return true;
+}
+
+bool sparse_linear_prefill48(const std::vector<mllm_sparse_operand> &ops, int32_t tokens, unsigned int *err,
+                             cudaStream_t st, mllm_status *status) {
+    return tokens <= 128 ? sparse_linear_prefill48_n<128>(ops, tokens, err, st, status)
+                         : sparse_linear_prefill48_n<256>(ops, tokens, err, st, status);
 }
 
 // The per-warp kernels for up to 16 tokens; every operand has rows > 0 and cols > 0.
