@@ -301,10 +301,11 @@ typedef struct {
  * i.e. y = x W*^T, with bf16 products accumulated in fp32 (tensor cores), for 1 <= tokens
  * <= 16384. Decode-sized calls (up to 64 tokens) are bound by reading the compressed weight,
  * which operands whose cols are a multiple of 128 read once per call (above 16 tokens the
- * others run as groups of 16 tokens). Above 64 tokens (prefill), 2:4 operands whose cols are
- * a multiple of 128 run on the sparse tensor cores in units of 128 rows x 128 tokens (each
- * unit over all columns, no unit split between CTAs); 4:8 operands run as groups of 64 tokens
- * and other widths as groups of 16.
+ * others run as groups of 16 tokens). Above 64 tokens (prefill), operands whose cols are a
+ * multiple of 128 run in units over all columns, no unit split between CTAs: 2:4 on the
+ * sparse tensor cores (two 128-row tiles x 128 tokens), 4:8 expanded to dense once per
+ * 64-column stage for 256 tokens (128 for calls of at most 128 tokens); other widths run as
+ * groups of 16 tokens.
  * Operands may differ in shape and are processed in one launch per 16 of them; rows == 0
  * operands are skipped and cols == 0 gives y = 0 (pointers other than y may then be NULL).
  * workspace: device memory of mllm_sparse_linear_workspace_bytes() bytes, zero-filled by the
