@@ -230,6 +230,32 @@ __device__ __forceinline__ float gumbel_unit(uint32_t unit_bits, const NlogCtx &
     return -nlog(t, L.tab);
 }
 
+// ---------------------------------------------------------------------------- paired forms
+//
+// The same arithmetic on two independent values at once with the fp32x2 instructions of
+// sm_100 (__ffma2_rn, __fmul2_rn, __fadd2_rn: each component rounds exactly as __fmaf_rn,
+// __fmul_rn, __fadd_rn), so every result is bit-identical to the scalar form while a pair
+// costs one instruction where the scalar form costs two. Table lookups, integer steps and
+// the special-function instructions stay per value.
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// (-nlog(x.x), -nlog(x.y)): the negation folded into the last add, (-T) + (-p) = -(T + p).
+__device__ __forceinline__ float2 neg_nlog2(float2 x, const float2 *__restrict__ tab) {
+    const float2 ca = tab[((__float_as_uint(x.x) + 0x408000u) >> 16) - kNlogIndexBias];
+    const float2 cb = tab[((__float_as_uint(x.y) + 0x408000u) >> 16) - kNlogIndexBias];
+    const float2 r = make_float2(__fmaf_rn(x.x, ca.x, -1.0f), __fmaf_rn(x.y, cb.x, -1.0f));
+    const float2 q = __ffma2_rn(r, f2(kOneThird), f2(-0.5f));
+    const float2 rq = __fmul2_rn(r, q);
+    const float2 p = __ffma2_rn(rq, r, r);
+    return make_float2(__fadd_rn(-ca.y, -p.x), __fadd_rn(-cb.y, -p.y));
+}
+
+// gumbel_unit of two fields.
+__device__ __forceinline__ float2 gumbel_unit2(uint32_t ua, uint32_t ub, const NlogCtx &L) {
+    const float2 eps = __fadd2_rn(make_float2(__uint_as_float(ua), __uint_as_float(ub)), f2(-1.0f));
+    return neg_nlog2(neg_nlog2(eps, L.tab), L.tab);
+}
+
 // Copy the table into shared memory (all threads; __syncthreads() before use).
 __device__ __forceinline__ void load_tab(float2 *s_tab) {
     const float4 *src = reinterpret_cast<const float4 *>(g_noise_table.cT);

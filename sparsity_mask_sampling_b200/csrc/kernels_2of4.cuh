@@ -89,6 +89,20 @@ __device__ __forceinline__ void store12(float *base, int64_t b0, bool two, const
     }
 }
 
+// load12 / store12 as six pairs (elements 2k, 2k+1).
+__device__ __forceinline__ void load12x2(const float *base, int64_t b0, bool two, float2 v[6]) {
+    float t[12];
+    load12(base, b0, two, t);
+#pragma unroll
+    for (int k = 0; k < 6; ++k) v[k] = make_float2(t[2 * k], t[2 * k + 1]);
+}
+__device__ __forceinline__ void store12x2(float *base, int64_t b0, bool two, const float2 v[6]) {
+    float t[12];
+#pragma unroll
+    for (int k = 0; k < 6; ++k) { t[2 * k] = v[k].x; t[2 * k + 1] = v[k].y; }
+    store12(base, b0, two, t);
+}
+
 // --------------------------------------------------------------------------- per-block math
 
 // Gumbel noise of the block's six candidates at the step of sc: one Philox call, six fields.
@@ -133,6 +147,49 @@ __device__ __forceinline__ void soft_mask_comp(const float e[6], float r, float 
     mc[1] = (e[1] + e[2] + e[5]) * r;
     mc[2] = (e[0] + e[2] + e[3]) * r;
     mc[3] = (e[0] + e[1] + e[4]) * r;
+}
+
+// --------------------------------------------------------------------------- paired forms
+// (bit-identical to the scalar helpers above; see the paired forms in device_common.cuh)
+
+// noise6 as three pairs (g0 g1), (g2 g3), (g4 g5).
+__device__ __forceinline__ void noise6x2(const StepScalars &sc, uint64_t gid, const NlogCtx &L, float2 g[3]) {
+    if (!sc.noise_on) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k) g[k] = make_float2(0.f, 0.f);
+        return;
+    }
+    uint32_t u[6];
+    fields21_unit(block_words(sc, gid, 0u), u);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) g[k] = gumbel_unit2(u[2 * k], u[2 * k + 1], L);
+}
+
+// soft_index with the logits and noise as pairs (pi2[k] = (pi_2k, pi_2k+1)).
+__device__ __forceinline__ void soft_index2(const float2 pi2[3], const float2 g[3], float kappa, float c2,
+                                            float e[6], float &r) {
+    float2 w[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k) w[k] = __ffma2_rn(f2(kappa), pi2[k], g[k]);
+    const float mx = fmaxf(fmaxf(fmaxf(w[0].x, w[0].y), fmaxf(w[1].x, w[1].y)), fmaxf(w[2].x, w[2].y));
+    const float mc = __fmul_rn(mx, c2);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const float2 a = __ffma2_rn(w[k], f2(c2), f2(-mc));
+        e[2 * k] = ex2_approx(a.x);
+        e[2 * k + 1] = ex2_approx(a.y);
+    }
+    const float s = __fadd_rn(__fadd_rn(__fadd_rn(e[0], e[1]), __fadd_rn(e[2], e[3])), __fadd_rn(e[4], e[5]));
+    r = rcp_approx(s);
+}
+
+// AdamW, PyTorch step order, two elements.
+__device__ __forceinline__ void adamw2(float2 &p, float2 &m, float2 &v, float2 g, const StepScalars &s) {
+    const float2 pd = __fmul2_rn(p, f2(s.decay));
+    m = __ffma2_rn(f2(s.beta1), m, __fmul2_rn(f2(s.one_minus_beta1), g));
+    v = __ffma2_rn(f2(s.beta2), v, __fmul2_rn(f2(s.one_minus_beta2), __fmul2_rn(g, g)));
+    const float2 denom = __ffma2_rn(make_float2(sqrt_approx(v.x), sqrt_approx(v.y)), f2(s.inv_sqrt_bc2), f2(s.eps));
+    p = __ffma2_rn(f2(-s.step_size), make_float2(__fdividef(m.x, denom.x), __fdividef(m.y, denom.y)), pd);
 }
 
 // AdamW, PyTorch step order, one element.
@@ -308,28 +365,34 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_adam_fwd_kernel(const __grid_
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
-        float w[8], gw[8], pi[12], mo[12], vo[12], x[8], msv[8];
+        float w[8], gw[8], x[8], msv[8];
+        float2 pi[6], mo[6], vo[6];  // pairs (2k, 2k+1); block h holds pairs 3h .. 3h+2
         load_vals<kW32>(d.W, b0, two, w);
         load_vals<kG32>(d.G, b0, two, gw);
-        load12(d.pi, b0, two, pi);
-        load12(d.m, b0, two, mo);
-        load12(d.v, b0, two, vo);
+        load12x2(d.pi, b0, two, pi);
+        load12x2(d.m, b0, two, mo);
+        load12x2(d.v, b0, two, vo);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const uint64_t gid = d.gid0 + b0 + h;
             {   // backward + AdamW, step t
-                float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
-                noise6(sb, gid, L, g);
-                soft_index(pi + 6 * h, g, sb.kappa, sb.c2, e, r);
+                float2 g[3];
+                float e[6], r, ms[4], mc[4], P[4], Q[4];
+                noise6x2(sb, gid, L, g);
+                soft_index2(pi + 3 * h, g, sb.kappa, sb.c2, e, r);
                 soft_mask(e, r, ms);
                 soft_mask_comp(e, r, mc);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float wj = w[4 * h + j];
-                    const float u = __fmaf_rn(-__fmul_rn(sb.two_lambda, __fmul_rn(wj, wj)), ms[j],
-                                              __fmul_rn(gw[4 * h + j], wj));
-                    P[j] = __fmul_rn(mc[j], u);
-                    Q[j] = __fmul_rn(ms[j], u);
+                for (int k = 0; k < 2; ++k) {  // positions 2k, 2k+1
+                    const float2 wj = make_float2(w[4 * h + 2 * k], w[4 * h + 2 * k + 1]);
+                    const float2 gj = make_float2(gw[4 * h + 2 * k], gw[4 * h + 2 * k + 1]);
+                    const float2 msj = make_float2(ms[2 * k], ms[2 * k + 1]);
+                    const float2 mcj = make_float2(mc[2 * k], mc[2 * k + 1]);
+                    // u_j = G_j W_j - 2 lambda W_j^2 M_j, as fma(-(2 lambda W_j^2), M_j, G_j W_j)
+                    const float2 u = __ffma2_rn(__fmul2_rn(f2(-sb.two_lambda), __fmul2_rn(wj, wj)), msj, __fmul2_rn(gj, wj));
+                    const float2 pp = __fmul2_rn(mcj, u), qq = __fmul2_rn(msj, u);
+                    P[2 * k] = pp.x; P[2 * k + 1] = pp.y;
+                    Q[2 * k] = qq.x; Q[2 * k + 1] = qq.y;
                 }
                 float D[6];
                 D[0] = (P[0] + P[1]) - (Q[2] + Q[3]);
@@ -339,36 +402,44 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_adam_fwd_kernel(const __grid_
                 D[4] = (P[1] + P[2]) - (Q[0] + Q[3]);
                 D[5] = (P[2] + P[3]) - (Q[0] + Q[1]);
                 const float cr = __fmul_rn(sb.kappa_over_tau, r);
-                float grad[6];
+                float2 grad[3];
 #pragma unroll
-                for (int i = 0; i < C; ++i) {
-                    grad[i] = __fmul_rn(__fmul_rn(cr, e[i]), D[i]);
-                    adamw(pi[6 * h + i], mo[6 * h + i], vo[6 * h + i], grad[i], sb);
+                for (int k = 0; k < 3; ++k) {
+                    grad[k] = __fmul2_rn(__fmul2_rn(f2(cr), make_float2(e[2 * k], e[2 * k + 1])),
+                                         make_float2(D[2 * k], D[2 * k + 1]));
+                    adamw2(pi[3 * h + k], mo[3 * h + k], vo[3 * h + k], grad[k], sb);
                 }
                 if (d.grad && (h == 0 || two)) {
                     float2 *gp = reinterpret_cast<float2 *>(d.grad + (b0 + h) * C);
-                    gp[0] = make_float2(grad[0], grad[1]);
-                    gp[1] = make_float2(grad[2], grad[3]);
-                    gp[2] = make_float2(grad[4], grad[5]);
+                    gp[0] = grad[0];
+                    gp[1] = grad[1];
+                    gp[2] = grad[2];
                 }
             }
             {   // forward, step t+1, from the updated logits
-                float g[6], e[6], r, ms[4];
-                noise6(sf, gid, L, g);
-                soft_index(pi + 6 * h, g, sf.kappa, sf.c2, e, r);
+                float2 g[3];
+                float e[6], r, ms[4];
+                noise6x2(sf, gid, L, g);
+                soft_index2(pi + 3 * h, g, sf.kappa, sf.c2, e, r);
                 soft_mask(e, r, ms);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float xj = __fmul_rn(w[4 * h + j], ms[j]);
-                    x[4 * h + j] = xj;
-                    msv[4 * h + j] = ms[j];
-                    if (h == 0 || two) acc = __fmaf_rn(xj, xj, acc);
+                for (int k = 0; k < 2; ++k) {
+                    const float2 xj = __fmul2_rn(make_float2(w[4 * h + 2 * k], w[4 * h + 2 * k + 1]),
+                                                 make_float2(ms[2 * k], ms[2 * k + 1]));
+                    x[4 * h + 2 * k] = xj.x;
+                    x[4 * h + 2 * k + 1] = xj.y;
+                    msv[4 * h + 2 * k] = ms[2 * k];
+                    msv[4 * h + 2 * k + 1] = ms[2 * k + 1];
+                    if (h == 0 || two) {
+                        acc = __fmaf_rn(xj.x, xj.x, acc);
+                        acc = __fmaf_rn(xj.y, xj.y, acc);
+                    }
                 }
             }
         }
-        store12(d.pi, b0, two, pi);
-        store12(d.m, b0, two, mo);
-        store12(d.v, b0, two, vo);
+        store12x2(d.pi, b0, two, pi);
+        store12x2(d.m, b0, two, mo);
+        store12x2(d.v, b0, two, vo);
         store_vals<kW32>(d.X, b0, two, x);
         if (d.soft) {
             float4 *sp = reinterpret_cast<float4 *>(d.soft + b0 * 4);
