@@ -257,22 +257,30 @@ __global__ void __launch_bounds__(kThreads) fwd_kernel(const __grid_constant__ G
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
-        float w[8], pi[12];
+        float w[8];
+        float2 pi[6];
         load_vals<kW32>(d.W, b0, two, w);
-        load12(d.pi, b0, two, pi);
+        load12x2(d.pi, b0, two, pi);
         float x[8], msv[8];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float g[6], e[6], r, ms[4];
-            noise6(sc, d.gid0 + b0 + h, L, g);
-            soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, r);
+            float2 g[3];
+            float e[6], r, ms[4];
+            noise6x2(sc, d.gid0 + b0 + h, L, g);
+            soft_index2(pi + 3 * h, g, sc.kappa, sc.c2, e, r);
             soft_mask(e, r, ms);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float xj = __fmul_rn(w[4 * h + j], ms[j]);
-                x[4 * h + j] = xj;
-                msv[4 * h + j] = ms[j];
-                if (h == 0 || two) acc = __fmaf_rn(xj, xj, acc);
+            for (int k = 0; k < 2; ++k) {
+                const float2 xj = __fmul2_rn(make_float2(w[4 * h + 2 * k], w[4 * h + 2 * k + 1]),
+                                             make_float2(ms[2 * k], ms[2 * k + 1]));
+                x[4 * h + 2 * k] = xj.x;
+                x[4 * h + 2 * k + 1] = xj.y;
+                msv[4 * h + 2 * k] = ms[2 * k];
+                msv[4 * h + 2 * k + 1] = ms[2 * k + 1];
+                if (h == 0 || two) {
+                    acc = __fmaf_rn(xj.x, xj.x, acc);
+                    acc = __fmaf_rn(xj.y, xj.y, acc);
+                }
             }
         }
         store_vals<kW32>(d.X, b0, two, x);
@@ -299,28 +307,32 @@ __global__ void __launch_bounds__(kThreads) bwd_adam_kernel(const __grid_constan
         const int64_t b0 = ((t - d.work_begin) * kThreads + threadIdx.x) * 2;
         if (b0 >= d.nblocks) continue;
         const bool two = b0 + 1 < d.nblocks;
-        float w[8], gw[8], pi[12], mo[12], vo[12];
+        float w[8], gw[8];
+        float2 pi[6], mo[6], vo[6], grad[6];
         load_vals<kW32>(d.W, b0, two, w);
         load_vals<kG32>(d.G, b0, two, gw);
-        load12(d.pi, b0, two, pi);
-        load12(d.m, b0, two, mo);
-        load12(d.v, b0, two, vo);
-        float grad[12];
+        load12x2(d.pi, b0, two, pi);
+        load12x2(d.m, b0, two, mo);
+        load12x2(d.v, b0, two, vo);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
-            noise6(sc, d.gid0 + b0 + h, L, g);
-            soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, r);
+            float2 g[3];
+            float e[6], r, ms[4], mc[4], P[4], Q[4];
+            noise6x2(sc, d.gid0 + b0 + h, L, g);
+            soft_index2(pi + 3 * h, g, sc.kappa, sc.c2, e, r);
             soft_mask(e, r, ms);
             soft_mask_comp(e, r, mc);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float wj = w[4 * h + j];
+            for (int k = 0; k < 2; ++k) {  // positions 2k, 2k+1
+                const float2 wj = make_float2(w[4 * h + 2 * k], w[4 * h + 2 * k + 1]);
+                const float2 gj = make_float2(gw[4 * h + 2 * k], gw[4 * h + 2 * k + 1]);
+                const float2 msj = make_float2(ms[2 * k], ms[2 * k + 1]);
+                const float2 mcj = make_float2(mc[2 * k], mc[2 * k + 1]);
                 // u_j = G_j W_j - 2 lambda W_j^2 M_j (G_j W_j is exact for bf16 inputs)
-                const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j],
-                                          __fmul_rn(gw[4 * h + j], wj));
-                P[j] = __fmul_rn(mc[j], u);
-                Q[j] = __fmul_rn(ms[j], u);
+                const float2 u = __ffma2_rn(__fmul2_rn(f2(-sc.two_lambda), __fmul2_rn(wj, wj)), msj, __fmul2_rn(gj, wj));
+                const float2 pp = __fmul2_rn(mcj, u), qq = __fmul2_rn(msj, u);
+                P[2 * k] = pp.x; P[2 * k + 1] = pp.y;
+                Q[2 * k] = qq.x; Q[2 * k + 1] = qq.y;
             }
             float D[6];
             D[0] = (P[0] + P[1]) - (Q[2] + Q[3]);
@@ -331,16 +343,16 @@ __global__ void __launch_bounds__(kThreads) bwd_adam_kernel(const __grid_constan
             D[5] = (P[2] + P[3]) - (Q[0] + Q[1]);
             const float cr = __fmul_rn(sc.kappa_over_tau, r);
 #pragma unroll
-            for (int i = 0; i < C; ++i) {
-                const float gi = __fmul_rn(__fmul_rn(cr, e[i]), D[i]);
-                grad[6 * h + i] = gi;
-                adamw(pi[6 * h + i], mo[6 * h + i], vo[6 * h + i], gi, sc);
+            for (int k = 0; k < 3; ++k) {
+                grad[3 * h + k] = __fmul2_rn(__fmul2_rn(f2(cr), make_float2(e[2 * k], e[2 * k + 1])),
+                                             make_float2(D[2 * k], D[2 * k + 1]));
+                adamw2(pi[3 * h + k], mo[3 * h + k], vo[3 * h + k], grad[3 * h + k], sc);
             }
         }
-        store12(d.pi, b0, two, pi);
-        store12(d.m, b0, two, mo);
-        store12(d.v, b0, two, vo);
-        if (d.grad) store12(d.grad, b0, two, grad);
+        store12x2(d.pi, b0, two, pi);
+        store12x2(d.m, b0, two, mo);
+        store12x2(d.v, b0, two, vo);
+        if (d.grad) store12x2(d.grad, b0, two, grad);
     }
 }
 

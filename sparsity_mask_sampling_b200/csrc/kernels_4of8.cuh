@@ -138,48 +138,87 @@ __device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) 
 
 // --------------------------------------------------------------------------- per-block math
 
+// The per-block math below runs on the paired fp32 instructions of sm_100 (__ffma2_rn,
+// __fmul2_rn, __fadd2_rn), two candidates or two positions per instruction; each component
+// rounds exactly as the scalar form and every sum keeps its order, so the results are
+// bit-identical to one-at-a-time evaluation. w2[k] holds candidates 2k and 2k+1.
+constexpr int C2 = C / 2;
+
 // Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates, and their maximum.
 __device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
-                                           const NlogCtx &L, float w[C]) {
+                                           const NlogCtx &L, float2 w2[C2]) {
     float mx = -INFINITY;
+    const float2 *pi2 = reinterpret_cast<const float2 *>(pi_row);  // rows are 280 B: 8-byte aligned
 #pragma unroll
     for (int gr = 0; gr < 12; ++gr) {
-        uint32_t f[6];
-        if (sc.noise_on) fields21(block_words(sc, gid, (uint32_t)gr), f);
+        uint32_t u[6];
+        if (sc.noise_on) fields21_unit(block_words(sc, gid, (uint32_t)gr), u);
 #pragma unroll
-        for (int k = 0; k < 6; ++k) {
-            const int c = 6 * gr + k;
+        for (int k = 0; k < 3; ++k) {
+            const int c = 6 * gr + 2 * k;
             if (c < C) {
-                const float g = sc.noise_on ? gumbel(f[k], L) : 0.f;
-                w[c] = __fmaf_rn(sc.kappa, pi_row[c], g);
-                mx = fmaxf(mx, w[c]);
+                const float2 g = sc.noise_on ? gumbel_unit2(u[2 * k], u[2 * k + 1], L) : make_float2(0.f, 0.f);
+                const float2 wc = __ffma2_rn(f2(sc.kappa), pi2[c / 2], g);
+                w2[c / 2] = wc;
+                mx = fmaxf(fmaxf(mx, wc.x), wc.y);
             }
         }
     }
     return mx;
 }
 
-// e_c = 2^((w_c - max) c2) in place; returns sum e; ms[j] = sum_{c: j in S_c} e_c and, when
-// kComp, mc[j] = sum_{c: j not in S_c} e_c.
+// Add e to the accumulators of the positions in the 8-bit set `bits` (acc2[p] holds
+// positions 2p, 2p+1): one paired add where both positions of a pair are in the set.
+template <uint32_t bits>
+__device__ __forceinline__ void add_to(float2 acc2[4], float e) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t b = (bits >> (2 * p)) & 3u;
+        if (b == 3u) acc2[p] = __fadd2_rn(acc2[p], f2(e));
+        else if (b == 1u) acc2[p].x = __fadd_rn(acc2[p].x, e);
+        else if (b == 2u) acc2[p].y = __fadd_rn(acc2[p].y, e);
+    }
+}
+
+// e_c = 2^((w_c - max) c2) in place; returns sum e; ms2 = sums over c with j in S_c and, when
+// kComp, mc2 = sums over c with j not in S_c (pairs of positions).
 template <bool kComp>
-__device__ __forceinline__ float soft_sums(float w[C], float mx, float c2, float ms[8], float mc[8]) {
+__device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, float2 ms2[4], float2 mc2[4]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { ms[j] = 0.f; mc[j] = 0.f; }
+    for (int p = 0; p < 4; ++p) { ms2[p] = make_float2(0.f, 0.f); mc2[p] = make_float2(0.f, 0.f); }
     float s = 0.f;
-    const float mc2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
-    static_for<0, C>([&](auto I) {
-        constexpr int c = decltype(I)::value;
-        constexpr uint32_t mk = cand_mask(c);
-        const float e = ex2_approx(__fmaf_rn(w[c], c2, -mc2));
-        w[c] = e;
-        s += e;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (mk & (1u << j)) ms[j] += e;
-            else if (kComp) mc[j] += e;
-        }
+    const float m2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
+    static_for<0, C2>([&](auto I) {
+        constexpr int k = decltype(I)::value;
+        const float2 a = __ffma2_rn(w2[k], f2(c2), f2(-m2));
+        const float e0 = ex2_approx(a.x), e1 = ex2_approx(a.y);
+        w2[k] = make_float2(e0, e1);
+        s += e0;
+        add_to<cand_mask(2 * k)>(ms2, e0);
+        if (kComp) add_to<(~cand_mask(2 * k)) & 0xFFu>(mc2, e0);
+        s += e1;
+        add_to<cand_mask(2 * k + 1)>(ms2, e1);
+        if (kComp) add_to<(~cand_mask(2 * k + 1)) & 0xFFu>(mc2, e1);
     });
     return s;
+}
+
+// AdamW, PyTorch step order, two elements (bit-identical to adamw on each).
+__device__ __forceinline__ void adamw2(float2 &p, float2 &m, float2 &v, float2 g, const StepScalars &s) {
+    const float2 pd = __fmul2_rn(p, f2(s.decay));
+    m = __ffma2_rn(f2(s.beta1), m, __fmul2_rn(f2(s.one_minus_beta1), g));
+    v = __ffma2_rn(f2(s.beta2), v, __fmul2_rn(f2(s.one_minus_beta2), __fmul2_rn(g, g)));
+    const float2 denom = __ffma2_rn(make_float2(sqrt_approx(v.x), sqrt_approx(v.y)), f2(s.inv_sqrt_bc2), f2(s.eps));
+    p = __ffma2_rn(f2(-s.step_size), make_float2(__fdividef(m.x, denom.x), __fdividef(m.y, denom.y)), pd);
+}
+__device__ __forceinline__ void adamw4(float4 &p, float4 &m, float4 &v, float4 g, const StepScalars &s) {
+    float2 pa = make_float2(p.x, p.y), pb = make_float2(p.z, p.w), ma = make_float2(m.x, m.y),
+           mb = make_float2(m.z, m.w), va = make_float2(v.x, v.y), vb = make_float2(v.z, v.w);
+    adamw2(pa, ma, va, make_float2(g.x, g.y), s);
+    adamw2(pb, mb, vb, make_float2(g.z, g.w), s);
+    p = make_float4(pa.x, pa.y, pb.x, pb.y);
+    m = make_float4(ma.x, ma.y, mb.x, mb.y);
+    v = make_float4(va.x, va.y, vb.x, vb.y);
 }
 
 // AdamW, PyTorch step order, one element.
@@ -196,30 +235,34 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
 // Q_j = M_j u_j, u_j = G_j W_j - 2 lambda W_j^2 M_j.
 __device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8], const float gw[8], uint64_t gid,
                                          const StepScalars &sc, const NlogCtx &L, float *grow) {
-    float w[C], ms[8], mc[8];
-    const float mx = perturbed(pi_row, gid, sc, L, w);
-    const float r = rcp_approx(soft_sums<true>(w, mx, sc.c2, ms, mc));
+    float2 w2[C2], ms2[4], mc2[4];
+    const float mx = perturbed(pi_row, gid, sc, L, w2);
+    const float r = rcp_approx(soft_sums<true>(w2, mx, sc.c2, ms2, mc2));
     float P[8], Q[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        ms[j] = __fmul_rn(ms[j], r);
-        mc[j] = __fmul_rn(mc[j], r);
-        const float wj = wt[j];
-        const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j], __fmul_rn(gw[j], wj));
-        P[j] = __fmul_rn(mc[j], u);
-        Q[j] = __fmul_rn(ms[j], u);
+    for (int p = 0; p < 4; ++p) {  // positions 2p, 2p+1
+        const float2 ms = __fmul2_rn(ms2[p], f2(r)), mc = __fmul2_rn(mc2[p], f2(r));
+        const float2 wj = make_float2(wt[2 * p], wt[2 * p + 1]), gj = make_float2(gw[2 * p], gw[2 * p + 1]);
+        // fma(-(2 lambda W^2), M, G W)
+        const float2 u = __ffma2_rn(__fmul2_rn(f2(-sc.two_lambda), __fmul2_rn(wj, wj)), ms, __fmul2_rn(gj, wj));
+        const float2 pp = __fmul2_rn(mc, u), qq = __fmul2_rn(ms, u);
+        P[2 * p] = pp.x; P[2 * p + 1] = pp.y;
+        Q[2 * p] = qq.x; Q[2 * p + 1] = qq.y;
     }
     const float cr = __fmul_rn(sc.kappa_over_tau, r);
-    static_for<0, C>([&](auto I) {
-        constexpr int c = decltype(I)::value;
-        constexpr uint32_t mk = cand_mask(c);
-        float kept = 0.f, pruned = 0.f;
+    float2 *grow2 = reinterpret_cast<float2 *>(grow);  // rows are 280 B: 8-byte aligned
+    static_for<0, C2>([&](auto I) {
+        constexpr int k = decltype(I)::value;
+        constexpr uint32_t mk0 = cand_mask(2 * k), mk1 = cand_mask(2 * k + 1);  // compile-time masks
+        float kept0 = 0.f, pruned0 = 0.f, kept1 = 0.f, pruned1 = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            if (mk & (1u << j)) kept += P[j];
-            else pruned += Q[j];
+            if (mk0 & (1u << j)) kept0 += P[j];
+            else pruned0 += Q[j];
+            if (mk1 & (1u << j)) kept1 += P[j];
+            else pruned1 += Q[j];
         }
-        grow[c] = __fmul_rn(__fmul_rn(cr, w[c]), kept - pruned);
+        grow2[k] = __fmul2_rn(__fmul2_rn(f2(cr), w2[k]), make_float2(kept0 - pruned0, kept1 - pruned1));
     });
 }
 
@@ -227,14 +270,17 @@ __device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8],
 // regulariser partial added to acc.
 __device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], uint64_t gid, const StepScalars &sc,
                                         const NlogCtx &L, float ms[8], float x[8], float &acc) {
-    float w[C], mc[8];
-    const float mx = perturbed(pi_row, gid, sc, L, w);
-    const float r = rcp_approx(soft_sums<false>(w, mx, sc.c2, ms, mc));
+    float2 w2[C2], ms2[4], mc2[4];
+    const float mx = perturbed(pi_row, gid, sc, L, w2);
+    const float r = rcp_approx(soft_sums<false>(w2, mx, sc.c2, ms2, mc2));
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        ms[j] = __fmul_rn(ms[j], r);
-        x[j] = __fmul_rn(wt[j], ms[j]);
-        acc = __fmaf_rn(x[j], x[j], acc);
+    for (int p = 0; p < 4; ++p) {
+        const float2 m = __fmul2_rn(ms2[p], f2(r));
+        const float2 xx = __fmul2_rn(make_float2(wt[2 * p], wt[2 * p + 1]), m);
+        ms[2 * p] = m.x; ms[2 * p + 1] = m.y;
+        x[2 * p] = xx.x; x[2 * p + 1] = xx.y;
+        acc = __fmaf_rn(xx.x, xx.x, acc);
+        acc = __fmaf_rn(xx.y, xx.y, acc);
     }
 }
 
@@ -264,10 +310,7 @@ __device__ __forceinline__ void adam_tile(float *s_pi, const float *s_gr, int n,
             if (i < n4) {
                 float4 p4 = reinterpret_cast<const float4 *>(s_pi)[i];
                 const float4 g4 = reinterpret_cast<const float4 *>(s_gr)[i];
-                adamw(p4.x, m4[u].x, v4[u].x, g4.x, sc);
-                adamw(p4.y, m4[u].y, v4[u].y, g4.y, sc);
-                adamw(p4.z, m4[u].z, v4[u].z, g4.z, sc);
-                adamw(p4.w, m4[u].w, v4[u].w, g4.w, sc);
+                adamw4(p4, m4[u], v4[u], g4, sc);
                 if (kKeep) reinterpret_cast<float4 *>(s_pi)[i] = p4;
                 __stcs(reinterpret_cast<float4 *>(pi) + i, p4);
                 __stcs(reinterpret_cast<float4 *>(mm) + i, m4[u]);
@@ -403,7 +446,7 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
 // forward runs, the next tile's logits land in the buffer its gradients used, and its m, v
 // are fetched into L2 at the start of the tile, ahead of the AdamW pass.
 template <bool kW32, bool kG32>
-__global__ void __launch_bounds__(kCtaThreads) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
+__global__ void __launch_bounds__(kCtaThreads, 2) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
                                                                    const StepScalars sb, const StepScalars sf,
                                                                    double *partials, unsigned int *ticket,
                                                                    double *reg_out, int accumulate) {
