@@ -140,21 +140,27 @@ __device__ __forceinline__ void gen_stage(unsigned char *tile, const Op &d, int6
         uint4 packed = make_uint4(0u, 0u, 0u, 0u);
         if (row < d.rows) {
             const int64_t b0 = row * bpr + ((j * kChunk + 8 * c) >> 2);  // even: a pair of blocks
-            float w[8], pi[12], x[8], msv[8];
+            float w[8], x[8], msv[8];
+            float2 pi[6];
             k24::load_vals<false>(d.W, b0, true, w);
-            k24::load12(d.pi, b0, true, pi);
+            k24::load12x2(d.pi, b0, true, pi);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                float g[6], e[6], rr, ms[4];
-                k24::noise6(sc, d.gid0 + b0 + h, L, g);
-                k24::soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, rr);
+                float2 g[3];
+                float e[6], rr, ms[4];
+                k24::noise6x2(sc, d.gid0 + b0 + h, L, g);
+                k24::soft_index2(pi + 3 * h, g, sc.kappa, sc.c2, e, rr);
                 k24::soft_mask(e, rr, ms);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float xq = __fmul_rn(w[4 * h + q], ms[q]);
-                    x[4 * h + q] = xq;
+                for (int q = 0; q < 4; q += 2) {
+                    const float2 xq = __fmul2_rn(make_float2(w[4 * h + q], w[4 * h + q + 1]),
+                                                 make_float2(ms[q], ms[q + 1]));
+                    x[4 * h + q] = xq.x;
+                    x[4 * h + q + 1] = xq.y;
                     msv[4 * h + q] = ms[q];
-                    acc = __fmaf_rn(xq, xq, acc);
+                    msv[4 * h + q + 1] = ms[q + 1];
+                    acc = __fmaf_rn(xq.x, xq.x, acc);
+                    acc = __fmaf_rn(xq.y, xq.y, acc);
                 }
             }
             packed = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
@@ -473,26 +479,32 @@ __device__ __forceinline__ void bwd_decode(const BwdGroup &g, int64_t t, int &op
 // pair's eight entries of G (fp32) from gp: the arithmetic of k24::bwd_adam_kernel.
 __device__ __forceinline__ void pair_bwd_adam(const Op &d, int64_t b0, const float *gp, const StepScalars &sc,
                                               const NlogCtx &L) {
-    float w[8], gw[8], pi[12], mo[12], vo[12], grad[12];
+    float w[8], gw[8];
+    float2 pi[6], mo[6], vo[6], grad[6];
     k24::load_vals<false>(d.W, b0, true, w);
     const float4 g0 = *reinterpret_cast<const float4 *>(gp), g1 = *reinterpret_cast<const float4 *>(gp + 4);
     gw[0] = g0.x; gw[1] = g0.y; gw[2] = g0.z; gw[3] = g0.w; gw[4] = g1.x; gw[5] = g1.y; gw[6] = g1.z; gw[7] = g1.w;
-    k24::load12(d.pi, b0, true, pi);
-    k24::load12(d.m, b0, true, mo);
-    k24::load12(d.v, b0, true, vo);
+    k24::load12x2(d.pi, b0, true, pi);
+    k24::load12x2(d.m, b0, true, mo);
+    k24::load12x2(d.v, b0, true, vo);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        float g[6], e[6], r, ms[4], mc[4], P[4], Q[4];
-        k24::noise6(sc, d.gid0 + b0 + h, L, g);
-        k24::soft_index(pi + 6 * h, g, sc.kappa, sc.c2, e, r);
+        float2 g[3];
+        float e[6], r, ms[4], mc[4], P[4], Q[4];
+        k24::noise6x2(sc, d.gid0 + b0 + h, L, g);
+        k24::soft_index2(pi + 3 * h, g, sc.kappa, sc.c2, e, r);
         k24::soft_mask(e, r, ms);
         k24::soft_mask_comp(e, r, mc);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float wj = w[4 * h + j];
-            const float u = __fmaf_rn(-__fmul_rn(sc.two_lambda, __fmul_rn(wj, wj)), ms[j], __fmul_rn(gw[4 * h + j], wj));
-            P[j] = __fmul_rn(mc[j], u);
-            Q[j] = __fmul_rn(ms[j], u);
+        for (int k = 0; k < 2; ++k) {  // positions 2k, 2k+1
+            const float2 wj = make_float2(w[4 * h + 2 * k], w[4 * h + 2 * k + 1]);
+            const float2 gj = make_float2(gw[4 * h + 2 * k], gw[4 * h + 2 * k + 1]);
+            const float2 msj = make_float2(ms[2 * k], ms[2 * k + 1]);
+            const float2 mcj = make_float2(mc[2 * k], mc[2 * k + 1]);
+            const float2 u = __ffma2_rn(__fmul2_rn(f2(-sc.two_lambda), __fmul2_rn(wj, wj)), msj, __fmul2_rn(gj, wj));
+            const float2 pp = __fmul2_rn(mcj, u), qq = __fmul2_rn(msj, u);
+            P[2 * k] = pp.x; P[2 * k + 1] = pp.y;
+            Q[2 * k] = qq.x; Q[2 * k + 1] = qq.y;
         }
         float D[6];
         D[0] = (P[0] + P[1]) - (Q[2] + Q[3]);
@@ -503,16 +515,16 @@ __device__ __forceinline__ void pair_bwd_adam(const Op &d, int64_t b0, const flo
         D[5] = (P[2] + P[3]) - (Q[0] + Q[1]);
         const float cr = __fmul_rn(sc.kappa_over_tau, r);
 #pragma unroll
-        for (int i = 0; i < 6; ++i) {
-            const float gi = __fmul_rn(__fmul_rn(cr, e[i]), D[i]);
-            grad[6 * h + i] = gi;
-            k24::adamw(pi[6 * h + i], mo[6 * h + i], vo[6 * h + i], gi, sc);
+        for (int k = 0; k < 3; ++k) {
+            grad[3 * h + k] = __fmul2_rn(__fmul2_rn(f2(cr), make_float2(e[2 * k], e[2 * k + 1])),
+                                         make_float2(D[2 * k], D[2 * k + 1]));
+            k24::adamw2(pi[3 * h + k], mo[3 * h + k], vo[3 * h + k], grad[3 * h + k], sc);
         }
     }
-    k24::store12(d.pi, b0, true, pi);
-    k24::store12(d.m, b0, true, mo);
-    k24::store12(d.v, b0, true, vo);
-    if (d.grad) k24::store12(d.grad, b0, true, grad);
+    k24::store12x2(d.pi, b0, true, pi);
+    k24::store12x2(d.m, b0, true, mo);
+    k24::store12x2(d.v, b0, true, vo);
+    if (d.grad) k24::store12x2(d.grad, b0, true, grad);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) masked_linear_bwd_adam_kernel(const __grid_constant__ BwdGroup grp,
