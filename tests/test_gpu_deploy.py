@@ -359,7 +359,7 @@ def test_side_streams_and_concurrent_host_threads(orc, tokens):
 # ------------------------------------------------------------------------------ prefill sizes
 
 @pytest.mark.parametrize("nm", [(2, 4), (4, 8)])
-@pytest.mark.parametrize("tokens", [65, 128, 200, 512])
+@pytest.mark.parametrize("tokens", [65, 128, 200, 300, 512])
 def test_prefill_sized_calls(orc, ws, nm, tokens):
     """More than 64 tokens: operands whose columns are whole 128-column stages run on the
     prefill kernels (2:4: units of two 128-row tiles x 128 tokens; 4:8: 128 rows x 256
