@@ -671,7 +671,7 @@ def config_leg(w, dev, peak, reps=10):
     return res
 
 
-def masked_linear_leg(dev, peak, tokens=256, reps=10):
+def masked_linear_leg(dev, peak, tokens=256, reps=10, bwd_tokens=2048):
     """The sampler inside the frozen network's linear layers (s.3.2 "Frozen LLM Backbone"), on
     the LLaMA-2-7B layer's seven matrices at `tokens` tokens (seeded synthetic activations A
     and output gradients dY, bf16). Fused: mllm_masked_linear_fwd (Y = A X^T with X made in
@@ -748,6 +748,28 @@ def masked_linear_leg(dev, peak, tokens=256, reps=10):
         res[k] = round(v, 4)
     res["fwd_speedup"] = round(t["unfused_fwd_ms"] / t["fused_fwd_ms"], 3)
     res["bwd_adam_speedup"] = round(t["unfused_bwd_adam_ms"] / t["fused_bwd_adam_ms"], 3)
+    # The backward sums over the tokens (its MMA's K), so one call takes a whole sequence:
+    # the same two backward plans at bwd_tokens tokens.
+    if bwd_tokens and bwd_tokens != tokens:
+        ios_l, As_l, dYs_l = [], [], []
+        for i, m in enumerate(w.matrices):
+            A = inputs.weights(bwd_tokens, m.cols, "bf16", 1.0, seed=500 + i, device=dev)
+            dY = inputs.upstream_grad(bwd_tokens, m.rows, "bf16", 1e-3, seed=600 + i, device=dev)
+            ios_l.append((A, None, dY))
+            As_l.append(A)
+            dYs_l.append(dY)
+
+        def unfused_bwd_l():
+            for mb, A, dY in zip(mats, As_l, dYs_l):
+                torch.matmul(dY.t(), A, out=mb.G)
+            pkg.mllm_sample_bwd_adam(arr, (2, 4), hp)
+
+        fb = timed(lambda: pkg.mllm_masked_linear_bwd_adam(farr, ios_l, (2, 4), bwd_tokens, hp, mlws))
+        ub = timed(unfused_bwd_l)
+        res["bwd_tokens"] = bwd_tokens
+        res["fused_bwd_adam_ms_at_bwd_tokens"] = round(fb, 4)
+        res["unfused_bwd_adam_ms_at_bwd_tokens"] = round(ub, 4)
+        res["bwd_adam_speedup_at_bwd_tokens"] = round(ub / fb, 3)
     # HBM bytes per block and step. Fused: forward reads W + logits (32), backward reads W and
     # logits/m/v and writes logits/m/v (152). Unfused as timed here: sampler forward 40 + the
     # GEMM's read of X 8, the GEMM's write of G 8 + sampler backward 160. (A loop built on the

@@ -239,7 +239,9 @@ mllm_status mllm_masked_linear_fwd(const mllm_matrix *mats, const mllm_linear_io
  * regulariser's term, AdamW on logits, adam_m, adam_v in place (grad_logits_out receives dpi
  * when non-NULL). G is formed tile by tile in tensor and shared memory and never written to
  * global memory. io[i].x and io[i].dy are the forward's activations and dL/dY; 1 <= tokens
- * <= 256; W bf16, cols % 64 == 0, rows % 8 == 0, 2:4 only (MLLM_ERR_UNSUPPORTED otherwise).
+ * <= 1048576 (the tokens are the products' summation index, run in stages of 64 tokens, so a
+ * whole batch's tokens can go in one call); W bf16, cols % 64 == 0, rows % 8 == 0, 2:4 only
+ * (MLLM_ERR_UNSUPPORTED otherwise).
  * workspace as for mllm_masked_linear_fwd (only its error word is used here). Reads W, x, dy. */
 mllm_status mllm_masked_linear_bwd_adam(const mllm_matrix *mats, const mllm_linear_io *io, int32_t n_mats,
                                         mllm_nm nm, int32_t tokens, const mllm_hparams *hp, void *workspace,

@@ -62,7 +62,8 @@ constexpr int kProdWarps = 16;      // producer / epilogue warps
 constexpr int kProd = 32 * kProdWarps;
 constexpr int kThreads = kProd + 64;  // + the copy warp and the MMA warp
 constexpr int kStages = 3;
-constexpr int kMaxTokens = 256;     // one MMA's N
+constexpr int kMaxTokens = 256;     // one MMA's N (the forward)
+constexpr int kMaxBwdTokens = 1 << 20;  // the backward's K: tokens in 64-token stages
 constexpr int kMaxCtas = 160;       // grid cap (one CTA per SM); sizes the partial-tile workspace
 
 template <int kN> constexpr int xbox_bytes() { return kN * 128; }

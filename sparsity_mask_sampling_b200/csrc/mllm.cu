@@ -704,7 +704,8 @@ mllm_status validate_mlin(const mllm_matrix *mats, const mllm_linear_io *io, int
     mllm_status s = validate_mats(mats, n_mats, nm, need);
     if (s != MLLM_OK) return s;
     if (nm.m != 4) return MLLM_ERR_UNSUPPORTED;
-    if (!io || tokens < 1 || tokens > mlin::kMaxTokens) return MLLM_ERR_INVALID_ARG;
+    // the forward's tokens are one MMA's N; the backward's are the MMA's K, in 64-token stages
+    if (!io || tokens < 1 || tokens > (fwd ? mlin::kMaxTokens : mlin::kMaxBwdTokens)) return MLLM_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_mats; ++i) {
         const mllm_matrix &a = mats[i];
         if (a.w_dtype != MLLM_BF16) return MLLM_ERR_UNSUPPORTED;

@@ -243,7 +243,7 @@ def test_masked_linear_validation(M):
         assert _mlin(M, [mat], [io], nm=(4, 8), bwd=bwd) == M.MLLM_ERR_UNSUPPORTED
         assert _mlin(M, [_mat(M, rows=128, cols=128, w_dtype=1)], [io], bwd=bwd) == M.MLLM_ERR_UNSUPPORTED
         assert _mlin(M, [_mat(M, rows=128, cols=96)], [io], bwd=bwd) == M.MLLM_ERR_UNSUPPORTED
-        for tokens in (0, -1, 257):
+        for tokens in (0, -1, 1048577 if bwd else 257):
             assert _mlin(M, [mat], [io], tokens=tokens, bwd=bwd) == M.MLLM_ERR_INVALID_ARG, tokens
         assert _mlin(M, [mat], [M.LinearIO(x=0, y=0xB000, dy=0xC000)], bwd=bwd) == M.MLLM_ERR_INVALID_ARG
         assert _mlin(M, [mat], [M.LinearIO(x=0xA008, y=0xB000, dy=0xC000)], bwd=bwd) == M.MLLM_ERR_MISALIGNED

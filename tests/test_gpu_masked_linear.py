@@ -146,7 +146,12 @@ def _bwd_check(orc, mb, A, dY, hp, pi0, m0, v0, rows_idx=None):
     f = orc.sample_fwd(2, 4, Wv.reshape(-1, 4), pi, gids, hp.kappa, hp.tau, hp.seed, hp.step)
     S = orc.candidates(2, 4).astype(np.float64)
     wdg = (np.abs(Wv) * dG).reshape(-1, 4)
-    prop = (hp.kappa / hp.tau) * f["y"] * (np.abs(S[None, :, :] - f["msoft"][:, None, :]) * wdg[:, None, :]).sum(-1)
+    # |d dpi_i / d u_j| / ((kappa/tau) y_i): the complement 1 - M_j for j in S_i, taken as the
+    # oracle's sum of the soft-index weights of the candidates without j (1 - M_j in floating
+    # point is 0 once M_j is within 2^-53 of 1, while that sum still carries the sensitivity),
+    # and M_j otherwise
+    sens = S[None, :, :] * f["mcomp"][:, None, :] + (1.0 - S[None, :, :]) * f["msoft"][:, None, :]
+    prop = (hp.kappa / hp.tau) * f["y"] * (sens * wdg[:, None, :]).sum(-1)
     floor = _tol.grad_floor(Wv.reshape(-1, 4), G.reshape(-1, 4), hp.kappa, hp.tau, hp.lambda_)
     g_tol = 1e-4 * scale + prop + floor
     g_gpu = mb.grad_logits.view(r_all, c // 4, 6)[rt].cpu().numpy().reshape(-1, 6)
@@ -184,10 +189,11 @@ def _bwd_layer(shapes, tokens, seed, outliers=0.0):
     return mats, ios, As, dYs, state
 
 
-@pytest.mark.parametrize("tokens", [1, 40, 64, 100, 256])
+@pytest.mark.parametrize("tokens", [1, 40, 64, 100, 256, 300, 1000])
 def test_masked_linear_backward_adam_parity(orc, mlws, tokens):
     """Ragged tiles in both directions (200 rows, 192 = 1.5 column tiles), grouped matrices,
-    token counts below, at and between the 64-token stages."""
+    token counts below, at and between the 64-token stages, and past the forward's 256 (the
+    backward sums over the tokens in stages)."""
     shapes = [(256, 128), (200, 192), (64, 64)]
     mats, ios, As, dYs, state = _bwd_layer(shapes, tokens, seed=700 + tokens)
     hp = Hparams(kappa=250.0, tau=0.6, lambda_=1e-5, lr=5e-4, adam_step=3, step=2, seed=0xB0B)
@@ -198,15 +204,17 @@ def test_masked_linear_backward_adam_parity(orc, mlws, tokens):
     assert mlws[-16:].view(torch.int32)[0].item() == 0  # error word
 
 
-def test_masked_linear_backward_adam_llama2_7b_layer(orc, mlws):
-    """The LLaMA-2-7B layer's seven matrices at 256 tokens in one call (12,352 tiles of
-    128 x 128 over the persistent grid); sampled rows checked."""
+@pytest.mark.parametrize("tokens", [256, 2048])
+def test_masked_linear_backward_adam_llama2_7b_layer(orc, mlws, tokens):
+    """The LLaMA-2-7B layer's seven matrices in one call (12,352 tiles of 128 x 128 over the
+    persistent grid), at 256 tokens and at 2048 (past the forward's limit: the backward sums
+    over the tokens in stages); sampled rows checked."""
     from sparsity_mask_sampling_b200 import configs
 
     w = configs.WORKLOADS["llama2_7b_layer_2of4"]
-    mats, ios, As, dYs, state = _bwd_layer([(m.rows, m.cols) for m in w.matrices], 256, seed=900, outliers=0.01)
+    mats, ios, As, dYs, state = _bwd_layer([(m.rows, m.cols) for m in w.matrices], tokens, seed=900, outliers=0.01)
     hp = Hparams(kappa=480.0, tau=0.1, lambda_=1e-5, lr=5e-4, adam_step=40, step=39, seed=5)
-    mllm_masked_linear_bwd_adam(mats, ios, (2, 4), 256, hp, mlws)
+    mllm_masked_linear_bwd_adam(mats, ios, (2, 4), tokens, hp, mlws)
     torch.cuda.synchronize()
     rng = np.random.default_rng(1)
     for mb, A, dY, (pi, m0, v0) in zip(mats, As, dYs, state):
