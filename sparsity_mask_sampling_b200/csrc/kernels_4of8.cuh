@@ -22,8 +22,14 @@ constexpr int C = 70;
 constexpr int kCtaThreads = 128;
 constexpr int kBlocksPerCta = kCtaThreads;  // one block per thread
 constexpr int kTileFloats = kBlocksPerCta * C;
-constexpr int kFwdDynSmem = kTileFloats * (int)sizeof(float);
+// The forward's CTA is two independent 128-thread halves that share one logarithm table:
+// each half stages and computes its own tiles and meets only on its own named barrier, so an
+// SM holds 16 warps (two such CTAs) where 128-thread CTAs, each with its own table, fit 12.
+constexpr int kFwdHalves = 2;
+constexpr int kFwdThreads = kFwdHalves * kCtaThreads;
+constexpr int kFwdDynSmem = kFwdHalves * kTileFloats * (int)sizeof(float);
 constexpr int kBwdDynSmem = 2 * kTileFloats * (int)sizeof(float);
+constexpr int kStepDynSmem = kTileFloats * (int)sizeof(float);  // the one-launch step: one tile buffer
 
 // Keep mask (bit j = position j) of candidate i: the i-th 4-subset of {0..7} in
 // lexicographic order of ascending index tuples. Only ever evaluated at compile time.
@@ -70,30 +76,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
-__device__ __forceinline__ void stage_in(float *dst, const float *src, int n) {
+// lt: the thread's index among the kCtaThreads threads that share the tile.
+__device__ __forceinline__ void stage_in(float *dst, const float *src, int n, int lt = threadIdx.x) {
     const int n4 = n >> 2;  // whole 16-byte chunks
-    for (int i = threadIdx.x; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
-    if ((n & 3) && threadIdx.x == 0) {  // n = nb*70 is even: at most one 8-byte tail
+    for (int i = lt; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
+    if ((n & 3) && lt == 0) {  // n = nb*70 is even: at most one 8-byte tail
         *reinterpret_cast<float2 *>(dst + 4 * n4) = __ldcs(reinterpret_cast<const float2 *>(src + 4 * n4));
     }
     cp_async_wait_all();
-}
-
-// The same copies without the wait: the tile lands while the CTA works on something else;
-// the caller waits (cp_async_wait_pending) and synchronises the CTA before reading it. The 8-byte
-// tail of an odd block count goes through an 8-byte cp.async.
-__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
-    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void stage_in_async(float *dst, const float *src, int n) {
-    const int n4 = n >> 2;
-    for (int i = threadIdx.x; i < n4; i += kCtaThreads) cp_async16(dst + 4 * i, src + 4 * i);
-    if ((n & 3) && threadIdx.x == 0) cp_async8(dst + 4 * n4, src + 4 * n4);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_pending() {
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void stage_out(float *dst, const float *src, int n) {
@@ -167,40 +157,108 @@ __device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, co
     return mx;
 }
 
-// Add e to the accumulators of the positions in the 8-bit set `bits` (acc2[p] holds
-// positions 2p, 2p+1): one paired add where both positions of a pair are in the set.
-template <uint32_t bits>
-__device__ __forceinline__ void add_to(float2 acc2[4], float e) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const uint32_t b = (bits >> (2 * p)) & 3u;
-        if (b == 3u) acc2[p] = __fadd2_rn(acc2[p], f2(e));
-        else if (b == 1u) acc2[p].x = __fadd_rn(acc2[p].x, e);
-        else if (b == 2u) acc2[p].y = __fadd_rn(acc2[p].y, e);
-    }
+// Sums over candidates, formed per half of the block. A candidate's four kept positions are
+// a subset of positions 0-3 (its low half) and a subset of positions 4-7 (its high half);
+// each of the 16 subsets of a half occurs among the 70 candidates. In the forward each e_c
+// goes into one of 16 buckets by its low half and one of 16 by its high half; the sum over
+// the candidates that keep position j (or prune it) is the sum of the 8 buckets of j's half
+// whose subset holds j (or lacks it). In the backward a candidate's
+// sum_{j kept} P_j - sum_{j pruned} Q_j is D_lo[low half] + D_hi[high half], where
+// D[s] = sum_{j in s} P_j - sum_{j in the half, not in s} Q_j is formed once per subset. The
+// terms are those of Eq.7 and its derivative; only the association of the fp32 additions
+// differs from sums taken in candidate order.
+__host__ __device__ constexpr uint32_t lo4(int c) { return cand_mask(c) & 0xFu; }
+__host__ __device__ constexpr uint32_t hi4(int c) { return cand_mask(c) >> 4; }
+__host__ __device__ constexpr bool first_lo(int c) {
+    for (int k = 0; k < c; ++k)
+        if (lo4(k) == lo4(c)) return false;
+    return true;
+}
+__host__ __device__ constexpr bool first_hi(int c) {
+    for (int k = 0; k < c; ++k)
+        if (hi4(k) == hi4(c)) return false;
+    return true;
+}
+__host__ __device__ constexpr int top_bit(int s) {
+    int b = -1;
+    for (; s; s >>= 1) ++b;
+    return b;
+}
+
+// Sum of the buckets B[s] whose subset s holds bit kBit (kHas) or lacks it, in ascending s.
+template <int kBit, bool kHas>
+__device__ __forceinline__ float bucket_sum(const float B[16]) {
+    constexpr int s0 = kHas ? (1 << kBit) : 0;  // the smallest such subset
+    float acc = B[s0];
+    static_for<s0 + 1, 16>([&](auto I) {
+        constexpr int s = decltype(I)::value;
+        if constexpr (((s >> kBit) & 1) == (kHas ? 1 : 0)) acc = __fadd_rn(acc, B[s]);
+    });
+    return acc;
 }
 
 // e_c = 2^((w_c - max) c2) in place; returns sum e; ms2 = sums over c with j in S_c and, when
-// kComp, mc2 = sums over c with j not in S_c (pairs of positions).
+// kComp, mc2 = sums over c with j not in S_c (pairs of positions 2p, 2p+1).
 template <bool kComp>
 __device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, float2 ms2[4], float2 mc2[4]) {
-#pragma unroll
-    for (int p = 0; p < 4; ++p) { ms2[p] = make_float2(0.f, 0.f); mc2[p] = make_float2(0.f, 0.f); }
-    float s = 0.f;
+    float BL[16], BH[16];  // buckets by low-half and by high-half subset
     const float m2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
+    auto put = [&](auto I, float e) {
+        constexpr int c = decltype(I)::value;
+        if constexpr (first_lo(c)) BL[lo4(c)] = e;
+        else BL[lo4(c)] = __fadd_rn(BL[lo4(c)], e);
+        if constexpr (first_hi(c)) BH[hi4(c)] = e;
+        else BH[hi4(c)] = __fadd_rn(BH[hi4(c)], e);
+    };
     static_for<0, C2>([&](auto I) {
         constexpr int k = decltype(I)::value;
         const float2 a = __ffma2_rn(w2[k], f2(c2), f2(-m2));
         const float e0 = ex2_approx(a.x), e1 = ex2_approx(a.y);
         w2[k] = make_float2(e0, e1);
-        s += e0;
-        add_to<cand_mask(2 * k)>(ms2, e0);
-        if (kComp) add_to<(~cand_mask(2 * k)) & 0xFFu>(mc2, e0);
-        s += e1;
-        add_to<cand_mask(2 * k + 1)>(ms2, e1);
-        if (kComp) add_to<(~cand_mask(2 * k + 1)) & 0xFFu>(mc2, e1);
+        put(std::integral_constant<int, 2 * k>{}, e0);
+        put(std::integral_constant<int, 2 * k + 1>{}, e1);
     });
-    return s;
+    ms2[0] = make_float2(bucket_sum<0, true>(BL), bucket_sum<1, true>(BL));
+    ms2[1] = make_float2(bucket_sum<2, true>(BL), bucket_sum<3, true>(BL));
+    ms2[2] = make_float2(bucket_sum<0, true>(BH), bucket_sum<1, true>(BH));
+    ms2[3] = make_float2(bucket_sum<2, true>(BH), bucket_sum<3, true>(BH));
+    if (kComp) {
+        mc2[0] = make_float2(bucket_sum<0, false>(BL), bucket_sum<1, false>(BL));
+        mc2[1] = make_float2(bucket_sum<2, false>(BL), bucket_sum<3, false>(BL));
+        mc2[2] = make_float2(bucket_sum<0, false>(BH), bucket_sum<1, false>(BH));
+        mc2[3] = make_float2(bucket_sum<2, false>(BH), bucket_sum<3, false>(BH));
+    }
+    // sum e: every candidate sits in exactly one low-half bucket (a pairwise tree over them)
+    float t8[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t8[q] = __fadd_rn(BL[2 * q], BL[2 * q + 1]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) t8[q] = __fadd_rn(t8[2 * q], t8[2 * q + 1]);
+    return __fadd_rn(__fadd_rn(t8[0], t8[1]), __fadd_rn(t8[2], t8[3]));
+}
+
+// D[s] = sum_{j in s} P_j - sum_{j in the half, not in s} Q_j for the 16 subsets s of the
+// half kBase..kBase+3 (subset sums in ascending position order).
+template <int kBase>
+__device__ __forceinline__ void half_diffs(const float P[8], const float Q[8], float D[16]) {
+    float SP[16], SQ[16];
+    static_for<1, 16>([&](auto I) {
+        constexpr int s = decltype(I)::value;
+        constexpr int hb = top_bit(s), rest = s & ~(1 << hb);
+        if constexpr (rest == 0) {
+            SP[s] = P[kBase + hb];
+            SQ[s] = Q[kBase + hb];
+        } else {
+            SP[s] = __fadd_rn(SP[rest], P[kBase + hb]);
+            SQ[s] = __fadd_rn(SQ[rest], Q[kBase + hb]);
+        }
+    });
+    D[0] = -SQ[15];
+    D[15] = SP[15];
+    static_for<1, 15>([&](auto I) {
+        constexpr int s = decltype(I)::value;
+        D[s] = __fsub_rn(SP[s], SQ[15 ^ s]);
+    });
 }
 
 // AdamW, PyTorch step order, two elements (bit-identical to adamw on each).
@@ -249,20 +307,16 @@ __device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8],
         P[2 * p] = pp.x; P[2 * p + 1] = pp.y;
         Q[2 * p] = qq.x; Q[2 * p + 1] = qq.y;
     }
+    float DL[16], DH[16];
+    half_diffs<0>(P, Q, DL);
+    half_diffs<4>(P, Q, DH);
     const float cr = __fmul_rn(sc.kappa_over_tau, r);
     float2 *grow2 = reinterpret_cast<float2 *>(grow);  // rows are 280 B: 8-byte aligned
     static_for<0, C2>([&](auto I) {
         constexpr int k = decltype(I)::value;
-        constexpr uint32_t mk0 = cand_mask(2 * k), mk1 = cand_mask(2 * k + 1);  // compile-time masks
-        float kept0 = 0.f, pruned0 = 0.f, kept1 = 0.f, pruned1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (mk0 & (1u << j)) kept0 += P[j];
-            else pruned0 += Q[j];
-            if (mk1 & (1u << j)) kept1 += P[j];
-            else pruned1 += Q[j];
-        }
-        grow2[k] = __fmul2_rn(__fmul2_rn(f2(cr), w2[k]), make_float2(kept0 - pruned0, kept1 - pruned1));
+        const float d0 = __fadd_rn(DL[lo4(2 * k)], DH[hi4(2 * k)]);
+        const float d1 = __fadd_rn(DL[lo4(2 * k + 1)], DH[hi4(2 * k + 1)]);
+        grow2[k] = __fmul2_rn(__fmul2_rn(f2(cr), w2[k]), make_float2(d0, d1));
     });
 }
 
@@ -330,11 +384,59 @@ __device__ __forceinline__ void adam_tile(float *s_pi, const float *s_gr, int n,
     }
 }
 
+// AdamW over a tile whose gradients sit in s_buf (flat, coalesced float4s): the logits are
+// read again from global memory (staged from there at the start of the tile, so they are
+// still in L2), m and v from global memory (prefetched into L2); the updated logits overwrite
+// the gradients in s_buf and are stored with m, v (and the gradient when gout). Each float4
+// is read and rewritten by the same thread, so the update in place needs no barrier.
+__device__ __forceinline__ void adam_tile_inplace(float *s_buf, int n, float *__restrict__ pi,
+                                                  float *__restrict__ mm, float *__restrict__ vv,
+                                                  float *__restrict__ gout, const StepScalars &sc) {
+    const int n4 = n >> 2;
+    constexpr int kUnroll = 4;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += kCtaThreads * kUnroll) {
+        float4 p4[kUnroll], m4[kUnroll], v4[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kCtaThreads;
+            if (i < n4) {
+                p4[u] = __ldcg(reinterpret_cast<const float4 *>(pi) + i);
+                m4[u] = __ldcs(reinterpret_cast<const float4 *>(mm) + i);
+                v4[u] = __ldcs(reinterpret_cast<const float4 *>(vv) + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int i = i0 + u * kCtaThreads;
+            if (i < n4) {
+                const float4 g4 = reinterpret_cast<const float4 *>(s_buf)[i];
+                adamw4(p4[u], m4[u], v4[u], g4, sc);
+                reinterpret_cast<float4 *>(s_buf)[i] = p4[u];
+                __stcs(reinterpret_cast<float4 *>(pi) + i, p4[u]);
+                __stcs(reinterpret_cast<float4 *>(mm) + i, m4[u]);
+                __stcs(reinterpret_cast<float4 *>(vv) + i, v4[u]);
+                if (gout) __stcs(reinterpret_cast<float4 *>(gout) + i, g4);
+            }
+        }
+    }
+    if ((n & 3) && threadIdx.x == 0) {  // 2-float tail of a tile with an odd block count
+        for (int i = 4 * n4; i < n; ++i) {
+            const float g = s_buf[i];
+            float p = __ldcg(pi + i), m = mm[i], v = vv[i];
+            adamw(p, m, v, g, sc);
+            s_buf[i] = p;
+            pi[i] = p; mm[i] = m; vv[i] = v;
+            if (gout) gout[i] = g;
+        }
+    }
+}
+
 // CTA-level deterministic reduction of the regulariser partials, then the last CTA (ticket)
-// combines all per-CTA partials in index order and resets the ticket.
+// combines all per-CTA partials in index order and resets the ticket. kThr: the CTA's threads.
+template <int kThr = kCtaThreads>
 __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned int *ticket, double *reg_out,
                                            int accumulate) {
-    __shared__ double s_w[kCtaThreads / 32];
+    __shared__ double s_w[kThr / 32];
     __shared__ bool s_last;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
@@ -344,7 +446,7 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
     __syncthreads();
     if (threadIdx.x == 0) {
         double tt = 0.0;
-        for (int i = 0; i < kCtaThreads / 32; ++i) tt += s_w[i];
+        for (int i = 0; i < kThr / 32; ++i) tt += s_w[i];
         partials[blockIdx.x] = tt;
         __threadfence();
         s_last = (atomicAdd(ticket, 1u) == gridDim.x - 1);
@@ -353,7 +455,7 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
     if (!s_last) return;
     __threadfence();
     double tt = 0.0;
-    for (unsigned int i = threadIdx.x; i < gridDim.x; i += kCtaThreads) tt += __ldcg(partials + i);
+    for (unsigned int i = threadIdx.x; i < gridDim.x; i += kThr) tt += __ldcg(partials + i);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tt += __shfl_xor_sync(0xFFFFFFFFu, tt, o);
     __syncthreads();
@@ -361,7 +463,7 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
     __syncthreads();
     if (threadIdx.x == 0) {
         double tot = 0.0;
-        for (int i = 0; i < kCtaThreads / 32; ++i) tot += s_w[i];
+        for (int i = 0; i < kThr / 32; ++i) tot += s_w[i];
         *reg_out = accumulate ? (*reg_out + tot) : tot;
         *ticket = 0u;
     }
@@ -369,31 +471,39 @@ __device__ __forceinline__ void reduce_reg(float acc, double *partials, unsigned
 
 // --------------------------------------------------------------------------- kernels
 
+// Named barrier of half h (ids 1 and 2 as immediates; id 0 is the CTA-wide barrier).
+__device__ __forceinline__ void half_sync(int h) {
+    if (h) asm volatile("bar.sync 2, %0;" ::"n"(kCtaThreads) : "memory");
+    else asm volatile("bar.sync 1, %0;" ::"n"(kCtaThreads) : "memory");
+}
+
 template <bool kW32>
-__global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant__ Group grp,
+__global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const __grid_constant__ Group grp,
                                                           const StepScalars sc, double *partials,
                                                           unsigned int *ticket, double *reg_out,
                                                           int accumulate) {
     __shared__ __align__(16) float2 s_tab[kNlogEntries];
-    extern __shared__ __align__(16) float s_dyn[];  // [kTileFloats] logits of the tile
-    float *s_pi = s_dyn;
+    extern __shared__ __align__(16) float s_dyn[];  // [kFwdHalves][kTileFloats] logits of each half's tile
+    const int h = (int)threadIdx.x / kCtaThreads, lt = (int)threadIdx.x % kCtaThreads;
+    float *s_pi = s_dyn + h * kTileFloats;
     load_tab(s_tab);
+    __syncthreads();
     const NlogCtx L{s_tab};
     float acc = 0.f;
     int mi = 0;
-    for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
+    for (int64_t t = (int64_t)blockIdx.x * kFwdHalves + h; t < grp.total_work; t += (int64_t)gridDim.x * kFwdHalves) {
         mi = next_mat(grp, mi, t);
         const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
-        __syncthreads();  // previous tile's readers are done (and the table is loaded)
-        stage_in(s_pi, d.pi + tb0 * C, nb * C);
-        __syncthreads();
-        if ((int)threadIdx.x < nb) {
-            const int64_t b = tb0 + threadIdx.x;
+        half_sync(h);  // the half's previous tile's readers are done
+        stage_in(s_pi, d.pi + tb0 * C, nb * C, lt);
+        half_sync(h);
+        if (lt < nb) {
+            const int64_t b = tb0 + lt;
             float wt[8], ms[8], x[8];
             load8<kW32>(d.W, b, wt);
-            fwd_row(s_pi + threadIdx.x * C, wt, d.gid0 + b, sc, L, ms, x, acc);
+            fwd_row(s_pi + lt * C, wt, d.gid0 + b, sc, L, ms, x, acc);
             store8<kW32>(d.X, b, x);
             if (d.soft) {
                 float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
@@ -402,7 +512,7 @@ __global__ void __launch_bounds__(kCtaThreads) fwd_kernel(const __grid_constant_
             }
         }
     }
-    if (reg_out) reduce_reg(acc, partials, ticket, reg_out, accumulate);
+    if (reg_out) reduce_reg<kFwdThreads>(acc, partials, ticket, reg_out, accumulate);
 }
 
 template <bool kW32, bool kG32>
@@ -440,58 +550,57 @@ __global__ void __launch_bounds__(kCtaThreads) bwd_adam_kernel(const __grid_cons
 }
 
 // Backward + AdamW of step t fused with the forward of step t+1 (mllm_sample_bwd_adam_fwd):
-// per tile, the gradient of every block (noise of step t) into one buffer, the flat AdamW
-// pass (updated logits kept in shared memory), then the forward of step t+1 from the updated
-// logits. The tile's logits are read from HBM once. Two tile buffers alternate: while a tile's
-// forward runs, the next tile's logits land in the buffer its gradients used, and its m, v
-// are fetched into L2 at the start of the tile, ahead of the AdamW pass.
+// per tile, the gradient of every block (noise of step t) written over the block's logits in
+// the one tile buffer (each thread reads its whole row before it writes it), the flat AdamW
+// pass (updated logits back into the buffer), then the forward of step t+1 from the updated
+// logits. One 35.8 KB buffer per CTA lets three CTAs share an SM. The logits are read from
+// HBM once: the AdamW pass reads them again from L2, and each tile start asks L2 for the
+// tile's m and v and for the CTA's next tile of logits.
 template <bool kW32, bool kG32>
-__global__ void __launch_bounds__(kCtaThreads, 2) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
+__global__ void __launch_bounds__(kCtaThreads, 3) bwd_adam_fwd_kernel(const __grid_constant__ Group grp,
                                                                    const StepScalars sb, const StepScalars sf,
                                                                    double *partials, unsigned int *ticket,
                                                                    double *reg_out, int accumulate) {
     __shared__ __align__(16) float2 s_tab[kNlogEntries];
-    extern __shared__ __align__(16) float s_dyn[];  // [2 * kTileFloats]: two tile buffers
+    extern __shared__ __align__(16) float s_buf[];  // [kTileFloats]: logits, gradients, updated logits
     load_tab(s_tab);
     const NlogCtx L{s_tab};
     float acc = 0.f;
-    int cur = 0;
-    auto stage = [&](float *dst, int64_t t) {
-        const MatDesc &d = grp.d[find_mat(grp, t)];
-        const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
-        stage_in_async(dst, d.pi + tb0 * C, (int)imin64(kBlocksPerCta, d.nblocks - tb0) * C);
-    };
-    if ((int64_t)blockIdx.x < grp.total_work) stage(s_dyn, blockIdx.x);
     int mi = 0;
     for (int64_t t = blockIdx.x; t < grp.total_work; t += gridDim.x) {
         mi = next_mat(grp, mi, t);
         const MatDesc &d = grp.d[mi];
         const int64_t tb0 = (t - d.work_begin) * kBlocksPerCta;
         const int nb = (int)imin64(kBlocksPerCta, d.nblocks - tb0);
-        float *s_pi = s_dyn + cur * kTileFloats, *s_gr = s_dyn + (cur ^ 1) * kTileFloats;
-        cp_async_wait_pending();
-        __syncthreads();  // the tile's logits (and the table) are in; the other buffer is free
         if (threadIdx.x == 0) {
             prefetch_l2(d.m + tb0 * C, nb * C * 4);
             prefetch_l2(d.v + tb0 * C, nb * C * 4);
+            const int64_t tn = t + gridDim.x;
+            if (tn < grp.total_work) {
+                const MatDesc &dn = grp.d[next_mat(grp, mi, tn)];
+                const int64_t nb0 = (tn - dn.work_begin) * kBlocksPerCta;
+                prefetch_l2(dn.pi + nb0 * C, (int)imin64(kBlocksPerCta, dn.nblocks - nb0) * C * 4);
+            }
         }
+        __syncthreads();  // the previous tile's readers are done (and the table is loaded)
+        stage_in(s_buf, d.pi + tb0 * C, nb * C);
+        __syncthreads();
         const bool mine = (int)threadIdx.x < nb;
         const int64_t b = tb0 + threadIdx.x;
-        float wt[8];
         if (mine) {
-            float gw[8];
+            float wt[8], gw[8];
             load8<kW32>(d.W, b, wt);
             load8<kG32>(d.G, b, gw);
-            grad_row(s_pi + threadIdx.x * C, wt, gw, d.gid0 + b, sb, L, s_gr + threadIdx.x * C);
+            grad_row(s_buf + threadIdx.x * C, wt, gw, d.gid0 + b, sb, L, s_buf + threadIdx.x * C);
         }
         __syncthreads();
-        adam_tile<true>(s_pi, s_gr, nb * C, d.pi + tb0 * C, d.m + tb0 * C, d.v + tb0 * C,
-                        d.grad ? d.grad + tb0 * C : nullptr, sb);
-        __syncthreads();  // updated logits in s_pi; the gradient buffer is free
-        if (t + gridDim.x < grp.total_work) stage(s_gr, t + gridDim.x);
+        adam_tile_inplace(s_buf, nb * C, d.pi + tb0 * C, d.m + tb0 * C, d.v + tb0 * C,
+                          d.grad ? d.grad + tb0 * C : nullptr, sb);
+        __syncthreads();  // updated logits in s_buf
         if (mine) {
-            float ms[8], x[8];
-            fwd_row(s_pi + threadIdx.x * C, wt, d.gid0 + b, sf, L, ms, x, acc);
+            float wt[8], ms[8], x[8];
+            load8<kW32>(d.W, b, wt);  // read again (from L2) rather than held through the tile
+            fwd_row(s_buf + threadIdx.x * C, wt, d.gid0 + b, sf, L, ms, x, acc);
             store8<kW32>(d.X, b, x);
             if (d.soft) {
                 float4 *sp = reinterpret_cast<float4 *>(d.soft + b * 8);
@@ -499,7 +608,6 @@ __global__ void __launch_bounds__(kCtaThreads, 2) bwd_adam_fwd_kernel(const __gr
                 sp[1] = make_float4(ms[4], ms[5], ms[6], ms[7]);
             }
         }
-        cur ^= 1;
     }
     if (reg_out) reduce_reg(acc, partials, ticket, reg_out, accumulate);
 }
@@ -655,11 +763,17 @@ __global__ void __launch_bounds__(kThreads) noise_kernel(int C,
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const uint64_t gid = gids[i];
         for (int gr = 0; gr * 6 < C; ++gr) {
-            uint32_t f[6];
-            fields21(block_words(seed, gid, step, (uint32_t)gr), f);
-            for (int k = 0; k < 6; ++k) {
+            // the samplers' own path: fields placed as the bits of 1 + eps, two draws per
+            // paired evaluation (C is even)
+            uint32_t u[6];
+            fields21_unit(block_words(seed, gid, step, (uint32_t)gr), u);
+            for (int k = 0; k < 6; k += 2) {
                 const int c = 6 * gr + k;
-                if (c < C) out[i * C + c] = gumbel(f[k], L);
+                if (c < C) {
+                    const float2 g = gumbel_unit2(u[k], u[k + 1], L);
+                    out[i * C + c] = g.x;
+                    out[i * C + c + 1] = g.y;
+                }
             }
         }
     }

@@ -72,6 +72,9 @@ int64_t grid_for(const void *fn, int threads, int dyn_smem, int64_t work, int64_
     return std::max<int64_t>(1, std::min<int64_t>({work, g, cap}));
 }
 
+// CTAs the 4:8 forward can use on a group: each CTA's two halves take one tile each.
+int64_t k48_fwd_ctas(const Group &g) { return (g.total_work + k48::kFwdHalves - 1) / k48::kFwdHalves; }
+
 mllm_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return MLLM_OK;
     g_last_cuda = (int32_t)e;
@@ -887,9 +890,9 @@ mllm_status mllm_sample_fwd(const mllm_matrix *mats, int32_t n_mats, mllm_nm nm,
             else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         } else {
             const void *fn = w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>;
-            const int64_t grid = grid_for(fn, k48::kCtaThreads, k48::kFwdDynSmem, g.total_work, kMaxReduceCtas);
-            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
-            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            const int64_t grid = grid_for(fn, k48::kFwdThreads, k48::kFwdDynSmem, k48_fwd_ctas(g), kMaxReduceCtas);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kFwdThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kFwdThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         }
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -911,13 +914,14 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
     const bool is24 = nm.m == 4;
     const void *fn = is24 ? (w32 ? (const void *)k24::fwd_kernel<true> : (const void *)k24::fwd_kernel<false>)
                           : (w32 ? (const void *)k48::fwd_kernel<true> : (const void *)k48::fwd_kernel<false>);
-    const int threads = is24 ? kThreads : k48::kCtaThreads;
+    const int threads = is24 ? kThreads : k48::kFwdThreads;
     const int dyn_smem = is24 ? 0 : k48::kFwdDynSmem;
+    auto ctas_wanted = [&](const Group &g) { return is24 ? g.total_work : k48_fwd_ctas(g); };
     const std::vector<Group> groups = make_groups(mats, n_mats, nm.m, is24 ? Kind::Sample24 : Kind::Sample48);
     // every launch's scratch need (one partial per CTA) is checked before anything runs
     for (const Group &g : groups) {
         if (g.total_work == 0) continue;
-        if (grid_for(fn, threads, dyn_smem, g.total_work, kMaxReduceCtas) > kNoallocMaxCtas) return MLLM_ERR_WORKSPACE;
+        if (grid_for(fn, threads, dyn_smem, ctas_wanted(g), kMaxReduceCtas) > kNoallocMaxCtas) return MLLM_ERR_WORKSPACE;
     }
     void *scratch = nullptr;
     if ((s = noalloc_scratch(&scratch)) != MLLM_OK) return s;
@@ -930,13 +934,13 @@ mllm_status mllm_sample_fwd_noalloc(const mllm_matrix *mats, int32_t n_mats, mll
         if (g.total_work == 0) continue;
         if ((s = cuda_status(cudaMemsetAsync(ticket, 0, sizeof(unsigned int), st))) != MLLM_OK) return s;
         const int accumulate = wrote_reg ? 1 : 0;
-        const int64_t grid = grid_for(fn, threads, dyn_smem, g.total_work, kMaxReduceCtas);
+        const int64_t grid = grid_for(fn, threads, dyn_smem, ctas_wanted(g), kMaxReduceCtas);
         if (is24) {
             if (w32) k24::fwd_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
             else k24::fwd_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         } else {
-            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
-            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kCtaThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            if (w32) k48::fwd_kernel<true><<<(unsigned)grid, k48::kFwdThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
+            else k48::fwd_kernel<false><<<(unsigned)grid, k48::kFwdThreads, k48::kFwdDynSmem, st>>>(g, sc, partials, ticket, reg_sum_out, accumulate);
         }
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
         wrote_reg = true;
@@ -1017,10 +1021,10 @@ mllm_status mllm_sample_bwd_adam_fwd(const mllm_matrix *mats, int32_t n_mats, ml
             else if (g32) MLLM_LAUNCH_FUSED(k24, kThreads, 0, false, true);
             else MLLM_LAUNCH_FUSED(k24, kThreads, 0, false, false);
         } else {
-            if (w32 && g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, true);
-            else if (w32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, true, false);
-            else if (g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, true);
-            else MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kBwdDynSmem, false, false);
+            if (w32 && g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kStepDynSmem, true, true);
+            else if (w32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kStepDynSmem, true, false);
+            else if (g32) MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kStepDynSmem, false, true);
+            else MLLM_LAUNCH_FUSED(k48, k48::kCtaThreads, k48::kStepDynSmem, false, false);
         }
 #undef MLLM_LAUNCH_FUSED
         if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
