@@ -134,27 +134,41 @@ __device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) 
 // bit-identical to one-at-a-time evaluation. w2[k] holds candidates 2k and 2k+1.
 constexpr int C2 = C / 2;
 
-// Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates, and their maximum.
-__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
-                                           const NlogCtx &L, float2 w2[C2]) {
+// max(a, b, c) in one instruction (the three-input form of max.f32, sm_100); NaN operands
+// are passed over as by fmaxf.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates (noise of `step` under
+// the seed's round keys rk), and their maximum.
+__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, uint32_t step, float kappa,
+                                           bool noise_on, const uint32_t (&rk)[20], const NlogCtx &L,
+                                           float2 w2[C2]) {
     float mx = -INFINITY;
     const float2 *pi2 = reinterpret_cast<const float2 *>(pi_row);  // rows are 280 B: 8-byte aligned
 #pragma unroll
     for (int gr = 0; gr < 12; ++gr) {
         uint32_t u[6];
-        if (sc.noise_on) fields21_unit(block_words(sc, gid, (uint32_t)gr), u);
+        if (noise_on) fields21_unit(block_words(rk, step, gid, (uint32_t)gr), u);
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int c = 6 * gr + 2 * k;
             if (c < C) {
-                const float2 g = sc.noise_on ? gumbel_unit2(u[2 * k], u[2 * k + 1], L) : make_float2(0.f, 0.f);
-                const float2 wc = __ffma2_rn(f2(sc.kappa), pi2[c / 2], g);
+                const float2 g = noise_on ? gumbel_unit2(u[2 * k], u[2 * k + 1], L) : make_float2(0.f, 0.f);
+                const float2 wc = __ffma2_rn(f2(kappa), pi2[c / 2], g);
                 w2[c / 2] = wc;
-                mx = fmaxf(fmaxf(mx, wc.x), wc.y);
+                mx = fmax3(mx, wc.x, wc.y);
             }
         }
     }
     return mx;
+}
+__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
+                                           const NlogCtx &L, float2 w2[C2]) {
+    return perturbed(pi_row, gid, sc.step, sc.kappa, sc.noise_on, sc.rk, L, w2);
 }
 
 // Sums over candidates, formed per half of the block. A candidate's four kept positions are
@@ -200,7 +214,8 @@ __device__ __forceinline__ float bucket_sum(const float B[16]) {
 // e_c = 2^((w_c - max) c2) in place; returns sum e; ms2 = sums over c with j in S_c and, when
 // kComp, mc2 = sums over c with j not in S_c (pairs of positions 2p, 2p+1).
 template <bool kComp>
-__device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, float2 ms2[4], float2 mc2[4]) {
+__device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, float2 ms2[4], float2 mc2[4],
+                                           bool comp = kComp) {
     float BL[16], BH[16];  // buckets by low-half and by high-half subset
     const float m2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
     auto put = [&](auto I, float e) {
@@ -222,7 +237,7 @@ __device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, fl
     ms2[1] = make_float2(bucket_sum<2, true>(BL), bucket_sum<3, true>(BL));
     ms2[2] = make_float2(bucket_sum<0, true>(BH), bucket_sum<1, true>(BH));
     ms2[3] = make_float2(bucket_sum<2, true>(BH), bucket_sum<3, true>(BH));
-    if (kComp) {
+    if (kComp && comp) {
         mc2[0] = make_float2(bucket_sum<0, false>(BL), bucket_sum<1, false>(BL));
         mc2[1] = make_float2(bucket_sum<2, false>(BL), bucket_sum<3, false>(BL));
         mc2[2] = make_float2(bucket_sum<0, false>(BH), bucket_sum<1, false>(BH));
@@ -288,14 +303,13 @@ __device__ __forceinline__ void adamw(float &p, float &m, float &v, float g, con
     p = __fmaf_rn(-s.step_size, __fdividef(m, denom), pd);
 }
 
-// Gradient of one block's logits (Eq.6-Eq.8 backward, noise of step sc.step) into grow[C]:
+// Gradient of one block's logits (Eq.6-Eq.8 backward) into grow[C] from e_c (in w2),
+// r = 1 / sum e and the position sums ms2, mc2 of the step's noise:
 // dpi_c = (kappa/tau) y_c (sum_{j in S_c} P_j - sum_{j not in S_c} Q_j), P_j = (1 - M_j) u_j,
 // Q_j = M_j u_j, u_j = G_j W_j - 2 lambda W_j^2 M_j.
-__device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8], const float gw[8], uint64_t gid,
-                                         const StepScalars &sc, const NlogCtx &L, float *grow) {
-    float2 w2[C2], ms2[4], mc2[4];
-    const float mx = perturbed(pi_row, gid, sc, L, w2);
-    const float r = rcp_approx(soft_sums<true>(w2, mx, sc.c2, ms2, mc2));
+__device__ __forceinline__ void grad_tail(const float2 w2[C2], float r, const float2 ms2[4], const float2 mc2[4],
+                                          const float wt[8], const float gw[8], const StepScalars &sc,
+                                          float *grow) {
     float P[8], Q[8];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {  // positions 2p, 2p+1
@@ -320,13 +334,19 @@ __device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8],
     });
 }
 
-// Forward of one block (Eq.5-Eq.8): soft mask ms[8] and soft-masked weights x[8] (fp32),
-// regulariser partial added to acc.
-__device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], uint64_t gid, const StepScalars &sc,
-                                        const NlogCtx &L, float ms[8], float x[8], float &acc) {
+// The same from the block's logits (noise of step sc.step).
+__device__ __forceinline__ void grad_row(const float *pi_row, const float wt[8], const float gw[8], uint64_t gid,
+                                         const StepScalars &sc, const NlogCtx &L, float *grow) {
     float2 w2[C2], ms2[4], mc2[4];
     const float mx = perturbed(pi_row, gid, sc, L, w2);
-    const float r = rcp_approx(soft_sums<false>(w2, mx, sc.c2, ms2, mc2));
+    const float r = rcp_approx(soft_sums<true>(w2, mx, sc.c2, ms2, mc2));
+    grad_tail(w2, r, ms2, mc2, wt, gw, sc, grow);
+}
+
+// Forward of one block (Eq.5-Eq.8) from r = 1 / sum e and the position sums ms2: soft mask
+// ms[8] and soft-masked weights x[8] (fp32), regulariser partial added to acc.
+__device__ __forceinline__ void fwd_tail(const float2 ms2[4], float r, const float wt[8], float ms[8], float x[8],
+                                         float &acc) {
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const float2 m = __fmul2_rn(ms2[p], f2(r));
@@ -336,6 +356,15 @@ __device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], 
         acc = __fmaf_rn(xx.x, xx.x, acc);
         acc = __fmaf_rn(xx.y, xx.y, acc);
     }
+}
+
+// The same from the block's logits (noise of step sc.step).
+__device__ __forceinline__ void fwd_row(const float *pi_row, const float wt[8], uint64_t gid, const StepScalars &sc,
+                                        const NlogCtx &L, float ms[8], float x[8], float &acc) {
+    float2 w2[C2], ms2[4], mc2[4];
+    const float mx = perturbed(pi_row, gid, sc, L, w2);
+    const float r = rcp_approx(soft_sums<false>(w2, mx, sc.c2, ms2, mc2));
+    fwd_tail(ms2, r, wt, ms, x, acc);
 }
 
 // AdamW over a tile as one flat, coalesced array of float4: logits and gradients from shared
