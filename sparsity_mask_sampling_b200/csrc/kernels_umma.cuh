@@ -135,11 +135,16 @@ __device__ __forceinline__ bool um_bar_or(bool p) {
 template <int kCount>
 __device__ __forceinline__ void um_bar() { asm volatile("barrier.cta.sync 1, %0;\n" ::"n"(kCount) : "memory"); }
 
-// Warp-uniform bounded wait that also gives up once *abort is set.
+// Warp-uniform bounded wait that also gives up once *abort is set. The clock and the abort
+// flag are read once per 8 polls (each poll is a try_wait, which itself suspends the warp
+// for a bounded time), so a waiting warp takes few issue slots from the working ones.
 __device__ __forceinline__ bool um_wait(unsigned bar, unsigned parity, const volatile int *abort) {
+    if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
     const unsigned long long t0 = __shfl_sync(0xFFFFFFFFu, globaltimer_ns(), 0);
     while (true) {
-        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k)
+            if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
         if (__any_sync(0xFFFFFFFFu, *abort != 0)) return false;
         if (__shfl_sync(0xFFFFFFFFu, globaltimer_ns(), 0) - t0 > kTmWaitNs) return false;
     }
