@@ -190,11 +190,6 @@ __device__ __forceinline__ uint4 block_words(const StepScalars &sc, uint64_t gid
     return philox4x32_10_rk(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), sc.step, group), sc.rk);
 }
 
-// The same with the step given apart from the seed's round keys.
-__device__ __forceinline__ uint4 block_words(const uint32_t (&rk)[20], uint32_t step, uint64_t gid, uint32_t group) {
-    return philox4x32_10_rk(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), step, group), rk);
-}
-
 // eps = (2k+1) 2^-22: the bit pattern of 1 + (2k+1) 2^-22 minus 1 (both exact).
 __device__ __forceinline__ float uniform_from_field(uint32_t k) {
     return __fadd_rn(__uint_as_float(0x3F800002u | (k << 2)), -1.0f);

@@ -134,6 +134,11 @@ __device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) 
 // bit-identical to one-at-a-time evaluation. w2[k] holds candidates 2k and 2k+1.
 constexpr int C2 = C / 2;
 
+// block_words with the step given apart from the seed's round keys.
+__device__ __forceinline__ uint4 block_words_rk(const uint32_t (&rk)[20], uint32_t step, uint64_t gid, uint32_t group) {
+    return philox4x32_10_rk(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), step, group), rk);
+}
+
 // max(a, b, c) in one instruction (the three-input form of max.f32, sm_100); NaN operands
 // are passed over as by fmaxf.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -152,7 +157,7 @@ __device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, ui
 #pragma unroll
     for (int gr = 0; gr < 12; ++gr) {
         uint32_t u[6];
-        if (noise_on) fields21_unit(block_words(rk, step, gid, (uint32_t)gr), u);
+        if (noise_on) fields21_unit(block_words_rk(rk, step, gid, (uint32_t)gr), u);
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int c = 6 * gr + 2 * k;
