@@ -134,11 +134,6 @@ __device__ __forceinline__ void store8(void *base, int64_t b, const float x[8]) 
 // bit-identical to one-at-a-time evaluation. w2[k] holds candidates 2k and 2k+1.
 constexpr int C2 = C / 2;
 
-// block_words with the step given apart from the seed's round keys.
-__device__ __forceinline__ uint4 block_words_rk(const uint32_t (&rk)[20], uint32_t step, uint64_t gid, uint32_t group) {
-    return philox4x32_10_rk(make_uint4((uint32_t)gid, (uint32_t)(gid >> 32), step, group), rk);
-}
-
 // max(a, b, c) in one instruction (the three-input form of max.f32, sm_100); NaN operands
 // are passed over as by fmaxf.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -147,33 +142,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates (noise of `step` under
-// the seed's round keys rk), and their maximum.
-__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, uint32_t step, float kappa,
-                                           bool noise_on, const uint32_t (&rk)[20], const NlogCtx &L,
-                                           float2 w2[C2]) {
+// Perturbed logits w_c = fma(kappa, pi_c, g_c) for all 70 candidates, and their maximum.
+__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
+                                           const NlogCtx &L, float2 w2[C2]) {
     float mx = -INFINITY;
     const float2 *pi2 = reinterpret_cast<const float2 *>(pi_row);  // rows are 280 B: 8-byte aligned
 #pragma unroll
     for (int gr = 0; gr < 12; ++gr) {
         uint32_t u[6];
-        if (noise_on) fields21_unit(block_words_rk(rk, step, gid, (uint32_t)gr), u);
+        if (sc.noise_on) fields21_unit(block_words(sc, gid, (uint32_t)gr), u);
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int c = 6 * gr + 2 * k;
             if (c < C) {
-                const float2 g = noise_on ? gumbel_unit2(u[2 * k], u[2 * k + 1], L) : make_float2(0.f, 0.f);
-                const float2 wc = __ffma2_rn(f2(kappa), pi2[c / 2], g);
+                const float2 g = sc.noise_on ? gumbel_unit2(u[2 * k], u[2 * k + 1], L) : make_float2(0.f, 0.f);
+                const float2 wc = __ffma2_rn(f2(sc.kappa), pi2[c / 2], g);
                 w2[c / 2] = wc;
                 mx = fmax3(mx, wc.x, wc.y);
             }
         }
     }
     return mx;
-}
-__device__ __forceinline__ float perturbed(const float *pi_row, uint64_t gid, const StepScalars &sc,
-                                           const NlogCtx &L, float2 w2[C2]) {
-    return perturbed(pi_row, gid, sc.step, sc.kappa, sc.noise_on, sc.rk, L, w2);
 }
 
 // Sums over candidates, formed per half of the block. A candidate's four kept positions are
@@ -219,8 +208,7 @@ __device__ __forceinline__ float bucket_sum(const float B[16]) {
 // e_c = 2^((w_c - max) c2) in place; returns sum e; ms2 = sums over c with j in S_c and, when
 // kComp, mc2 = sums over c with j not in S_c (pairs of positions 2p, 2p+1).
 template <bool kComp>
-__device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, float2 ms2[4], float2 mc2[4],
-                                           bool comp = kComp) {
+__device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, float2 ms2[4], float2 mc2[4]) {
     float BL[16], BH[16];  // buckets by low-half and by high-half subset
     const float m2 = __fmul_rn(mx, c2);  // (w - max) c2 = w c2 - fl(max c2): a common rounding that cancels
     auto put = [&](auto I, float e) {
@@ -242,7 +230,7 @@ __device__ __forceinline__ float soft_sums(float2 w2[C2], float mx, float c2, fl
     ms2[1] = make_float2(bucket_sum<2, true>(BL), bucket_sum<3, true>(BL));
     ms2[2] = make_float2(bucket_sum<0, true>(BH), bucket_sum<1, true>(BH));
     ms2[3] = make_float2(bucket_sum<2, true>(BH), bucket_sum<3, true>(BH));
-    if (kComp && comp) {
+    if (kComp) {
         mc2[0] = make_float2(bucket_sum<0, false>(BL), bucket_sum<1, false>(BL));
         mc2[1] = make_float2(bucket_sum<2, false>(BL), bucket_sum<3, false>(BL));
         mc2[2] = make_float2(bucket_sum<0, false>(BH), bucket_sum<1, false>(BH));
