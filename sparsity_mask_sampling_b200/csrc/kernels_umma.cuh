@@ -657,36 +657,42 @@ __global__ void __launch_bounds__(kPfThreads, 1) sparse_linear_prefill_kernel(co
 // ------------------------------------------------------------------ 4:8 on the dense tensor cores
 //
 // 4:8 has no hardware sparse mode. Per 128-column stage, kU8Warps warps expand the compressed
-// tile into a dense 128 x 128 bf16 tile in shared memory (two 128 x 64 atoms in the K-major,
-// 128-byte swizzled layout of the MMA's descriptors), and one thread issues eight dense
-// tcgen05.mma (kind::f16, K = 16) on it. A 4:8 block (four kept values in position order and
-// the code p0 | p1 << 3 | p2 << 6 | p3 << 9) expands into exactly one 16-byte chunk of eight
-// bf16. Word i of the chunk (positions 2i, 2i+1) is prmt(prmt(v0v1, 0, A[p0p1].i), v2v3,
-// B[p2p3].i): table A places the first pair and zero-fills, table B places the second pair
-// and keeps the rest (u8_table_entry). Each CTA builds both 64-entry tables in shared memory,
-// 8 interleaved copies each, so that the 16-byte lookups of a quarter-warp never share a bank. Thread t
-// expands row t % 128, part t / 128 of the stage (64 / kU8Warps blocks, within one atom), and
-// arrives on the stage's "expanded" barrier; a separate MMA warp waits for all arrivals and
-// issues the stage's MMAs, so the expanding warps never wait on one another within a tile
-// (they meet once per tile, for the epilogue).
-// A stage: values 16 KB | x, two kNTok x 64 boxes | metadata, 128 rows x 16 codes (4 KB) |
-// the dense tile (32 KB). One CTA per SM with three stages; tensor memory holds only the
-// accumulator (64 columns). Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 and the
-// token slice w / 4. Copy warp, bounded waits, work split and partial tiles as above; a warp
-// whose wait runs out stops working and leaves with the others at the end of the tile.
+// tile into a dense 128 x 128 bf16 tile in tensor memory (row m in lane m, 64 columns of two
+// bf16 each in K order), and one thread issues eight dense tcgen05.mma (kind::f16, K = 16)
+// that read A from tensor memory and the activations from shared memory. A 4:8 block (four
+// kept values in position order and the code p0 | p1 << 3 | p2 << 6 | p3 << 9) expands into
+// exactly four 32-bit columns. Column i of a block (positions 2i, 2i+1) is
+// prmt(prmt(v0v1, 0, A[p0p1].i), v2v3, B[p2p3].i): table A places the first pair and
+// zero-fills, table B places the second pair and keeps the rest (u8_table_entry). Each CTA
+// builds both 64-entry tables in shared memory, 8 interleaved copies each, so that the
+// 16-byte lookups of a quarter-warp never share a bank. Thread t expands row t % 128, part
+// t / 128 of the stage (64 / kU8Warps blocks: 16 columns, one tcgen05.st of its own lane),
+// and arrives on the stage's "expanded" barrier after its store has completed; a separate MMA
+// warp waits for all arrivals and issues the stage's MMAs, so the expanding warps never wait
+// on one another within a tile (they meet once per tile, for the epilogue). The dense tile
+// never enters shared memory, so a stage is only what the copy engine lands: values 16 KB |
+// x, two kNTok x 64 boxes | metadata, 128 rows x 16 codes (4 KB); five or six stages in
+// flight. Tensor memory: the accumulator in columns 0-63, stage s's dense tile in columns
+// 64 + 64 s (it is rewritten only after the stage's MMAs have completed, which the copy warp
+// waits for before it refills the stage). One CTA per SM. Epilogue: warp w reads TMEM lanes
+// 32 (w % 4) .. +31 and the token slice w / 4. Copy warp, bounded waits, work split and
+// partial tiles as above; a warp whose wait runs out stops working and leaves with the others
+// at the end of the tile.
 
 constexpr int kU8Warps = 16;         // expansion / epilogue warps (a multiple of 4, at most 16)
 constexpr int kU8Threads = 32 * kU8Warps + 64;  // + the copy warp and the MMA warp
 constexpr int kU8NStep = 8 * (kU8Warps / 4) > 16 ? 8 * (kU8Warps / 4) : 16;  // N is a multiple of this
-constexpr int kU8Stages = 3;
-constexpr unsigned kU8TmemCols = 64;
+constexpr unsigned kU8TmemCols = 512;  // accumulator at 0 (N <= 64 columns), the stages' dense tiles from kU8ACol
+constexpr unsigned kU8ACol = 64;       // a stage's dense 128 x 128 bf16 tile: 64 columns (2 values per column)
 
 template <int kNTok> constexpr int u8_tx() { return kUmRows * 128 + 2 * um_xbox_bytes<kNTok>() + kUmRows * 32; }
-template <int kNTok> constexpr int u8_a_off() { return (u8_tx<kNTok>() + 1023) / 1024 * 1024; }
-template <int kNTok> constexpr int u8_stage_bytes() { return u8_a_off<kNTok>() + 2 * kUmRows * 128; }
+template <int kNTok> constexpr int u8_stage_bytes() { return (u8_tx<kNTok>() + 1023) / 1024 * 1024; }
+// Stages in flight: as many as shared memory holds beside the selector tables, at most six
+// (six dense tiles fill tensor memory beside the accumulator).
+template <int kNTok> constexpr int u8_stages() { return kNTok <= 48 ? 6 : 5; }
 constexpr int kU8TabCopies = 8;      // one copy per lane of a quarter-warp: conflict-free 16-byte lookups
 constexpr int kU8TabBytes = 2 * 64 * kU8TabCopies * 16;  // tables A and B
-template <int kNTok> constexpr int u8_smem_bytes() { return kU8Stages * u8_stage_bytes<kNTok>() + 1024 + kU8TabBytes; }
+template <int kNTok> constexpr int u8_smem_bytes() { return u8_stages<kNTok>() * u8_stage_bytes<kNTok>() + 1024 + kU8TabBytes; }
 
 // Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
 // N = kNTok, M = 128.
@@ -701,6 +707,28 @@ __device__ __forceinline__ void umma_dense(unsigned d_tmem, uint64_t adesc, uint
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// The same with A read from tensor memory (a_tmem: lane 0, first column of the K-slice; A
+// K-major, two bf16 per 32-bit column).
+__device__ __forceinline__ void umma_dense_ta(unsigned d_tmem, unsigned a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's lane from w[16], then wait for the store.
+__device__ __forceinline__ void tmem_st16(unsigned taddr, const uint32_t (&w)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};\n" ::"r"(taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]),
+        "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
 
 // 8 consecutive accumulator columns of this thread's lane (see tmem_ld16).
@@ -752,12 +780,14 @@ __device__ __forceinline__ void u8_issue(const TmGroup &tg, const Cursor &c, uns
     tma_load_2d(stage + kUmRows * 128 + 2 * um_xbox_bytes<kNTok>(), &mp.meta, 16 * j, row0, bar);
 }
 
-// Row r, part pt of a stage (kBlk = 64 / kU8Warps blocks from block kBlk pt; a part lies in
-// one atom) into the dense tile.
-__device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char *dense, const uint4 *tab_a,
-                                          const uint4 *tab_b, int meta_off, int r, int pt) {
-    constexpr int kBlk = 64 / kU8Warps;  // 8 or 4 blocks, 2 per 16-byte value chunk
-    const int b0 = kBlk * pt, atom = b0 >> 3;
+// Row r, part pt of a stage (kBlk = 64 / kU8Warps blocks from block kBlk pt) expanded into
+// its 4 kBlk 32-bit columns of the row's dense K-slice: block b's eight values are columns
+// 4 (b - kBlk pt) .. +3, two bf16 per column in K order (the layout tcgen05.mma reads A in
+// from tensor memory).
+template <int kBlk>
+__device__ __forceinline__ void u8_expand(const unsigned char *st, const uint4 *tab_a, const uint4 *tab_b,
+                                          int meta_off, int r, int pt, uint32_t (&w)[4 * kBlk]) {
+    const int b0 = kBlk * pt;
     uint32_t codes[kBlk / 2];
     if constexpr (kBlk == 8) {
         const uint4 cw = lds128(st + meta_off + r * 32 + b0 * 2);
@@ -766,7 +796,6 @@ __device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char
         const uint2 cw = *reinterpret_cast<const uint2 *>(st + meta_off + r * 32 + b0 * 2);
         codes[0] = cw.x; codes[1] = cw.y;
     }
-    unsigned char *row = dense + atom * (kUmRows * 128) + r * 128;
 #pragma unroll
     for (int c = 0; c < kBlk / 2; ++c) {
         const int cl = (b0 >> 1) + c;  // value chunk within the row
@@ -776,13 +805,11 @@ __device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned char
             const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
             const uint32_t code = (codes[c] >> (16 * h)) & 0xFFFu;
             const uint4 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
-            uint4 o;
-            o.x = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
-            o.y = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
-            o.z = __byte_perm(__byte_perm(lo, 0u, sa.z), hi, sb.z);
-            o.w = __byte_perm(__byte_perm(lo, 0u, sa.w), hi, sb.w);
-            const int b = (2 * cl + h) & 7;  // dense chunk within the atom
-            *reinterpret_cast<uint4 *>(row + ((b ^ (r & 7)) << 4)) = o;
+            uint32_t *o = w + 4 * (2 * c + h);
+            o[0] = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
+            o[1] = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
+            o[2] = __byte_perm(__byte_perm(lo, 0u, sa.z), hi, sb.z);
+            o[3] = __byte_perm(__byte_perm(lo, 0u, sa.w), hi, sb.w);
         }
     }
 }
@@ -805,9 +832,13 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
                                                                             int arm_only_first) {
     static_assert(kNTok % 16 == 0 && kNTok >= 16 && kNTok <= kMaxTokens, "N of an M = 128 MMA");
     static_assert(2 * (u8_smem_bytes<kNTok>() + 1024) > 233472, "one CTA per SM");
+    static_assert(u8_smem_bytes<kNTok>() + 1024 <= 232448, "fits one SM");
+    static_assert(kU8ACol >= (unsigned)kNTok && kU8ACol + 64u * u8_stages<kNTok>() <= kU8TmemCols,
+                  "accumulator and dense tiles fit tensor memory");
+    static_assert(kU8Warps == 16, "four threads per row, one x16 store of 16 columns each");
     static_assert(kU8Warps % 4 == 0 && kU8Warps <= 16 && kNTok % (8 * (kU8Warps / 4)) == 0,
                   "each epilogue warp takes a multiple of 8 token columns");
-    constexpr int kD = kU8Stages, kStage = u8_stage_bytes<kNTok>(), kAOff = u8_a_off<kNTok>();
+    constexpr int kD = u8_stages<kNTok>(), kStage = u8_stage_bytes<kNTok>();
     constexpr int kMetaOff = kUmRows * 128 + 2 * um_xbox_bytes<kNTok>();
     constexpr int kHalf = kNTok / (kU8Warps / 4);  // token columns per epilogue warp
     constexpr int kBar = 32 * kU8Warps;
@@ -904,13 +935,13 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
             if (lane == 0) {
                 tc_fence_after();
                 const unsigned sa = ring_s + s * kStage;
-                const uint64_t a0 = um_desc(sa + kAOff), a1 = um_desc(sa + kAOff + kUmRows * 128),
-                               b0 = um_desc(sa + kUmRows * 128),
+                const unsigned ta = tbase + kU8ACol + 64u * (unsigned)s;  // the stage's dense tile
+                const uint64_t b0 = um_desc(sa + kUmRows * 128),
                                b1 = um_desc(sa + kUmRows * 128 + um_xbox_bytes<kNTok>());
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    umma_dense(tbase, ((j >> 2) ? a1 : a0) + (uint64_t)(2 * (j & 3)),
-                               ((j >> 2) ? b1 : b0) + (uint64_t)(2 * (j & 3)), kIdesc, (fresh && j == 0) ? 0u : 1u);
+                for (int j = 0; j < 8; ++j)  // K = 16 per MMA: 8 columns of A
+                    umma_dense_ta(tbase, ta + 8u * (unsigned)j, ((j >> 2) ? b1 : b0) + (uint64_t)(2 * (j & 3)),
+                                  kIdesc, (fresh && j == 0) ? 0u : 1u);
                 umma_commit(empty0 + 8 * s);
                 if (piece_end) umma_commit(accb);
             }
@@ -928,6 +959,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
         const int r = threadIdx.x & (kUmRows - 1), pt = threadIdx.x >> 7;
         const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
         const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
+        const unsigned tdense = tbase + ((unsigned)(32 * q) << 16) + kU8ACol + 16u * (unsigned)pt;  // row r's part
         const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
         Cursor cc = sk_decode(grp, lo);
         unsigned acc_phase = 0u;
@@ -939,8 +971,10 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
             // it meets the others at the end of the tile, where all of them leave together.
             if (!failed) {
                 if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
-                    u8_expand(st, st + kAOff, tab_a, tab_b, kMetaOff, r, pt);
-                    fence_proxy_async();  // the dense tile, written here, is read by the tensor cores
+                    uint32_t w[16];
+                    u8_expand<64 / kU8Warps>(st, tab_a, tab_b, kMetaOff, r, pt, w);
+                    tmem_st16(tdense + 64u * (unsigned)s, w);  // into the stage's dense tile in tensor memory
+                    tc_fence_before();
                     mbar_arrive(exp0 + 8 * s);
                 } else {
                     failed = true;
