@@ -3,25 +3,30 @@
 // y = x W*^T from the packed 4:8 hard mask (MaskLLM serves the masked network from its hard
 // mask after training: paper-graph-ui summary of arXiv 2409.17481, s.3.2 "Information flow at
 // inference"; s.5 Table 16 times 128- and 2048-token prompts). 4:8 has no hardware sparse
-// mode, so each stage of compressed blocks is expanded to a dense bf16 tile in shared memory
+// mode, so each stage of compressed blocks is expanded to a dense bf16 tile in tensor memory
 // (the byte-permute expansion of sparse_linear_umma48_kernel, same selector tables) and fed to
-// dense tcgen05.mma (kind::f16). Unlike the decode kernel, which expands every weight once per
-// group of at most 64 tokens, a stage here is expanded once for 256 tokens: the MMA's N is 256
-// and the accumulator (128 rows x 256 tokens of fp32) fills 256 tensor-memory columns (calls
-// of at most 128 tokens use N = 128 and 128 columns, with four stages instead of three).
+// dense tcgen05.mma (kind::f16) that reads A from tensor memory and the activations from
+// shared memory. Unlike the decode kernel, which expands every weight once per group of at
+// most 64 tokens, a stage here is expanded once for 256 tokens: the MMA's N is 256 and the
+// accumulator (128 rows x 256 tokens of fp32) fills 256 tensor-memory columns (calls of at most
+// 128 tokens use N = 128 and 128 columns, with six stages instead of four).
 //
 // A unit is (operand, 128-row tile, N-token chunk) over all columns, in stages of 64 columns
 // (eight 4:8 blocks per row). Per stage the copy warp lands, on one mbarrier, the N x 64 box
-// of x (128-byte swizzle, the MMA's K-major layout), the 128 x 32 box of compressed values and
-// the 128 x 8 box of codes; the 16 expansion warps write the 128 x 64 dense atom (128-byte
-// swizzle) and arrive on the stage's "expanded" barrier; the MMA warp issues four MMAs
-// (K = 16) and commits them to the stage's "empty" barrier, and at a unit's last stage to the
-// accumulator barrier; then the same 16 warps store the unit's y (warp w: TMEM lane quarter
-// w % 4, a quarter of the unit's tokens). Units are dealt round-robin to one CTA per SM in the
-// order of the 2:4 prefill kernel (row-tile groups, token chunk by token chunk), so a weight
-// strip is read from HBM about once per launch. Rows and tokens past the call are zero-filled
-// by the tensor maps and not stored. Every wait is bounded; a timeout sets the error word and
-// the CTA winds down as the other tensor-memory kernels do.
+// of x (128-byte swizzle, the MMA's K-major layout), the 128 x 32 box of compressed values
+// (64-byte swizzle) and the 128 x 8 box of codes; each of the 16 expansion warps takes the 32
+// rows of its tensor-memory lane quarter (warp % 4) and a quarter of the stage's columns
+// (warp / 4), writes its rows' 8 dense columns with one tcgen05.st and arrives on the stage's
+// "expanded" barrier; the MMA warp issues four MMAs (K = 16) and commits them to the stage's
+// "empty" barrier, and at a unit's last stage to the accumulator barrier; then the same 16
+// warps store the unit's y (warp w: TMEM lane quarter w % 4, a quarter of the unit's tokens).
+// Tensor memory: the accumulator in columns 0 .. N-1, stage s's dense tile (32 columns) from
+// column N + 32 s; a tile is rewritten only after its stage's MMAs have completed (the copy
+// warp waits for that before it refills the stage). Units are dealt round-robin to one CTA
+// per SM in the order of the 2:4 prefill kernel (row-tile groups, token chunk by token chunk),
+// so a weight strip is read from HBM about once per launch. Rows and tokens past the call are
+// zero-filled by the tensor maps and not stored. Every wait is bounded; a timeout sets the
+// error word and the CTA winds down as the other tensor-memory kernels do.
 #pragma once
 
 #include "kernels_umma.cuh"
@@ -32,15 +37,15 @@ namespace spl {
 // Tokens per unit (the MMA's N): 256, or 128 for calls of at most 128 tokens (a 256-token
 // unit would compute half of its columns on zero-filled tokens).
 template <int kTok> struct P8 {
-    static constexpr int kXOff = 0;                              // x: kTok tokens x 64 columns
-    static constexpr int kDenseOff = kTok * 128;                 // the dense atom: 128 rows x 64 columns (16 KB)
-    static constexpr int kValOff = kDenseOff + kUmRows * 128;    // values: 128 rows x 32 bf16 (8 KB, unswizzled)
+    static constexpr int kXOff = 0;                              // x: kTok tokens x 64 columns (128-byte swizzle)
+    static constexpr int kValOff = kTok * 128;                   // values: 128 rows x 32 bf16 (8 KB, 64-byte swizzle)
     static constexpr int kMetaOff = kValOff + kUmRows * 64;      // codes: 128 rows x 8 uint16 (2 KB)
     static constexpr int kStageTx = kTok * 128 + kUmRows * 64 + kUmRows * 16;  // bytes the copy engine lands
     static constexpr int kStage = (kMetaOff + kUmRows * 16 + 1023) / 1024 * 1024;
-    static constexpr int kStages = kTok == 256 ? 3 : 4;
+    static constexpr int kStages = kTok == 256 ? 4 : 6;
     static constexpr int kSmem = kStages * kStage + 1024 + kU8TabBytes;
-    static constexpr unsigned kTmemCols = kTok;
+    static constexpr unsigned kACol = kTok;                      // stage s's dense tile: 32 columns from kACol + 32 s
+    static constexpr unsigned kTmemCols = 512;
     // Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
     // N = kTok, M = 128.
     static constexpr uint32_t kIdesc =
@@ -60,27 +65,36 @@ __device__ __forceinline__ void p8_issue(const PfGroup &g, const PfCur &c, int64
 }
 
 // Thread (r, pt) of the stage: row r, blocks 2 pt and 2 pt + 1 (one 16-byte value chunk, one
-// word of two codes) into dense chunks 2 pt + h of row r. Four consecutive threads share a
-// row, so a quarter-warp reads 128 contiguous bytes of values.
+// word of two codes) into the row's dense columns 8 pt .. 8 pt + 7 (two bf16 per column in K
+// order). The values box lands with the 64-byte swizzle (16-byte chunk c of row r at chunk
+// c ^ ((r >> 1) & 3)), so the 32 rows a warp reads at one pt fall on distinct banks in each
+// quarter-warp; each thread reads its row's 16 bytes of codes whole and keeps word pt.
 template <int kTok>
-__device__ __forceinline__ void p8_expand(unsigned char *st, const uint4 *tab_a, const uint4 *tab_b, int r, int pt) {
+__device__ __forceinline__ void p8_expand(const unsigned char *st, const uint4 *tab_a, const uint4 *tab_b, int r, int pt,
+                                          uint32_t (&w)[8]) {
     using K = P8<kTok>;
-    const uint4 v = lds128(st + K::kValOff + r * 64 + pt * 16);
-    const uint32_t cw = lds32(st + K::kMetaOff + r * 16 + pt * 4);
-    unsigned char *row = st + K::kDenseOff + r * 128;
+    const uint4 v = lds128(st + K::kValOff + r * 64 + ((pt ^ ((r >> 1) & 3)) << 4));
+    const uint4 c4 = lds128(st + K::kMetaOff + r * 16);
+    const uint32_t cw = pt == 0 ? c4.x : pt == 1 ? c4.y : pt == 2 ? c4.z : c4.w;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
         const uint32_t code = (cw >> (16 * h)) & 0xFFFu;
         const uint4 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
-        uint4 o;
-        o.x = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
-        o.y = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
-        o.z = __byte_perm(__byte_perm(lo, 0u, sa.z), hi, sb.z);
-        o.w = __byte_perm(__byte_perm(lo, 0u, sa.w), hi, sb.w);
-        const int b = 2 * pt + h;
-        *reinterpret_cast<uint4 *>(row + ((b ^ (r & 7)) << 4)) = o;
+        uint32_t *o = w + 4 * h;
+        o[0] = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
+        o[1] = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
+        o[2] = __byte_perm(__byte_perm(lo, 0u, sa.z), hi, sb.z);
+        o[3] = __byte_perm(__byte_perm(lo, 0u, sa.w), hi, sb.w);
     }
+}
+
+// 8 consecutive 32-bit columns of this thread's lane from w[8], then wait for the store.
+__device__ __forceinline__ void tmem_st8(unsigned taddr, const uint32_t (&w)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(taddr),
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
 
 template <int kTok>
@@ -89,6 +103,8 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
     using K = P8<kTok>;
     static_assert(K::kSmem + 1024 <= 232448, "fits one SM");
     static_assert(kU8Warps == 16, "four threads per row, 128 rows");
+    static_assert(K::kACol + 32u * K::kStages <= K::kTmemCols, "accumulator and dense tiles fit tensor memory");
+    static_assert(K::kValOff % 512 == 0 && K::kStage % 512 == 0, "64-byte-swizzled values box on a 512-byte boundary");
     constexpr int kD = K::kStages, kP8Stage = K::kStage, kQTok = kTok / 4;  // epilogue: tokens per warp
     constexpr int kBar = 32 * kU8Warps;
     constexpr uint32_t kIdesc = K::kIdesc;
@@ -179,11 +195,12 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
                 if (lane == 0) {
                     tc_fence_after();
                     const unsigned st = ring_s + s * kP8Stage;
-                    const uint64_t a0 = um_desc(st + K::kDenseOff), b0 = um_desc(st + K::kXOff);
+                    const unsigned ta = tbase + K::kACol + 32u * (unsigned)s;  // the stage's dense tile
+                    const uint64_t b0 = um_desc(st + K::kXOff);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        umma_dense(tbase, a0 + (uint64_t)(2 * k), b0 + (uint64_t)(2 * k), kIdesc,
-                                   (j == 0 && k == 0) ? 0u : 1u);
+                    for (int k = 0; k < 4; ++k)  // K = 16 per MMA: 8 columns of A
+                        umma_dense_ta(tbase, ta + 8u * (unsigned)k, b0 + (uint64_t)(2 * k), kIdesc,
+                                      (j == 0 && k == 0) ? 0u : 1u);
                     umma_commit(empty0 + 8 * s);
                     if (j == nch - 1) umma_commit(accb);
                 }
@@ -197,9 +214,10 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
         }
     } else {
         // ------------------------------------------------------------ expansion / epilogue warps
-        const int r = threadIdx.x >> 2, pt = threadIdx.x & 3;  // expansion: row, part
-        const int q = warp & 3, sl = warp >> 2;                // epilogue: TMEM lane quarter, token slice
+        const int q = warp & 3, sl = warp >> 2;                // TMEM lane quarter; token slice / part
+        const int r = 32 * q + lane, pt = sl;                  // expansion: row (this lane), part
         const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(kQTok * sl);
+        const unsigned tdense = tbase + ((unsigned)(32 * q) << 16) + K::kACol + 8u * (unsigned)pt;
         const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
         unsigned acc_phase = 0u;
         bool failed = false;
@@ -211,8 +229,10 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
                 const int s = f % kD;
                 if (!failed) {
                     if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
-                        p8_expand<kTok>(ring + s * kP8Stage, tab_a, tab_b, r, pt);
-                        fence_proxy_async();  // the dense atom, written here, is read by the tensor cores
+                        uint32_t w[8];
+                        p8_expand<kTok>(ring + s * kP8Stage, tab_a, tab_b, r, pt, w);
+                        tmem_st8(tdense + 32u * (unsigned)s, w);  // into the stage's dense tile in tensor memory
+                        tc_fence_before();
                         mbar_arrive(exp0 + 8 * s);
                     } else {
                         failed = true;

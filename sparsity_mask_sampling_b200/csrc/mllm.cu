@@ -516,7 +516,7 @@ bool sparse_linear_prefill48_n(const std::vector<mllm_sparse_operand> &ops_in, i
             units += d.npairs * nt;
             const uint64_t rows = (uint64_t)o.rows, cols = (uint64_t)o.cols;
             if (!(encode_2d(&pg.maps[k].vals, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.pack_values, cols / 2, rows, cols, 32,
-                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                            spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_64B) &&
                   encode_2d(&pg.maps[k].meta, CU_TENSOR_MAP_DATA_TYPE_UINT16, o.pack_meta, cols / 8, rows, cols / 4, 8,
                             spl::kUmRows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   encode_2d(&pg.maps[k].x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o.x, cols, (uint64_t)tokens, 2 * cols, 64,
