@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(kThreads) stats24_kernel(const __grid_constant
             for (int i = 0; i < 6; ++i) mx = fmaxf(mx, kappa * p[i]);
             float s = 0.f;
 #pragma unroll
-            for (int i = 0; i < 6; ++i) s += expf(kappa * p[i] - mx);
-            acc[0] += 1.0 / (double)s;
+            for (int i = 0; i < 6; ++i) s += __expf(kappa * p[i] - mx);
+            acc[0] += (double)__frcp_rn(s);  // the block's term in fp32, the sum over blocks in fp64
             const uint32_t mk = k24::cand_mask(k), m0 = k24::top2_mask(w + 4 * h);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -142,9 +142,9 @@ __global__ void __launch_bounds__(kThreads) stats48_kernel(const __grid_constant
         float s = 0.f;
         for (int c2 = 0; c2 < k48::C / 2; ++c2) {
             const float2 v = __ldcs(row + c2);
-            s += expf(kappa * v.x - mx) + expf(kappa * v.y - mx);
+            s += __expf(kappa * v.x - mx) + __expf(kappa * v.y - mx);
         }
-        acc[0] += 1.0 / (double)s;
+        acc[0] += (double)__frcp_rn(s);  // the block's term in fp32, the sum over blocks in fp64
         float key[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) key[j] = (w[j] != w[j]) ? -1.0f : fabsf(w[j]);
@@ -172,10 +172,11 @@ __global__ void __launch_bounds__(kThreads) stats48_kernel(const __grid_constant
 // ------------------------------------------------------------------ candidate-index codec
 
 // D indices per uint32 word, base C, least significant digit first.
+// Words w0 .. of the code (w0 > 0: the tail after encode4_kernel's groups).
 __global__ void __launch_bounds__(kThreads) encode_kernel(const uint8_t *__restrict__ idx, int64_t n, int C,
-                                                          int D, uint32_t *__restrict__ out) {
+                                                          int D, uint32_t *__restrict__ out, int64_t w0 = 0) {
     const int64_t words = (n + D - 1) / D;
-    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < words;
+    for (int64_t wi = w0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < words;
          wi += (int64_t)gridDim.x * blockDim.x) {
         uint32_t v = 0;
         for (int t = D - 1; t >= 0; --t) {  // Horner, most significant digit first
@@ -187,15 +188,82 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const uint8_t *__restr
 }
 
 __global__ void __launch_bounds__(kThreads) decode_kernel(const uint32_t *__restrict__ in, int64_t n, int C,
-                                                          int D, uint8_t *__restrict__ idx) {
+                                                          int D, uint8_t *__restrict__ idx, int64_t w0 = 0) {
     const int64_t words = (n + D - 1) / D;
-    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < words;
+    for (int64_t wi = w0 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < words;
          wi += (int64_t)gridDim.x * blockDim.x) {
         uint32_t v = in[wi];
         for (int t = 0; t < D; ++t) {
             const int64_t i = wi * D + t;
             if (i < n) idx[i] = (uint8_t)(v % (uint32_t)C);
             v /= (uint32_t)C;
+        }
+    }
+}
+
+// The same for whole groups of 4 words per thread with vector accesses (the digits of 4
+// words, 4 D bytes, are read as D 32-bit words; the 4 words are written as one 16-byte
+// store): group g covers indices 4 D g .. 4 D g + 4 D - 1. idx must be 4-byte aligned (16-byte
+// when D % 4 == 0) and out 16-byte aligned; the caller runs the scalar kernel on the tail.
+template <int C, int D>
+__global__ void __launch_bounds__(kThreads) encode4_kernel(const uint8_t *__restrict__ idx, int64_t groups,
+                                                           uint32_t *__restrict__ out) {
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (int64_t)gridDim.x * blockDim.x) {
+        uint32_t b[D];  // bytes 4 k .. 4 k + 3 of the group in b[k]
+        if constexpr (D % 4 == 0) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(idx + 4 * D * g);
+#pragma unroll
+            for (int k = 0; k < D / 4; ++k) {
+                const uint4 v = __ldcs(p + k);
+                b[4 * k] = v.x; b[4 * k + 1] = v.y; b[4 * k + 2] = v.z; b[4 * k + 3] = v.w;
+            }
+        } else {
+            const uint32_t *p = reinterpret_cast<const uint32_t *>(idx + 4 * D * g);
+#pragma unroll
+            for (int k = 0; k < D; ++k) b[k] = __ldcs(p + k);
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int t = D - 1; t >= 0; --t) {  // Horner, most significant digit first
+                const int byte = D * j + t;
+                v = v * (uint32_t)C + __byte_perm(b[byte >> 2], 0u, 0x4440u | (uint32_t)(byte & 3));
+            }
+            w[j] = v;
+        }
+        __stcs(reinterpret_cast<uint4 *>(out) + g, make_uint4(w[0], w[1], w[2], w[3]));
+    }
+}
+
+template <int C, int D>
+__global__ void __launch_bounds__(kThreads) decode4_kernel(const uint32_t *__restrict__ in, int64_t groups,
+                                                           uint8_t *__restrict__ idx) {
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 wv = __ldcs(reinterpret_cast<const uint4 *>(in) + g);
+        const uint32_t wa[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t b[D];
+#pragma unroll
+        for (int k = 0; k < D; ++k) b[k] = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t v = wa[j];
+#pragma unroll
+            for (int t = 0; t < D; ++t) {
+                const int byte = D * j + t;
+                b[byte >> 2] |= (v % (uint32_t)C) << (8 * (byte & 3));
+                v /= (uint32_t)C;
+            }
+        }
+        if constexpr (D % 4 == 0) {
+            uint4 *p = reinterpret_cast<uint4 *>(idx + 4 * D * g);
+#pragma unroll
+            for (int k = 0; k < D / 4; ++k) __stcs(p + k, make_uint4(b[4 * k], b[4 * k + 1], b[4 * k + 2], b[4 * k + 3]));
+        } else {
+            uint32_t *p = reinterpret_cast<uint32_t *>(idx + 4 * D * g);
+#pragma unroll
+            for (int k = 0; k < D; ++k) __stcs(p + k, b[k]);
         }
     }
 }

@@ -1137,13 +1137,31 @@ static mllm_status codec_args(mllm_nm nm, const void *src, const void *dst, int6
     return check_ptr(dst, n > 0);
 }
 
+// The codec's vector kernels read or write the indices as 32-bit (D % 4 == 0: 16-byte) words
+// and the code as 16-byte vectors.
+static bool codec_vector_ok(const void *idx, const void *words, int D) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(idx), b = reinterpret_cast<uintptr_t>(words);
+    return (b & 15u) == 0 && (a & ((D % 4 == 0) ? 15u : 3u)) == 0;
+}
+
 mllm_status mllm_encode_candidates(mllm_nm nm, const uint8_t *idx, int64_t n, uint32_t *words, void *stream) {
     int C, D;
     mllm_status s = codec_args(nm, idx, words, n, &C, &D);
     if (s != MLLM_OK || n == 0) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t w = (n + D - 1) / D;
-    const int64_t grid = std::min<int64_t>((w + kThreads - 1) / kThreads, 65535 * 16);
-    diag::encode_kernel<<<(unsigned)grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(idx, n, C, D, words);
+    // whole groups of 4 words with vector accesses where the pointers allow, the rest word by word
+    const int64_t groups = codec_vector_ok(idx, words, D) ? n / (4 * (int64_t)D) : 0;
+    if (groups > 0) {
+        const int64_t grid = std::min<int64_t>((groups + kThreads - 1) / kThreads, 65535 * 16);
+        if (C == 6) diag::encode4_kernel<6, 12><<<(unsigned)grid, kThreads, 0, st>>>(idx, groups, words);
+        else diag::encode4_kernel<70, 5><<<(unsigned)grid, kThreads, 0, st>>>(idx, groups, words);
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    }
+    if (4 * groups < w) {
+        const int64_t grid = std::min<int64_t>((w - 4 * groups + kThreads - 1) / kThreads, 65535 * 16);
+        diag::encode_kernel<<<(unsigned)grid, kThreads, 0, st>>>(idx, n, C, D, words, 4 * groups);
+    }
     return cuda_status(cudaGetLastError());
 }
 
@@ -1151,9 +1169,19 @@ mllm_status mllm_decode_candidates(mllm_nm nm, const uint32_t *words, int64_t n,
     int C, D;
     mllm_status s = codec_args(nm, words, idx, n, &C, &D);
     if (s != MLLM_OK || n == 0) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t w = (n + D - 1) / D;
-    const int64_t grid = std::min<int64_t>((w + kThreads - 1) / kThreads, 65535 * 16);
-    diag::decode_kernel<<<(unsigned)grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(words, n, C, D, idx);
+    const int64_t groups = codec_vector_ok(idx, words, D) ? n / (4 * (int64_t)D) : 0;
+    if (groups > 0) {
+        const int64_t grid = std::min<int64_t>((groups + kThreads - 1) / kThreads, 65535 * 16);
+        if (C == 6) diag::decode4_kernel<6, 12><<<(unsigned)grid, kThreads, 0, st>>>(words, groups, idx);
+        else diag::decode4_kernel<70, 5><<<(unsigned)grid, kThreads, 0, st>>>(words, groups, idx);
+        if ((s = cuda_status(cudaGetLastError())) != MLLM_OK) return s;
+    }
+    if (4 * groups < w) {
+        const int64_t grid = std::min<int64_t>((w - 4 * groups + kThreads - 1) / kThreads, 65535 * 16);
+        diag::decode_kernel<<<(unsigned)grid, kThreads, 0, st>>>(words, n, C, D, idx, 4 * groups);
+    }
     return cuda_status(cudaGetLastError());
 }
 
