@@ -1,6 +1,6 @@
 // kernels_umma.cuh -- the serving product on the fifth-generation tensor cores: 2:4 at 17-64
 // tokens with tcgen05.mma.sp (operands in shared memory, sparsity metadata and accumulators in
-// tensor memory), and 4:8 at 1-64 tokens with blocks expanded to a dense tile in shared memory
+// tensor memory), and 4:8 at 1-64 tokens with blocks expanded to a dense tile in tensor memory
 // and dense tcgen05.mma (below, "4:8 on the dense tensor cores").
 //
 // The product is y = x W*^T with W* = W (.) M* in the form mllm_hard_pack writes (two kept
