@@ -1138,7 +1138,8 @@ static mllm_status codec_args(mllm_nm nm, const void *src, const void *dst, int6
 }
 
 // The codec's vector kernels read or write the indices as 32-bit (D % 4 == 0: 16-byte) words
-// and the code as 16-byte vectors.
+// and the code as 16-byte vectors (the entry points' pointer checks already ask for 16-byte
+// alignment; this keeps the kernels' own requirement next to them).
 static bool codec_vector_ok(const void *idx, const void *words, int D) {
     const uintptr_t a = reinterpret_cast<uintptr_t>(idx), b = reinterpret_cast<uintptr_t>(words);
     return (b & 15u) == 0 && (a & ((D % 4 == 0) ? 15u : 3u)) == 0;
