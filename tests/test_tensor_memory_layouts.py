@@ -79,3 +79,23 @@ def test_4of8_zero_filled_code_expands_to_zero():
     """Rows past the matrix arrive zero-filled (values 0, code 0): the chunk must be zero."""
     sa, sb = u8_table_entry(0, False), u8_table_entry(0, True)
     assert [byte_perm(byte_perm(0, 0, sa[i]), 0, sb[i]) for i in range(4)] == [0, 0, 0, 0]
+
+
+def test_4of8_prefill_value_reads_undo_the_64_byte_swizzle():
+    """The 4:8 prefill kernel lands each stage's 128-row x 64-byte box of compressed values
+    with the tensor map's 64-byte swizzle (on a 512-byte boundary: 16-byte chunk c of row r at
+    chunk c ^ ((r >> 1) & 3)); the thread of row r and part pt reads its chunk at that place,
+    and the eight consecutive rows a quarter-warp reads at one part fall on eight distinct
+    four-bank groups (no bank conflict)."""
+    def landed(off):  # byte offset of logical byte `off` of the box after the 64-byte swizzle
+        return off ^ (((off >> 7) & 3) << 4)
+
+    def read_at(r, pt):  # the kernel's address of row r, part pt
+        return r * 64 + ((pt ^ ((r >> 1) & 3)) << 4)
+
+    for r in range(128):
+        for pt in range(4):
+            assert landed(r * 64 + pt * 16) == read_at(r, pt)
+    for q0 in range(0, 128, 8):
+        for pt in range(4):
+            assert len({(read_at(r, pt) // 16) % 8 for r in range(q0, q0 + 8)}) == 8
