@@ -1,4 +1,4 @@
-"""Host models of two pieces of index arithmetic in the tensor-memory serving kernels.
+"""Host models of index arithmetic in the tensor-memory serving kernels.
 
 1. 2:4 sparsity metadata in tensor memory (kernels_umma.cuh). For a kind::f16 sparse MMA with
    M = 128 and K = 32, the 4-bit code of block b (columns 4b..4b+3, b = 0..7) of row m sits in
@@ -8,6 +8,8 @@
 2. 4:8 expansion (kernels_umma.cuh, u8_table_entry): a block's four values in position order
    (v0 v1 in one word, v2 v3 in the other) become a dense chunk of eight bf16 through
    prmt(prmt(v0v1, 0, A[p0 p1]), v2v3, B[p2 p3]) per word; this checks all 70 position sets.
+   The four words are the block's four 32-bit columns of the dense tile in tensor memory.
+3. 4:8 prefill (kernels_pf48.cuh): the reads of the 64-byte-swizzled box of compressed values.
 """
 import itertools
 import random
