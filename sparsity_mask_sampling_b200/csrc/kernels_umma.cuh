@@ -720,7 +720,8 @@ __device__ __forceinline__ void umma_dense_ta(unsigned d_tmem, unsigned a_tmem, 
         : "memory");
 }
 
-// 16 consecutive 32-bit columns of this thread's lane from w[16], then wait for the store.
+// 16 consecutive 32-bit columns of this thread's lane from w[16]; the store completes
+// asynchronously (tmem_st_wait waits for all of the warp's earlier stores).
 __device__ __forceinline__ void tmem_st16(unsigned taddr, const uint32_t (&w)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -728,8 +729,8 @@ __device__ __forceinline__ void tmem_st16(unsigned taddr, const uint32_t (&w)[16
         "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]),
         "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
         : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 // 8 consecutive accumulator columns of this thread's lane (see tmem_ld16).
 __device__ __forceinline__ void tmem_ld8(unsigned taddr, float *v) {
@@ -964,6 +965,20 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
         Cursor cc = sk_decode(grp, lo);
         unsigned acc_phase = 0u;
         bool failed = false;
+        // With six stages in flight, a stage's store into tensor memory is waited for (and the
+        // stage handed to the MMA warp) only after the next stage's expansion, so the store's
+        // latency overlaps it (1-32 tokens: 1 % faster); with five (above 48 tokens) the lost
+        // stage costs more (2 %), so there each stage is handed over at once.
+        constexpr bool kDefer = kD >= 6;
+        int pending = -1;
+        auto hand_over = [&]() {
+            if (pending >= 0) {
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(exp0 + 8 * pending);
+                pending = -1;
+            }
+        };
         for (int f = 0; f < n; ++f) {
             const int s = f % kD;
             unsigned char *st = ring + s * kStage;
@@ -973,10 +988,12 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
                 if (um_wait(full0 + 8 * s, (f / kD) & 1, &s_abort)) {
                     uint32_t w[16];
                     u8_expand<64 / kU8Warps>(st, tab_a, tab_b, kMetaOff, r, pt, w);
+                    hand_over();
                     tmem_st16(tdense + 64u * (unsigned)s, w);  // into the stage's dense tile in tensor memory
-                    tc_fence_before();
-                    mbar_arrive(exp0 + 8 * s);
+                    pending = s;
+                    if (!kDefer) hand_over();
                 } else {
+                    hand_over();
                     failed = true;
                     if (lane == 0 && !s_abort) {
                         atomicOr(err, 1u);
@@ -986,6 +1003,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
             }
             const SkOp &d = grp.d[cc.op];
             const bool piece_end = (cc.j == d.nch - 1) || (f == n - 1);
+            if (piece_end) hand_over();
             if (piece_end) {
                 const bool acc_ok = !failed && um_wait(accb, acc_phase, &s_abort);
                 acc_phase ^= 1u;
