@@ -692,7 +692,9 @@ template <int kNTok> constexpr int u8_stage_bytes() { return (u8_tx<kNTok>() + 1
 template <int kNTok> constexpr int u8_stages() { return kNTok <= 48 ? 6 : 5; }
 constexpr int kU8TabCopies = 8;      // one copy per lane of a quarter-warp: conflict-free 16-byte lookups
 constexpr int kU8TabBytes = 2 * 64 * kU8TabCopies * 16;  // tables A and B
-template <int kNTok> constexpr int u8_smem_bytes() { return u8_stages<kNTok>() * u8_stage_bytes<kNTok>() + 1024 + kU8TabBytes; }
+// The two 8 KB selector tables come first, on an 8 KB boundary (so that a lookup's address is
+// the table's base OR'ed with the entry's and the copy's bits), then the stages.
+template <int kNTok> constexpr int u8_smem_bytes() { return u8_stages<kNTok>() * u8_stage_bytes<kNTok>() + 8192 + kU8TabBytes; }
 
 // Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
 // N = kNTok, M = 128.
@@ -785,8 +787,22 @@ __device__ __forceinline__ void u8_issue(const TmGroup &tg, const Cursor &c, uns
 // its 4 kBlk 32-bit columns of the row's dense K-slice: block b's eight values are columns
 // 4 (b - kBlk pt) .. +3, two bf16 per column in K order (the layout tcgen05.mma reads A in
 // from tensor memory).
+// 16-byte load from a shared-memory address.
+__device__ __forceinline__ uint4 lds128_at(unsigned addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+// Row r, part pt of a stage (kBlk = 64 / kU8Warps blocks from block kBlk pt) expanded into
+// its 4 kBlk 32-bit columns of the row's dense K-slice: block b's eight values are columns
+// 4 (b - kBlk pt) .. +3, two bf16 per column in K order (the layout tcgen05.mma reads A in
+// from tensor memory). ta / tb: shared-memory addresses of this lane's copy of entry 0 of
+// tables A and B (8 KB aligned but for the copy's bits 4-6), so that the entry of a 6-bit
+// pair code p is ta | p << 7: each lookup address is one shift and one masked OR of the
+// block's code word.
 template <int kBlk>
-__device__ __forceinline__ void u8_expand(const unsigned char *st, const uint4 *tab_a, const uint4 *tab_b,
+__device__ __forceinline__ void u8_expand(const unsigned char *st, unsigned ta, unsigned tb,
                                           int meta_off, int r, int pt, uint32_t (&w)[4 * kBlk]) {
     const int b0 = kBlk * pt;
     uint32_t codes[kBlk / 2];
@@ -801,11 +817,14 @@ __device__ __forceinline__ void u8_expand(const unsigned char *st, const uint4 *
     for (int c = 0; c < kBlk / 2; ++c) {
         const int cl = (b0 >> 1) + c;  // value chunk within the row
         const uint4 v = lds128(st + r * 128 + ((cl ^ (r & 7)) << 4));
+        const uint32_t cw = codes[c];  // block 2c + 0 in bits 0-11, block 2c + 1 in bits 16-27
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
-            const uint32_t code = (codes[c] >> (16 * h)) & 0xFFFu;
-            const uint4 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
+            // pair codes p0p1 (code bits 0-5) and p2p3 (bits 6-11) placed at bits 7-12
+            const uint32_t ka = (h ? (cw >> 9) : (cw << 7)) & 0x1F80u;
+            const uint32_t kb = (h ? (cw >> 15) : (cw << 1)) & 0x1F80u;
+            const uint4 sa = lds128_at(ta | ka), sb = lds128_at(tb | kb);
             uint32_t *o = w + 4 * (2 * c + h);
             o[0] = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
             o[1] = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
@@ -857,10 +876,10 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
     const int64_t lo = cta * total / G, hi = (cta + 1) * total / G;
     const int n = (int)(hi - lo);
     const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_u8);
-    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
-    unsigned char *ring = s_dyn_u8 + pad;
-    const unsigned ring_s = dyn_s + pad;
-    uint4 *tab = reinterpret_cast<uint4 *>(ring + kD * kStage);  // A: entries [0, 64), B: [64, 128), x copies
+    const unsigned tab_s = (dyn_s + 8191u) & ~8191u;  // tables A, B: 8 KB each on 8 KB boundaries
+    uint4 *tab = reinterpret_cast<uint4 *>(s_dyn_u8 + (tab_s - dyn_s));  // A: entries [0, 64), B: [64, 128), x copies
+    const unsigned ring_s = tab_s + (unsigned)kU8TabBytes;  // 1 KB aligned
+    unsigned char *ring = s_dyn_u8 + (ring_s - dyn_s);
     const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
     const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
     const unsigned exp0 = (unsigned)__cvta_generic_to_shared(&s_exp[0]);
@@ -961,7 +980,7 @@ __global__ void __launch_bounds__(kU8Threads, 1) sparse_linear_umma48_kernel(con
         const int q = warp & 3, ch = warp >> 2;  // TMEM lane quarter, token slice of the epilogue
         const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(ch * kHalf);
         const unsigned tdense = tbase + ((unsigned)(32 * q) << 16) + kU8ACol + 16u * (unsigned)pt;  // row r's part
-        const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
+        const unsigned tab_a = tab_s + 16u * (unsigned)(lane & (kU8TabCopies - 1)), tab_b = tab_a + 64u * 16u * kU8TabCopies;
         Cursor cc = sk_decode(grp, lo);
         unsigned acc_phase = 0u;
         bool failed = false;
