@@ -43,7 +43,7 @@ template <int kTok> struct P8 {
     static constexpr int kStageTx = kTok * 128 + kUmRows * 64 + kUmRows * 16;  // bytes the copy engine lands
     static constexpr int kStage = (kMetaOff + kUmRows * 16 + 1023) / 1024 * 1024;
     static constexpr int kStages = kTok == 256 ? 4 : 6;
-    static constexpr int kSmem = kStages * kStage + 1024 + kU8TabBytes;
+    static constexpr int kSmem = kStages * kStage + 8192 + kU8TabBytes;  // tables first, 8 KB aligned
     static constexpr unsigned kACol = kTok;                      // stage s's dense tile: 32 columns from kACol + 32 s
     static constexpr unsigned kTmemCols = 512;
     // Instruction descriptor of kind::f16: dense, f32 accumulator, bf16 A and B (K-major),
@@ -69,8 +69,10 @@ __device__ __forceinline__ void p8_issue(const PfGroup &g, const PfCur &c, int64
 // order). The values box lands with the 64-byte swizzle (16-byte chunk c of row r at chunk
 // c ^ ((r >> 1) & 3)), so the 32 rows a warp reads at one pt fall on distinct banks in each
 // quarter-warp; each thread reads its row's 16 bytes of codes whole and keeps word pt.
+// ta / tb: shared-memory addresses of this lane's copy of entry 0 of the selector tables (8 KB
+// aligned but for the copy's bits), the entry of pair code p at ta | p << 7 (u8_expand).
 template <int kTok>
-__device__ __forceinline__ void p8_expand(const unsigned char *st, const uint4 *tab_a, const uint4 *tab_b, int r, int pt,
+__device__ __forceinline__ void p8_expand(const unsigned char *st, unsigned ta, unsigned tb, int r, int pt,
                                           uint32_t (&w)[8]) {
     using K = P8<kTok>;
     const uint4 v = lds128(st + K::kValOff + r * 64 + ((pt ^ ((r >> 1) & 3)) << 4));
@@ -79,8 +81,9 @@ __device__ __forceinline__ void p8_expand(const unsigned char *st, const uint4 *
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const uint32_t lo = h ? v.z : v.x, hi = h ? v.w : v.y;
-        const uint32_t code = (cw >> (16 * h)) & 0xFFFu;
-        const uint4 sa = tab_a[(code & 63u) * kU8TabCopies], sb = tab_b[(code >> 6) * kU8TabCopies];
+        const uint32_t ka = (h ? (cw >> 9) : (cw << 7)) & 0x1F80u;
+        const uint32_t kb = (h ? (cw >> 15) : (cw << 1)) & 0x1F80u;
+        const uint4 sa = lds128_at(ta | ka), sb = lds128_at(tb | kb);
         uint32_t *o = w + 4 * h;
         o[0] = __byte_perm(__byte_perm(lo, 0u, sa.x), hi, sb.x);
         o[1] = __byte_perm(__byte_perm(lo, 0u, sa.y), hi, sb.y);
@@ -115,10 +118,10 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t G = gridDim.x, u0 = blockIdx.x, u1 = pg.total_units;
     const unsigned dyn_s = (unsigned)__cvta_generic_to_shared(s_dyn_p8);
-    const unsigned pad = (1024u - (dyn_s & 1023u)) & 1023u;
-    unsigned char *ring = s_dyn_p8 + pad;
-    const unsigned ring_s = dyn_s + pad;
-    uint4 *tab = reinterpret_cast<uint4 *>(ring + kD * kP8Stage);  // A: entries [0, 64), B: [64, 128), x copies
+    const unsigned tab_s = (dyn_s + 8191u) & ~8191u;  // tables A, B: 8 KB each on 8 KB boundaries
+    uint4 *tab = reinterpret_cast<uint4 *>(s_dyn_p8 + (tab_s - dyn_s));  // A: entries [0, 64), B: [64, 128), x copies
+    const unsigned ring_s = tab_s + (unsigned)kU8TabBytes;  // 1 KB aligned
+    unsigned char *ring = s_dyn_p8 + (ring_s - dyn_s);
     const unsigned full0 = (unsigned)__cvta_generic_to_shared(&s_full[0]);
     const unsigned empty0 = (unsigned)__cvta_generic_to_shared(&s_empty[0]);
     const unsigned exp0 = (unsigned)__cvta_generic_to_shared(&s_exp[0]);
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(kP8Threads, 1) sparse_linear_prefill48_kernel(
         const int r = 32 * q + lane, pt = sl;                  // expansion: row (this lane), part
         const unsigned tq = tbase + ((unsigned)(32 * q) << 16) + (unsigned)(kQTok * sl);
         const unsigned tdense = tbase + ((unsigned)(32 * q) << 16) + K::kACol + 8u * (unsigned)pt;
-        const uint4 *tab_a = tab + (lane & (kU8TabCopies - 1)), *tab_b = tab_a + 64 * kU8TabCopies;
+        const unsigned tab_a = tab_s + 16u * (unsigned)(lane & (kU8TabCopies - 1)), tab_b = tab_a + 64u * 16u * kU8TabCopies;
         unsigned acc_phase = 0u;
         bool failed = false;
         int f = 0;
